@@ -1,0 +1,208 @@
+/*
+ * jolt.h -- C ABI of the JoLT / FlashJoLT KV-cache compressor for NVIDIA B200 (sm_100a).
+ *
+ * What it computes (sources: "A JoLT for the KV cache: Near-Lossless KV Cache Compression
+ * via Joint Rank-bit Allocation", abstract; "A JoLT for the KV Cache: Near-Lossless KV
+ * Cache Compression via Joint Tucker and JL-Residual Allocation for LLMs", introduction):
+ * per layer group and separately for keys and values, the grouped prefill cache
+ * X[l, h, t, d] (layers x heads x tokens x features) is factored by a partial Tucker
+ * decomposition on the token and feature modes only, X[l,h] ~ U C[l,h] W^T; the
+ * truncation residual is rotated by a random orthogonal (Johnson-Lindenstrauss) rotation
+ * and quantised to b bits; one Lagrangian dual picks (token rank, feature rank, bits)
+ * for every unit under one global byte budget.  JoLT takes the token factor from an
+ * exact eigen-decomposition; FlashJoLT from a randomized SVD sketch Y = X_(T) Omega.
+ *
+ * Readings of what the pages leave open (all fixed here):
+ *   - unit u = 2*g + kv: layer group g (layers_per_group consecutive layers), kv 0 = K, 1 = V;
+ *     S = layers_per_group * n_heads slices per unit, M = S * head_dim;
+ *   - rotation along the features of every row: rho = r diag(sigma) H_D / sqrt(D), H_D the
+ *     Sylvester Hadamard matrix, sigma from splitmix64 (seed, stream 2<<32 | u, index d);
+ *   - quantiser: blocks of 16 consecutive rotated features, lo = fp16 round-down(min),
+ *     step = fp16 round-up((max - lo)/(2^b - 1)), code = round-half-even((rho - lo)/step);
+ *   - stored factors U (T x r_T), W (D x r_D), core (S x r_T x r_D) in bf16; the decoder
+ *     forms U P' with P' = bf16((C W^T) diag(sigma) H_D / sqrt(D)) and un-rotates the sum
+ *     of that and the dequantised residual;
+ *   - budget = total blob bytes including the 64-byte global header and 64 bytes per unit.
+ *
+ * Conventions for every call:
+ *   - every pointer named *_dev is device memory the caller owns; the library keeps no
+ *     pointer after the call returns and allocates no device memory of its own (the one
+ *     exception: eigen-solver and Cholesky calls go through a cuSOLVER handle that the
+ *     library creates once per thread and device, which holds cuSOLVER's own state);
+ *   - calls are stream-ordered on `stream` (a cudaStream_t, NULL = legacy default stream)
+ *     and return before the GPU work finishes, except where a call says it synchronises;
+ *   - argument errors are detected on the host and returned before anything is launched;
+ *     errors found on the device (non-finite input, infeasible budget, factorisation
+ *     breakdown) are written to the blob's header status word and returned by the next
+ *     call that synchronises (jolt_read_header, jolt_decompress);
+ *   - on any non-OK return, jolt_last_error() gives a one-line message (thread-local).
+ */
+#ifndef JOLT_H_
+#define JOLT_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  JOLT_OK = 0,
+  JOLT_ERR_INVALID_ARG = 1,        /* null pointer, bad enum, bad candidate list */
+  JOLT_ERR_UNSUPPORTED_SHAPE = 2,  /* head_dim not in {16,32,64,128}, n_tokens % 16, ... */
+  JOLT_ERR_WORKSPACE_TOO_SMALL = 3,
+  JOLT_ERR_OUTPUT_TOO_SMALL = 4,   /* blob capacity below the budget */
+  JOLT_ERR_BUDGET_INFEASIBLE = 5,  /* budget below every unit's fewest-bytes choice */
+  JOLT_ERR_NUMERIC = 6,            /* NaN/Inf in the cache, or an eigen/Cholesky breakdown */
+  JOLT_ERR_TIMEOUT = 7,            /* reserved: a bounded device wait gave up */
+  JOLT_ERR_CUDA = 8,               /* a CUDA runtime or cuSOLVER call failed */
+  JOLT_ERR_BAD_BLOB = 9            /* blob header failed validation */
+} jolt_status;
+
+typedef enum { JOLT_BF16 = 0, JOLT_F32 = 1 } jolt_dtype;
+typedef enum { JOLT_EXACT = 0, JOLT_RANDOMIZED = 1 } jolt_method;
+
+/* Shape of ONE of the two cache tensors K and V, both [n_layers, n_heads, n_tokens, head_dim],
+ * row-major, element type `dtype`.  n_layers % layers_per_group == 0. */
+typedef struct {
+  int32_t n_layers;
+  int32_t n_heads;
+  int32_t n_tokens;
+  int32_t head_dim;
+  int32_t layers_per_group;
+  int32_t dtype; /* jolt_dtype */
+} jolt_shape;
+
+#define JOLT_MAX_CANDIDATES 8
+
+/* Candidate sets of the allocation (ascending, no repeats) and the token-factor method.
+ * Choice index c = (i_T * n_feature_ranks + i_D) * n_bits + i_b. */
+typedef struct {
+  int32_t n_token_ranks;
+  int32_t token_ranks[JOLT_MAX_CANDIDATES];   /* 1 <= r_T <= n_tokens (and <= M) */
+  int32_t n_feature_ranks;
+  int32_t feature_ranks[JOLT_MAX_CANDIDATES]; /* 1 <= r_D <= head_dim */
+  int32_t n_bits;
+  int32_t bits[JOLT_MAX_CANDIDATES];          /* 0 <= b <= 8; 0 = no residual */
+  int32_t method;                             /* jolt_method */
+  int32_t oversample;                         /* FlashJoLT sketch width = max r_T + oversample */
+  int32_t power_iters;                        /* FlashJoLT power iterations */
+} jolt_options;
+
+/* Per-unit record of a compressed blob, as returned by jolt_read_header. */
+typedef struct {
+  int32_t r_T, r_D, bits, choice;
+  uint64_t off_U, off_W, off_C, off_codes, off_scales; /* byte offsets inside the blob */
+  double distortion;  /* table value || X_u - decode(encode(X_u)) ||_F^2 of the choice */
+} jolt_unit_record;
+
+/* Library version string. */
+const char* jolt_version(void);
+
+/* Message of the last non-OK status returned on this thread. */
+const char* jolt_last_error(void);
+
+/* Sizes the caller must provide.
+ *   ws_bytes   : device workspace for jolt_compress / jolt_factor / jolt_table / jolt_encode
+ *   blob_bytes : the largest blob any budget can produce (every unit at its largest choice)
+ *   dws_bytes  : device workspace for jolt_decompress
+ * Returns INVALID_ARG / UNSUPPORTED_SHAPE for shapes or options the library rejects. */
+jolt_status jolt_workspace_size(const jolt_shape* shape, const jolt_options* opts, size_t* ws_bytes,
+                                size_t* blob_bytes, size_t* dws_bytes);
+
+/* Number of units (2 * n_layers / layers_per_group) and of choices per unit. */
+jolt_status jolt_counts(const jolt_shape* shape, const jolt_options* opts, int32_t* n_units,
+                        int32_t* n_choices);
+
+/* Payload bytes of every choice (identical for all units), n_choices uint64 on the HOST.
+ * Formula: pad16(2 T r_T) + pad16(2 D r_D) + pad16(2 S r_T r_D)
+ *        + [b > 0] (pad16(nblk * 2b) + pad16(nblk * 4)),  nblk = S T D / 16.
+ * ("a single Lagrangian dual allocates ... under a global byte constraint", abstract.) */
+jolt_status jolt_choice_bytes(const jolt_shape* shape, const jolt_options* opts, uint64_t* bytes_host);
+
+/* Whole compress ("JoLT ... treats grouped prefill caches as fourth-order tensors and applies
+ * partial Tucker decomposition along the token and feature modes ... A rotated low-bit
+ * quantizer captures the truncation residual, and a single Lagrangian dual allocates
+ * per-group Tucker ranks and residual bit-widths under a global byte constraint", abstract).
+ *   k_dev, v_dev : input caches (read only), shape/dtype as `shape`
+ *   budget_bytes : total blob bytes allowed (headers included)
+ *   seed         : seeds the rotation signs and the FlashJoLT sketch
+ *   blob_dev     : output, capacity blob_cap >= budget_bytes; layout: 64-byte header,
+ *                  64 bytes per unit, then per unit U, W, core, codes, scales (16-B aligned)
+ *   ws_dev       : workspace of ws_bytes >= jolt_workspace_size().ws_bytes
+ * Asynchronous.  Infeasible budget / non-finite input are reported in the blob header. */
+jolt_status jolt_compress(const jolt_shape* shape, const void* k_dev, const void* v_dev, const jolt_options* opts,
+                          uint64_t budget_bytes, uint64_t seed, void* blob_dev, size_t blob_cap, void* ws_dev,
+                          size_t ws_bytes, void* stream);
+
+/* Stage 1: token and feature factors of every unit (partial Tucker, token and feature modes;
+ * "FlashJoLT replaces the exact token-mode SVD with a randomized approximation", abstract).
+ *   u_dev : [n_units][n_tokens][ld_u] fp32, unrounded token factor (leading max r_T columns)
+ *   w_dev : [n_units][head_dim][ld_w] fp32, unrounded feature factor (leading max r_D columns)
+ *   ld_u >= max r_T, ld_w >= max r_D.  Columns ordered by descending singular value, the
+ *   entry of largest magnitude of every column positive.  Asynchronous. */
+jolt_status jolt_factor(const jolt_shape* shape, const void* k_dev, const void* v_dev, const jolt_options* opts,
+                        uint64_t seed, float* u_dev, int64_t ld_u, float* w_dev, int64_t ld_w, void* ws_dev,
+                        size_t ws_bytes, void* stream);
+
+/* Stage 2: stored core and distortion table from given bf16 factors.
+ *   u_bf16_dev : [n_units][n_tokens][ld_u] bf16 (leading max r_T columns used)
+ *   w_bf16_dev : [n_units][head_dim][ld_w] bf16 (leading max r_D columns used)
+ *   core_dev   : out [n_units][S][max r_T][max r_D] bf16, C = bf16(U^T bf16(X W)) per slice
+ *   table_dev  : out [n_units][n_choices] fp64, || X - decode(encode_c(X)) ||_F^2
+ * Asynchronous. */
+jolt_status jolt_table(const jolt_shape* shape, const void* k_dev, const void* v_dev, const jolt_options* opts,
+                       uint64_t seed, const void* u_bf16_dev, int64_t ld_u, const void* w_bf16_dev, int64_t ld_w,
+                       void* core_dev, double* table_dev, void* ws_dev, size_t ws_bytes, void* stream);
+
+/* Stage 3: the single Lagrangian dual ("a single Lagrangian dual allocates per-group Tucker
+ * ranks and residual bit-widths under a global byte constraint", abstract; "per layer group
+ * and separately for keys and values, under one byte budget", introduction).
+ *   dist_dev [n_units][n_choices] fp64, bytes_dev [n_units][n_choices] uint64 (device),
+ *   budget_bytes: payload bytes available (headers NOT included here).
+ *   choice_dev [n_units] int32 out, lambda_dev [1] fp64 out (+inf when infeasible),
+ *   status_dev [1] uint32 out: 0 ok, 4 infeasible.
+ * Rule: lambda = 0 if the distortion-minimising choices fit; else lo = 0, hi = 1 doubled
+ * until the choices fit, then 200 bisection halvings; answer = choices at hi.  Per unit,
+ * argmin D + lambda*B in fp64 (no fused multiply-add), ties to fewer bytes then lower index.
+ * Asynchronous; one CTA. */
+jolt_status jolt_allocate(const double* dist_dev, const uint64_t* bytes_dev, int32_t n_units, int32_t n_choices,
+                          uint64_t budget_bytes, int32_t* choice_dev, double* lambda_dev, uint32_t* status_dev,
+                          void* stream);
+
+/* Stage 4: write the blob for given factors, core and choices (choice_dev [n_units] int32,
+ * dist_dev [n_units][n_choices] fp64 recorded in the unit headers).  Same factor layouts as
+ * jolt_table.  Asynchronous. */
+jolt_status jolt_encode(const jolt_shape* shape, const void* k_dev, const void* v_dev, const jolt_options* opts,
+                        uint64_t seed, const void* u_bf16_dev, int64_t ld_u, const void* w_bf16_dev, int64_t ld_w,
+                        const void* core_dev, const int32_t* choice_dev, const double* dist_dev, void* blob_dev,
+                        size_t blob_cap, void* ws_dev, size_t ws_bytes, void* stream);
+
+/* Read and validate a blob's headers (SYNCHRONISES the stream).  records: n_units entries
+ * (capacity `cap`).  Returns the device-side status recorded in the header
+ * (BUDGET_INFEASIBLE, NUMERIC, OUTPUT_TOO_SMALL) or BAD_BLOB for a corrupt header. */
+jolt_status jolt_read_header(const void* blob_dev, jolt_shape* shape_out, uint64_t* total_bytes,
+                             jolt_unit_record* records, int32_t cap, void* stream);
+
+/* Decompress ("a fused ... kernel evaluates attention directly over the stored factors",
+ * abstract: this is the dense reconstruction from the same stored factors):
+ * X_hat = (U P' + dequant(codes)) diag(sigma) H_D / sqrt(D) per unit.
+ *   out_dtype: JOLT_BF16 or JOLT_F32; k_out_dev, v_out_dev: [n_layers, H, T, D].
+ * Reads the headers first (SYNCHRONISES once), then runs asynchronously. */
+jolt_status jolt_decompress(const void* blob_dev, int32_t out_dtype, void* k_out_dev, void* v_out_dev, void* ws_dev,
+                            size_t ws_bytes, void* stream);
+
+/* Per-unit sums of squares (relative Frobenius error, "relative Frobenius error 0.009 (K)
+ * and 0.006 (V)", introduction): sq_dev[2*u] = ||X_u||^2, sq_dev[2*u+1] = ||X_u - Y_u||^2
+ * (fp64), X and Y of the same shape; y may be NULL (then only ||X_u||^2).  ydtype is Y's
+ * element type.  Asynchronous. */
+jolt_status jolt_frobenius(const jolt_shape* shape, const void* k_dev, const void* v_dev, const void* ky_dev,
+                           const void* vy_dev, int32_t ydtype, double* sq_dev, void* ws_dev, size_t ws_bytes,
+                           void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* JOLT_H_ */

@@ -1,0 +1,631 @@
+// Streaming kernels of the compress / decompress path.
+//
+// The residual of every candidate is formed in the rotated basis: the cache tile is
+// rotated once (sign flip + Walsh-Hadamard along the features), and the candidate's
+// reconstruction U_s[:, :r_T] P'(r_D)[:r_T] comes straight out of the tensor cores with
+// the rotation already folded into P' = bf16((C_s W_s^T) Phi).  The per-candidate work
+// is then a subtraction, a 16-wide block min/max and the quantiser for every bit-width.
+#pragma once
+
+#include "common.cuh"
+#include "gemm.cuh"
+
+namespace jolt {
+
+constexpr int MAXC = 8;   // candidates per set (token ranks, feature ranks, bit-widths)
+
+struct CacheView {
+  const void* k;          // [n_layers, H, T, D]
+  const void* v;
+  int dtype;              // 0 bf16, 1 fp32
+  int n_layers, H, T, D, Lg, S;
+  long long unit_elems;   // S * T * D
+  __host__ __device__ const void* unit_ptr(int u) const {
+    const char* base = (const char*)((u & 1) ? v : k);
+    return base + (long long)(u >> 1) * unit_elems * (dtype ? 4 : 2);
+  }
+};
+
+struct Cands {
+  int nT, nD, nB;
+  int rT[MAXC], rD[MAXC], bits[MAXC];
+};
+
+// ---------------------------------------------------------------------------------------
+// exact fp16 directed-rounding helpers
+// ---------------------------------------------------------------------------------------
+__device__ __forceinline__ float fp16_rd(float x) { return __half2float(__float2half_rd(x)); }
+
+// smallest fp16 s with s * levels >= mx - lo (exact), i.e. fp16 round-up of (mx - lo)/levels;
+// 0 when mx <= lo.  A float estimate is corrected by one fp16 ulp with exact fp64 checks.
+__device__ __forceinline__ float quant_step(float mx, float lo, int levels, float inv_levels) {
+  if (!(mx > lo)) return 0.f;
+  double need = (double)mx - (double)lo;
+  float q = (mx - lo) * inv_levels;
+  unsigned short u = __half_as_ushort(__float2half_ru(q));
+  double s = (double)__half2float(__ushort_as_half(u));
+  if (s * (double)levels < need) {
+    u = (unsigned short)(u + 1);
+  } else if (u > 0) {
+    unsigned short d = (unsigned short)(u - 1);
+    double sd = (double)__half2float(__ushort_as_half(d));
+    if (sd * (double)levels >= need) u = d;
+  }
+  return __half2float(__ushort_as_half(u));
+}
+
+// round-half-even to integer of a non-negative float below 2^22 via the 1.5*2^23 shift
+__device__ __forceinline__ float rne_int(float q) {
+  const float magic = 12582912.0f;
+  return __fsub_rn(__fadd_rn(q, magic), magic);
+}
+
+// ---------------------------------------------------------------------------------------
+// fused residual / rotation / quantiser tile machinery (mma.sync m16n8k16 fragments)
+//
+// A CTA owns ROWS = 64 consecutive tokens of one slice (4 warps x 16 rows) and the full
+// feature width D.  Thread (warp w, lane) holds rows g = lane/4 and g+8 of its warp's 16
+// and, for every n8 tile j, columns 8j + 2(lane%4) + {0,1}.  A 16-wide quantisation block
+// m is n8 tiles 2m and 2m+1: four values per thread, completed across the lane quad.
+// ---------------------------------------------------------------------------------------
+constexpr int TROWS = 64;
+constexpr int TTHREADS = 128;
+constexpr int KC = 64;  // token-rank chunk staged per pipeline step
+
+template <int D>
+struct TileFrag {
+  static constexpr int NT = D / 8;
+  float v[2][NT][2];
+};
+
+// rotate the tile's rows (sigma, Walsh-Hadamard, 1/sqrt(D)) into smem as fp32
+template <int D, typename TX>
+__device__ __forceinline__ void rotate_tile_to_smem(const TX* X, int T, int t0, const float* sig, float* xs) {
+  // xs: [TROWS][D + 4]
+  for (int r = threadIdx.x; r < TROWS; r += blockDim.x) {
+    float v[D];
+    int t = t0 + r;
+    if (t < T) {
+      const TX* row = X + (long long)t * D;
+#pragma unroll
+      for (int d = 0; d < D; ++d) v[d] = ld_as_float(row + d) * sig[d];
+    } else {
+#pragma unroll
+      for (int d = 0; d < D; ++d) v[d] = 0.f;
+    }
+    fwht_regs<D>(v);
+    const float sc = (float)(1.0 / sqrt((double)D));
+#pragma unroll
+    for (int d = 0; d < D; ++d) xs[r * (D + 4) + d] = v[d] * sc;
+  }
+}
+
+template <int D>
+__device__ __forceinline__ void frag_from_smem(const float* xs, TileFrag<D>& f) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    int r = warp * 16 + (lane >> 2) + h * 8;
+#pragma unroll
+    for (int j = 0; j < TileFrag<D>::NT; ++j) {
+      int c = j * 8 + (lane & 3) * 2;
+      f.v[h][j][0] = xs[r * (D + 4) + c];
+      f.v[h][j][1] = xs[r * (D + 4) + c + 1];
+    }
+  }
+}
+
+// Staged operands for the reconstruction MMA:  sU [TROWS][KC] (K-contiguous, swizzled)
+//                                             sP [KC][D]     (D-contiguous, swizzled)
+template <int D>
+struct ReconSmem {
+  static constexpr int U_ELEMS = TROWS * KC;
+  static constexpr int P_ELEMS = KC * D;
+  static constexpr int STAGE = U_ELEMS + P_ELEMS;
+};
+
+__device__ __forceinline__ int su_off(int row, int ch) { return row * KC + ((ch ^ (row & 7)) << 3); }
+template <int D>
+__device__ __forceinline__ int sp_off(int krow, int ch) {
+  constexpr int CH = D / 8;
+  return krow * D + ((CH >= 8 ? (ch ^ (krow & 7)) : (ch ^ (krow & (CH - 1)))) << 3);
+}
+
+// issue cp.async of U rows [t0, t0+64) x k [k0, k0+KC) and P' rows k [k0, k0+KC)
+template <int D>
+__device__ __forceinline__ void recon_load_stage(bf16* st, const bf16* U, long long ldU, int T, int t0,
+                                                 const bf16* P, int kmax, int k0) {
+  using namespace gemm_detail;
+  bf16* sU = st;
+  bf16* sP = st + ReconSmem<D>::U_ELEMS;
+  constexpr int UCH = TROWS * KC / 8;  // 512 chunks
+  for (int c = threadIdx.x; c < UCH; c += blockDim.x) {
+    int row = c / (KC / 8), ch = c % (KC / 8);
+    int t = t0 + row, k = k0 + ch * 8;
+    bool valid = (t < T) && (k < kmax);
+    const bf16* src = valid ? U + (long long)t * ldU + k : U;
+    cp_async16(smem_u32(sU + su_off(row, ch)), src, valid);
+  }
+  constexpr int PCH = KC * D / 8;
+  for (int c = threadIdx.x; c < PCH; c += blockDim.x) {
+    int krow = c / (D / 8), ch = c % (D / 8);
+    int k = k0 + krow;
+    bool valid = k < kmax;
+    const bf16* src = valid ? P + (long long)k * D + ch * 8 : P;
+    cp_async16(smem_u32(sP + sp_off<D>(krow, ch)), src, valid);
+  }
+}
+
+// accumulate the k16 slab at chunk offset kk (absolute token rank kabs) of a staged chunk,
+// keeping only the ranks in [klo, khi)
+template <int D>
+__device__ __forceinline__ void recon_mma_k16(const bf16* st, int kk, int kabs, int klo, int khi,
+                                              float (*acc)[4]) {
+  using namespace gemm_detail;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const bf16* sU = st;
+  const bf16* sP = st + ReconSmem<D>::U_ELEMS;
+  uint32_t a[4];
+  {
+    int row = warp * 16 + (lane & 15);
+    int ch = (kk >> 3) + (lane >> 4);
+    ldsm_x4(smem_u32(sU + su_off(row, ch)), a[0], a[1], a[2], a[3]);
+  }
+  if (klo > kabs || khi < kabs + 16) {
+    // zero the bf16 halves whose k falls outside [klo, khi)
+    int kq = kabs + (lane & 3) * 2;
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      int kb = kq + ((r >> 1) << 3);
+      uint32_t m = 0;
+      if (kb >= klo && kb < khi) m |= 0x0000FFFFu;
+      if (kb + 1 >= klo && kb + 1 < khi) m |= 0xFFFF0000u;
+      a[r] &= m;
+    }
+  }
+  constexpr int NT = D / 8;
+#pragma unroll
+  for (int np = 0; np < NT / 2; ++np) {
+    uint32_t r0, r1, r2, r3;
+    int krow = kk + (lane & 7) + (((lane >> 3) & 1) << 3);
+    int ch = np * 2 + (lane >> 4);
+    ldsm_x4_t(smem_u32(sP + sp_off<D>(krow, ch)), r0, r1, r2, r3);
+    mma16816(acc[np * 2 + 0], a, r0, r1);
+    mma16816(acc[np * 2 + 1], a, r2, r3);
+  }
+}
+
+// Walk the token-rank axis [0, kmax) in KC chunks; call epi(i) whenever the
+// accumulated prefix reaches cut[i] (cuts ascending, all <= kmax).
+template <int D, typename Epi>
+__device__ __forceinline__ void recon_walk(bf16* smem_stages, const bf16* U, long long ldU, int T, int t0,
+                                           const bf16* P, int kmax, const int* cuts, int ncuts,
+                                           float (*acc)[4], Epi&& epi) {
+  using namespace gemm_detail;
+  const int nchunks = (kmax + KC - 1) / KC;
+  int ci = 0;
+  while (ci < ncuts && cuts[ci] <= 0) { epi(ci); ++ci; }
+  recon_load_stage<D>(smem_stages, U, ldU, T, t0, P, kmax, 0);
+  cp_async_commit();
+  for (int c = 0; c < nchunks; ++c) {
+    if (c + 1 < nchunks)
+      recon_load_stage<D>(smem_stages + ((c + 1) & 1) * ReconSmem<D>::STAGE, U, ldU, T, t0, P, kmax, (c + 1) * KC);
+    cp_async_commit();
+    cp_async_wait<1>();
+    __syncthreads();
+    const bf16* st = smem_stages + (c & 1) * ReconSmem<D>::STAGE;
+    for (int kk = 0; kk < KC; kk += 16) {
+      int k = c * KC + kk;
+      if (k >= kmax) break;
+      int lo = k;
+      while (lo < k + 16 && lo < kmax) {
+        int hi = min(k + 16, kmax);
+        if (ci < ncuts && cuts[ci] > lo && cuts[ci] < hi) hi = cuts[ci];
+        recon_mma_k16<D>(st, kk, k, lo, hi, acc);
+        lo = hi;
+        while (ci < ncuts && cuts[ci] == lo) { epi(ci); ++ci; }
+      }
+    }
+    __syncthreads();
+  }
+  cp_async_wait<0>();
+}
+
+// per-row block min / max of rho = x' - acc over block m (n8 tiles 2m, 2m+1), quad-reduced
+template <int D>
+__device__ __forceinline__ void block_vals(const TileFrag<D>& xf, float (*acc)[4], int h, int m, float* r) {
+  r[0] = xf.v[h][2 * m][0] - acc[2 * m][h * 2 + 0];
+  r[1] = xf.v[h][2 * m][1] - acc[2 * m][h * 2 + 1];
+  r[2] = xf.v[h][2 * m + 1][0] - acc[2 * m + 1][h * 2 + 0];
+  r[3] = xf.v[h][2 * m + 1][1] - acc[2 * m + 1][h * 2 + 1];
+}
+
+__device__ __forceinline__ void quad_minmax(float& mn, float& mx) {
+  mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, 1));
+  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+  mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, 2));
+  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+}
+
+// ---------------------------------------------------------------------------------------
+// distortion table kernel: grid (tiles, S, units); writes fp64 partial sums per CTA
+// ---------------------------------------------------------------------------------------
+struct TableArgs {
+  CacheView cv;
+  const bf16* U;        // [unit][T][ldU]
+  long long ldU, sU;
+  const bf16* P;        // [unit][iD][S][rTmax][D]
+  long long sP_unit, sP_rd;
+  int rTmax;
+  Cands cand;
+  uint64_t seed;
+  double* partial;      // [unit][S][tiles][nD][nT][nB]
+  int tiles;
+};
+
+template <int D, typename TX>
+__global__ void __launch_bounds__(TTHREADS) table_kernel(TableArgs a) {
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  float* xs = reinterpret_cast<float*>(smem_raw);                          // TROWS x (D+4)
+  bf16* stages = reinterpret_cast<bf16*>(smem_raw + TROWS * (D + 4) * 4);   // 2 stages
+  __shared__ float sig[D];
+  __shared__ float red[4][MAXC];
+
+  const int tile = blockIdx.x, s = blockIdx.y, u = blockIdx.z;
+  const int T = a.cv.T;
+  const int t0 = tile * TROWS;
+  const TX* X = reinterpret_cast<const TX*>(a.cv.unit_ptr(u)) + (long long)s * T * D;
+  for (int d = threadIdx.x; d < D; d += blockDim.x) sig[d] = rotation_sign(a.seed, u, d);
+  __syncthreads();
+  rotate_tile_to_smem<D, TX>(X, T, t0, sig, xs);
+  __syncthreads();
+  TileFrag<D> xf;
+  frag_from_smem<D>(xs, xf);
+  __syncthreads();
+
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const Cands& cd = a.cand;
+  const bf16* U = a.U + (long long)u * a.sU;
+  constexpr int NT = D / 8;
+  double* out = a.partial + (((long long)u * a.cv.S + s) * a.tiles + tile) * (long long)(cd.nD * cd.nT * cd.nB);
+
+  for (int iD = 0; iD < cd.nD; ++iD) {
+    const bf16* P = a.P + (long long)u * a.sP_unit + iD * a.sP_rd + (long long)s * a.rTmax * D;
+    float acc[NT][4];
+#pragma unroll
+    for (int j = 0; j < NT; ++j)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[j][e] = 0.f;
+
+    auto epi = [&](int iT) {
+      float err[MAXC];
+#pragma unroll
+      for (int ib = 0; ib < MAXC; ++ib) err[ib] = 0.f;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+#pragma unroll
+        for (int m = 0; m < D / 16; ++m) {
+          float r[4];
+          block_vals<D>(xf, acc, h, m, r);
+          float mn = fminf(fminf(r[0], r[1]), fminf(r[2], r[3]));
+          float mx = fmaxf(fmaxf(r[0], r[1]), fmaxf(r[2], r[3]));
+          quad_minmax(mn, mx);
+          float lo = fp16_rd(mn);
+          float dd[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) dd[i] = r[i] - lo;
+#pragma unroll
+          for (int ib = 0; ib < MAXC; ++ib) {
+            if (ib >= cd.nB) break;
+            int b = cd.bits[ib];
+            if (b == 0) {
+#pragma unroll
+              for (int i = 0; i < 4; ++i) err[ib] = fmaf(r[i], r[i], err[ib]);
+              continue;
+            }
+            int levels = (1 << b) - 1;
+            float step = quant_step(mx, lo, levels, 1.0f / (float)levels);
+            if (!(isfinite(lo) && isfinite(step))) {
+              err[ib] = INFINITY;
+              continue;
+            }
+            float inv = step > 0.f ? 1.0f / step : 0.f;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              float code = rne_int(dd[i] * inv);
+              float e = fmaf(-code, step, dd[i]);
+              err[ib] = fmaf(e, e, err[ib]);
+            }
+          }
+        }
+      }
+      // reduce over the warp, then over the 4 warps in fixed order (fp64)
+#pragma unroll
+      for (int ib = 0; ib < MAXC; ++ib) {
+        if (ib >= cd.nB) break;
+        float v = err[ib];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+        if (lane == 0) red[warp][ib] = v;
+      }
+      __syncthreads();
+      if (threadIdx.x < cd.nB) {
+        double v = 0.0;
+        for (int w = 0; w < 4; ++w) v += (double)red[w][threadIdx.x];
+        out[(iD * cd.nT + iT) * cd.nB + threadIdx.x] = v;
+      }
+      __syncthreads();
+    };
+    recon_walk<D>(stages, U, a.ldU, T, t0, P, cd.rT[cd.nT - 1], cd.rT, cd.nT, acc, epi);
+  }
+}
+
+template <int D>
+inline size_t table_smem() {
+  return (size_t)TROWS * (D + 4) * 4 + 2 * (size_t)ReconSmem<D>::STAGE * sizeof(bf16);
+}
+
+// ---------------------------------------------------------------------------------------
+// unit record header (device layout of the compressed blob; 64 bytes each)
+// ---------------------------------------------------------------------------------------
+struct BlobHeader {      // 64 bytes at offset 0
+  uint32_t magic, version, n_units, status;
+  int32_t n_layers, n_heads, n_tokens, head_dim, layers_per_group, dtype, block, reserved;
+  uint64_t seed, total_bytes;
+};
+struct UnitHeader {      // 64 bytes per unit after the global header
+  int32_t r_T, r_D, bits, choice;
+  uint64_t off_U, off_W, off_C, off_codes, off_scales;
+  double distortion;
+};
+static_assert(sizeof(BlobHeader) == 64, "header");
+static_assert(sizeof(UnitHeader) == 64, "unit header");
+constexpr uint32_t kMagic = 0x544C4F4Au;  // "JOLT"
+constexpr uint32_t kVersion = 1u;
+
+// ---------------------------------------------------------------------------------------
+// encode kernel: chosen (r_T, r_D, b) per unit from the blob's unit table
+// grid (tiles, S, units)
+// ---------------------------------------------------------------------------------------
+struct EncodeArgs {
+  CacheView cv;
+  const bf16* U;
+  long long ldU, sU;
+  const bf16* P;
+  long long sP_unit, sP_rd;
+  int rTmax;
+  Cands cand;
+  uint64_t seed;
+  unsigned char* blob;
+};
+
+template <int D, typename TX>
+__global__ void __launch_bounds__(TTHREADS) encode_kernel(EncodeArgs a) {
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  float* xs = reinterpret_cast<float*>(smem_raw);
+  bf16* stages = reinterpret_cast<bf16*>(smem_raw + TROWS * (D + 4) * 4);
+  __shared__ float sig[D];
+
+  const int tile = blockIdx.x, s = blockIdx.y, u = blockIdx.z;
+  const int T = a.cv.T;
+  const int t0 = tile * TROWS;
+  const UnitHeader uh = reinterpret_cast<const UnitHeader*>(a.blob + sizeof(BlobHeader))[u];
+  const BlobHeader* gh = reinterpret_cast<const BlobHeader*>(a.blob);
+  if (gh->status != 0) return;
+  const int b = uh.bits;
+  if (b == 0) return;
+  int iD = 0;
+  while (iD < a.cand.nD && a.cand.rD[iD] != uh.r_D) ++iD;
+
+  const TX* X = reinterpret_cast<const TX*>(a.cv.unit_ptr(u)) + (long long)s * T * D;
+  for (int d = threadIdx.x; d < D; d += blockDim.x) sig[d] = rotation_sign(a.seed, u, d);
+  __syncthreads();
+  rotate_tile_to_smem<D, TX>(X, T, t0, sig, xs);
+  __syncthreads();
+  TileFrag<D> xf;
+  frag_from_smem<D>(xs, xf);
+  __syncthreads();
+
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  constexpr int NT = D / 8;
+  const bf16* U = a.U + (long long)u * a.sU;
+  const bf16* P = a.P + (long long)u * a.sP_unit + iD * a.sP_rd + (long long)s * a.rTmax * D;
+  float acc[NT][4];
+#pragma unroll
+  for (int j = 0; j < NT; ++j)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) acc[j][e] = 0.f;
+
+  const int levels = (1 << b) - 1;
+  const float inv_levels = 1.0f / (float)levels;
+  unsigned char* codes = a.blob + uh.off_codes;
+  __half2* scales = reinterpret_cast<__half2*>(a.blob + uh.off_scales);
+  const int q = lane & 3;
+
+  auto epi = [&](int) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      int t = t0 + warp * 16 + (lane >> 2) + h * 8;
+#pragma unroll
+      for (int m = 0; m < D / 16; ++m) {
+        float r[4];
+        block_vals<D>(xf, acc, h, m, r);
+        float mn = fminf(fminf(r[0], r[1]), fminf(r[2], r[3]));
+        float mx = fmaxf(fmaxf(r[0], r[1]), fmaxf(r[2], r[3]));
+        quad_minmax(mn, mx);
+        float lo = fp16_rd(mn);
+        float step = quant_step(mx, lo, levels, inv_levels);
+        float inv = step > 0.f ? 1.0f / step : 0.f;
+        // columns inside the block held by this thread: 2q, 2q+1, 8+2q, 9+2q
+        uint32_t w[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          int col = (i >> 1) * 8 + 2 * q + (i & 1);
+          float c = rne_int((r[i] - lo) * inv);
+          c = fminf(fmaxf(c, 0.f), (float)levels);
+          uint32_t code = (uint32_t)c;
+          int pos = col * b;
+          w[pos >> 5] |= code << (pos & 31);
+          if ((pos & 31) + b > 32) w[(pos >> 5) + 1] |= code >> (32 - (pos & 31));
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          w[i] |= __shfl_xor_sync(0xffffffffu, w[i], 1);
+          w[i] |= __shfl_xor_sync(0xffffffffu, w[i], 2);
+        }
+        if (q == 0 && t < T) {
+          long long blk = ((long long)s * T + t) * (D / 16) + m;
+          unsigned char* dst = codes + blk * (2 * b);
+          for (int byte = 0; byte < 2 * b; ++byte) dst[byte] = (unsigned char)(w[byte >> 2] >> ((byte & 3) * 8));
+          scales[blk] = __halves2half2(__float2half_rn(lo), __float2half_rn(step));
+        }
+      }
+    }
+  };
+  int cut = uh.r_T;
+  recon_walk<D>(stages, U, a.ldU, T, t0, P, cut, &cut, 1, acc, epi);
+}
+
+// ---------------------------------------------------------------------------------------
+// decode kernel: X_hat = (U P' + dequant) Phi^T ; grid (tiles, S, units)
+// P' here is the decoder's own operator built from the stored core and feature factor
+// ---------------------------------------------------------------------------------------
+struct DecodeArgs {
+  const unsigned char* blob;
+  const bf16* U;         // [unit][T][ldU] aligned copy of the stored token factors
+  long long ldU, sU;
+  const bf16* P;         // [unit][S][rTmax][D]
+  long long sP_unit;
+  int rTmax;
+  int T, S, Lg;
+  uint64_t seed;
+  void* k_out;
+  void* v_out;
+  int out_f32;
+};
+
+template <int D>
+__device__ __forceinline__ void fwht_frag_row(TileFrag<D>& f, int h) {
+  // butterflies inside the thread: stride 1 (e) and strides 8..D/2 (n8 tile index)
+  constexpr int NT = D / 8;
+#pragma unroll
+  for (int j = 0; j < NT; ++j) {
+    float x0 = f.v[h][j][0], x1 = f.v[h][j][1];
+    f.v[h][j][0] = x0 + x1;
+    f.v[h][j][1] = x0 - x1;
+  }
+  // strides 2 and 4 across the lane quad
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int sh = 1; sh <= 2; sh <<= 1) {
+    bool upper = (lane & sh) != 0;
+#pragma unroll
+    for (int j = 0; j < NT; ++j)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        float mine = f.v[h][j][e];
+        float other = __shfl_xor_sync(0xffffffffu, mine, sh);
+        f.v[h][j][e] = upper ? other - mine : mine + other;
+      }
+  }
+#pragma unroll
+  for (int hs = 1; hs < NT; hs <<= 1) {
+#pragma unroll
+    for (int j = 0; j < NT; ++j) {
+      if (j & hs) continue;
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        float x0 = f.v[h][j][e], x1 = f.v[h][j + hs][e];
+        f.v[h][j][e] = x0 + x1;
+        f.v[h][j + hs][e] = x0 - x1;
+      }
+    }
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(TTHREADS) decode_kernel(DecodeArgs a) {
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  bf16* stages = reinterpret_cast<bf16*>(smem_raw);
+  __shared__ float sig[D];
+  const int tile = blockIdx.x, s = blockIdx.y, u = blockIdx.z;
+  const int T = a.T;
+  const int t0 = tile * TROWS;
+  const UnitHeader uh = reinterpret_cast<const UnitHeader*>(a.blob + sizeof(BlobHeader))[u];
+  for (int d = threadIdx.x; d < D; d += blockDim.x) sig[d] = rotation_sign(a.seed, u, d);
+  __syncthreads();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  constexpr int NT = D / 8;
+  const bf16* U = a.U + (long long)u * a.sU;
+  const bf16* P = a.P + (long long)u * a.sP_unit + (long long)s * a.rTmax * D;
+  float acc[NT][4];
+#pragma unroll
+  for (int j = 0; j < NT; ++j)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) acc[j][e] = 0.f;
+  int cut = uh.r_T;
+  recon_walk<D>(stages, U, a.ldU, T, t0, P, uh.r_T, &cut, 1, acc, [](int) {});
+
+  TileFrag<D> f;
+  const int b = uh.bits;
+  const int q = lane & 3;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    int t = t0 + warp * 16 + (lane >> 2) + h * 8;
+    bool valid = t < T;
+#pragma unroll
+    for (int m = 0; m < D / 16; ++m) {
+      float deq[4] = {0.f, 0.f, 0.f, 0.f};
+      if (b > 0 && valid) {
+        long long blk = ((long long)s * T + t) * (D / 16) + m;
+        const unsigned char* src = a.blob + uh.off_codes + blk * (2 * b);
+        uint32_t w[4] = {0u, 0u, 0u, 0u};
+        for (int byte = 0; byte < 2 * b; ++byte) w[byte >> 2] |= (uint32_t)src[byte] << ((byte & 3) * 8);
+        __half2 sc = reinterpret_cast<const __half2*>(a.blob + uh.off_scales)[blk];
+        float lo = __low2float(sc), step = __high2float(sc);
+        const uint32_t mask = (1u << b) - 1u;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          int col = (i >> 1) * 8 + 2 * q + (i & 1);
+          int pos = col * b;
+          uint32_t code = w[pos >> 5] >> (pos & 31);
+          if ((pos & 31) + b > 32) code |= w[(pos >> 5) + 1] << (32 - (pos & 31));
+          code &= mask;
+          deq[i] = fmaf((float)code, step, lo);
+        }
+      }
+      f.v[h][2 * m][0] = acc[2 * m][h * 2 + 0] + deq[0];
+      f.v[h][2 * m][1] = acc[2 * m][h * 2 + 1] + deq[1];
+      f.v[h][2 * m + 1][0] = acc[2 * m + 1][h * 2 + 0] + deq[2];
+      f.v[h][2 * m + 1][1] = acc[2 * m + 1][h * 2 + 1] + deq[3];
+    }
+    fwht_frag_row<D>(f, h);
+    if (!valid) continue;
+    const float sc = (float)(1.0 / sqrt((double)D));
+    const int g = u >> 1;
+    long long row_off = ((long long)s * T + t) * D;          // row inside the unit
+    long long unit_off = (long long)g * a.S * T * D;         // unit inside K or V
+    void* outp = (u & 1) ? a.v_out : a.k_out;
+#pragma unroll
+    for (int j = 0; j < NT; ++j) {
+      int c = j * 8 + 2 * q;
+      float y0 = f.v[h][j][0] * sc * sig[c];
+      float y1 = f.v[h][j][1] * sc * sig[c + 1];
+      long long off = unit_off + row_off + c;
+      if (a.out_f32) {
+        float2* o = reinterpret_cast<float2*>(reinterpret_cast<float*>(outp) + off);
+        *o = make_float2(y0, y1);
+      } else {
+        __nv_bfloat162* o = reinterpret_cast<__nv_bfloat162*>(reinterpret_cast<bf16*>(outp) + off);
+        *o = __floats2bfloat162_rn(y0, y1);
+      }
+    }
+  }
+}
+
+template <int D>
+inline size_t decode_smem() {
+  return 2 * (size_t)ReconSmem<D>::STAGE * sizeof(bf16);
+}
+
+}  // namespace jolt

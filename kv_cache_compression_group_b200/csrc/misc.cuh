@@ -1,0 +1,494 @@
+// Small kernels around the factor, allocation and packing steps.
+#pragma once
+
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace jolt {
+
+// out[b][i] = sum_s part[b][s][i]  in a fixed order (s ascending), fp64
+template <typename TP>
+__global__ void reduce_splits_kernel(const TP* part, double* out, int nbatch, int nsplit, long long n) {
+  long long total = (long long)nbatch * n;
+  for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < total;
+       idx += (long long)gridDim.x * blockDim.x) {
+    long long b = idx / n, i = idx - b * n;
+    const TP* p = part + b * nsplit * n + i;
+    double acc = 0.0;
+    for (int s = 0; s < nsplit; ++s) acc += (double)p[(long long)s * n];
+    out[idx] = acc;
+  }
+}
+
+// every diagonal entry of the unit's feature Gram must be finite (a NaN/Inf anywhere in
+// the cache reaches the diagonal through x*x)
+__global__ void gram_diag_check_kernel(const double* G, int n, int nunits, uint32_t* status) {
+  int u = blockIdx.x;
+  if (u >= nunits) return;
+  for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    double v = G[(long long)u * n * n + (long long)i * n + i];
+    if (!isfinite(v)) raise_status(status, DEV_ERR_NONFINITE);
+  }
+}
+
+// Leading r eigenvectors in descending eigenvalue order (ties: lower original index first)
+// from an ascending eigen-solver output (eigenvectors in columns, column-major, lda),
+// the entry of largest magnitude made positive (ties: lowest row).
+// Writes row-major n x ldo fp32 (optional), bf16 (optional) and the eigenvalues (optional).
+__global__ void eig_select_kernel(const double* vals, const double* vecs, int n, long long lda,
+                                  long long sval, long long svec, int r, float* out_f32, bf16* out_bf16,
+                                  long long ldo, long long sout, double* out_vals) {
+  const int j = blockIdx.x, u = blockIdx.y;
+  const double* w = vals + (long long)u * sval;
+  // the j-th largest: with ties broken towards the lower index, descending order of an
+  // ascending list is position n-1-j unless equal neighbours exist; resolve exactly.
+  __shared__ int src;
+  if (threadIdx.x == 0) {
+    // count of entries strictly greater, then pick among equals the lowest index
+    int pos = n - 1 - j;
+    double v = w[pos];
+    int first_eq = pos;
+    while (first_eq > 0 && w[first_eq - 1] == v) --first_eq;
+    int last_eq = pos;
+    while (last_eq < n - 1 && w[last_eq + 1] == v) ++last_eq;
+    int rank_in_group = (last_eq - pos);  // 0 for the first (largest-position) in descending walk
+    src = first_eq + rank_in_group;
+    if (out_vals) out_vals[(long long)u * r + j] = v;
+  }
+  __syncthreads();
+  const double* col = vecs + (long long)u * svec + (long long)src * lda;
+  __shared__ double bestv[256];
+  __shared__ int besti[256];
+  double bv = -1.0;
+  int bi = 0x7fffffff;
+  for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    double a = fabs(col[i]);
+    if (a > bv || (a == bv && i < bi)) { bv = a; bi = i; }
+  }
+  bestv[threadIdx.x] = bv;
+  besti[threadIdx.x] = bi;
+  __syncthreads();
+  for (int st = blockDim.x / 2; st > 0; st >>= 1) {
+    if ((int)threadIdx.x < st) {
+      double ov = bestv[threadIdx.x + st];
+      int oi = besti[threadIdx.x + st];
+      if (ov > bestv[threadIdx.x] || (ov == bestv[threadIdx.x] && oi < besti[threadIdx.x])) {
+        bestv[threadIdx.x] = ov;
+        besti[threadIdx.x] = oi;
+      }
+    }
+    __syncthreads();
+  }
+  const double sgn = col[besti[0]] < 0 ? -1.0 : 1.0;
+  for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    double v = sgn * col[i];
+    long long o = (long long)u * sout + (long long)i * ldo + j;
+    if (out_f32) out_f32[o] = (float)v;
+    if (out_bf16) out_bf16[o] = __float2bfloat16_rn((float)v);
+  }
+}
+
+// Same sign convention on the columns of a row-major fp32 matrix (in place), plus bf16 copy
+__global__ void col_sign_fix_kernel(float* A, long long lda, long long sA, int n, int r, bf16* out_bf16,
+                                    long long ldo, long long so) {
+  const int j = blockIdx.x, u = blockIdx.y;
+  float* a = A + (long long)u * sA;
+  __shared__ float bestv[256];
+  __shared__ int besti[256];
+  float bv = -1.f;
+  int bi = 0x7fffffff;
+  for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    float x = fabsf(a[(long long)i * lda + j]);
+    if (x > bv || (x == bv && i < bi)) { bv = x; bi = i; }
+  }
+  bestv[threadIdx.x] = bv;
+  besti[threadIdx.x] = bi;
+  __syncthreads();
+  for (int st = blockDim.x / 2; st > 0; st >>= 1) {
+    if ((int)threadIdx.x < st) {
+      float ov = bestv[threadIdx.x + st];
+      int oi = besti[threadIdx.x + st];
+      if (ov > bestv[threadIdx.x] || (ov == bestv[threadIdx.x] && oi < besti[threadIdx.x])) {
+        bestv[threadIdx.x] = ov;
+        besti[threadIdx.x] = oi;
+      }
+    }
+    __syncthreads();
+  }
+  const float sgn = a[(long long)besti[0] * lda + j] < 0 ? -1.f : 1.f;
+  __syncthreads();
+  for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    float v = sgn * a[(long long)i * lda + j];
+    a[(long long)i * lda + j] = v;
+    if (out_bf16) out_bf16[(long long)u * so + (long long)i * ldo + j] = __float2bfloat16_rn(v);
+  }
+}
+
+// FlashJoLT test matrix: Omega[m][j] = bf16(gaussian(seed, OMEGA stream of unit, m*k + j)),
+// zero in the padding columns k <= j < ld
+__global__ void omega_kernel(bf16* om, int M, int k, long long ld, long long sunit, uint64_t seed, int unit0,
+                             int nunits) {
+  long long total = (long long)nunits * M * ld;
+  for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < total;
+       idx += (long long)gridDim.x * blockDim.x) {
+    long long u = idx / ((long long)M * ld);
+    long long rem = idx - u * M * ld;
+    long long m = rem / ld, j = rem - m * ld;
+    // one rounding from double to bf16 (round to nearest even)
+    om[u * sunit + m * ld + j] =
+        j < k ? __double2bfloat16(gaussian(seed, stream_id(kStreamOmega, unit0 + (int)u), (uint64_t)(m * k + j)))
+              : __float2bfloat16_rn(0.f);
+  }
+}
+
+// fp32 -> bf16 hi + bf16 lo with hi + lo ~ x (2^-17 relative)
+__global__ void split_bf16_kernel(const float* x, bf16* hi, bf16* lo, long long n) {
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
+    float v = x[i];
+    bf16 h = __float2bfloat16_rn(v);
+    hi[i] = h;
+    lo[i] = __float2bfloat16_rn(v - __bfloat162float(h));
+  }
+}
+
+// rows of fp32 [nrows][D] -> bf16(FWHT(sigma * row) / sqrt(D)) ; sigma of unit (row / rows_per_unit)
+template <int D>
+__global__ void rotate_rows_kernel(const float* in, bf16* out, long long nrows, long long rows_per_unit,
+                                   const int* unit_of_batch, uint64_t seed) {
+  long long r = blockIdx.x * (long long)blockDim.x + threadIdx.x;
+  if (r >= nrows) return;
+  int u = unit_of_batch[r / rows_per_unit];
+  float v[D];
+  const float* row = in + r * D;
+#pragma unroll
+  for (int d = 0; d < D; ++d) v[d] = row[d] * rotation_sign(seed, u, d);
+  fwht_regs<D>(v);
+  const float sc = (float)(1.0 / sqrt((double)D));
+  bf16* o = out + r * D;
+#pragma unroll
+  for (int d = 0; d < D; ++d) o[d] = __float2bfloat16_rn(v[d] * sc);
+}
+
+// zero the strict upper triangle of column-major n x n matrices (lda)
+__global__ void tril_zero_kernel(double* A, int n, long long lda, long long sA, int nbatch) {
+  long long total = (long long)nbatch * n * n;
+  for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < total;
+       idx += (long long)gridDim.x * blockDim.x) {
+    long long b = idx / ((long long)n * n);
+    long long rem = idx - b * n * n;
+    long long col = rem / n, row = rem - col * n;
+    if (row < col) A[b * sA + col * lda + row] = 0.0;
+  }
+}
+
+__global__ void info_check_kernel(const int* info, int n, uint32_t* status, uint32_t bits) {
+  int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n && info[i] != 0) raise_status(status, bits);
+}
+
+// fp32 -> fp64 copy (for the eigen solver input) with optional scale per column
+__global__ void f32_to_f64_kernel(const float* in, double* out, long long n) {
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x)
+    out[i] = (double)in[i];
+}
+
+// V[:, j] *= 1/sqrt(lambda_j) (row-major n x ld fp32) and flag non-positive eigenvalues
+__global__ void scale_cols_kernel(float* V, const double* lam, int n, int r, long long ld, long long sV,
+                                  long long slam, int nunits, uint32_t* status) {
+  long long total = (long long)nunits * n * r;
+  for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < total;
+       idx += (long long)gridDim.x * blockDim.x) {
+    long long u = idx / ((long long)n * r);
+    long long rem = idx - u * n * r;
+    long long i = rem / r, j = rem - i * r;
+    double l = lam[u * slam + j];
+    if (!(l > 0.0)) {
+      raise_status(status, DEV_ERR_FACTOR);
+      l = 1.0;
+    }
+    V[u * sV + i * ld + j] = (float)((double)V[u * sV + i * ld + j] / sqrt(l));
+  }
+}
+
+// ------------------------------------------------------------------------------------------
+// distortion table finalisation, byte table and the Lagrangian dual
+// ------------------------------------------------------------------------------------------
+// table[u][(iT*nD + iD)*nB + ib] = sum over (slice, tile) of partial[u][s][tile][(iD*nT+iT)*nB+ib]
+__global__ void table_reduce_kernel(const double* partial, double* table, int nunits, int S, int tiles, int nT,
+                                    int nD, int nB) {
+  const int nc = nT * nD * nB;
+  int idx = blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= nunits * nc) return;
+  int u = idx / nc, c = idx - u * nc;
+  int ib = c % nB, iD = (c / nB) % nD, iT = c / (nB * nD);
+  int pc = (iD * nT + iT) * nB + ib;
+  const double* p = partial + (long long)u * S * tiles * nc + pc;
+  double acc = 0.0;
+  for (long long st = 0; st < (long long)S * tiles; ++st) acc += p[st * nc];
+  table[idx] = acc;
+}
+
+__host__ __device__ inline unsigned long long pad16u(unsigned long long n) { return (n + 15ull) / 16ull * 16ull; }
+
+// stored bytes of one unit for (r_T, r_D, b): U, W, core in bf16, codes (2b bytes per block
+// of 16) and one fp16 (lo, step) pair per block, each array padded to 16 bytes
+__host__ __device__ inline unsigned long long unit_payload_bytes(int T, int D, int S, int rT, int rD, int b) {
+  unsigned long long n = pad16u(2ull * T * rT) + pad16u(2ull * D * rD) + pad16u(2ull * S * rT * rD);
+  if (b > 0) {
+    unsigned long long nblk = (unsigned long long)S * T * (D / 16);
+    n += pad16u(nblk * 2ull * b) + pad16u(nblk * 4ull);
+  }
+  return n;
+}
+
+__global__ void bytes_table_kernel(unsigned long long* B, int nunits, int T, int D, int S, Cands cd) {
+  const int nc = cd.nT * cd.nD * cd.nB;
+  int idx = blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= nunits * nc) return;
+  int c = idx % nc;
+  int ib = c % cd.nB, iD = (c / cd.nB) % cd.nD, iT = c / (cd.nB * cd.nD);
+  B[idx] = unit_payload_bytes(T, D, S, cd.rT[iT], cd.rD[iD], cd.bits[ib]);
+}
+
+// argmin_c D[c] + lam*B[c] with two separate roundings; ties -> fewer bytes -> lower index
+__device__ __forceinline__ int lagrangian_argmin(const double* Dr, const unsigned long long* Br, int nc, double lam) {
+  double bv = 0.0;
+  unsigned long long bb = 0ull;
+  int bc = -1;
+  for (int c = 0; c < nc; ++c) {
+    double v = __dadd_rn(Dr[c], __dmul_rn(lam, (double)Br[c]));
+    bool better = (bc < 0) || (v < bv) || (v == bv && Br[c] < bb);
+    // NaN never occurs: D is finite or +inf and lam*B is finite or +inf
+    if (better) { bv = v; bb = Br[c]; bc = c; }
+  }
+  return bc;
+}
+
+struct AllocArgs {
+  const double* D;
+  const unsigned long long* B;
+  int nunits, nc;
+  unsigned long long budget;       // bytes available to the payload (headers already taken out)
+  int* choice;                     // [nunits]
+  double* lambda;                  // [1]
+  uint32_t* status;
+  // blob filling (optional)
+  unsigned char* blob;
+  unsigned long long blob_cap;
+  unsigned long long header_bytes;
+  int T, D_, S;
+  Cands cd;
+  BlobHeader hdr;                  // global header prototype (passed by value)
+  const int32_t* forced;           // optional caller choices: skip the search, fill the headers
+};
+
+__device__ unsigned long long alloc_F(const AllocArgs& a, double lam, int* sch, unsigned long long* sB) {
+  for (int u = threadIdx.x; u < a.nunits; u += blockDim.x) {
+    int c = lagrangian_argmin(a.D + (long long)u * a.nc, a.B + (long long)u * a.nc, a.nc, lam);
+    sch[u] = c;
+    sB[u] = a.B[(long long)u * a.nc + c];
+  }
+  __syncthreads();
+  unsigned long long tot = 0ull;
+  for (int u = 0; u < a.nunits; ++u) tot += sB[u];
+  __syncthreads();
+  return tot;
+}
+
+// one CTA: the bisection on lambda, then the unit headers and byte offsets of the blob
+__global__ void allocate_kernel(AllocArgs a) {
+  extern __shared__ unsigned char sm[];
+  int* sch = reinterpret_cast<int*>(sm);
+  unsigned long long* sB = reinterpret_cast<unsigned long long*>(sm + ((a.nunits * 4 + 15) / 16) * 16);
+  __shared__ double s_lam;
+  __shared__ int s_state;  // 0 ok, 1 infeasible
+  // feasibility: every unit at its fewest-bytes choice
+  if (a.forced) {
+    for (int u = threadIdx.x; u < a.nunits; u += blockDim.x) sch[u] = a.forced[u];
+    __syncthreads();
+    if (threadIdx.x == 0) s_lam = 0.0;
+    __syncthreads();
+  }
+  if (threadIdx.x == 0 && !a.forced) {
+    unsigned long long minB = 0ull;
+    for (int u = 0; u < a.nunits; ++u) {
+      unsigned long long m = ~0ull;
+      for (int c = 0; c < a.nc; ++c) m = min(m, a.B[(long long)u * a.nc + c]);
+      minB += m;
+    }
+    s_state = minB > a.budget ? 1 : 0;
+  }
+  if (a.forced && threadIdx.x == 0) s_state = 0;
+  __syncthreads();
+  if (s_state) {
+    if (threadIdx.x == 0) {
+      raise_status(a.status, DEV_ERR_INFEASIBLE);
+      a.lambda[0] = __longlong_as_double(0x7ff0000000000000LL);
+      if (a.blob) {
+        BlobHeader h = a.hdr;
+        h.status = DEV_ERR_INFEASIBLE;
+        h.total_bytes = 0;
+        *reinterpret_cast<BlobHeader*>(a.blob) = h;
+      }
+    }
+    return;
+  }
+  double lam = 0.0;
+  unsigned long long F = a.forced ? 0ull : alloc_F(a, 0.0, sch, sB);
+  if (!a.forced && F > a.budget) {
+    double lo = 0.0, hi = 1.0;
+    for (int it = 0; it < 2100; ++it) {
+      if (alloc_F(a, hi, sch, sB) <= a.budget) break;
+      hi = __dmul_rn(hi, 2.0);
+    }
+    for (int it = 0; it < 200; ++it) {
+      double mid = __dadd_rn(lo, __dmul_rn(__dadd_rn(hi, -lo), 0.5));
+      if (alloc_F(a, mid, sch, sB) <= a.budget) hi = mid;
+      else lo = mid;
+    }
+    lam = hi;
+    F = alloc_F(a, hi, sch, sB);
+  }
+  if (threadIdx.x == 0) s_lam = lam;
+  __syncthreads();
+  if (!a.forced) {
+    for (int u = threadIdx.x; u < a.nunits; u += blockDim.x) a.choice[u] = sch[u];
+    if (threadIdx.x == 0) a.lambda[0] = s_lam;
+  }
+  if (!a.blob || threadIdx.x != 0) return;
+  // unit headers and payload offsets, in unit order
+  unsigned long long off = a.header_bytes;
+  UnitHeader* uh = reinterpret_cast<UnitHeader*>(a.blob + sizeof(BlobHeader));
+  for (int u = 0; u < a.nunits; ++u) {
+    int c = sch[u];
+    int ib = c % a.cd.nB, iD = (c / a.cd.nB) % a.cd.nD, iT = c / (a.cd.nB * a.cd.nD);
+    int rT = a.cd.rT[iT], rD = a.cd.rD[iD], b = a.cd.bits[ib];
+    UnitHeader h;
+    h.r_T = rT;
+    h.r_D = rD;
+    h.bits = b;
+    h.choice = c;
+    h.off_U = off;
+    h.off_W = h.off_U + pad16u(2ull * a.T * rT);
+    h.off_C = h.off_W + pad16u(2ull * a.D_ * rD);
+    h.off_codes = h.off_C + pad16u(2ull * a.S * rT * rD);
+    unsigned long long nblk = (unsigned long long)a.S * a.T * (a.D_ / 16);
+    h.off_scales = h.off_codes + (b > 0 ? pad16u(nblk * 2ull * b) : 0ull);
+    h.distortion = a.D[(long long)u * a.nc + c];
+    uh[u] = h;
+    off += a.B[(long long)u * a.nc + c];
+  }
+  BlobHeader g = a.hdr;
+  g.total_bytes = off;
+  g.status = off > a.blob_cap ? DEV_ERR_CAPACITY : 0u;
+  if (g.status) raise_status(a.status, DEV_ERR_CAPACITY);
+  *reinterpret_cast<BlobHeader*>(a.blob) = g;
+}
+
+// copy the chosen prefixes of U (T x r_T), W (D x r_D) and the core (S x r_T x r_D) into the blob
+__global__ void copy_factors_kernel(unsigned char* blob, const bf16* U, long long ldU, long long sU,
+                                    const bf16* W, long long ldW, long long sW, const bf16* C, long long ldC,
+                                    long long sC_slice, long long sC_unit, int T, int D, int S) {
+  const int u = blockIdx.y;
+  const BlobHeader* gh = reinterpret_cast<const BlobHeader*>(blob);
+  if (gh->status != 0) return;
+  const UnitHeader h = reinterpret_cast<const UnitHeader*>(blob + sizeof(BlobHeader))[u];
+  bf16* oU = reinterpret_cast<bf16*>(blob + h.off_U);
+  bf16* oW = reinterpret_cast<bf16*>(blob + h.off_W);
+  bf16* oC = reinterpret_cast<bf16*>(blob + h.off_C);
+  long long nU = (long long)T * h.r_T, nW = (long long)D * h.r_D, nC = (long long)S * h.r_T * h.r_D;
+  long long tot = nU + nW + nC;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < tot; i += (long long)gridDim.x * blockDim.x) {
+    if (i < nU) {
+      long long t = i / h.r_T, j = i - t * h.r_T;
+      oU[i] = U[u * sU + t * ldU + j];
+    } else if (i < nU + nW) {
+      long long k = i - nU;
+      long long d = k / h.r_D, j = k - d * h.r_D;
+      oW[k] = W[u * sW + d * ldW + j];
+    } else {
+      long long k = i - nU - nW;
+      long long s = k / ((long long)h.r_T * h.r_D);
+      long long rem = k - s * h.r_T * h.r_D;
+      long long r = rem / h.r_D, q = rem - r * h.r_D;
+      oC[k] = C[u * sC_unit + s * sC_slice + r * ldC + q];
+    }
+  }
+}
+
+__global__ void iota_kernel(int* out, int n) {
+  int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) out[i] = i;
+}
+
+// device-side errors of the factor stage go into the blob header status word
+__global__ void fold_status_kernel(const uint32_t* status, unsigned char* blob) {
+  BlobHeader* h = reinterpret_cast<BlobHeader*>(blob);
+  uint32_t s = *status;
+  if (s) h->status |= s;
+}
+
+// dense rows x cols bf16 (ld = cols) -> rows x ldo, zero padded columns
+__global__ void copy2d_kernel(const bf16* src, long long rows, int cols, bf16* dst, long long ldo) {
+  long long tot = rows * ldo;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < tot; i += (long long)gridDim.x * blockDim.x) {
+    long long r = i / ldo, j = i - r * ldo;
+    dst[i] = j < cols ? src[r * cols + j] : __float2bfloat16_rn(0.f);
+  }
+}
+
+// copy a unit's U from the blob (T x r_T) into an aligned workspace (T x ld)
+__global__ void unpack_u_kernel(const unsigned char* blob, bf16* out, long long ld, long long sunit, int T) {
+  const int u = blockIdx.y;
+  const UnitHeader h = reinterpret_cast<const UnitHeader*>(blob + sizeof(BlobHeader))[u];
+  const bf16* src = reinterpret_cast<const bf16*>(blob + h.off_U);
+  long long tot = (long long)T * ld;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < tot; i += (long long)gridDim.x * blockDim.x) {
+    long long t = i / ld, j = i - t * ld;
+    out[u * sunit + i] = j < h.r_T ? src[t * h.r_T + j] : __float2bfloat16_rn(0.f);
+  }
+}
+
+// per-unit sums of squares of X and of X - Y over one of K / V (grid (nblk, groups));
+// partial sums land at part[(unit * nblk + block) * 2 + {0, 1}] with unit = 2 g + kv
+template <typename TX, typename TY>
+__global__ void frob_partial_kernel(const TX* X, const TY* Y, long long n_per_unit, int kv, double* part, int nblk) {
+  const int g = blockIdx.y, u = 2 * g + kv;
+  __shared__ double s1[256], s2[256];
+  double a = 0.0, b = 0.0;
+  const TX* x = X + (long long)g * n_per_unit;
+  const TY* y = Y ? Y + (long long)g * n_per_unit : nullptr;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n_per_unit; i += (long long)nblk * blockDim.x) {
+    double xv = (double)ld_as_float(x + i);
+    a += xv * xv;
+    if (y) {
+      double d = xv - (double)ld_as_float(y + i);
+      b += d * d;
+    }
+  }
+  s1[threadIdx.x] = a;
+  s2[threadIdx.x] = b;
+  __syncthreads();
+  for (int st = blockDim.x / 2; st > 0; st >>= 1) {
+    if ((int)threadIdx.x < st) {
+      s1[threadIdx.x] += s1[threadIdx.x + st];
+      s2[threadIdx.x] += s2[threadIdx.x + st];
+    }
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    part[((long long)u * nblk + blockIdx.x) * 2 + 0] = s1[0];
+    part[((long long)u * nblk + blockIdx.x) * 2 + 1] = s2[0];
+  }
+}
+
+__global__ void frob_final_kernel(const double* part, int nunits, int nblk, double* sq) {
+  int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= nunits * 2) return;
+  int u = i >> 1, w = i & 1;
+  double acc = 0.0;
+  for (int b = 0; b < nblk; ++b) acc += part[((long long)u * nblk + b) * 2 + w];
+  sq[i] = acc;
+}
+
+}  // namespace jolt
