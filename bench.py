@@ -1,0 +1,382 @@
+"""KV compress throughput of the JoLT / FlashJoLT library on a Mistral-7B-shaped cache.
+
+One step = jolt_compress of the whole cache (K and V, 32 layers x 8 KV heads x 1024 tokens
+x 128 features, bf16) at the 2x budget, then again at the 3x budget.  `value` is input
+GB/s over the timed steps (inputs resident in HBM, L2 flushed between steps), `e2e` is
+the same metric through the public API with the caches copied in from pinned host memory
+and the blobs read back every step.  For N > 1 every rank compresses its own cache (weak
+scaling; the units of different caches are independent, so no collective is involved).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--method randomized|exact]
+  python bench.py --impl reference ...   # the float64 CPU oracle on a bounded sample
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "KV compress throughput (input GB/s) at 2x/3x budget"
+RATIOS = (2.0, 3.0)
+L2_BYTES = 126 * 1024 * 1024
+# FP32 pipe: 148 SMs x 128 lanes, one FMA-class instruction per lane per clock
+SMS, FP32_LANES = 148, 128
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="jolt", choices=["jolt", "reference"])
+    ap.add_argument("--method", default="randomized", choices=["randomized", "exact"])
+    ap.add_argument("--workload", default="mistral7b")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extras", action="store_true", help="skip the exact-arm and decompress side figures")
+    return ap.parse_args()
+
+
+def workload_config(w, method, opts):
+    return {
+        "workload": f"{w.name}: K and V [{w.n_layers}, {w.n_heads}, {w.T}, {w.D}] {w.dtype}, "
+                    f"layer groups of {w.layers_per_group}, {'FlashJoLT' if method == 'randomized' else 'JoLT'} "
+                    f"compress at {'/'.join(f'{r:g}x' for r in RATIOS)} budgets",
+        "n_layers": w.n_layers, "n_kv_heads": w.n_heads, "n_tokens": w.T, "head_dim": w.D,
+        "layers_per_group": w.layers_per_group, "method": method,
+        "token_ranks": list(opts.token_ranks), "feature_ranks": list(opts.feature_ranks),
+        "bits": list(opts.bits), "oversample": opts.oversample, "power_iters": opts.power_iters,
+        "budgets_bytes": [int(w.bf16_bytes() / r) for r in RATIOS],
+        "generator": f"{w.n_components} rank-one terms, s_i = exp(-i/{w.decay:g}), noise {w.noise}, "
+                     f"key scales lognormal(0, {w.key_sigma})",
+        "l2": "flushed between steps (write of a 256 MiB buffer)",
+    }
+
+
+# ------------------------------------------------------------------------------------------
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms while running."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.rows = []
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.th = threading.Thread(target=self._read, daemon=True)
+            self.th.start()
+        except FileNotFoundError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.rows.append([x.strip() for x in line.split(",")])
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm = [float(r[1]) for r in self.rows if len(r) >= 9 and r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in self.rows if len(r) >= 9 and r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = set()
+        for r in self.rows:
+            if len(r) < 9:
+                continue
+            for n, v in zip(names, r[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        sm.sort()
+        return {"sm_mhz": sm[len(sm) // 2] if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------------------------------
+# roofline model of the library's stages (algorithmic work per launch)
+# ------------------------------------------------------------------------------------------
+def table_alu_ops(w, opts, n_units):
+    """Quantiser arithmetic of the distortion table: per element and (r_T, r_D) candidate,
+    1 residual subtraction + 2 block min/max + 1 offset from lo, then per bit-width b > 0:
+    scale-and-round (1 FMA with the shift constant), 1 subtraction back to the integer,
+    1 FMA for the error and 1 FMA to accumulate its square; b = 0 is 1 FMA."""
+    per = 4 + sum(4 if b > 0 else 1 for b in opts.bits)
+    elems = n_units * w.layers_per_group * w.n_heads * w.T * w.D
+    return elems * len(opts.token_ranks) * len(opts.feature_ranks) * per, per
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "sm_max_mhz": 1965.0}, "fallback"
+
+
+# ------------------------------------------------------------------------------------------
+def oracle_sample(w, opts_j, seed, ratio, K=None, V=None):
+    """The float64 oracle as it stands on one unit (the keys of layer group 0) of the workload:
+    factors, distortion table, allocation at the unit's share of the budget, encoding."""
+    import numpy as np
+    import oracle as O
+    from kv_cache_compression_group_b200 import synth
+    if K is None:
+        K = synth.make_cache(w, seed, kv=0, layers=range(0, w.layers_per_group))
+    X = synth.to_f64(K)
+    oo = O.Options(opts_j.token_ranks, opts_j.feature_ranks, opts_j.bits, opts_j.method,
+                   opts_j.oversample, opts_j.power_iters)
+    t0 = time.perf_counter()
+    f = O.unit_factors(X, 0, 0, oo, seed)
+    tab = O.distortion_table(X, f.U_s, f.W_s, f.C_s, f.sigma, oo).reshape(1, -1)
+    S = w.layers_per_group * w.n_heads
+    B = O.bytes_table(w.T, w.D, S, oo).reshape(1, -1)
+    budget = int(X.size * 2 / ratio) - O.header_bytes(1)
+    al = O.allocate(tab, B, budget)
+    if al.status == "ok":
+        O.encode_unit(X, f, oo, int(al.choice[0]), float(tab[0, al.choice[0]]))
+    dt = time.perf_counter() - t0
+    return dt, X.size * 2
+
+
+def cpu_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        n = max([i.get("num_threads", 1) for i in info] or [1])
+    except Exception:
+        n = 1
+    return n, len(os.sched_getaffinity(0))
+
+
+# ------------------------------------------------------------------------------------------
+def run_reference(args, rank, world):
+    """The oracle on the host cores: each step is one unit of the workload at 2x or 3x."""
+    from kv_cache_compression_group_b200 import synth, jolt as J
+    if rank != 0:
+        return
+    w = synth.WORKLOADS[args.workload]
+    opts = J.default_options(w.T, w.D, args.method)
+    K = synth.make_cache(w, 0, kv=0, layers=range(0, w.layers_per_group))
+    times, nbytes = [], 0
+    for i in range(args.warmup + args.steps):
+        dt, nb = oracle_sample(w, opts, 0, RATIOS[i % 2], K=K)
+        if i >= args.warmup:
+            times.append(dt)
+            nbytes += nb
+    tot = sum(times)
+    value = nbytes / tot / 1e9
+    threads, cores = cpu_threads()
+    sample = (f"one unit per step (keys of layer group 0: [{w.layers_per_group}, {w.n_heads}, {w.T}, {w.D}] bf16, "
+              f"{w.layers_per_group * w.n_heads * w.T * w.D * 2 / 2**20:.0f} MiB), budgets alternating 2x / 3x")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": tot / len(times) * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(w, args.method, opts),
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": threads, "host_cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------------------------------
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+
+    import torch
+    import torch.distributed as dist
+    from datetime import timedelta
+    from kv_cache_compression_group_b200 import synth, jolt as J
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+
+    w = synth.WORKLOADS[args.workload]
+    opts = J.default_options(w.T, w.D, args.method)
+    seed = rank
+    K, V = synth.make_cache(w, seed)
+    Kd, Vd = K.to(dev), V.to(dev)
+    comp = J.Compressor(w.n_layers, w.n_heads, w.T, w.D, w.layers_per_group, K.dtype, opts, dev)
+    budgets = [int(w.bf16_bytes() / r) for r in RATIOS]
+    blobs = [torch.empty(min(b, comp.blob_max), dtype=torch.uint8, device=dev) for b in budgets]
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(Ks, Vs):
+        for b, blob in zip(budgets, blobs):
+            comp.compress(Ks, Vs, b, seed, blob=blob)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step(Kd, Vd)
+    torch.cuda.synchronize()
+    # validity of what is timed: the blobs decode and respect their budgets
+    for b, blob in zip(budgets, blobs):
+        _, total, _ = J.read_header(blob)
+        assert total <= b
+
+    # ---- timed region: device-resident inputs ------------------------------------------
+    clocks = ClockSampler(local)
+    clocks.start()
+    barrier()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    n0 = J.launch_count()
+    J.profile_begin()
+    for i in range(args.steps):
+        flush.zero_()
+        ev[i][0].record(stream)
+        step(Kd, Vd)
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    prof = J.profile_end()
+    launches = J.launch_count() - n0
+    barrier()
+    clk = clocks.stop()
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    t_ms = sum(step_ms)
+    if world > 1:
+        tt = torch.tensor([t_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        t_ms = float(tt.item())
+    in_bytes = w.input_bytes()
+    value = world * args.steps * len(RATIOS) * in_bytes / (t_ms / 1e3) / 1e9
+
+    # ---- end to end through the public API: pinned host in, blobs out ---------------------
+    Kh, Vh = K.pin_memory(), V.pin_memory()
+    Kbuf, Vbuf = torch.empty_like(Kd), torch.empty_like(Vd)
+    host_blobs = [torch.empty(bl.numel(), dtype=torch.uint8).pin_memory() for bl in blobs]
+    d2h = 0
+
+    def e2e_step():
+        nonlocal d2h
+        Kbuf.copy_(Kh, non_blocking=True)
+        Vbuf.copy_(Vh, non_blocking=True)
+        step(Kbuf, Vbuf)
+        d2h = 0
+        for bl, hb in zip(blobs, host_blobs):
+            hb.copy_(bl, non_blocking=True)
+            d2h += bl.numel()
+
+    for _ in range(max(1, args.warmup)):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        tt = torch.tensor([e_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e_ms = float(tt.item())
+    e2e = {"value": world * args.steps * len(RATIOS) * in_bytes / (e_ms / 1e3) / 1e9, "unit": "GB/s",
+           "h2d_bytes_per_step": 2 * K.numel() * K.element_size(), "d2h_bytes_per_step": d2h,
+           "ms_per_step": e_ms / args.steps}
+
+    # ---- roofline of the dominant stage ----------------------------------------------------
+    peaks, peak_src = load_peaks()
+    stages = {k: {"ms_total": v[0], "launches": v[1], "ms_per_launch": v[0] / max(1, v[1])} for k, v in prof.items()}
+    dom = max(prof.items(), key=lambda kv: kv[1][0])[0] if prof else None
+    roofline = None
+    if "table_kernel" in prof:
+        ms, n, _ = prof["table_kernel"]
+        ops, per = table_alu_ops(w, opts, comp.n_units)
+        mhz = float(peaks.get("sm_max_mhz", 1965.0))
+        peak = SMS * FP32_LANES * mhz * 1e6 / 1e12
+        achieved = ops / (ms / n / 1e3) / 1e12
+        roofline = {"kernel": "table_kernel", "bound": "alu", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                    "frac": achieved / peak, "traffic": None,
+                    "note": f"peak = {SMS} SMs x {FP32_LANES} FP32 lanes x {mhz:.0f} MHz ({peak_src} max clock); "
+                            f"algorithmic work = {per} FP32-pipe ops per element per (r_T, r_D) candidate",
+                    "dominant_stage": dom}
+
+    out = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": t_ms / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": workload_config(w, args.method, opts),
+        "e2e": e2e, "gpu_launches": int(launches), "clocks": clk, "roofline": roofline,
+        "stages": stages,
+    }
+
+    if rank == 0 and not args.no_extras:
+        # side figures: the exact (JoLT) arm and decompress, on the same cache
+        ex = {}
+        for meth in ("exact", "randomized"):
+            o2 = J.default_options(w.T, w.D, meth)
+            c2 = J.Compressor(w.n_layers, w.n_heads, w.T, w.D, w.layers_per_group, K.dtype, o2, dev)
+            c2.compress(Kd, Vd, budgets[0], seed, blob=blobs[0])
+            torch.cuda.synchronize()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            c2.compress(Kd, Vd, budgets[0], seed, blob=blobs[0])
+            b.record(stream)
+            torch.cuda.synchronize()
+            ms = a.elapsed_time(b)
+            Ko, Vo = c2.decompress(blobs[0])
+            torch.cuda.synchronize()
+            a.record(stream)
+            Ko, Vo = c2.decompress(blobs[0], K_out=Ko, V_out=Vo)
+            b.record(stream)
+            torch.cuda.synchronize()
+            dms = a.elapsed_time(b)
+            ek, evv = J.relative_errors(Kd, Vd, Ko.float(), Vo.float(), w.layers_per_group)
+            ex[meth] = {"compress_2x_ms": ms, "compress_2x_gbs": in_bytes / ms / 1e6,
+                        "latency_per_layer_group_ms": ms / w.n_groups, "decompress_ms": dms,
+                        "decompress_out_gbs": in_bytes / dms / 1e6, "rel_err_K": ek, "rel_err_V": evv}
+        ex["flashjolt_speedup_over_jolt"] = ex["exact"]["compress_2x_ms"] / ex["randomized"]["compress_2x_ms"]
+        out["arms_2x"] = ex
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        dt, nb = oracle_sample(w, opts, 0, RATIOS[0])
+        threads, cores = cpu_threads()
+        out["cpu_baseline"] = {"value": nb / dt / 1e9, "unit": "GB/s", "cores": threads, "host_cores": cores,
+                               "kind": "oracle",
+                               "sample": f"one unit (keys of layer group 0, [{w.layers_per_group}, {w.n_heads}, "
+                                         f"{w.T}, {w.D}] bf16) at the 2x budget, {dt:.1f} s"}
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -118,13 +118,14 @@ jolt_status jolt_counts(const jolt_shape* shape, const jolt_options* opts, int32
 /* Payload bytes of every choice (identical for all units), n_choices uint64 on the HOST.
  * Formula: pad16(2 T r_T) + pad16(2 D r_D) + pad16(2 S r_T r_D)
  *        + [b > 0] (pad16(nblk * 2b) + pad16(nblk * 4)),  nblk = S T D / 16.
- * ("a single Lagrangian dual allocates ... under a global byte constraint", abstract.) */
+ * (The abstract of "A JoLT for the KV cache ... Joint Rank-bit Allocation" sets one global
+ * byte limit over all groups; this is the byte count each choice is charged.) */
 jolt_status jolt_choice_bytes(const jolt_shape* shape, const jolt_options* opts, uint64_t* bytes_host);
 
-/* Whole compress ("JoLT ... treats grouped prefill caches as fourth-order tensors and applies
- * partial Tucker decomposition along the token and feature modes ... A rotated low-bit
- * quantizer captures the truncation residual, and a single Lagrangian dual allocates
- * per-group Tucker ranks and residual bit-widths under a global byte constraint", abstract).
+/* Whole compress (abstract of "A JoLT for the KV cache ... Joint Rank-bit Allocation": the
+ * grouped cache is a fourth-order tensor factored on its token and feature modes; a
+ * rotated few-bit quantiser stores the truncation residual; one Lagrangian dual sets the
+ * ranks and bit-widths of every group under a single global byte limit).
  *   k_dev, v_dev : input caches (read only), shape/dtype as `shape`
  *   budget_bytes : total blob bytes allowed (headers included)
  *   seed         : seeds the rotation signs and the FlashJoLT sketch
@@ -136,8 +137,8 @@ jolt_status jolt_compress(const jolt_shape* shape, const void* k_dev, const void
                           uint64_t budget_bytes, uint64_t seed, void* blob_dev, size_t blob_cap, void* ws_dev,
                           size_t ws_bytes, void* stream);
 
-/* Stage 1: token and feature factors of every unit (partial Tucker, token and feature modes;
- * "FlashJoLT replaces the exact token-mode SVD with a randomized approximation", abstract).
+/* Stage 1: token and feature factors of every unit (partial Tucker on the token and feature
+ * modes; FlashJoLT swaps the exact token-mode SVD for a randomized one, abstract).
  *   u_dev : [n_units][n_tokens][ld_u] fp32, unrounded token factor (leading max r_T columns)
  *   w_dev : [n_units][head_dim][ld_w] fp32, unrounded feature factor (leading max r_D columns)
  *   ld_u >= max r_T, ld_w >= max r_D.  Columns ordered by descending singular value, the
@@ -156,9 +157,23 @@ jolt_status jolt_table(const jolt_shape* shape, const void* k_dev, const void* v
                        uint64_t seed, const void* u_bf16_dev, int64_t ld_u, const void* w_bf16_dev, int64_t ld_w,
                        void* core_dev, double* table_dev, void* ws_dev, size_t ws_bytes, void* stream);
 
-/* Stage 3: the single Lagrangian dual ("a single Lagrangian dual allocates per-group Tucker
- * ranks and residual bit-widths under a global byte constraint", abstract; "per layer group
- * and separately for keys and values, under one byte budget", introduction).
+/* Stage 2b: the rotated reconstruction operators the table, encoder and decoder use
+ * (the residual is rotated before quantisation, introduction of "... Joint Tucker and
+ * JL-Residual Allocation for LLMs"; folding the rotation into the operator is this
+ * library's form of it):
+ *   P'[i_D][u][s] = bf16( (C[u][s][:, :r_D] W[u][:, :r_D]^T) diag(sigma_u) H_D / sqrt(D) )
+ *   core_dev   : [n_units][S][max r_T][max r_D] bf16 (as written by jolt_table)
+ *   w_bf16_dev : [n_units][head_dim][ld_w] bf16
+ *   p_dev      : out [n_feature_ranks][n_units][S][max r_T][head_dim] bf16
+ * Asynchronous. */
+jolt_status jolt_recon_operator(const jolt_shape* shape, const jolt_options* opts, uint64_t seed,
+                                const void* core_dev, const void* w_bf16_dev, int64_t ld_w, void* p_dev, void* ws_dev,
+                                size_t ws_bytes, void* stream);
+
+/* Stage 3: the single Lagrangian dual (abstract of "A JoLT for the KV cache ... Joint Rank-bit
+ * Allocation"; introduction of "... Joint Tucker and JL-Residual Allocation for LLMs": ranks
+ * and bit-widths are set per layer group, for keys and values separately, against one
+ * shared byte budget).
  *   dist_dev [n_units][n_choices] fp64, bytes_dev [n_units][n_choices] uint64 (device),
  *   budget_bytes: payload bytes available (headers NOT included here).
  *   choice_dev [n_units] int32 out, lambda_dev [1] fp64 out (+inf when infeasible),
@@ -185,21 +200,32 @@ jolt_status jolt_encode(const jolt_shape* shape, const void* k_dev, const void* 
 jolt_status jolt_read_header(const void* blob_dev, jolt_shape* shape_out, uint64_t* total_bytes,
                              jolt_unit_record* records, int32_t cap, void* stream);
 
-/* Decompress ("a fused ... kernel evaluates attention directly over the stored factors",
- * abstract: this is the dense reconstruction from the same stored factors):
+/* Decompress: the dense reconstruction from the stored factors (the abstract's decode kernel
+ * reads the same factors; this call materialises them):
  * X_hat = (U P' + dequant(codes)) diag(sigma) H_D / sqrt(D) per unit.
  *   out_dtype: JOLT_BF16 or JOLT_F32; k_out_dev, v_out_dev: [n_layers, H, T, D].
  * Reads the headers first (SYNCHRONISES once), then runs asynchronously. */
 jolt_status jolt_decompress(const void* blob_dev, int32_t out_dtype, void* k_out_dev, void* v_out_dev, void* ws_dev,
                             size_t ws_bytes, void* stream);
 
-/* Per-unit sums of squares (relative Frobenius error, "relative Frobenius error 0.009 (K)
- * and 0.006 (V)", introduction): sq_dev[2*u] = ||X_u||^2, sq_dev[2*u+1] = ||X_u - Y_u||^2
+/* Per-unit sums of squares (the introduction reports the relative Frobenius error of K and
+ * of V separately): sq_dev[2*u] = ||X_u||^2, sq_dev[2*u+1] = ||X_u - Y_u||^2
  * (fp64), X and Y of the same shape; y may be NULL (then only ||X_u||^2).  ydtype is Y's
  * element type.  Asynchronous. */
 jolt_status jolt_frobenius(const jolt_shape* shape, const void* k_dev, const void* v_dev, const void* ky_dev,
                            const void* vy_dev, int32_t ydtype, double* sq_dev, void* ws_dev, size_t ws_bytes,
                            void* stream);
+
+/* Stage timing for measurement (no counterpart on the pages).  jolt_profile_begin starts
+ * recording CUDA events around every internal stage launched by this thread (on the call's
+ * stream); jolt_profile_end stops, SYNCHRONISES on the recorded events and writes one line
+ * per stage, "name total_ms launches units\n", into buf (capacity cap, NUL-terminated).
+ * Recording adds two event records per stage and changes no result. */
+jolt_status jolt_profile_begin(void);
+/* Number of kernels this library has launched in the process so far (its own kernels; work
+ * launched inside cuSOLVER is not counted). */
+uint64_t jolt_launch_count(void);
+jolt_status jolt_profile_end(char* buf, size_t cap);
 
 #ifdef __cplusplus
 }

@@ -16,11 +16,14 @@ namespace jolt {
 
 struct GemmOperand {
   const void* ptr = nullptr;
+  const void* ptr_odd = nullptr;  // if set: entry e reads (e odd ? ptr_odd : ptr) + (e/2) * sbatch
+                                  // (the K / V alternation of units u = 2 g + kv)
+  int bdiv = 1;                   // batch b uses entry e = b / bdiv (operands shared by bdiv batches)
   long long ld = 0;           // stride of the non-contiguous index inside a block
   long long sbatch = 0;       // stride between batch entries
-  long long kblk = 1LL << 40; // K index = kb * kblk + kr
+  int kshift = 40;            // K index = kb * 2^kshift + kr
   long long skblk = 0;        //   -> kb * skblk + kr * (stride of K)
-  long long xblk = 1LL << 40; // M (or N) index split the same way
+  int xshift = 40;            // M (or N) index split the same way
   long long sxblk = 0;
   bool kmajor = true;         // true: K is the contiguous index
 };
@@ -39,12 +42,22 @@ struct GemmParams {
 };
 
 __host__ __device__ __forceinline__ long long opnd_offset(const GemmOperand& o, long long x, long long k) {
-  long long xb = x / o.xblk, xr = x - xb * o.xblk;
-  long long kb = k / o.kblk, kr = k - kb * o.kblk;
+  long long xb = x >> o.xshift, xr = x & ((1LL << o.xshift) - 1);
+  long long kb = k >> o.kshift, kr = k & ((1LL << o.kshift) - 1);
   long long off = xb * o.sxblk + kb * o.skblk;
   if (o.kmajor) off += xr * o.ld + kr;
   else off += xr + kr * o.ld;
   return off;
+}
+
+__host__ __device__ __forceinline__ const void* opnd_base_t(const GemmOperand& o, int b, int esize) {
+  const int e = b / o.bdiv;
+  const char* base = (const char*)((o.ptr_odd && (e & 1)) ? o.ptr_odd : o.ptr);
+  long long idx = o.ptr_odd ? (long long)(e >> 1) : (long long)e;
+  return base + idx * o.sbatch * esize;
+}
+__host__ __device__ __forceinline__ const void* opnd_base(const GemmOperand& o, int b) {
+  return opnd_base_t(o, b, 2);
 }
 
 // ------------------------------------------------------------------------------------------
@@ -147,8 +160,8 @@ __global__ void __launch_bounds__(256) gemm_bf16_kernel(GemmParams p) {
   const int kbeg = split * p.kchunk;
   const int kend = min(p.K, kbeg + p.kchunk);
 
-  const bf16* Ab = reinterpret_cast<const bf16*>(p.A.ptr) + (long long)b * p.A.sbatch;
-  const bf16* Bb = reinterpret_cast<const bf16*>(p.B.ptr) + (long long)b * p.B.sbatch;
+  const bf16* Ab = reinterpret_cast<const bf16*>(opnd_base(p.A, b));
+  const bf16* Bb = reinterpret_cast<const bf16*>(opnd_base(p.B, b));
 
   float acc[4][4][4];
 #pragma unroll
@@ -272,7 +285,7 @@ inline cudaError_t launch_gemm_bf16(const GemmParams& p, cudaStream_t st) {
   if (q.kchunk <= 0) q.kchunk = q.K;
   dim3 grid((unsigned)ceil_div(q.N, gemm_detail::BN), (unsigned)ceil_div(q.M, gemm_detail::BM),
             (unsigned)(q.batch * q.splits));
-  gemm_bf16_kernel<<<grid, gemm_detail::THREADS, gemm_bf16_smem(), st>>>(q);
+  count_launch(), gemm_bf16_kernel<<<grid, gemm_detail::THREADS, gemm_bf16_smem(), st>>>(q);
   return cudaGetLastError();
 }
 
@@ -290,8 +303,8 @@ __global__ void __launch_bounds__(256) gemm_simt_kernel(GemmParams p) {
   const int b = bz / p.splits, split = bz - b * p.splits;
   const int kbeg = split * p.kchunk;
   const int kend = min(p.K, kbeg + p.kchunk);
-  const TA* A = reinterpret_cast<const TA*>(p.A.ptr) + (long long)b * p.A.sbatch;
-  const TB* B = reinterpret_cast<const TB*>(p.B.ptr) + (long long)b * p.B.sbatch;
+  const TA* A = reinterpret_cast<const TA*>(opnd_base_t(p.A, b, (int)sizeof(TA)));
+  const TB* B = reinterpret_cast<const TB*>(opnd_base_t(p.B, b, (int)sizeof(TB)));
   Acc acc[4][4];
 #pragma unroll
   for (int i = 0; i < 4; ++i)
@@ -353,7 +366,7 @@ inline cudaError_t launch_gemm_simt(const GemmParams& p, cudaStream_t st) {
   GemmParams q = p;
   if (q.kchunk <= 0) q.kchunk = q.K;
   dim3 grid((unsigned)ceil_div(q.N, 64), (unsigned)ceil_div(q.M, 64), (unsigned)(q.batch * q.splits));
-  gemm_simt_kernel<TA, TB, Acc><<<grid, 256, 0, st>>>(q);
+  count_launch(), gemm_simt_kernel<TA, TB, Acc><<<grid, 256, 0, st>>>(q);
   return cudaGetLastError();
 }
 

@@ -74,6 +74,50 @@ jolt_status solver_get(cudaStream_t st, Solver** out) {
 }
 
 // ------------------------------------------------------------------------------------------
+// optional stage timing: CUDA events recorded around each stage on the launch stream
+// ------------------------------------------------------------------------------------------
+struct ProfRec {
+  std::string name;
+  cudaEvent_t a, b;
+  long long units;  // work items the stage processed (for per-launch figures)
+};
+struct Profiler {
+  bool on = false;
+  std::vector<ProfRec> recs;
+  std::vector<cudaEvent_t> pool;
+  cudaEvent_t get() {
+    if (!pool.empty()) {
+      cudaEvent_t e = pool.back();
+      pool.pop_back();
+      return e;
+    }
+    cudaEvent_t e;
+    cudaEventCreate(&e);
+    return e;
+  }
+};
+thread_local Profiler g_prof;
+
+struct ProfScope {
+  ProfRec rec;
+  cudaStream_t st;
+  bool on;
+  ProfScope(const char* name, cudaStream_t s, long long units = 1) : st(s), on(g_prof.on) {
+    if (!on) return;
+    rec.name = name;
+    rec.units = units;
+    rec.a = g_prof.get();
+    rec.b = g_prof.get();
+    cudaEventRecord(rec.a, st);
+  }
+  ~ProfScope() {
+    if (!on) return;
+    cudaEventRecord(rec.b, st);
+    g_prof.recs.push_back(rec);
+  }
+};
+
+// ------------------------------------------------------------------------------------------
 // plan: derived sizes and workspace layout
 // ------------------------------------------------------------------------------------------
 struct Bump {
@@ -97,8 +141,9 @@ struct Plan {
   // workspace offsets (bytes)
   size_t o_status, o_gd_part, o_gd, o_evals, o_Wf, o_Ws, o_Uf, o_Us, o_core, o_zc, o_ptmp, o_P, o_partial,
       o_table, o_bytes, o_choice, o_lambda, o_hdr, o_umap, o_info, o_solver;
-  // token factor scratch (per unit, reused)
-  size_t o_gt_part, o_gt, o_vsel, o_lam, o_omega, o_Y, o_Yt, o_Zm, o_Zt, o_h, o_l, o_Bm, o_G;
+  // token factor scratch (all units)
+  size_t o_gt32, o_gt, o_vsel, o_lam, o_omega, o_Y, o_Zm, o_h, o_l, o_gpart, o_G, o_ptrs;
+  int qr_split_max;       // split-K of the Cholesky-QR Grams
   size_t ws_total;
   int tiles;
   size_t blob_max;
@@ -186,26 +231,51 @@ jolt_status make_plan(const jolt_shape* sh, const jolt_options* op, Plan* p) {
   p->gt_split = p->m_side ? (int)ceil_div(p->T, 4096) : (p->S < 16 ? p->S : 16);
   if (p->gt_split > 64) p->gt_split = 64;
 
-  // cuSOLVER device workspace: a bound of twice the LAPACK syevd requirement
-  // (1 + 6n + 2n^2 doubles) for the largest eigenproblem; the actual need is queried and
-  // checked against it at run time, so the plan itself never touches the GPU.
+  const int NU = p->NU, T = p->T, S = p->S, M = p->M;
+  // Cholesky-QR Grams: split-K so every fp32 partial sums at most 256 terms
   {
-    long long nmax = D;
-    if (op->method == JOLT_EXACT) nmax = p->m_side ? p->M : p->T;
-    else nmax = p->k > nmax ? p->k : nmax;
-    if (nmax < D) nmax = D;
-    p->solver_dev = (size_t)(2 * (1 + 6 * nmax + 2 * nmax * nmax) * 8 + (4 << 20));
+    long long mrows = op->method == JOLT_RANDOMIZED ? (M > T ? M : T) : (p->m_side ? T : 0);
+    p->qr_split_max = mrows > 0 ? (int)ceil_div(mrows, 256) : 1;
+  }
+  // cuSOLVER device workspace: with a device present the batched eigen solver is asked for
+  // its exact need; without one (size queries on a host) a bound is used.
+  {
+    long long ntok = op->method == JOLT_EXACT ? (p->m_side ? M : T) : p->k;
+    p->solver_dev = 0;
     p->solver_host = 0;
+    int ndev = 0;
+    bool queried = false;
+    if (cudaGetDeviceCount(&ndev) == cudaSuccess && ndev > 0) {
+      Solver* s = nullptr;
+      if (solver_get(0, &s) == JOLT_OK) {
+        queried = true;
+        for (long long n : {(long long)D, ntok}) {
+          size_t dv = 0, hv = 0;
+          if (cusolverDnXsyevBatched_bufferSize(s->h, s->params, CUSOLVER_EIG_MODE_VECTOR, CUBLAS_FILL_MODE_LOWER, n,
+                                                CUDA_R_64F, nullptr, n, CUDA_R_64F, nullptr, CUDA_R_64F, &dv, &hv,
+                                                NU) != CUSOLVER_STATUS_SUCCESS) {
+            queried = false;
+            break;
+          }
+          p->solver_dev = dv > p->solver_dev ? dv : p->solver_dev;
+          p->solver_host = hv > p->solver_host ? hv : p->solver_host;
+        }
+      }
+    }
+    cudaGetLastError();
+    if (!queried) {
+      long long nmax = ntok > D ? ntok : D;
+      p->solver_dev = (size_t)NU * (size_t)(8 * (1 + 6 * nmax + 2 * nmax * nmax) * 8) + (16 << 20);
+    }
   }
 
-  const int NU = p->NU, T = p->T, S = p->S, M = p->M;
   Bump b;
   p->o_status = b.take(256);
   p->o_gd_part = b.take((size_t)NU * p->gd_split * D * D * 4);
   p->o_gd = b.take((size_t)NU * D * D * 8);
   {
     long long ntok = op->method == JOLT_EXACT ? (p->m_side ? M : T) : p->kp;
-    long long nev = (long long)NU * D > ntok ? (long long)NU * D : ntok;
+    long long nev = (long long)NU * (D > ntok ? D : ntok);
     p->o_evals = b.take((size_t)nev * 8 + 256);
   }
   p->o_Wf = b.take((size_t)NU * D * p->ldW * 4);
@@ -213,8 +283,8 @@ jolt_status make_plan(const jolt_shape* sh, const jolt_options* op, Plan* p) {
   p->o_Uf = b.take((size_t)NU * T * p->ldU * 4);
   p->o_Us = b.take((size_t)NU * T * p->ldU * 2);
   p->o_core = b.take((size_t)NU * S * p->rTmax * p->ldC * 2);
-  p->o_zc = b.take((size_t)S * T * p->ldW * 2);                        // per unit, reused
-  p->o_ptmp = b.take((size_t)S * p->rTmax * D * 4);                    // per unit, reused
+  p->o_zc = b.take((size_t)NU * S * T * p->ldW * 2);
+  p->o_ptmp = b.take((size_t)NU * S * p->rTmax * D * 4);
   p->o_P = b.take((size_t)NU * p->cd.nD * S * p->rTmax * D * 2);
   p->o_partial = b.take((size_t)NU * S * p->tiles * p->nC * 8);
   p->o_table = b.take((size_t)NU * p->nC * 8);
@@ -223,35 +293,36 @@ jolt_status make_plan(const jolt_shape* sh, const jolt_options* op, Plan* p) {
   p->o_lambda = b.take(8);
   p->o_hdr = b.take(64);
   p->o_umap = b.take((size_t)NU * S * 4 + 64);
-  p->o_info = b.take(64);
+  p->o_info = b.take((size_t)NU * 4 + 64);
   p->o_solver = b.take(p->solver_dev + 256);
   // token factor scratch
-  p->o_gt_part = p->o_gt = p->o_vsel = p->o_lam = p->o_omega = 0;
-  p->o_Y = p->o_Yt = p->o_Zm = p->o_Zt = p->o_h = p->o_l = p->o_Bm = p->o_G = 0;
+  p->o_gt32 = p->o_gt = p->o_vsel = p->o_lam = p->o_omega = 0;
+  p->o_Y = p->o_Zm = p->o_h = p->o_l = p->o_gpart = p->o_G = p->o_ptrs = 0;
+  const int kq = op->method == JOLT_RANDOMIZED ? p->kp : p->ldU;   // width of the QR'ed blocks
   if (op->method == JOLT_EXACT) {
     long long n = p->m_side ? M : T;
-    p->o_gt_part = b.take((size_t)p->gt_split * n * n * 4);
-    p->o_gt = b.take((size_t)n * n * 8);
-    p->o_lam = b.take((size_t)p->rTmax * 8 + 256);
+    p->o_gt32 = b.take((size_t)NU * n * n * 4);
+    p->o_gt = b.take((size_t)NU * n * n * 8);
+    p->o_lam = b.take((size_t)NU * p->rTmax * 8 + 256);
     if (p->m_side) {
-      p->o_vsel = b.take((size_t)M * p->ldU * 4);
-      p->o_h = b.take((size_t)M * p->ldU * 2);
-      p->o_l = b.take((size_t)M * p->ldU * 2);
-      p->o_Yt = b.take((size_t)T * p->ldU * 4);
-      p->o_G = b.take((size_t)p->ldU * p->ldU * 8);
+      p->o_vsel = b.take((size_t)NU * M * p->ldU * 4);
+      p->o_h = b.take((size_t)NU * M * p->ldU * 2);
+      p->o_l = b.take((size_t)NU * M * p->ldU * 2);
     }
   } else {
     const int kp = p->kp;
     long long big = M > T ? M : T;
-    p->o_omega = b.take((size_t)M * kp * 2);
-    p->o_Y = b.take((size_t)T * kp * 4);
-    p->o_Yt = b.take((size_t)big * kp * 4);
-    p->o_Zm = b.take((size_t)M * kp * 4);
-    p->o_h = b.take((size_t)big * kp * 2);
-    p->o_l = b.take((size_t)big * kp * 2);
-    p->o_Bm = b.take((size_t)kp * M * 4);
-    p->o_G = b.take((size_t)kp * kp * 8);
-    p->o_vsel = b.take((size_t)kp * p->ldU * 4);
+    p->o_omega = b.take((size_t)NU * M * kp * 2);
+    p->o_Y = b.take((size_t)NU * T * kp * 4);
+    p->o_Zm = b.take((size_t)NU * M * kp * 4);
+    p->o_h = b.take((size_t)NU * big * kp * 2);
+    p->o_l = b.take((size_t)NU * big * kp * 2);
+    p->o_vsel = b.take((size_t)NU * kp * p->ldU * 4);
+  }
+  if (op->method == JOLT_RANDOMIZED || p->m_side) {
+    p->o_gpart = b.take((size_t)NU * p->qr_split_max * kq * kq * 4);
+    p->o_G = b.take((size_t)NU * kq * kq * 8);
+    p->o_ptrs = b.take((size_t)NU * 8 + 64);
   }
   p->ws_total = b.off;
 
@@ -270,7 +341,7 @@ jolt_status make_plan(const jolt_shape* sh, const jolt_options* op, Plan* p) {
   p->d_U = d.take((size_t)NU * T * p->ldU * 2);
   p->d_W = d.take((size_t)NU * D * p->ldW * 2);
   p->d_C = d.take((size_t)NU * S * p->rTmax * p->ldC * 2);
-  p->d_ptmp = d.take((size_t)S * p->rTmax * D * 4);
+  p->d_ptmp = d.take((size_t)NU * S * p->rTmax * D * 4);
   p->d_P = d.take((size_t)NU * S * p->rTmax * D * 2);
   p->d_umap = d.take((size_t)NU * S * 4 + 64);
   p->dws_total = d.off;
@@ -297,6 +368,12 @@ jolt_status gemm(const GemmParams& p, int ta, int tb, cudaStream_t st) {
   else return fail(JOLT_ERR_INVALID_ARG, "gemm type combination %d/%d", ta, tb);
   if (e != cudaSuccess) return fail(JOLT_ERR_CUDA, "gemm launch: %s", cudaGetErrorString(e));
   return JOLT_OK;
+}
+
+int ilog2(int v) {
+  int s = 0;
+  while ((1 << s) < v) ++s;
+  return s;
 }
 
 unsigned grid1d(long long n, int threads = 256) {
@@ -338,7 +415,7 @@ GemmOperand xt_rowmajor(const Ctx& c, const void* x) {
   o.ptr = x;
   o.kmajor = true;       // as A (T x M): contiguous along the M index inside a slice
   o.ld = c.p.D;
-  o.kblk = c.p.D;
+  o.kshift = ilog2(c.p.D);
   o.skblk = (long long)c.p.T * c.p.D;
   return o;
 }
@@ -355,92 +432,104 @@ jolt_status solver_ws(const Ctx& c, Solver* s, size_t dv, size_t hv, void** host
   return JOLT_OK;
 }
 
-jolt_status sym_eig(const Ctx& c, double* A, int64_t n, double* w) {
+// batched: nbatch matrices of n x n stored back to back (lda = n), eigenvalues n per matrix
+jolt_status sym_eig_batched(const Ctx& c, double* A, int64_t n, double* w, int64_t nbatch) {
+  ProfScope ps("sym_eig", c.st, nbatch);
   Solver* s = nullptr;
   JTRY(solver_get(c.st, &s));
   size_t dv = 0, hv = 0;
-  SOLVER_TRY(cusolverDnXsyevd_bufferSize(s->h, s->params, CUSOLVER_EIG_MODE_VECTOR, CUBLAS_FILL_MODE_LOWER, n,
-                                         CUDA_R_64F, A, n, CUDA_R_64F, w, CUDA_R_64F, &dv, &hv));
+  SOLVER_TRY(cusolverDnXsyevBatched_bufferSize(s->h, s->params, CUSOLVER_EIG_MODE_VECTOR, CUBLAS_FILL_MODE_LOWER, n,
+                                               CUDA_R_64F, A, n, CUDA_R_64F, w, CUDA_R_64F, &dv, &hv, nbatch));
   void* host = nullptr;
   JTRY(solver_ws(c, s, dv, hv, &host));
-  SOLVER_TRY(cusolverDnXsyevd(s->h, s->params, CUSOLVER_EIG_MODE_VECTOR, CUBLAS_FILL_MODE_LOWER, n, CUDA_R_64F, A, n,
-                              CUDA_R_64F, w, CUDA_R_64F, c.at<void>(c.p.o_solver), dv, host, hv,
-                              c.at<int>(c.p.o_info)));
-  info_check_kernel<<<1, 32, 0, c.st>>>(c.at<int>(c.p.o_info), 1, c.status(), DEV_ERR_FACTOR);
+  for (int64_t b = 0; b < nbatch; ++b) {
+    count_launch(), sanitize_sym_kernel<<<1, 1024, 0, c.st>>>(A + b * n * n, (int)n, n, c.status());
+  }
+  CUDA_TRY(cudaGetLastError());
+  SOLVER_TRY(cusolverDnXsyevBatched(s->h, s->params, CUSOLVER_EIG_MODE_VECTOR, CUBLAS_FILL_MODE_LOWER, n, CUDA_R_64F,
+                                    A, n, CUDA_R_64F, w, CUDA_R_64F, c.at<void>(c.p.o_solver), dv, host, hv,
+                                    c.at<int>(c.p.o_info), nbatch));
+  count_launch(), info_check_kernel<<<(unsigned)ceil_div(nbatch, 32), 32, 0, c.st>>>(c.at<int>(c.p.o_info),
+                                                                                   (int)nbatch, c.status(),
+                                                                                   DEV_ERR_FACTOR);
   CUDA_TRY(cudaGetLastError());
   return JOLT_OK;
 }
 
-// Q = Y R^{-1} with R^T R = Y^T Y (Cholesky QR), twice; Y is m x k fp32 row-major (ld),
-// overwritten by Q.  tmp: m x ld fp32; G: k x k fp64 (ld = gld)
-jolt_status cholqr2(const Ctx& c, float* Y, int64_t m, int k, int ld, float* tmp, double* G, int gld) {
+// Cholesky QR of every unit's m x k block Y (fp32, row pitch ld, unit stride m*ld), in
+// place: G = Y^T Y (fp32 partial sums of <= 256 terms, added in fp64), G = L L^T (batched
+// Cholesky), Q = Y L^{-T} (row-wise triangular solve).  `passes` = 2 gives CholeskyQR2.
+jolt_status cholqr_batched(const Ctx& c, float* Y, long long m, int k, int ld, int passes) {
+  const Plan& p = c.p;
+  ProfScope ps("cholesky_qr", c.st, p.NU);
   Solver* s = nullptr;
   JTRY(solver_get(c.st, &s));
-  size_t dv1 = 0, hv1 = 0, dv2 = 0, hv2 = 0;
-  SOLVER_TRY(cusolverDnXpotrf_bufferSize(s->h, s->params, CUBLAS_FILL_MODE_LOWER, k, CUDA_R_64F, G, gld, CUDA_R_64F,
-                                         &dv1, &hv1));
-  SOLVER_TRY(cusolverDnXtrtri_bufferSize(s->h, CUBLAS_FILL_MODE_LOWER, CUBLAS_DIAG_NON_UNIT, k, CUDA_R_64F, G, gld,
-                                         &dv2, &hv2));
-  void* host1 = nullptr;
-  JTRY(solver_ws(c, s, dv1 > dv2 ? dv1 : dv2, hv1 > hv2 ? hv1 : hv2, &host1));
-  for (int pass = 0; pass < 2; ++pass) {
-    CUDA_TRY(cudaMemsetAsync(G, 0, (size_t)gld * gld * 8, c.st));
-    CUDA_TRY(cudaMemsetAsync(tmp, 0, (size_t)m * ld * 4, c.st));
+  float* gpart = c.at<float>(p.o_gpart);
+  double* G = c.at<double>(p.o_G);
+  double** ptrs = c.at<double*>(p.o_ptrs);
+  int* info = c.at<int>(p.o_info);
+  const int ns = (int)ceil_div(m, 256);
+  const int gld = ld;
+  for (int pass = 0; pass < passes; ++pass) {
+    ProfScope ps1("qr_gram", c.st, p.NU);
     GemmParams g;
     g.M = k;
     g.N = k;
     g.K = (int)m;
+    g.batch = p.NU;
     g.A.ptr = Y;
     g.A.kmajor = false;
     g.A.ld = ld;
-    g.B.ptr = Y;
-    g.B.kmajor = false;
-    g.B.ld = ld;
-    g.C = G;
+    g.A.sbatch = m * ld;
+    g.B = g.A;
+    g.C = gpart;
     g.ldc = gld;
-    g.c_type = 2;
+    g.sbatchC = (long long)ns * k * gld;
+    g.ssplitC = (long long)k * gld;
+    g.splits = ns;
+    g.kchunk = 256;
+    g.c_type = 0;
     JTRY(gemm(g, 1, 1, c.st));
-    SOLVER_TRY(cusolverDnXpotrf(s->h, s->params, CUBLAS_FILL_MODE_LOWER, k, CUDA_R_64F, G, gld, CUDA_R_64F,
-                                c.at<void>(c.p.o_solver), dv1, host1, hv1, c.at<int>(c.p.o_info)));
-    info_check_kernel<<<1, 32, 0, c.st>>>(c.at<int>(c.p.o_info), 1, c.status(), DEV_ERR_FACTOR);
-    SOLVER_TRY(cusolverDnXtrtri(s->h, CUBLAS_FILL_MODE_LOWER, CUBLAS_DIAG_NON_UNIT, k, CUDA_R_64F, G, gld,
-                                c.at<void>(c.p.o_solver), dv2, host1, hv2, c.at<int>(c.p.o_info)));
-    info_check_kernel<<<1, 32, 0, c.st>>>(c.at<int>(c.p.o_info), 1, c.status(), DEV_ERR_FACTOR);
-    tril_zero_kernel<<<grid1d((long long)k * k), 256, 0, c.st>>>(G, k, gld, 0, 1);
-    // Q = Y L^{-T}: B(kk, n) = Linv(n, kk) stored column-major at n + kk*gld
-    GemmParams q;
-    q.M = (int)m;
-    q.N = k;
-    q.K = k;
-    q.A.ptr = Y;
-    q.A.kmajor = true;
-    q.A.ld = ld;
-    q.B.ptr = G;
-    q.B.kmajor = false;
-    q.B.ld = gld;
-    q.C = tmp;
-    q.ldc = ld;
-    q.c_type = 0;
-    JTRY(gemm(q, 1, 2, c.st));
-    CUDA_TRY(cudaMemcpyAsync(Y, tmp, (size_t)m * ld * 4, cudaMemcpyDeviceToDevice, c.st));
+    const long long n = (long long)k * gld;
+    count_launch(), reduce_splits_kernel<float><<<grid1d((long long)p.NU * n), 256, 0, c.st>>>(gpart, G, p.NU, ns, n);
+    count_launch(), sanitize_sym_batched_kernel<<<p.NU, 1024, 0, c.st>>>(G, k, gld, n, c.status());
+    count_launch(), ptr_array_kernel<<<1, 64, 0, c.st>>>(ptrs, G, n, p.NU);
+    CUDA_TRY(cudaGetLastError());
+    ProfScope ps2("qr_potrf", c.st, p.NU);
+    SOLVER_TRY(cusolverDnDpotrfBatched(s->h, CUBLAS_FILL_MODE_LOWER, k, ptrs, gld, info, p.NU));
+    count_launch(), info_check_kernel<<<(unsigned)ceil_div(p.NU, 32), 32, 0, c.st>>>(info, p.NU, c.status(),
+                                                                                      DEV_ERR_FACTOR);
+    ProfScope ps3("qr_trsm", c.st, p.NU);
+    if (k <= 512) {
+      size_t sm = trsm_smem(64, k);
+      CUDA_TRY(cudaFuncSetAttribute(trsm_rows_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm));
+      count_launch(), trsm_rows_kernel<64><<<dim3((unsigned)ceil_div(m, 64), p.NU), 64, sm, c.st>>>(
+          Y, ld, m * ld, m, k, G, gld, n);
+    } else {
+      size_t sm = trsm_smem(32, k);
+      CUDA_TRY(cudaFuncSetAttribute(trsm_rows_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm));
+      count_launch(), trsm_rows_kernel<32><<<dim3((unsigned)ceil_div(m, 32), p.NU), 32, sm, c.st>>>(
+          Y, ld, m * ld, m, k, G, gld, n);
+    }
+    CUDA_TRY(cudaGetLastError());
   }
-  CUDA_TRY(cudaGetLastError());
   return JOLT_OK;
 }
 
-// C (m x n fp32) = X-product with an fp32 operand F given as bf16 hi + lo splits, or
-// directly when the cache is fp32.  Operand roles are given by the caller.
-jolt_status gemm_xf(const Ctx& c, GemmParams g, bool f_is_A, const float* F, long long nF, int fld_unused) {
-  (void)fld_unused;
+// C = (X-product with an fp32 operand F).  For a bf16 cache F is split as hi + lo bf16
+// (hi + lo = F to 2^-17) and the two tensor-core products are summed; for an fp32 cache
+// the product runs in fp32 directly.
+jolt_status gemm_xf(const Ctx& c, GemmParams g, bool f_is_A, const float* F, long long nF) {
+  ProfScope ps("sketch_product", c.st, c.p.NU);
   const bool xbf = c.p.dtype == JOLT_BF16;
   if (!xbf) {
     if (f_is_A) g.A.ptr = F;
     else g.B.ptr = F;
-    return gemm(g, f_is_A ? 1 : 1, 1, c.st);
+    return gemm(g, 1, 1, c.st);
   }
   bf16* hi = c.at<bf16>(c.p.o_h);
   bf16* lo = c.at<bf16>(c.p.o_l);
-  split_bf16_kernel<<<grid1d(nF), 256, 0, c.st>>>(F, hi, lo, nF);
+  count_launch(), split_bf16_kernel<<<grid1d(nF), 256, 0, c.st>>>(F, hi, lo, nF);
   CUDA_TRY(cudaGetLastError());
   GemmParams g1 = g, g2 = g;
   if (f_is_A) {
@@ -459,29 +548,51 @@ jolt_status gemm_xf(const Ctx& c, GemmParams g, bool f_is_A, const float* F, lon
 
 int xtype(const Ctx& c) { return c.p.dtype == JOLT_BF16 ? 0 : 1; }
 
+// the cache of every unit as a batched operand: X_(T) (T x M, rows t, columns (l,h,d))
+GemmOperand xt_units(const Ctx& c) {
+  GemmOperand o = xt_rowmajor(c, c.k);
+  o.ptr_odd = c.v;
+  o.sbatch = (long long)c.p.S * c.p.T * c.p.D;
+  return o;
+}
+// X_(T)^T (M x T): contiguous along (l,h,d) inside a slice, t stride D
+GemmOperand xtT_units(const Ctx& c) {
+  GemmOperand o;
+  o.ptr = c.k;
+  o.ptr_odd = c.v;
+  o.sbatch = (long long)c.p.S * c.p.T * c.p.D;
+  o.kmajor = false;
+  o.ld = c.p.D;
+  o.xshift = ilog2(c.p.D);
+  o.sxblk = (long long)c.p.T * c.p.D;
+  return o;
+}
+
 // ------------------------------------------------------------------------------------------
 // stage 1a: feature factor W of every unit
 // ------------------------------------------------------------------------------------------
-jolt_status run_feature_factor(const Ctx& c, float* Wf, long long ldWf, bf16* Ws, long long ldWs) {
+jolt_status run_feature_factor(const Ctx& c, float* Wf, long long ldWf, bf16* Ws) {
   const Plan& p = c.p;
+  ProfScope ps("feature_factor", c.st, p.NU);
   const int D = p.D;
   float* part = c.at<float>(p.o_gd_part);
   const long long rows = (long long)p.S * p.T;
   const int kchunk = (int)round_up(ceil_div(rows, p.gd_split), 32);
-  for (int kv = 0; kv < 2; ++kv) {
+  {
     GemmParams g;
     g.M = D;
     g.N = D;
     g.K = (int)rows;
-    g.batch = p.G;
-    g.A.ptr = kv ? c.v : c.k;
+    g.batch = p.NU;
+    g.A.ptr = c.k;
+    g.A.ptr_odd = c.v;
     g.A.kmajor = false;
     g.A.ld = D;
     g.A.sbatch = rows * D;
     g.B = g.A;
-    g.C = part + (size_t)kv * p.gd_split * D * D;
+    g.C = part;
     g.ldc = D;
-    g.sbatchC = 2LL * p.gd_split * D * D;
+    g.sbatchC = (long long)p.gd_split * D * D;
     g.ssplitC = (long long)D * D;
     g.splits = p.gd_split;
     g.kchunk = kchunk;
@@ -489,198 +600,188 @@ jolt_status run_feature_factor(const Ctx& c, float* Wf, long long ldWf, bf16* Ws
     JTRY(gemm(g, xtype(c), xtype(c), c.st));
   }
   double* G = c.at<double>(p.o_gd);
-  reduce_splits_kernel<float><<<grid1d((long long)p.NU * D * D), 256, 0, c.st>>>(part, G, p.NU, p.gd_split,
-                                                                                 (long long)D * D);
-  gram_diag_check_kernel<<<p.NU, 128, 0, c.st>>>(G, D, p.NU, c.status());
+  count_launch(), reduce_splits_kernel<float><<<grid1d((long long)p.NU * D * D), 256, 0, c.st>>>(
+      part, G, p.NU, p.gd_split, (long long)D * D);
+  count_launch(), gram_diag_check_kernel<<<p.NU, 128, 0, c.st>>>(G, D, p.NU, c.status());
   CUDA_TRY(cudaGetLastError());
   double* w = c.at<double>(p.o_evals);
-  for (int u = 0; u < p.NU; ++u) {
-    JTRY(sym_eig(c, G + (size_t)u * D * D, D, w + (size_t)u * D));
-  }
-  eig_select_kernel<<<dim3(p.rDmax, p.NU), 128, 0, c.st>>>(w, G, D, D, D, (long long)D * D, p.rDmax, Wf, Ws, ldWf,
-                                                           (long long)D * ldWf, nullptr);
+  JTRY(sym_eig_batched(c, G, D, w, p.NU));
+  count_launch(), eig_select_kernel<<<dim3(p.rDmax, p.NU), 128, 0, c.st>>>(
+      w, G, D, D, D, (long long)D * D, p.rDmax, Wf, Ws, ldWf, (long long)D * ldWf, nullptr);
   CUDA_TRY(cudaGetLastError());
-  (void)ldWs;
   return JOLT_OK;
 }
 
 // ------------------------------------------------------------------------------------------
-// stage 1b: token factor U of one unit (exact or randomized)
+// stage 1b: token factor U of every unit
 // ------------------------------------------------------------------------------------------
-jolt_status run_token_exact(const Ctx& c, int u, float* Uf, long long ldUf) {
+jolt_status run_token_exact(const Ctx& c, float* Uf, long long ldUf) {
   const Plan& p = c.p;
-  const int T = p.T, M = p.M, D = p.D;
-  const void* X = c.view().unit_ptr(u);
-  const int n = p.m_side ? M : T;
-  float* part = c.at<float>(p.o_gt_part);
+  ProfScope ps("token_factor_exact", c.st, p.NU);
+  const int T = p.T, M = p.M;
+  const long long n = p.m_side ? M : T;
+  float* G32 = c.at<float>(p.o_gt32);
   double* G = c.at<double>(p.o_gt);
-  GemmParams g;
-  g.C = part;
-  g.ldc = n;
-  g.c_type = 0;
-  g.splits = p.gt_split;
-  g.ssplitC = (long long)n * n;
-  if (!p.m_side) {
-    g.M = T;
-    g.N = T;
-    g.K = M;
-    g.A = xt_rowmajor(c, X);
-    g.B = g.A;  // B = X_(T)^T is K-major with the same addressing
-    g.kchunk = (int)round_up(ceil_div(M, p.gt_split), D);
-  } else {
-    g.M = M;
-    g.N = M;
-    g.K = T;
-    GemmOperand a;
-    a.ptr = X;
-    a.kmajor = false;     // contiguous along the (s,d) index inside a slice
-    a.ld = D;             // t stride
-    a.xblk = D;
-    a.sxblk = (long long)T * D;
-    g.A = a;
-    g.B = a;
-    g.kchunk = (int)round_up(ceil_div(T, p.gt_split), 32);
+  {
+    GemmParams g;
+    g.batch = p.NU;
+    g.C = G32;
+    g.ldc = n;
+    g.sbatchC = n * n;
+    g.c_type = 0;
+    if (!p.m_side) {
+      g.M = T;   // G_T = X_(T) X_(T)^T
+      g.N = T;
+      g.K = M;
+      g.A = xt_units(c);
+      g.B = g.A;
+    } else {
+      g.M = M;   // G_M = X_(T)^T X_(T)
+      g.N = M;
+      g.K = T;
+      g.A = xtT_units(c);
+      g.B = g.A;
+    }
+    JTRY(gemm(g, xtype(c), xtype(c), c.st));
   }
-  JTRY(gemm(g, xtype(c), xtype(c), c.st));
-  reduce_splits_kernel<float><<<grid1d((long long)n * n), 256, 0, c.st>>>(part, G, 1, p.gt_split, (long long)n * n);
+  count_launch(), f32_to_f64_kernel<<<grid1d((long long)p.NU * n * n), 256, 0, c.st>>>(G32, G, (long long)p.NU * n * n);
   CUDA_TRY(cudaGetLastError());
   double* w = c.at<double>(p.o_evals);
-  JTRY(sym_eig(c, G, n, w));
+  JTRY(sym_eig_batched(c, G, n, w, p.NU));
   if (!p.m_side) {
-    eig_select_kernel<<<dim3(p.rTmax, 1), 256, 0, c.st>>>(w, G, n, n, 0, 0, p.rTmax, Uf, nullptr, ldUf, 0, nullptr);
+    count_launch(), eig_select_kernel<<<dim3(p.rTmax, p.NU), 256, 0, c.st>>>(
+        w, G, (int)n, n, n, n * n, p.rTmax, Uf, nullptr, ldUf, (long long)T * ldUf, nullptr);
     CUDA_TRY(cudaGetLastError());
     return JOLT_OK;
   }
-  // T > M: U = X_(T) V Lambda^{-1/2}, then Cholesky-QR re-orthonormalisation
+  // T > M: U = X_(T) V Lambda^{-1/2}, then CholeskyQR2 re-orthonormalisation
   float* V = c.at<float>(p.o_vsel);
   double* lam = c.at<double>(p.o_lam);
-  eig_select_kernel<<<dim3(p.rTmax, 1), 256, 0, c.st>>>(w, G, n, n, 0, 0, p.rTmax, V, nullptr, p.ldU, 0, lam);
-  scale_cols_kernel<<<grid1d((long long)M * p.rTmax), 256, 0, c.st>>>(V, lam, M, p.rTmax, p.ldU, 0, 0, 1, c.status());
+  count_launch(), eig_select_kernel<<<dim3(p.rTmax, p.NU), 256, 0, c.st>>>(
+      w, G, (int)n, n, n, n * n, p.rTmax, V, nullptr, p.ldU, (long long)M * p.ldU, lam);
+  count_launch(), scale_cols_kernel<<<grid1d((long long)p.NU * M * p.rTmax), 256, 0, c.st>>>(
+      V, lam, M, p.rTmax, p.ldU, (long long)M * p.ldU, p.rTmax, p.NU, c.status());
   CUDA_TRY(cudaGetLastError());
   GemmParams y;
   y.M = T;
   y.N = p.rTmax;
   y.K = M;
-  y.A = xt_rowmajor(c, X);
+  y.batch = p.NU;
+  y.A = xt_units(c);
   y.B.kmajor = false;
   y.B.ld = p.ldU;
+  y.B.sbatch = (long long)M * p.ldU;
   y.C = Uf;
   y.ldc = ldUf;
+  y.sbatchC = (long long)T * ldUf;
   y.c_type = 0;
-  if (xtype(c) == 0) JTRY(gemm_xf(c, y, false, V, (long long)M * p.ldU, p.ldU));
-  else {
-    y.B.ptr = V;
-    JTRY(gemm(y, 1, 1, c.st));
-  }
-  JTRY(cholqr2(c, Uf, T, p.rTmax, (int)ldUf, c.at<float>(p.o_Yt), c.at<double>(p.o_G), p.ldU));
+  JTRY(gemm_xf(c, y, false, V, (long long)p.NU * M * p.ldU));
+  JTRY(cholqr_batched(c, Uf, T, p.rTmax, (int)ldUf, 2));
   return JOLT_OK;
 }
 
-jolt_status run_token_randomized(const Ctx& c, int u, float* Uf, long long ldUf) {
+// FlashJoLT: randomized subspace iteration (sketch, orthonormalise after every product),
+// then the Rayleigh-Ritz step.  B B^T with B = Q^T X_(T) is Z^T Z for Z = X_(T)^T Q.
+jolt_status run_token_randomized(const Ctx& c, float* Uf, long long ldUf) {
   const Plan& p = c.p;
-  const int T = p.T, M = p.M, D = p.D, k = p.k, kp = p.kp;
-  const void* X = c.view().unit_ptr(u);
+  ProfScope ps("token_factor_randomized", c.st, p.NU);
+  const int T = p.T, M = p.M, k = p.k, kp = p.kp, NU = p.NU;
   bf16* Om = c.at<bf16>(p.o_omega);
   float* Y = c.at<float>(p.o_Y);
-  float* tmp = c.at<float>(p.o_Yt);
   float* Z = c.at<float>(p.o_Zm);
-  double* G = c.at<double>(p.o_G);
-  CUDA_TRY(cudaMemsetAsync(Y, 0, (size_t)T * kp * 4, c.st));
-  CUDA_TRY(cudaMemsetAsync(Z, 0, (size_t)M * kp * 4, c.st));
-  omega_kernel<<<grid1d((long long)M * kp), 256, 0, c.st>>>(Om, M, k, kp, 0, c.seed, u, 1);
+  CUDA_TRY(cudaMemsetAsync(Y, 0, (size_t)NU * T * kp * 4, c.st));
+  CUDA_TRY(cudaMemsetAsync(Z, 0, (size_t)NU * M * kp * 4, c.st));
+  count_launch(), omega_kernel<<<grid1d((long long)NU * M * kp), 256, 0, c.st>>>(Om, M, k, kp, (long long)M * kp,
+                                                                                  c.seed, 0, NU);
   CUDA_TRY(cudaGetLastError());
-  // Y = X_(T) Omega
-  GemmParams g;
-  g.M = T;
-  g.N = k;
-  g.K = M;
-  g.A = xt_rowmajor(c, X);
-  g.B.ptr = Om;
-  g.B.kmajor = false;
-  g.B.ld = kp;
-  g.C = Y;
-  g.ldc = kp;
-  g.c_type = 0;
-  JTRY(gemm(g, xtype(c), 0, c.st));
-  JTRY(cholqr2(c, Y, T, k, kp, tmp, G, kp));
-  // X_(T)^T as A (M x T): contiguous along (s,d) inside a slice, t stride D
-  GemmOperand xtT;
-  xtT.ptr = X;
-  xtT.kmajor = false;
-  xtT.ld = D;
-  xtT.xblk = D;
-  xtT.sxblk = (long long)T * D;
-  for (int it = 0; it < p.q; ++it) {
-    GemmParams z;
-    z.M = M;
-    z.N = k;
-    z.K = T;
-    z.A = xtT;
-    z.B.kmajor = false;
-    z.B.ld = kp;
-    z.C = Z;
-    z.ldc = kp;
-    z.c_type = 0;
-    JTRY(gemm_xf(c, z, false, Y, (long long)T * kp, kp));
-    JTRY(cholqr2(c, Z, M, k, kp, tmp, G, kp));
-    GemmParams y = g;
-    y.B.kmajor = false;
-    y.B.ld = kp;
-    JTRY(gemm_xf(c, y, false, Z, (long long)M * kp, kp));
-    JTRY(cholqr2(c, Y, T, k, kp, tmp, G, kp));
+  // products with X_(T) (Y side, T x k) and X_(T)^T (Z side, M x k)
+  GemmParams gy;
+  gy.M = T;
+  gy.N = k;
+  gy.K = M;
+  gy.batch = NU;
+  gy.A = xt_units(c);
+  gy.B.kmajor = false;
+  gy.B.ld = kp;
+  gy.C = Y;
+  gy.ldc = kp;
+  gy.sbatchC = (long long)T * kp;
+  gy.c_type = 0;
+  GemmParams gz = gy;
+  gz.M = M;
+  gz.K = T;
+  gz.A = xtT_units(c);
+  gz.C = Z;
+  gz.sbatchC = (long long)M * kp;
+  {
+    ProfScope ps0("sketch_product", c.st, NU);
+    GemmParams g0 = gy;  // Y = X_(T) Omega
+    g0.B.ptr = Om;
+    g0.B.sbatch = (long long)M * kp;
+    JTRY(gemm(g0, xtype(c), 0, c.st));
   }
-  // B = Q^T X_(T) (k x M), then the k x k matrix B B^T
-  float* Bm = c.at<float>(p.o_Bm);
-  GemmParams bq;
-  bq.M = k;
-  bq.N = M;
-  bq.K = T;
-  bq.A.kmajor = false;  // A(i, t) = Q[t][i]
-  bq.A.ld = kp;
-  GemmOperand xn;       // B(t, (s,d)) = X[s][t][d]: contiguous along (s,d) inside a slice
-  xn.ptr = X;
-  xn.kmajor = false;
-  xn.ld = D;
-  xn.xblk = D;
-  xn.sxblk = (long long)T * D;
-  bq.B = xn;
-  bq.C = Bm;
-  bq.ldc = M;
-  bq.c_type = 0;
-  JTRY(gemm_xf(c, bq, true, Y, (long long)T * kp, kp));
-  CUDA_TRY(cudaMemsetAsync(G, 0, (size_t)kp * kp * 8, c.st));
-  GemmParams gg;
-  gg.M = k;
-  gg.N = k;
-  gg.K = M;
-  gg.A.ptr = Bm;
-  gg.A.kmajor = true;
-  gg.A.ld = M;
-  gg.B.ptr = Bm;
-  gg.B.kmajor = true;
-  gg.B.ld = M;
-  gg.C = G;
-  gg.ldc = k;
-  gg.c_type = 2;
-  JTRY(gemm(gg, 1, 1, c.st));
+  gy.B.sbatch = (long long)M * kp;   // Y = X_(T) Qz : B = Qz (M x k)
+  gz.B.sbatch = (long long)T * kp;   // Z = X_(T)^T Q : B = Q (T x k)
+  JTRY(cholqr_batched(c, Y, T, k, kp, p.q == 0 ? 2 : 1));
+  for (int it = 0; it < p.q; ++it) {
+    JTRY(gemm_xf(c, gz, false, Y, (long long)NU * T * kp));
+    JTRY(cholqr_batched(c, Z, M, k, kp, 1));
+    JTRY(gemm_xf(c, gy, false, Z, (long long)NU * M * kp));
+    JTRY(cholqr_batched(c, Y, T, k, kp, it + 1 == p.q ? 2 : 1));
+  }
+  // Rayleigh-Ritz: S = Z^T Z with Z = X_(T)^T Q  (k x k per unit)
+  JTRY(gemm_xf(c, gz, false, Y, (long long)NU * T * kp));
+  float* gpart = c.at<float>(p.o_gpart);
+  double* S = c.at<double>(p.o_G);
+  const int ns = (int)ceil_div(M, 256);
+  {
+    ProfScope ps1("ritz_gram", c.st, NU);
+    GemmParams g;
+    g.M = k;
+    g.N = k;
+    g.K = M;
+    g.batch = NU;
+    g.A.ptr = Z;
+    g.A.kmajor = false;
+    g.A.ld = kp;
+    g.A.sbatch = (long long)M * kp;
+    g.B = g.A;
+    g.C = gpart;
+    g.ldc = k;
+    g.sbatchC = (long long)ns * k * k;
+    g.ssplitC = (long long)k * k;
+    g.splits = ns;
+    g.kchunk = 256;
+    g.c_type = 0;
+    JTRY(gemm(g, 1, 1, c.st));
+    count_launch(), reduce_splits_kernel<float><<<grid1d((long long)NU * k * k), 256, 0, c.st>>>(
+        gpart, S, NU, ns, (long long)k * k);
+    CUDA_TRY(cudaGetLastError());
+  }
   double* w = c.at<double>(p.o_evals);
-  JTRY(sym_eig(c, G, k, w));
+  JTRY(sym_eig_batched(c, S, k, w, NU));
   float* V = c.at<float>(p.o_vsel);
-  eig_select_kernel<<<dim3(p.rTmax, 1), 256, 0, c.st>>>(w, G, k, k, 0, 0, p.rTmax, V, nullptr, p.ldU, 0, nullptr);
+  count_launch(), eig_select_kernel<<<dim3(p.rTmax, NU), 256, 0, c.st>>>(
+      w, S, k, k, k, (long long)k * k, p.rTmax, V, nullptr, p.ldU, (long long)kp * p.ldU, nullptr);
   CUDA_TRY(cudaGetLastError());
   // U = Q V
+  ProfScope ps2("ritz_vectors", c.st, NU);
   GemmParams uq;
   uq.M = T;
   uq.N = p.rTmax;
   uq.K = k;
+  uq.batch = NU;
   uq.A.ptr = Y;
   uq.A.kmajor = true;
   uq.A.ld = kp;
+  uq.A.sbatch = (long long)T * kp;
   uq.B.ptr = V;
   uq.B.kmajor = false;
   uq.B.ld = p.ldU;
+  uq.B.sbatch = (long long)kp * p.ldU;
   uq.C = Uf;
   uq.ldc = ldUf;
+  uq.sbatchC = (long long)T * ldUf;
   uq.c_type = 0;
   JTRY(gemm(uq, 1, 1, c.st));
   return JOLT_OK;
@@ -689,16 +790,13 @@ jolt_status run_token_randomized(const Ctx& c, int u, float* Uf, long long ldUf)
 jolt_status run_factor(const Ctx& c, float* Uf, long long ldUf, float* Wf, long long ldWf, bf16* Us, bf16* Ws) {
   const Plan& p = c.p;
   CUDA_TRY(cudaMemsetAsync(c.status(), 0, 4, c.st));
-  JTRY(run_feature_factor(c, Wf, ldWf, Ws, ldWf));
-  for (int u = 0; u < p.NU; ++u) {
-    float* U = Uf + (size_t)u * p.T * ldUf;
-    if (p.method == JOLT_EXACT) JTRY(run_token_exact(c, u, U, ldUf));
-    else JTRY(run_token_randomized(c, u, U, ldUf));
-  }
+  JTRY(run_feature_factor(c, Wf, ldWf, Ws));
+  if (p.method == JOLT_EXACT) JTRY(run_token_exact(c, Uf, ldUf));
+  else JTRY(run_token_randomized(c, Uf, ldUf));
   // sign convention of the token factor columns (the randomized and back-projected routes
   // need it; for the eigenvector route it is already in place) and the bf16 copy
-  col_sign_fix_kernel<<<dim3(p.rTmax, p.NU), 256, 0, c.st>>>(Uf, ldUf, (long long)p.T * ldUf, p.T, p.rTmax, Us,
-                                                             ldUf, (long long)p.T * ldUf);
+  count_launch(), col_sign_fix_kernel<<<dim3(p.rTmax, p.NU), 256, 0, c.st>>>(
+      Uf, ldUf, (long long)p.T * ldUf, p.T, p.rTmax, Us, ldUf, (long long)p.T * ldUf);
   CUDA_TRY(cudaGetLastError());
   return JOLT_OK;
 }
@@ -708,52 +806,56 @@ jolt_status run_factor(const Ctx& c, float* Uf, long long ldUf, float* Wf, long 
 // ------------------------------------------------------------------------------------------
 jolt_status run_core(const Ctx& c, const bf16* Us, long long ldU, const bf16* Ws, long long ldW, bf16* core) {
   const Plan& p = c.p;
+  ProfScope ps("core", c.st, p.NU);
   const int T = p.T, D = p.D, S = p.S;
   bf16* Zc = c.at<bf16>(p.o_zc);
-  for (int u = 0; u < p.NU; ++u) {
-    const void* X = c.view().unit_ptr(u);
-    // Z = bf16(X_(D) W_s)   ((S T) x rDmax)
-    GemmParams z;
-    z.M = S * T;
-    z.N = p.rDmax;
-    z.K = D;
-    z.A.ptr = X;
-    z.A.kmajor = true;
-    z.A.ld = D;
-    z.B.ptr = Ws + (size_t)u * D * ldW;
-    z.B.kmajor = false;
-    z.B.ld = ldW;
-    z.C = Zc;
-    z.ldc = p.ldW;
-    z.c_type = 1;
-    JTRY(gemm(z, xtype(c), 0, c.st));
-    // C_s = bf16(U_s^T Z_s) per slice  (rTmax x rDmax)
-    GemmParams cc;
-    cc.M = p.rTmax;
-    cc.N = p.rDmax;
-    cc.K = T;
-    cc.batch = S;
-    cc.A.ptr = Us + (size_t)u * T * ldU;
-    cc.A.kmajor = false;
-    cc.A.ld = ldU;
-    cc.A.sbatch = 0;
-    cc.B.ptr = Zc;
-    cc.B.kmajor = false;
-    cc.B.ld = p.ldW;
-    cc.B.sbatch = (long long)T * p.ldW;
-    cc.C = core + (size_t)u * S * p.rTmax * p.ldC;
-    cc.ldc = p.ldC;
-    cc.sbatchC = (long long)p.rTmax * p.ldC;
-    cc.c_type = 1;
-    JTRY(gemm(cc, 0, 0, c.st));
-  }
+  // Z = bf16(X_(D) W_s)   ((S T) x rDmax per unit)
+  GemmParams z;
+  z.M = S * T;
+  z.N = p.rDmax;
+  z.K = D;
+  z.batch = p.NU;
+  z.A.ptr = c.k;
+  z.A.ptr_odd = c.v;
+  z.A.kmajor = true;
+  z.A.ld = D;
+  z.A.sbatch = (long long)S * T * D;
+  z.B.ptr = Ws;
+  z.B.kmajor = false;
+  z.B.ld = ldW;
+  z.B.sbatch = (long long)D * ldW;
+  z.C = Zc;
+  z.ldc = p.ldW;
+  z.sbatchC = (long long)S * T * p.ldW;
+  z.c_type = 1;
+  JTRY(gemm(z, xtype(c), 0, c.st));
+  // C_s = bf16(U_s^T Z_s) per (unit, slice)  (rTmax x rDmax)
+  GemmParams cc;
+  cc.M = p.rTmax;
+  cc.N = p.rDmax;
+  cc.K = T;
+  cc.batch = p.NU * S;
+  cc.A.ptr = Us;
+  cc.A.kmajor = false;
+  cc.A.ld = ldU;
+  cc.A.sbatch = (long long)T * ldU;
+  cc.A.bdiv = S;
+  cc.B.ptr = Zc;
+  cc.B.kmajor = false;
+  cc.B.ld = p.ldW;
+  cc.B.sbatch = (long long)T * p.ldW;
+  cc.C = core;
+  cc.ldc = p.ldC;
+  cc.sbatchC = (long long)p.rTmax * p.ldC;
+  cc.c_type = 1;
+  JTRY(gemm(cc, 0, 0, c.st));
   return JOLT_OK;
 }
 
 template <int D>
 void launch_rotate_rows(const float* in, bf16* out, long long nrows, long long rows_per_unit, const int* umap,
                         uint64_t seed, cudaStream_t st) {
-  rotate_rows_kernel<D><<<(unsigned)ceil_div(nrows, 64), 64, 0, st>>>(in, out, nrows, rows_per_unit, umap, seed);
+  count_launch(), rotate_rows_kernel<D><<<(unsigned)ceil_div(nrows, 64), 64, 0, st>>>(in, out, nrows, rows_per_unit, umap, seed);
 }
 
 jolt_status rotate_rows(const Ctx& c, const float* in, bf16* out, long long nrows, long long rows_per_unit,
@@ -794,8 +896,36 @@ jolt_status pmat_unit(const Ctx& c, int u, const bf16* core_u, long long ldC, in
   return JOLT_OK;
 }
 
+// P'(r_D) of every unit: bf16(rotate(C_s[:, :rT, :r_D] W_s[:, :r_D]^T)); out layout
+// [unit][S][rTslice][D] (unit stride S*rTslice*D)
+jolt_status pmat_all(const Ctx& c, const bf16* core, long long ldC, int rT, int rTslice, const bf16* Ws, long long ldW,
+                     int rD, float* ptmp, bf16* out, const int* umap) {
+  const Plan& p = c.p;
+  GemmParams g;
+  g.M = rT;
+  g.N = p.D;
+  g.K = rD;
+  g.batch = p.NU * p.S;
+  g.A.ptr = core;
+  g.A.kmajor = true;
+  g.A.ld = ldC;
+  g.A.sbatch = (long long)rT * ldC;
+  g.B.ptr = Ws;
+  g.B.kmajor = true;  // B(j, d) = W_s[d][j]
+  g.B.ld = ldW;
+  g.B.sbatch = (long long)p.D * ldW;
+  g.B.bdiv = p.S;
+  g.C = ptmp;
+  g.ldc = p.D;
+  g.sbatchC = (long long)rTslice * p.D;
+  g.c_type = 0;
+  JTRY(gemm(g, 0, 0, c.st));
+  JTRY(rotate_rows(c, ptmp, out, (long long)p.NU * p.S * rTslice, (long long)p.S * rTslice, umap));
+  return JOLT_OK;
+}
+
 jolt_status fill_umap(const Ctx& c, int* umap, int n) {
-  iota_kernel<<<(unsigned)ceil_div(n, 128), 128, 0, c.st>>>(umap, n);
+  count_launch(), iota_kernel<<<(unsigned)ceil_div(n, 128), 128, 0, c.st>>>(umap, n);
   CUDA_TRY(cudaGetLastError());
   return JOLT_OK;
 }
@@ -804,7 +934,7 @@ template <int D, typename TX>
 jolt_status launch_table_T(const Ctx& c, const TableArgs& a) {
   size_t sm = table_smem<D>();
   CUDA_TRY(cudaFuncSetAttribute(table_kernel<D, TX>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm));
-  table_kernel<D, TX><<<dim3(c.p.tiles, c.p.S, c.p.NU), TTHREADS, sm, c.st>>>(a);
+  count_launch(), table_kernel<D, TX><<<dim3(c.p.tiles, c.p.S, c.p.NU), TTHREADS, sm, c.st>>>(a);
   CUDA_TRY(cudaGetLastError());
   return JOLT_OK;
 }
@@ -821,13 +951,14 @@ jolt_status run_table(const Ctx& c, const bf16* Us, long long ldU, const bf16* W
   bf16* P = c.at<bf16>(p.o_P);
   int* umap = c.at<int>(p.o_umap);
   JTRY(fill_umap(c, umap, p.NU));
-  const long long sP_rd = (long long)p.S * p.rTmax * p.D;
-  const long long sP_unit = p.cd.nD * sP_rd;
-  for (int u = 0; u < p.NU; ++u)
+  const long long sP_unit = (long long)p.S * p.rTmax * p.D;
+  const long long sP_rd = p.NU * sP_unit;
+  {
+    ProfScope ps("recon_operator", c.st, p.NU);
     for (int iD = 0; iD < p.cd.nD; ++iD)
-      JTRY(pmat_unit(c, u, core + (size_t)u * p.S * p.rTmax * p.ldC, p.ldC, p.rTmax, p.rTmax,
-                     Ws + (size_t)u * p.D * ldW, ldW, p.cd.rD[iD], c.at<float>(p.o_ptmp), P + u * sP_unit + iD * sP_rd,
-                     umap));
+      JTRY(pmat_all(c, core, p.ldC, p.rTmax, p.rTmax, Ws, ldW, p.cd.rD[iD], c.at<float>(p.o_ptmp), P + iD * sP_rd,
+                    umap));
+  }
   TableArgs a;
   a.cv = c.view();
   a.U = Us;
@@ -841,13 +972,16 @@ jolt_status run_table(const Ctx& c, const bf16* Us, long long ldU, const bf16* W
   a.seed = c.seed;
   a.partial = c.at<double>(p.o_partial);
   a.tiles = p.tiles;
-  switch (p.D) {
-    case 16: JTRY(launch_table_D<16>(c, a)); break;
-    case 32: JTRY(launch_table_D<32>(c, a)); break;
-    case 64: JTRY(launch_table_D<64>(c, a)); break;
-    default: JTRY(launch_table_D<128>(c, a)); break;
+  {
+    ProfScope ps("table_kernel", c.st, p.NU);
+    switch (p.D) {
+      case 16: JTRY(launch_table_D<16>(c, a)); break;
+      case 32: JTRY(launch_table_D<32>(c, a)); break;
+      case 64: JTRY(launch_table_D<64>(c, a)); break;
+      default: JTRY(launch_table_D<128>(c, a)); break;
+    }
   }
-  table_reduce_kernel<<<(unsigned)ceil_div((long long)p.NU * p.nC, 128), 128, 0, c.st>>>(
+  count_launch(), table_reduce_kernel<<<(unsigned)ceil_div((long long)p.NU * p.nC, 128), 128, 0, c.st>>>(
       a.partial, table, p.NU, p.S, p.tiles, p.cd.nT, p.cd.nD, p.cd.nB);
   CUDA_TRY(cudaGetLastError());
   return JOLT_OK;
@@ -860,7 +994,7 @@ template <int D, typename TX>
 jolt_status launch_encode_T(const Ctx& c, const EncodeArgs& a) {
   size_t sm = table_smem<D>();
   CUDA_TRY(cudaFuncSetAttribute(encode_kernel<D, TX>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm));
-  encode_kernel<D, TX><<<dim3(c.p.tiles, c.p.S, c.p.NU), TTHREADS, sm, c.st>>>(a);
+  count_launch(), encode_kernel<D, TX><<<dim3(c.p.tiles, c.p.S, c.p.NU), TTHREADS, sm, c.st>>>(a);
   CUDA_TRY(cudaGetLastError());
   return JOLT_OK;
 }
@@ -890,8 +1024,9 @@ BlobHeader header_proto(const Plan& p, uint64_t seed) {
 jolt_status run_allocate(const Ctx& c, const double* table, unsigned long long budget_payload, unsigned char* blob,
                          size_t blob_cap, const int32_t* forced_choice) {
   const Plan& p = c.p;
+  ProfScope ps("allocate", c.st, 1);
   unsigned long long* B = c.at<unsigned long long>(p.o_bytes);
-  bytes_table_kernel<<<(unsigned)ceil_div((long long)p.NU * p.nC, 128), 128, 0, c.st>>>(B, p.NU, p.T, p.D, p.S, p.cd);
+  count_launch(), bytes_table_kernel<<<(unsigned)ceil_div((long long)p.NU * p.nC, 128), 128, 0, c.st>>>(B, p.NU, p.T, p.D, p.S, p.cd);
   CUDA_TRY(cudaGetLastError());
   AllocArgs a;
   memset(&a, 0, sizeof a);
@@ -913,7 +1048,7 @@ jolt_status run_allocate(const Ctx& c, const double* table, unsigned long long b
   a.hdr = header_proto(p, c.seed);
   size_t sm = (size_t)((p.NU * 4 + 15) / 16) * 16 + (size_t)p.NU * 8;
   a.forced = forced_choice;  // caller's choices (jolt_encode): same header filling, no search
-  allocate_kernel<<<1, 128, sm, c.st>>>(a);
+  count_launch(), allocate_kernel<<<1, 512, sm, c.st>>>(a);
   CUDA_TRY(cudaGetLastError());
   return JOLT_OK;
 }
@@ -927,19 +1062,20 @@ jolt_status run_encode(const Ctx& c, const bf16* Us, long long ldU, const bf16* 
   a.ldU = ldU;
   a.sU = (long long)p.T * ldU;
   a.P = c.at<bf16>(p.o_P);
-  a.sP_rd = (long long)p.S * p.rTmax * p.D;
-  a.sP_unit = p.cd.nD * a.sP_rd;
+  a.sP_unit = (long long)p.S * p.rTmax * p.D;
+  a.sP_rd = p.NU * a.sP_unit;
   a.rTmax = p.rTmax;
   a.cand = p.cd;
   a.seed = c.seed;
   a.blob = blob;
+  ProfScope ps("encode", c.st, p.NU);
   switch (p.D) {
     case 16: JTRY(launch_encode_D<16>(c, a)); break;
     case 32: JTRY(launch_encode_D<32>(c, a)); break;
     case 64: JTRY(launch_encode_D<64>(c, a)); break;
     default: JTRY(launch_encode_D<128>(c, a)); break;
   }
-  copy_factors_kernel<<<dim3(64, p.NU), 256, 0, c.st>>>(blob, Us, ldU, (long long)p.T * ldU, Ws, ldW,
+  count_launch(), copy_factors_kernel<<<dim3(64, p.NU), 256, 0, c.st>>>(blob, Us, ldU, (long long)p.T * ldU, Ws, ldW,
                                                          (long long)p.D * ldW, core, p.ldC, (long long)p.rTmax * p.ldC,
                                                          (long long)p.S * p.rTmax * p.ldC, p.T, p.D, p.S);
   CUDA_TRY(cudaGetLastError());
@@ -978,6 +1114,53 @@ extern "C" {
 const char* jolt_version(void) { return "jolt-b200 1.0 (sm_100a)"; }
 
 const char* jolt_last_error(void) { return g_err.c_str(); }
+
+uint64_t jolt_launch_count(void) { return launch_counter().load(); }
+
+jolt_status jolt_profile_begin(void) {
+  for (auto& r : g_prof.recs) {
+    g_prof.pool.push_back(r.a);
+    g_prof.pool.push_back(r.b);
+  }
+  g_prof.recs.clear();
+  g_prof.on = true;
+  return JOLT_OK;
+}
+
+jolt_status jolt_profile_end(char* buf, size_t cap) {
+  g_prof.on = false;
+  std::vector<std::string> names;
+  std::vector<double> ms;
+  std::vector<long long> cnt, units;
+  for (auto& r : g_prof.recs) {
+    CUDA_TRY(cudaEventSynchronize(r.b));
+    float t = 0.f;
+    CUDA_TRY(cudaEventElapsedTime(&t, r.a, r.b));
+    size_t i = 0;
+    while (i < names.size() && names[i] != r.name) ++i;
+    if (i == names.size()) {
+      names.push_back(r.name);
+      ms.push_back(0.0);
+      cnt.push_back(0);
+      units.push_back(0);
+    }
+    ms[i] += t;
+    cnt[i] += 1;
+    units[i] += r.units;
+  }
+  std::string out;
+  char line[256];
+  for (size_t i = 0; i < names.size(); ++i) {
+    snprintf(line, sizeof line, "%s %.6f %lld %lld\n", names[i].c_str(), ms[i], cnt[i], units[i]);
+    out += line;
+  }
+  if (buf && cap) {
+    size_t n = out.size() < cap - 1 ? out.size() : cap - 1;
+    memcpy(buf, out.data(), n);
+    buf[n] = 0;
+  }
+  return JOLT_OK;
+}
 
 jolt_status jolt_workspace_size(const jolt_shape* shape, const jolt_options* opts, size_t* ws_bytes,
                                 size_t* blob_bytes, size_t* dws_bytes) {
@@ -1038,6 +1221,30 @@ jolt_status jolt_table(const jolt_shape* shape, const void* k_dev, const void* v
   return run_table(c, (const bf16*)u_bf16_dev, ld_u, (const bf16*)w_bf16_dev, ld_w, (bf16*)core_dev, table_dev);
 }
 
+jolt_status jolt_recon_operator(const jolt_shape* shape, const jolt_options* opts, uint64_t seed,
+                                const void* core_dev, const void* w_bf16_dev, int64_t ld_w, void* p_dev, void* ws_dev,
+                                size_t ws_bytes, void* stream) {
+  Plan p;
+  JTRY(make_plan(shape, opts, &p));
+  JTRY(check_ws(p, ws_dev, ws_bytes));
+  JTRY(check_aligned(core_dev, "core"));
+  JTRY(check_aligned(w_bf16_dev, "w_bf16"));
+  JTRY(check_aligned(p_dev, "p"));
+  if (ld_w < p.rDmax || ld_w % 8) return fail(JOLT_ERR_INVALID_ARG, "ld_w must cover the largest rank, multiple of 8");
+  Ctx c{p, (unsigned char*)ws_dev, (cudaStream_t)stream, nullptr, nullptr, seed};
+  int* umap = c.at<int>(p.o_umap);
+  JTRY(fill_umap(c, umap, p.NU));
+  const long long sP_rd = (long long)p.NU * p.S * p.rTmax * p.D;
+  const bf16* core = (const bf16*)core_dev;
+  const bf16* Ws = (const bf16*)w_bf16_dev;
+  bf16* P = (bf16*)p_dev;
+  ProfScope ps("recon_operator", c.st, p.NU);
+  for (int iD = 0; iD < p.cd.nD; ++iD)
+    JTRY(pmat_all(c, core, p.ldC, p.rTmax, p.rTmax, Ws, ld_w, p.cd.rD[iD], c.at<float>(p.o_ptmp), P + iD * sP_rd,
+                  umap));
+  return JOLT_OK;
+}
+
 jolt_status jolt_allocate(const double* dist_dev, const uint64_t* bytes_dev, int32_t n_units, int32_t n_choices,
                           uint64_t budget_bytes, int32_t* choice_dev, double* lambda_dev, uint32_t* status_dev,
                           void* stream) {
@@ -1056,7 +1263,7 @@ jolt_status jolt_allocate(const double* dist_dev, const uint64_t* bytes_dev, int
   a.lambda = lambda_dev;
   a.status = status_dev;
   size_t sm = (size_t)((n_units * 4 + 15) / 16) * 16 + (size_t)n_units * 8;
-  allocate_kernel<<<1, 128, sm, st>>>(a);
+  count_launch(), allocate_kernel<<<1, 512, sm, st>>>(a);
   CUDA_TRY(cudaGetLastError());
   return JOLT_OK;
 }
@@ -1082,14 +1289,12 @@ jolt_status jolt_encode(const jolt_shape* shape, const void* k_dev, const void* 
   bf16* P = c.at<bf16>(p.o_P);
   int* umap = c.at<int>(p.o_umap);
   JTRY(fill_umap(c, umap, p.NU));
-  const long long sP_rd = (long long)p.S * p.rTmax * p.D;
+  const long long sP_rd = (long long)p.NU * p.S * p.rTmax * p.D;
   const bf16* core = (const bf16*)core_dev;
   const bf16* Ws = (const bf16*)w_bf16_dev;
-  for (int u = 0; u < p.NU; ++u)
-    for (int iD = 0; iD < p.cd.nD; ++iD)
-      JTRY(pmat_unit(c, u, core + (size_t)u * p.S * p.rTmax * p.ldC, p.ldC, p.rTmax, p.rTmax,
-                     Ws + (size_t)u * p.D * ld_w, ld_w, p.cd.rD[iD], c.at<float>(p.o_ptmp),
-                     P + u * p.cd.nD * sP_rd + iD * sP_rd, umap));
+  for (int iD = 0; iD < p.cd.nD; ++iD)
+    JTRY(pmat_all(c, core, p.ldC, p.rTmax, p.rTmax, Ws, ld_w, p.cd.rD[iD], c.at<float>(p.o_ptmp), P + iD * sP_rd,
+                  umap));
   JTRY(run_allocate(c, dist_dev, 0, (unsigned char*)blob_dev, blob_cap, choice_dev));
   return run_encode(c, (const bf16*)u_bf16_dev, ld_u, Ws, ld_w, core, (unsigned char*)blob_dev);
 }
@@ -1120,7 +1325,7 @@ jolt_status jolt_compress(const jolt_shape* shape, const void* k_dev, const void
   JTRY(run_allocate(c, table, budget_bytes - hdr, (unsigned char*)blob_dev, blob_cap, nullptr));
   JTRY(run_encode(c, Us, p.ldU, Ws, p.ldW, core, (unsigned char*)blob_dev));
   // device-side errors of the factor stage are folded into the header status
-  fold_status_kernel<<<1, 1, 0, c.st>>>(c.status(), (unsigned char*)blob_dev);
+  count_launch(), fold_status_kernel<<<1, 1, 0, c.st>>>(c.status(), (unsigned char*)blob_dev);
   CUDA_TRY(cudaGetLastError());
   return JOLT_OK;
 }
@@ -1208,9 +1413,9 @@ jolt_status jolt_decompress(const void* blob_dev, int32_t out_dtype, void* k_out
     bf16* Uu = Ucp + (size_t)u * p.T * p.ldU;
     bf16* Wu = Wcp + (size_t)u * p.D * p.ldW;
     bf16* Cu = Ccp + (size_t)u * p.S * p.rTmax * p.ldC;
-    copy2d_kernel<<<grid1d((long long)p.T * p.ldU), 256, 0, st>>>((const bf16*)(blob + r.off_U), p.T, r.r_T, Uu, p.ldU);
-    copy2d_kernel<<<grid1d((long long)p.D * p.ldW), 256, 0, st>>>((const bf16*)(blob + r.off_W), p.D, r.r_D, Wu, p.ldW);
-    copy2d_kernel<<<grid1d((long long)p.S * r.r_T * p.ldC), 256, 0, st>>>((const bf16*)(blob + r.off_C),
+    count_launch(), copy2d_kernel<<<grid1d((long long)p.T * p.ldU), 256, 0, st>>>((const bf16*)(blob + r.off_U), p.T, r.r_T, Uu, p.ldU);
+    count_launch(), copy2d_kernel<<<grid1d((long long)p.D * p.ldW), 256, 0, st>>>((const bf16*)(blob + r.off_W), p.D, r.r_D, Wu, p.ldW);
+    count_launch(), copy2d_kernel<<<grid1d((long long)p.S * r.r_T * p.ldC), 256, 0, st>>>((const bf16*)(blob + r.off_C),
                                                                           (long long)p.S * r.r_T, r.r_D, Cu, p.ldC);
     CUDA_TRY(cudaGetLastError());
     JTRY(pmat_unit(c, u, Cu, p.ldC, r.r_T, p.rTmax, Wu, p.ldW, r.r_D, ptmp, P + u * sP_unit, umap));
@@ -1231,12 +1436,13 @@ jolt_status jolt_decompress(const void* blob_dev, int32_t out_dtype, void* k_out
   a.v_out = v_out_dev;
   a.out_f32 = out_dtype == JOLT_F32;
   dim3 grid(p.tiles, p.S, p.NU);
+  ProfScope ps("decode_kernel", st, p.NU);
   switch (p.D) {
 #define DEC_CASE(DD)                                                                                     \
   case DD: {                                                                                             \
     CUDA_TRY(cudaFuncSetAttribute(decode_kernel<DD>, cudaFuncAttributeMaxDynamicSharedMemorySize,        \
                                   (int)decode_smem<DD>()));                                              \
-    decode_kernel<DD><<<grid, TTHREADS, decode_smem<DD>(), st>>>(a);                                     \
+    count_launch(), decode_kernel<DD><<<grid, TTHREADS, decode_smem<DD>(), st>>>(a);                                     \
     break;                                                                                               \
   }
     DEC_CASE(16)
@@ -1268,18 +1474,18 @@ jolt_status jolt_frobenius(const jolt_shape* shape, const void* k_dev, const voi
     dim3 grid(nblk, G);
     if (shape->dtype == JOLT_BF16) {
       if (ydtype == JOLT_F32)
-        frob_partial_kernel<bf16, float><<<grid, 256, 0, st>>>((const bf16*)X, (const float*)Y, n, kv, part, nblk);
+        count_launch(), frob_partial_kernel<bf16, float><<<grid, 256, 0, st>>>((const bf16*)X, (const float*)Y, n, kv, part, nblk);
       else
-        frob_partial_kernel<bf16, bf16><<<grid, 256, 0, st>>>((const bf16*)X, (const bf16*)Y, n, kv, part, nblk);
+        count_launch(), frob_partial_kernel<bf16, bf16><<<grid, 256, 0, st>>>((const bf16*)X, (const bf16*)Y, n, kv, part, nblk);
     } else {
       if (ydtype == JOLT_F32)
-        frob_partial_kernel<float, float><<<grid, 256, 0, st>>>((const float*)X, (const float*)Y, n, kv, part, nblk);
+        count_launch(), frob_partial_kernel<float, float><<<grid, 256, 0, st>>>((const float*)X, (const float*)Y, n, kv, part, nblk);
       else
-        frob_partial_kernel<float, bf16><<<grid, 256, 0, st>>>((const float*)X, (const bf16*)Y, n, kv, part, nblk);
+        count_launch(), frob_partial_kernel<float, bf16><<<grid, 256, 0, st>>>((const float*)X, (const bf16*)Y, n, kv, part, nblk);
     }
     CUDA_TRY(cudaGetLastError());
   }
-  frob_final_kernel<<<(unsigned)ceil_div(2 * NU, 128), 128, 0, st>>>(part, NU, nblk, sq_dev);
+  count_launch(), frob_final_kernel<<<(unsigned)ceil_div(2 * NU, 128), 128, 0, st>>>(part, NU, nblk, sq_dev);
   CUDA_TRY(cudaGetLastError());
   return JOLT_OK;
 }

@@ -32,32 +32,74 @@ struct Cands {
 };
 
 // ---------------------------------------------------------------------------------------
-// exact fp16 directed-rounding helpers
+// exact fp16 directed rounding and the quantiser step, in FP32-pipe integer / float ops
+// (fp16 normal values are the floats whose low 13 mantissa bits are zero; other ranges
+// go through the conversion instructions)
 // ---------------------------------------------------------------------------------------
-__device__ __forceinline__ float fp16_rd(float x) { return __half2float(__float2half_rd(x)); }
+constexpr float kFp16MinNormal = 6.103515625e-05f;  // 2^-14
+constexpr float kFp16Max = 65504.f;
 
-// smallest fp16 s with s * levels >= mx - lo (exact), i.e. fp16 round-up of (mx - lo)/levels;
-// 0 when mx <= lo.  A float estimate is corrected by one fp16 ulp with exact fp64 checks.
-__device__ __forceinline__ float quant_step(float mx, float lo, int levels, float inv_levels) {
-  if (!(mx > lo)) return 0.f;
-  double need = (double)mx - (double)lo;
-  float q = (mx - lo) * inv_levels;
-  unsigned short u = __half_as_ushort(__float2half_ru(q));
-  double s = (double)__half2float(__ushort_as_half(u));
-  if (s * (double)levels < need) {
-    u = (unsigned short)(u + 1);
-  } else if (u > 0) {
-    unsigned short d = (unsigned short)(u - 1);
-    double sd = (double)__half2float(__ushort_as_half(d));
-    if (sd * (double)levels >= need) u = d;
+// fp16 round toward -inf (as __float2half_rd)
+__device__ __forceinline__ float rd16(float x) {
+  const float ax = fabsf(x);
+  if (ax >= kFp16MinNormal && ax <= kFp16Max) {
+    uint32_t u = __float_as_uint(x);
+    if (x >= 0.f) u &= ~0x1FFFu;
+    else if (u & 0x1FFFu) u = (u | 0x1FFFu) + 1u;
+    return __uint_as_float(u);
   }
-  return __half2float(__ushort_as_half(u));
+  return __half2float(__float2half_rd(x));
 }
 
-// round-half-even to integer of a non-negative float below 2^22 via the 1.5*2^23 shift
-__device__ __forceinline__ float rne_int(float q) {
-  const float magic = 12582912.0f;
-  return __fsub_rn(__fadd_rn(q, magic), magic);
+// fp16 round toward +inf of a positive float (as __float2half_ru)
+__device__ __forceinline__ float ru16_pos(float q) {
+  if (q >= kFp16MinNormal && q <= kFp16Max) {
+    uint32_t u = __float_as_uint(q);
+    if (u & 0x1FFFu) u = (u | 0x1FFFu) + 1u;
+    return __uint_as_float(u);
+  }
+  return __half2float(__float2half_ru(q));
+}
+
+// neighbouring fp16 values of a positive fp16 value s
+__device__ __forceinline__ float next16_up(float s) {
+  if (s >= kFp16MinNormal && s < kFp16Max) return __uint_as_float(__float_as_uint(s) + 0x2000u);
+  return __half2float(__ushort_as_half((unsigned short)(__half_as_ushort(__float2half_rn(s)) + 1)));
+}
+__device__ __forceinline__ float next16_down(float s) {
+  if (s > kFp16MinNormal && s <= kFp16Max) return __uint_as_float(__float_as_uint(s) - 0x2000u);
+  unsigned short h = __half_as_ushort(__float2half_rn(s));
+  return h ? __half2float(__ushort_as_half((unsigned short)(h - 1))) : 0.f;
+}
+
+// a >= mx - lo, decided exactly (R is the rounded difference)
+__device__ __forceinline__ bool ge_exact(float a, float mx, float lo, float R) {
+  if (a > R * 1.0000002384185791f) return true;
+  if (a < R * 0.9999997615814209f) return false;
+  return (double)a >= (double)mx - (double)lo;
+}
+
+// quantiser step: the smallest fp16 s with s * levels >= mx - lo exactly (the fp16
+// round-up of (mx - lo)/levels); 0 when mx <= lo.  A float estimate is corrected by one
+// fp16 step where needed.
+__device__ __forceinline__ float quant_step(float mx, float lo, float flev, float inv_lev) {
+  if (!(mx > lo)) return 0.f;
+  const float R = mx - lo;
+  float s = ru16_pos(R * inv_lev);
+  if (!(s <= kFp16Max)) return s;  // +inf: this block cannot be stored with this many bits
+  if (!ge_exact(s * flev, mx, lo, R)) {
+    s = next16_up(s);
+  } else {
+    float sp = next16_down(s);
+    if (sp > 0.f && ge_exact(sp * flev, mx, lo, R)) s = sp;
+  }
+  return s;
+}
+
+// round-half-even of d * inv to an integer-valued float: one FMA onto the 1.5*2^23 shift
+constexpr float kRoundShift = 12582912.0f;
+__device__ __forceinline__ float code_of(float d, float inv) {
+  return __fsub_rn(__fmaf_rn(d, inv, kRoundShift), kRoundShift);
 }
 
 // ---------------------------------------------------------------------------------------
@@ -231,20 +273,116 @@ __device__ __forceinline__ void recon_walk(bf16* smem_stages, const bf16* U, lon
   cp_async_wait<0>();
 }
 
-// per-row block min / max of rho = x' - acc over block m (n8 tiles 2m, 2m+1), quad-reduced
+// ---------------------------------------------------------------------------------------
+// residual tile in shared memory: the fragment owners write rho = x' - acc, then every
+// thread quantises whole 16-wide blocks of one row (row = tid % 64, blocks of one half row)
+// ---------------------------------------------------------------------------------------
 template <int D>
-__device__ __forceinline__ void block_vals(const TileFrag<D>& xf, float (*acc)[4], int h, int m, float* r) {
-  r[0] = xf.v[h][2 * m][0] - acc[2 * m][h * 2 + 0];
-  r[1] = xf.v[h][2 * m][1] - acc[2 * m][h * 2 + 1];
-  r[2] = xf.v[h][2 * m + 1][0] - acc[2 * m + 1][h * 2 + 0];
-  r[3] = xf.v[h][2 * m + 1][1] - acc[2 * m + 1][h * 2 + 1];
+struct RhoTile {
+  static constexpr int LD = D + 4;                 // row pitch (floats)
+  static constexpr int BLK_PER_ROW = D / 16;
+  static constexpr int BLK_PER_THREAD = (TROWS * BLK_PER_ROW) / TTHREADS;  // 4 for D = 128
+  static constexpr size_t BYTES = (size_t)TROWS * LD * 4;
+};
+
+template <int D>
+__device__ __forceinline__ void write_rho(float* rho, const TileFrag<D>& xf, float (*acc)[4]) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int r = warp * 16 + (lane >> 2) + h * 8;
+#pragma unroll
+    for (int j = 0; j < D / 8; ++j) {
+      const int c = j * 8 + (lane & 3) * 2;
+      float2 v = make_float2(xf.v[h][j][0] - acc[j][h * 2 + 0], xf.v[h][j][1] - acc[j][h * 2 + 1]);
+      *reinterpret_cast<float2*>(rho + r * RhoTile<D>::LD + c) = v;
+    }
+  }
 }
 
-__device__ __forceinline__ void quad_minmax(float& mn, float& mx) {
-  mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, 1));
-  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-  mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, 2));
-  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+// blocks handled by this thread: row tid % 64, blocks [ (tid / 64) * BPT, +BPT ) of that row;
+// D = 16 has one block per row, held by the first 64 threads
+template <int D>
+__device__ __forceinline__ int block_row() { return threadIdx.x % TROWS; }
+template <int D>
+__device__ __forceinline__ int block_first() {
+  return (RhoTile<D>::BLK_PER_THREAD > 0) ? (threadIdx.x / TROWS) * RhoTile<D>::BLK_PER_THREAD : 0;
+}
+template <int D>
+__host__ __device__ constexpr int blocks_per_thread() { return RhoTile<D>::BLK_PER_THREAD > 0 ? RhoTile<D>::BLK_PER_THREAD : 1; }
+
+__device__ __forceinline__ void load16(const float* src, float* v) {
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    float4 t = reinterpret_cast<const float4*>(src)[q];
+    v[4 * q + 0] = t.x;
+    v[4 * q + 1] = t.y;
+    v[4 * q + 2] = t.z;
+    v[4 * q + 3] = t.w;
+  }
+}
+
+__device__ __forceinline__ void minmax16(const float* v, float& mn, float& mx) {
+  float a0 = fminf(v[0], v[1]), a1 = fminf(v[2], v[3]), a2 = fminf(v[4], v[5]), a3 = fminf(v[6], v[7]);
+  float a4 = fminf(v[8], v[9]), a5 = fminf(v[10], v[11]), a6 = fminf(v[12], v[13]), a7 = fminf(v[14], v[15]);
+  mn = fminf(fminf(fminf(a0, a1), fminf(a2, a3)), fminf(fminf(a4, a5), fminf(a6, a7)));
+  float b0 = fmaxf(v[0], v[1]), b1 = fmaxf(v[2], v[3]), b2 = fmaxf(v[4], v[5]), b3 = fmaxf(v[6], v[7]);
+  float b4 = fmaxf(v[8], v[9]), b5 = fmaxf(v[10], v[11]), b6 = fmaxf(v[12], v[13]), b7 = fmaxf(v[14], v[15]);
+  mx = fmaxf(fmaxf(fmaxf(b0, b1), fmaxf(b2, b3)), fmaxf(fmaxf(b4, b5), fmaxf(b6, b7)));
+}
+
+// per-bit-width constants of the candidate set (b = 0 marks "no residual")
+struct BitConsts {
+  float flev[MAXC], inv[MAXC];
+  int bits[MAXC];
+  int n;
+};
+__device__ __forceinline__ BitConsts bit_consts(const Cands& cd) {
+  BitConsts k;
+  k.n = cd.nB;
+#pragma unroll
+  for (int i = 0; i < MAXC; ++i) {
+    int b = i < cd.nB ? cd.bits[i] : 0;
+    k.bits[i] = b;
+    k.flev[i] = (float)((1 << b) - 1);
+    k.inv[i] = b > 0 ? 1.0f / k.flev[i] : 0.f;
+  }
+  return k;
+}
+
+// squared quantisation error of one 16-wide block for every bit-width (added into err)
+__device__ __forceinline__ void block_errors(const float* v, const BitConsts& k, float* err) {
+  float mn, mx;
+  minmax16(v, mn, mx);
+  const float lo = rd16(mn);
+  float d[16];
+#pragma unroll
+  for (int j = 0; j < 16; ++j) d[j] = v[j] - lo;
+#pragma unroll
+  for (int ib = 0; ib < MAXC; ++ib) {
+    if (ib >= k.n) break;
+    if (k.bits[ib] == 0) {
+      float e0 = 0.f;
+#pragma unroll
+      for (int j = 0; j < 16; ++j) e0 = fmaf(v[j], v[j], e0);
+      err[ib] += e0;
+      continue;
+    }
+    const float step = quant_step(mx, lo, k.flev[ib], k.inv[ib]);
+    if (!(isfinite(lo) && step <= kFp16Max)) {
+      err[ib] = INFINITY;
+      continue;
+    }
+    const float inv = step > 0.f ? __frcp_rn(step) : 0.f;
+    float e2 = 0.f;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      const float c = code_of(d[j], inv);
+      const float e = fmaf(-c, step, d[j]);
+      e2 = fmaf(e, e, e2);
+    }
+    err[ib] += e2;
+  }
 }
 
 // ---------------------------------------------------------------------------------------
@@ -263,13 +401,18 @@ struct TableArgs {
   int tiles;
 };
 
+template <int D>
+inline size_t table_smem() {
+  return RhoTile<D>::BYTES + 2 * (size_t)ReconSmem<D>::STAGE * sizeof(bf16);
+}
+
 template <int D, typename TX>
 __global__ void __launch_bounds__(TTHREADS) table_kernel(TableArgs a) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
-  float* xs = reinterpret_cast<float*>(smem_raw);                          // TROWS x (D+4)
-  bf16* stages = reinterpret_cast<bf16*>(smem_raw + TROWS * (D + 4) * 4);   // 2 stages
+  float* rho = reinterpret_cast<float*>(smem_raw);                                   // TROWS x LD
+  bf16* stages = reinterpret_cast<bf16*>(smem_raw + RhoTile<D>::BYTES);                // 2 stages
   __shared__ float sig[D];
-  __shared__ float red[4][MAXC];
+  __shared__ float red[TTHREADS / 32][MAXC];
 
   const int tile = blockIdx.x, s = blockIdx.y, u = blockIdx.z;
   const int T = a.cv.T;
@@ -277,17 +420,20 @@ __global__ void __launch_bounds__(TTHREADS) table_kernel(TableArgs a) {
   const TX* X = reinterpret_cast<const TX*>(a.cv.unit_ptr(u)) + (long long)s * T * D;
   for (int d = threadIdx.x; d < D; d += blockDim.x) sig[d] = rotation_sign(a.seed, u, d);
   __syncthreads();
-  rotate_tile_to_smem<D, TX>(X, T, t0, sig, xs);
+  rotate_tile_to_smem<D, TX>(X, T, t0, sig, rho);   // x' staged through the rho buffer
   __syncthreads();
   TileFrag<D> xf;
-  frag_from_smem<D>(xs, xf);
+  frag_from_smem<D>(rho, xf);
   __syncthreads();
 
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const Cands& cd = a.cand;
+  const BitConsts kb = bit_consts(cd);
   const bf16* U = a.U + (long long)u * a.sU;
   constexpr int NT = D / 8;
   double* out = a.partial + (((long long)u * a.cv.S + s) * a.tiles + tile) * (long long)(cd.nD * cd.nT * cd.nB);
+  const int brow = block_row<D>();
+  const bool has_blocks = (RhoTile<D>::BLK_PER_THREAD > 0) || threadIdx.x < TROWS;
 
   for (int iD = 0; iD < cd.nD; ++iD) {
     const bf16* P = a.P + (long long)u * a.sP_unit + iD * a.sP_rd + (long long)s * a.rTmax * D;
@@ -298,48 +444,20 @@ __global__ void __launch_bounds__(TTHREADS) table_kernel(TableArgs a) {
       for (int e = 0; e < 4; ++e) acc[j][e] = 0.f;
 
     auto epi = [&](int iT) {
+      write_rho<D>(rho, xf, acc);
+      __syncthreads();
       float err[MAXC];
 #pragma unroll
       for (int ib = 0; ib < MAXC; ++ib) err[ib] = 0.f;
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-#pragma unroll
-        for (int m = 0; m < D / 16; ++m) {
-          float r[4];
-          block_vals<D>(xf, acc, h, m, r);
-          float mn = fminf(fminf(r[0], r[1]), fminf(r[2], r[3]));
-          float mx = fmaxf(fmaxf(r[0], r[1]), fmaxf(r[2], r[3]));
-          quad_minmax(mn, mx);
-          float lo = fp16_rd(mn);
-          float dd[4];
-#pragma unroll
-          for (int i = 0; i < 4; ++i) dd[i] = r[i] - lo;
-#pragma unroll
-          for (int ib = 0; ib < MAXC; ++ib) {
-            if (ib >= cd.nB) break;
-            int b = cd.bits[ib];
-            if (b == 0) {
-#pragma unroll
-              for (int i = 0; i < 4; ++i) err[ib] = fmaf(r[i], r[i], err[ib]);
-              continue;
-            }
-            int levels = (1 << b) - 1;
-            float step = quant_step(mx, lo, levels, 1.0f / (float)levels);
-            if (!(isfinite(lo) && isfinite(step))) {
-              err[ib] = INFINITY;
-              continue;
-            }
-            float inv = step > 0.f ? 1.0f / step : 0.f;
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              float code = rne_int(dd[i] * inv);
-              float e = fmaf(-code, step, dd[i]);
-              err[ib] = fmaf(e, e, err[ib]);
-            }
-          }
+      if (has_blocks) {
+#pragma unroll 1
+        for (int q = 0; q < blocks_per_thread<D>(); ++q) {
+          float v[16];
+          load16(rho + brow * RhoTile<D>::LD + (block_first<D>() + q) * 16, v);
+          block_errors(v, kb, err);
         }
       }
-      // reduce over the warp, then over the 4 warps in fixed order (fp64)
+      // reduce over the warp, then over the warps in fixed order (fp64)
 #pragma unroll
       for (int ib = 0; ib < MAXC; ++ib) {
         if (ib >= cd.nB) break;
@@ -351,18 +469,13 @@ __global__ void __launch_bounds__(TTHREADS) table_kernel(TableArgs a) {
       __syncthreads();
       if (threadIdx.x < cd.nB) {
         double v = 0.0;
-        for (int w = 0; w < 4; ++w) v += (double)red[w][threadIdx.x];
+        for (int w = 0; w < TTHREADS / 32; ++w) v += (double)red[w][threadIdx.x];
         out[(iD * cd.nT + iT) * cd.nB + threadIdx.x] = v;
       }
-      __syncthreads();
     };
     recon_walk<D>(stages, U, a.ldU, T, t0, P, cd.rT[cd.nT - 1], cd.rT, cd.nT, acc, epi);
+    __syncthreads();
   }
-}
-
-template <int D>
-inline size_t table_smem() {
-  return (size_t)TROWS * (D + 4) * 4 + 2 * (size_t)ReconSmem<D>::STAGE * sizeof(bf16);
 }
 
 // ---------------------------------------------------------------------------------------
@@ -402,8 +515,8 @@ struct EncodeArgs {
 template <int D, typename TX>
 __global__ void __launch_bounds__(TTHREADS) encode_kernel(EncodeArgs a) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
-  float* xs = reinterpret_cast<float*>(smem_raw);
-  bf16* stages = reinterpret_cast<bf16*>(smem_raw + TROWS * (D + 4) * 4);
+  float* rho = reinterpret_cast<float*>(smem_raw);
+  bf16* stages = reinterpret_cast<bf16*>(smem_raw + RhoTile<D>::BYTES);
   __shared__ float sig[D];
 
   const int tile = blockIdx.x, s = blockIdx.y, u = blockIdx.z;
@@ -420,13 +533,12 @@ __global__ void __launch_bounds__(TTHREADS) encode_kernel(EncodeArgs a) {
   const TX* X = reinterpret_cast<const TX*>(a.cv.unit_ptr(u)) + (long long)s * T * D;
   for (int d = threadIdx.x; d < D; d += blockDim.x) sig[d] = rotation_sign(a.seed, u, d);
   __syncthreads();
-  rotate_tile_to_smem<D, TX>(X, T, t0, sig, xs);
+  rotate_tile_to_smem<D, TX>(X, T, t0, sig, rho);
   __syncthreads();
   TileFrag<D> xf;
-  frag_from_smem<D>(xs, xf);
+  frag_from_smem<D>(rho, xf);
   __syncthreads();
 
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   constexpr int NT = D / 8;
   const bf16* U = a.U + (long long)u * a.sU;
   const bf16* P = a.P + (long long)u * a.sP_unit + iD * a.sP_rd + (long long)s * a.rTmax * D;
@@ -436,50 +548,51 @@ __global__ void __launch_bounds__(TTHREADS) encode_kernel(EncodeArgs a) {
 #pragma unroll
     for (int e = 0; e < 4; ++e) acc[j][e] = 0.f;
 
-  const int levels = (1 << b) - 1;
-  const float inv_levels = 1.0f / (float)levels;
+  const float flev = (float)((1 << b) - 1);
+  const float inv_lev = 1.0f / flev;
   unsigned char* codes = a.blob + uh.off_codes;
   __half2* scales = reinterpret_cast<__half2*>(a.blob + uh.off_scales);
-  const int q = lane & 3;
+  const int brow = block_row<D>();
+  const bool has_blocks = (RhoTile<D>::BLK_PER_THREAD > 0) || threadIdx.x < TROWS;
 
   auto epi = [&](int) {
+    write_rho<D>(rho, xf, acc);
+    __syncthreads();
+    const int t = t0 + brow;
+    if (!has_blocks || t >= T) return;
+#pragma unroll 1
+    for (int q = 0; q < blocks_per_thread<D>(); ++q) {
+      const int m = block_first<D>() + q;
+      float v[16];
+      load16(rho + brow * RhoTile<D>::LD + m * 16, v);
+      float mn, mx;
+      minmax16(v, mn, mx);
+      const float lo = rd16(mn);
+      const float step = quant_step(mx, lo, flev, inv_lev);
+      const float inv = (step > 0.f && step <= kFp16Max) ? __frcp_rn(step) : 0.f;
+      uint32_t w[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      int t = t0 + warp * 16 + (lane >> 2) + h * 8;
-#pragma unroll
-      for (int m = 0; m < D / 16; ++m) {
-        float r[4];
-        block_vals<D>(xf, acc, h, m, r);
-        float mn = fminf(fminf(r[0], r[1]), fminf(r[2], r[3]));
-        float mx = fmaxf(fmaxf(r[0], r[1]), fmaxf(r[2], r[3]));
-        quad_minmax(mn, mx);
-        float lo = fp16_rd(mn);
-        float step = quant_step(mx, lo, levels, inv_levels);
-        float inv = step > 0.f ? 1.0f / step : 0.f;
-        // columns inside the block held by this thread: 2q, 2q+1, 8+2q, 9+2q
-        uint32_t w[4] = {0u, 0u, 0u, 0u};
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          int col = (i >> 1) * 8 + 2 * q + (i & 1);
-          float c = rne_int((r[i] - lo) * inv);
-          c = fminf(fmaxf(c, 0.f), (float)levels);
-          uint32_t code = (uint32_t)c;
-          int pos = col * b;
-          w[pos >> 5] |= code << (pos & 31);
-          if ((pos & 31) + b > 32) w[(pos >> 5) + 1] |= code >> (32 - (pos & 31));
-        }
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          w[i] |= __shfl_xor_sync(0xffffffffu, w[i], 1);
-          w[i] |= __shfl_xor_sync(0xffffffffu, w[i], 2);
-        }
-        if (q == 0 && t < T) {
-          long long blk = ((long long)s * T + t) * (D / 16) + m;
-          unsigned char* dst = codes + blk * (2 * b);
-          for (int byte = 0; byte < 2 * b; ++byte) dst[byte] = (unsigned char)(w[byte >> 2] >> ((byte & 3) * 8));
-          scales[blk] = __halves2half2(__float2half_rn(lo), __float2half_rn(step));
-        }
+      for (int j = 0; j < 16; ++j) {
+        float c = code_of(v[j] - lo, inv);
+        c = fminf(fmaxf(c, 0.f), flev);
+        const uint32_t code = (uint32_t)c;
+        const int pos = j * b;
+        w[pos >> 5] |= code << (pos & 31);
+        if ((pos & 31) + b > 32) w[(pos >> 5) + 1] |= code >> (32 - (pos & 31));
       }
+      const long long blk = ((long long)s * T + t) * (D / 16) + m;
+      unsigned char* dst = codes + blk * (2 * b);
+      // 2b bytes; the block start is 2b-aligned
+      if (b == 8) {
+        *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+      } else if (b == 4) {
+        *reinterpret_cast<uint2*>(dst) = make_uint2(w[0], w[1]);
+      } else if (b == 2) {
+        *reinterpret_cast<uint32_t*>(dst) = w[0];
+      } else {
+        for (int byte = 0; byte < 2 * b; ++byte) dst[byte] = (unsigned char)(w[byte >> 2] >> ((byte & 3) * 8));
+      }
+      scales[blk] = __halves2half2(__float2half_rn(lo), __float2half_rn(step));
     }
   };
   int cut = uh.r_T;

@@ -181,6 +181,117 @@ __global__ void tril_zero_kernel(double* A, int n, long long lda, long long sA, 
   }
 }
 
+// Guard in front of every eigen / Cholesky call: if the cache was flagged non-finite, or the
+// matrix itself holds a NaN / Inf, the matrix is replaced by the identity (the status word
+// records the error), so the solver only ever sees finite input.  One block per call.
+__global__ void sanitize_sym_kernel(double* A, int n, long long lda, uint32_t* status) {
+  __shared__ int bad;
+  if (threadIdx.x == 0) bad = (*status & DEV_ERR_NONFINITE) ? 1 : 0;
+  __syncthreads();
+  for (long long i = threadIdx.x; i < (long long)n * n && !bad; i += blockDim.x) {
+    long long r = i / n, c = i - r * n;
+    if (!isfinite(A[c * lda + r])) bad = 1;
+  }
+  __syncthreads();
+  if (!bad) return;
+  if (threadIdx.x == 0) raise_status(status, DEV_ERR_NONFINITE);
+  for (long long i = threadIdx.x; i < (long long)n * n; i += blockDim.x) {
+    long long r = i / n, c = i - r * n;
+    A[c * lda + r] = (r == c) ? 1.0 : 0.0;
+  }
+}
+
+// batched guard: one block per matrix (stride sA between matrices)
+__global__ void sanitize_sym_batched_kernel(double* A, int n, long long lda, long long sA, uint32_t* status) {
+  double* M = A + blockIdx.x * sA;
+  __shared__ int bad;
+  if (threadIdx.x == 0) bad = (*status & DEV_ERR_NONFINITE) ? 1 : 0;
+  __syncthreads();
+  for (long long i = threadIdx.x; i < (long long)n * n && !bad; i += blockDim.x) {
+    long long r = i / n, c = i - r * n;
+    if (!isfinite(M[c * lda + r])) bad = 1;
+  }
+  __syncthreads();
+  if (!bad) return;
+  if (threadIdx.x == 0) raise_status(status, DEV_ERR_NONFINITE);
+  for (long long i = threadIdx.x; i < (long long)n * n; i += blockDim.x) {
+    long long r = i / n, c = i - r * n;
+    M[c * lda + r] = (r == c) ? 1.0 : 0.0;
+  }
+}
+
+// device pointer array for the batched Cholesky: P[u] = A + u * sA
+__global__ void ptr_array_kernel(double** P, double* A, long long sA, int n) {
+  int u = blockIdx.x * blockDim.x + threadIdx.x;
+  if (u < n) P[u] = A + (long long)u * sA;
+}
+
+// Q = Y L^{-T} in place (Q L^T = Y), row by row, for every unit: Y [rows x k] fp32 (ld,
+// stride sY per unit), L lower triangular k x k, column-major fp64 (lda, stride sL).  A CTA
+// owns RT rows (one thread each); columns go in blocks of 32: the block's right-hand side is
+// updated with the already solved columns (L rows staged through shared memory in chunks),
+// then the 32 x 32 diagonal triangle is solved in registers.
+constexpr int TRSM_NB = 32;
+constexpr int TRSM_PC = 256;
+template <int RT>
+__global__ void __launch_bounds__(RT) trsm_rows_kernel(float* Y, long long ld, long long sY, long long rows, int k,
+                                                       const double* L, long long lda, long long sL) {
+  extern __shared__ __align__(16) float tsm[];
+  const int ldq = k + 1;
+  float* Qs = tsm;                          // RT x ldq: solved columns of this CTA's rows
+  float* Lp = Qs + RT * ldq;                // TRSM_NB x (TRSM_PC + 1): chunk of L rows
+  float* Ld = Lp + TRSM_NB * (TRSM_PC + 1); // TRSM_NB x (TRSM_NB + 1): diagonal block
+  const int u = blockIdx.y;
+  const long long row = (long long)blockIdx.x * RT + threadIdx.x;
+  const bool valid = row < rows;
+  float* y = Y + (long long)u * sY + row * ld;
+  const double* Lu = L + (long long)u * sL;
+  for (int J = 0; J < k; J += TRSM_NB) {
+    const int nb = min(TRSM_NB, k - J);
+    float acc[TRSM_NB];
+#pragma unroll
+    for (int c = 0; c < TRSM_NB; ++c) acc[c] = (valid && c < nb) ? y[J + c] : 0.f;
+    for (int pc = 0; pc < J; pc += TRSM_PC) {
+      const int np = min(TRSM_PC, J - pc);
+      __syncthreads();
+      for (int idx = threadIdx.x; idx < TRSM_NB * np; idx += RT) {
+        int c = idx / np, q = idx - c * np;
+        Lp[c * (TRSM_PC + 1) + q] = c < nb ? (float)Lu[(long long)(pc + q) * lda + (J + c)] : 0.f;
+      }
+      __syncthreads();
+      for (int q = 0; q < np; ++q) {
+        const float qv = Qs[threadIdx.x * ldq + pc + q];
+#pragma unroll
+        for (int c = 0; c < TRSM_NB; ++c) acc[c] = fmaf(-qv, Lp[c * (TRSM_PC + 1) + q], acc[c]);
+      }
+    }
+    __syncthreads();
+    for (int idx = threadIdx.x; idx < TRSM_NB * TRSM_NB; idx += RT) {
+      int c = idx / TRSM_NB, q = idx - c * TRSM_NB;
+      Ld[c * (TRSM_NB + 1) + q] = (c < nb && q < nb) ? (float)Lu[(long long)(J + q) * lda + (J + c)] : 0.f;
+    }
+    __syncthreads();
+    float x[TRSM_NB];
+#pragma unroll
+    for (int c = 0; c < TRSM_NB; ++c) {
+      float v = acc[c];
+#pragma unroll
+      for (int q = 0; q < c; ++q) v = fmaf(-x[q], Ld[c * (TRSM_NB + 1) + q], v);
+      const float dgl = Ld[c * (TRSM_NB + 1) + c];
+      x[c] = (c < nb && dgl != 0.f) ? v / dgl : 0.f;
+    }
+#pragma unroll
+    for (int c = 0; c < TRSM_NB; ++c)
+      if (c < nb) Qs[threadIdx.x * ldq + J + c] = x[c];
+  }
+  if (!valid) return;
+  for (int c = 0; c < k; ++c) y[c] = Qs[threadIdx.x * ldq + c];
+}
+
+inline size_t trsm_smem(int RT, int k) {
+  return ((size_t)RT * (k + 1) + (size_t)TRSM_NB * (TRSM_PC + 1) + (size_t)TRSM_NB * (TRSM_NB + 1)) * 4;
+}
+
 __global__ void info_check_kernel(const int* info, int n, uint32_t* status, uint32_t bits) {
   int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i < n && info[i] != 0) raise_status(status, bits);
@@ -250,20 +361,9 @@ __global__ void bytes_table_kernel(unsigned long long* B, int nunits, int T, int
   B[idx] = unit_payload_bytes(T, D, S, cd.rT[iT], cd.rD[iD], cd.bits[ib]);
 }
 
-// argmin_c D[c] + lam*B[c] with two separate roundings; ties -> fewer bytes -> lower index
-__device__ __forceinline__ int lagrangian_argmin(const double* Dr, const unsigned long long* Br, int nc, double lam) {
-  double bv = 0.0;
-  unsigned long long bb = 0ull;
-  int bc = -1;
-  for (int c = 0; c < nc; ++c) {
-    double v = __dadd_rn(Dr[c], __dmul_rn(lam, (double)Br[c]));
-    bool better = (bc < 0) || (v < bv) || (v == bv && Br[c] < bb);
-    // NaN never occurs: D is finite or +inf and lam*B is finite or +inf
-    if (better) { bv = v; bb = Br[c]; bc = c; }
-  }
-  return bc;
-}
-
+// Per unit, argmin_c D[c] + lam*B[c] with two separate roundings (no fused multiply-add);
+// ties go to fewer bytes, then to the lower choice index.  D is finite or +inf and lam*B is
+// finite or +inf, so no NaN is compared.
 struct AllocArgs {
   const double* D;
   const unsigned long long* B;
@@ -282,11 +382,33 @@ struct AllocArgs {
   const int32_t* forced;           // optional caller choices: skip the search, fill the headers
 };
 
+// F(lam): every unit's Lagrangian choice (one warp per unit, lanes over the choices, then a
+// lexicographic (value, bytes, index) reduction), and the total bytes
 __device__ unsigned long long alloc_F(const AllocArgs& a, double lam, int* sch, unsigned long long* sB) {
-  for (int u = threadIdx.x; u < a.nunits; u += blockDim.x) {
-    int c = lagrangian_argmin(a.D + (long long)u * a.nc, a.B + (long long)u * a.nc, a.nc, lam);
-    sch[u] = c;
-    sB[u] = a.B[(long long)u * a.nc + c];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+  for (int u = warp; u < a.nunits; u += nwarps) {
+    const double* Dr = a.D + (long long)u * a.nc;
+    const unsigned long long* Br = a.B + (long long)u * a.nc;
+    double bv = 0.0;
+    unsigned long long bb = 0ull;
+    int bc = -1;
+    for (int c = lane; c < a.nc; c += 32) {
+      double v = __dadd_rn(Dr[c], __dmul_rn(lam, (double)Br[c]));
+      bool better = (bc < 0) || (v < bv) || (v == bv && Br[c] < bb);
+      if (better) { bv = v; bb = Br[c]; bc = c; }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      double ov = __shfl_xor_sync(0xffffffffu, bv, o);
+      unsigned long long ob = __shfl_xor_sync(0xffffffffu, bb, o);
+      int oc = __shfl_xor_sync(0xffffffffu, bc, o);
+      bool take = (oc >= 0) && ((bc < 0) || (ov < bv) || (ov == bv && (ob < bb || (ob == bb && oc < bc))));
+      if (take) { bv = ov; bb = ob; bc = oc; }
+    }
+    if (lane == 0) {
+      sch[u] = bc;
+      sB[u] = Br[bc];
+    }
   }
   __syncthreads();
   unsigned long long tot = 0ull;

@@ -27,7 +27,8 @@ STATUS_NAMES = {
 EXPORTED = [
     "jolt_version", "jolt_last_error", "jolt_workspace_size", "jolt_counts", "jolt_choice_bytes",
     "jolt_compress", "jolt_factor", "jolt_table", "jolt_allocate", "jolt_encode", "jolt_read_header",
-    "jolt_decompress", "jolt_frobenius",
+    "jolt_decompress", "jolt_frobenius", "jolt_profile_begin", "jolt_profile_end", "jolt_recon_operator",
+    "jolt_launch_count",
 ]
 
 
@@ -84,7 +85,12 @@ def lib():
             "jolt_read_header": [vp, pS, ctypes.POINTER(u64), ctypes.POINTER(CUnitRecord), i32, vp],
             "jolt_decompress": [vp, i32, vp, vp, vp, sz, vp],
             "jolt_frobenius": [pS, vp, vp, vp, vp, i32, vp, vp, sz, vp],
+            "jolt_recon_operator": [pS, pO, u64, vp, vp, ctypes.c_int64, vp, vp, sz, vp],
+            "jolt_profile_begin": [],
+            "jolt_profile_end": [ctypes.c_char_p, sz],
         }
+        L.jolt_launch_count.argtypes = []
+        L.jolt_launch_count.restype = ctypes.c_uint64
         for name, args in sigs.items():
             f = getattr(L, name)
             f.argtypes = args
@@ -251,6 +257,18 @@ class Compressor:
                                 _ptr(tab), self._ws_ptr(self.ws), self.ws_bytes, _stream(stream)))
         return core, tab
 
+    def recon_operator(self, core, W_bf16, seed: int = 0, stream=None):
+        """Rotated reconstruction operators P' [n_feature_ranks, units, S, max r_T, D] (bf16)."""
+        o = self.opts
+        S = self.shape.layers_per_group * self.shape.n_heads
+        P = torch.zeros((len(o.feature_ranks), self.n_units, S, max(o.token_ranks), self.shape.head_dim),
+                        dtype=torch.bfloat16, device=core.device)
+        W_bf16 = W_bf16.contiguous()
+        _check(lib().jolt_recon_operator(ctypes.byref(self.shape), ctypes.byref(self._copts), int(seed),
+                                         _ptr(core.contiguous()), _ptr(W_bf16), W_bf16.shape[-1], _ptr(P),
+                                         self._ws_ptr(self.ws), self.ws_bytes, _stream(stream)))
+        return P
+
     def encode(self, K, V, U_bf16, W_bf16, core, choice, dist, seed: int = 0, cap: int | None = None, stream=None):
         _check_cache(K, V)
         cap = self.blob_max if cap is None else cap
@@ -318,6 +336,27 @@ def frobenius(K, V, K_hat=None, V_hat=None, layers_per_group=1, stream=None):
     _check(lib().jolt_frobenius(ctypes.byref(shape), _ptr(K), _ptr(V), _ptr(K_hat), _ptr(V_hat), yd, _ptr(sq),
                                 _ptr(ws), ws.numel(), _stream(stream)))
     return sq.view(2 * G, 2)
+
+
+def launch_count() -> int:
+    """Kernels launched by the library in this process so far."""
+    return int(lib().jolt_launch_count())
+
+
+def profile_begin():
+    """Start recording CUDA events around every library stage on this thread."""
+    _check(lib().jolt_profile_begin())
+
+
+def profile_end():
+    """Stop recording; returns {stage: (total_ms, launches, units)} (synchronises)."""
+    buf = ctypes.create_string_buffer(1 << 16)
+    _check(lib().jolt_profile_end(buf, len(buf)))
+    out = {}
+    for line in buf.value.decode().splitlines():
+        name, ms, n, u = line.split()
+        out[name] = (float(ms), int(n), int(u))
+    return out
 
 
 def relative_errors(K, V, K_hat, V_hat, layers_per_group):

@@ -195,7 +195,7 @@ def unit_payload_bytes(T: int, D: int, S: int, r_T: int, r_D: int, b: int, block
     """Stored bytes of one unit: U (T x r_T), W (D x r_D), core (S x r_T x r_D) in bf16,
     plus, when b > 0, the packed b-bit codes (block*b/8 bytes per block) and one fp16
     (lo, step) pair per block.  Every array starts on a 16-byte boundary and the padding
-    counts ([Abstract]: "global byte constraint")."""
+    counts against the global byte limit ([Abstract])."""
     n = 2 * T * r_T
     n = pad16(n) + pad16(2 * D * r_D) + pad16(2 * S * r_T * r_D)
     if b > 0:
@@ -210,8 +210,8 @@ def header_bytes(n_units: int) -> int:
 
 # ----------------------------------------------------------------------------------------
 # Tensor views: the grouped prefill cache of one unit u = (group g, K or V) is the
-# fourth-order tensor X[l, h, t, d] over its L_g layers ([Abstract]: "treats grouped
-# prefill caches as fourth-order tensors"; [Blog], [Intro]: keys and values separately).
+# fourth-order tensor X[l, h, t, d] over its L_g layers ([Abstract]: the grouped prefill
+# cache is handled as a fourth-order tensor; [Blog], [Intro]: keys and values separately).
 # ----------------------------------------------------------------------------------------
 def units_of(K: np.ndarray, V: np.ndarray, layers_per_group: int):
     """Yield (g, kv, X_unit[L_g, H, T, D]) in unit order u = 2 g + kv."""
@@ -290,8 +290,8 @@ def token_factor_exact(X: np.ndarray, r: int) -> np.ndarray:
 
 def token_factor_randomized(X: np.ndarray, r: int, oversample: int, power_iters: int,
                             seed: int, group: int, kv: int) -> np.ndarray:
-    """FlashJoLT: randomized token-mode SVD ([Abstract]: "replaces the exact token-mode SVD
-    with a randomized approximation").  Randomized subspace iteration in the form of
+    """FlashJoLT: randomized token-mode SVD in place of the exact one ([Abstract]).
+    Randomized subspace iteration in the form of
     Halko, Martinsson & Tropp (SIAM Review 2011), Algorithm 4.4: sketch Y = X_(T) Omega,
     orthonormalise after every product, then a Rayleigh-Ritz step (small SVD of
     B = Q^T X_(T) through the eigenvectors of B B^T)."""
@@ -333,8 +333,8 @@ def stored_core(X: np.ndarray, U_s: np.ndarray, W_s: np.ndarray) -> np.ndarray:
 
 
 # ----------------------------------------------------------------------------------------
-# Johnson-Lindenstrauss rotation of the residual ([Intro]: "JL rotated low-bit residual";
-# [Blog]: "Johnson-Lindenstrauss rotation"; [Wiki]: "random orthogonal rotation").
+# Johnson-Lindenstrauss rotation of the residual ([Intro], [Blog], [Wiki] "Methodology": a
+# random orthogonal rotation is applied before the few-bit quantiser).
 # Reading: along the feature axis of every row, rho = r diag(sigma) H_D / sqrt(D) with
 # H_D the Sylvester Hadamard matrix and sigma random signs; Phi = diag(sigma) H_D/sqrt(D)
 # is orthogonal, so the rotation preserves the residual's energy.
@@ -380,8 +380,8 @@ def recon_operator(C_s: np.ndarray, W_s: np.ndarray, sigma: np.ndarray, r_D: int
 
 
 # ----------------------------------------------------------------------------------------
-# Low-bit residual quantiser ([Abstract]: "A rotated low-bit quantizer captures the
-# truncation residual").  Reading: asymmetric min-max round-to-nearest per block of 16
+# Low-bit residual quantiser ([Abstract]: the truncation residual is stored by a rotated
+# few-bit quantiser).  Reading: asymmetric min-max round-to-nearest per block of 16
 # consecutive rotated features; lo = fp16 round-down of the block minimum, step =
 # fp16 round-up of (max - lo)/(2^b - 1); code = round-half-even((rho - lo)/step).
 # ----------------------------------------------------------------------------------------
@@ -450,10 +450,10 @@ def unpack_codes(packed: np.ndarray, b: int, block: int = 16) -> np.ndarray:
 
 
 # ----------------------------------------------------------------------------------------
-# Distortion table and the single Lagrangian dual ([Abstract]: "a single Lagrangian dual
-# allocates per-group Tucker ranks and residual bit-widths under a global byte
-# constraint"; [Intro]: "per layer group and separately for keys and values, under one
-# byte budget"; [Radio] "The Core Mechanism": bytes may move between K and V).
+# Distortion table and the single Lagrangian dual ([Abstract]: one dual sets the Tucker
+# ranks and residual bit-widths of every group under a single global byte limit; [Intro]:
+# per layer group, keys and values separately, one budget; [Radio] "The Core Mechanism":
+# bytes can move between the K and V sides).
 # ----------------------------------------------------------------------------------------
 def rotated_input(X: np.ndarray, sigma: np.ndarray) -> np.ndarray:
     return rotate(X, sigma)

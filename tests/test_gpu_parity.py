@@ -1,0 +1,350 @@
+"""Parity of the CUDA library (through the C ABI) with the float64 oracle on the same
+seeded inputs.  Tolerances:
+  factor subspaces        : largest principal-angle sine <= 1e-3 where the relative eigengap
+                            at the cut is >= 1e-4 (elsewhere the subspace is not determined)
+  stored core             : <= 1e-2 of entries differ, each by at most one bf16 step
+  reconstruction operator : same bound as the core (bf16 rounding of fp32 vs fp64 sums)
+  distortion table        : 1e-6 relative + 2 sqrt(entry) * 64 u_32 ||X|| (fp32 residual vs fp64)
+  block scales            : equal, except where the oracle's block minimum / maximum lies within
+                            w = 2^-17 (max|x'| + max|x_hat|) of an fp16 rounding boundary (the
+                            fp32 residual's absolute error); then the library's scale must be
+                            the rounding of a value inside that window
+  codes                   : <= 1e-4 of codes differ (under the library's scales), and only where
+                            the oracle's scaled value lies within w / step of a rounding tie
+  allocation              : bit-exact choices and lambda given identical tables
+  end to end              : relative Frobenius error within 1e-4 absolute of the oracle's
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from kv_cache_compression_group_b200 import jolt as J
+from kv_cache_compression_group_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+TINY_OPTS = ((4, 8, 16, 32), (4, 8, 16), (0, 2, 3, 4))
+
+
+def _case(name):
+    if name.startswith("tiny"):
+        w = synth.WORKLOADS["tiny"]
+        rt, rd, bits = TINY_OPTS
+        ratio = 2.0
+    elif name.startswith("mistral4"):
+        w = synth.small_workload("mistral7b", n_layers=4)
+        o = J.default_options(w.T, w.D)
+        rt, rd, bits = o.token_ranks, o.feature_ranks, o.bits
+        ratio = 2.0
+    elif name.startswith("mistral8"):
+        w = synth.small_workload("mistral7b", n_layers=8, n_heads=4)
+        o = J.default_options(w.T, w.D)
+        rt, rd, bits = o.token_ranks, o.feature_ranks, o.bits
+        ratio = 3.0
+    method = "randomized" if name.endswith("rand") else "exact"
+    return w, J.Options(rt, rd, bits, method), O.Options(rt, rd, bits, method), ratio
+
+
+CASES = ["tiny-exact", "tiny-rand", "mistral4-exact", "mistral4-rand", "mistral8-rand"]
+_cache = {}
+
+
+def _setup(name):
+    if name in _cache:
+        return _cache[name]
+    w, jo, oo, ratio = _case(name)
+    K, V = synth.make_cache(w, 0)
+    Kn, Vn = synth.to_f64(K), synth.to_f64(V)
+    budget = int(w.bf16_bytes() / ratio)
+    res = O.compress(Kn, Vn, w.layers_per_group, oo, budget, 0)
+    comp = J.Compressor(w.n_layers, w.n_heads, w.T, w.D, w.layers_per_group, K.dtype, jo)
+    units = list(O.units_of(Kn, Vn, w.layers_per_group))
+    d = dict(w=w, jo=jo, oo=oo, K=K.cuda(), V=V.cuda(), Kn=Kn, Vn=Vn, budget=budget, res=res, comp=comp,
+             units=units)
+    _cache[name] = d
+    return d
+
+
+def _bf16(a):
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(torch.bfloat16).cuda()
+
+
+def _sin_theta(U1, U2):
+    return float(np.linalg.norm(U2 - U1 @ (U1.T @ U2), 2))
+
+
+def _relgaps(vals, cuts):
+    v = np.sort(np.asarray(vals))[::-1]
+    out = []
+    for r in cuts:
+        out.append((v[r - 1] - v[r]) / v[0] if r < len(v) else 1.0)
+    return out
+
+
+@pytest.mark.parametrize("name", CASES)
+def test_factor_subspaces(name):
+    d = _setup(name)
+    U, W = d["comp"].factor(d["K"], d["V"], 0)
+    U = U.double().cpu().numpy()
+    W = W.double().cpu().numpy()
+    checked = 0
+    for u, f in enumerate(d["res"].factors):
+        X = d["units"][u][2]
+        A = O.token_unfolding(X)
+        gt = np.linalg.eigvalsh(A @ A.T if A.shape[0] <= A.shape[1] else A.T @ A)
+        for r, g in zip(d["oo"].token_ranks, _relgaps(gt, d["oo"].token_ranks)):
+            s = _sin_theta(f.U[:, :r], U[u][:, :r])
+            if g >= 1e-4:
+                assert s <= 1e-3, (u, r, s, g)
+                checked += 1
+        for r, g in zip(d["oo"].feature_ranks, _relgaps(f.w_eigvals, d["oo"].feature_ranks)):
+            s = _sin_theta(f.W[:, :r], W[u][:, :r])
+            if g >= 1e-4:
+                assert s <= 1e-3, (u, r, s, g)
+                checked += 1
+        assert np.abs(U[u].T @ U[u] - np.eye(U.shape[2])).max() < 1e-4
+        assert np.abs(W[u].T @ W[u] - np.eye(W.shape[2])).max() < 1e-4
+    assert checked > 0
+
+
+def _oracle_factors(d):
+    facs = d["res"].factors
+    Us = _bf16(np.stack([f.U_s for f in facs]))
+    Ws = _bf16(np.stack([f.W_s for f in facs]))
+    return facs, Us, Ws
+
+
+def _ulp_close(got, want, slack):
+    """fraction of entries that differ, and whether every difference is within one bf16 step
+    of the value plus `slack` (the absolute error the fp32 sums before the rounding may carry)."""
+    diff = got != want
+    frac = diff.mean()
+    step = np.abs(want) * 2.0 ** -7 * 1.0001 + slack
+    ok = np.all(np.abs(got - want)[diff] <= np.broadcast_to(step, want.shape)[diff])
+    return frac, ok
+
+
+@pytest.mark.parametrize("name", CASES)
+def test_core_table_and_operator(name):
+    d = _setup(name)
+    facs, Us, Ws = _oracle_factors(d)
+    core, tab = d["comp"].table(d["K"], d["V"], Us, Ws, 0)
+    core = core.double().cpu().numpy()
+    tab = tab.cpu().numpy()
+    P = d["comp"].recon_operator(torch.from_numpy(core).to(torch.bfloat16).cuda(), Ws, 0).double().cpu().numpy()
+    Lg, H = d["w"].layers_per_group, d["w"].n_heads
+    for u, f in enumerate(facs):
+        X = d["units"][u][2]
+        want = O.stored_core(X, f.U_s, f.W_s).reshape(core[u].shape)
+        # two bf16 rounding points (Z = bf16(X W), C = bf16(U^T Z)): fp32 sums flip a rounding
+        # of Z now and then (one bf16 step, 2^-8 relative), and a flipped Z entry moves every
+        # core sum that uses it by up to 2^-8 max|U| max|Z|; allow four such flips per sum
+        Z = O.bf16_rn(np.einsum("lhtd,dq->lhtq", X, f.W_s)).reshape(-1, X.shape[2], f.W_s.shape[1])
+        slack = 4 * 2.0 ** -8 * np.abs(f.U_s).max(0)[None, :, None] * np.abs(Z).max(1)[:, None, :]
+        frac, ok = _ulp_close(core[u], want, slack)
+        assert frac <= 1e-2 and ok, (u, frac)
+        Cg = core[u].reshape(Lg, H, *core[u].shape[1:])
+        for iD, rD in enumerate(d["oo"].feature_ranks):
+            Pw = O.recon_operator(Cg, f.W_s, f.sigma, rD).reshape(P[iD, u].shape)
+            frac, ok = _ulp_close(P[iD, u], Pw, 2.0 ** -16 * np.abs(Pw).max(-1, keepdims=True))
+            assert frac <= 1e-3 and ok, (u, rD, frac)
+        # the table kernel against the oracle's table built from the same stored core.
+        # The library forms rho in fp32: |d rho| <= c u_32 |x| per element, so an entry
+        # sum_i e_i^2 moves by at most 2 sqrt(entry) ||d rho|| (+ ties, which move e^2 by
+        # the same order); c = 64 covers the accumulation depth of the reconstruction.
+        tw = O.distortion_table(X, f.U_s, f.W_s, Cg, f.sigma, d["oo"]).reshape(-1)
+        fin = np.isfinite(tw)
+        assert np.array_equal(fin, np.isfinite(tab[u]))
+        xnorm = float(np.linalg.norm(X))
+        tol = 1e-6 * tw[fin] + 2 * np.sqrt(tw[fin]) * 64 * 2.0 ** -24 * xnorm
+        assert np.all(np.abs(tab[u][fin] - tw[fin]) <= tol), (u, np.max(np.abs(tab[u][fin] - tw[fin]) / tol))
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_allocation_bit_exact(seed):
+    rng = np.random.default_rng(seed)
+    nu = int(rng.integers(2, 21))
+    nc = int(rng.integers(8, 97))
+    B = rng.integers(1000, 10_000_000, size=(nu, nc)).astype(np.int64)
+    D = 1e9 / B * rng.uniform(0.2, 5.0, size=(nu, nc))
+    if seed % 2:
+        D[rng.random((nu, nc)) < 0.1] = np.inf      # unstorable choices
+        D[:, 0] = 1e12                              # fewest-bytes choice always finite
+        B[:, 0] = B.min() // 2
+    lo, hi = int(B.min(1).sum()), int(B.max(1).sum())
+    for budget in (lo, (lo + hi) // 3, (lo + hi) // 2, hi, hi * 2):
+        al = O.allocate(D, B, budget)
+        ch, lam, st = J.allocate(torch.from_numpy(D).cuda(), torch.from_numpy(B).cuda(), budget)
+        assert st.item() == 0
+        assert list(ch.cpu().numpy()) == list(al.choice), budget
+        assert lam.cpu().numpy()[0].tobytes() == np.float64(al.lam).tobytes(), (lam.item(), al.lam)
+    ch, lam, st = J.allocate(torch.from_numpy(D).cuda(), torch.from_numpy(B).cuda(), lo - 1)
+    assert st.item() == 4 and math.isinf(lam.item())
+
+
+def test_allocation_bit_exact_on_oracle_tables():
+    for name in ("tiny-exact", "mistral4-exact"):
+        d = _setup(name)
+        res = d["res"]
+        avail = d["budget"] - O.header_bytes(res.table.shape[0])
+        for frac in (0.6, 0.8, 1.0, 1.3):
+            b = int(avail * frac)
+            al = O.allocate(res.table, res.bytes, b)
+            ch, lam, st = J.allocate(torch.from_numpy(res.table).cuda(), torch.from_numpy(res.bytes).cuda(), b)
+            if al.status == "infeasible":
+                assert st.item() == 4
+                continue
+            assert list(ch.cpu().numpy()) == list(al.choice)
+            assert lam.cpu().numpy()[0].tobytes() == np.float64(al.lam).tobytes()
+
+
+def _blob_unit(blob_np, u, rec, w, block=16):
+    S = w.layers_per_group * w.n_heads
+    T, D = w.T, w.D
+
+    def bf(off, n):
+        return torch.from_numpy(blob_np[off:off + 2 * n].copy()).view(torch.bfloat16).double().numpy()
+
+    Ub = bf(rec["off_U"], T * rec["r_T"]).reshape(T, rec["r_T"])
+    Wb = bf(rec["off_W"], D * rec["r_D"]).reshape(D, rec["r_D"])
+    Cb = bf(rec["off_C"], S * rec["r_T"] * rec["r_D"]).reshape(S, rec["r_T"], rec["r_D"])
+    out = dict(U=Ub, W=Wb, C=Cb)
+    b = rec["bits"]
+    if b:
+        nblk = S * T * D // block
+        packed = blob_np[rec["off_codes"]:rec["off_codes"] + nblk * 2 * b].reshape(nblk, 2 * b)
+        out["codes"] = O.unpack_codes(packed, b).reshape(nblk, block)
+        sc = blob_np[rec["off_scales"]:rec["off_scales"] + nblk * 4].copy().view(np.float16).astype(np.float64)
+        out["lo"], out["step"] = sc[0::2], sc[1::2]
+    return out
+
+
+@pytest.mark.parametrize("name", CASES)
+def test_encode_codes_and_factors(name):
+    d = _setup(name)
+    res, w = d["res"], d["w"]
+    facs, Us, Ws = _oracle_factors(d)
+    core = _bf16(np.stack([f.C_s.reshape(-1, f.C_s.shape[-2], f.C_s.shape[-1]) for f in facs]))
+    choice = torch.tensor([r.choice for r in res.units], dtype=torch.int32)
+    dist = torch.from_numpy(res.table)
+    blob = d["comp"].encode(d["K"], d["V"], Us, Ws, core, choice, dist, 0)
+    _, total, recs = J.read_header(blob)
+    assert total == res.total_bytes
+    P = d["comp"].recon_operator(core, Ws, 0).double().cpu().numpy()
+    bnp = blob.cpu().numpy()
+    n_codes = n_bad = n_scales = n_scale_bad = 0
+    for u, (rec_o, rec_g) in enumerate(zip(res.units, recs)):
+        assert (rec_g["r_T"], rec_g["r_D"], rec_g["bits"]) == (rec_o.r_T, rec_o.r_D, rec_o.b)
+        g = _blob_unit(bnp, u, rec_g, w)
+        assert np.array_equal(g["U"], rec_o.U_s) and np.array_equal(g["W"], rec_o.W_s)
+        assert np.array_equal(g["C"], rec_o.C_s.reshape(g["C"].shape))
+        if not rec_o.b:
+            continue
+        # residual with the library's own reconstruction operator (same bf16 operands on both sides)
+        iD = d["oo"].feature_ranks.index(rec_o.r_D)
+        X = d["units"][u][2]
+        Pg = P[iD, u][:, :rec_o.r_T, :].reshape(w.layers_per_group, w.n_heads, rec_o.r_T, w.D)
+        rho = O.rotated_input(X, rec_o.sigma) - np.einsum("tr,lhrd->lhtd", rec_o.U_s, Pg)
+        codes, lo, step, _, _ = O.quantize(rho, rec_o.b)
+        codes, lo, step = codes.reshape(-1, 16), lo.reshape(-1), step.reshape(-1)
+        rb = rho.reshape(-1, 16)
+        # the library forms rho in fp32 from x' and the reconstruction: its error is absolute,
+        # bounded here per block by 2^-17 (max |x'| + max |x_hat|)
+        xr = O.rotated_input(X, rec_o.sigma).reshape(-1, 16)
+        win = 2.0 ** -17 * (np.abs(xr).max(1) + np.abs(xr - rb).max(1))
+        n_scales += lo.size
+        same = (g["lo"] == lo) & (g["step"] == step)
+        bad = np.nonzero(~same)[0]
+        n_scale_bad += bad.size
+        if bad.size:
+            # every differing scale is the rounding of a block minimum / maximum inside the window
+            L = (1 << rec_o.b) - 1
+            mn, mx, wb = rb[bad].min(1), rb[bad].max(1), win[bad]
+            lo_ok = (g["lo"][bad] >= O.fp16_rd(mn - wb)) & (g["lo"][bad] <= O.fp16_rd(mn + wb))
+            st_lo = O.fp16_ru(np.maximum(mx - wb - g["lo"][bad], 0) / L)
+            st_hi = O.fp16_ru((mx + wb - g["lo"][bad]) / L)
+            st_ok = (g["step"][bad] >= st_lo) & (g["step"][bad] <= st_hi)
+            assert np.all(lo_ok & st_ok), bad[~(lo_ok & st_ok)][:5]
+        # codes under the library's own scales, from the oracle's rho
+        gl, gs = g["lo"][:, None], g["step"][:, None]
+        q = (rb - gl) / np.where(gs > 0, gs, 1.0)
+        want = np.where(gs > 0, np.clip(np.rint(q), 0, (1 << rec_o.b) - 1), 0)
+        diff = g["codes"] != want
+        n_codes += want.size
+        n_bad += int(diff.sum())
+        if diff.any():
+            tie = np.abs(q - np.floor(q) - 0.5)
+            tw = (win[:, None] / np.where(gs > 0, gs, 1.0)) + 1e-6
+            assert np.all(tie[diff] <= np.broadcast_to(tw, tie.shape)[diff]), tie[diff].max()
+    assert n_scale_bad <= max(4, 2e-3 * n_scales), (n_scale_bad, n_scales)
+    if n_codes:
+        assert n_bad <= max(1, 1e-4 * n_codes), (n_bad, n_codes)
+
+
+@pytest.mark.parametrize("name", CASES)
+def test_end_to_end_against_oracle(name):
+    d = _setup(name)
+    comp, res, w = d["comp"], d["res"], d["w"]
+    blob = comp.compress(d["K"], d["V"], d["budget"], 0)
+    _, total, recs = J.read_header(blob)
+    assert total <= d["budget"]
+    assert [(r["r_T"], r["r_D"], r["bits"]) for r in recs] == [(u.r_T, u.r_D, u.b) for u in res.units]
+    Kh, Vh = comp.decompress(blob, torch.float32)
+    ek, ev = J.relative_errors(d["K"], d["V"], Kh, Vh, w.layers_per_group)
+    Ko, Vo = O.decompress(res)
+    assert abs(ek - O.relative_error(d["Kn"], Ko)) <= 1e-4
+    assert abs(ev - O.relative_error(d["Vn"], Vo)) <= 1e-4
+    # round trip: the measured error of every unit is the table entry it was chosen by
+    sq = J.frobenius(d["K"], d["V"], Kh, Vh, w.layers_per_group).cpu().numpy()
+    for u, r in enumerate(recs):
+        assert abs(sq[u, 1] - r["distortion"]) <= 1e-5 * max(sq[u, 1], 1e-30) + 1e-9 * sq[u, 0]
+    # bf16 output is the bf16 rounding of the fp32 output
+    Kb, Vb = comp.decompress(blob, torch.bfloat16)
+    assert torch.equal(Kb, Kh.to(torch.bfloat16)) and torch.equal(Vb, Vh.to(torch.bfloat16))
+    # deterministic: a second compress gives the same bytes
+    blob2 = comp.compress(d["K"], d["V"], d["budget"], 0)
+    assert torch.equal(blob[:total], blob2[:total])
+
+
+def test_device_side_errors():
+    d = _setup("tiny-exact")
+    comp, w = d["comp"], d["w"]
+    blob = comp.compress(d["K"], d["V"], O.header_bytes(comp.n_units) + 16, 0)
+    with pytest.raises(J.JoltError) as e:
+        J.read_header(blob)
+    assert e.value.name == "BUDGET_INFEASIBLE"
+    K = d["K"].clone()
+    K[0, 0, 3, 5] = float("nan")
+    blob = comp.compress(K, d["V"], d["budget"], 0)
+    with pytest.raises(J.JoltError) as e:
+        J.read_header(blob)
+    assert e.value.name == "NUMERIC"
+    with pytest.raises(J.JoltError) as e:
+        comp.compress(d["K"], d["V"], d["budget"], 0, blob=torch.empty(100, dtype=torch.uint8, device="cuda"))
+    assert e.value.name == "OUTPUT_TOO_SMALL"
+    bad = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    with pytest.raises(J.JoltError) as e:
+        comp.decompress(bad)
+    assert e.value.name == "BAD_BLOB"
+
+
+def test_edge_candidate_sets():
+    """Residual-free (bits {0}) and full-rank feature factor (r_D = D) choices."""
+    w = synth.WORKLOADS["tiny"]
+    K, V = synth.make_cache(w, 1)
+    Kn, Vn = synth.to_f64(K), synth.to_f64(V)
+    for rt, rd, bits, ratio in (((8, 32), (8, 16), (0,), 1.5), ((32,), (16,), (0, 8), 0.6)):
+        jo, oo = J.Options(rt, rd, bits), O.Options(rt, rd, bits)
+        budget = int(w.bf16_bytes() / ratio)
+        res = O.compress(Kn, Vn, w.layers_per_group, oo, budget, 1)
+        comp = J.Compressor(w.n_layers, w.n_heads, w.T, w.D, w.layers_per_group, K.dtype, jo)
+        blob = comp.compress(K.cuda(), V.cuda(), budget, 1)
+        _, total, recs = J.read_header(blob)
+        assert [(r["r_T"], r["r_D"], r["bits"]) for r in recs] == [(u.r_T, u.r_D, u.b) for u in res.units]
+        Kh, Vh = comp.decompress(blob, torch.float32)
+        ek, ev = J.relative_errors(K.cuda(), V.cuda(), Kh, Vh, w.layers_per_group)
+        Ko, Vo = O.decompress(res)
+        assert abs(ek - O.relative_error(Kn, Ko)) <= 1e-4 and abs(ev - O.relative_error(Vn, Vo)) <= 1e-4
