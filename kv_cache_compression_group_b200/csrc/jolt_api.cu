@@ -142,7 +142,7 @@ struct Plan {
   size_t o_status, o_gd_part, o_gd, o_evals, o_Wf, o_Ws, o_Uf, o_Us, o_core, o_zc, o_ptmp, o_P, o_partial,
       o_table, o_bytes, o_choice, o_lambda, o_hdr, o_umap, o_info, o_solver;
   // token factor scratch (all units)
-  size_t o_gt32, o_gt, o_vsel, o_lam, o_omega, o_Y, o_Zm, o_h, o_l, o_gpart, o_G, o_ptrs;
+  size_t o_gt32, o_gt, o_vsel, o_lam, o_omega, o_Y, o_Zm, o_h, o_l, o_gpart, o_G, o_ptrs, o_shift;
   int qr_split_max;       // split-K of the Cholesky-QR Grams
   size_t ws_total;
   int tiles;
@@ -294,6 +294,7 @@ jolt_status make_plan(const jolt_shape* sh, const jolt_options* op, Plan* p) {
   p->o_hdr = b.take(64);
   p->o_umap = b.take((size_t)NU * S * 4 + 64);
   p->o_info = b.take((size_t)NU * 4 + 64);
+  p->o_shift = b.take((size_t)NU * 8 + 64);
   p->o_solver = b.take(p->solver_dev + 256);
   // token factor scratch
   p->o_gt32 = p->o_gt = p->o_vsel = p->o_lam = p->o_omega = 0;
@@ -322,8 +323,8 @@ jolt_status make_plan(const jolt_shape* sh, const jolt_options* op, Plan* p) {
   if (op->method == JOLT_RANDOMIZED || p->m_side) {
     p->o_gpart = b.take((size_t)NU * p->qr_split_max * kq * kq * 4);
     p->o_G = b.take((size_t)NU * kq * kq * 8);
-    p->o_ptrs = b.take((size_t)NU * 8 + 64);
   }
+  p->o_ptrs = b.take((size_t)NU * 8 + 64);
   p->ws_total = b.off;
 
   // largest possible blob
@@ -452,6 +453,18 @@ jolt_status sym_eig_batched(const Ctx& c, double* A, int64_t n, double* w, int64
   count_launch(), info_check_kernel<<<(unsigned)ceil_div(nbatch, 32), 32, 0, c.st>>>(c.at<int>(c.p.o_info),
                                                                                    (int)nbatch, c.status(),
                                                                                    DEV_ERR_FACTOR);
+  CUDA_TRY(cudaGetLastError());
+  return JOLT_OK;
+}
+
+// Leading r eigenvectors (descending, sign-fixed) of nbatch symmetric n x n matrices S (fp64,
+// lda = n, stride n*n; overwritten by the solver), through cuSOLVER's batched eigen solver.
+jolt_status sym_eig_top(const Ctx& c, double* S, int n, int nbatch, int r, float* out_f32, bf16* out_bf16,
+                        long long ldo, long long sout, double* out_vals) {
+  double* w = c.at<double>(c.p.o_evals);
+  JTRY(sym_eig_batched(c, S, n, w, nbatch));
+  count_launch(), eig_select_kernel<<<dim3(r, nbatch), 256, 0, c.st>>>(w, S, n, n, n, (long long)n * n, r, out_f32,
+                                                                       out_bf16, ldo, sout, out_vals);
   CUDA_TRY(cudaGetLastError());
   return JOLT_OK;
 }
@@ -604,12 +617,7 @@ jolt_status run_feature_factor(const Ctx& c, float* Wf, long long ldWf, bf16* Ws
       part, G, p.NU, p.gd_split, (long long)D * D);
   count_launch(), gram_diag_check_kernel<<<p.NU, 128, 0, c.st>>>(G, D, p.NU, c.status());
   CUDA_TRY(cudaGetLastError());
-  double* w = c.at<double>(p.o_evals);
-  JTRY(sym_eig_batched(c, G, D, w, p.NU));
-  count_launch(), eig_select_kernel<<<dim3(p.rDmax, p.NU), 128, 0, c.st>>>(
-      w, G, D, D, D, (long long)D * D, p.rDmax, Wf, Ws, ldWf, (long long)D * ldWf, nullptr);
-  CUDA_TRY(cudaGetLastError());
-  return JOLT_OK;
+  return sym_eig_top(c, G, D, p.NU, p.rDmax, Wf, Ws, ldWf, (long long)D * ldWf, nullptr);
 }
 
 // ------------------------------------------------------------------------------------------
@@ -646,19 +654,11 @@ jolt_status run_token_exact(const Ctx& c, float* Uf, long long ldUf) {
   }
   count_launch(), f32_to_f64_kernel<<<grid1d((long long)p.NU * n * n), 256, 0, c.st>>>(G32, G, (long long)p.NU * n * n);
   CUDA_TRY(cudaGetLastError());
-  double* w = c.at<double>(p.o_evals);
-  JTRY(sym_eig_batched(c, G, n, w, p.NU));
-  if (!p.m_side) {
-    count_launch(), eig_select_kernel<<<dim3(p.rTmax, p.NU), 256, 0, c.st>>>(
-        w, G, (int)n, n, n, n * n, p.rTmax, Uf, nullptr, ldUf, (long long)T * ldUf, nullptr);
-    CUDA_TRY(cudaGetLastError());
-    return JOLT_OK;
-  }
+  if (!p.m_side) return sym_eig_top(c, G, (int)n, p.NU, p.rTmax, Uf, nullptr, ldUf, (long long)T * ldUf, nullptr);
   // T > M: U = X_(T) V Lambda^{-1/2}, then CholeskyQR2 re-orthonormalisation
   float* V = c.at<float>(p.o_vsel);
   double* lam = c.at<double>(p.o_lam);
-  count_launch(), eig_select_kernel<<<dim3(p.rTmax, p.NU), 256, 0, c.st>>>(
-      w, G, (int)n, n, n, n * n, p.rTmax, V, nullptr, p.ldU, (long long)M * p.ldU, lam);
+  JTRY(sym_eig_top(c, G, (int)n, p.NU, p.rTmax, V, nullptr, p.ldU, (long long)M * p.ldU, lam));
   count_launch(), scale_cols_kernel<<<grid1d((long long)p.NU * M * p.rTmax), 256, 0, c.st>>>(
       V, lam, M, p.rTmax, p.ldU, (long long)M * p.ldU, p.rTmax, p.NU, c.status());
   CUDA_TRY(cudaGetLastError());
@@ -758,12 +758,8 @@ jolt_status run_token_randomized(const Ctx& c, float* Uf, long long ldUf) {
         gpart, S, NU, ns, (long long)k * k);
     CUDA_TRY(cudaGetLastError());
   }
-  double* w = c.at<double>(p.o_evals);
-  JTRY(sym_eig_batched(c, S, k, w, NU));
   float* V = c.at<float>(p.o_vsel);
-  count_launch(), eig_select_kernel<<<dim3(p.rTmax, NU), 256, 0, c.st>>>(
-      w, S, k, k, k, (long long)k * k, p.rTmax, V, nullptr, p.ldU, (long long)kp * p.ldU, nullptr);
-  CUDA_TRY(cudaGetLastError());
+  JTRY(sym_eig_top(c, S, k, NU, p.rTmax, V, nullptr, p.ldU, (long long)kp * p.ldU, nullptr));
   // U = Q V
   ProfScope ps2("ritz_vectors", c.st, NU);
   GemmParams uq;
