@@ -41,7 +41,27 @@ def parse():
     ap.add_argument("--workload", default="mistral7b")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extras", action="store_true", help="skip the exact-arm and decompress side figures")
+    ap.add_argument("--profile-case", default=None, choices=["mistral7b_4layers"],
+                    help="run one compress of a small case (for ncu captures) and exit")
     return ap.parse_args()
+
+
+def profile_case(args):
+    """One FlashJoLT (or JoLT) compress + decompress of a 4-layer Mistral-shaped cache (16 MiB of
+    K and V): a case small enough for an ncu capture, with the same kernels as the full run."""
+    import torch
+    from kv_cache_compression_group_b200 import synth, jolt as J
+    w = synth.small_workload("mistral7b", n_layers=4)
+    K, V = synth.make_cache(w, 0)
+    Kd, Vd = K.cuda(), V.cuda()
+    opts = J.default_options(w.T, w.D, args.method)
+    comp = J.Compressor(w.n_layers, w.n_heads, w.T, w.D, w.layers_per_group, K.dtype, opts)
+    for _ in range(2):
+        blob = comp.compress(Kd, Vd, w.bf16_bytes() // 2, 0)
+        Kh, Vh = comp.decompress(blob)
+    torch.cuda.synchronize()
+    print(json.dumps({"profile_case": args.profile_case, "method": args.method,
+                      "total_bytes": J.read_header(blob)[1]}))
 
 
 def workload_config(w, method, opts):
@@ -208,6 +228,8 @@ def main():
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         return run_reference(args, rank, world)
+    if args.profile_case:
+        return profile_case(args)
 
     import torch
     import torch.distributed as dist
