@@ -216,6 +216,21 @@ jolt_status jolt_frobenius(const jolt_shape* shape, const void* k_dev, const voi
                            const void* vy_dev, int32_t ydtype, double* sq_dev, void* ws_dev, size_t ws_bytes,
                            void* stream);
 
+/* jolt_frobenius without a workspace argument (the paper has no counterpart: this is a
+ * convenience of the library).  For callers that cannot allocate device memory themselves,
+ * e.g. a host program whose device memory is entirely owned by another allocator: the
+ * partial sums go to a 64 KiB array compiled into the library, which every device that loads
+ * the library holds until the process exits.  Same arguments and results as jolt_frobenius.
+ *   - at most 64 units (2 * n_layers / layers_per_group <= 64); more returns
+ *     JOLT_ERR_WORKSPACE_TOO_SMALL with a message naming the limit;
+ *   - the first call on each device looks up the array's device address with that device
+ *     current (a one-time set-up); make that first call before any stream capture;
+ *   - all calls share the one array: two calls whose GPU work overlaps (different streams or
+ *     threads without ordering between them) race on it and may return wrong sums;
+ *   - allocates nothing.  Asynchronous. */
+jolt_status jolt_frobenius_noalloc(const jolt_shape* shape, const void* k_dev, const void* v_dev, const void* ky_dev,
+                                   const void* vy_dev, int32_t ydtype, double* sq_dev, void* stream);
+
 /* Stage timing for measurement (no counterpart on the pages).  jolt_profile_begin starts
  * recording CUDA events around every internal stage launched by this thread (on the call's
  * stream); jolt_profile_end stops, SYNCHRONISES on the recorded events and writes one line

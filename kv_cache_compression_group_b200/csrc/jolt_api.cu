@@ -2,6 +2,7 @@
 #include <cusolverDn.h>
 
 #include <cstdarg>
+#include <mutex>
 #include <cstdio>
 #include <cstring>
 #include <string>
@@ -1486,4 +1487,83 @@ jolt_status jolt_frobenius(const jolt_shape* shape, const void* k_dev, const voi
   return JOLT_OK;
 }
 
+// ------------------------------------------------------------------------------------------
+// Allocation-free variant of jolt_frobenius.  Its per-block partial sums live in a file-scope
+// device array instead of a caller-provided workspace, for callers that cannot allocate
+// device memory themselves: for instance a host program whose device memory is entirely
+// owned by another allocator, or one that must not call the CUDA allocator at all on its
+// path.  The array is part of this library's image: every device that loads the library
+// holds it until the process exits.
+// ------------------------------------------------------------------------------------------
 }  // extern "C"
+
+namespace {
+constexpr int kNoAllocBlocks = 64;                       // partial-sum blocks per unit
+constexpr int kNoAllocMaxUnits = 64;                     // 2 * n_layers / layers_per_group
+constexpr int kNoAllocSlots = kNoAllocMaxUnits * kNoAllocBlocks * 2;
+static __device__ __align__(256) double g_frob_scratch[kNoAllocSlots];  // 64 KiB
+
+// device address of g_frob_scratch, looked up once per device with that device current
+struct NoAllocScratch {
+  std::mutex mu;
+  double* ptr[64] = {};
+};
+NoAllocScratch& noalloc_scratch() {
+  static NoAllocScratch s;
+  return s;
+}
+}  // namespace
+
+extern "C" jolt_status jolt_frobenius_noalloc(const jolt_shape* shape, const void* k_dev, const void* v_dev,
+                                              const void* ky_dev, const void* vy_dev, int32_t ydtype,
+                                              double* sq_dev, void* stream) {
+  if (!shape || !k_dev || !v_dev || !sq_dev) return fail(JOLT_ERR_INVALID_ARG, "null pointer");
+  if ((ky_dev == nullptr) != (vy_dev == nullptr)) return fail(JOLT_ERR_INVALID_ARG, "give both or neither of ky, vy");
+  if (shape->n_layers < 1 || shape->layers_per_group < 1 || shape->n_layers % shape->layers_per_group)
+    return fail(JOLT_ERR_INVALID_ARG, "shape");
+  const int G = shape->n_layers / shape->layers_per_group, NU = 2 * G;
+  if (NU > kNoAllocMaxUnits)
+    return fail(JOLT_ERR_WORKSPACE_TOO_SMALL, "jolt_frobenius_noalloc handles at most %d units (got %d); use jolt_frobenius",
+                kNoAllocMaxUnits, NU);
+  int dev = 0;
+  CUDA_TRY(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return fail(JOLT_ERR_INVALID_ARG, "device ordinal %d out of range", dev);
+  double* part = nullptr;
+  {
+    NoAllocScratch& sc = noalloc_scratch();
+    std::lock_guard<std::mutex> lk(sc.mu);
+    if (!sc.ptr[dev]) {
+      void* p = nullptr;
+      CUDA_TRY(cudaGetSymbolAddress(&p, g_frob_scratch));
+      sc.ptr[dev] = static_cast<double*>(p);
+    }
+    part = sc.ptr[dev];
+  }
+  const long long n = (long long)shape->layers_per_group * shape->n_heads * shape->n_tokens * shape->head_dim;
+  cudaStream_t st = (cudaStream_t)stream;
+  // every partial slot read below is written first by the same call: nothing to clear
+  for (int kv = 0; kv < 2; ++kv) {
+    const void* X = kv ? v_dev : k_dev;
+    const void* Y = kv ? vy_dev : ky_dev;
+    dim3 grid(kNoAllocBlocks, G);
+    if (shape->dtype == JOLT_BF16) {
+      if (ydtype == JOLT_F32)
+        count_launch(), frob_partial_kernel<bf16, float><<<grid, 256, 0, st>>>((const bf16*)X, (const float*)Y, n, kv,
+                                                                               part, kNoAllocBlocks);
+      else
+        count_launch(), frob_partial_kernel<bf16, bf16><<<grid, 256, 0, st>>>((const bf16*)X, (const bf16*)Y, n, kv,
+                                                                              part, kNoAllocBlocks);
+    } else {
+      if (ydtype == JOLT_F32)
+        count_launch(), frob_partial_kernel<float, float><<<grid, 256, 0, st>>>((const float*)X, (const float*)Y, n,
+                                                                                kv, part, kNoAllocBlocks);
+      else
+        count_launch(), frob_partial_kernel<float, bf16><<<grid, 256, 0, st>>>((const float*)X, (const bf16*)Y, n, kv,
+                                                                               part, kNoAllocBlocks);
+    }
+    CUDA_TRY(cudaGetLastError());
+  }
+  count_launch(), frob_final_kernel<<<(unsigned)ceil_div(2 * NU, 128), 128, 0, st>>>(part, NU, kNoAllocBlocks, sq_dev);
+  CUDA_TRY(cudaGetLastError());
+  return JOLT_OK;
+}

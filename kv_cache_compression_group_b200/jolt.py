@@ -28,7 +28,7 @@ EXPORTED = [
     "jolt_version", "jolt_last_error", "jolt_workspace_size", "jolt_counts", "jolt_choice_bytes",
     "jolt_compress", "jolt_factor", "jolt_table", "jolt_allocate", "jolt_encode", "jolt_read_header",
     "jolt_decompress", "jolt_frobenius", "jolt_profile_begin", "jolt_profile_end", "jolt_recon_operator",
-    "jolt_launch_count",
+    "jolt_launch_count", "jolt_frobenius_noalloc",
 ]
 
 
@@ -85,6 +85,7 @@ def lib():
             "jolt_read_header": [vp, pS, ctypes.POINTER(u64), ctypes.POINTER(CUnitRecord), i32, vp],
             "jolt_decompress": [vp, i32, vp, vp, vp, sz, vp],
             "jolt_frobenius": [pS, vp, vp, vp, vp, i32, vp, vp, sz, vp],
+            "jolt_frobenius_noalloc": [pS, vp, vp, vp, vp, i32, vp, vp],
             "jolt_recon_operator": [pS, pO, u64, vp, vp, ctypes.c_int64, vp, vp, sz, vp],
             "jolt_profile_begin": [],
             "jolt_profile_end": [ctypes.c_char_p, sz],
@@ -357,6 +358,18 @@ def profile_end():
         name, ms, n, u = line.split()
         out[name] = (float(ms), int(n), int(u))
     return out
+
+
+def frobenius_noalloc(K, V, K_hat=None, V_hat=None, layers_per_group=1, stream=None):
+    """As frobenius(), through the entry point that needs no workspace (its scratch is a
+    fixed array inside the library; calls whose GPU work overlaps must not be mixed)."""
+    shape = make_shape(K, layers_per_group)
+    G = K.shape[0] // layers_per_group
+    sq = torch.zeros(2 * 2 * G, dtype=torch.float64, device=K.device)
+    yd = JOLT_F32 if (K_hat is not None and K_hat.dtype == torch.float32) else JOLT_BF16
+    _check(lib().jolt_frobenius_noalloc(ctypes.byref(shape), _ptr(K), _ptr(V), _ptr(K_hat), _ptr(V_hat), yd,
+                                        _ptr(sq), _stream(stream)))
+    return sq.view(2 * G, 2)
 
 
 def relative_errors(K, V, K_hat, V_hat, layers_per_group):
