@@ -29,6 +29,10 @@ RATIOS = (2.0, 3.0)
 L2_BYTES = 126 * 1024 * 1024
 # FP32 pipe: 148 SMs x 128 lanes, one FMA-class instruction per lane per clock
 SMS, FP32_LANES = 148, 128
+# DRAM bytes (read + write) of one table_kernel launch over the 16 units of the bench workload:
+# an ncu capture of 2 units (profiles/table_kernel_mistral7b_4layers.md) scaled by 8.  None
+# whenever the kernel has changed since that capture.
+TABLE_KERNEL_TRAFFIC_BYTES = 277.6e6
 
 
 def parse():
@@ -344,7 +348,7 @@ def main():
         peak = SMS * FP32_LANES * mhz * 1e6 / 1e12
         achieved = ops / (ms / n / 1e3) / 1e12
         roofline = {"kernel": "table_kernel", "bound": "alu", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                    "frac": achieved / peak, "traffic": None,
+                    "frac": achieved / peak, "traffic": TABLE_KERNEL_TRAFFIC_BYTES,
                     "note": f"peak = {SMS} SMs x {FP32_LANES} FP32 lanes x {mhz:.0f} MHz ({peak_src} max clock); "
                             f"algorithmic work = {per} FP32-pipe ops per element per (r_T, r_D) candidate",
                     "dominant_stage": dom}
