@@ -361,6 +361,140 @@ __global__ void __launch_bounds__(256) gemm_simt_kernel(GemmParams p) {
   }
 }
 
+// ------------------------------------------------------------------------------------------
+// fp32 x fp32 GEMM on the CUDA cores, register tiled: 128 x 128 CTA tile, 256 threads, 8 x 8
+// outputs per thread (two 4 x 4 sub-blocks 64 apart), k-steps of 8 double-buffered in shared
+// memory, 16-byte loads where an operand run is aligned and in range.
+// ------------------------------------------------------------------------------------------
+namespace sgemm_detail {
+constexpr int BM = 128, BN = 128, BK = 8, THREADS = 256;
+
+// load the BK x 128 slice (k0.., x0..) of an operand into s[BK][128] (x fastest)
+__device__ __forceinline__ void load_slice(float (*s)[BM], const GemmOperand& o, const float* base, int x0, int k0,
+                                           int Xext, int kend, int tid) {
+  if (!o.kmajor) {
+    // contiguous along x: thread -> (k row tid/32, four x from (tid%32)*4)
+    const int kr = tid >> 5, xc = (tid & 31) * 4;
+    const int k = k0 + kr, x = x0 + xc;
+    float v[4] = {0.f, 0.f, 0.f, 0.f};
+    if (k < kend) {
+      const float* src = base + opnd_offset(o, x, k);
+      const bool vec = (x + 3 < Xext) && (o.xshift >= 31 || ((x & ((1 << o.xshift) - 1)) + 3) < (1 << o.xshift)) &&
+                       ((reinterpret_cast<uintptr_t>(src) & 15) == 0);
+      if (vec) {
+        float4 t = *reinterpret_cast<const float4*>(src);
+        v[0] = t.x; v[1] = t.y; v[2] = t.z; v[3] = t.w;
+      } else {
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          if (x + e < Xext) v[e] = base[opnd_offset(o, x + e, k)];
+      }
+    }
+    *reinterpret_cast<float4*>(&s[kr][xc]) = make_float4(v[0], v[1], v[2], v[3]);
+  } else {
+    // contiguous along k: thread -> (x row tid/2, four k from (tid%2)*4), stored transposed
+    const int xr = tid >> 1, kc = (tid & 1) * 4;
+    const int x = x0 + xr, k = k0 + kc;
+    float v[4] = {0.f, 0.f, 0.f, 0.f};
+    if (x < Xext && k < kend) {
+      const float* src = base + opnd_offset(o, x, k);
+      const bool vec = (k + 3 < kend) && ((reinterpret_cast<uintptr_t>(src) & 15) == 0) &&
+                       (o.kshift >= 31 || ((k & ((1 << o.kshift) - 1)) + 3) < (1 << o.kshift));
+      if (vec) {
+        float4 t = *reinterpret_cast<const float4*>(src);
+        v[0] = t.x; v[1] = t.y; v[2] = t.z; v[3] = t.w;
+      } else {
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          if (k + e < kend) v[e] = base[opnd_offset(o, x, k + e)];
+      }
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) s[kc + e][xr] = v[e];
+  }
+}
+}  // namespace sgemm_detail
+
+__global__ void __launch_bounds__(256, 2) sgemm_kernel(GemmParams p) {
+  using namespace sgemm_detail;
+  __shared__ __align__(16) float As[2][BK][BM];
+  __shared__ __align__(16) float Bs[2][BK][BN];
+  const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
+  const int m0 = blockIdx.y * BM, n0 = blockIdx.x * BN;
+  const int bz = blockIdx.z;
+  const int b = bz / p.splits, split = bz - b * p.splits;
+  const int kbeg = split * p.kchunk;
+  const int kend = min(p.K, kbeg + p.kchunk);
+  const float* A = reinterpret_cast<const float*>(opnd_base_t(p.A, b, 4));
+  const float* B = reinterpret_cast<const float*>(opnd_base_t(p.B, b, 4));
+  float acc[8][8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
+  const int ntiles = kend > kbeg ? (kend - kbeg + BK - 1) / BK : 0;
+  if (ntiles > 0) {
+    load_slice(As[0], p.A, A, m0, kbeg, p.M, kend, tid);
+    load_slice(Bs[0], p.B, B, n0, kbeg, p.N, kend, tid);
+  }
+  __syncthreads();
+  for (int t = 0; t < ntiles; ++t) {
+    const int cur = t & 1;
+    if (t + 1 < ntiles) {
+      load_slice(As[cur ^ 1], p.A, A, m0, kbeg + (t + 1) * BK, p.M, kend, tid);
+      load_slice(Bs[cur ^ 1], p.B, B, n0, kbeg + (t + 1) * BK, p.N, kend, tid);
+    }
+#pragma unroll
+    for (int kk = 0; kk < BK; ++kk) {
+      float a[8], bb[8];
+      const float4 a0 = *reinterpret_cast<const float4*>(&As[cur][kk][ty * 4]);
+      const float4 a1 = *reinterpret_cast<const float4*>(&As[cur][kk][64 + ty * 4]);
+      const float4 b0 = *reinterpret_cast<const float4*>(&Bs[cur][kk][tx * 4]);
+      const float4 b1 = *reinterpret_cast<const float4*>(&Bs[cur][kk][64 + tx * 4]);
+      a[0] = a0.x; a[1] = a0.y; a[2] = a0.z; a[3] = a0.w; a[4] = a1.x; a[5] = a1.y; a[6] = a1.z; a[7] = a1.w;
+      bb[0] = b0.x; bb[1] = b0.y; bb[2] = b0.z; bb[3] = b0.w; bb[4] = b1.x; bb[5] = b1.y; bb[6] = b1.z; bb[7] = b1.w;
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(a[i], bb[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+  const long long cbase = (long long)b * p.sbatchC + (long long)split * p.ssplitC;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int m = m0 + (i < 4 ? ty * 4 + i : 64 + ty * 4 + i - 4);
+    if (m >= p.M) continue;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int n = n0 + (j < 4 ? tx * 4 + j : 64 + tx * 4 + j - 4);
+      if (n >= p.N) continue;
+      const long long off = cbase + (long long)m * p.ldc + n;
+      const float v = p.alpha * acc[i][j];
+      if (p.c_type == 2) {
+        double* C = reinterpret_cast<double*>(p.C) + off;
+        *C = (p.beta != 0.f) ? (double)v + (double)p.beta * *C : (double)v;
+      } else if (p.c_type == 0) {
+        float* C = reinterpret_cast<float*>(p.C) + off;
+        *C = (p.beta != 0.f) ? v + p.beta * *C : v;
+      } else {
+        bf16* C = reinterpret_cast<bf16*>(p.C) + off;
+        *C = __float2bfloat16_rn(p.beta != 0.f ? v + p.beta * __bfloat162float(*C) : v);
+      }
+    }
+  }
+}
+
+inline cudaError_t launch_sgemm(const GemmParams& p, cudaStream_t st) {
+  GemmParams q = p;
+  if (q.kchunk <= 0) q.kchunk = q.K;
+  dim3 grid((unsigned)ceil_div(q.N, sgemm_detail::BN), (unsigned)ceil_div(q.M, sgemm_detail::BM),
+            (unsigned)(q.batch * q.splits));
+  count_launch();
+  sgemm_kernel<<<grid, sgemm_detail::THREADS, 0, st>>>(q);
+  return cudaGetLastError();
+}
+
 template <typename TA, typename TB, typename Acc>
 inline cudaError_t launch_gemm_simt(const GemmParams& p, cudaStream_t st) {
   GemmParams q = p;

@@ -143,7 +143,8 @@ struct Plan {
   size_t o_status, o_gd_part, o_gd, o_evals, o_Wf, o_Ws, o_Uf, o_Us, o_core, o_zc, o_ptmp, o_P, o_partial,
       o_table, o_bytes, o_choice, o_lambda, o_hdr, o_umap, o_info, o_solver;
   // token factor scratch (all units)
-  size_t o_gt32, o_gt, o_vsel, o_lam, o_omega, o_Y, o_Zm, o_h, o_l, o_gpart, o_G, o_ptrs, o_shift;
+  size_t o_gt32, o_gt, o_vsel, o_lam, o_omega, o_Y, o_Zm, o_h, o_l, o_gpart, o_G, o_ptrs, o_shift, o_Lr, o_Linv,
+      o_qtmp;
   int qr_split_max;       // split-K of the Cholesky-QR Grams
   size_t ws_total;
   int tiles;
@@ -321,9 +322,14 @@ jolt_status make_plan(const jolt_shape* sh, const jolt_options* op, Plan* p) {
     p->o_l = b.take((size_t)NU * big * kp * 2);
     p->o_vsel = b.take((size_t)NU * kp * p->ldU * 4);
   }
+  p->o_Lr = p->o_Linv = p->o_qtmp = 0;
   if (op->method == JOLT_RANDOMIZED || p->m_side) {
+    long long mrows = op->method == JOLT_RANDOMIZED ? (M > T ? M : T) : T;
     p->o_gpart = b.take((size_t)NU * p->qr_split_max * kq * kq * 4);
     p->o_G = b.take((size_t)NU * kq * kq * 8);
+    p->o_Lr = b.take((size_t)NU * kq * kq * 4);
+    p->o_Linv = b.take((size_t)NU * kq * kq * 4);
+    p->o_qtmp = b.take((size_t)NU * mrows * kq * 4);
   }
   p->o_ptrs = b.take((size_t)NU * 8 + 64);
   p->ws_total = b.off;
@@ -357,6 +363,7 @@ jolt_status gemm(const GemmParams& p, int ta, int tb, cudaStream_t st) {
   cudaError_t e;
   const bool dacc = p.c_type == 2;
   if (ta == 0 && tb == 0) e = launch_gemm_bf16(p, st);
+  else if (ta == 1 && tb == 1 && p.c_type != 2) e = launch_sgemm(p, st);
 #define GEMM_CASE(A, B, TA, TB)                                                              \
   else if (ta == A && tb == B) e = dacc ? launch_gemm_simt<TA, TB, double>(p, st)           \
                                         : launch_gemm_simt<TA, TB, float>(p, st);
@@ -444,9 +451,7 @@ jolt_status sym_eig_batched(const Ctx& c, double* A, int64_t n, double* w, int64
                                                CUDA_R_64F, A, n, CUDA_R_64F, w, CUDA_R_64F, &dv, &hv, nbatch));
   void* host = nullptr;
   JTRY(solver_ws(c, s, dv, hv, &host));
-  for (int64_t b = 0; b < nbatch; ++b) {
-    count_launch(), sanitize_sym_kernel<<<1, 1024, 0, c.st>>>(A + b * n * n, (int)n, n, c.status());
-  }
+  count_launch(), sanitize_sym_batched_kernel<<<(unsigned)nbatch, 1024, 0, c.st>>>(A, (int)n, n, n * n, c.status());
   CUDA_TRY(cudaGetLastError());
   SOLVER_TRY(cusolverDnXsyevBatched(s->h, s->params, CUSOLVER_EIG_MODE_VECTOR, CUBLAS_FILL_MODE_LOWER, n, CUDA_R_64F,
                                     A, n, CUDA_R_64F, w, CUDA_R_64F, c.at<void>(c.p.o_solver), dv, host, hv,
@@ -514,17 +519,40 @@ jolt_status cholqr_batched(const Ctx& c, float* Y, long long m, int k, int ld, i
     count_launch(), info_check_kernel<<<(unsigned)ceil_div(p.NU, 32), 32, 0, c.st>>>(info, p.NU, c.status(),
                                                                                       DEV_ERR_FACTOR);
     ProfScope ps3("qr_trsm", c.st, p.NU);
-    if (k <= 512) {
-      size_t sm = trsm_smem(64, k);
-      CUDA_TRY(cudaFuncSetAttribute(trsm_rows_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm));
-      count_launch(), trsm_rows_kernel<64><<<dim3((unsigned)ceil_div(m, 64), p.NU), 64, sm, c.st>>>(
-          Y, ld, m * ld, m, k, G, gld, n);
-    } else {
-      size_t sm = trsm_smem(32, k);
-      CUDA_TRY(cudaFuncSetAttribute(trsm_rows_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm));
-      count_launch(), trsm_rows_kernel<32><<<dim3((unsigned)ceil_div(m, 32), p.NU), 32, sm, c.st>>>(
-          Y, ld, m * ld, m, k, G, gld, n);
+    // Q = Y L^{-T}: L^{-1} by column-parallel forward substitution, then a GEMM
+    float* Lr = c.at<float>(p.o_Lr);
+    float* Li = c.at<float>(p.o_Linv);
+    float* Qt = c.at<float>(p.o_qtmp);
+    count_launch(), lower_to_rowmajor_kernel<<<grid1d((long long)p.NU * k * k), 256, 0, c.st>>>(
+        G, k, gld, n, Lr, gld, (long long)k * gld, p.NU);
+    {
+      const int nth = 32 * (int)(ceil_div(ceil_div(k, TRI_NB), 1) < 32 ? ceil_div(k, TRI_NB) : 32);
+      const size_t sm = trinv_smem(nth);
+      CUDA_TRY(cudaFuncSetAttribute(trinv_blocked_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm));
+      count_launch(), trinv_blocked_kernel<<<p.NU, nth, sm, c.st>>>(Lr, k, gld, (long long)k * gld, Li, c.status());
     }
+    CUDA_TRY(cudaGetLastError());
+    GemmParams q;
+    q.M = (int)m;
+    q.N = k;
+    q.K = k;
+    q.batch = p.NU;
+    q.A.ptr = Y;
+    q.A.kmajor = true;
+    q.A.ld = ld;
+    q.A.sbatch = m * ld;
+    q.B.ptr = Li;       // B(i, j) = L^{-1}[j][i]: row j of L^{-1} is contiguous in i
+    q.B.kmajor = true;
+    q.B.ld = gld;
+    q.B.sbatch = (long long)k * gld;
+    q.C = Qt;
+    q.ldc = ld;
+    q.sbatchC = m * ld;
+    q.c_type = 0;
+    JTRY(gemm(q, 1, 1, c.st));
+    // copy the k columns back (the padding columns of Y stay as they are)
+    CUDA_TRY(cudaMemcpy2DAsync(Y, (size_t)ld * 4, Qt, (size_t)ld * 4, (size_t)k * 4, (size_t)(p.NU * m),
+                               cudaMemcpyDeviceToDevice, c.st));
     CUDA_TRY(cudaGetLastError());
   }
   return JOLT_OK;

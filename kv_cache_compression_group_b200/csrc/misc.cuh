@@ -226,70 +226,99 @@ __global__ void ptr_array_kernel(double** P, double* A, long long sA, int n) {
   if (u < n) P[u] = A + (long long)u * sA;
 }
 
-// Q = Y L^{-T} in place (Q L^T = Y), row by row, for every unit: Y [rows x k] fp32 (ld,
-// stride sY per unit), L lower triangular k x k, column-major fp64 (lda, stride sL).  A CTA
-// owns RT rows (one thread each); columns go in blocks of 32: the block's right-hand side is
-// updated with the already solved columns (L rows staged through shared memory in chunks),
-// then the 32 x 32 diagonal triangle is solved in registers.
-constexpr int TRSM_NB = 32;
-constexpr int TRSM_PC = 256;
-template <int RT>
-__global__ void __launch_bounds__(RT) trsm_rows_kernel(float* Y, long long ld, long long sY, long long rows, int k,
-                                                       const double* L, long long lda, long long sL) {
-  extern __shared__ __align__(16) float tsm[];
-  const int ldq = k + 1;
-  float* Qs = tsm;                          // RT x ldq: solved columns of this CTA's rows
-  float* Lp = Qs + RT * ldq;                // TRSM_NB x (TRSM_PC + 1): chunk of L rows
-  float* Ld = Lp + TRSM_NB * (TRSM_PC + 1); // TRSM_NB x (TRSM_NB + 1): diagonal block
-  const int u = blockIdx.y;
-  const long long row = (long long)blockIdx.x * RT + threadIdx.x;
-  const bool valid = row < rows;
-  float* y = Y + (long long)u * sY + row * ld;
-  const double* Lu = L + (long long)u * sL;
-  for (int J = 0; J < k; J += TRSM_NB) {
-    const int nb = min(TRSM_NB, k - J);
-    float acc[TRSM_NB];
-#pragma unroll
-    for (int c = 0; c < TRSM_NB; ++c) acc[c] = (valid && c < nb) ? y[J + c] : 0.f;
-    for (int pc = 0; pc < J; pc += TRSM_PC) {
-      const int np = min(TRSM_PC, J - pc);
-      __syncthreads();
-      for (int idx = threadIdx.x; idx < TRSM_NB * np; idx += RT) {
-        int c = idx / np, q = idx - c * np;
-        Lp[c * (TRSM_PC + 1) + q] = c < nb ? (float)Lu[(long long)(pc + q) * lda + (J + c)] : 0.f;
-      }
-      __syncthreads();
-      for (int q = 0; q < np; ++q) {
-        const float qv = Qs[threadIdx.x * ldq + pc + q];
-#pragma unroll
-        for (int c = 0; c < TRSM_NB; ++c) acc[c] = fmaf(-qv, Lp[c * (TRSM_PC + 1) + q], acc[c]);
-      }
-    }
-    __syncthreads();
-    for (int idx = threadIdx.x; idx < TRSM_NB * TRSM_NB; idx += RT) {
-      int c = idx / TRSM_NB, q = idx - c * TRSM_NB;
-      Ld[c * (TRSM_NB + 1) + q] = (c < nb && q < nb) ? (float)Lu[(long long)(J + q) * lda + (J + c)] : 0.f;
-    }
-    __syncthreads();
-    float x[TRSM_NB];
-#pragma unroll
-    for (int c = 0; c < TRSM_NB; ++c) {
-      float v = acc[c];
-#pragma unroll
-      for (int q = 0; q < c; ++q) v = fmaf(-x[q], Ld[c * (TRSM_NB + 1) + q], v);
-      const float dgl = Ld[c * (TRSM_NB + 1) + c];
-      x[c] = (c < nb && dgl != 0.f) ? v / dgl : 0.f;
-    }
-#pragma unroll
-    for (int c = 0; c < TRSM_NB; ++c)
-      if (c < nb) Qs[threadIdx.x * ldq + J + c] = x[c];
+// lower-triangular L (column-major fp64, lda, stride sL) -> row-major fp32 [k][ld] (stride so),
+// zero above the diagonal
+__global__ void lower_to_rowmajor_kernel(const double* L, int k, long long lda, long long sL, float* out, long long ld,
+                                         long long so, int nbatch) {
+  const long long tot = (long long)nbatch * k * k;
+  for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < tot;
+       idx += (long long)gridDim.x * blockDim.x) {
+    const long long u = idx / ((long long)k * k), rem = idx - u * k * k;
+    const long long i = rem / k, j = rem - i * k;
+    out[u * so + i * ld + j] = j <= i ? (float)L[u * sL + j * lda + i] : 0.f;
   }
-  if (!valid) return;
-  for (int c = 0; c < k; ++c) y[c] = Qs[threadIdx.x * ldq + c];
 }
 
-inline size_t trsm_smem(int RT, int k) {
-  return ((size_t)RT * (k + 1) + (size_t)TRSM_NB * (TRSM_PC + 1) + (size_t)TRSM_NB * (TRSM_NB + 1)) * 4;
+// X = L^{-1} for every unit (L: row-major fp32 lower [k][ld], X: row-major fp32 [k][ld], both
+// with unit stride sL), blocked by 32: block row I is X_II = inv(L_II) (one warp, forward
+// substitution per column) and, for every block column J < I (one warp each),
+// X_IJ = -X_II (sum_{J<=P<I} L_IP X_PJ).  Block rows go in order; one CTA per unit.
+constexpr int TRI_NB = 32;
+__global__ void __launch_bounds__(1024) trinv_blocked_kernel(const float* L, int k, long long ld, long long sL,
+                                                             float* X, uint32_t* status) {
+  extern __shared__ __align__(16) float tri_sm[];
+  float* Xd = tri_sm;                              // X_II, 32 x 33
+  float* acc_s = tri_sm + TRI_NB * (TRI_NB + 1);   // per warp 32 x 33
+  const int u = blockIdx.x;
+  const float* Lu = L + (long long)u * sL;
+  float* Xu = X + (long long)u * sL;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+  const int nb = (k + TRI_NB - 1) / TRI_NB;
+  // zero the strict upper part once
+  for (long long idx = threadIdx.x; idx < (long long)k * k; idx += blockDim.x) {
+    const long long r = idx / k, cc = idx - r * k;
+    if (cc > r) Xu[r * ld + cc] = 0.f;
+  }
+  for (int I = 0; I < nb; ++I) {
+    const int i0 = I * TRI_NB, ni = min(TRI_NB, k - i0);
+    // 1. X_II by warp 0: lane j owns column j of the diagonal block
+    if (warp == 0) {
+      float x[TRI_NB];
+#pragma unroll
+      for (int r = 0; r < TRI_NB; ++r) {
+        float v = (r == lane) ? 1.f : 0.f;
+        if (r < ni) {
+          const float* Lr = Lu + (long long)(i0 + r) * ld + i0;
+#pragma unroll
+          for (int q = 0; q < r; ++q) v = fmaf(-Lr[q], x[q], v);
+          const float d = Lr[r];
+          if (!(d != 0.f)) raise_status(status, DEV_ERR_FACTOR);
+          x[r] = (lane <= r && lane < ni) ? v / d : 0.f;
+        } else {
+          x[r] = 0.f;
+        }
+      }
+#pragma unroll
+      for (int r = 0; r < TRI_NB; ++r) Xd[r * (TRI_NB + 1) + lane] = x[r];
+    }
+    __syncthreads();
+    if (warp == 0 && lane < ni)
+      for (int r = 0; r < ni; ++r) Xu[(long long)(i0 + r) * ld + i0 + lane] = Xd[r * (TRI_NB + 1) + lane];
+    // 2. off-diagonal blocks of block row I: warp w handles block columns J = w, w + nwarps, ...
+    for (int J = warp; J < I; J += nwarps) {
+      const int j0 = J * TRI_NB;
+      // acc[r][c] (lane = row r): sum_{P=J}^{I-1} L_IP X_PJ
+      float acc[TRI_NB];
+#pragma unroll
+      for (int c = 0; c < TRI_NB; ++c) acc[c] = 0.f;
+      if (lane < ni) {
+        const float* Lr = Lu + (long long)(i0 + lane) * ld;
+        for (int p = j0; p < i0; ++p) {
+          const float l = Lr[p];
+          const float* Xp = Xu + (long long)p * ld + j0;
+#pragma unroll
+          for (int c = 0; c < TRI_NB; ++c) acc[c] = fmaf(l, Xp[c], acc[c]);
+        }
+      }
+      float* as = acc_s + warp * TRI_NB * (TRI_NB + 1);
+#pragma unroll
+      for (int c = 0; c < TRI_NB; ++c) as[lane * (TRI_NB + 1) + c] = acc[c];
+      __syncwarp();
+      // X_IJ[r][c] = -sum_q X_II[r][q] acc[q][c]   (lane = column c)
+      const int nj = min(TRI_NB, k - j0);
+      for (int r = 0; r < ni; ++r) {
+        float v = 0.f;
+        for (int q = 0; q <= r; ++q) v = fmaf(Xd[r * (TRI_NB + 1) + q], as[q * (TRI_NB + 1) + lane], v);
+        if (lane < nj) Xu[(long long)(i0 + r) * ld + j0 + lane] = -v;
+      }
+      __syncwarp();
+    }
+    __syncthreads();
+  }
+}
+
+inline size_t trinv_smem(int nthreads) {
+  return (size_t)(TRI_NB * (TRI_NB + 1)) * 4 * (1 + nthreads / 32);
 }
 
 __global__ void info_check_kernel(const int* info, int n, uint32_t* status, uint32_t bits) {
