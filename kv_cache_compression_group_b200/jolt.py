@@ -148,12 +148,16 @@ class Options:
 
 
 def default_options(T: int, D: int, method: str = "exact", bits=(0, 1, 2, 3, 4, 8)) -> Options:
-    """Candidate sets used for the Mistral / LLaMA shaped workloads: token ranks
-    T/32, T/16, T/8, T/4 (128..1024 beyond 4096 tokens), feature ranks D/4..D."""
+    """Candidate sets used for the Mistral / LLaMA shaped workloads: token ranks T/32, T/16, T/8
+    and 15T/64 (128..960 from 4096 tokens on: 128, 256, 512, 960), feature ranks D/4..D.
+
+    The largest token rank is 15T/64 rather than T/4 so that FlashJoLT's sketch (largest rank
+    + 10 = 250 at 1024 tokens) stays within 256 columns, where the batched eigen solver of the
+    Rayleigh-Ritz step runs at about half the time it needs at 266."""
     if T <= 4096:
-        rt = tuple(max(8, T // d) for d in (32, 16, 8, 4))
+        rt = tuple(max(8, T // d) for d in (32, 16, 8)) + (max(8, (15 * T // 64) // 8 * 8),)
     else:
-        rt = (128, 256, 512, 1024)
+        rt = (128, 256, 512, 960)
     rd = (D // 4, D // 2, 3 * D // 4, D)
     return Options(rt, rd, tuple(bits), method)
 
