@@ -45,17 +45,21 @@ def parse():
     ap.add_argument("--workload", default="mistral7b")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extras", action="store_true", help="skip the exact-arm and decompress side figures")
-    ap.add_argument("--profile-case", default=None, choices=["mistral7b_4layers"],
-                    help="run one compress of a small case (for ncu captures) and exit")
+    ap.add_argument("--profile-case", default=None, choices=["mistral7b_4layers", "mistral7b"],
+                    help="run two compress + decompress calls of one case (for ncu captures) and exit")
     return ap.parse_args()
 
 
 def profile_case(args):
-    """One FlashJoLT (or JoLT) compress + decompress of a 4-layer Mistral-shaped cache (16 MiB of
-    K and V): a case small enough for an ncu capture, with the same kernels as the full run."""
+    """Two FlashJoLT (or JoLT) compress + decompress calls of one case, for ncu captures:
+    mistral7b_4layers (16 MiB of K and V) or the full Mistral-shaped cache (128 MiB, about
+    1 GiB of workspace with FlashJoLT), with the same kernels as the timed run."""
     import torch
     from kv_cache_compression_group_b200 import synth, jolt as J
-    w = synth.small_workload("mistral7b", n_layers=4)
+    if args.profile_case == "mistral7b":
+        w = synth.WORKLOADS["mistral7b"]
+    else:
+        w = synth.small_workload("mistral7b", n_layers=4)
     K, V = synth.make_cache(w, 0)
     Kd, Vd = K.cuda(), V.cuda()
     opts = J.default_options(w.T, w.D, args.method)

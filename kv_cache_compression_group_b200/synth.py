@@ -14,6 +14,8 @@ the two see bit-identical inputs.
 """
 from __future__ import annotations
 
+import os
+from concurrent.futures import ThreadPoolExecutor
 from dataclasses import dataclass, asdict
 
 import numpy as np
@@ -104,22 +106,36 @@ def slice_f64(w: Workload, seed: int, kv: int, layer: int, head: int) -> np.ndar
     return x
 
 
-def make_cache(w: Workload, seed: int = 0, kv: int | None = None, layers: range | None = None):
+def make_cache(w: Workload, seed: int = 0, kv: int | None = None, layers: range | None = None,
+               workers: int | None = None):
     """K and V as CPU torch tensors [n_layers, H, T, D] in the workload's dtype.
 
     With ``kv`` given, returns only that tensor; with ``layers`` given, only those layers
     (the slices are drawn independently, so any sub-range is bit-identical to the same
-    layers of the full tensor).
+    layers of the full tensor).  Slices are generated on ``workers`` threads (default: the
+    CPUs this process may use); every slice has its own stream, so the result does not
+    depend on the thread count.
     """
     tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
     lay = range(w.n_layers) if layers is None else layers
+    if workers is None:
+        workers = max(1, len(os.sched_getaffinity(0)))
     out = []
     for which in ((0, 1) if kv is None else (kv,)):
         t = torch.empty((len(lay), w.n_heads, w.T, w.D), dtype=tdt)
-        for li, layer in enumerate(lay):
-            for h in range(w.n_heads):
-                x = slice_f64(w, seed, which, layer, h)
-                t[li, h] = torch.from_numpy(x.astype(np.float32)).to(tdt)
+
+        def fill(job, which=which, t=t):
+            li, layer, h = job
+            x = slice_f64(w, seed, which, layer, h)
+            t[li, h] = torch.from_numpy(x.astype(np.float32)).to(tdt)
+
+        jobs = [(li, layer, h) for li, layer in enumerate(lay) for h in range(w.n_heads)]
+        if workers > 1 and len(jobs) > 1:
+            with ThreadPoolExecutor(workers) as ex:
+                list(ex.map(fill, jobs))
+        else:
+            for j in jobs:
+                fill(j)
         out.append(t)
     return tuple(out) if kv is None else out[0]
 

@@ -1,0 +1,140 @@
+"""The library at the full workload sizes, in the launch configuration the benchmark times.
+
+At these sizes the float64 checker cannot redo whole compress calls, so every case checks
+  * properties that hold at any size: the byte budget is never exceeded; every unit's
+    measured round-trip error equals the distortion-table entry it was chosen by (table,
+    encoder and decoder agree); decompression is deterministic in its dtype;
+  * sampled outputs the checker computes one by one: for two sampled units, a range of
+    token rows of every slice is decoded by the checker from the library's stored bytes
+    and compared with the library's own decompression, and the checker re-quantises the
+    residual of those rows (formed from the stored factors) and compares scales and codes;
+  * on the Mistral-shaped cache (cheap enough for the checker's own factor step) the
+    token and feature factors of the sampled units against the checker's, with the same
+    randomized sketch, as in the small-size parity tests.
+Tolerances are the ones of the small-size parity tests.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from kv_cache_compression_group_b200 import jolt as J
+from kv_cache_compression_group_b200 import synth
+from blob_helpers import as_record, blob_unit, check_codes
+
+pytestmark = pytest.mark.gpu
+
+FULL = [
+    ("mistral7b", "randomized", (2.0, 3.0)),
+    ("mistral7b", "exact", (2.0,)),
+    ("llama2_13b", "randomized", (2.0, 3.0, 4.0)),
+    ("llama31_8b_64k", "randomized", (2.0, 3.0, 4.0, 5.0)),
+    # the compression-time sweep on the Mistral-shaped generator
+    ("sweep_T512", "exact", (2.0,)), ("sweep_T512", "randomized", (3.0,)),
+    ("sweep_T2048", "exact", (3.0,)), ("sweep_T2048", "randomized", (2.0,)),
+    ("sweep_T8192", "randomized", (2.0, 3.0)), ("sweep_T32768", "randomized", (2.0,)),
+]
+
+
+def _workload(name):
+    if name.startswith("sweep_T"):
+        return synth.sweep_workload(int(name[len("sweep_T"):]))
+    return synth.WORKLOADS[name]
+SEED = 0
+ROWS = 64  # token rows of every slice checked per sampled unit
+
+
+def _unit_x(K, V, w, u, rows=None):
+    """Unit u of the CPU caches in float64 (only token rows [t0, t1) if given)."""
+    g, kv = u // 2, u % 2
+    src = (K if kv == 0 else V)[g * w.layers_per_group:(g + 1) * w.layers_per_group]
+    if rows is not None:
+        src = src[:, :, rows[0]:rows[1]]
+    return synth.to_f64(src.contiguous())
+
+
+def _sampled_rows_check(blob_np, rec, w, u, K, V):
+    """Decode and re-encode token rows [t0, t0 + ROWS) of every slice with the checker."""
+    g, kv = u // 2, u % 2
+    t0 = (w.T - ROWS) if u % 4 == 3 else (u * 37) % (w.T - ROWS + 1)
+    gb = blob_unit(blob_np, rec, w, rows=(t0, t0 + ROWS))
+    r = as_record(gb, w, rec, g, kv, SEED)
+    Xrows = _unit_x(K, V, w, u, (t0, t0 + ROWS))
+    xr = O.rotated_input(Xrows, r.sigma)
+    P = O.recon_operator(r.C_s, r.W_s, r.sigma, r.r_D)
+    rho = xr - np.einsum("tr,lhrd->lhtd", r.U_s, P, optimize=True)
+    counts = check_codes(gb, rho, xr, r.b) if r.b else (0, 0, 0, 0)
+    return t0, Xrows, O.decode_unit(r), counts
+
+
+@pytest.mark.parametrize("name,method,ratios", FULL)
+def test_full_size(name, method, ratios):
+    w = _workload(name)
+    K, V = synth.make_cache(w, SEED)
+    Kd, Vd = K.cuda(), V.cuda()
+    opts = J.default_options(w.T, w.D, method)
+    comp = J.Compressor(w.n_layers, w.n_heads, w.T, w.D, w.layers_per_group, K.dtype, opts)
+    nu = comp.n_units
+    sample = (0, nu - 1)
+    n_scales = n_scale_bad = n_codes = n_code_bad = 0
+    for ratio in ratios:
+        budget = int(w.bf16_bytes() / ratio)
+        blob = comp.compress(Kd, Vd, budget, SEED)
+        _, total, recs = J.read_header(blob)
+        assert total <= budget
+        Kh, Vh = comp.decompress(blob, torch.float32)
+        sq = J.frobenius(Kd, Vd, Kh, Vh, w.layers_per_group).cpu().numpy()
+        for u, r in enumerate(recs):
+            assert abs(sq[u, 1] - r["distortion"]) <= 1e-5 * max(sq[u, 1], 1e-30) + 1e-9 * sq[u, 0], (u, ratio)
+        Kb, _ = comp.decompress(blob, torch.bfloat16)
+        assert torch.equal(Kb, Kh.to(torch.bfloat16))
+        del Kb
+        blob_np = blob[:total].cpu().numpy()
+        for u in sample:
+            t0, X, Xo, counts = _sampled_rows_check(blob_np, recs[u], w, u, K, V)
+            ns, nsb, nc, ncb = counts
+            n_scales, n_scale_bad, n_codes, n_code_bad = (n_scales + ns, n_scale_bad + nsb, n_codes + nc,
+                                                          n_code_bad + ncb)
+            g, kv = u // 2, u % 2
+            Xl = (Kh if kv == 0 else Vh)[g * w.layers_per_group:(g + 1) * w.layers_per_group, :, t0:t0 + ROWS]
+            Xl = Xl.double().cpu().numpy()
+            # fp32 decoder against the float64 one over the same stored bytes
+            assert np.abs(Xl - Xo).max() <= 2.0 ** -18 * (np.abs(Xo).max() + np.abs(X).max()), (u, ratio)
+        del Kh, Vh
+    assert n_scale_bad <= max(4, 2e-3 * n_scales), (n_scale_bad, n_scales)
+    if n_codes:
+        assert n_code_bad <= max(1, 1e-4 * n_codes), (n_code_bad, n_codes)
+
+
+def test_full_size_factors_mistral():
+    """Token and feature factors of sampled units of the full Mistral-shaped cache against
+    the checker's (same seed, so the same Gaussian sketch for FlashJoLT)."""
+    w = synth.WORKLOADS["mistral7b"]
+    K, V = synth.make_cache(w, SEED)
+    Kd, Vd = K.cuda(), V.cuda()
+    for method in ("randomized", "exact"):
+        opts = J.default_options(w.T, w.D, method)
+        oo = O.Options(opts.token_ranks, opts.feature_ranks, opts.bits, method)
+        comp = J.Compressor(w.n_layers, w.n_heads, w.T, w.D, w.layers_per_group, K.dtype, opts)
+        U, W = comp.factor(Kd, Vd, SEED)
+        U, W = U.double().cpu().numpy(), W.double().cpu().numpy()
+        checked = 0
+        for u in (0, comp.n_units - 1):
+            X = _unit_x(K, V, w, u)
+            f = O.unit_factors(X, u // 2, u % 2, oo, SEED)
+            A = O.token_unfolding(X)
+            gt = np.linalg.eigvalsh(A @ A.T)[::-1]
+            for r in oo.token_ranks:
+                gap = (gt[r - 1] - gt[r]) / gt[0]
+                if gap >= 1e-4:
+                    s = np.linalg.norm(f.U[:, :r] - U[u][:, :r] @ (U[u][:, :r].T @ f.U[:, :r]), 2)
+                    assert s <= 1e-3, (method, u, r, s)
+                    checked += 1
+            wv = np.sort(f.w_eigvals)[::-1]
+            for r in oo.feature_ranks:
+                gap = (wv[r - 1] - wv[r]) / wv[0] if r < len(wv) else 1.0
+                if gap >= 1e-4:
+                    s = np.linalg.norm(f.W[:, :r] - W[u][:, :r] @ (W[u][:, :r].T @ f.W[:, :r]), 2)
+                    assert s <= 1e-3, (method, u, r, s)
+                    checked += 1
+        assert checked > 0

@@ -23,6 +23,7 @@ import torch
 import oracle as O
 from kv_cache_compression_group_b200 import jolt as J
 from kv_cache_compression_group_b200 import synth
+from blob_helpers import blob_unit, check_codes
 
 pytestmark = pytest.mark.gpu
 
@@ -201,27 +202,6 @@ def test_allocation_bit_exact_on_oracle_tables():
             assert lam.cpu().numpy()[0].tobytes() == np.float64(al.lam).tobytes()
 
 
-def _blob_unit(blob_np, u, rec, w, block=16):
-    S = w.layers_per_group * w.n_heads
-    T, D = w.T, w.D
-
-    def bf(off, n):
-        return torch.from_numpy(blob_np[off:off + 2 * n].copy()).view(torch.bfloat16).double().numpy()
-
-    Ub = bf(rec["off_U"], T * rec["r_T"]).reshape(T, rec["r_T"])
-    Wb = bf(rec["off_W"], D * rec["r_D"]).reshape(D, rec["r_D"])
-    Cb = bf(rec["off_C"], S * rec["r_T"] * rec["r_D"]).reshape(S, rec["r_T"], rec["r_D"])
-    out = dict(U=Ub, W=Wb, C=Cb)
-    b = rec["bits"]
-    if b:
-        nblk = S * T * D // block
-        packed = blob_np[rec["off_codes"]:rec["off_codes"] + nblk * 2 * b].reshape(nblk, 2 * b)
-        out["codes"] = O.unpack_codes(packed, b).reshape(nblk, block)
-        sc = blob_np[rec["off_scales"]:rec["off_scales"] + nblk * 4].copy().view(np.float16).astype(np.float64)
-        out["lo"], out["step"] = sc[0::2], sc[1::2]
-    return out
-
-
 @pytest.mark.parametrize("name", CASES)
 def test_encode_codes_and_factors(name):
     d = _setup(name)
@@ -238,7 +218,7 @@ def test_encode_codes_and_factors(name):
     n_codes = n_bad = n_scales = n_scale_bad = 0
     for u, (rec_o, rec_g) in enumerate(zip(res.units, recs)):
         assert (rec_g["r_T"], rec_g["r_D"], rec_g["bits"]) == (rec_o.r_T, rec_o.r_D, rec_o.b)
-        g = _blob_unit(bnp, u, rec_g, w)
+        g = blob_unit(bnp, rec_g, w)
         assert np.array_equal(g["U"], rec_o.U_s) and np.array_equal(g["W"], rec_o.W_s)
         assert np.array_equal(g["C"], rec_o.C_s.reshape(g["C"].shape))
         if not rec_o.b:
@@ -247,38 +227,13 @@ def test_encode_codes_and_factors(name):
         iD = d["oo"].feature_ranks.index(rec_o.r_D)
         X = d["units"][u][2]
         Pg = P[iD, u][:, :rec_o.r_T, :].reshape(w.layers_per_group, w.n_heads, rec_o.r_T, w.D)
-        rho = O.rotated_input(X, rec_o.sigma) - np.einsum("tr,lhrd->lhtd", rec_o.U_s, Pg)
-        codes, lo, step, _, _ = O.quantize(rho, rec_o.b)
-        codes, lo, step = codes.reshape(-1, 16), lo.reshape(-1), step.reshape(-1)
-        rb = rho.reshape(-1, 16)
-        # the library forms rho in fp32 from x' and the reconstruction: its error is absolute,
-        # bounded here per block by 2^-17 (max |x'| + max |x_hat|)
-        xr = O.rotated_input(X, rec_o.sigma).reshape(-1, 16)
-        win = 2.0 ** -17 * (np.abs(xr).max(1) + np.abs(xr - rb).max(1))
-        n_scales += lo.size
-        same = (g["lo"] == lo) & (g["step"] == step)
-        bad = np.nonzero(~same)[0]
-        n_scale_bad += bad.size
-        if bad.size:
-            # every differing scale is the rounding of a block minimum / maximum inside the window
-            L = (1 << rec_o.b) - 1
-            mn, mx, wb = rb[bad].min(1), rb[bad].max(1), win[bad]
-            lo_ok = (g["lo"][bad] >= O.fp16_rd(mn - wb)) & (g["lo"][bad] <= O.fp16_rd(mn + wb))
-            st_lo = O.fp16_ru(np.maximum(mx - wb - g["lo"][bad], 0) / L)
-            st_hi = O.fp16_ru((mx + wb - g["lo"][bad]) / L)
-            st_ok = (g["step"][bad] >= st_lo) & (g["step"][bad] <= st_hi)
-            assert np.all(lo_ok & st_ok), bad[~(lo_ok & st_ok)][:5]
-        # codes under the library's own scales, from the oracle's rho
-        gl, gs = g["lo"][:, None], g["step"][:, None]
-        q = (rb - gl) / np.where(gs > 0, gs, 1.0)
-        want = np.where(gs > 0, np.clip(np.rint(q), 0, (1 << rec_o.b) - 1), 0)
-        diff = g["codes"] != want
-        n_codes += want.size
-        n_bad += int(diff.sum())
-        if diff.any():
-            tie = np.abs(q - np.floor(q) - 0.5)
-            tw = (win[:, None] / np.where(gs > 0, gs, 1.0)) + 1e-6
-            assert np.all(tie[diff] <= np.broadcast_to(tw, tie.shape)[diff]), tie[diff].max()
+        xr = O.rotated_input(X, rec_o.sigma)
+        rho = xr - np.einsum("tr,lhrd->lhtd", rec_o.U_s, Pg)
+        ns, nsb, nc, ncb = check_codes(g, rho, xr, rec_o.b)
+        n_scales += ns
+        n_scale_bad += nsb
+        n_codes += nc
+        n_bad += ncb
     assert n_scale_bad <= max(4, 2e-3 * n_scales), (n_scale_bad, n_scales)
     if n_codes:
         assert n_bad <= max(1, 1e-4 * n_codes), (n_bad, n_codes)
