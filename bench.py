@@ -29,10 +29,9 @@ RATIOS = (2.0, 3.0)
 L2_BYTES = 126 * 1024 * 1024
 # FP32 pipe: 148 SMs x 128 lanes, one FMA-class instruction per lane per clock
 SMS, FP32_LANES = 148, 128
-# DRAM bytes (read + write) of one table_kernel launch over the 16 units of the bench workload:
-# an ncu capture of 2 units (profiles/table_kernel_mistral7b_4layers.md) scaled by 8.  None
-# whenever the kernel has changed since that capture.
-TABLE_KERNEL_TRAFFIC_BYTES = 277.6e6
+# DRAM bytes (read + write) of one table_kernel launch over the 16 units of the bench workload
+# from an ncu capture of that kernel (profiles/); None whenever the kernel has changed since.
+TABLE_KERNEL_TRAFFIC_BYTES = None
 
 
 def parse():
@@ -231,27 +230,23 @@ def run_reference(args, rank, world):
 # ------------------------------------------------------------------------------------------
 def main():
     args = parse()
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    from kv_cache_compression_group_b200 import ranks
+    rank, world, local = ranks.dist_env()
     if args.impl == "reference":
         return run_reference(args, rank, world)
     if args.profile_case:
         return profile_case(args)
 
     import torch
-    import torch.distributed as dist
-    from datetime import timedelta
     from kv_cache_compression_group_b200 import synth, jolt as J
 
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    if world > 1:
-        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+    ranks.init(world, "nccl", dev)
 
     w = synth.WORKLOADS[args.workload]
     opts = J.default_options(w.T, w.D, args.method)
-    seed = rank
+    seed = ranks.rank_seed(rank)
     K, V = synth.make_cache(w, seed)
     Kd, Vd = K.to(dev), V.to(dev)
     comp = J.Compressor(w.n_layers, w.n_heads, w.T, w.D, w.layers_per_group, K.dtype, opts, dev)
@@ -265,8 +260,7 @@ def main():
             comp.compress(Ks, Vs, b, seed, blob=blob)
 
     def barrier():
-        if world > 1:
-            dist.barrier()
+        ranks.barrier(world)
 
     for _ in range(args.warmup):
         flush.zero_()
@@ -284,25 +278,20 @@ def main():
     torch.cuda.synchronize()
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     n0 = J.launch_count()
-    J.profile_begin()
     for i in range(args.steps):
         flush.zero_()
         ev[i][0].record(stream)
         step(Kd, Vd)
         ev[i][1].record(stream)
     torch.cuda.synchronize()
-    prof = J.profile_end()
     launches = J.launch_count() - n0
     barrier()
     clk = clocks.stop()
     step_ms = [a.elapsed_time(b) for a, b in ev]
     t_ms = sum(step_ms)
-    if world > 1:
-        tt = torch.tensor([t_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        t_ms = float(tt.item())
+    t_ms = ranks.max_over_ranks(t_ms, world, dev)
     in_bytes = w.input_bytes()
-    value = world * args.steps * len(RATIOS) * in_bytes / (t_ms / 1e3) / 1e9
+    value = ranks.aggregate_gbs(world, args.steps * len(RATIOS) * in_bytes, t_ms)
 
     # ---- end to end through the public API: pinned host in, blobs out ---------------------
     Kh, Vh = K.pin_memory(), V.pin_memory()
@@ -331,14 +320,19 @@ def main():
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
-    e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        tt = torch.tensor([e_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e_ms = float(tt.item())
-    e2e = {"value": world * args.steps * len(RATIOS) * in_bytes / (e_ms / 1e3) / 1e9, "unit": "GB/s",
+    e_ms = ranks.max_over_ranks(e0.elapsed_time(e1), world, dev)
+    e2e = {"value": ranks.aggregate_gbs(world, args.steps * len(RATIOS) * in_bytes, e_ms), "unit": "GB/s",
            "h2d_bytes_per_step": 2 * K.numel() * K.element_size(), "d2h_bytes_per_step": d2h,
            "ms_per_step": e_ms / args.steps}
+
+    # ---- stage breakdown: a separate pass with per-stage events (these calls run without
+    # the CUDA graphs of the timed region, so stage sums exceed the timed step) ------------
+    J.profile_begin()
+    for _ in range(2):
+        flush.zero_()
+        step(Kd, Vd)
+    torch.cuda.synchronize()
+    prof = J.profile_end()
 
     # ---- roofline of the dominant stage ----------------------------------------------------
     peaks, peak_src = load_peaks()
@@ -401,9 +395,8 @@ def main():
                                "kind": "oracle",
                                "sample": f"one unit (keys of layer group 0, [{w.layers_per_group}, {w.n_heads}, "
                                          f"{w.T}, {w.D}] bf16) at the 2x budget, {dt:.1f} s"}
-    if world > 1:
-        dist.barrier()
-        dist.destroy_process_group()
+    ranks.barrier(world)
+    ranks.shutdown(world)
     if rank == 0:
         print(json.dumps(out), flush=True)
 

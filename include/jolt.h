@@ -55,7 +55,7 @@ typedef enum {
   JOLT_ERR_OUTPUT_TOO_SMALL = 4,   /* blob capacity below the budget */
   JOLT_ERR_BUDGET_INFEASIBLE = 5,  /* budget below every unit's fewest-bytes choice */
   JOLT_ERR_NUMERIC = 6,            /* NaN/Inf in the cache, or an eigen/Cholesky breakdown */
-  JOLT_ERR_TIMEOUT = 7,            /* reserved: a bounded device wait gave up */
+  JOLT_ERR_TIMEOUT = 7,            /* a bounded device-side wait (tensor-core pipeline) gave up */
   JOLT_ERR_CUDA = 8,               /* a CUDA runtime or cuSOLVER call failed */
   JOLT_ERR_BAD_BLOB = 9            /* blob header failed validation */
 } jolt_status;
@@ -230,6 +230,18 @@ jolt_status jolt_frobenius(const jolt_shape* shape, const void* k_dev, const voi
  *   - allocates nothing.  Asynchronous. */
 jolt_status jolt_frobenius_noalloc(const jolt_shape* shape, const void* k_dev, const void* v_dev, const void* ky_dev,
                                    const void* vy_dev, int32_t ydtype, double* sq_dev, void* stream);
+
+/* CUDA graphs of compress calls (no counterpart on the pages; on by default).  With graphs
+ * on, jolt_compress captures its stages once per distinct argument set (shape, options,
+ * every pointer and size, budget, seed, device; up to 8 per host thread, least recently used
+ * dropped) on a private stream and afterwards replays the captured graph on the caller's
+ * stream: the same kernels on the same buffers, with one launch.  The captured graph reads
+ * the caller's buffers at replay time, so changing their contents between calls is fine;
+ * freeing a buffer and passing a new one at the same address with the same size is also
+ * fine.  Calls made while stage timing is on, or on a stream that is itself being
+ * captured, run directly.  jolt_set_graphs(0) turns graphs off for this thread and drops
+ * its cached graphs. */
+void jolt_set_graphs(int32_t enable);
 
 /* Stage timing for measurement (no counterpart on the pages).  jolt_profile_begin starts
  * recording CUDA events around every internal stage launched by this thread (on the call's

@@ -17,7 +17,16 @@ inline std::atomic<unsigned long long>& launch_counter() {
   static std::atomic<unsigned long long> n{0};
   return n;
 }
-inline void count_launch() { launch_counter().fetch_add(1, std::memory_order_relaxed); }
+// while this thread captures a CUDA graph, its launches are counted here instead (they run
+// when the graph is launched, and are added to the process count at every launch)
+inline unsigned long long*& capture_counter() {
+  thread_local unsigned long long* c = nullptr;
+  return c;
+}
+inline void count_launch() {
+  if (capture_counter()) ++*capture_counter();
+  else launch_counter().fetch_add(1, std::memory_order_relaxed);
+}
 
 typedef __nv_bfloat16 bf16;
 
@@ -28,6 +37,7 @@ enum : uint32_t {
   DEV_ERR_INFEASIBLE = 4u,    // budget below the fewest-bytes choice of every unit
   DEV_ERR_BLOB = 8u,          // a compressed record failed validation
   DEV_ERR_CAPACITY = 16u,     // output buffer smaller than the chosen payload
+  DEV_ERR_TIMEOUT = 32u,      // a bounded device-side wait gave up
 };
 
 // ---- splitmix64 (Steele, Lea & Flood, OOPSLA 2014) ------------------------------------

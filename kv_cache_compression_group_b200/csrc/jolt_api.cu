@@ -13,6 +13,7 @@
 #include "gemm.cuh"
 #include "kernels.cuh"
 #include "misc.cuh"
+#include "umma.cuh"
 
 using namespace jolt;
 
@@ -55,22 +56,46 @@ struct Solver {
   int device = -1;
   std::vector<char> host_ws;
 };
-thread_local Solver g_solver;
+thread_local Solver g_solver[2];   // [0]: the caller's stream, [1]: the auxiliary stream
 
-jolt_status solver_get(cudaStream_t st, Solver** out) {
+jolt_status solver_get(cudaStream_t st, Solver** out, int idx = 0) {
   int dev = 0;
   CUDA_TRY(cudaGetDevice(&dev));
-  if (g_solver.h == nullptr || g_solver.device != dev) {
-    if (g_solver.h) {
-      cusolverDnDestroyParams(g_solver.params);
-      cusolverDnDestroy(g_solver.h);
+  Solver& sv = g_solver[idx];
+  if (sv.h == nullptr || sv.device != dev) {
+    if (sv.h) {
+      cusolverDnDestroyParams(sv.params);
+      cusolverDnDestroy(sv.h);
     }
-    SOLVER_TRY(cusolverDnCreate(&g_solver.h));
-    SOLVER_TRY(cusolverDnCreateParams(&g_solver.params));
-    g_solver.device = dev;
+    SOLVER_TRY(cusolverDnCreate(&sv.h));
+    SOLVER_TRY(cusolverDnCreateParams(&sv.params));
+    sv.device = dev;
   }
-  SOLVER_TRY(cusolverDnSetStream(g_solver.h, st));
-  *out = &g_solver;
+  SOLVER_TRY(cusolverDnSetStream(sv.h, st));
+  *out = &sv;
+  return JOLT_OK;
+}
+
+// An auxiliary stream (one per host thread and device) on which the feature factor runs
+// concurrently with the token factor; fork / join through events on the caller's stream,
+// so the pair is legal inside stream capture.
+struct Aux {
+  cudaStream_t st = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+  int device = -1;
+};
+thread_local Aux g_aux;
+
+jolt_status aux_get(Aux** out) {
+  int dev = 0;
+  CUDA_TRY(cudaGetDevice(&dev));
+  if (g_aux.st == nullptr || g_aux.device != dev) {
+    CUDA_TRY(cudaStreamCreateWithFlags(&g_aux.st, cudaStreamNonBlocking));
+    CUDA_TRY(cudaEventCreateWithFlags(&g_aux.fork, cudaEventDisableTiming));
+    CUDA_TRY(cudaEventCreateWithFlags(&g_aux.join, cudaEventDisableTiming));
+    g_aux.device = dev;
+  }
+  *out = &g_aux;
   return JOLT_OK;
 }
 
@@ -137,14 +162,14 @@ struct Plan {
   bool m_side;            // exact token factor through the M x M Gram (T > M)
   int gd_split;           // split-K of the feature Gram
   int gt_split;           // split-K of the token Gram
-  size_t solver_dev;      // cuSOLVER device workspace
+  size_t solver_dev;      // cuSOLVER device workspace (token factor)
+  size_t fsolver_dev;     // cuSOLVER device workspace (feature factor, on the auxiliary stream)
   size_t solver_host;
   // workspace offsets (bytes)
   size_t o_status, o_gd_part, o_gd, o_evals, o_Wf, o_Ws, o_Uf, o_Us, o_core, o_zc, o_ptmp, o_P, o_partial,
-      o_table, o_bytes, o_choice, o_lambda, o_hdr, o_umap, o_info, o_solver;
+      o_table, o_bytes, o_choice, o_lambda, o_hdr, o_umap, o_info, o_solver, o_fsolver, o_finfo, o_fevals;
   // token factor scratch (all units)
-  size_t o_gt32, o_gt, o_vsel, o_lam, o_omega, o_Y, o_Zm, o_h, o_l, o_gpart, o_G, o_ptrs, o_shift, o_Lr, o_Linv,
-      o_qtmp;
+  size_t o_gt32, o_gt, o_vsel, o_lam, o_omega, o_Y, o_Zm, o_h, o_l, o_gpart, o_G, o_ptrs, o_Lr, o_Linv;
   int qr_split_max;       // split-K of the Cholesky-QR Grams
   size_t ws_total;
   int tiles;
@@ -244,6 +269,7 @@ jolt_status make_plan(const jolt_shape* sh, const jolt_options* op, Plan* p) {
   {
     long long ntok = op->method == JOLT_EXACT ? (p->m_side ? M : T) : p->k;
     p->solver_dev = 0;
+    p->fsolver_dev = 0;
     p->solver_host = 0;
     int ndev = 0;
     bool queried = false;
@@ -259,15 +285,16 @@ jolt_status make_plan(const jolt_shape* sh, const jolt_options* op, Plan* p) {
             queried = false;
             break;
           }
-          p->solver_dev = dv > p->solver_dev ? dv : p->solver_dev;
+          if (n == D) p->fsolver_dev = dv;
+          if (n == ntok) p->solver_dev = dv > p->solver_dev ? dv : p->solver_dev;
           p->solver_host = hv > p->solver_host ? hv : p->solver_host;
         }
       }
     }
     cudaGetLastError();
     if (!queried) {
-      long long nmax = ntok > D ? ntok : D;
-      p->solver_dev = (size_t)NU * (size_t)(8 * (1 + 6 * nmax + 2 * nmax * nmax) * 8) + (16 << 20);
+      p->solver_dev = (size_t)NU * (size_t)(8 * (1 + 6 * ntok + 2 * ntok * ntok) * 8) + (16 << 20);
+      p->fsolver_dev = (size_t)NU * (size_t)(8 * (1 + 6 * (long long)D + 2 * (long long)D * D) * 8) + (16 << 20);
     }
   }
 
@@ -296,8 +323,10 @@ jolt_status make_plan(const jolt_shape* sh, const jolt_options* op, Plan* p) {
   p->o_hdr = b.take(64);
   p->o_umap = b.take((size_t)NU * S * 4 + 64);
   p->o_info = b.take((size_t)NU * 4 + 64);
-  p->o_shift = b.take((size_t)NU * 8 + 64);
   p->o_solver = b.take(p->solver_dev + 256);
+  p->o_fsolver = b.take(p->fsolver_dev + 256);
+  p->o_finfo = b.take((size_t)NU * 4 + 64);
+  p->o_fevals = b.take((size_t)NU * D * 8 + 256);
   // token factor scratch
   p->o_gt32 = p->o_gt = p->o_vsel = p->o_lam = p->o_omega = 0;
   p->o_Y = p->o_Zm = p->o_h = p->o_l = p->o_gpart = p->o_G = p->o_ptrs = 0;
@@ -322,16 +351,14 @@ jolt_status make_plan(const jolt_shape* sh, const jolt_options* op, Plan* p) {
     p->o_l = b.take((size_t)NU * big * kp * 2);
     p->o_vsel = b.take((size_t)NU * kp * p->ldU * 4);
   }
-  p->o_Lr = p->o_Linv = p->o_qtmp = 0;
+  p->o_Lr = p->o_Linv = 0;
   if (op->method == JOLT_RANDOMIZED || p->m_side) {
-    long long mrows = op->method == JOLT_RANDOMIZED ? (M > T ? M : T) : T;
     p->o_gpart = b.take((size_t)NU * p->qr_split_max * kq * kq * 4);
     p->o_G = b.take((size_t)NU * kq * kq * 8);
-    p->o_Lr = b.take((size_t)NU * kq * kq * 4);
-    p->o_Linv = b.take((size_t)NU * kq * kq * 4);
-    p->o_qtmp = b.take((size_t)NU * mrows * kq * 4);
+    p->o_Lr = b.take((size_t)NU * kq * kq * 4);   // L as fp32 row-major
+    p->o_ptrs = b.take((size_t)NU * 8 + 64);
+    p->o_Linv = b.take((size_t)NU * round_up(kq, 32) * 32 * 4);   // inverses of the 32 x 32 diagonal blocks
   }
-  p->o_ptrs = b.take((size_t)NU * 8 + 64);
   p->ws_total = b.off;
 
   // largest possible blob
@@ -399,6 +426,7 @@ struct Ctx {
   const void* k;
   const void* v;
   uint64_t seed;
+  int side = 0;   // 1: the feature factor on the auxiliary stream (own eigen-solver workspace)
   template <typename T>
   T* at(size_t off) const { return reinterpret_cast<T*>(ws + off); }
   uint32_t* status() const { return at<uint32_t>(p.o_status); }
@@ -434,8 +462,8 @@ GemmOperand xt_rowmajor(const Ctx& c, const void* x) {
 // ------------------------------------------------------------------------------------------
 // the solver's device workspace must fit the plan's bound; host workspace grows on demand
 jolt_status solver_ws(const Ctx& c, Solver* s, size_t dv, size_t hv, void** host) {
-  if (dv > c.p.solver_dev)
-    return fail(JOLT_ERR_WORKSPACE_TOO_SMALL, "cuSOLVER needs %zu device bytes, plan holds %zu", dv, c.p.solver_dev);
+  const size_t cap = c.side ? c.p.fsolver_dev : c.p.solver_dev;
+  if (dv > cap) return fail(JOLT_ERR_WORKSPACE_TOO_SMALL, "cuSOLVER needs %zu device bytes, plan holds %zu", dv, cap);
   if (s->host_ws.size() < hv) s->host_ws.resize(hv);
   *host = hv ? s->host_ws.data() : nullptr;
   return JOLT_OK;
@@ -445,7 +473,9 @@ jolt_status solver_ws(const Ctx& c, Solver* s, size_t dv, size_t hv, void** host
 jolt_status sym_eig_batched(const Ctx& c, double* A, int64_t n, double* w, int64_t nbatch) {
   ProfScope ps("sym_eig", c.st, nbatch);
   Solver* s = nullptr;
-  JTRY(solver_get(c.st, &s));
+  JTRY(solver_get(c.st, &s, c.side));
+  void* dws = c.at<void>(c.side ? c.p.o_fsolver : c.p.o_solver);
+  int* info = c.at<int>(c.side ? c.p.o_finfo : c.p.o_info);
   size_t dv = 0, hv = 0;
   SOLVER_TRY(cusolverDnXsyevBatched_bufferSize(s->h, s->params, CUSOLVER_EIG_MODE_VECTOR, CUBLAS_FILL_MODE_LOWER, n,
                                                CUDA_R_64F, A, n, CUDA_R_64F, w, CUDA_R_64F, &dv, &hv, nbatch));
@@ -454,10 +484,8 @@ jolt_status sym_eig_batched(const Ctx& c, double* A, int64_t n, double* w, int64
   count_launch(), sanitize_sym_batched_kernel<<<(unsigned)nbatch, 1024, 0, c.st>>>(A, (int)n, n, n * n, c.status());
   CUDA_TRY(cudaGetLastError());
   SOLVER_TRY(cusolverDnXsyevBatched(s->h, s->params, CUSOLVER_EIG_MODE_VECTOR, CUBLAS_FILL_MODE_LOWER, n, CUDA_R_64F,
-                                    A, n, CUDA_R_64F, w, CUDA_R_64F, c.at<void>(c.p.o_solver), dv, host, hv,
-                                    c.at<int>(c.p.o_info), nbatch));
-  count_launch(), info_check_kernel<<<(unsigned)ceil_div(nbatch, 32), 32, 0, c.st>>>(c.at<int>(c.p.o_info),
-                                                                                   (int)nbatch, c.status(),
+                                    A, n, CUDA_R_64F, w, CUDA_R_64F, dws, dv, host, hv, info, nbatch));
+  count_launch(), info_check_kernel<<<(unsigned)ceil_div(nbatch, 32), 32, 0, c.st>>>(info, (int)nbatch, c.status(),
                                                                                    DEV_ERR_FACTOR);
   CUDA_TRY(cudaGetLastError());
   return JOLT_OK;
@@ -467,17 +495,29 @@ jolt_status sym_eig_batched(const Ctx& c, double* A, int64_t n, double* w, int64
 // lda = n, stride n*n; overwritten by the solver), through cuSOLVER's batched eigen solver.
 jolt_status sym_eig_top(const Ctx& c, double* S, int n, int nbatch, int r, float* out_f32, bf16* out_bf16,
                         long long ldo, long long sout, double* out_vals) {
-  double* w = c.at<double>(c.p.o_evals);
+  double* w = c.at<double>(c.side ? c.p.o_fevals : c.p.o_evals);
   JTRY(sym_eig_batched(c, S, n, w, nbatch));
-  count_launch(), eig_select_kernel<<<dim3(r, nbatch), 256, 0, c.st>>>(w, S, n, n, n, (long long)n * n, r, out_f32,
+  count_launch(), eig_select_kernel<<<dim3(r, nbatch), 256, 0, c.st>>>(w, S, n, n, 1, n, (long long)n * n, r, out_f32,
                                                                        out_bf16, ldo, sout, out_vals);
   CUDA_TRY(cudaGetLastError());
   return JOLT_OK;
 }
 
 // Cholesky QR of every unit's m x k block Y (fp32, row pitch ld, unit stride m*ld), in
-// place: G = Y^T Y (fp32 partial sums of <= 256 terms, added in fp64), G = L L^T (batched
-// Cholesky), Q = Y L^{-T} (row-wise triangular solve).  `passes` = 2 gives CholeskyQR2.
+// place: G = Y^T Y (fp32 partial sums of <= 256 terms, added in fp64), G = L L^T (cuSOLVER's
+// batched Cholesky, fp64), Q = Y L^{-T} (blocked row-panel solve).  `passes` = 2 gives
+// CholeskyQR2.
+template <int RB>
+jolt_status launch_trsm_panel(const Ctx& c, float* Y, long long m, int k, int ld, const float* Lr, long long ldl,
+                              long long sL, const float* Dinv, long long sD) {
+  const size_t sm = trsm_smem(RB, k);
+  CUDA_TRY(cudaFuncSetAttribute(trsm_panel_kernel<RB>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm));
+  count_launch(), trsm_panel_kernel<RB><<<dim3((unsigned)ceil_div(m, RB), c.p.NU), 256, sm, c.st>>>(
+      Y, m, k, ld, m * ld, Lr, ldl, sL, Dinv, sD);
+  CUDA_TRY(cudaGetLastError());
+  return JOLT_OK;
+}
+
 jolt_status cholqr_batched(const Ctx& c, float* Y, long long m, int k, int ld, int passes) {
   const Plan& p = c.p;
   ProfScope ps("cholesky_qr", c.st, p.NU);
@@ -489,6 +529,7 @@ jolt_status cholqr_batched(const Ctx& c, float* Y, long long m, int k, int ld, i
   int* info = c.at<int>(p.o_info);
   const int ns = (int)ceil_div(m, 256);
   const int gld = ld;
+  if (k > 1024) return fail(JOLT_ERR_UNSUPPORTED_SHAPE, "Cholesky QR of more than 1024 columns");
   for (int pass = 0; pass < passes; ++pass) {
     ProfScope ps1("qr_gram", c.st, p.NU);
     GemmParams g;
@@ -518,42 +559,16 @@ jolt_status cholqr_batched(const Ctx& c, float* Y, long long m, int k, int ld, i
     SOLVER_TRY(cusolverDnDpotrfBatched(s->h, CUBLAS_FILL_MODE_LOWER, k, ptrs, gld, info, p.NU));
     count_launch(), info_check_kernel<<<(unsigned)ceil_div(p.NU, 32), 32, 0, c.st>>>(info, p.NU, c.status(),
                                                                                       DEV_ERR_FACTOR);
+    CUDA_TRY(cudaGetLastError());
     ProfScope ps3("qr_trsm", c.st, p.NU);
-    // Q = Y L^{-T}: L^{-1} by column-parallel forward substitution, then a GEMM
     float* Lr = c.at<float>(p.o_Lr);
-    float* Li = c.at<float>(p.o_Linv);
-    float* Qt = c.at<float>(p.o_qtmp);
-    count_launch(), lower_to_rowmajor_kernel<<<grid1d((long long)p.NU * k * k), 256, 0, c.st>>>(
-        G, k, gld, n, Lr, gld, (long long)k * gld, p.NU);
-    {
-      const int nth = 32 * (int)(ceil_div(ceil_div(k, TRI_NB), 1) < 32 ? ceil_div(k, TRI_NB) : 32);
-      const size_t sm = trinv_smem(nth);
-      CUDA_TRY(cudaFuncSetAttribute(trinv_blocked_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm));
-      count_launch(), trinv_blocked_kernel<<<p.NU, nth, sm, c.st>>>(Lr, k, gld, (long long)k * gld, Li, c.status());
-    }
+    float* Dinv = c.at<float>(p.o_Linv);
+    const int nbk = (int)ceil_div(k, TS_NB);
+    const long long sL = (long long)k * gld, sD = (long long)nbk * TS_NB * TS_NB;
+    count_launch(), trsm_prep_kernel<<<dim3(nbk, p.NU), 32, 0, c.st>>>(G, k, gld, n, Lr, gld, sL, Dinv, sD);
     CUDA_TRY(cudaGetLastError());
-    GemmParams q;
-    q.M = (int)m;
-    q.N = k;
-    q.K = k;
-    q.batch = p.NU;
-    q.A.ptr = Y;
-    q.A.kmajor = true;
-    q.A.ld = ld;
-    q.A.sbatch = m * ld;
-    q.B.ptr = Li;       // B(i, j) = L^{-1}[j][i]: row j of L^{-1} is contiguous in i
-    q.B.kmajor = true;
-    q.B.ld = gld;
-    q.B.sbatch = (long long)k * gld;
-    q.C = Qt;
-    q.ldc = ld;
-    q.sbatchC = m * ld;
-    q.c_type = 0;
-    JTRY(gemm(q, 1, 1, c.st));
-    // copy the k columns back (the padding columns of Y stay as they are)
-    CUDA_TRY(cudaMemcpy2DAsync(Y, (size_t)ld * 4, Qt, (size_t)ld * 4, (size_t)k * 4, (size_t)(p.NU * m),
-                               cudaMemcpyDeviceToDevice, c.st));
-    CUDA_TRY(cudaGetLastError());
+    if (k <= 512) JTRY(launch_trsm_panel<64>(c, Y, m, k, ld, Lr, gld, sL, Dinv, sD));
+    else JTRY(launch_trsm_panel<32>(c, Y, m, k, ld, Lr, gld, sL, Dinv, sD));
   }
   return JOLT_OK;
 }
@@ -590,6 +605,47 @@ jolt_status gemm_xf(const Ctx& c, GemmParams g, bool f_is_A, const float* F, lon
 
 int xtype(const Ctx& c) { return c.p.dtype == JOLT_BF16 ? 0 : 1; }
 
+// the X-products of the sketch run on the tcgen05 kernel when the cache is bf16 and a
+// 64-wide feature box stays inside one slice
+bool umma_ok(const Plan& p) { return p.dtype == JOLT_BF16 && p.D % 64 == 0 && p.T % 64 == 0; }
+
+// tensor maps of the K and V caches as slices (X_(T) modes) or as rows (X_(D) modes)
+jolt_status cache_maps(const Ctx& c, bool rows, CUtensorMap* mk, CUtensorMap* mv) {
+  const Plan& p = c.p;
+  const bool ok = rows ? (map_cache_rows(mk, c.k, p.nL, p.H, p.T, p.D) && map_cache_rows(mv, c.v, p.nL, p.H, p.T, p.D))
+                       : (map_cache_xt(mk, c.k, p.nL, p.H, p.T, p.D) && map_cache_xt(mv, c.v, p.nL, p.H, p.T, p.D));
+  if (!ok) return fail(JOLT_ERR_CUDA, "tensor map of the cache refused");
+  return JOLT_OK;
+}
+
+jolt_status umma_run(const UmmaMaps& m, const UmmaArgs& a, int nb, cudaStream_t st) {
+  cudaError_t e = launch_umma(m, a, nb, st);
+  if (e != cudaSuccess) return fail(JOLT_ERR_CUDA, "tensor-core GEMM: %s", cudaGetErrorString(e));
+  return JOLT_OK;
+}
+
+// z_side = false: out (T x k per unit) = X_(T) F, F = M x kp ; z_side = true: out (M x k) =
+// X_(T)^T F, F = T x kp.  F is bf16 (F16, one operand) or fp32 (F32, split into hi + lo).
+jolt_status umma_product(const Ctx& c, bool z_side, const bf16* F16, const float* F32, float* out) {
+  const Plan& p = c.p;
+  ProfScope ps("sketch_product", c.st, p.NU);
+  const bf16* f0 = F16;
+  const bf16* f1 = nullptr;
+  if (F32) {
+    bf16* hi = c.at<bf16>(p.o_h);
+    bf16* lo = c.at<bf16>(p.o_l);
+    const long long nF = (long long)p.NU * (z_side ? p.T : p.M) * p.kp;
+    count_launch(), split_bf16_kernel<<<grid1d(nF), 256, 0, c.st>>>(F32, hi, lo, nF);
+    CUDA_TRY(cudaGetLastError());
+    f0 = hi;
+    f1 = lo;
+  }
+  cudaError_t e = umma_x_product(c.k, c.v, p.nL, p.H, p.T, p.D, p.S, p.NU, z_side, f0, f1, p.kp, p.k, out, p.kp,
+                                 c.status(), c.st);
+  if (e != cudaSuccess) return fail(JOLT_ERR_CUDA, "tensor-core X-product: %s", cudaGetErrorString(e));
+  return JOLT_OK;
+}
+
 // the cache of every unit as a batched operand: X_(T) (T x M, rows t, columns (l,h,d))
 GemmOperand xt_units(const Ctx& c) {
   GemmOperand o = xt_rowmajor(c, c.k);
@@ -619,8 +675,30 @@ jolt_status run_feature_factor(const Ctx& c, float* Wf, long long ldWf, bf16* Ws
   const int D = p.D;
   float* part = c.at<float>(p.o_gd_part);
   const long long rows = (long long)p.S * p.T;
-  const int kchunk = (int)round_up(ceil_div(rows, p.gd_split), 32);
-  {
+  if (umma_ok(p)) {
+    // G_D partial sums on the tensor cores: A = B = X_(D) (one shared tile per K block)
+    UmmaMaps m;
+    JTRY(cache_maps(c, true, &m.a0, &m.a1));
+    m.b0 = m.a0;
+    m.b1 = m.a1;
+    UmmaArgs a;
+    a.M = a.N = D;
+    a.K = (int)rows;
+    a.batch = p.NU;
+    a.splits = p.gd_split;
+    a.kchunk = (int)round_up(ceil_div(rows, p.gd_split), 64);
+    a.A.mode = UM_ROW_MN;
+    a.A.rows = rows;
+    a.B = a.A;
+    a.b_is_a = true;
+    a.C = part;
+    a.ldc = D;
+    a.sC = (long long)p.gd_split * D * D;
+    a.ssplit = (long long)D * D;
+    a.status = c.status();
+    JTRY(umma_run(m, a, 1, c.st));
+  } else {
+    const int kchunk = (int)round_up(ceil_div(rows, p.gd_split), 32);
     GemmParams g;
     g.M = D;
     g.N = D;
@@ -679,7 +757,27 @@ jolt_status run_token_exact(const Ctx& c, float* Uf, long long ldUf) {
       g.A = xtT_units(c);
       g.B = g.A;
     }
-    JTRY(gemm(g, xtype(c), xtype(c), c.st));
+    if (umma_ok(p)) {
+      UmmaMaps m;
+      JTRY(cache_maps(c, false, &m.a0, &m.a1));
+      m.b0 = m.a0;
+      m.b1 = m.a1;
+      UmmaArgs a;
+      a.M = a.N = (int)n;
+      a.K = p.m_side ? T : M;
+      a.batch = p.NU;
+      a.A.mode = p.m_side ? UM_XT_MN : UM_XT_K;
+      a.A.S = p.S;
+      a.A.d_shift = ilog2(p.D);
+      a.B = a.A;
+      a.C = G32;
+      a.ldc = n;
+      a.sC = n * n;
+      a.status = c.status();
+      JTRY(umma_run(m, a, 1, c.st));
+    } else {
+      JTRY(gemm(g, xtype(c), xtype(c), c.st));
+    }
   }
   count_launch(), f32_to_f64_kernel<<<grid1d((long long)p.NU * n * n), 256, 0, c.st>>>(G32, G, (long long)p.NU * n * n);
   CUDA_TRY(cudaGetLastError());
@@ -704,7 +802,18 @@ jolt_status run_token_exact(const Ctx& c, float* Uf, long long ldUf) {
   y.ldc = ldUf;
   y.sbatchC = (long long)T * ldUf;
   y.c_type = 0;
-  JTRY(gemm_xf(c, y, false, V, (long long)p.NU * M * p.ldU));
+  if (umma_ok(p)) {
+    bf16* hi = c.at<bf16>(p.o_h);
+    bf16* lo = c.at<bf16>(p.o_l);
+    const long long nF = (long long)p.NU * M * p.ldU;
+    count_launch(), split_bf16_kernel<<<grid1d(nF), 256, 0, c.st>>>(V, hi, lo, nF);
+    CUDA_TRY(cudaGetLastError());
+    cudaError_t e = umma_x_product(c.k, c.v, p.nL, p.H, T, p.D, p.S, p.NU, false, hi, lo, p.ldU, p.rTmax, Uf, ldUf,
+                                   c.status(), c.st);
+    if (e != cudaSuccess) return fail(JOLT_ERR_CUDA, "tensor-core X-product: %s", cudaGetErrorString(e));
+  } else {
+    JTRY(gemm_xf(c, y, false, V, (long long)p.NU * M * p.ldU));
+  }
   JTRY(cholqr_batched(c, Uf, T, p.rTmax, (int)ldUf, 2));
   return JOLT_OK;
 }
@@ -742,7 +851,10 @@ jolt_status run_token_randomized(const Ctx& c, float* Uf, long long ldUf) {
   gz.A = xtT_units(c);
   gz.C = Z;
   gz.sbatchC = (long long)M * kp;
-  {
+  const bool tc = umma_ok(p);
+  if (tc) {
+    JTRY(umma_product(c, false, Om, nullptr, Y));   // Y = X_(T) Omega
+  } else {
     ProfScope ps0("sketch_product", c.st, NU);
     GemmParams g0 = gy;  // Y = X_(T) Omega
     g0.B.ptr = Om;
@@ -751,15 +863,21 @@ jolt_status run_token_randomized(const Ctx& c, float* Uf, long long ldUf) {
   }
   gy.B.sbatch = (long long)M * kp;   // Y = X_(T) Qz : B = Qz (M x k)
   gz.B.sbatch = (long long)T * kp;   // Z = X_(T)^T Q : B = Q (T x k)
+  auto z_of = [&](const float* Q) -> jolt_status {  // Z = X_(T)^T Q
+    return tc ? umma_product(c, true, nullptr, Q, Z) : gemm_xf(c, gz, false, Q, (long long)NU * T * kp);
+  };
+  auto y_of = [&](const float* Qz) -> jolt_status {  // Y = X_(T) Qz
+    return tc ? umma_product(c, false, nullptr, Qz, Y) : gemm_xf(c, gy, false, Qz, (long long)NU * M * kp);
+  };
   JTRY(cholqr_batched(c, Y, T, k, kp, p.q == 0 ? 2 : 1));
   for (int it = 0; it < p.q; ++it) {
-    JTRY(gemm_xf(c, gz, false, Y, (long long)NU * T * kp));
+    JTRY(z_of(Y));
     JTRY(cholqr_batched(c, Z, M, k, kp, 1));
-    JTRY(gemm_xf(c, gy, false, Z, (long long)NU * M * kp));
+    JTRY(y_of(Z));
     JTRY(cholqr_batched(c, Y, T, k, kp, it + 1 == p.q ? 2 : 1));
   }
   // Rayleigh-Ritz: S = Z^T Z with Z = X_(T)^T Q  (k x k per unit)
-  JTRY(gemm_xf(c, gz, false, Y, (long long)NU * T * kp));
+  JTRY(z_of(Y));
   float* gpart = c.at<float>(p.o_gpart);
   double* S = c.at<double>(p.o_G);
   const int ns = (int)ceil_div(M, 256);
@@ -815,9 +933,20 @@ jolt_status run_token_randomized(const Ctx& c, float* Uf, long long ldUf) {
 jolt_status run_factor(const Ctx& c, float* Uf, long long ldUf, float* Wf, long long ldWf, bf16* Us, bf16* Ws) {
   const Plan& p = c.p;
   CUDA_TRY(cudaMemsetAsync(c.status(), 0, 4, c.st));
-  JTRY(run_feature_factor(c, Wf, ldWf, Ws));
+  // the feature factor (its Gram and a small eigen solve) runs on the auxiliary stream while
+  // the token factor runs on the caller's; the two share only the status word (atomic OR)
+  Aux* ax = nullptr;
+  JTRY(aux_get(&ax));
+  CUDA_TRY(cudaEventRecord(ax->fork, c.st));
+  CUDA_TRY(cudaStreamWaitEvent(ax->st, ax->fork, 0));
+  Ctx cf = c;
+  cf.st = ax->st;
+  cf.side = 1;
+  JTRY(run_feature_factor(cf, Wf, ldWf, Ws));
+  CUDA_TRY(cudaEventRecord(ax->join, ax->st));
   if (p.method == JOLT_EXACT) JTRY(run_token_exact(c, Uf, ldUf));
   else JTRY(run_token_randomized(c, Uf, ldUf));
+  CUDA_TRY(cudaStreamWaitEvent(c.st, ax->join, 0));
   // sign convention of the token factor columns (the randomized and back-projected routes
   // need it; for the eigenvector route it is already in place) and the bf16 copy
   count_launch(), col_sign_fix_kernel<<<dim3(p.rTmax, p.NU), 256, 0, c.st>>>(
@@ -834,6 +963,47 @@ jolt_status run_core(const Ctx& c, const bf16* Us, long long ldU, const bf16* Ws
   ProfScope ps("core", c.st, p.NU);
   const int T = p.T, D = p.D, S = p.S;
   bf16* Zc = c.at<bf16>(p.o_zc);
+  if (umma_ok(p)) {
+    // Z = bf16(X_(D) W_s) : A = X_(D) rows (K-major), B = W_s (D x rDmax, MN-major)
+    UmmaMaps m;
+    JTRY(cache_maps(c, true, &m.a0, &m.a1));
+    if (!map_dense(&m.b0, Ws, ldW, D, p.NU)) return fail(JOLT_ERR_CUDA, "tensor map of W refused");
+    m.b1 = m.b0;
+    UmmaArgs a;
+    a.M = S * T;
+    a.N = p.rDmax;
+    a.K = D;
+    a.batch = p.NU;
+    a.A.mode = UM_ROW_K;
+    a.A.rows = (long long)S * T;
+    a.B.mode = UM_DENSE_MN;
+    a.C = Zc;
+    a.c_bf16 = 1;
+    a.ldc = p.ldW;
+    a.sC = (long long)S * T * p.ldW;
+    a.status = c.status();
+    JTRY(umma_run(m, a, 1, c.st));
+    // C_s = bf16(U_s^T Z_s) per (unit, slice): A = U_s^T (MN-major, shared by the S slices)
+    UmmaMaps m2;
+    if (!map_dense(&m2.a0, Us, ldU, T, p.NU) || !map_dense(&m2.b0, Zc, p.ldW, T, (long long)p.NU * S))
+      return fail(JOLT_ERR_CUDA, "tensor map of U / Z refused");
+    m2.a1 = m2.a0;
+    m2.b1 = m2.b0;
+    UmmaArgs a2;
+    a2.M = p.rTmax;
+    a2.N = p.rDmax;
+    a2.K = T;
+    a2.batch = p.NU * S;
+    a2.A.mode = UM_DENSE_MN;
+    a2.A.ediv = S;
+    a2.B.mode = UM_DENSE_MN;
+    a2.C = core;
+    a2.c_bf16 = 1;
+    a2.ldc = p.ldC;
+    a2.sC = (long long)p.rTmax * p.ldC;
+    a2.status = c.status();
+    return umma_run(m2, a2, 1, c.st);
+  }
   // Z = bf16(X_(D) W_s)   ((S T) x rDmax per unit)
   GemmParams z;
   z.M = S * T;
@@ -959,7 +1129,7 @@ template <int D, typename TX>
 jolt_status launch_table_T(const Ctx& c, const TableArgs& a) {
   size_t sm = table_smem<D>();
   CUDA_TRY(cudaFuncSetAttribute(table_kernel<D, TX>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm));
-  count_launch(), table_kernel<D, TX><<<dim3(c.p.tiles, c.p.S, c.p.NU), TTHREADS, sm, c.st>>>(a);
+  count_launch(), table_kernel<D, TX><<<dim3(c.p.tiles, c.p.S, c.p.NU), table_threads<D>(), sm, c.st>>>(a);
   CUDA_TRY(cudaGetLastError());
   return JOLT_OK;
 }
@@ -1324,6 +1494,133 @@ jolt_status jolt_encode(const jolt_shape* shape, const void* k_dev, const void* 
   return run_encode(c, (const bf16*)u_bf16_dev, ld_u, Ws, ld_w, core, (unsigned char*)blob_dev);
 }
 
+// the compress stages of one call, enqueued on c.st
+jolt_status compress_body(const Ctx& c, uint64_t budget_bytes, unsigned long long hdr, void* blob_dev,
+                          size_t blob_cap) {
+  const Plan& p = c.p;
+  float* Uf = c.at<float>(p.o_Uf);
+  float* Wf = c.at<float>(p.o_Wf);
+  bf16* Us = c.at<bf16>(p.o_Us);
+  bf16* Ws = c.at<bf16>(p.o_Ws);
+  JTRY(run_factor(c, Uf, p.ldU, Wf, p.ldW, Us, Ws));
+  bf16* core = c.at<bf16>(p.o_core);
+  double* table = c.at<double>(p.o_table);
+  JTRY(run_table(c, Us, p.ldU, Ws, p.ldW, core, table));
+  JTRY(run_allocate(c, table, budget_bytes - hdr, (unsigned char*)blob_dev, blob_cap, nullptr));
+  JTRY(run_encode(c, Us, p.ldU, Ws, p.ldW, core, (unsigned char*)blob_dev));
+  // device-side errors of the factor stage are folded into the header status
+  count_launch(), fold_status_kernel<<<1, 1, 0, c.st>>>(c.status(), (unsigned char*)blob_dev);
+  CUDA_TRY(cudaGetLastError());
+  return JOLT_OK;
+}
+
+// ------------------------------------------------------------------------------------------
+// CUDA graphs of whole compress calls.  A call whose arguments (shape, options, every
+// pointer and size, budget, seed, device) equal those of an earlier call of this thread
+// replays that call's graph: the same kernels on the same buffers, launched with one
+// cudaGraphLaunch instead of ~2000 stream launches (most of them inside cuSOLVER's batched
+// eigen solver and Cholesky).  The graph is captured on a private stream and launched on
+// the caller's; a call that cannot be captured runs directly.
+// ------------------------------------------------------------------------------------------
+struct GraphKey {
+  jolt_shape sh;
+  jolt_options op;
+  const void *k, *v;
+  uint64_t budget, seed;
+  void* blob;
+  size_t cap;
+  void* ws;
+  size_t ws_bytes;
+  int device;
+};
+struct GraphEntry {
+  GraphKey key;
+  cudaGraphExec_t exec = nullptr;
+  unsigned long long launches = 0;
+  unsigned long long last = 0;
+  bool failed = false;    // capture not possible for these arguments: run directly
+};
+constexpr size_t kMaxGraphs = 8;
+struct GraphCache {
+  std::vector<GraphEntry> e;
+  unsigned long long tick = 0;
+  cudaStream_t cap_stream = nullptr;
+  int cap_device = -1;
+  bool on = true;
+  ~GraphCache() {
+    for (auto& g : e)
+      if (g.exec) cudaGraphExecDestroy(g.exec);
+  }
+};
+thread_local GraphCache g_graphs;
+
+void graph_insert(GraphCache& gc, const GraphEntry& ent) {
+  if (gc.e.size() >= kMaxGraphs) {
+    size_t lru = 0;
+    for (size_t i = 1; i < gc.e.size(); ++i)
+      if (gc.e[i].last < gc.e[lru].last) lru = i;
+    if (gc.e[lru].exec) cudaGraphExecDestroy(gc.e[lru].exec);
+    gc.e.erase(gc.e.begin() + lru);
+  }
+  gc.e.push_back(ent);
+}
+
+// first call with a key: runs directly (so every lazily created library resource exists);
+// second call: captured and launched; later calls: replayed
+jolt_status compress_graph(const Ctx& c, const GraphKey& key, uint64_t budget_bytes, unsigned long long hdr,
+                           void* blob_dev, size_t blob_cap) {
+  GraphCache& gc = g_graphs;
+  ++gc.tick;
+  GraphEntry* hit = nullptr;
+  for (auto& g : gc.e)
+    if (memcmp(&g.key, &key, sizeof key) == 0) hit = &g;
+  if (!hit) {
+    GraphEntry ent;
+    ent.key = key;
+    ent.last = gc.tick;
+    graph_insert(gc, ent);
+    return compress_body(c, budget_bytes, hdr, blob_dev, blob_cap);
+  }
+  hit->last = gc.tick;
+  if (hit->failed) return compress_body(c, budget_bytes, hdr, blob_dev, blob_cap);
+  if (hit->exec) {
+    CUDA_TRY(cudaGraphLaunch(hit->exec, c.st));
+    launch_counter().fetch_add(hit->launches, std::memory_order_relaxed);
+    return JOLT_OK;
+  }
+  if (gc.cap_stream == nullptr || gc.cap_device != key.device) {
+    CUDA_TRY(cudaStreamCreateWithFlags(&gc.cap_stream, cudaStreamNonBlocking));
+    gc.cap_device = key.device;
+  }
+  // resources the body creates on first use exist already (the first call ran directly);
+  // capture the body on the private stream; the graph is launched on the caller's stream,
+  // which orders it after the caller's earlier work
+  Ctx cc = c;
+  cc.st = gc.cap_stream;
+  unsigned long long counted = 0;
+  cudaGraph_t graph = nullptr;
+  jolt_status st = JOLT_OK;
+  bool ok = false;
+  if (cudaStreamBeginCapture(gc.cap_stream, cudaStreamCaptureModeThreadLocal) == cudaSuccess) {
+    capture_counter() = &counted;
+    st = compress_body(cc, budget_bytes, hdr, blob_dev, blob_cap);
+    capture_counter() = nullptr;
+    const cudaError_t e = cudaStreamEndCapture(gc.cap_stream, &graph);
+    ok = st == JOLT_OK && e == cudaSuccess && graph && cudaGraphInstantiateWithFlags(&hit->exec, graph, 0) == cudaSuccess;
+    if (graph) cudaGraphDestroy(graph);
+  }
+  cudaGetLastError();   // a refused capture leaves no sticky error
+  if (!ok) {
+    hit->failed = true;
+    hit->exec = nullptr;
+    return compress_body(c, budget_bytes, hdr, blob_dev, blob_cap);
+  }
+  hit->launches = counted;
+  CUDA_TRY(cudaGraphLaunch(hit->exec, c.st));
+  launch_counter().fetch_add(hit->launches, std::memory_order_relaxed);
+  return JOLT_OK;
+}
+
 jolt_status jolt_compress(const jolt_shape* shape, const void* k_dev, const void* v_dev, const jolt_options* opts,
                           uint64_t budget_bytes, uint64_t seed, void* blob_dev, size_t blob_cap, void* ws_dev,
                           size_t ws_bytes, void* stream) {
@@ -1339,20 +1636,33 @@ jolt_status jolt_compress(const jolt_shape* shape, const void* k_dev, const void
   const unsigned long long hdr = 64ull + 64ull * p.NU;
   if (budget_bytes < hdr) return fail(JOLT_ERR_BUDGET_INFEASIBLE, "budget below the headers (%llu bytes)", hdr);
   Ctx c{p, (unsigned char*)ws_dev, (cudaStream_t)stream, k_dev, v_dev, seed};
-  float* Uf = c.at<float>(p.o_Uf);
-  float* Wf = c.at<float>(p.o_Wf);
-  bf16* Us = c.at<bf16>(p.o_Us);
-  bf16* Ws = c.at<bf16>(p.o_Ws);
-  JTRY(run_factor(c, Uf, p.ldU, Wf, p.ldW, Us, Ws));
-  bf16* core = c.at<bf16>(p.o_core);
-  double* table = c.at<double>(p.o_table);
-  JTRY(run_table(c, Us, p.ldU, Ws, p.ldW, core, table));
-  JTRY(run_allocate(c, table, budget_bytes - hdr, (unsigned char*)blob_dev, blob_cap, nullptr));
-  JTRY(run_encode(c, Us, p.ldU, Ws, p.ldW, core, (unsigned char*)blob_dev));
-  // device-side errors of the factor stage are folded into the header status
-  count_launch(), fold_status_kernel<<<1, 1, 0, c.st>>>(c.status(), (unsigned char*)blob_dev);
-  CUDA_TRY(cudaGetLastError());
-  return JOLT_OK;
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  CUDA_TRY(cudaStreamIsCapturing(c.st, &cs));
+  if (!g_graphs.on || g_prof.on || cs != cudaStreamCaptureStatusNone)
+    return compress_body(c, budget_bytes, hdr, blob_dev, blob_cap);
+  GraphKey key;
+  memset(&key, 0, sizeof key);
+  key.sh = *shape;
+  key.op = *opts;
+  key.k = k_dev;
+  key.v = v_dev;
+  key.budget = budget_bytes;
+  key.seed = seed;
+  key.blob = blob_dev;
+  key.cap = blob_cap;
+  key.ws = ws_dev;
+  key.ws_bytes = ws_bytes;
+  CUDA_TRY(cudaGetDevice(&key.device));
+  return compress_graph(c, key, budget_bytes, hdr, blob_dev, blob_cap);
+}
+
+void jolt_set_graphs(int32_t enable) {
+  g_graphs.on = enable != 0;
+  if (!g_graphs.on) {
+    for (auto& g : g_graphs.e)
+      if (g.exec) cudaGraphExecDestroy(g.exec);
+    g_graphs.e.clear();
+  }
 }
 
 jolt_status jolt_read_header(const void* blob_dev, jolt_shape* shape_out, uint64_t* total_bytes,
@@ -1379,6 +1689,7 @@ jolt_status jolt_read_header(const void* blob_dev, jolt_shape* shape_out, uint64
                              cudaMemcpyDeviceToHost, st));
     CUDA_TRY(cudaStreamSynchronize(st));
   }
+  if (h.status & DEV_ERR_TIMEOUT) return fail(JOLT_ERR_TIMEOUT, "a bounded device-side wait gave up");
   if (h.status & DEV_ERR_INFEASIBLE) return fail(JOLT_ERR_BUDGET_INFEASIBLE, "budget infeasible (device)");
   if (h.status & (DEV_ERR_NONFINITE | DEV_ERR_FACTOR))
     return fail(JOLT_ERR_NUMERIC, "non-finite input or factorisation breakdown (status %u)", h.status);

@@ -114,9 +114,11 @@ constexpr int TROWS = 64;
 constexpr int TTHREADS = 128;
 constexpr int KC = 64;  // token-rank chunk staged per pipeline step
 
-template <int D>
+// SPLIT = 2: two warps share a 16-row group, each holding half of the D columns (the table
+// kernel, which runs eight warps per 64-row tile to halve the registers a thread holds)
+template <int D, int SPLIT = 1>
 struct TileFrag {
-  static constexpr int NT = D / 8;
+  static constexpr int NT = D / 8 / SPLIT;
   float v[2][NT][2];
 };
 
@@ -142,15 +144,46 @@ __device__ __forceinline__ void rotate_tile_to_smem(const TX* X, int T, int t0, 
   }
 }
 
-template <int D>
-__device__ __forceinline__ void frag_from_smem(const float* xs, TileFrag<D>& f) {
+// the same rotation with the whole CTA working in shared memory: x * sigma staged, then the
+// Walsh-Hadamard butterflies stage by stage (the order of fwht_regs, so the result is
+// bit-identical), then the 1/sqrt(D) scale; keeps no row in registers
+template <int D, typename TX>
+__device__ __forceinline__ void rotate_tile_smem(const TX* X, int T, int t0, const float* sig, float* xs) {
+  constexpr int LD = D + 4;
+  for (int idx = threadIdx.x; idx < TROWS * D; idx += blockDim.x) {
+    const int r = idx / D, d = idx - r * D, t = t0 + r;
+    xs[r * LD + d] = t < T ? ld_as_float(X + (long long)t * D + d) * sig[d] : 0.f;
+  }
+  __syncthreads();
+#pragma unroll
+  for (int h = 1; h < D; h <<= 1) {
+    for (int idx = threadIdx.x; idx < TROWS * D / 2; idx += blockDim.x) {
+      const int r = idx / (D / 2), p = idx - r * (D / 2);
+      const int i = (p / h) * 2 * h + (p % h);
+      const float a = xs[r * LD + i], b = xs[r * LD + i + h];
+      xs[r * LD + i] = a + b;
+      xs[r * LD + i + h] = a - b;
+    }
+    __syncthreads();
+  }
+  const float sc = (float)(1.0 / sqrt((double)D));
+  for (int idx = threadIdx.x; idx < TROWS * D; idx += blockDim.x) {
+    const int r = idx / D, d = idx - r * D;
+    xs[r * LD + d] *= sc;
+  }
+}
+
+template <int D, int SPLIT = 1>
+__device__ __forceinline__ void frag_from_smem(const float* xs, TileFrag<D, SPLIT>& f) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  constexpr int NT = TileFrag<D, SPLIT>::NT;
+  const int rg = warp / SPLIT, half = warp % SPLIT;
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
-    int r = warp * 16 + (lane >> 2) + h * 8;
+    int r = rg * 16 + (lane >> 2) + h * 8;
 #pragma unroll
-    for (int j = 0; j < TileFrag<D>::NT; ++j) {
-      int c = j * 8 + (lane & 3) * 2;
+    for (int j = 0; j < NT; ++j) {
+      int c = (half * NT + j) * 8 + (lane & 3) * 2;
       f.v[h][j][0] = xs[r * (D + 4) + c];
       f.v[h][j][1] = xs[r * (D + 4) + c + 1];
     }
@@ -200,16 +233,17 @@ __device__ __forceinline__ void recon_load_stage(bf16* st, const bf16* U, long l
 
 // accumulate the k16 slab at chunk offset kk (absolute token rank kabs) of a staged chunk,
 // keeping only the ranks in [klo, khi)
-template <int D>
+template <int D, int SPLIT = 1>
 __device__ __forceinline__ void recon_mma_k16(const bf16* st, int kk, int kabs, int klo, int khi,
                                               float (*acc)[4]) {
   using namespace gemm_detail;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int rg = warp / SPLIT, half = warp % SPLIT;
   const bf16* sU = st;
   const bf16* sP = st + ReconSmem<D>::U_ELEMS;
   uint32_t a[4];
   {
-    int row = warp * 16 + (lane & 15);
+    int row = rg * 16 + (lane & 15);
     int ch = (kk >> 3) + (lane >> 4);
     ldsm_x4(smem_u32(sU + su_off(row, ch)), a[0], a[1], a[2], a[3]);
   }
@@ -225,12 +259,12 @@ __device__ __forceinline__ void recon_mma_k16(const bf16* st, int kk, int kabs, 
       a[r] &= m;
     }
   }
-  constexpr int NT = D / 8;
+  constexpr int NT = D / 8 / SPLIT;   // n8 tiles of this warp
 #pragma unroll
   for (int np = 0; np < NT / 2; ++np) {
     uint32_t r0, r1, r2, r3;
     int krow = kk + (lane & 7) + (((lane >> 3) & 1) << 3);
-    int ch = np * 2 + (lane >> 4);
+    int ch = (half * NT / 2 + np) * 2 + (lane >> 4);
     ldsm_x4_t(smem_u32(sP + sp_off<D>(krow, ch)), r0, r1, r2, r3);
     mma16816(acc[np * 2 + 0], a, r0, r1);
     mma16816(acc[np * 2 + 1], a, r2, r3);
@@ -239,7 +273,7 @@ __device__ __forceinline__ void recon_mma_k16(const bf16* st, int kk, int kabs, 
 
 // Walk the token-rank axis [0, kmax) in KC chunks; call epi(i) whenever the
 // accumulated prefix reaches cut[i] (cuts ascending, all <= kmax).
-template <int D, typename Epi>
+template <int D, int SPLIT = 1, typename Epi>
 __device__ __forceinline__ void recon_walk(bf16* smem_stages, const bf16* U, long long ldU, int T, int t0,
                                            const bf16* P, int kmax, const int* cuts, int ncuts,
                                            float (*acc)[4], Epi&& epi) {
@@ -263,7 +297,7 @@ __device__ __forceinline__ void recon_walk(bf16* smem_stages, const bf16* U, lon
       while (lo < k + 16 && lo < kmax) {
         int hi = min(k + 16, kmax);
         if (ci < ncuts && cuts[ci] > lo && cuts[ci] < hi) hi = cuts[ci];
-        recon_mma_k16<D>(st, kk, k, lo, hi, acc);
+        recon_mma_k16<D, SPLIT>(st, kk, k, lo, hi, acc);
         lo = hi;
         while (ci < ncuts && cuts[ci] == lo) { epi(ci); ++ci; }
       }
@@ -277,23 +311,26 @@ __device__ __forceinline__ void recon_walk(bf16* smem_stages, const bf16* U, lon
 // residual tile in shared memory: the fragment owners write rho = x' - acc, then every
 // thread quantises whole 16-wide blocks of one row (row = tid % 64, blocks of one half row)
 // ---------------------------------------------------------------------------------------
-template <int D>
+template <int D, int THREADS = TTHREADS>
 struct RhoTile {
   static constexpr int LD = D + 4;                 // row pitch (floats)
   static constexpr int BLK_PER_ROW = D / 16;
-  static constexpr int BLK_PER_THREAD = (TROWS * BLK_PER_ROW) / TTHREADS;  // 4 for D = 128
+  static constexpr int BLOCKS = TROWS * BLK_PER_ROW;
+  static constexpr int BLK_PER_THREAD = BLOCKS / THREADS;  // 4 for D = 128 and 128 threads
   static constexpr size_t BYTES = (size_t)TROWS * LD * 4;
 };
 
-template <int D>
-__device__ __forceinline__ void write_rho(float* rho, const TileFrag<D>& xf, float (*acc)[4]) {
+template <int D, int SPLIT = 1>
+__device__ __forceinline__ void write_rho(float* rho, const TileFrag<D, SPLIT>& xf, float (*acc)[4]) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int rg = warp / SPLIT, half = warp % SPLIT;
+  constexpr int NT = TileFrag<D, SPLIT>::NT;
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
-    const int r = warp * 16 + (lane >> 2) + h * 8;
+    const int r = rg * 16 + (lane >> 2) + h * 8;
 #pragma unroll
-    for (int j = 0; j < D / 8; ++j) {
-      const int c = j * 8 + (lane & 3) * 2;
+    for (int j = 0; j < NT; ++j) {
+      const int c = (half * NT + j) * 8 + (lane & 3) * 2;
       float2 v = make_float2(xf.v[h][j][0] - acc[j][h * 2 + 0], xf.v[h][j][1] - acc[j][h * 2 + 1]);
       *reinterpret_cast<float2*>(rho + r * RhoTile<D>::LD + c) = v;
     }
@@ -301,15 +338,22 @@ __device__ __forceinline__ void write_rho(float* rho, const TileFrag<D>& xf, flo
 }
 
 // blocks handled by this thread: row tid % 64, blocks [ (tid / 64) * BPT, +BPT ) of that row;
-// D = 16 has one block per row, held by the first 64 threads
-template <int D>
+// with fewer blocks than threads, thread tid < BLOCKS holds block tid / 64 of row tid % 64
+template <int D, int THREADS = TTHREADS>
 __device__ __forceinline__ int block_row() { return threadIdx.x % TROWS; }
-template <int D>
+template <int D, int THREADS = TTHREADS>
 __device__ __forceinline__ int block_first() {
-  return (RhoTile<D>::BLK_PER_THREAD > 0) ? (threadIdx.x / TROWS) * RhoTile<D>::BLK_PER_THREAD : 0;
+  constexpr int BPT = RhoTile<D, THREADS>::BLK_PER_THREAD;
+  return BPT > 0 ? (int)(threadIdx.x / TROWS) * BPT : (int)(threadIdx.x / TROWS);
 }
-template <int D>
-__host__ __device__ constexpr int blocks_per_thread() { return RhoTile<D>::BLK_PER_THREAD > 0 ? RhoTile<D>::BLK_PER_THREAD : 1; }
+template <int D, int THREADS = TTHREADS>
+__host__ __device__ constexpr int blocks_per_thread() {
+  return RhoTile<D, THREADS>::BLK_PER_THREAD > 0 ? RhoTile<D, THREADS>::BLK_PER_THREAD : 1;
+}
+template <int D, int THREADS = TTHREADS>
+__device__ __forceinline__ bool has_blocks() {
+  return RhoTile<D, THREADS>::BLK_PER_THREAD > 0 || (int)threadIdx.x < RhoTile<D, THREADS>::BLOCKS;
+}
 
 __device__ __forceinline__ void load16(const float* src, float* v) {
 #pragma unroll
@@ -350,22 +394,29 @@ __device__ __forceinline__ BitConsts bit_consts(const Cands& cd) {
   return k;
 }
 
-// squared quantisation error of one 16-wide block for every bit-width (added into err)
+// squared quantisation error of one 16-wide block for every bit-width (added into err).
+// The per-element work runs on packed fp32 pairs (FFMA2 / FADD2: the same IEEE round-to-
+// nearest per lane as the scalar forms, half the instructions) with four partial sums, so
+// the dependent accumulation chain is four deep instead of sixteen.
 __device__ __forceinline__ void block_errors(const float* v, const BitConsts& k, float* err) {
   float mn, mx;
   minmax16(v, mn, mx);
   const float lo = rd16(mn);
-  float d[16];
+  float2 d[8];
 #pragma unroll
-  for (int j = 0; j < 16; ++j) d[j] = v[j] - lo;
+  for (int j = 0; j < 8; ++j) d[j] = __fadd2_rn(make_float2(v[2 * j], v[2 * j + 1]), make_float2(-lo, -lo));
 #pragma unroll
   for (int ib = 0; ib < MAXC; ++ib) {
     if (ib >= k.n) break;
     if (k.bits[ib] == 0) {
-      float e0 = 0.f;
+      float2 a0 = make_float2(0.f, 0.f), a1 = a0;
 #pragma unroll
-      for (int j = 0; j < 16; ++j) e0 = fmaf(v[j], v[j], e0);
-      err[ib] += e0;
+      for (int j = 0; j < 8; j += 2) {
+        const float2 x0 = make_float2(v[2 * j], v[2 * j + 1]), x1 = make_float2(v[2 * j + 2], v[2 * j + 3]);
+        a0 = __ffma2_rn(x0, x0, a0);
+        a1 = __ffma2_rn(x1, x1, a1);
+      }
+      err[ib] += (a0.x + a0.y) + (a1.x + a1.y);
       continue;
     }
     const float step = quant_step(mx, lo, k.flev[ib], k.inv[ib]);
@@ -374,14 +425,20 @@ __device__ __forceinline__ void block_errors(const float* v, const BitConsts& k,
       continue;
     }
     const float inv = step > 0.f ? __frcp_rn(step) : 0.f;
-    float e2 = 0.f;
+    const float2 inv2 = make_float2(inv, inv), nstep2 = make_float2(-step, -step);
+    const float2 sh = make_float2(kRoundShift, kRoundShift), nsh = make_float2(-kRoundShift, -kRoundShift);
+    float2 a0 = make_float2(0.f, 0.f), a1 = a0;
 #pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      const float c = code_of(d[j], inv);
-      const float e = fmaf(-c, step, d[j]);
-      e2 = fmaf(e, e, e2);
+    for (int j = 0; j < 8; j += 2) {
+      // code = rne(d / step) through the shift, e = d - code * step, e2 += e * e
+      const float2 c0 = __fadd2_rn(__ffma2_rn(d[j], inv2, sh), nsh);
+      const float2 c1 = __fadd2_rn(__ffma2_rn(d[j + 1], inv2, sh), nsh);
+      const float2 e0 = __ffma2_rn(c0, nstep2, d[j]);
+      const float2 e1 = __ffma2_rn(c1, nstep2, d[j + 1]);
+      a0 = __ffma2_rn(e0, e0, a0);
+      a1 = __ffma2_rn(e1, e1, a1);
     }
-    err[ib] += e2;
+    err[ib] += (a0.x + a0.y) + (a1.x + a1.y);
   }
 }
 
@@ -406,13 +463,21 @@ inline size_t table_smem() {
   return RhoTile<D>::BYTES + 2 * (size_t)ReconSmem<D>::STAGE * sizeof(bf16);
 }
 
+// the table kernel runs 2 warps per 16-row group (each half of the columns) where D >= 32
+template <int D>
+__host__ __device__ constexpr int table_split() { return D >= 32 ? 2 : 1; }
+template <int D>
+__host__ __device__ constexpr int table_threads() { return TTHREADS * table_split<D>(); }
+
 template <int D, typename TX>
-__global__ void __launch_bounds__(TTHREADS) table_kernel(TableArgs a) {
+__global__ void __launch_bounds__(table_threads<D>(), D >= 64 ? 2 : 1) table_kernel(TableArgs a) {
+  constexpr int SPLIT = table_split<D>();
+  constexpr int THREADS = table_threads<D>();
   extern __shared__ __align__(128) unsigned char smem_raw[];
   float* rho = reinterpret_cast<float*>(smem_raw);                                   // TROWS x LD
   bf16* stages = reinterpret_cast<bf16*>(smem_raw + RhoTile<D>::BYTES);                // 2 stages
   __shared__ float sig[D];
-  __shared__ float red[TTHREADS / 32][MAXC];
+  __shared__ float red[THREADS / 32][MAXC];
 
   const int tile = blockIdx.x, s = blockIdx.y, u = blockIdx.z;
   const int T = a.cv.T;
@@ -420,20 +485,20 @@ __global__ void __launch_bounds__(TTHREADS) table_kernel(TableArgs a) {
   const TX* X = reinterpret_cast<const TX*>(a.cv.unit_ptr(u)) + (long long)s * T * D;
   for (int d = threadIdx.x; d < D; d += blockDim.x) sig[d] = rotation_sign(a.seed, u, d);
   __syncthreads();
-  rotate_tile_to_smem<D, TX>(X, T, t0, sig, rho);   // x' staged through the rho buffer
+  rotate_tile_smem<D, TX>(X, T, t0, sig, rho);   // x' staged through the rho buffer
   __syncthreads();
-  TileFrag<D> xf;
-  frag_from_smem<D>(rho, xf);
+  TileFrag<D, SPLIT> xf;
+  frag_from_smem<D, SPLIT>(rho, xf);
   __syncthreads();
 
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const Cands& cd = a.cand;
   const BitConsts kb = bit_consts(cd);
   const bf16* U = a.U + (long long)u * a.sU;
-  constexpr int NT = D / 8;
+  constexpr int NT = TileFrag<D, SPLIT>::NT;
   double* out = a.partial + (((long long)u * a.cv.S + s) * a.tiles + tile) * (long long)(cd.nD * cd.nT * cd.nB);
-  const int brow = block_row<D>();
-  const bool has_blocks = (RhoTile<D>::BLK_PER_THREAD > 0) || threadIdx.x < TROWS;
+  const int brow = block_row<D, THREADS>();
+  const bool mine = has_blocks<D, THREADS>();
 
   for (int iD = 0; iD < cd.nD; ++iD) {
     const bf16* P = a.P + (long long)u * a.sP_unit + iD * a.sP_rd + (long long)s * a.rTmax * D;
@@ -444,16 +509,16 @@ __global__ void __launch_bounds__(TTHREADS) table_kernel(TableArgs a) {
       for (int e = 0; e < 4; ++e) acc[j][e] = 0.f;
 
     auto epi = [&](int iT) {
-      write_rho<D>(rho, xf, acc);
+      write_rho<D, SPLIT>(rho, xf, acc);
       __syncthreads();
       float err[MAXC];
 #pragma unroll
       for (int ib = 0; ib < MAXC; ++ib) err[ib] = 0.f;
-      if (has_blocks) {
+      if (mine) {
 #pragma unroll 1
-        for (int q = 0; q < blocks_per_thread<D>(); ++q) {
+        for (int q = 0; q < blocks_per_thread<D, THREADS>(); ++q) {
           float v[16];
-          load16(rho + brow * RhoTile<D>::LD + (block_first<D>() + q) * 16, v);
+          load16(rho + brow * RhoTile<D>::LD + (block_first<D, THREADS>() + q) * 16, v);
           block_errors(v, kb, err);
         }
       }
@@ -469,11 +534,11 @@ __global__ void __launch_bounds__(TTHREADS) table_kernel(TableArgs a) {
       __syncthreads();
       if (threadIdx.x < cd.nB) {
         double v = 0.0;
-        for (int w = 0; w < TTHREADS / 32; ++w) v += (double)red[w][threadIdx.x];
+        for (int w = 0; w < THREADS / 32; ++w) v += (double)red[w][threadIdx.x];
         out[(iD * cd.nT + iT) * cd.nB + threadIdx.x] = v;
       }
     };
-    recon_walk<D>(stages, U, a.ldU, T, t0, P, cd.rT[cd.nT - 1], cd.rT, cd.nT, acc, epi);
+    recon_walk<D, SPLIT>(stages, U, a.ldU, T, t0, P, cd.rT[cd.nT - 1], cd.rT, cd.nT, acc, epi);
     __syncthreads();
   }
 }

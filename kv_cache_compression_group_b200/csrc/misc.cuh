@@ -35,7 +35,8 @@ __global__ void gram_diag_check_kernel(const double* G, int n, int nunits, uint3
 // from an ascending eigen-solver output (eigenvectors in columns, column-major, lda),
 // the entry of largest magnitude made positive (ties: lowest row).
 // Writes row-major n x ldo fp32 (optional), bf16 (optional) and the eigenvalues (optional).
-__global__ void eig_select_kernel(const double* vals, const double* vecs, int n, long long lda,
+// eigenvector i of matrix u is vecs[u * svec + i * lda + row * inc]
+__global__ void eig_select_kernel(const double* vals, const double* vecs, int n, long long lda, long long inc,
                                   long long sval, long long svec, int r, float* out_f32, bf16* out_bf16,
                                   long long ldo, long long sout, double* out_vals) {
   const int j = blockIdx.x, u = blockIdx.y;
@@ -62,7 +63,7 @@ __global__ void eig_select_kernel(const double* vals, const double* vecs, int n,
   double bv = -1.0;
   int bi = 0x7fffffff;
   for (int i = threadIdx.x; i < n; i += blockDim.x) {
-    double a = fabs(col[i]);
+    double a = fabs(col[i * inc]);
     if (a > bv || (a == bv && i < bi)) { bv = a; bi = i; }
   }
   bestv[threadIdx.x] = bv;
@@ -79,9 +80,9 @@ __global__ void eig_select_kernel(const double* vals, const double* vecs, int n,
     }
     __syncthreads();
   }
-  const double sgn = col[besti[0]] < 0 ? -1.0 : 1.0;
+  const double sgn = col[besti[0] * inc] < 0 ? -1.0 : 1.0;
   for (int i = threadIdx.x; i < n; i += blockDim.x) {
-    double v = sgn * col[i];
+    double v = sgn * col[i * inc];
     long long o = (long long)u * sout + (long long)i * ldo + j;
     if (out_f32) out_f32[o] = (float)v;
     if (out_bf16) out_bf16[o] = __float2bfloat16_rn((float)v);
@@ -226,99 +227,139 @@ __global__ void ptr_array_kernel(double** P, double* A, long long sA, int n) {
   if (u < n) P[u] = A + (long long)u * sA;
 }
 
-// lower-triangular L (column-major fp64, lda, stride sL) -> row-major fp32 [k][ld] (stride so),
-// zero above the diagonal
-__global__ void lower_to_rowmajor_kernel(const double* L, int k, long long lda, long long sL, float* out, long long ld,
-                                         long long so, int nbatch) {
-  const long long tot = (long long)nbatch * k * k;
-  for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < tot;
-       idx += (long long)gridDim.x * blockDim.x) {
-    const long long u = idx / ((long long)k * k), rem = idx - u * k * k;
-    const long long i = rem / k, j = rem - i * k;
-    out[u * so + i * ld + j] = j <= i ? (float)L[u * sL + j * lda + i] : 0.f;
+// ------------------------------------------------------------------------------------------
+// Q = Y L^{-T} in place (the triangular solve of Cholesky QR), blocked by 32 columns:
+//   Q[:, J] = (Y[:, J] - Q[:, :J] L[J, :J]^T) inv(L[J, J])^T
+// trsm_prep_kernel: per (block J, unit) one warp writes rows J of L as fp32 row-major (zeros
+//   above the diagonal) and inv(L_JJ) (fp64 forward substitution, rounded to fp32);
+// trsm_panel_kernel<RB>: one CTA per RB rows of one unit keeps its rows of Y in shared memory
+//   and solves them block column by block column (GEMM update from staged chunks of L, then
+//   the product with inv(L_JJ)^T), then writes the k solved columns back.
+// ------------------------------------------------------------------------------------------
+constexpr int TS_NB = 32;
+constexpr int TS_PC = 128;
+
+__global__ void trsm_prep_kernel(const double* L, int k, long long gld, long long sG, float* Lr, long long ldl,
+                                 long long sL, float* Dinv, long long sD) {
+  const int J = blockIdx.x, u = blockIdx.y, lane = threadIdx.x;
+  const int J0 = J * TS_NB, nb = min(TS_NB, k - J0);
+  const double* Lu = L + (long long)u * sG;   // column-major: (i, j) at Lu[j * gld + i]
+  float* Lru = Lr + (long long)u * sL;
+  for (int r = 0; r < nb; ++r) {
+    const int i = J0 + r;
+    for (int c = lane; c < k; c += 32) Lru[(long long)i * ldl + c] = c <= i ? (float)Lu[(long long)c * gld + i] : 0.f;
   }
+  double x[TS_NB];
+#pragma unroll
+  for (int r = 0; r < TS_NB; ++r) {
+    double v = (r == lane) ? 1.0 : 0.0;
+    if (r < nb && lane < nb) {
+#pragma unroll
+      for (int q = 0; q < r; ++q) v = fma(-Lu[(long long)(J0 + q) * gld + J0 + r], x[q], v);
+      x[r] = lane <= r ? v / Lu[(long long)(J0 + r) * gld + J0 + r] : 0.0;
+    } else {
+      x[r] = 0.0;
+    }
+  }
+  float* D = Dinv + (long long)u * sD + (long long)J * TS_NB * TS_NB;
+#pragma unroll
+  for (int r = 0; r < TS_NB; ++r) D[r * TS_NB + lane] = (float)x[r];
 }
 
-// X = L^{-1} for every unit (L: row-major fp32 lower [k][ld], X: row-major fp32 [k][ld], both
-// with unit stride sL), blocked by 32: block row I is X_II = inv(L_II) (one warp, forward
-// substitution per column) and, for every block column J < I (one warp each),
-// X_IJ = -X_II (sum_{J<=P<I} L_IP X_PJ).  Block rows go in order; one CTA per unit.
-constexpr int TRI_NB = 32;
-__global__ void __launch_bounds__(1024) trinv_blocked_kernel(const float* L, int k, long long ld, long long sL,
-                                                             float* X, uint32_t* status) {
-  extern __shared__ __align__(16) float tri_sm[];
-  float* Xd = tri_sm;                              // X_II, 32 x 33
-  float* acc_s = tri_sm + TRI_NB * (TRI_NB + 1);   // per warp 32 x 33
-  const int u = blockIdx.x;
-  const float* Lu = L + (long long)u * sL;
-  float* Xu = X + (long long)u * sL;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
-  const int nb = (k + TRI_NB - 1) / TRI_NB;
-  // zero the strict upper part once
-  for (long long idx = threadIdx.x; idx < (long long)k * k; idx += blockDim.x) {
-    const long long r = idx / k, cc = idx - r * k;
-    if (cc > r) Xu[r * ld + cc] = 0.f;
-  }
-  for (int I = 0; I < nb; ++I) {
-    const int i0 = I * TRI_NB, ni = min(TRI_NB, k - i0);
-    // 1. X_II by warp 0: lane j owns column j of the diagonal block
-    if (warp == 0) {
-      float x[TRI_NB];
-#pragma unroll
-      for (int r = 0; r < TRI_NB; ++r) {
-        float v = (r == lane) ? 1.f : 0.f;
-        if (r < ni) {
-          const float* Lr = Lu + (long long)(i0 + r) * ld + i0;
-#pragma unroll
-          for (int q = 0; q < r; ++q) v = fmaf(-Lr[q], x[q], v);
-          const float d = Lr[r];
-          if (!(d != 0.f)) raise_status(status, DEV_ERR_FACTOR);
-          x[r] = (lane <= r && lane < ni) ? v / d : 0.f;
-        } else {
-          x[r] = 0.f;
-        }
-      }
-#pragma unroll
-      for (int r = 0; r < TRI_NB; ++r) Xd[r * (TRI_NB + 1) + lane] = x[r];
-    }
-    __syncthreads();
-    if (warp == 0 && lane < ni)
-      for (int r = 0; r < ni; ++r) Xu[(long long)(i0 + r) * ld + i0 + lane] = Xd[r * (TRI_NB + 1) + lane];
-    // 2. off-diagonal blocks of block row I: warp w handles block columns J = w, w + nwarps, ...
-    for (int J = warp; J < I; J += nwarps) {
-      const int j0 = J * TRI_NB;
-      // acc[r][c] (lane = row r): sum_{P=J}^{I-1} L_IP X_PJ
-      float acc[TRI_NB];
-#pragma unroll
-      for (int c = 0; c < TRI_NB; ++c) acc[c] = 0.f;
-      if (lane < ni) {
-        const float* Lr = Lu + (long long)(i0 + lane) * ld;
-        for (int p = j0; p < i0; ++p) {
-          const float l = Lr[p];
-          const float* Xp = Xu + (long long)p * ld + j0;
-#pragma unroll
-          for (int c = 0; c < TRI_NB; ++c) acc[c] = fmaf(l, Xp[c], acc[c]);
-        }
-      }
-      float* as = acc_s + warp * TRI_NB * (TRI_NB + 1);
-#pragma unroll
-      for (int c = 0; c < TRI_NB; ++c) as[lane * (TRI_NB + 1) + c] = acc[c];
-      __syncwarp();
-      // X_IJ[r][c] = -sum_q X_II[r][q] acc[q][c]   (lane = column c)
-      const int nj = min(TRI_NB, k - j0);
-      for (int r = 0; r < ni; ++r) {
-        float v = 0.f;
-        for (int q = 0; q <= r; ++q) v = fmaf(Xd[r * (TRI_NB + 1) + q], as[q * (TRI_NB + 1) + lane], v);
-        if (lane < nj) Xu[(long long)(i0 + r) * ld + j0 + lane] = -v;
-      }
-      __syncwarp();
-    }
-    __syncthreads();
-  }
+// row pitches: multiples of 4 floats (16-byte vector loads) that are 4 mod 32, so the rows a
+// warp reads together fall on distinct banks
+__host__ __device__ inline int trsm_pitch(int k) { return (int)round_up(k, TS_NB) + 4; }
+constexpr int TS_LP = TS_PC + 4;
+inline size_t trsm_smem(int rb, int k) {
+  return ((size_t)rb * trsm_pitch(k) + (size_t)TS_NB * TS_LP + (size_t)TS_NB * (TS_NB + 1)) * sizeof(float);
 }
 
-inline size_t trinv_smem(int nthreads) {
-  return (size_t)(TRI_NB * (TRI_NB + 1)) * 4 * (1 + nthreads / 32);
+template <int RB>
+__global__ void __launch_bounds__(256) trsm_panel_kernel(float* Y, long long m, int k, long long ld, long long sY,
+                                                         const float* Lr, long long ldl, long long sL,
+                                                         const float* Dinv, long long sD) {
+  extern __shared__ __align__(16) float ts_sm[];
+  const int P = trsm_pitch(k), kq = P - 4;
+  float* panel = ts_sm;                        // RB x P
+  float* lch = panel + RB * P;                 // 32 x TS_LP
+  float* dv = lch + TS_NB * TS_LP;             // 32 x 33
+  const int u = blockIdx.y, tid = threadIdx.x;
+  const long long r0 = (long long)blockIdx.x * RB;
+  float* Yu = Y + (long long)u * sY;
+  const float* Lu = Lr + (long long)u * sL;
+  const float* Du = Dinv + (long long)u * sD;
+  for (int idx = tid; idx < RB * kq; idx += blockDim.x) {
+    const int r = idx / kq, c = idx - r * kq;
+    panel[r * P + c] = (r0 + r < m && c < k) ? Yu[(r0 + r) * ld + c] : 0.f;
+  }
+  __syncthreads();
+  constexpr int RI = RB / 32;
+  const int ty = tid >> 3, tx = tid & 7;
+  for (int J0 = 0; J0 < k; J0 += TS_NB) {
+    float acc[RI][4];
+#pragma unroll
+    for (int i = 0; i < RI; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) acc[i][j] = panel[(ty + 32 * i) * P + J0 + tx + 8 * j];
+    for (int p0 = 0; p0 < J0; p0 += TS_PC) {
+      const int pc = min(TS_PC, J0 - p0);
+      __syncthreads();
+      for (int idx = tid; idx < TS_NB * TS_PC; idx += blockDim.x) {
+        const int rr = idx / TS_PC, cc = idx - rr * TS_PC;
+        lch[rr * TS_LP + cc] = (cc < pc && J0 + rr < k) ? Lu[(long long)(J0 + rr) * ldl + p0 + cc] : 0.f;
+      }
+      __syncthreads();
+      // pc is a multiple of 4 (block columns of 32, chunks of 128): four p per vector load
+      for (int p = 0; p < pc; p += 4) {
+        float4 q[RI], l[4];
+#pragma unroll
+        for (int i = 0; i < RI; ++i) q[i] = *reinterpret_cast<const float4*>(panel + (ty + 32 * i) * P + p0 + p);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) l[j] = *reinterpret_cast<const float4*>(lch + (tx + 8 * j) * TS_LP + p);
+#pragma unroll
+        for (int i = 0; i < RI; ++i)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            float a = acc[i][j];
+            a = fmaf(-q[i].x, l[j].x, a);
+            a = fmaf(-q[i].y, l[j].y, a);
+            a = fmaf(-q[i].z, l[j].z, a);
+            a = fmaf(-q[i].w, l[j].w, a);
+            acc[i][j] = a;
+          }
+      }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int i = 0; i < RI; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) panel[(ty + 32 * i) * P + J0 + tx + 8 * j] = acc[i][j];
+    for (int idx = tid; idx < TS_NB * TS_NB; idx += blockDim.x)
+      dv[(idx / TS_NB) * (TS_NB + 1) + (idx % TS_NB)] = Du[(long long)(J0 / TS_NB) * TS_NB * TS_NB + idx];
+    __syncthreads();
+    float out[RI][4];
+#pragma unroll
+    for (int i = 0; i < RI; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float* row = panel + (ty + 32 * i) * P + J0;
+        const float* dr = dv + (tx + 8 * j) * (TS_NB + 1);
+        float s = 0.f;
+#pragma unroll
+        for (int q = 0; q < TS_NB; ++q) s = fmaf(row[q], dr[q], s);
+        out[i][j] = s;
+      }
+    __syncthreads();
+#pragma unroll
+    for (int i = 0; i < RI; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) panel[(ty + 32 * i) * P + J0 + tx + 8 * j] = out[i][j];
+    __syncthreads();
+  }
+  for (int idx = tid; idx < RB * kq; idx += blockDim.x) {
+    const int r = idx / kq, c = idx - r * kq;
+    if (r0 + r < m && c < k) Yu[(r0 + r) * ld + c] = panel[r * P + c];
+  }
 }
 
 __global__ void info_check_kernel(const int* info, int n, uint32_t* status, uint32_t bits) {

@@ -28,7 +28,7 @@ EXPORTED = [
     "jolt_version", "jolt_last_error", "jolt_workspace_size", "jolt_counts", "jolt_choice_bytes",
     "jolt_compress", "jolt_factor", "jolt_table", "jolt_allocate", "jolt_encode", "jolt_read_header",
     "jolt_decompress", "jolt_frobenius", "jolt_profile_begin", "jolt_profile_end", "jolt_recon_operator",
-    "jolt_launch_count", "jolt_frobenius_noalloc",
+    "jolt_launch_count", "jolt_frobenius_noalloc", "jolt_set_graphs",
 ]
 
 
@@ -92,6 +92,8 @@ def lib():
         }
         L.jolt_launch_count.argtypes = []
         L.jolt_launch_count.restype = ctypes.c_uint64
+        L.jolt_set_graphs.argtypes = [i32]
+        L.jolt_set_graphs.restype = None
         for name, args in sigs.items():
             f = getattr(L, name)
             f.argtypes = args
@@ -346,6 +348,11 @@ def frobenius(K, V, K_hat=None, V_hat=None, layers_per_group=1, stream=None):
 def launch_count() -> int:
     """Kernels launched by the library in this process so far."""
     return int(lib().jolt_launch_count())
+
+
+def set_graphs(enable: bool):
+    """CUDA graphs of repeated compress calls on this thread (on by default)."""
+    lib().jolt_set_graphs(1 if enable else 0)
 
 
 def profile_begin():

@@ -60,7 +60,9 @@ def check_codes(g, rho, xr, b):
     bounded per block by w = 2^-17 (max |x'| + max |x_hat|).  A differing scale must be the
     rounding of a block minimum / maximum inside that window; codes are compared under the
     library's own scales and may differ only where the oracle's scaled value lies within
-    w / step of a rounding tie.  Returns (n_scales, n_scale_bad, n_codes, n_code_bad)."""
+    w / step of a rounding tie.  Returns (n_scales, n_scale_bad, n_codes, n_code_bad); a
+    differing scale is only possible in a block whose window straddles an fp16 rounding
+    boundary, and their number is asserted not to exceed the number of such blocks."""
     codes, lo, step, _, _ = O.quantize(rho, b)
     codes, lo, step = codes.reshape(-1, 16), lo.reshape(-1), step.reshape(-1)
     rb = rho.reshape(-1, 16)
@@ -68,6 +70,12 @@ def check_codes(g, rho, xr, b):
     win = 2.0 ** -17 * (np.abs(xr).max(1) + np.abs(xr - rb).max(1))
     same = (g["lo"] == lo) & (g["step"] == step)
     bad = np.nonzero(~same)[0]
+    # blocks whose window straddles an fp16 rounding boundary of lo or of step
+    L = (1 << b) - 1
+    mn_all, mx_all = rb.min(1), rb.max(1)
+    st_lo_all = O.fp16_rd(mn_all - win) != O.fp16_rd(mn_all + win)
+    st_st_all = O.fp16_ru(np.maximum(mx_all - win - lo, 0) / L) != O.fp16_ru((mx_all + win - lo) / L)
+    n_straddle = int(np.count_nonzero(st_lo_all | st_st_all))
     if bad.size:
         L = (1 << b) - 1
         mn, mx, wb = rb[bad].min(1), rb[bad].max(1), win[bad]
@@ -76,6 +84,7 @@ def check_codes(g, rho, xr, b):
         st_hi = O.fp16_ru((mx + wb - g["lo"][bad]) / L)
         st_ok = (g["step"][bad] >= st_lo) & (g["step"][bad] <= st_hi)
         assert np.all(lo_ok & st_ok), bad[~(lo_ok & st_ok)][:5]
+    assert bad.size <= n_straddle, (bad.size, n_straddle)
     gl, gs = g["lo"][:, None], g["step"][:, None]
     q = (rb - gl) / np.where(gs > 0, gs, 1.0)
     want = np.where(gs > 0, np.clip(np.rint(q), 0, (1 << b) - 1), 0)
