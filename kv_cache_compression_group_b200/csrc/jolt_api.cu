@@ -14,6 +14,8 @@
 #include "kernels.cuh"
 #include "misc.cuh"
 #include "umma.cuh"
+#include "eig_cluster.cuh"
+#include "chol_cluster.cuh"
 
 using namespace jolt;
 
@@ -167,7 +169,7 @@ struct Plan {
   size_t solver_host;
   // workspace offsets (bytes)
   size_t o_status, o_gd_part, o_gd, o_evals, o_Wf, o_Ws, o_Uf, o_Us, o_core, o_zc, o_ptmp, o_P, o_partial,
-      o_table, o_bytes, o_choice, o_lambda, o_hdr, o_umap, o_info, o_solver, o_fsolver, o_finfo, o_fevals;
+      o_table, o_bytes, o_choice, o_lambda, o_hdr, o_umap, o_info, o_solver, o_fsolver, o_finfo, o_fevals, o_eigvec, o_eigscr;
   // token factor scratch (all units)
   size_t o_gt32, o_gt, o_vsel, o_lam, o_omega, o_Y, o_Zm, o_h, o_l, o_gpart, o_G, o_ptrs, o_Lr, o_Linv;
   int qr_split_max;       // split-K of the Cholesky-QR Grams
@@ -329,7 +331,7 @@ jolt_status make_plan(const jolt_shape* sh, const jolt_options* op, Plan* p) {
   p->o_fevals = b.take((size_t)NU * D * 8 + 256);
   // token factor scratch
   p->o_gt32 = p->o_gt = p->o_vsel = p->o_lam = p->o_omega = 0;
-  p->o_Y = p->o_Zm = p->o_h = p->o_l = p->o_gpart = p->o_G = p->o_ptrs = 0;
+  p->o_Y = p->o_Zm = p->o_h = p->o_l = p->o_gpart = p->o_G = p->o_ptrs = p->o_eigvec = p->o_eigscr = 0;
   const int kq = op->method == JOLT_RANDOMIZED ? p->kp : p->ldU;   // width of the QR'ed blocks
   if (op->method == JOLT_EXACT) {
     long long n = p->m_side ? M : T;
@@ -350,6 +352,10 @@ jolt_status make_plan(const jolt_shape* sh, const jolt_options* op, Plan* p) {
     p->o_h = b.take((size_t)NU * big * kp * 2);
     p->o_l = b.take((size_t)NU * big * kp * 2);
     p->o_vsel = b.take((size_t)NU * kp * p->ldU * 4);
+    if (p->k >= 2 && p->k <= eigc::MAXN) {
+      p->o_eigvec = b.take((size_t)NU * p->k * p->k * 8);
+      p->o_eigscr = b.take((size_t)NU * eigc::scratch_doubles(p->k) * 8);
+    }
   }
   p->o_Lr = p->o_Linv = 0;
   if (op->method == JOLT_RANDOMIZED || p->m_side) {
@@ -496,6 +502,21 @@ jolt_status sym_eig_batched(const Ctx& c, double* A, int64_t n, double* w, int64
 jolt_status sym_eig_top(const Ctx& c, double* S, int n, int nbatch, int r, float* out_f32, bf16* out_bf16,
                         long long ldo, long long sout, double* out_vals) {
   double* w = c.at<double>(c.side ? c.p.o_fevals : c.p.o_evals);
+  if (c.p.o_eigscr && n == c.p.k && n >= 2 && n <= eigc::MAXN) {
+    // the Rayleigh-Ritz problem: one 8-CTA cluster per matrix
+    ProfScope ps("sym_eig", c.st, nbatch);
+    double* V = c.at<double>(c.p.o_eigvec);
+    double* scr = c.at<double>(c.p.o_eigscr);
+    const size_t sm = eigc::smem_bytes();
+    CUDA_TRY(cudaFuncSetAttribute(sym_eig_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm));
+    count_launch(), sym_eig_cluster_kernel<<<(unsigned)(nbatch * eigc::CL), eigc::THREADS, sm, c.st>>>(
+        S, n, (long long)n * n, w, n, V, scr, c.status());
+    CUDA_TRY(cudaGetLastError());
+    count_launch(), eig_select_kernel<<<dim3(r, nbatch), 256, 0, c.st>>>(w, V, n, 1, n, n, (long long)n * n, r,
+                                                                         out_f32, out_bf16, ldo, sout, out_vals);
+    CUDA_TRY(cudaGetLastError());
+    return JOLT_OK;
+  }
   JTRY(sym_eig_batched(c, S, n, w, nbatch));
   count_launch(), eig_select_kernel<<<dim3(r, nbatch), 256, 0, c.st>>>(w, S, n, n, 1, n, (long long)n * n, r, out_f32,
                                                                        out_bf16, ldo, sout, out_vals);
@@ -553,20 +574,30 @@ jolt_status cholqr_batched(const Ctx& c, float* Y, long long m, int k, int ld, i
     const long long n = (long long)k * gld;
     count_launch(), reduce_splits_kernel<float><<<grid1d((long long)p.NU * n), 256, 0, c.st>>>(gpart, G, p.NU, ns, n);
     count_launch(), sanitize_sym_batched_kernel<<<p.NU, 1024, 0, c.st>>>(G, k, gld, n, c.status());
-    count_launch(), ptr_array_kernel<<<1, 64, 0, c.st>>>(ptrs, G, n, p.NU);
     CUDA_TRY(cudaGetLastError());
-    ProfScope ps2("qr_potrf", c.st, p.NU);
-    SOLVER_TRY(cusolverDnDpotrfBatched(s->h, CUBLAS_FILL_MODE_LOWER, k, ptrs, gld, info, p.NU));
-    count_launch(), info_check_kernel<<<(unsigned)ceil_div(p.NU, 32), 32, 0, c.st>>>(info, p.NU, c.status(),
-                                                                                      DEV_ERR_FACTOR);
-    CUDA_TRY(cudaGetLastError());
-    ProfScope ps3("qr_trsm", c.st, p.NU);
     float* Lr = c.at<float>(p.o_Lr);
     float* Dinv = c.at<float>(p.o_Linv);
     const int nbk = (int)ceil_div(k, TS_NB);
     const long long sL = (long long)k * gld, sD = (long long)nbk * TS_NB * TS_NB;
-    count_launch(), trsm_prep_kernel<<<dim3(nbk, p.NU), 32, 0, c.st>>>(G, k, gld, n, Lr, gld, sL, Dinv, sD);
-    CUDA_TRY(cudaGetLastError());
+    if (k <= cholc::MAXN) {
+      // L (fp32) and the inverses of its diagonal blocks: one 8-CTA cluster per unit
+      ProfScope ps2("qr_potrf", c.st, p.NU);
+      const size_t sm = cholc::smem_bytes();
+      CUDA_TRY(cudaFuncSetAttribute(chol_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm));
+      count_launch(), chol_cluster_kernel<<<(unsigned)(p.NU * cholc::CL), cholc::THREADS, sm, c.st>>>(
+          G, k, gld, n, Lr, gld, sL, Dinv, sD, c.status());
+      CUDA_TRY(cudaGetLastError());
+    } else {
+      count_launch(), ptr_array_kernel<<<1, 64, 0, c.st>>>(ptrs, G, n, p.NU);
+      CUDA_TRY(cudaGetLastError());
+      ProfScope ps2("qr_potrf", c.st, p.NU);
+      SOLVER_TRY(cusolverDnDpotrfBatched(s->h, CUBLAS_FILL_MODE_LOWER, k, ptrs, gld, info, p.NU));
+      count_launch(), info_check_kernel<<<(unsigned)ceil_div(p.NU, 32), 32, 0, c.st>>>(info, p.NU, c.status(),
+                                                                                        DEV_ERR_FACTOR);
+      count_launch(), trsm_prep_kernel<<<dim3(nbk, p.NU), 32, 0, c.st>>>(G, k, gld, n, Lr, gld, sL, Dinv, sD);
+      CUDA_TRY(cudaGetLastError());
+    }
+    ProfScope ps3("qr_trsm", c.st, p.NU);
     if (k <= 512) JTRY(launch_trsm_panel<64>(c, Y, m, k, ld, Lr, gld, sL, Dinv, sD));
     else JTRY(launch_trsm_panel<32>(c, Y, m, k, ld, Lr, gld, sL, Dinv, sD));
   }
@@ -1050,7 +1081,14 @@ jolt_status run_core(const Ctx& c, const bf16* Us, long long ldU, const bf16* Ws
 template <int D>
 void launch_rotate_rows(const float* in, bf16* out, long long nrows, long long rows_per_unit, const int* umap,
                         uint64_t seed, cudaStream_t st) {
-  count_launch(), rotate_rows_kernel<D><<<(unsigned)ceil_div(nrows, 64), 64, 0, st>>>(in, out, nrows, rows_per_unit, umap, seed);
+  if constexpr (D >= 32) {
+    const long long blocks = ceil_div(nrows, 8) < 148 * 16 ? ceil_div(nrows, 8) : 148 * 16;   // 8 warps per block
+    count_launch(), rotate_rows_warp_kernel<D><<<(unsigned)blocks, 256, 0, st>>>(in, out, nrows, rows_per_unit, umap,
+                                                                               seed);
+  } else {
+    count_launch(), rotate_rows_kernel<D><<<(unsigned)ceil_div(nrows, 64), 64, 0, st>>>(in, out, nrows, rows_per_unit,
+                                                                                      umap, seed);
+  }
 }
 
 jolt_status rotate_rows(const Ctx& c, const float* in, bf16* out, long long nrows, long long rows_per_unit,

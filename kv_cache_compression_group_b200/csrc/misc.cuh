@@ -170,6 +170,66 @@ __global__ void rotate_rows_kernel(const float* in, bf16* out, long long nrows, 
   for (int d = 0; d < D; ++d) o[d] = __float2bfloat16_rn(v[d] * sc);
 }
 
+// The same rotation with one warp per row (D >= 32): lane l holds the E = D/32 consecutive
+// elements [l E, l E + E), so loads and stores are coalesced; the Walsh-Hadamard stages of
+// stride < E run inside the thread, the others across lanes (shfl_xor); each output is the
+// same sum or difference of the same two values as in fwht_regs, so the result is bitwise
+// the same.  The signs of a unit are recomputed only when a warp's row changes unit.
+template <int D>
+__global__ void rotate_rows_warp_kernel(const float* in, bf16* out, long long nrows, long long rows_per_unit,
+                                        const int* unit_of_batch, uint64_t seed) {
+  constexpr int E = D / 32;
+  const int lane = threadIdx.x & 31;
+  const long long warp0 = (blockIdx.x * (long long)blockDim.x + threadIdx.x) >> 5;
+  const long long nwarps = ((long long)gridDim.x * blockDim.x) >> 5;
+  const float sc = (float)(1.0 / sqrt((double)D));
+  int ucur = -1;
+  float sg[E];
+  for (long long r = warp0; r < nrows; r += nwarps) {
+    const int u = unit_of_batch[r / rows_per_unit];
+    if (u != ucur) {
+#pragma unroll
+      for (int e = 0; e < E; ++e) sg[e] = rotation_sign(seed, u, lane * E + e);
+      ucur = u;
+    }
+    float v[E];
+    const float* row = in + r * D + lane * E;
+    if (E == 4) {
+      const float4 t = *reinterpret_cast<const float4*>(row);
+      v[0] = t.x;
+      v[E > 1 ? 1 : 0] = t.y;
+      v[E > 2 ? 2 : 0] = t.z;
+      v[E > 3 ? 3 : 0] = t.w;
+    } else {
+#pragma unroll
+      for (int e = 0; e < E; ++e) v[e] = row[e];
+    }
+#pragma unroll
+    for (int e = 0; e < E; ++e) v[e] *= sg[e];
+#pragma unroll
+    for (int h = 1; h < E; h <<= 1)
+#pragma unroll
+      for (int e = 0; e < E; ++e)
+        if (!(e & h)) {
+          const float a = v[e], b = v[e + h];
+          v[e] = a + b;
+          v[e + h] = a - b;
+        }
+#pragma unroll
+    for (int hl = 1; hl < 32; hl <<= 1) {
+      const bool upper = (lane & hl) != 0;
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        const float mine = v[e], other = __shfl_xor_sync(0xffffffffu, mine, hl);
+        v[e] = upper ? other - mine : mine + other;
+      }
+    }
+    bf16* o = out + r * D + lane * E;
+#pragma unroll
+    for (int e = 0; e < E; ++e) o[e] = __float2bfloat16_rn(v[e] * sc);
+  }
+}
+
 // zero the strict upper triangle of column-major n x n matrices (lda)
 __global__ void tril_zero_kernel(double* A, int n, long long lda, long long sA, int nbatch) {
   long long total = (long long)nbatch * n * n;
