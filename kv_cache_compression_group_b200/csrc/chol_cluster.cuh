@@ -1,15 +1,15 @@
 // Cholesky factor G = L L^T of one symmetric positive definite n x n fp64 matrix
 // (n <= 256) per thread-block cluster of 8 CTAs, for the orthonormalisation step of
 // Cholesky QR.  CTA q keeps columns [32q, 32q + 32) of G in its shared memory.  Panel step
-// J (J = 0 .. 7): CTA J factors its 32 columns (one column after another inside the CTA)
-// and writes the finished panel into the shared memory of every CTA to its right
+// J (J = 0 .. 7): CTA J factors its 32 columns (the diagonal block by one warp, the rows
+// below by a triangular solve per row) and writes the finished panel into the shared memory of every CTA to its right
 // (distributed shared memory; two panel buffers alternate), one cluster barrier, then every
 // CTA to the right subtracts the panel's rank-32 update from its own columns.  At the end
 // every CTA writes its columns of L as fp32 (row-major, zeros above the diagonal) and the
 // inverse of its 32 x 32 diagonal block (fp64 forward substitution, rounded to fp32): the
 // operands of the row-panel triangular solve.  A non-positive or non-finite pivot raises
-// DEV_ERR_FACTOR (the pivot is replaced by 1 so the cluster finishes).  Every thread of
-// every CTA passes the same sequence of cluster barriers.
+// DEV_ERR_FACTOR (the pivot is replaced by 1 so the cluster finishes), a non-finite entry
+// DEV_ERR_NONFINITE.  Every thread of every CTA passes the same sequence of cluster barriers.
 #pragma once
 
 #include <cooperative_groups.h>
@@ -49,36 +49,62 @@ __global__ void __cluster_dims__(cholc::CL, 1, 1) __launch_bounds__(cholc::THREA
   const int c0 = q * NC;
   const int nblk = (n + NC - 1) / NC;
 
+  bool bad = false;
   for (int idx = tid; idx < MAXN * NC; idx += blockDim.x) {
     const int r = idx / NC, lc = idx - r * NC, c = c0 + lc;
-    As[r * LD + lc] = (r < n && c < n && r >= c) ? Gu[(long long)c * gld + r] : 0.0;
+    const double a = (r < n && c < n && r >= c) ? Gu[(long long)c * gld + r] : 0.0;
+    if (!isfinite(a)) bad = true;
+    As[r * LD + lc] = a;
   }
+  if (bad) raise_status(status, DEV_ERR_NONFINITE);
   __syncthreads();
 
   for (int J = 0; J < CL; ++J) {
     const int buf = J & 1;
     if (q == J && J < nblk) {
-      // factor my 32 columns
+      // factor my 32 columns: the 32 x 32 diagonal block by warp 0 (lane = row), then every
+      // row below solves x L_JJ^T = a (one thread per row)
       const int nb = min(NC, n - c0);
-      for (int jj = 0; jj < nb; ++jj) {
-        const int c = c0 + jj;
-        double d = As[c * LD + jj];
-        if (!(d > 0.0) || !isfinite(d)) {
-          if (tid == 0) raise_status(status, DEV_ERR_FACTOR);
-          d = 1.0;
+      if (tid < 32) {
+        const int lane = tid;
+        for (int jj = 0; jj < nb; ++jj) {
+          double d = As[(c0 + jj) * LD + jj];
+          if (!(d > 0.0) || !isfinite(d)) {
+            if (lane == 0) raise_status(status, DEV_ERR_FACTOR);
+            d = 1.0;
+          }
+          d = sqrt(d);
+          __syncwarp();
+          if (lane == jj) As[(c0 + jj) * LD + jj] = d;
+          if (lane > jj && lane < nb) As[(c0 + lane) * LD + jj] /= d;
+          __syncwarp();
+          if (lane > jj && lane < nb) {
+            const double lij = As[(c0 + lane) * LD + jj];
+            for (int p = jj + 1; p <= lane; ++p)
+              As[(c0 + lane) * LD + p] = fma(-lij, As[(c0 + p) * LD + jj], As[(c0 + lane) * LD + p]);
+          }
+          __syncwarp();
         }
-        d = sqrt(d);
-        __syncthreads();
-        for (int r = c + 1 + tid; r < n; r += blockDim.x) As[r * LD + jj] /= d;
-        if (tid == 0) As[c * LD + jj] = d;
-        __syncthreads();
-        // the later columns of the panel: A[r][c'] -= L[r][c] L[c'][c] for r >= c'
-        for (int idx = tid; idx < (n - c - 1) * (nb - jj - 1); idx += blockDim.x) {
-          const int r = c + 1 + idx / (nb - jj - 1), lc2 = jj + 1 + idx % (nb - jj - 1);
-          if (r >= c0 + lc2) As[r * LD + lc2] = fma(-As[r * LD + jj], As[(c0 + lc2) * LD + jj], As[r * LD + lc2]);
-        }
-        __syncthreads();
       }
+      __syncthreads();
+      for (int r = c0 + nb + tid; r < n; r += blockDim.x) {
+        double x[NC];
+#pragma unroll
+        for (int jj = 0; jj < NC; ++jj) x[jj] = jj < nb ? As[r * LD + jj] : 0.0;
+#pragma unroll
+        for (int jj = 0; jj < NC; ++jj) {
+          if (jj < nb) {
+            double v = x[jj];
+#pragma unroll
+            for (int p = 0; p < jj; ++p) v = fma(-x[p], As[(c0 + jj) * LD + p], v);
+            x[jj] = v / As[(c0 + jj) * LD + jj];
+          }
+        }
+#pragma unroll
+        for (int jj = 0; jj < NC; ++jj)
+          if (jj < nb) As[r * LD + jj] = x[jj];
+      }
+      __syncthreads();
       // the finished panel to every CTA on my right
       for (int t = q + 1; t < CL; ++t) {
         double* dst = cluster.map_shared_rank(pb, t) + buf * MAXN * LD;

@@ -573,8 +573,6 @@ jolt_status cholqr_batched(const Ctx& c, float* Y, long long m, int k, int ld, i
     JTRY(gemm(g, 1, 1, c.st));
     const long long n = (long long)k * gld;
     count_launch(), reduce_splits_kernel<float><<<grid1d((long long)p.NU * n), 256, 0, c.st>>>(gpart, G, p.NU, ns, n);
-    count_launch(), sanitize_sym_batched_kernel<<<p.NU, 1024, 0, c.st>>>(G, k, gld, n, c.status());
-    CUDA_TRY(cudaGetLastError());
     float* Lr = c.at<float>(p.o_Lr);
     float* Dinv = c.at<float>(p.o_Linv);
     const int nbk = (int)ceil_div(k, TS_NB);
@@ -588,6 +586,7 @@ jolt_status cholqr_batched(const Ctx& c, float* Y, long long m, int k, int ld, i
           G, k, gld, n, Lr, gld, sL, Dinv, sD, c.status());
       CUDA_TRY(cudaGetLastError());
     } else {
+      count_launch(), sanitize_sym_batched_kernel<<<p.NU, 1024, 0, c.st>>>(G, k, gld, n, c.status());
       count_launch(), ptr_array_kernel<<<1, 64, 0, c.st>>>(ptrs, G, n, p.NU);
       CUDA_TRY(cudaGetLastError());
       ProfScope ps2("qr_potrf", c.st, p.NU);
@@ -598,7 +597,10 @@ jolt_status cholqr_batched(const Ctx& c, float* Y, long long m, int k, int ld, i
       CUDA_TRY(cudaGetLastError());
     }
     ProfScope ps3("qr_trsm", c.st, p.NU);
-    if (k <= 512) JTRY(launch_trsm_panel<64>(c, Y, m, k, ld, Lr, gld, sL, Dinv, sD));
+    // rows per CTA: 128 (4 rows x 4 columns per thread) when the panel fits and there are
+    // enough rows to fill the GPU, else 64, else 32 for wide blocks
+    if (k <= 256 && m * p.NU >= 128LL * 148 * 2) JTRY(launch_trsm_panel<128>(c, Y, m, k, ld, Lr, gld, sL, Dinv, sD));
+    else if (k <= 512) JTRY(launch_trsm_panel<64>(c, Y, m, k, ld, Lr, gld, sL, Dinv, sD));
     else JTRY(launch_trsm_panel<32>(c, Y, m, k, ld, Lr, gld, sL, Dinv, sD));
   }
   return JOLT_OK;
@@ -1163,13 +1165,22 @@ jolt_status fill_umap(const Ctx& c, int* umap, int n) {
   return JOLT_OK;
 }
 
-template <int D, typename TX>
-jolt_status launch_table_T(const Ctx& c, const TableArgs& a) {
+template <int D, typename TX, typename BITS>
+jolt_status launch_table_B(const Ctx& c, const TableArgs& a) {
   size_t sm = table_smem<D>();
-  CUDA_TRY(cudaFuncSetAttribute(table_kernel<D, TX>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm));
-  count_launch(), table_kernel<D, TX><<<dim3(c.p.tiles, c.p.S, c.p.NU), table_threads<D>(), sm, c.st>>>(a);
+  CUDA_TRY(cudaFuncSetAttribute(table_kernel<D, TX, BITS>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm));
+  count_launch(), table_kernel<D, TX, BITS><<<dim3(c.p.tiles, c.p.S, c.p.NU), table_threads<D>(), sm, c.st>>>(a);
   CUDA_TRY(cudaGetLastError());
   return JOLT_OK;
+}
+
+// the default bit-width set {0,1,2,3,4,8} has its own instantiation (constants folded)
+template <int D, typename TX>
+jolt_status launch_table_T(const Ctx& c, const TableArgs& a) {
+  const Cands& cd = c.p.cd;
+  const bool dflt = cd.nB == 6 && cd.bits[0] == 0 && cd.bits[1] == 1 && cd.bits[2] == 2 && cd.bits[3] == 3 &&
+                    cd.bits[4] == 4 && cd.bits[5] == 8;
+  return dflt ? launch_table_B<D, TX, DefaultBits>(c, a) : launch_table_B<D, TX, void>(c, a);
 }
 
 template <int D>

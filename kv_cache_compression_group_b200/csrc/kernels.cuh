@@ -7,6 +7,8 @@
 // is then a subtraction, a 16-wide block min/max and the quantiser for every bit-width.
 #pragma once
 
+#include <type_traits>
+
 #include "common.cuh"
 #include "gemm.cuh"
 
@@ -442,6 +444,63 @@ __device__ __forceinline__ void block_errors(const float* v, const BitConsts& k,
   }
 }
 
+// The same errors for a bit-width set fixed at compile time (the default candidate set
+// {0,1,2,3,4,8}): the per-width constants fold into the code and the loop over widths is
+// unrolled without branches; the arithmetic of every width is the same as above.
+template <int B>
+__device__ __forceinline__ void bit_error(const float* v, const float2* d, float mx, float lo, float& err) {
+  if constexpr (B == 0) {
+    float2 a0 = make_float2(0.f, 0.f), a1 = a0;
+#pragma unroll
+    for (int j = 0; j < 8; j += 2) {
+      const float2 x0 = make_float2(v[2 * j], v[2 * j + 1]), x1 = make_float2(v[2 * j + 2], v[2 * j + 3]);
+      a0 = __ffma2_rn(x0, x0, a0);
+      a1 = __ffma2_rn(x1, x1, a1);
+    }
+    err += (a0.x + a0.y) + (a1.x + a1.y);
+  } else {
+    constexpr float flev = (float)((1 << B) - 1);
+    const float inv_lev = 1.0f / flev;
+    const float step = quant_step(mx, lo, flev, inv_lev);
+    if (!(isfinite(lo) && step <= kFp16Max)) {
+      err = INFINITY;
+      return;
+    }
+    const float inv = step > 0.f ? __frcp_rn(step) : 0.f;
+    const float2 inv2 = make_float2(inv, inv), nstep2 = make_float2(-step, -step);
+    const float2 sh = make_float2(kRoundShift, kRoundShift), nsh = make_float2(-kRoundShift, -kRoundShift);
+    float2 a0 = make_float2(0.f, 0.f), a1 = a0;
+#pragma unroll
+    for (int j = 0; j < 8; j += 2) {
+      const float2 c0 = __fadd2_rn(__ffma2_rn(d[j], inv2, sh), nsh);
+      const float2 c1 = __fadd2_rn(__ffma2_rn(d[j + 1], inv2, sh), nsh);
+      const float2 e0 = __ffma2_rn(c0, nstep2, d[j]);
+      const float2 e1 = __ffma2_rn(c1, nstep2, d[j + 1]);
+      a0 = __ffma2_rn(e0, e0, a0);
+      a1 = __ffma2_rn(e1, e1, a1);
+    }
+    err += (a0.x + a0.y) + (a1.x + a1.y);
+  }
+}
+
+template <int... Bs>
+struct BitSet {
+  static constexpr int N = sizeof...(Bs);
+};
+using DefaultBits = BitSet<0, 1, 2, 3, 4, 8>;
+
+template <int... Bs>
+__device__ __forceinline__ void block_errors_fixed(const float* v, float* err, BitSet<Bs...>) {
+  float mn, mx;
+  minmax16(v, mn, mx);
+  const float lo = rd16(mn);
+  float2 d[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) d[j] = __fadd2_rn(make_float2(v[2 * j], v[2 * j + 1]), make_float2(-lo, -lo));
+  int i = 0;
+  (bit_error<Bs>(v, d, mx, lo, err[i++]), ...);
+}
+
 // ---------------------------------------------------------------------------------------
 // distortion table kernel: grid (tiles, S, units); writes fp64 partial sums per CTA
 // ---------------------------------------------------------------------------------------
@@ -469,7 +528,7 @@ __host__ __device__ constexpr int table_split() { return D >= 32 ? 2 : 1; }
 template <int D>
 __host__ __device__ constexpr int table_threads() { return TTHREADS * table_split<D>(); }
 
-template <int D, typename TX>
+template <int D, typename TX, typename BITS>
 __global__ void __launch_bounds__(table_threads<D>(), D >= 64 ? 2 : 1) table_kernel(TableArgs a) {
   constexpr int SPLIT = table_split<D>();
   constexpr int THREADS = table_threads<D>();
@@ -519,7 +578,8 @@ __global__ void __launch_bounds__(table_threads<D>(), D >= 64 ? 2 : 1) table_ker
         for (int q = 0; q < blocks_per_thread<D, THREADS>(); ++q) {
           float v[16];
           load16(rho + brow * RhoTile<D>::LD + (block_first<D, THREADS>() + q) * 16, v);
-          block_errors(v, kb, err);
+          if constexpr (std::is_same<BITS, void>::value) block_errors(v, kb, err);
+          else block_errors_fixed(v, err, BITS{});
         }
       }
       // reduce over the warp, then over the warps in fixed order (fp64)
