@@ -11,9 +11,9 @@
 //   2. every eigenvalue of T by multisection on Sturm counts (8 threads per eigenvalue, each
 //      round shrinks the bracket ninefold);
 //   3. every eigenvector of T by inverse iteration (one thread each: tridiagonal LU with
-//      partial pivoting, three solves from a splitmix64 start vector); eigenvalues closer
-//      than 1e-10 ||T|| are redone in order, orthogonalised against the earlier members of
-//      their cluster inside every step;
+//      partial pivoting, two solves from a splitmix64 start vector); the vectors of
+//      eigenvalues closer than 1e-10 ||T|| span their cluster's invariant subspace and are
+//      orthonormalised in order by one warp (modified Gram-Schmidt);
 //   4. back-transformation V = H_0 ... H_{n-3} Z, CTA q on eigenvectors [32q, 32q + 32).
 // Output: w ascending; V[r * n + i] = component r of the unit eigenvector of w[i].
 // Non-finite input raises DEV_ERR_NONFINITE.  Every thread of every CTA passes the same
@@ -128,6 +128,44 @@ __device__ void tri_solve_normalise(const double* U0, const double* U1, const do
   }
   const double inv = nrm > 0.0 && isfinite(nrm) ? 1.0 / sqrt(nrm) : 0.0;
   for (int k = 0; k < n; ++k) x[(long long)k * n + i] *= inv;
+}
+
+// the same solve with the vector in shared memory (x[k * xs + il]) and the factors of global
+// column i
+__device__ void tri_solve_normalise_sm(const double* U0, const double* U1, const double* U2, const double* L,
+                                       const double* P, int n, double* x, int il, int xs, int i) {
+  for (int k = 0; k + 1 < n; ++k) {
+    const long long o = (long long)k * n + i;
+    double bk = x[k * xs + il], bk1 = x[(k + 1) * xs + il];
+    if (P[o] != 0.0) {
+      const double t = bk;
+      bk = bk1;
+      bk1 = t;
+    }
+    bk1 -= L[o] * bk;
+    x[k * xs + il] = bk;
+    x[(k + 1) * xs + il] = bk1;
+  }
+  double x1 = 0.0, x2 = 0.0, nrm = 0.0;
+  for (int k = n - 1; k >= 0; --k) {
+    const long long o = (long long)k * n + i;
+    double s = x[k * xs + il];
+    if (k + 1 < n) s -= U1[o] * x1;
+    if (k + 2 < n) s -= U2[o] * x2;
+    s /= U0[o];
+    x[k * xs + il] = s;
+    nrm = fma(s, s, nrm);
+    x2 = x1;
+    x1 = s;
+  }
+  const double inv = nrm > 0.0 && isfinite(nrm) ? 1.0 / sqrt(nrm) : 0.0;
+  for (int k = 0; k < n; ++k) x[k * xs + il] *= inv;
+}
+
+__device__ __forceinline__ double warp_sum(double v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
 }
 
 __device__ __forceinline__ double start_value(int i, int k) {
@@ -312,35 +350,45 @@ __global__ void __cluster_dims__(eigc::CL, 1, 1) __launch_bounds__(eigc::THREADS
   const double tiny = 2.220446049250313e-16 * fmax(norm, 2.2250738585072014e-308);
   const double ctol = 1e-10 * norm;
 
-  // 3. eigenvectors of T (one thread per eigenvector of this CTA), into V
+  // 3. eigenvectors of T (one thread per eigenvector of this CTA; the iterate in shared
+  //    memory, the factors in global memory), two solves, then into V
   if (tid < NC && c0 + tid < n) {
     const int i = c0 + tid;
+    double* xs = As;   // [MAXN][NC], free until the back-transformation
     eigc::tri_lu(sd, se, n, wu[i], tiny, U0, U1, U2, Lm, Pv, i);
-    for (int k = 0; k < n; ++k) Vu[(long long)k * n + i] = eigc::start_value(i, k);
-    for (int it = 0; it < 3; ++it) eigc::tri_solve_normalise(U0, U1, U2, Lm, Pv, n, Vu, i);
+    for (int k = 0; k < n; ++k) xs[k * NC + tid] = eigc::start_value(i, k);
+    for (int it = 0; it < 2; ++it) eigc::tri_solve_normalise_sm(U0, U1, U2, Lm, Pv, n, xs, tid, NC, i);
+    for (int k = 0; k < n; ++k) Vu[(long long)k * n + i] = xs[k * NC + tid];
   }
   __threadfence();
   cluster.sync();
-  // nearly equal eigenvalues: redone in order by one thread of the cluster
-  if (q == 0 && tid == 0) {
+  // eigenvalues closer than ctol: their vectors span the cluster's invariant subspace; one
+  // warp of the cluster orthonormalises them in order (modified Gram-Schmidt)
+  if (q == 0 && tid < 32) {
+    const int lane = tid;
     int cs0 = 0;
+    double wprev = wu[0];
     for (int i = 1; i < n; ++i) {
-      if (wu[i] - wu[i - 1] >= ctol) {
+      const double wi = wu[i];
+      const bool tight = wi - wprev < ctol;
+      wprev = wi;
+      if (!tight) {
         cs0 = i;
         continue;
       }
-      for (int it = 0; it < 4; ++it) {
-        for (int jj = cs0; jj < i; ++jj) {
-          double dot = 0.0;
-          for (int k = 0; k < n; ++k) dot = fma(Vu[(long long)k * n + jj], Vu[(long long)k * n + i], dot);
-          for (int k = 0; k < n; ++k) Vu[(long long)k * n + i] = fma(-dot, Vu[(long long)k * n + jj], Vu[(long long)k * n + i]);
-        }
-        double nrm = 0.0;
-        for (int k = 0; k < n; ++k) nrm = fma(Vu[(long long)k * n + i], Vu[(long long)k * n + i], nrm);
-        const double inv = nrm > 0.0 ? 1.0 / sqrt(nrm) : 0.0;
-        for (int k = 0; k < n; ++k) Vu[(long long)k * n + i] *= inv;
-        if (it < 3) eigc::tri_solve_normalise(U0, U1, U2, Lm, Pv, n, Vu, i);
+      for (int jj = cs0; jj < i; ++jj) {
+        double dot = 0.0;
+        for (int k = lane; k < n; k += 32) dot = fma(Vu[(long long)k * n + jj], Vu[(long long)k * n + i], dot);
+        dot = eigc::warp_sum(dot);
+        for (int k = lane; k < n; k += 32) Vu[(long long)k * n + i] = fma(-dot, Vu[(long long)k * n + jj], Vu[(long long)k * n + i]);
+        __syncwarp();
       }
+      double nrm = 0.0;
+      for (int k = lane; k < n; k += 32) nrm = fma(Vu[(long long)k * n + i], Vu[(long long)k * n + i], nrm);
+      nrm = eigc::warp_sum(nrm);
+      const double inv = nrm > 0.0 ? 1.0 / sqrt(nrm) : 0.0;
+      for (int k = lane; k < n; k += 32) Vu[(long long)k * n + i] *= inv;
+      __syncwarp();
     }
   }
   __threadfence();

@@ -15,7 +15,6 @@
 #include "misc.cuh"
 #include "umma.cuh"
 #include "eig_cluster.cuh"
-#include "chol_cluster.cuh"
 
 using namespace jolt;
 
@@ -577,18 +576,10 @@ jolt_status cholqr_batched(const Ctx& c, float* Y, long long m, int k, int ld, i
     float* Dinv = c.at<float>(p.o_Linv);
     const int nbk = (int)ceil_div(k, TS_NB);
     const long long sL = (long long)k * gld, sD = (long long)nbk * TS_NB * TS_NB;
-    if (k <= cholc::MAXN) {
-      // L (fp32) and the inverses of its diagonal blocks: one 8-CTA cluster per unit
-      ProfScope ps2("qr_potrf", c.st, p.NU);
-      const size_t sm = cholc::smem_bytes();
-      CUDA_TRY(cudaFuncSetAttribute(chol_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm));
-      count_launch(), chol_cluster_kernel<<<(unsigned)(p.NU * cholc::CL), cholc::THREADS, sm, c.st>>>(
-          G, k, gld, n, Lr, gld, sL, Dinv, sD, c.status());
-      CUDA_TRY(cudaGetLastError());
-    } else {
-      count_launch(), sanitize_sym_batched_kernel<<<p.NU, 1024, 0, c.st>>>(G, k, gld, n, c.status());
-      count_launch(), ptr_array_kernel<<<1, 64, 0, c.st>>>(ptrs, G, n, p.NU);
-      CUDA_TRY(cudaGetLastError());
+    count_launch(), sanitize_sym_batched_kernel<<<p.NU, 1024, 0, c.st>>>(G, k, gld, n, c.status());
+    count_launch(), ptr_array_kernel<<<1, 64, 0, c.st>>>(ptrs, G, n, p.NU);
+    CUDA_TRY(cudaGetLastError());
+    {
       ProfScope ps2("qr_potrf", c.st, p.NU);
       SOLVER_TRY(cusolverDnDpotrfBatched(s->h, CUBLAS_FILL_MODE_LOWER, k, ptrs, gld, info, p.NU));
       count_launch(), info_check_kernel<<<(unsigned)ceil_div(p.NU, 32), 32, 0, c.st>>>(info, p.NU, c.status(),
@@ -597,10 +588,8 @@ jolt_status cholqr_batched(const Ctx& c, float* Y, long long m, int k, int ld, i
       CUDA_TRY(cudaGetLastError());
     }
     ProfScope ps3("qr_trsm", c.st, p.NU);
-    // rows per CTA: 128 (4 rows x 4 columns per thread) when the panel fits and there are
-    // enough rows to fill the GPU, else 64, else 32 for wide blocks
-    if (k <= 256 && m * p.NU >= 128LL * 148 * 2) JTRY(launch_trsm_panel<128>(c, Y, m, k, ld, Lr, gld, sL, Dinv, sD));
-    else if (k <= 512) JTRY(launch_trsm_panel<64>(c, Y, m, k, ld, Lr, gld, sL, Dinv, sD));
+    // rows per CTA: 64 (two CTAs per SM), 32 for wide blocks
+    if (k <= 512) JTRY(launch_trsm_panel<64>(c, Y, m, k, ld, Lr, gld, sL, Dinv, sD));
     else JTRY(launch_trsm_panel<32>(c, Y, m, k, ld, Lr, gld, sL, Dinv, sD));
   }
   return JOLT_OK;
