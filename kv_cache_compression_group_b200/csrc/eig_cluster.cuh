@@ -34,9 +34,11 @@ constexpr int MAXN = CL * NC;    // 256
 constexpr int THREADS = 256;
 constexpr int SUB = 8;           // threads per eigenvalue in the multisection
 // shared memory (doubles): A [MAXN][NC + 1] | v[2][MAXN] | w[2][MAXN] | d | e | beta [MAXN] |
-// p [NC] | red[2][CL] | tmp[THREADS]
+// p [NC] | red[2][RED] | tmp[THREADS]
 constexpr int A_LD = NC + 1;
-constexpr size_t SMEM_DOUBLES = (size_t)MAXN * A_LD + 4 * MAXN + 3 * MAXN + NC + 2 * CL + THREADS;
+constexpr int WARPS = THREADS / 32;
+constexpr int RED = CL * WARPS;  // partial-sum slots per buffer: one per (CTA, warp)
+constexpr size_t SMEM_DOUBLES = (size_t)MAXN * A_LD + 4 * MAXN + 3 * MAXN + NC + 2 * RED + THREADS;
 inline size_t smem_bytes() { return SMEM_DOUBLES * sizeof(double); }
 // global scratch per matrix (doubles): reflectors n*n | LU 5*n*n
 __host__ __device__ inline size_t scratch_doubles(int n) { return (size_t)6 * n * n; }
@@ -178,7 +180,7 @@ __device__ __forceinline__ double start_value(int i, int k) {
 // eigc::smem_bytes().  A: input matrices (lower triangle of column-major n x n, stride sA);
 // w: eigenvalues (stride sw); V: eigenvectors (row-major n x n per matrix, stride n*n);
 // scr: eigc::scratch_doubles(n) per matrix.
-__global__ void __cluster_dims__(eigc::CL, 1, 1) __launch_bounds__(eigc::THREADS)
+__global__ void __cluster_dims__(eigc::CL, 1, 1) __launch_bounds__(eigc::THREADS, 2)
     sym_eig_cluster_kernel(const double* A, int n, long long sA, double* w, long long sw, double* V, double* scr,
                            uint32_t* status) {
   using namespace eigc;
@@ -194,8 +196,8 @@ __global__ void __cluster_dims__(eigc::CL, 1, 1) __launch_bounds__(eigc::THREADS
   double* se = sd + MAXN;                  // [MAXN]
   double* sb = se + MAXN;                  // [MAXN]
   double* sp = sb + MAXN;                  // [NC]
-  double* red = sp + NC;                   // [2][CL]
-  double* tmp = red + 2 * CL;              // [THREADS]
+  double* red = sp + NC;                   // [2][RED]
+  double* tmp = red + 2 * RED;             // [THREADS]
   const double* Au = A + (long long)u * sA;
   double* wu = w + (long long)u * sw;
   double* Vu = V + (long long)u * n * n;
@@ -224,12 +226,13 @@ __global__ void __cluster_dims__(eigc::CL, 1, 1) __launch_bounds__(eigc::THREADS
   for (int j = 0; j + 2 < n; ++j) {
     const int buf = j & 1, owner = j / NC, lc = j - owner * NC;
     if (q == owner) {
+      // every warp forms the same norm (same order), so no CTA barrier is needed here
       double part = 0.0;
-      for (int r = j + 2 + tid; r < n; r += blockDim.x) {
+      for (int r = j + 2 + (tid & 31); r < n; r += 32) {
         const double x = As[r * A_LD + lc];
         part = fma(x, x, part);
       }
-      const double tail2 = block_sum(part, tmp);
+      const double tail2 = warp_sum(part);
       const double x0 = As[(j + 1) * A_LD + lc];
       double beta = 0.0, alpha = x0;
       if (tail2 > 0.0) {
@@ -268,14 +271,15 @@ __global__ void __cluster_dims__(eigc::CL, 1, 1) __launch_bounds__(eigc::THREADS
       const double pc = (c > j && c < n) ? beta * s : 0.0;
       if (part == 0)
         for (int t = 0; t < CL; ++t) cluster.map_shared_rank(wb, t)[buf * MAXN + c] = pc;
-      const double pv = block_sum(part == 0 ? pc * v[c] : 0.0, tmp);
-      if (tid == 0)
-        for (int t = 0; t < CL; ++t) cluster.map_shared_rank(red, t)[buf * CL + q] = pv;
+      // one partial sum of p.v per warp, into slot (q, warp) of every CTA
+      const double pv = warp_sum(part == 0 ? pc * v[c] : 0.0);
+      if ((tid & 31) == 0)
+        for (int t = 0; t < CL; ++t) cluster.map_shared_rank(red, t)[buf * RED + q * WARPS + (tid >> 5)] = pv;
     }
     cluster.sync();   // (B) p and the partial sums of p.v everywhere
     if (beta != 0.0) {
       double ptv = 0.0;
-      for (int t = 0; t < CL; ++t) ptv += red[buf * CL + t];
+      for (int t = 0; t < RED; ++t) ptv += red[buf * RED + t];
       const double K = 0.5 * beta * ptv;
       // A -= v w^T + w v^T with w = p - K v (each CTA forms w itself from the gathered p)
       const int lcol = tid & (NC - 1), c = c0 + lcol;
@@ -327,6 +331,7 @@ __global__ void __cluster_dims__(eigc::CL, 1, 1) __launch_bounds__(eigc::THREADS
     // every lane of the warp takes part in every shuffle
     for (int it = 0; it < 24; ++it) {
       const bool done = b - a <= 2.220446049250313e-16 * fmax(fabs(a), fabs(b)) + pivmin;
+      if (__all_sync(0xffffffffu, done)) break;   // the whole warp has converged
       const double x = a + (b - a) * (double)(sub + 1) / (double)(SUB + 1);
       const int cnt = (i < n && !done) ? eigc::sturm_count(sd, e2, n, x, pivmin) : 0;
       double na = a, nb = b;

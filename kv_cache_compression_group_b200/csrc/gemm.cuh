@@ -39,6 +39,7 @@ struct GemmParams {
   int splits = 1;             // split-K: split s covers [s*kchunk, (s+1)*kchunk)
   int kchunk = 0;
   long long ssplitC = 0;      // output stride between splits
+  bool sym = false;           // C = A^T A (A = B): tiles above the diagonal are skipped (sgemm)
 };
 
 __host__ __device__ __forceinline__ long long opnd_offset(const GemmOperand& o, long long x, long long k) {
@@ -155,6 +156,7 @@ __global__ void __launch_bounds__(256) gemm_bf16_kernel(GemmParams p) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int wm = warp >> 2, wn = warp & 3;  // 2 x 4 warps, warp tile 64 x 32
   const int m0 = blockIdx.y * BM, n0 = blockIdx.x * BN;
+  if (p.sym && blockIdx.x > blockIdx.y) return;   // mirrored from the tile below the diagonal
   const int bz = blockIdx.z;
   const int b = bz / p.splits, split = bz - b * p.splits;
   const int kbeg = split * p.kchunk;

@@ -394,6 +394,7 @@ jolt_status make_plan(const jolt_shape* sh, const jolt_options* op, Plan* p) {
 jolt_status gemm(const GemmParams& p, int ta, int tb, cudaStream_t st) {
   cudaError_t e;
   const bool dacc = p.c_type == 2;
+  if (p.sym && !(ta == 1 && tb == 1 && !dacc)) return fail(JOLT_ERR_INVALID_ARG, "symmetric GEMM needs fp32 operands");
   if (ta == 0 && tb == 0) e = launch_gemm_bf16(p, st);
   else if (ta == 1 && tb == 1 && p.c_type != 2) e = launch_sgemm(p, st);
 #define GEMM_CASE(A, B, TA, TB)                                                              \
@@ -569,9 +570,11 @@ jolt_status cholqr_batched(const Ctx& c, float* Y, long long m, int k, int ld, i
     g.splits = ns;
     g.kchunk = 256;
     g.c_type = 0;
+    g.sym = true;
     JTRY(gemm(g, 1, 1, c.st));
     const long long n = (long long)k * gld;
-    count_launch(), reduce_splits_kernel<float><<<grid1d((long long)p.NU * n), 256, 0, c.st>>>(gpart, G, p.NU, ns, n);
+    count_launch(), reduce_splits_sym_kernel<float><<<grid1d((long long)p.NU * k * k), 256, 0, c.st>>>(
+        gpart, G, p.NU, ns, k, gld, sgemm_detail::BM);
     float* Lr = c.at<float>(p.o_Lr);
     float* Dinv = c.at<float>(p.o_Linv);
     const int nbk = (int)ceil_div(k, TS_NB);
@@ -922,9 +925,10 @@ jolt_status run_token_randomized(const Ctx& c, float* Uf, long long ldUf) {
     g.splits = ns;
     g.kchunk = 256;
     g.c_type = 0;
+    g.sym = true;
     JTRY(gemm(g, 1, 1, c.st));
-    count_launch(), reduce_splits_kernel<float><<<grid1d((long long)NU * k * k), 256, 0, c.st>>>(
-        gpart, S, NU, ns, (long long)k * k);
+    count_launch(), reduce_splits_sym_kernel<float><<<grid1d((long long)NU * k * k), 256, 0, c.st>>>(
+        gpart, S, NU, ns, k, k, sgemm_detail::BM);
     CUDA_TRY(cudaGetLastError());
   }
   float* V = c.at<float>(p.o_vsel);

@@ -20,6 +20,25 @@ __global__ void reduce_splits_kernel(const TP* part, double* out, int nbatch, in
   }
 }
 
+// the same sum for a symmetric k x k result whose split partials hold only the tiles on and
+// below the diagonal (tile edge te): entry (r, c) of an upper tile is read at (c, r)
+template <typename TP>
+__global__ void reduce_splits_sym_kernel(const TP* part, double* out, int nbatch, int nsplit, int k, long long ld,
+                                         int te) {
+  const long long n = (long long)k * ld;
+  const long long total = (long long)nbatch * k * k;
+  for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < total;
+       idx += (long long)gridDim.x * blockDim.x) {
+    const long long b = idx / ((long long)k * k), rem = idx - b * k * k;
+    const int r = (int)(rem / k), c = (int)(rem - (long long)r * k);
+    const long long src = (c / te > r / te) ? (long long)c * ld + r : (long long)r * ld + c;
+    const TP* p = part + b * nsplit * n + src;
+    double acc = 0.0;
+    for (int s = 0; s < nsplit; ++s) acc += (double)p[(long long)s * n];
+    out[b * n + (long long)r * ld + c] = acc;
+  }
+}
+
 // every diagonal entry of the unit's feature Gram must be finite (a NaN/Inf anywhere in
 // the cache reaches the diagonal through x*x)
 __global__ void gram_diag_check_kernel(const double* G, int n, int nunits, uint32_t* status) {
