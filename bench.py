@@ -47,6 +47,9 @@ def parse():
     ap.add_argument("--no-extras", action="store_true", help="skip the exact-arm and decompress side figures")
     ap.add_argument("--profile-case", default=None, choices=["mistral7b_4layers", "mistral7b"],
                     help="run two compress + decompress calls of one case (for ncu captures) and exit")
+    ap.add_argument("--sweep", action="store_true",
+                    help="one JSON line per workload of the other shapes (LLaMA-2-13B, LLaMA-3.1-8B/64K) and "
+                         "per context length of the Mistral-shaped sweep, JoLT and FlashJoLT, then exit")
     return ap.parse_args()
 
 
@@ -70,6 +73,61 @@ def profile_case(args):
     torch.cuda.synchronize()
     print(json.dumps({"profile_case": args.profile_case, "method": args.method,
                       "total_bytes": J.read_header(blob)[1]}))
+
+
+def sweep(args):
+    """Compress and decompress throughput of the other workload shapes: LLaMA-2-13B and
+    LLaMA-3.1-8B/64K (FlashJoLT, 2x / 3x), and the Mistral-shaped generator at T = 512 ..
+    32768 (FlashJoLT; JoLT up to T = 2048, 2x).  Each case: the first call runs directly, the second is
+    captured as a CUDA graph, then three replays are timed with CUDA events (inputs resident
+    in HBM; the 126 MB L2 holds a small part of the larger caches)."""
+    import torch
+    from kv_cache_compression_group_b200 import synth, jolt as J
+    cases = [("llama2_13b", "randomized", (2.0, 3.0)), ("llama31_8b_64k", "randomized", (2.0, 3.0))]
+    for T in (512, 1024, 2048, 8192, 32768):
+        for meth in (("exact", "randomized") if T <= 2048 else ("randomized",)):
+            cases.append((f"sweep_T{T}", meth, (2.0,)))
+    cache = {}
+    for name, meth, ratios in cases:
+        w = synth.sweep_workload(int(name[7:])) if name.startswith("sweep_T") else synth.WORKLOADS[name]
+        if name not in cache:
+            cache.clear()
+            K, V = synth.make_cache(w, 0)
+            cache[name] = (K.cuda(), V.cuda())
+            del K, V
+        Kd, Vd = cache[name]
+        opts = J.default_options(w.T, w.D, meth)
+        comp = J.Compressor(w.n_layers, w.n_heads, w.T, w.D, w.layers_per_group, Kd.dtype, opts)
+        for ratio in ratios:
+            budget = int(w.bf16_bytes() / ratio)
+            blob = torch.empty(min(budget, comp.blob_max), dtype=torch.uint8, device="cuda")
+            for _ in range(3):
+                comp.compress(Kd, Vd, budget, 0, blob=blob)
+            torch.cuda.synchronize()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            for _ in range(3):
+                comp.compress(Kd, Vd, budget, 0, blob=blob)
+            b.record()
+            torch.cuda.synchronize()
+            ms = a.elapsed_time(b) / 3
+            _, total, _ = J.read_header(blob)
+            Ko, Vo = comp.decompress(blob)
+            torch.cuda.synchronize()
+            a.record()
+            Ko, Vo = comp.decompress(blob, K_out=Ko, V_out=Vo)
+            b.record()
+            torch.cuda.synchronize()
+            dms = a.elapsed_time(b)
+            ek, ev = J.relative_errors(Kd, Vd, Ko, Vo, w.layers_per_group)
+            del Ko, Vo
+            print(json.dumps({"sweep": name, "method": meth, "ratio": ratio, "shape": [w.n_layers, w.n_heads, w.T, w.D],
+                              "input_bytes": w.input_bytes(), "compress_ms": ms, "compress_gbs": w.input_bytes() / ms / 1e6,
+                              "latency_per_layer_group_ms": ms / w.n_groups, "decompress_ms": dms,
+                              "decompress_out_gbs": w.input_bytes() / dms / 1e6, "total_bytes": total,
+                              "rel_err_K": ek, "rel_err_V": ev, "token_ranks": list(opts.token_ranks)}), flush=True)
+        del comp
+        torch.cuda.empty_cache()
 
 
 def workload_config(w, method, opts):
@@ -237,6 +295,8 @@ def main():
         return run_reference(args, rank, world)
     if args.profile_case:
         return profile_case(args)
+    if args.sweep:
+        return sweep(args)
 
     import torch
     from kv_cache_compression_group_b200 import synth, jolt as J
