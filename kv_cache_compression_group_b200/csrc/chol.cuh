@@ -1,0 +1,384 @@
+// Cholesky QR of the sketch blocks for widths k <= 256: Q = Y L^{-T} with G = Y^T Y = L L^T.
+//
+// Three kernels, all in fp64 up to the last product:
+//   chol_factor_kernel   one CTA per unit: the Cholesky factor L of the Gram, left-looking,
+//                        blocked by 32 columns; it also inverts each 32 x 32 diagonal block;
+//   tri_inv_kernel       one CTA per (32-column block, unit): that block column of W = L^{-1}
+//                        by block forward substitution (the block columns are independent);
+//   trsm_inv_kernel      one CTA per 64 rows of Y: Q = Y W^T in fp32 with every output
+//                        column independent (no sequential dependency across columns).
+// The Gram buffer G (column-major, ld gld, symmetric on entry) carries the factor between
+// them: L's rows below its diagonal blocks go to the lower triangle, the inverses of the
+// diagonal blocks to the upper triangle of their own diagonal block (W[i][c] at G[i*gld+c],
+// c <= i), both places the factorisation no longer reads.
+#pragma once
+
+#include "common.cuh"
+
+namespace jolt {
+
+constexpr int CF_NB = 32;
+constexpr int CF_MAXK = 256;
+constexpr int CF_THREADS = 256;
+constexpr int CF_P = CF_NB + 1;   // shared-memory pitch (doubles)
+inline size_t chol_factor_smem() { return 3 * (size_t)CF_MAXK * CF_P * sizeof(double); }
+
+// asynchronous global -> shared copies (the staging loads of all three kernels stay in flight
+// together instead of one round trip per element); src_bytes < size zero-fills the rest
+__device__ __forceinline__ void cf_cp8(void* dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 8;\n" ::"r"((uint32_t)__cvta_generic_to_shared(dst)),
+               "l"(src)
+               : "memory");
+}
+__device__ __forceinline__ void cf_cp16(void* dst, const void* src, int src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"((uint32_t)__cvta_generic_to_shared(dst)),
+               "l"(src), "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cf_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cf_wait() {
+  asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
+}
+
+// Non-finite Gram entries (or one met earlier in the cache): G := I (so W = I) and
+// DEV_ERR_NONFINITE.  A pivot that is not positive: DEV_ERR_FACTOR, the pivot taken as 1.
+__global__ void __launch_bounds__(CF_THREADS, 1)
+    chol_factor_kernel(double* G, int k, long long gld, long long sG, uint32_t* status) {
+  extern __shared__ __align__(16) double cf_sm[];
+  double* P = cf_sm;                      // [row - J0][col - J0] of the block column
+  double* const Lb0 = cf_sm + CF_MAXK * CF_P;   // two buffers [row - J0][q]: 32 finished columns
+  __shared__ double rdiag[CF_NB];
+  __shared__ int fail;
+  const int u = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  double* Gu = G + (long long)u * sG;
+  const int nbk = (k + CF_NB - 1) / CF_NB;
+
+  constexpr int NW = CF_THREADS / 32;
+  int bad = (tid == 0 && (*status & DEV_ERR_NONFINITE)) ? 1 : 0;
+  for (int c = warp; c < k; c += NW) {
+    double v[CF_MAXK / 32];
+#pragma unroll
+    for (int t = 0; t < CF_MAXK / 32; ++t) v[t] = lane + 32 * t < k ? Gu[(long long)c * gld + lane + 32 * t] : 0.0;
+#pragma unroll
+    for (int t = 0; t < CF_MAXK / 32; ++t)
+      if (!isfinite(v[t])) bad = 1;
+  }
+  if (tid == 0) fail = 0;
+  if (__syncthreads_or(bad)) {
+    if (tid == 0) raise_status(status, DEV_ERR_NONFINITE);
+    for (int c = warp; c < k; c += NW)
+      for (int i = lane; i < k; i += 32) Gu[(long long)c * gld + i] = i == c ? 1.0 : 0.0;
+    return;
+  }
+
+  const int tc = tid & 7, tr = tid >> 3;   // update tile: columns tc + 8 j, rows tr + 32 m
+  for (int J = 0; J < nbk; ++J) {
+    const int J0 = J * CF_NB, nb = min(CF_NB, k - J0), R = k - J0;
+    double acc[8][4];
+    // the Gram's block column, read through the symmetric upper part (rows and columns
+    // >= J0 there are not written before this block column is done)
+#pragma unroll
+    for (int m = 0; m < 8; ++m)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int lr = tr + 32 * m, c = tc + 8 * j;
+        acc[m][j] = (lr < R && c < nb) ? Gu[(long long)(J0 + lr) * gld + J0 + c] : 0.0;
+      }
+    // finished block column Q, rows J0.. (written to the lower triangle before the barrier
+    // that ended block column Q) -> buffer
+    auto stage = [&](int Q, double* buf) {
+#pragma unroll
+      for (int s = 0; s < CF_NB / NW; ++s) {
+        const int q = warp + NW * s;
+        const double* src = Gu + (long long)(Q * CF_NB + q) * gld + J0;
+#pragma unroll
+        for (int t = 0; t < CF_MAXK / 32; ++t) {
+          const int lr = lane + 32 * t;
+          if (lr < R) cf_cp8(buf + lr * CF_P + q, src + lr);
+        }
+      }
+      cf_commit();
+    };
+    if (J > 0) stage(0, Lb0);
+    for (int Q = 0; Q < J; ++Q) {
+      // the buffer of chunk Q + 1 was last read before the barrier ending chunk Q - 1
+      if (Q + 1 < J) {
+        stage(Q + 1, Lb0 + ((Q + 1) & 1) * (CF_MAXK * CF_P));
+        cf_wait<1>();
+      } else {
+        cf_wait<0>();
+      }
+      __syncthreads();
+      const double* Lc = Lb0 + (Q & 1) * (CF_MAXK * CF_P);
+#pragma unroll 4
+      for (int q = 0; q < CF_NB; ++q) {
+        double b[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) b[j] = Lc[(tc + 8 * j) * CF_P + q];
+#pragma unroll
+        for (int m = 0; m < 8; ++m) {
+          if (32 * m < R) {
+            const double a = Lc[(tr + 32 * m) * CF_P + q];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) acc[m][j] = fma(-a, b[j], acc[m][j]);
+          }
+        }
+      }
+      __syncthreads();
+    }
+#pragma unroll
+    for (int m = 0; m < 8; ++m)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int lr = tr + 32 * m, c = tc + 8 * j;
+        if (lr < R && c < nb) P[lr * CF_P + c] = acc[m][j];
+      }
+    __syncthreads();
+    // diagonal block: unblocked Cholesky by warp 0, lane r holding row r in registers
+    if (warp == 0) {
+      double a[CF_NB];
+#pragma unroll
+      for (int c = 0; c < CF_NB; ++c) a[c] = (lane < nb && c <= lane) ? P[lane * CF_P + c] : 0.0;
+#pragma unroll
+      for (int c = 0; c < CF_NB; ++c) {
+        if (c < nb) {
+          const double piv = __shfl_sync(0xffffffffu, a[c], c);
+          const bool ok = piv > 0.0 && isfinite(piv);
+          const double rd = ok ? rsqrt(piv) : 1.0;
+          if (lane == 0 && !ok) fail = 1;
+          if (lane == c) {
+            a[c] = ok ? piv * rd : 1.0;
+            rdiag[c] = rd;
+          } else if (lane > c) {
+            a[c] *= rd;
+          }
+#pragma unroll
+          for (int c2 = c + 1; c2 < CF_NB; ++c2) {
+            const double l2 = __shfl_sync(0xffffffffu, a[c], c2);   // L[c2][c]
+            if (lane >= c2) a[c2] = fma(-a[c], l2, a[c2]);
+          }
+        }
+      }
+#pragma unroll
+      for (int c = 0; c < CF_NB; ++c)
+        if (lane < nb && c <= lane) P[lane * CF_P + c] = a[c];
+    }
+    __syncthreads();
+    const int nbelow = R - nb;   // <= 224: threads of warps 0..6
+    if (tid < nbelow) {
+      // row of L below the diagonal block: x L_JJ^T = g (forward substitution)
+      double* row = P + (nb + tid) * CF_P;
+      double x[CF_NB];
+#pragma unroll
+      for (int c = 0; c < CF_NB; ++c) x[c] = c < nb ? row[c] : 0.0;
+#pragma unroll
+      for (int c = 0; c < CF_NB; ++c) {
+        if (c < nb) {
+          x[c] *= rdiag[c];
+#pragma unroll
+          for (int c2 = c + 1; c2 < CF_NB; ++c2)
+            if (c2 < nb) x[c2] = fma(-x[c], P[c2 * CF_P + c], x[c2]);
+        }
+      }
+#pragma unroll
+      for (int c = 0; c < CF_NB; ++c)
+        if (c < nb) row[c] = x[c];
+    } else if (warp == CF_THREADS / 32 - 1) {
+      // inverse of the diagonal block, lane = column (forward substitution), stored as
+      // W[J0 + r][J0 + lane] at G[(J0 + r) * gld + J0 + lane] for lane <= r
+      double x[CF_NB];
+#pragma unroll
+      for (int r = 0; r < CF_NB; ++r) {
+        double v = (r == lane) ? 1.0 : 0.0;
+        if (r < nb && lane < nb) {
+#pragma unroll
+          for (int q = 0; q < r; ++q) v = fma(-P[r * CF_P + q], x[q], v);
+          x[r] = lane <= r ? v * rdiag[r] : 0.0;
+          if (lane <= r) Gu[(long long)(J0 + r) * gld + J0 + lane] = x[r];
+        } else {
+          x[r] = 0.0;
+        }
+      }
+    }
+    __syncthreads();
+    // the rows below the diagonal block to the lower triangle (read by later block columns
+    // and by the inverse)
+    for (int c = warp; c < nb; c += NW) {
+      double* dst = Gu + (long long)(J0 + c) * gld + J0;
+      for (int lr = nb + lane; lr < R; lr += 32) dst[lr] = P[lr * CF_P + c];
+    }
+    __syncthreads();
+  }
+  if (tid == 0 && fail) raise_status(status, DEV_ERR_FACTOR);
+}
+
+// ------------------------------------------------------------------------------------------
+// Block column J of W = L^{-1}:  W_JJ = inv(L_JJ),  W_IJ = -inv(L_II) sum_{J<=K<I} L_IK W_KJ.
+// Written transposed and in fp32: WT[q][i] = W[i][q] for the rows q of block J (zeros for
+// i < J0 and for i >= k up to the padded width ldw).
+// ------------------------------------------------------------------------------------------
+constexpr int TI_LP = CF_MAXK + 1;
+inline size_t tri_inv_smem() {
+  return ((size_t)CF_MAXK * CF_P + (size_t)CF_NB * TI_LP + 2 * (size_t)CF_NB * CF_P) * sizeof(double);
+}
+
+__global__ void __launch_bounds__(CF_THREADS, 1)
+    tri_inv_kernel(const double* G, int k, long long gld, long long sG, float* WT, long long ldw, long long sW) {
+  extern __shared__ __align__(16) double ti_sm[];
+  double* X = ti_sm;                       // [i - J0][c]: rows of W's block column
+  double* Ls = X + CF_MAXK * CF_P;         // [r][q - J0]: L's rows of block I
+  double* Ds = Ls + CF_NB * TI_LP;         // inv(L_II)
+  double* Ts = Ds + CF_NB * CF_P;          // sum_K L_IK W_KJ
+  const int J = blockIdx.x, u = blockIdx.y, tid = threadIdx.x;
+  const int J0 = J * CF_NB, nbJ = min(CF_NB, k - J0);
+  const int nbk = (k + CF_NB - 1) / CF_NB;
+  const double* Gu = G + (long long)u * sG;
+  const int r = tid >> 3, cg = tid & 7;    // 32 x 32 outputs: row r, columns cg + 8 j
+
+  // the inverse of the 32 x 32 diagonal block I (lower; W[I0 + r][I0 + c] at G[(I0 + r) * gld + I0 + c])
+  auto stage_diag = [&](int I0, int nbI, double* dst) {
+    for (int idx = tid; idx < CF_NB * CF_NB; idx += CF_THREADS) {
+      const int rr = idx / CF_NB, c = idx % CF_NB;
+      if (rr < nbI && c <= rr) cf_cp8(dst + rr * CF_P + c, Gu + (long long)(I0 + rr) * gld + I0 + c);
+      else dst[rr * CF_P + c] = 0.0;
+    }
+  };
+  stage_diag(J0, nbJ, X);
+  cf_commit();
+  for (int I = J + 1; I < nbk; ++I) {
+    const int I0 = I * CF_NB, nbI = min(CF_NB, k - I0), KQ = I0 - J0;
+    __syncthreads();
+    for (int idx = tid; idx < KQ * CF_NB; idx += CF_THREADS) {
+      const int q = idx / CF_NB, rr = idx % CF_NB;
+      if (rr < nbI) cf_cp8(Ls + rr * TI_LP + q, Gu + (long long)(J0 + q) * gld + I0 + rr);
+      else Ls[rr * TI_LP + q] = 0.0;
+    }
+    stage_diag(I0, nbI, Ds);
+    cf_commit();
+    cf_wait<0>();
+    __syncthreads();
+    double acc[4] = {0.0, 0.0, 0.0, 0.0};
+#pragma unroll 4
+    for (int q = 0; q < KQ; ++q) {
+      const double a = Ls[r * TI_LP + q];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) acc[j] = fma(a, X[q * CF_P + cg + 8 * j], acc[j]);
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) Ts[r * CF_P + cg + 8 * j] = acc[j];
+    __syncthreads();
+    double out[4] = {0.0, 0.0, 0.0, 0.0};
+    for (int s = 0; s <= r; ++s) {
+      const double d = Ds[r * CF_P + s];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) out[j] = fma(d, Ts[s * CF_P + cg + 8 * j], out[j]);
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) X[(KQ + r) * CF_P + cg + 8 * j] = r < nbI ? -out[j] : 0.0;
+  }
+  cf_wait<0>();
+  __syncthreads();
+  float* Wu = WT + (long long)u * sW;
+  for (int c = tid >> 5; c < nbJ; c += CF_THREADS / 32)
+    for (int i = tid & 31; i < ldw; i += 32)
+      Wu[(long long)(J0 + c) * ldw + i] = (i >= J0 && i < k) ? (float)X[(i - J0) * CF_P + c] : 0.f;
+}
+
+// ------------------------------------------------------------------------------------------
+// Q = Y W^T in place, W lower triangular (k <= 256): a CTA keeps 64 rows of Y in shared
+// memory and stages WT 16 rows at a time (the next chunk in flight while the current one is
+// used); warp w computes rows 8w..8w+7, lane l the columns l + 32 j.  Column blocks j with
+// 32 j + 31 < q0 meet only zeros of W in the chunk at q0 and are skipped.
+// ------------------------------------------------------------------------------------------
+constexpr int TI_RB = 64;
+constexpr int TI_QC = 16;   // rows of WT per staged chunk (double-buffered)
+inline int trsm_inv_pitch(int kq) { return kq + 4; }
+inline size_t trsm_inv_smem(int kq) {
+  return ((size_t)TI_RB * trsm_inv_pitch(kq) + 2 * (size_t)TI_QC * kq) * sizeof(float);
+}
+
+__global__ void __launch_bounds__(CF_THREADS, 2)
+    trsm_inv_kernel(float* Y, long long m, int k, long long ld, long long sY, const float* WT, long long ldw,
+                    long long sW) {
+  extern __shared__ __align__(16) float tv_sm[];
+  const int kq = (k + 31) & ~31, P = kq + 4, nj = kq / 32;
+  float* panel = tv_sm;                                      // TI_RB x P
+  float* const wt0 = panel + TI_RB * P;                      // two buffers TI_QC x kq
+  const int u = blockIdx.y, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const long long r0 = (long long)blockIdx.x * TI_RB;
+  float* Yu = Y + (long long)u * sY;
+  const float* Wu = WT + (long long)u * sW;
+  // rows r0.. of Y (16-byte copies: ld is a multiple of 4 floats; columns >= k and rows >= m
+  // are zero-filled)
+  for (int rr = warp; rr < TI_RB; rr += CF_THREADS / 32)
+    for (int c = 4 * lane; c < kq; c += 128) {
+      const bool row_ok = r0 + rr < m;
+      const int nbytes = row_ok ? 4 * max(0, min(4, k - c)) : 0;
+      cf_cp16(panel + rr * P + c, nbytes > 0 ? Yu + (r0 + rr) * ld + c : Yu, nbytes);
+    }
+  auto stage = [&](int q0, float* buf) {
+    for (int q = warp; q < TI_QC; q += CF_THREADS / 32)
+      for (int c = 4 * lane; c < kq; c += 128) {
+        const bool ok = q0 + q < k;
+        cf_cp16(buf + q * kq + c, ok ? Wu + (long long)(q0 + q) * ldw + c : Wu, ok ? 16 : 0);
+      }
+    cf_commit();
+  };
+  stage(0, wt0);   // committed together with the panel
+  float acc[8][8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
+  const int nch = (k + TI_QC - 1) / TI_QC;
+  for (int ch = 0; ch < nch; ++ch) {
+    const int q0 = ch * TI_QC;
+    // the buffer of chunk ch + 1 was last read before the barrier ending chunk ch - 1
+    if (ch + 1 < nch) {
+      stage(q0 + TI_QC, wt0 + ((ch + 1) & 1) * (TI_QC * kq));
+      cf_wait<1>();
+    } else {
+      cf_wait<0>();
+    }
+    __syncthreads();
+    const float* wt = wt0 + (ch & 1) * (TI_QC * kq);
+    const int jmin = q0 / 32;   // column blocks j with 32 j + 31 < q0 meet only zeros of W
+#pragma unroll 1
+    for (int q = 0; q < TI_QC; q += 4) {
+      float w[8][4];
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) w[j][e] = (j >= jmin && j < nj) ? wt[(q + e) * kq + lane + 32 * j] : 0.f;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float4 y = *reinterpret_cast<const float4*>(panel + (warp * 8 + i) * P + q0 + q);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          if (j >= jmin && j < nj) {
+            float a = acc[i][j];
+            a = fmaf(y.x, w[j][0], a);
+            a = fmaf(y.y, w[j][1], a);
+            a = fmaf(y.z, w[j][2], a);
+            a = fmaf(y.w, w[j][3], a);
+            acc[i][j] = a;
+          }
+        }
+      }
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const long long rr = r0 + warp * 8 + i;
+    if (rr >= m) continue;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int c = lane + 32 * j;
+      if (j < nj && c < k) Yu[rr * ld + c] = acc[i][j];
+    }
+  }
+}
+
+}  // namespace jolt

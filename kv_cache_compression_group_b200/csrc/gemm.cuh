@@ -371,14 +371,16 @@ __global__ void __launch_bounds__(256) gemm_simt_kernel(GemmParams p) {
 namespace sgemm_detail {
 constexpr int BM = 128, BN = 128, BK = 8, THREADS = 256;
 
-// load the BK x 128 slice (k0.., x0..) of an operand into s[BK][128] (x fastest)
-__device__ __forceinline__ void load_slice(float (*s)[BM], const GemmOperand& o, const float* base, int x0, int k0,
-                                           int Xext, int kend, int tid) {
+// The BK x 128 slice (k0.., x0..) of an operand, in two steps so that the global loads of the
+// next slice are in flight while the current one is multiplied: fetch_slice reads this
+// thread's four values into registers, store_slice puts them into s[BK][128] (x fastest).
+__device__ __forceinline__ void fetch_slice(float* v, const GemmOperand& o, const float* base, int x0, int k0,
+                                            int Xext, int kend, int tid) {
+  v[0] = v[1] = v[2] = v[3] = 0.f;
   if (!o.kmajor) {
     // contiguous along x: thread -> (k row tid/32, four x from (tid%32)*4)
     const int kr = tid >> 5, xc = (tid & 31) * 4;
     const int k = k0 + kr, x = x0 + xc;
-    float v[4] = {0.f, 0.f, 0.f, 0.f};
     if (k < kend) {
       const float* src = base + opnd_offset(o, x, k);
       const bool vec = (x + 3 < Xext) && (o.xshift >= 31 || ((x & ((1 << o.xshift) - 1)) + 3) < (1 << o.xshift)) &&
@@ -392,12 +394,10 @@ __device__ __forceinline__ void load_slice(float (*s)[BM], const GemmOperand& o,
           if (x + e < Xext) v[e] = base[opnd_offset(o, x + e, k)];
       }
     }
-    *reinterpret_cast<float4*>(&s[kr][xc]) = make_float4(v[0], v[1], v[2], v[3]);
   } else {
-    // contiguous along k: thread -> (x row tid/2, four k from (tid%2)*4), stored transposed
+    // contiguous along k: thread -> (x row tid/2, four k from (tid%2)*4)
     const int xr = tid >> 1, kc = (tid & 1) * 4;
     const int x = x0 + xr, k = k0 + kc;
-    float v[4] = {0.f, 0.f, 0.f, 0.f};
     if (x < Xext && k < kend) {
       const float* src = base + opnd_offset(o, x, k);
       const bool vec = (k + 3 < kend) && ((reinterpret_cast<uintptr_t>(src) & 15) == 0) &&
@@ -411,6 +411,15 @@ __device__ __forceinline__ void load_slice(float (*s)[BM], const GemmOperand& o,
           if (k + e < kend) v[e] = base[opnd_offset(o, x, k + e)];
       }
     }
+  }
+}
+__device__ __forceinline__ void store_slice(float (*s)[BM], const GemmOperand& o, const float* v, int tid) {
+  if (!o.kmajor) {
+    const int kr = tid >> 5, xc = (tid & 31) * 4;
+    *reinterpret_cast<float4*>(&s[kr][xc]) = make_float4(v[0], v[1], v[2], v[3]);
+  } else {
+    // stored transposed
+    const int xr = tid >> 1, kc = (tid & 1) * 4;
 #pragma unroll
     for (int e = 0; e < 4; ++e) s[kc + e][xr] = v[e];
   }
@@ -423,6 +432,7 @@ __global__ void __launch_bounds__(256, 2) sgemm_kernel(GemmParams p) {
   __shared__ __align__(16) float Bs[2][BK][BN];
   const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
   const int m0 = blockIdx.y * BM, n0 = blockIdx.x * BN;
+  if (p.sym && blockIdx.x > blockIdx.y) return;   // mirrored from the tile below the diagonal
   const int bz = blockIdx.z;
   const int b = bz / p.splits, split = bz - b * p.splits;
   const int kbeg = split * p.kchunk;
@@ -435,16 +445,20 @@ __global__ void __launch_bounds__(256, 2) sgemm_kernel(GemmParams p) {
 #pragma unroll
     for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
   const int ntiles = kend > kbeg ? (kend - kbeg + BK - 1) / BK : 0;
+  float va[4], vb[4];
   if (ntiles > 0) {
-    load_slice(As[0], p.A, A, m0, kbeg, p.M, kend, tid);
-    load_slice(Bs[0], p.B, B, n0, kbeg, p.N, kend, tid);
+    fetch_slice(va, p.A, A, m0, kbeg, p.M, kend, tid);
+    fetch_slice(vb, p.B, B, n0, kbeg, p.N, kend, tid);
+    store_slice(As[0], p.A, va, tid);
+    store_slice(Bs[0], p.B, vb, tid);
   }
   __syncthreads();
   for (int t = 0; t < ntiles; ++t) {
     const int cur = t & 1;
-    if (t + 1 < ntiles) {
-      load_slice(As[cur ^ 1], p.A, A, m0, kbeg + (t + 1) * BK, p.M, kend, tid);
-      load_slice(Bs[cur ^ 1], p.B, B, n0, kbeg + (t + 1) * BK, p.N, kend, tid);
+    const bool more = t + 1 < ntiles;
+    if (more) {
+      fetch_slice(va, p.A, A, m0, kbeg + (t + 1) * BK, p.M, kend, tid);
+      fetch_slice(vb, p.B, B, n0, kbeg + (t + 1) * BK, p.N, kend, tid);
     }
 #pragma unroll
     for (int kk = 0; kk < BK; ++kk) {
@@ -459,6 +473,11 @@ __global__ void __launch_bounds__(256, 2) sgemm_kernel(GemmParams p) {
       for (int i = 0; i < 8; ++i)
 #pragma unroll
         for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(a[i], bb[j], acc[i][j]);
+    }
+    // the other buffer was last read before the previous barrier
+    if (more) {
+      store_slice(As[cur ^ 1], p.A, va, tid);
+      store_slice(Bs[cur ^ 1], p.B, vb, tid);
     }
     __syncthreads();
   }

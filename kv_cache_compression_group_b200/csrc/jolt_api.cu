@@ -15,6 +15,7 @@
 #include "misc.cuh"
 #include "umma.cuh"
 #include "eig_cluster.cuh"
+#include "chol.cuh"
 
 using namespace jolt;
 
@@ -360,7 +361,8 @@ jolt_status make_plan(const jolt_shape* sh, const jolt_options* op, Plan* p) {
   if (op->method == JOLT_RANDOMIZED || p->m_side) {
     p->o_gpart = b.take((size_t)NU * p->qr_split_max * kq * kq * 4);
     p->o_G = b.take((size_t)NU * kq * kq * 8);
-    p->o_Lr = b.take((size_t)NU * kq * kq * 4);   // L as fp32 row-major
+    // L as fp32 row-major, or (k <= 256) the transposed inverse of L at the padded width
+    p->o_Lr = b.take((size_t)NU * round_up(kq, 32) * round_up(kq, 32) * 4);
     p->o_ptrs = b.take((size_t)NU * 8 + 64);
     p->o_Linv = b.take((size_t)NU * round_up(kq, 32) * 32 * 4);   // inverses of the 32 x 32 diagonal blocks
   }
@@ -552,6 +554,8 @@ jolt_status cholqr_batched(const Ctx& c, float* Y, long long m, int k, int ld, i
   const int gld = ld;
   if (k > 1024) return fail(JOLT_ERR_UNSUPPORTED_SHAPE, "Cholesky QR of more than 1024 columns");
   for (int pass = 0; pass < passes; ++pass) {
+    const long long n = (long long)k * gld;
+    {
     ProfScope ps1("qr_gram", c.st, p.NU);
     GemmParams g;
     g.M = k;
@@ -572,17 +576,42 @@ jolt_status cholqr_batched(const Ctx& c, float* Y, long long m, int k, int ld, i
     g.c_type = 0;
     g.sym = true;
     JTRY(gemm(g, 1, 1, c.st));
-    const long long n = (long long)k * gld;
     count_launch(), reduce_splits_sym_kernel<float><<<grid1d((long long)p.NU * k * k), 256, 0, c.st>>>(
         gpart, G, p.NU, ns, k, gld, sgemm_detail::BM);
+    }
     float* Lr = c.at<float>(p.o_Lr);
     float* Dinv = c.at<float>(p.o_Linv);
     const int nbk = (int)ceil_div(k, TS_NB);
     const long long sL = (long long)k * gld, sD = (long long)nbk * TS_NB * TS_NB;
-    count_launch(), sanitize_sym_batched_kernel<<<p.NU, 1024, 0, c.st>>>(G, k, gld, n, c.status());
-    count_launch(), ptr_array_kernel<<<1, 64, 0, c.st>>>(ptrs, G, n, p.NU);
-    CUDA_TRY(cudaGetLastError());
+    if (k <= CF_MAXK && ld % 4 == 0) {
+      // own factor, block-column inverse and inverse product (chol.cuh; 16-byte row loads)
+      const int kq32 = (int)round_up(k, 32);
+      float* WT = Lr;
+      const long long sW = (long long)kq32 * kq32;
+      {
+        ProfScope ps2("qr_factor", c.st, p.NU);
+        CUDA_TRY(cudaFuncSetAttribute(chol_factor_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)chol_factor_smem()));
+        count_launch(), chol_factor_kernel<<<p.NU, CF_THREADS, chol_factor_smem(), c.st>>>(G, k, gld, n, c.status());
+        CUDA_TRY(cudaGetLastError());
+        CUDA_TRY(cudaFuncSetAttribute(tri_inv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)tri_inv_smem()));
+        count_launch(), tri_inv_kernel<<<dim3(nbk, p.NU), CF_THREADS, tri_inv_smem(), c.st>>>(G, k, gld, n, WT, kq32,
+                                                                                               sW);
+        CUDA_TRY(cudaGetLastError());
+      }
+      ProfScope ps3("qr_trsm", c.st, p.NU);
+      const size_t sm = trsm_inv_smem(kq32);
+      CUDA_TRY(cudaFuncSetAttribute(trsm_inv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm));
+      count_launch(), trsm_inv_kernel<<<dim3((unsigned)ceil_div(m, TI_RB), p.NU), CF_THREADS, sm, c.st>>>(
+          Y, m, k, ld, m * ld, WT, kq32, sW);
+      CUDA_TRY(cudaGetLastError());
+      continue;
+    }
     {
+      count_launch(), sanitize_sym_batched_kernel<<<p.NU, 1024, 0, c.st>>>(G, k, gld, n, c.status());
+      count_launch(), ptr_array_kernel<<<1, 64, 0, c.st>>>(ptrs, G, n, p.NU);
+      CUDA_TRY(cudaGetLastError());
       ProfScope ps2("qr_potrf", c.st, p.NU);
       SOLVER_TRY(cusolverDnDpotrfBatched(s->h, CUBLAS_FILL_MODE_LOWER, k, ptrs, gld, info, p.NU));
       count_launch(), info_check_kernel<<<(unsigned)ceil_div(p.NU, 32), 32, 0, c.st>>>(info, p.NU, c.status(),
