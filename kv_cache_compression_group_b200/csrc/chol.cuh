@@ -21,7 +21,6 @@ constexpr int CF_NB = 32;
 constexpr int CF_MAXK = 256;
 constexpr int CF_THREADS = 256;
 constexpr int CF_P = CF_NB + 1;   // shared-memory pitch (doubles)
-inline size_t chol_factor_smem() { return 3 * (size_t)CF_MAXK * CF_P * sizeof(double); }
 
 // asynchronous global -> shared copies (the staging loads of all three kernels stay in flight
 // together instead of one round trip per element); src_bytes < size zero-fills the rest
@@ -41,91 +40,83 @@ __device__ __forceinline__ void cf_wait() {
   asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
 }
 
+// Shared memory of the factor: the block column P (R x 32), the factored diagonal block L11,
+// its inverse (stored transposed) and the finished columns left of the block column
+// (R x J0, pitch J0 + 1), whose largest size for k <= 256 is 128 x 129 at J0 = 128.
+constexpr int CF_LEFT_MAX = 128 * 129;
+inline size_t chol_factor_smem() {
+  return ((size_t)CF_MAXK * CF_P + 2 * (size_t)CF_NB * CF_P + CF_LEFT_MAX) * sizeof(double);
+}
+
 // Non-finite Gram entries (or one met earlier in the cache): G := I (so W = I) and
 // DEV_ERR_NONFINITE.  A pivot that is not positive: DEV_ERR_FACTOR, the pivot taken as 1.
+// Per block column J (rows J0..k, R of them), all 256 threads in every phase:
+//   1. the finished columns 0..J0 of those rows are copied to shared memory in one batch;
+//   2. the block column of the Gram minus their products (registers, 8 x 4 per thread);
+//   3. the diagonal block factored column by column, one barrier per pivot;
+//   4. its inverse by right-looking forward substitution, one barrier per row;
+//   5. the rows below: L21 = A21 inv(L11)^T, 28 rows x 1 column per thread;
+//   6. L21 to the Gram's lower triangle, inv(L11) to the upper part of its diagonal block.
 __global__ void __launch_bounds__(CF_THREADS, 1)
     chol_factor_kernel(double* G, int k, long long gld, long long sG, uint32_t* status) {
   extern __shared__ __align__(16) double cf_sm[];
-  double* P = cf_sm;                      // [row - J0][col - J0] of the block column
-  double* const Lb0 = cf_sm + CF_MAXK * CF_P;   // two buffers [row - J0][q]: 32 finished columns
+  double* P = cf_sm;                      // [row - J0][col - J0]
+  double* Ls = P + CF_MAXK * CF_P;        // L11 [r][c]
+  double* XT = Ls + CF_NB * CF_P;         // inv(L11) transposed: XT[c][r] = inv(L11)[r][c]
+  double* Lleft = XT + CF_NB * CF_P;      // [row - J0][q], q < J0
   __shared__ double rdiag[CF_NB];
   __shared__ int fail;
+  constexpr int NW = CF_THREADS / 32;
   const int u = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   double* Gu = G + (long long)u * sG;
   const int nbk = (k + CF_NB - 1) / CF_NB;
-
-  constexpr int NW = CF_THREADS / 32;
   int bad = (tid == 0 && (*status & DEV_ERR_NONFINITE)) ? 1 : 0;
-  for (int c = warp; c < k; c += NW) {
-    double v[CF_MAXK / 32];
-#pragma unroll
-    for (int t = 0; t < CF_MAXK / 32; ++t) v[t] = lane + 32 * t < k ? Gu[(long long)c * gld + lane + 32 * t] : 0.0;
-#pragma unroll
-    for (int t = 0; t < CF_MAXK / 32; ++t)
-      if (!isfinite(v[t])) bad = 1;
-  }
   if (tid == 0) fail = 0;
-  if (__syncthreads_or(bad)) {
-    if (tid == 0) raise_status(status, DEV_ERR_NONFINITE);
-    for (int c = warp; c < k; c += NW)
-      for (int i = lane; i < k; i += 32) Gu[(long long)c * gld + i] = i == c ? 1.0 : 0.0;
-    return;
-  }
 
   const int tc = tid & 7, tr = tid >> 3;   // update tile: columns tc + 8 j, rows tr + 32 m
   for (int J = 0; J < nbk; ++J) {
-    const int J0 = J * CF_NB, nb = min(CF_NB, k - J0), R = k - J0;
+    const int J0 = J * CF_NB, nb = min(CF_NB, k - J0), R = k - J0, lp = J0 + 1;
+    // 1. L[J0 + lr][q], q < J0 (written before the barrier that ended block column q / 32)
+    for (int q = warp; q < J0; q += NW) {
+      const double* src = Gu + (long long)q * gld + J0;
+#pragma unroll
+      for (int t = 0; t < CF_MAXK / 32; ++t) {
+        const int lr = lane + 32 * t;
+        if (lr < R) cf_cp8(Lleft + lr * lp + q, src + lr);
+      }
+    }
+    cf_commit();
+    // 2. the Gram's block column through its symmetric upper part (never overwritten there);
+    //    every Gram entry is read here once up to symmetry, so the finiteness check is here
     double acc[8][4];
-    // the Gram's block column, read through the symmetric upper part (rows and columns
-    // >= J0 there are not written before this block column is done)
 #pragma unroll
     for (int m = 0; m < 8; ++m)
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const int lr = tr + 32 * m, c = tc + 8 * j;
         acc[m][j] = (lr < R && c < nb) ? Gu[(long long)(J0 + lr) * gld + J0 + c] : 0.0;
+        if (!isfinite(acc[m][j])) bad = 1;
       }
-    // finished block column Q, rows J0.. (written to the lower triangle before the barrier
-    // that ended block column Q) -> buffer
-    auto stage = [&](int Q, double* buf) {
+    cf_wait<0>();
+    if (__syncthreads_or(bad)) {
+      if (tid == 0) raise_status(status, DEV_ERR_NONFINITE);
+      for (int c = warp; c < k; c += NW)
+        for (int i = lane; i < k; i += 32) Gu[(long long)c * gld + i] = i == c ? 1.0 : 0.0;
+      return;
+    }
+#pragma unroll 2
+    for (int q = 0; q < J0; ++q) {
+      double b[4];
 #pragma unroll
-      for (int s = 0; s < CF_NB / NW; ++s) {
-        const int q = warp + NW * s;
-        const double* src = Gu + (long long)(Q * CF_NB + q) * gld + J0;
+      for (int j = 0; j < 4; ++j) b[j] = Lleft[(tc + 8 * j) * lp + q];
 #pragma unroll
-        for (int t = 0; t < CF_MAXK / 32; ++t) {
-          const int lr = lane + 32 * t;
-          if (lr < R) cf_cp8(buf + lr * CF_P + q, src + lr);
+      for (int m = 0; m < 8; ++m) {
+        if (32 * m < R) {
+          const double a = Lleft[(tr + 32 * m) * lp + q];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) acc[m][j] = fma(-a, b[j], acc[m][j]);
         }
       }
-      cf_commit();
-    };
-    if (J > 0) stage(0, Lb0);
-    for (int Q = 0; Q < J; ++Q) {
-      // the buffer of chunk Q + 1 was last read before the barrier ending chunk Q - 1
-      if (Q + 1 < J) {
-        stage(Q + 1, Lb0 + ((Q + 1) & 1) * (CF_MAXK * CF_P));
-        cf_wait<1>();
-      } else {
-        cf_wait<0>();
-      }
-      __syncthreads();
-      const double* Lc = Lb0 + (Q & 1) * (CF_MAXK * CF_P);
-#pragma unroll 4
-      for (int q = 0; q < CF_NB; ++q) {
-        double b[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) b[j] = Lc[(tc + 8 * j) * CF_P + q];
-#pragma unroll
-        for (int m = 0; m < 8; ++m) {
-          if (32 * m < R) {
-            const double a = Lc[(tr + 32 * m) * CF_P + q];
-#pragma unroll
-            for (int j = 0; j < 4; ++j) acc[m][j] = fma(-a, b[j], acc[m][j]);
-          }
-        }
-      }
-      __syncthreads();
     }
 #pragma unroll
     for (int m = 0; m < 8; ++m)
@@ -135,78 +126,82 @@ __global__ void __launch_bounds__(CF_THREADS, 1)
         if (lr < R && c < nb) P[lr * CF_P + c] = acc[m][j];
       }
     __syncthreads();
-    // diagonal block: unblocked Cholesky by warp 0, lane r holding row r in registers
-    if (warp == 0) {
-      double a[CF_NB];
+    // 3. diagonal block: thread (r = tid / 8, s = tid % 8) updates columns s + 8 i of row r;
+    //    a step reads only column c and writes only columns > c
+    {
+      const int r = tid >> 3, s8 = tid & 7;
+      for (int c = 0; c < nb; ++c) {
+        const double piv = P[c * CF_P + c];
+        const bool ok = piv > 0.0 && isfinite(piv);
+        const double rd = ok ? rsqrt(piv) : 1.0;
+        if (r > c && r < nb) {
+          const double lrc = P[r * CF_P + c] * rd;   // L[r][c]
 #pragma unroll
-      for (int c = 0; c < CF_NB; ++c) a[c] = (lane < nb && c <= lane) ? P[lane * CF_P + c] : 0.0;
-#pragma unroll
-      for (int c = 0; c < CF_NB; ++c) {
-        if (c < nb) {
-          const double piv = __shfl_sync(0xffffffffu, a[c], c);
-          const bool ok = piv > 0.0 && isfinite(piv);
-          const double rd = ok ? rsqrt(piv) : 1.0;
-          if (lane == 0 && !ok) fail = 1;
-          if (lane == c) {
-            a[c] = ok ? piv * rd : 1.0;
-            rdiag[c] = rd;
-          } else if (lane > c) {
-            a[c] *= rd;
+          for (int i = 0; i < 4; ++i) {
+            const int c2 = s8 + 8 * i;
+            if (c2 > c && c2 <= r) P[r * CF_P + c2] = fma(-lrc, P[c2 * CF_P + c] * rd, P[r * CF_P + c2]);
           }
-#pragma unroll
-          for (int c2 = c + 1; c2 < CF_NB; ++c2) {
-            const double l2 = __shfl_sync(0xffffffffu, a[c], c2);   // L[c2][c]
-            if (lane >= c2) a[c2] = fma(-a[c], l2, a[c2]);
-          }
+          if (s8 == 0) Ls[r * CF_P + c] = lrc;
         }
+        if (tid == 0) {
+          Ls[c * CF_P + c] = ok ? piv * rd : 1.0;
+          rdiag[c] = rd;
+          if (!ok) fail = 1;
+        }
+        __syncthreads();
       }
-#pragma unroll
-      for (int c = 0; c < CF_NB; ++c)
-        if (lane < nb && c <= lane) P[lane * CF_P + c] = a[c];
     }
-    __syncthreads();
-    const int nbelow = R - nb;   // <= 224: threads of warps 0..6
-    if (tid < nbelow) {
-      // row of L below the diagonal block: x L_JJ^T = g (forward substitution)
-      double* row = P + (nb + tid) * CF_P;
-      double x[CF_NB];
-#pragma unroll
-      for (int c = 0; c < CF_NB; ++c) x[c] = c < nb ? row[c] : 0.0;
-#pragma unroll
-      for (int c = 0; c < CF_NB; ++c) {
-        if (c < nb) {
-          x[c] *= rdiag[c];
-#pragma unroll
-          for (int c2 = c + 1; c2 < CF_NB; ++c2)
-            if (c2 < nb) x[c2] = fma(-x[c], P[c2 * CF_P + c], x[c2]);
+    // 4. inv(L11): thread (column j = lane, rows w + 8 s) keeps its rows' running sums; row r
+    //    is final once the rows above it are, and its owner publishes it
+    {
+      // running sums of rows warp, warp + 8, warp + 16, warp + 24 (scalars: kept in registers)
+      double x0 = (warp == lane && lane < nb) ? 1.0 : 0.0, x1 = (warp + 8 == lane && lane < nb) ? 1.0 : 0.0;
+      double x2 = (warp + 16 == lane && lane < nb) ? 1.0 : 0.0, x3 = (warp + 24 == lane && lane < nb) ? 1.0 : 0.0;
+      for (int r = 0; r < nb; ++r) {
+        if (warp == (r & 7)) {
+          const int s4 = r >> 3;
+          const double xv = s4 == 0 ? x0 : s4 == 1 ? x1 : s4 == 2 ? x2 : x3;
+          XT[lane * CF_P + r] = (lane <= r) ? xv * rdiag[r] : 0.0;
         }
+        __syncthreads();
+        const double xr = XT[lane * CF_P + r];
+        if (warp > r && warp < nb) x0 = fma(-Ls[warp * CF_P + r], xr, x0);
+        if (warp + 8 > r && warp + 8 < nb) x1 = fma(-Ls[(warp + 8) * CF_P + r], xr, x1);
+        if (warp + 16 > r && warp + 16 < nb) x2 = fma(-Ls[(warp + 16) * CF_P + r], xr, x2);
+        if (warp + 24 > r && warp + 24 < nb) x3 = fma(-Ls[(warp + 24) * CF_P + r], xr, x3);
       }
+    }
+    // 5. rows below the diagonal block: L21[lr][c] = sum_{q <= c} A21[lr][q] inv(L11)[c][q]
+    const int nbelow = R - nb;
+    double o[(CF_MAXK - CF_NB) / NW];
 #pragma unroll
-      for (int c = 0; c < CF_NB; ++c)
-        if (c < nb) row[c] = x[c];
-    } else if (warp == CF_THREADS / 32 - 1) {
-      // inverse of the diagonal block, lane = column (forward substitution), stored as
-      // W[J0 + r][J0 + lane] at G[(J0 + r) * gld + J0 + lane] for lane <= r
-      double x[CF_NB];
+    for (int t = 0; t < (CF_MAXK - CF_NB) / NW; ++t) o[t] = 0.0;
+    if (nbelow > 0) {
+#pragma unroll 2
+      for (int q = 0; q < nb; ++q) {
+        const double xq = XT[q * CF_P + lane];   // inv(L11)[lane][q]
 #pragma unroll
-      for (int r = 0; r < CF_NB; ++r) {
-        double v = (r == lane) ? 1.0 : 0.0;
-        if (r < nb && lane < nb) {
-#pragma unroll
-          for (int q = 0; q < r; ++q) v = fma(-P[r * CF_P + q], x[q], v);
-          x[r] = lane <= r ? v * rdiag[r] : 0.0;
-          if (lane <= r) Gu[(long long)(J0 + r) * gld + J0 + lane] = x[r];
-        } else {
-          x[r] = 0.0;
+        for (int t = 0; t < (CF_MAXK - CF_NB) / NW; ++t) {
+          const int lr = nb + warp + NW * t;
+          if (NW * t < nbelow) o[t] = fma(lr < R ? P[lr * CF_P + q] : 0.0, xq, o[t]);
         }
       }
     }
     __syncthreads();
-    // the rows below the diagonal block to the lower triangle (read by later block columns
-    // and by the inverse)
+    // 6. outputs
+#pragma unroll
+    for (int t = 0; t < (CF_MAXK - CF_NB) / NW; ++t) {
+      const int lr = nb + warp + NW * t;
+      if (lr < R && lane < nb) P[lr * CF_P + lane] = o[t];
+    }
+    __syncthreads();
     for (int c = warp; c < nb; c += NW) {
       double* dst = Gu + (long long)(J0 + c) * gld + J0;
       for (int lr = nb + lane; lr < R; lr += 32) dst[lr] = P[lr * CF_P + c];
+    }
+    for (int idx = tid; idx < CF_NB * CF_NB; idx += CF_THREADS) {
+      const int r = idx / CF_NB, c = idx % CF_NB;
+      if (r < nb && c <= r) Gu[(long long)(J0 + r) * gld + J0 + c] = XT[c * CF_P + r];
     }
     __syncthreads();
   }
@@ -326,11 +321,13 @@ __global__ void __launch_bounds__(CF_THREADS, 2)
     cf_commit();
   };
   stage(0, wt0);   // committed together with the panel
-  float acc[8][8];
+  // accumulators of column blocks 2p and 2p + 1 side by side: packed fp32 FMAs (two IEEE
+  // fmas each, in the same order as scalar ones)
+  float2 acc[8][4];
 #pragma unroll
   for (int i = 0; i < 8; ++i)
 #pragma unroll
-    for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
+    for (int p = 0; p < 4; ++p) acc[i][p] = make_float2(0.f, 0.f);
   const int nch = (k + TI_QC - 1) / TI_QC;
   for (int ch = 0; ch < nch; ++ch) {
     const int q0 = ch * TI_QC;
@@ -343,26 +340,32 @@ __global__ void __launch_bounds__(CF_THREADS, 2)
     }
     __syncthreads();
     const float* wt = wt0 + (ch & 1) * (TI_QC * kq);
-    const int jmin = q0 / 32;   // column blocks j with 32 j + 31 < q0 meet only zeros of W
+    // column blocks j with 32 j + 31 < q0 meet only zeros of W: a pair is skipped when both
+    // of its blocks are (an inactive block of a live pair adds 0 * y = +0)
+    const int jmin = q0 / 32;
 #pragma unroll 1
     for (int q = 0; q < TI_QC; q += 4) {
-      float w[8][4];
+      float2 w[4][4];
 #pragma unroll
-      for (int j = 0; j < 8; ++j)
+      for (int pr = 0; pr < 4; ++pr)
 #pragma unroll
-        for (int e = 0; e < 4; ++e) w[j][e] = (j >= jmin && j < nj) ? wt[(q + e) * kq + lane + 32 * j] : 0.f;
+        for (int e = 0; e < 4; ++e) {
+          const int j0 = 2 * pr, j1 = 2 * pr + 1;
+          w[pr][e] = make_float2((j0 >= jmin && j0 < nj) ? wt[(q + e) * kq + lane + 32 * j0] : 0.f,
+                                 (j1 >= jmin && j1 < nj) ? wt[(q + e) * kq + lane + 32 * j1] : 0.f);
+        }
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         const float4 y = *reinterpret_cast<const float4*>(panel + (warp * 8 + i) * P + q0 + q);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          if (j >= jmin && j < nj) {
-            float a = acc[i][j];
-            a = fmaf(y.x, w[j][0], a);
-            a = fmaf(y.y, w[j][1], a);
-            a = fmaf(y.z, w[j][2], a);
-            a = fmaf(y.w, w[j][3], a);
-            acc[i][j] = a;
+        for (int pr = 0; pr < 4; ++pr) {
+          if (2 * pr + 1 >= jmin && 2 * pr < nj) {
+            float2 a = acc[i][pr];
+            a = __ffma2_rn(make_float2(y.x, y.x), w[pr][0], a);
+            a = __ffma2_rn(make_float2(y.y, y.y), w[pr][1], a);
+            a = __ffma2_rn(make_float2(y.z, y.z), w[pr][2], a);
+            a = __ffma2_rn(make_float2(y.w, y.w), w[pr][3], a);
+            acc[i][pr] = a;
           }
         }
       }
@@ -374,9 +377,10 @@ __global__ void __launch_bounds__(CF_THREADS, 2)
     const long long rr = r0 + warp * 8 + i;
     if (rr >= m) continue;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int c = lane + 32 * j;
-      if (j < nj && c < k) Yu[rr * ld + c] = acc[i][j];
+    for (int pr = 0; pr < 4; ++pr) {
+      const int c0 = lane + 64 * pr, c1 = c0 + 32;
+      if (2 * pr < nj && c0 < k) Yu[rr * ld + c0] = acc[i][pr].x;
+      if (2 * pr + 1 < nj && c1 < k) Yu[rr * ld + c1] = acc[i][pr].y;
     }
   }
 }
