@@ -50,14 +50,15 @@ inline size_t chol_factor_smem() {
 
 // Non-finite Gram entries (or one met earlier in the cache): G := I (so W = I) and
 // DEV_ERR_NONFINITE.  A pivot that is not positive: DEV_ERR_FACTOR, the pivot taken as 1.
-// Per block column J (rows J0..k, R of them), all 256 threads in every phase:
+// Per block column J (rows J0..k, R of them), all 512 threads in every phase:
 //   1. the finished columns 0..J0 of those rows are copied to shared memory in one batch;
-//   2. the block column of the Gram minus their products (registers, 8 x 4 per thread);
+//   2. the block column of the Gram minus their products (registers, 4 x 4 per thread);
 //   3. the diagonal block factored column by column, one barrier per pivot;
 //   4. its inverse by right-looking forward substitution, one barrier per row;
-//   5. the rows below: L21 = A21 inv(L11)^T, 28 rows x 1 column per thread;
+//   5. the rows below: L21 = A21 inv(L11)^T, 7 rows x 2 columns per thread;
 //   6. L21 to the Gram's lower triangle, inv(L11) to the upper part of its diagonal block.
-__global__ void __launch_bounds__(CF_THREADS, 1)
+constexpr int CF_FT = 512;   // threads of the factor kernel
+__global__ void __launch_bounds__(CF_FT, 1)
     chol_factor_kernel(double* G, int k, long long gld, long long sG, uint32_t* status) {
   extern __shared__ __align__(16) double cf_sm[];
   double* P = cf_sm;                      // [row - J0][col - J0]
@@ -66,14 +67,14 @@ __global__ void __launch_bounds__(CF_THREADS, 1)
   double* Lleft = XT + CF_NB * CF_P;      // [row - J0][q], q < J0
   __shared__ double rdiag[CF_NB];
   __shared__ int fail;
-  constexpr int NW = CF_THREADS / 32;
+  constexpr int NW = CF_FT / 32;
   const int u = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   double* Gu = G + (long long)u * sG;
   const int nbk = (k + CF_NB - 1) / CF_NB;
   int bad = (tid == 0 && (*status & DEV_ERR_NONFINITE)) ? 1 : 0;
   if (tid == 0) fail = 0;
 
-  const int tc = tid & 7, tr = tid >> 3;   // update tile: columns tc + 8 j, rows tr + 32 m
+  const int tc = tid & 7, tr = tid >> 3;   // update tile: columns tc + 8 j, rows tr + 64 m
   for (int J = 0; J < nbk; ++J) {
     const int J0 = J * CF_NB, nb = min(CF_NB, k - J0), R = k - J0, lp = J0 + 1;
     // 1. L[J0 + lr][q], q < J0 (written before the barrier that ended block column q / 32)
@@ -88,12 +89,12 @@ __global__ void __launch_bounds__(CF_THREADS, 1)
     cf_commit();
     // 2. the Gram's block column through its symmetric upper part (never overwritten there);
     //    every Gram entry is read here once up to symmetry, so the finiteness check is here
-    double acc[8][4];
+    double acc[4][4];
 #pragma unroll
-    for (int m = 0; m < 8; ++m)
+    for (int m = 0; m < 4; ++m)
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        const int lr = tr + 32 * m, c = tc + 8 * j;
+        const int lr = tr + 64 * m, c = tc + 8 * j;
         acc[m][j] = (lr < R && c < nb) ? Gu[(long long)(J0 + lr) * gld + J0 + c] : 0.0;
         if (!isfinite(acc[m][j])) bad = 1;
       }
@@ -110,26 +111,27 @@ __global__ void __launch_bounds__(CF_THREADS, 1)
 #pragma unroll
       for (int j = 0; j < 4; ++j) b[j] = Lleft[(tc + 8 * j) * lp + q];
 #pragma unroll
-      for (int m = 0; m < 8; ++m) {
-        if (32 * m < R) {
-          const double a = Lleft[(tr + 32 * m) * lp + q];
+      for (int m = 0; m < 4; ++m) {
+        if (64 * m < R) {
+          // rows past R would lie beyond the staged block (64-row granularity)
+          const double a = tr + 64 * m < R ? Lleft[(tr + 64 * m) * lp + q] : 0.0;
 #pragma unroll
           for (int j = 0; j < 4; ++j) acc[m][j] = fma(-a, b[j], acc[m][j]);
         }
       }
     }
 #pragma unroll
-    for (int m = 0; m < 8; ++m)
+    for (int m = 0; m < 4; ++m)
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        const int lr = tr + 32 * m, c = tc + 8 * j;
+        const int lr = tr + 64 * m, c = tc + 8 * j;
         if (lr < R && c < nb) P[lr * CF_P + c] = acc[m][j];
       }
     __syncthreads();
-    // 3. diagonal block: thread (r = tid / 8, s = tid % 8) updates columns s + 8 i of row r;
-    //    a step reads only column c and writes only columns > c
+    // 3. diagonal block: thread (r = tid / 16, s = tid % 16) updates columns s and s + 16 of
+    //    row r; a step reads only column c and writes only columns > c
     {
-      const int r = tid >> 3, s8 = tid & 7;
+      const int r = tid >> 4, s16 = tid & 15;
       for (int c = 0; c < nb; ++c) {
         const double piv = P[c * CF_P + c];
         const bool ok = piv > 0.0 && isfinite(piv);
@@ -137,11 +139,11 @@ __global__ void __launch_bounds__(CF_THREADS, 1)
         if (r > c && r < nb) {
           const double lrc = P[r * CF_P + c] * rd;   // L[r][c]
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int c2 = s8 + 8 * i;
+          for (int i = 0; i < 2; ++i) {
+            const int c2 = s16 + 16 * i;
             if (c2 > c && c2 <= r) P[r * CF_P + c2] = fma(-lrc, P[c2 * CF_P + c] * rd, P[r * CF_P + c2]);
           }
-          if (s8 == 0) Ls[r * CF_P + c] = lrc;
+          if (s16 == 0) Ls[r * CF_P + c] = lrc;
         }
         if (tid == 0) {
           Ls[c * CF_P + c] = ok ? piv * rd : 1.0;
@@ -151,55 +153,56 @@ __global__ void __launch_bounds__(CF_THREADS, 1)
         __syncthreads();
       }
     }
-    // 4. inv(L11): thread (column j = lane, rows w + 8 s) keeps its rows' running sums; row r
-    //    is final once the rows above it are, and its owner publishes it
+    // 4. inv(L11): thread (column j = lane, rows w and w + 16) keeps its rows' running sums;
+    //    row r is final once the rows above it are, and its owner publishes it
     {
-      // running sums of rows warp, warp + 8, warp + 16, warp + 24 (scalars: kept in registers)
-      double x0 = (warp == lane && lane < nb) ? 1.0 : 0.0, x1 = (warp + 8 == lane && lane < nb) ? 1.0 : 0.0;
-      double x2 = (warp + 16 == lane && lane < nb) ? 1.0 : 0.0, x3 = (warp + 24 == lane && lane < nb) ? 1.0 : 0.0;
+      double x0 = (warp == lane && lane < nb) ? 1.0 : 0.0, x1 = (warp + 16 == lane && lane < nb) ? 1.0 : 0.0;
       for (int r = 0; r < nb; ++r) {
-        if (warp == (r & 7)) {
-          const int s4 = r >> 3;
-          const double xv = s4 == 0 ? x0 : s4 == 1 ? x1 : s4 == 2 ? x2 : x3;
-          XT[lane * CF_P + r] = (lane <= r) ? xv * rdiag[r] : 0.0;
-        }
+        if (warp == (r & 15)) XT[lane * CF_P + r] = (lane <= r) ? (r < 16 ? x0 : x1) * rdiag[r] : 0.0;
         __syncthreads();
         const double xr = XT[lane * CF_P + r];
         if (warp > r && warp < nb) x0 = fma(-Ls[warp * CF_P + r], xr, x0);
-        if (warp + 8 > r && warp + 8 < nb) x1 = fma(-Ls[(warp + 8) * CF_P + r], xr, x1);
-        if (warp + 16 > r && warp + 16 < nb) x2 = fma(-Ls[(warp + 16) * CF_P + r], xr, x2);
-        if (warp + 24 > r && warp + 24 < nb) x3 = fma(-Ls[(warp + 24) * CF_P + r], xr, x3);
+        if (warp + 16 > r && warp + 16 < nb) x1 = fma(-Ls[(warp + 16) * CF_P + r], xr, x1);
       }
     }
-    // 5. rows below the diagonal block: L21[lr][c] = sum_{q <= c} A21[lr][q] inv(L11)[c][q]
-    const int nbelow = R - nb;
-    double o[(CF_MAXK - CF_NB) / NW];
+    // 5. rows below the diagonal block: L21[lr][c] = sum_{q <= c} A21[lr][q] inv(L11)[c][q];
+    //    thread: columns cl and cl + 16, rows nb + rg + 32 t
+    const int nbelow = R - nb, cl = tid & 15, rg = tid >> 4;
+    constexpr int RT = (CF_MAXK - CF_NB) / 32;   // 7
+    double o0[RT], o1[RT];
 #pragma unroll
-    for (int t = 0; t < (CF_MAXK - CF_NB) / NW; ++t) o[t] = 0.0;
+    for (int t = 0; t < RT; ++t) o0[t] = o1[t] = 0.0;
     if (nbelow > 0) {
 #pragma unroll 2
       for (int q = 0; q < nb; ++q) {
-        const double xq = XT[q * CF_P + lane];   // inv(L11)[lane][q]
+        const double xa = XT[q * CF_P + cl], xb = XT[q * CF_P + cl + 16];   // inv(L11)[c][q]
 #pragma unroll
-        for (int t = 0; t < (CF_MAXK - CF_NB) / NW; ++t) {
-          const int lr = nb + warp + NW * t;
-          if (NW * t < nbelow) o[t] = fma(lr < R ? P[lr * CF_P + q] : 0.0, xq, o[t]);
+        for (int t = 0; t < RT; ++t) {
+          const int lr = nb + rg + 32 * t;
+          if (32 * t < nbelow) {
+            const double a = lr < R ? P[lr * CF_P + q] : 0.0;
+            o0[t] = fma(a, xa, o0[t]);
+            o1[t] = fma(a, xb, o1[t]);
+          }
         }
       }
     }
     __syncthreads();
     // 6. outputs
 #pragma unroll
-    for (int t = 0; t < (CF_MAXK - CF_NB) / NW; ++t) {
-      const int lr = nb + warp + NW * t;
-      if (lr < R && lane < nb) P[lr * CF_P + lane] = o[t];
+    for (int t = 0; t < RT; ++t) {
+      const int lr = nb + rg + 32 * t;
+      if (lr < R) {
+        if (cl < nb) P[lr * CF_P + cl] = o0[t];
+        if (cl + 16 < nb) P[lr * CF_P + cl + 16] = o1[t];
+      }
     }
     __syncthreads();
     for (int c = warp; c < nb; c += NW) {
       double* dst = Gu + (long long)(J0 + c) * gld + J0;
       for (int lr = nb + lane; lr < R; lr += 32) dst[lr] = P[lr * CF_P + c];
     }
-    for (int idx = tid; idx < CF_NB * CF_NB; idx += CF_THREADS) {
+    for (int idx = tid; idx < CF_NB * CF_NB; idx += CF_FT) {
       const int r = idx / CF_NB, c = idx % CF_NB;
       if (r < nb && c <= r) Gu[(long long)(J0 + r) * gld + J0 + c] = XT[c * CF_P + r];
     }

@@ -592,7 +592,7 @@ jolt_status cholqr_batched(const Ctx& c, float* Y, long long m, int k, int ld, i
         ProfScope ps2("qr_factor", c.st, p.NU);
         CUDA_TRY(cudaFuncSetAttribute(chol_factor_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       (int)chol_factor_smem()));
-        count_launch(), chol_factor_kernel<<<p.NU, CF_THREADS, chol_factor_smem(), c.st>>>(G, k, gld, n, c.status());
+        count_launch(), chol_factor_kernel<<<p.NU, CF_FT, chol_factor_smem(), c.st>>>(G, k, gld, n, c.status());
         CUDA_TRY(cudaGetLastError());
         CUDA_TRY(cudaFuncSetAttribute(tri_inv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       (int)tri_inv_smem()));
