@@ -550,7 +550,16 @@ jolt_status cholqr_batched(const Ctx& c, float* Y, long long m, int k, int ld, i
   double* G = c.at<double>(p.o_G);
   double** ptrs = c.at<double*>(p.o_ptrs);
   int* info = c.at<int>(p.o_info);
-  const int ns = (int)ceil_div(m, 256);
+  // split-K chunk: 256 rows, halved (down to 64) while fewer than two CTAs per SM would run
+  // and the partial buffer (qr_split_max splits) still holds the splits
+  int kchunk = 256;
+  {
+    const long long nt = ceil_div(k, sgemm_detail::BM), tiles = nt * (nt + 1) / 2;
+    while (kchunk > 64 && (long long)p.NU * tiles * ceil_div(m, kchunk) < 2 * 148 &&
+           ceil_div(m, kchunk / 2) <= p.qr_split_max)
+      kchunk /= 2;
+  }
+  const int ns = (int)ceil_div(m, kchunk);
   const int gld = ld;
   if (k > 1024) return fail(JOLT_ERR_UNSUPPORTED_SHAPE, "Cholesky QR of more than 1024 columns");
   for (int pass = 0; pass < passes; ++pass) {
@@ -572,7 +581,7 @@ jolt_status cholqr_batched(const Ctx& c, float* Y, long long m, int k, int ld, i
     g.sbatchC = (long long)ns * k * gld;
     g.ssplitC = (long long)k * gld;
     g.splits = ns;
-    g.kchunk = 256;
+    g.kchunk = kchunk;
     g.c_type = 0;
     g.sym = true;
     JTRY(gemm(g, 1, 1, c.st));
