@@ -114,3 +114,12 @@ def test_struct_layouts():
     assert ctypes.sizeof(J.CShape) == 24
     assert ctypes.sizeof(J.COptions) == 4 * (3 + 3 * J.MAXC + 3)
     assert ctypes.sizeof(J.CUnitRecord) == 64
+
+
+def test_build_tracks_every_source_file():
+    """A kernel header missing from the rebuild check would leave a stale library in place."""
+    import os
+    from kv_cache_compression_group_b200 import build
+    on_disk = sorted(f for f in os.listdir(build.CSRC) if f.endswith((".cu", ".cuh")))
+    assert sorted(build.DEPS) == on_disk
+    assert all(s in build.DEPS for s in build.SOURCES)
