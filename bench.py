@@ -355,36 +355,76 @@ def main():
     value = ranks.aggregate_gbs(world, args.steps * len(RATIOS) * in_bytes, t_ms)
 
     # ---- end to end through the public API: pinned host in, blobs out ---------------------
+    # Every step copies its cache in from pinned host memory and its blobs out, inside the
+    # timed region. The copies run on a second stream, double-buffered: step i + 1's upload and
+    # step i's download overlap the compress of the neighbouring step. Events order every
+    # buffer reuse: an upload waits for the compress that last read its buffers, a download for
+    # the compress that wrote its blobs, and a compress for its upload. The upload into a slot
+    # is issued after that slot's previous download on the copy stream, so it also orders the
+    # compress that overwrites those blobs.
     Kh, Vh = K.pin_memory(), V.pin_memory()
-    Kbuf, Vbuf = torch.empty_like(Kd), torch.empty_like(Vd)
-    host_blobs = [torch.empty(bl.numel(), dtype=torch.uint8).pin_memory() for bl in blobs]
-    d2h = 0
+    Kb = [torch.empty_like(Kd), torch.empty_like(Kd)]
+    Vb = [torch.empty_like(Vd), torch.empty_like(Vd)]
+    dblobs = [blobs, [torch.empty_like(bl) for bl in blobs]]
+    host_blobs = [[torch.empty(bl.numel(), dtype=torch.uint8).pin_memory() for bl in blobs] for _ in range(2)]
+    cstream = torch.cuda.Stream(device=dev)
+    h2d_ev = [torch.cuda.Event(), torch.cuda.Event()]
+    done_ev = [torch.cuda.Event(), torch.cuda.Event()]
+    d2h = sum(bl.numel() for bl in blobs)
 
-    def e2e_step():
-        nonlocal d2h
-        Kbuf.copy_(Kh, non_blocking=True)
-        Vbuf.copy_(Vh, non_blocking=True)
-        step(Kbuf, Vbuf)
-        d2h = 0
-        for bl, hb in zip(blobs, host_blobs):
-            hb.copy_(bl, non_blocking=True)
-            d2h += bl.numel()
+    def upload(slot):
+        with torch.cuda.stream(cstream):
+            cstream.wait_event(done_ev[slot])
+            Kb[slot].copy_(Kh, non_blocking=True)
+            Vb[slot].copy_(Vh, non_blocking=True)
+            h2d_ev[slot].record(cstream)
 
-    for _ in range(max(1, args.warmup)):
-        e2e_step()
+    def download(slot):
+        with torch.cuda.stream(cstream):
+            cstream.wait_event(done_ev[slot])
+            for bl, hb in zip(dblobs[slot], host_blobs[slot]):
+                hb.copy_(bl, non_blocking=True)
+
+    def compute(slot):
+        stream.wait_event(h2d_ev[slot])
+        for b, bl in zip(budgets, dblobs[slot]):
+            comp.compress(Kb[slot], Vb[slot], b, seed, blob=bl)
+        done_ev[slot].record(stream)
+
+    def e2e_run(nsteps, start=None):
+        if start is not None:
+            cstream.wait_event(start)
+        upload(0)
+        for i in range(nsteps):
+            s = i % 2
+            if i + 1 < nsteps:
+                upload(1 - s)
+            compute(s)
+            download(s)
+        fin = torch.cuda.Event()
+        fin.record(cstream)
+        stream.wait_event(fin)
+
+    # each buffer slot's argument set runs directly once, is captured once, then replays
+    e2e_run(max(6, args.warmup))
     torch.cuda.synchronize()
+    for slot in range(2):
+        for b, bl in zip(budgets, dblobs[slot]):
+            _, total, _ = J.read_header(bl)
+            assert total <= b
     barrier()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for _ in range(args.steps):
-        e2e_step()
+    e2e_run(args.steps, start=e0)
     e1.record(stream)
     torch.cuda.synchronize()
     e_ms = ranks.max_over_ranks(e0.elapsed_time(e1), world, dev)
     e2e = {"value": ranks.aggregate_gbs(world, args.steps * len(RATIOS) * in_bytes, e_ms), "unit": "GB/s",
            "h2d_bytes_per_step": 2 * K.numel() * K.element_size(), "d2h_bytes_per_step": d2h,
-           "ms_per_step": e_ms / args.steps}
+           "ms_per_step": e_ms / args.steps,
+           "note": "copies on a second stream, double-buffered: step i+1's upload and step i's download "
+                   "overlap the neighbouring compress; all bytes of every step inside the timed region"}
 
     # ---- stage breakdown: a separate pass with per-stage events (these calls run without
     # the CUDA graphs of the timed region, so stage sums exceed the timed step) ------------
