@@ -1,0 +1,97 @@
+// Exact fp16 directed rounding and the quantiser step of the b-bit block quantiser.
+// Host and device: the device code is what the table and encode kernels run; the host
+// copy of the same source lets a CPU check compare it with the float64 definition.
+#pragma once
+
+#include <cuda_fp16.h>
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+namespace jolt {
+
+__host__ __device__ __forceinline__ uint32_t f32_bits(float x) {
+#ifdef __CUDA_ARCH__
+  return __float_as_uint(x);
+#else
+  uint32_t u;
+  memcpy(&u, &x, sizeof u);
+  return u;
+#endif
+}
+__host__ __device__ __forceinline__ float bits_f32(uint32_t u) {
+#ifdef __CUDA_ARCH__
+  return __uint_as_float(u);
+#else
+  float x;
+  memcpy(&x, &u, sizeof x);
+  return x;
+#endif
+}
+
+// ---------------------------------------------------------------------------------------
+// exact fp16 directed rounding and the quantiser step, in FP32-pipe integer / float ops
+// (fp16 normal values are the floats whose low 13 mantissa bits are zero; other ranges
+// go through the conversion instructions)
+// ---------------------------------------------------------------------------------------
+constexpr float kFp16MinNormal = 6.103515625e-05f;  // 2^-14
+constexpr float kFp16Max = 65504.f;
+
+// fp16 round toward -inf (as __float2half_rd)
+__host__ __device__ __forceinline__ float rd16(float x) {
+  const float ax = fabsf(x);
+  if (ax >= kFp16MinNormal && ax <= kFp16Max) {
+    uint32_t u = f32_bits(x);
+    if (x >= 0.f) u &= ~0x1FFFu;
+    else if (u & 0x1FFFu) u = (u | 0x1FFFu) + 1u;
+    return bits_f32(u);
+  }
+  return __half2float(__float2half_rd(x));
+}
+
+// fp16 round toward +inf of a positive float (as __float2half_ru)
+__host__ __device__ __forceinline__ float ru16_pos(float q) {
+  if (q >= kFp16MinNormal && q <= kFp16Max) {
+    uint32_t u = f32_bits(q);
+    if (u & 0x1FFFu) u = (u | 0x1FFFu) + 1u;
+    return bits_f32(u);
+  }
+  return __half2float(__float2half_ru(q));
+}
+
+// neighbouring fp16 values of a positive fp16 value s
+__host__ __device__ __forceinline__ float next16_up(float s) {
+  if (s >= kFp16MinNormal && s < kFp16Max) return bits_f32(f32_bits(s) + 0x2000u);
+  return __half2float(__ushort_as_half((unsigned short)(__half_as_ushort(__float2half_rn(s)) + 1)));
+}
+__host__ __device__ __forceinline__ float next16_down(float s) {
+  if (s > kFp16MinNormal && s <= kFp16Max) return bits_f32(f32_bits(s) - 0x2000u);
+  unsigned short h = __half_as_ushort(__float2half_rn(s));
+  return h ? __half2float(__ushort_as_half((unsigned short)(h - 1))) : 0.f;
+}
+
+// a >= mx - lo, decided exactly (R is the rounded difference)
+__host__ __device__ __forceinline__ bool ge_exact(float a, float mx, float lo, float R) {
+  if (a > R * 1.0000002384185791f) return true;
+  if (a < R * 0.9999997615814209f) return false;
+  return (double)a >= (double)mx - (double)lo;
+}
+
+// quantiser step: the smallest fp16 s with s * levels >= mx - lo exactly (the fp16
+// round-up of (mx - lo)/levels); 0 when mx <= lo.  A float estimate is corrected by one
+// fp16 step where needed.
+__host__ __device__ __forceinline__ float quant_step(float mx, float lo, float flev, float inv_lev) {
+  if (!(mx > lo)) return 0.f;
+  const float R = mx - lo;
+  float s = ru16_pos(R * inv_lev);
+  if (!(s <= kFp16Max)) return s;  // +inf: this block cannot be stored with this many bits
+  if (!ge_exact(s * flev, mx, lo, R)) {
+    s = next16_up(s);
+  } else {
+    float sp = next16_down(s);
+    if (sp > 0.f && ge_exact(sp * flev, mx, lo, R)) s = sp;
+  }
+  return s;
+}
+
+}  // namespace jolt

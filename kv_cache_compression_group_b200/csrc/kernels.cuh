@@ -10,6 +10,7 @@
 #include <type_traits>
 
 #include "common.cuh"
+#include "fp16_exact.cuh"
 #include "gemm.cuh"
 
 namespace jolt {
@@ -32,71 +33,6 @@ struct Cands {
   int nT, nD, nB;
   int rT[MAXC], rD[MAXC], bits[MAXC];
 };
-
-// ---------------------------------------------------------------------------------------
-// exact fp16 directed rounding and the quantiser step, in FP32-pipe integer / float ops
-// (fp16 normal values are the floats whose low 13 mantissa bits are zero; other ranges
-// go through the conversion instructions)
-// ---------------------------------------------------------------------------------------
-constexpr float kFp16MinNormal = 6.103515625e-05f;  // 2^-14
-constexpr float kFp16Max = 65504.f;
-
-// fp16 round toward -inf (as __float2half_rd)
-__device__ __forceinline__ float rd16(float x) {
-  const float ax = fabsf(x);
-  if (ax >= kFp16MinNormal && ax <= kFp16Max) {
-    uint32_t u = __float_as_uint(x);
-    if (x >= 0.f) u &= ~0x1FFFu;
-    else if (u & 0x1FFFu) u = (u | 0x1FFFu) + 1u;
-    return __uint_as_float(u);
-  }
-  return __half2float(__float2half_rd(x));
-}
-
-// fp16 round toward +inf of a positive float (as __float2half_ru)
-__device__ __forceinline__ float ru16_pos(float q) {
-  if (q >= kFp16MinNormal && q <= kFp16Max) {
-    uint32_t u = __float_as_uint(q);
-    if (u & 0x1FFFu) u = (u | 0x1FFFu) + 1u;
-    return __uint_as_float(u);
-  }
-  return __half2float(__float2half_ru(q));
-}
-
-// neighbouring fp16 values of a positive fp16 value s
-__device__ __forceinline__ float next16_up(float s) {
-  if (s >= kFp16MinNormal && s < kFp16Max) return __uint_as_float(__float_as_uint(s) + 0x2000u);
-  return __half2float(__ushort_as_half((unsigned short)(__half_as_ushort(__float2half_rn(s)) + 1)));
-}
-__device__ __forceinline__ float next16_down(float s) {
-  if (s > kFp16MinNormal && s <= kFp16Max) return __uint_as_float(__float_as_uint(s) - 0x2000u);
-  unsigned short h = __half_as_ushort(__float2half_rn(s));
-  return h ? __half2float(__ushort_as_half((unsigned short)(h - 1))) : 0.f;
-}
-
-// a >= mx - lo, decided exactly (R is the rounded difference)
-__device__ __forceinline__ bool ge_exact(float a, float mx, float lo, float R) {
-  if (a > R * 1.0000002384185791f) return true;
-  if (a < R * 0.9999997615814209f) return false;
-  return (double)a >= (double)mx - (double)lo;
-}
-
-// quantiser step: the smallest fp16 s with s * levels >= mx - lo exactly (the fp16
-// round-up of (mx - lo)/levels); 0 when mx <= lo.  A float estimate is corrected by one
-// fp16 step where needed.
-__device__ __forceinline__ float quant_step(float mx, float lo, float flev, float inv_lev) {
-  if (!(mx > lo)) return 0.f;
-  const float R = mx - lo;
-  float s = ru16_pos(R * inv_lev);
-  if (!(s <= kFp16Max)) return s;  // +inf: this block cannot be stored with this many bits
-  if (!ge_exact(s * flev, mx, lo, R)) {
-    s = next16_up(s);
-  } else {
-    float sp = next16_down(s);
-    if (sp > 0.f && ge_exact(sp * flev, mx, lo, R)) s = sp;
-  }
-  return s;
-}
 
 // round-half-even of d * inv to an integer-valued float: one FMA onto the 1.5*2^23 shift
 constexpr float kRoundShift = 12582912.0f;
