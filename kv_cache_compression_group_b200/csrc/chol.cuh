@@ -52,7 +52,8 @@ inline size_t chol_factor_smem() {
 // DEV_ERR_NONFINITE.  A pivot that is not positive: DEV_ERR_FACTOR, the pivot taken as 1.
 // Per block column J (rows J0..k, R of them), all 512 threads in every phase:
 //   1. the finished columns 0..J0 of those rows are copied to shared memory in one batch;
-//   2. the block column of the Gram minus their products (registers, 4 x 4 per thread);
+//   2. the block column of the Gram minus their products (registers, 4 x 4 per thread,
+//      the inner dimension split over the threads a short block column leaves idle);
 //   3. the diagonal block factored column by column, one barrier per pivot;
 //   4. its inverse by right-looking forward substitution, one barrier per row;
 //   5. the rows below: L21 = A21 inv(L11)^T, 7 rows x 2 columns per thread;
@@ -74,7 +75,6 @@ __global__ void __launch_bounds__(CF_FT, 1)
   int bad = (tid == 0 && (*status & DEV_ERR_NONFINITE)) ? 1 : 0;
   if (tid == 0) fail = 0;
 
-  const int tc = tid & 7, tr = tid >> 3;   // update tile: columns tc + 8 j, rows tr + 64 m
   for (int J = 0; J < nbk; ++J) {
     const int J0 = J * CF_NB, nb = min(CF_NB, k - J0), R = k - J0, lp = J0 + 1;
     // 1. L[J0 + lr][q], q < J0 (written before the barrier that ended block column q / 32)
@@ -87,15 +87,24 @@ __global__ void __launch_bounds__(CF_FT, 1)
       }
     }
     cf_commit();
-    // 2. the Gram's block column through its symmetric upper part (never overwritten there);
-    //    every Gram entry is read here once up to symmetry, so the finiteness check is here
+    // 2. the Gram's block column through its symmetric upper part (never overwritten there),
+    //    minus the products of the finished columns.  Thread tile: rows 4 trg .. 4 trg + 3,
+    //    columns tcc + 8 j.  A short block column leaves tiles for fewer threads than the
+    //    CTA has: the inner dimension is then split KS ways, split 0 starting from the Gram
+    //    and the others from zero, and split 0 adds the others' partial sums in split order
+    //    (they are parked in rows of P past R: at most 8192 doubles, P holds 8448).
+    //    Every Gram entry is read here once up to symmetry, so the finiteness check is here.
+    const int ntiles = 8 * ((R + 3) / 4);
+    const int KS = max(1, CF_FT / ntiles);
+    const int ti = tid % ntiles, ks = tid / ntiles, trg = ti >> 3, tcc = ti & 7;
+    const bool act = ks < KS;
     double acc[4][4];
 #pragma unroll
     for (int m = 0; m < 4; ++m)
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        const int lr = tr + 64 * m, c = tc + 8 * j;
-        acc[m][j] = (lr < R && c < nb) ? Gu[(long long)(J0 + lr) * gld + J0 + c] : 0.0;
+        const int lr = 4 * trg + m, c = tcc + 8 * j;
+        acc[m][j] = (ks == 0 && lr < R && c < nb) ? Gu[(long long)(J0 + lr) * gld + J0 + c] : 0.0;
         if (!isfinite(acc[m][j])) bad = 1;
       }
     cf_wait<0>();
@@ -105,28 +114,47 @@ __global__ void __launch_bounds__(CF_FT, 1)
         for (int i = lane; i < k; i += 32) Gu[(long long)c * gld + i] = i == c ? 1.0 : 0.0;
       return;
     }
+    if (act && J0 > 0) {
+      const int qc = (J0 + KS - 1) / KS, qb = ks * qc, qe = min(J0, qb + qc);
 #pragma unroll 2
-    for (int q = 0; q < J0; ++q) {
-      double b[4];
+      for (int q = qb; q < qe; ++q) {
+        double b[4];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) b[j] = Lleft[(tc + 8 * j) * lp + q];
+        for (int j = 0; j < 4; ++j) b[j] = Lleft[(tcc + 8 * j) * lp + q];
 #pragma unroll
-      for (int m = 0; m < 4; ++m) {
-        if (64 * m < R) {
-          // rows past R would lie beyond the staged block (64-row granularity)
-          const double a = tr + 64 * m < R ? Lleft[(tr + 64 * m) * lp + q] : 0.0;
+        for (int m = 0; m < 4; ++m) {
+          // rows past R would lie beyond the staged block
+          const double a = 4 * trg + m < R ? Lleft[(4 * trg + m) * lp + q] : 0.0;
 #pragma unroll
           for (int j = 0; j < 4; ++j) acc[m][j] = fma(-a, b[j], acc[m][j]);
         }
       }
     }
+    double* part = P + R * CF_P;   // partial sums of splits 1..KS-1
+    if (act && ks > 0) {
 #pragma unroll
-    for (int m = 0; m < 4; ++m)
+      for (int m = 0; m < 4; ++m)
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int lr = tr + 64 * m, c = tc + 8 * j;
-        if (lr < R && c < nb) P[lr * CF_P + c] = acc[m][j];
-      }
+        for (int j = 0; j < 4; ++j) part[((ks - 1) * ntiles + ti) * 16 + m * 4 + j] = acc[m][j];
+    }
+    __syncthreads();
+    if (ks == 0) {
+      for (int s2 = 1; s2 < KS; ++s2)
+#pragma unroll
+        for (int m = 0; m < 4; ++m)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) acc[m][j] += part[((s2 - 1) * ntiles + ti) * 16 + m * 4 + j];
+    }
+    __syncthreads();
+    if (ks == 0) {
+#pragma unroll
+      for (int m = 0; m < 4; ++m)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int lr = 4 * trg + m, c = tcc + 8 * j;
+          if (lr < R && c < nb) P[lr * CF_P + c] = acc[m][j];
+        }
+    }
     __syncthreads();
     // 3. diagonal block: thread (r = tid / 16, s = tid % 16) updates columns s and s + 16 of
     //    row r; a step reads only column c and writes only columns > c
