@@ -1,4 +1,5 @@
-// Exact fp16 directed rounding and the quantiser step of the b-bit block quantiser.
+// Exact fp16 directed rounding, the quantiser step, codes and code packing of the b-bit
+// block quantiser.
 // Host and device: the device code is what the table and encode kernels run; the host
 // copy of the same source lets a CPU check compare it with the float64 definition.
 #pragma once
@@ -92,6 +93,42 @@ __host__ __device__ __forceinline__ float quant_step(float mx, float lo, float f
     if (sp > 0.f && ge_exact(sp * flev, mx, lo, R)) s = sp;
   }
   return s;
+}
+
+// ---------------------------------------------------------------------------------------
+// codes of the b-bit block quantiser and their packing
+// ---------------------------------------------------------------------------------------
+// round-half-even of d * inv to an integer-valued float: one FMA onto the 1.5*2^23 shift
+constexpr float kRoundShift = 12582912.0f;
+__host__ __device__ __forceinline__ float code_of(float d, float inv) {
+#ifdef __CUDA_ARCH__
+  return __fsub_rn(__fmaf_rn(d, inv, kRoundShift), kRoundShift);
+#else
+  volatile float t = fmaf(d, inv, kRoundShift);   // one rounding, then an exact subtraction
+  return t - kRoundShift;
+#endif
+}
+
+// code of one value: round((v - lo) * inv) clamped to [0, levels]; inv is the correctly
+// rounded reciprocal of the fp16 step
+__host__ __device__ __forceinline__ uint32_t block_code(float v, float lo, float inv, float flev) {
+  float c = code_of(v - lo, inv);
+  c = fminf(fmaxf(c, 0.f), flev);
+  return (uint32_t)c;
+}
+
+// code j of a block occupies bits [j b, (j + 1) b) of the block's little-endian bit string,
+// held as four 32-bit words (2 b bytes for 16 codes)
+__host__ __device__ __forceinline__ void pack_code(uint32_t* w, int j, int b, uint32_t code) {
+  const int pos = j * b;
+  w[pos >> 5] |= code << (pos & 31);
+  if ((pos & 31) + b > 32) w[(pos >> 5) + 1] |= code >> (32 - (pos & 31));
+}
+__host__ __device__ __forceinline__ uint32_t unpack_code(const uint32_t* w, int j, int b) {
+  const int pos = j * b;
+  uint32_t code = w[pos >> 5] >> (pos & 31);
+  if ((pos & 31) + b > 32) code |= w[(pos >> 5) + 1] << (32 - (pos & 31));
+  return code & ((1u << b) - 1u);
 }
 
 }  // namespace jolt

@@ -34,12 +34,6 @@ struct Cands {
   int rT[MAXC], rD[MAXC], bits[MAXC];
 };
 
-// round-half-even of d * inv to an integer-valued float: one FMA onto the 1.5*2^23 shift
-constexpr float kRoundShift = 12582912.0f;
-__device__ __forceinline__ float code_of(float d, float inv) {
-  return __fsub_rn(__fmaf_rn(d, inv, kRoundShift), kRoundShift);
-}
-
 // ---------------------------------------------------------------------------------------
 // fused residual / rotation / quantiser tile machinery (mma.sync m16n8k16 fragments)
 //
@@ -633,14 +627,7 @@ __global__ void __launch_bounds__(TTHREADS) encode_kernel(EncodeArgs a) {
       const float inv = (step > 0.f && step <= kFp16Max) ? __frcp_rn(step) : 0.f;
       uint32_t w[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        float c = code_of(v[j] - lo, inv);
-        c = fminf(fmaxf(c, 0.f), flev);
-        const uint32_t code = (uint32_t)c;
-        const int pos = j * b;
-        w[pos >> 5] |= code << (pos & 31);
-        if ((pos & 31) + b > 32) w[(pos >> 5) + 1] |= code >> (32 - (pos & 31));
-      }
+      for (int j = 0; j < 16; ++j) pack_code(w, j, b, block_code(v[j], lo, inv, flev));
       const long long blk = ((long long)s * T + t) * (D / 16) + m;
       unsigned char* dst = codes + blk * (2 * b);
       // 2b bytes; the block start is 2b-aligned
@@ -757,16 +744,8 @@ __global__ void __launch_bounds__(TTHREADS) decode_kernel(DecodeArgs a) {
         for (int byte = 0; byte < 2 * b; ++byte) w[byte >> 2] |= (uint32_t)src[byte] << ((byte & 3) * 8);
         __half2 sc = reinterpret_cast<const __half2*>(a.blob + uh.off_scales)[blk];
         float lo = __low2float(sc), step = __high2float(sc);
-        const uint32_t mask = (1u << b) - 1u;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          int col = (i >> 1) * 8 + 2 * q + (i & 1);
-          int pos = col * b;
-          uint32_t code = w[pos >> 5] >> (pos & 31);
-          if ((pos & 31) + b > 32) code |= w[(pos >> 5) + 1] << (32 - (pos & 31));
-          code &= mask;
-          deq[i] = fmaf((float)code, step, lo);
-        }
+        for (int i = 0; i < 4; ++i) deq[i] = fmaf((float)unpack_code(w, (i >> 1) * 8 + 2 * q + (i & 1), b), step, lo);
       }
       f.v[h][2 * m][0] = acc[2 * m][h * 2 + 0] + deq[0];
       f.v[h][2 * m][1] = acc[2 * m][h * 2 + 1] + deq[1];

@@ -1,8 +1,15 @@
-"""The library's exact fp16 block scales (lo = fp16 round-down of the block minimum, step =
-smallest fp16 s with s * (2^b - 1) >= max - lo) compiled for the host from the same source
-the kernels use, compared bit for bit with the oracle's float64 definition on random and
-adversarial blocks: values at and next to fp16 numbers, steps landing exactly on fp16
-numbers, the fp16 subnormal range, overflow, equal minimum and maximum."""
+"""The library's block quantiser compiled for the host from the same source the kernels use,
+against the oracle:
+
+* the exact fp16 block scales (lo = fp16 round-down of the block minimum, step = smallest
+  fp16 s with s * (2^b - 1) >= max - lo), bit for bit, on random and adversarial blocks
+  (values at and next to fp16 numbers, steps landing exactly on fp16 numbers, the fp16
+  subnormal range, overflow, equal minimum and maximum);
+* the packed code bytes, bit for bit with the oracle's packing of the same codes, and their
+  unpacking;
+* the codes themselves: the library rounds (x - lo) * fp32(1/step), the oracle rounds
+  (x - lo) / step in float64, so they may differ only where the quotient lies within fp32
+  rounding of a half-integer."""
 import os
 import shutil
 import subprocess
@@ -60,6 +67,62 @@ def host_prog(tmp_path_factory):
     subprocess.run([nvcc, "-std=c++17", "-O2", "-Wno-deprecated-gpu-targets", "-I", CSRC, "-o", exe, os.path.join(ROOT, "tests", "quant_step_host.cu")],
                    check=True, capture_output=True)
     return exe
+
+
+def _compile(tmp_path_factory, name):
+    nvcc = shutil.which("nvcc")
+    if nvcc is None:
+        pytest.skip("nvcc not available")
+    exe = str(tmp_path_factory.mktemp(name) / name)
+    subprocess.run([nvcc, "-std=c++17", "-O2", "-Wno-deprecated-gpu-targets", "-I", CSRC, "-o", exe,
+                    os.path.join(ROOT, "tests", name + ".cu")], check=True, capture_output=True)
+    return exe
+
+
+@pytest.fixture(scope="module")
+def codes_prog(tmp_path_factory):
+    return _compile(tmp_path_factory, "quant_codes_host")
+
+
+@pytest.mark.parametrize("b", BITS)
+def test_codes_and_packing(codes_prog, b):
+    rng = np.random.default_rng(100 + b)
+    blocks = [(rng.standard_normal((3000, 16)) * s) for s in (1e-4, 0.05, 1.0, 30.0)]
+    # blocks whose values sit on and next to the quantiser's half-integer levels
+    lo = O.fp16_rd(rng.standard_normal(2000))
+    step = O.fp16_ru(np.abs(rng.standard_normal(2000)) * 0.1 + 1e-3)
+    k = rng.integers(0, (1 << b) - 1, (2000, 16)) + 0.5
+    x = lo[:, None] + k * step[:, None]
+    x[:, 0] = lo
+    x[:, 1] = lo + ((1 << b) - 1) * step
+    blocks.append(x)
+    v = np.concatenate(blocks).astype(np.float32)
+    out = subprocess.run([codes_prog], input=np.int32(b).tobytes() + v.tobytes(), capture_output=True,
+                         check=True).stdout
+    rec = np.frombuffer(out, dtype=np.dtype([("lo", "<f4"), ("step", "<f4"), ("codes", "u1", 16),
+                                             ("bytes", "u1", 16), ("back", "u1", 16)]))
+    assert rec.shape[0] == v.shape[0]
+    codes = rec["codes"].astype(np.int64)
+    nbytes = 2 * b
+    # packing: bit for bit the oracle's packing of the same codes; unpacking inverts it
+    np.testing.assert_array_equal(rec["bytes"][:, :nbytes], O.pack_codes(codes[:, None, :], b))
+    assert not rec["bytes"][:, nbytes:].any()
+    np.testing.assert_array_equal(rec["back"].astype(np.int64), codes)
+    np.testing.assert_array_equal(O.unpack_codes(rec["bytes"][:, :nbytes], b)[:, 0, :], codes)
+    # codes: the oracle's quantiser on the same fp32 block; differences only at ties
+    ref_codes, ref_lo, ref_step, _, ok = O.quantize(v.astype(np.float64), b)
+    ref_codes, ref_lo, ref_step, ok = ref_codes[:, 0, :], ref_lo[:, 0], ref_step[:, 0], ok[:, 0]
+    assert ok.all()
+    np.testing.assert_array_equal(rec["lo"].astype(np.float64), ref_lo)
+    np.testing.assert_array_equal(rec["step"].astype(np.float64), ref_step)
+    diff = codes != ref_codes
+    q = (v.astype(np.float64) - ref_lo[:, None]) / np.where(ref_step > 0, ref_step, 1.0)[:, None]
+    near_tie = np.abs(q - np.floor(q) - 0.5) <= 4 * np.finfo(np.float32).eps * np.maximum(np.abs(q), 1.0)
+    assert np.all(near_tie[diff])
+    assert np.all(np.abs(codes - ref_codes) <= 1)
+    # the stated bound on random blocks (the constructed blocks above are ties on purpose)
+    n_random = sum(x.shape[0] for x in blocks[:-1])
+    assert diff[:n_random].mean() <= 1e-4
 
 
 def test_block_scales_match_the_oracle_bit_for_bit(host_prog):
