@@ -37,6 +37,8 @@ Parity status (what pins each function, see tests/test_oracle_*.py):
   allocate                       -- exhaustive enumeration (Everett), budget never exceeded,
                                     lambda = 0 and infeasible special cases.
   compress / decompress          -- round trip error equals the table entry.
+  slice_attention_factored       -- equals softmax attention over the decompressed cache
+                                    (dense route) for every bit-width and both methods.
 """
 from __future__ import annotations
 
@@ -675,6 +677,56 @@ def decompress(res: CompressResult):
         sl = slice(rec.group * Lg, (rec.group + 1) * Lg)
         (K if rec.kv == 0 else V)[sl] = decode_unit(rec, res.opts.block)
     return K, V
+
+
+# ----------------------------------------------------------------------------------------
+# Decode-side attention over the stored factors ([Abstract]: the decode path evaluates
+# attention directly over the stored factors, without forming dense K and V tensors).
+# Reading: one decode step of queries q against every cached token of one (layer, head)
+# slice of a layer group.  With Phi = diag(sigma) H / sqrt(D), the decoder above stores the
+# slice as X_hat = (U_s P' + rho_hat) Phi^T, so
+#   scores:  X_hat q = U_s (P' q') + rho_hat q',   q' = Phi^T q  (rotate(q) as a row),
+#   values:  p^T X_hat = (p^T U_s P' + p^T rho_hat) Phi^T,
+# and rho_hat q' sums, per 16-wide block, lo * (sum of q' over the block) + step * (codes . q').
+# Scores are scaled by 1 / sqrt(D) before the softmax.
+# ----------------------------------------------------------------------------------------
+def softmax(s: np.ndarray) -> np.ndarray:
+    m = s.max(axis=-1, keepdims=True)
+    e = np.exp(s - m)
+    return e / e.sum(axis=-1, keepdims=True)
+
+
+def slice_scores_factored(rec: UnitRecord, l: int, h: int, q: np.ndarray, block: int = 16) -> np.ndarray:
+    """X_hat[l, h] q for queries q (nq, D) from the stored factors and codes: (nq, T)."""
+    D = q.shape[-1]
+    P = recon_operator(rec.C_s, rec.W_s, rec.sigma, rec.r_D)[l, h]      # (r_T, D), rotated
+    qr = rotate(np.asarray(q, dtype=np.float64), rec.sigma)             # q' as rows
+    s = (rec.U_s @ (P @ qr.T)).T                                        # (nq, T)
+    if rec.b > 0:
+        nb = D // block
+        qb = qr.reshape(qr.shape[0], nb, block)
+        s = s + np.einsum("tb,qb->qt", rec.lo[l, h], qb.sum(-1), optimize=True)
+        s = s + np.einsum("tb,tbj,qbj->qt", rec.step[l, h], rec.codes[l, h].astype(np.float64), qb,
+                          optimize=True)
+    return s
+
+
+def slice_values_factored(rec: UnitRecord, l: int, h: int, p: np.ndarray, block: int = 16) -> np.ndarray:
+    """p^T X_hat[l, h] for attention weights p (nq, T) from the stored factors: (nq, D)."""
+    P = recon_operator(rec.C_s, rec.W_s, rec.sigma, rec.r_D)[l, h]
+    y = (np.asarray(p, dtype=np.float64) @ rec.U_s) @ P                 # rotated basis
+    if rec.b > 0:
+        rhat = rec.lo[l, h][..., None] + rec.codes[l, h] * rec.step[l, h][..., None]   # (T, nb, block)
+        y = y + p @ rhat.reshape(rhat.shape[0], -1)
+    return unrotate(y, rec.sigma)
+
+
+def slice_attention_factored(recK: UnitRecord, recV: UnitRecord, l: int, h: int, q: np.ndarray,
+                             block: int = 16):
+    """One decode step over the stored factors: (softmax weights (nq, T), output (nq, D))."""
+    D = q.shape[-1]
+    p = softmax(slice_scores_factored(recK, l, h, q, block) / math.sqrt(D))
+    return p, slice_values_factored(recV, l, h, p, block)
 
 
 def relative_error(X: np.ndarray, Xhat: np.ndarray) -> float:
