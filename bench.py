@@ -45,7 +45,7 @@ def parse():
     ap.add_argument("--workload", default="mistral7b")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extras", action="store_true", help="skip the exact-arm and decompress side figures")
-    ap.add_argument("--profile-case", default=None, choices=["mistral7b_4layers", "mistral7b"],
+    ap.add_argument("--profile-case", default=None, choices=["mistral7b_4layers", "mistral7b", "llama31_8b_64k"],
                     help="run two compress + decompress calls of one case (for ncu captures) and exit")
     ap.add_argument("--sweep", action="store_true",
                     help="one JSON line per workload of the other shapes (LLaMA-2-13B, LLaMA-3.1-8B/64K) and "
@@ -59,8 +59,8 @@ def profile_case(args):
     1 GiB of workspace with FlashJoLT), with the same kernels as the timed run."""
     import torch
     from kv_cache_compression_group_b200 import synth, jolt as J
-    if args.profile_case == "mistral7b":
-        w = synth.WORKLOADS["mistral7b"]
+    if args.profile_case in ("mistral7b", "llama31_8b_64k"):
+        w = synth.WORKLOADS[args.profile_case]
     else:
         w = synth.small_workload("mistral7b", n_layers=4)
     K, V = synth.make_cache(w, 0)

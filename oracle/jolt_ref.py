@@ -15,10 +15,9 @@ the token and feature modes only; the truncation residual is rotated by a random
 orthogonal (Johnson-Lindenstrauss) rotation and quantised to a few bits; one
 Lagrangian dual picks the Tucker ranks and residual bit-widths of every group
 under one global byte budget; FlashJoLT replaces the exact token-mode SVD by a
-randomized one.  Everything else below is a stated reading (listed in the
-design notes): Gram/eigen factor route, random-sign Walsh-Hadamard rotation
-along the features, 16-wide min-max blocks with fp16 scales, bf16 factor storage,
-the byte formula and the bisection rule.
+randomized one.  Everything else below is a stated reading: the Gram/eigen factor
+route, the random-sign Walsh-Hadamard rotation along the features, 16-wide min-max
+blocks with fp16 scales, bf16 factor storage, the byte formula and the bisection rule.
 
 Every step runs in float64 except at the storage rounding points the format
 defines (bf16 factors and reconstruction operator, fp16 block scales).  No
@@ -31,14 +30,26 @@ Parity status (what pins each function, see tests/test_oracle_*.py):
   feature_factor, token_factor_* -- full-rank exactness, energy split, Eckart-Young,
                                     exact Tucker generator, T-side vs M-side route,
                                     randomized == exact when the sketch covers the rank.
+  tucker_core / tucker_reconstruct -- full-rank exactness, energy split, Eckart-Young.
+  stored_core                    -- hand-worked example of both bf16 roundings; exact
+                                    sub-block under row / column selections; within two
+                                    bf16 roundings of tucker_core.
+  recon_operator / decode_unit   -- hand-worked example of the rotated operator; at b = 0
+                                    the decoder equals tucker_reconstruct of the stored
+                                    factors within the bf16 rounding of P'; full rank with
+                                    roundings removed reconstructs exactly.
   quantize / pack_codes          -- brute-force nearest level on tiny blocks, tie cases,
-                                    bit-level unpack.
+                                    bit-level unpack, hand-worked block.
   unit_payload_bytes             -- byte count of the actual packed arrays.
+  distortion_table / encode_unit -- round trip error equals the table entry; zero at full
+                                    rank without roundings.
   allocate                       -- exhaustive enumeration (Everett), budget never exceeded,
                                     lambda = 0 and infeasible special cases.
   compress / decompress          -- round trip error equals the table entry.
   slice_attention_factored       -- equals softmax attention over the decompressed cache
                                     (dense route) for every bit-width and both methods.
+Planted mistakes (a transposed core, an unrounded Z, Phi^T for Phi, an unrotated
+operator) are each shown to fail one of these pins.
 """
 from __future__ import annotations
 

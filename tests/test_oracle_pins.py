@@ -334,3 +334,181 @@ def test_round_trip_equals_table_entry(method):
         sl = slice(rec.group * 2, rec.group * 2 + 2)
         e = np.sum((X[sl] - Xh[sl]) ** 2)
         assert abs(e - rec.distortion) <= 1e-12 * np.sum(X[sl] ** 2)
+
+
+# ------------------------------------------------------------------ stored format
+# The stored core, the rotated reconstruction operator and the decoder are pinned against
+# hand-worked examples, exact column selections and the textbook Tucker forms above
+# (tucker_core / tucker_reconstruct, themselves pinned by the closed forms of this file),
+# never against themselves.  Each check is also run on a copy of the oracle function with
+# one plausible mistake planted, and must reject it.
+import oracle.jolt_ref as JR
+
+_U8 = 2.0 ** -8     # unit roundoff of bf16 (8 significant bits)
+
+
+def _golden_map(golden_dir, name):
+    return dict((r.split()[0], [float(v) for v in r.split()[1:]]) for r in _read_golden(golden_dir, name))
+
+
+def _core_worked_example(stored_core_fn, golden_dir):
+    g = _golden_map(golden_dir, "stored_core_worked_example.txt")
+    t = int(g["t"][0])
+    X = np.tile(np.array(g["x_row"]), (t, 1))[None, None]        # (1, 1, T, 2)
+    W_s = np.ones((2, 1))
+    U_s = np.ones((t, 1))
+    return float(stored_core_fn(X, U_s, W_s)[0, 0, 0, 0]), g
+
+
+def test_stored_core_worked_example(golden_dir):
+    got, g = _core_worked_example(O.stored_core, golden_dir)
+    assert got == g["core"][0]
+    # the unrounded Tucker core of the same slice is the textbook value
+    X = np.tile(np.array(g["x_row"]), (int(g["t"][0]), 1))[None, None]
+    assert float(O.tucker_core(X, np.ones((X.shape[2], 1)), np.ones((2, 1)))[0, 0, 0, 0]) == g["core_unrounded"][0]
+
+
+def _core_by_selection(stored_core_fn):
+    """U_s, W_s that pick rows / columns (exact in bf16): the core of a bf16-exact slice is
+    then the selected sub-block, C[l,h][r, q] = X[l,h][rows[r], cols[q]], with no rounding.
+    Returns the largest deviation."""
+    rng = np.random.default_rng(21)
+    Lg, H, T, D = 2, 3, 12, 16
+    X = O.bf16_rn(rng.standard_normal((Lg, H, T, D)))
+    rows = np.array([7, 2, 11, 0])
+    cols = np.array([5, 14, 3, 9])
+    U_s = np.zeros((T, 4))
+    U_s[rows, np.arange(4)] = 1.0
+    W_s = np.zeros((D, 4))
+    W_s[cols, np.arange(4)] = 1.0
+    want = X[:, :, rows][:, :, :, cols]
+    got = stored_core_fn(X, U_s, W_s)
+    if got.shape != want.shape:
+        return math.inf
+    return float(np.max(np.abs(got - want)))
+
+
+def test_stored_core_selects_the_sub_block():
+    assert _core_by_selection(O.stored_core) == 0.0
+
+
+def _core_vs_tucker(stored_core_fn):
+    """stored_core against the unrounded Tucker core U_s^T X W_s: two bf16 roundings, so
+    |C_s - C| <= u (|U_s|^T |X W_s|) (1 + u) + u |C| (1 + u)^2 entry by entry.  Returns the
+    largest ratio of the deviation to that bound."""
+    rng = np.random.default_rng(22)
+    X = O.bf16_rn(_rand_cache(rng, 2, 2, 40, 16) * 3.0)
+    _, W = O.feature_factor(X)
+    U = O.token_factor_exact(X, 10)
+    U_s, W_s = O.bf16_rn(U), O.bf16_rn(W[:, :6])
+    C = O.tucker_core(X, U_s, W_s)
+    Cs = stored_core_fn(X, U_s, W_s)
+    if Cs.shape != C.shape:
+        return math.inf
+    Z = np.abs(np.einsum("lhtd,dq->lhtq", X, W_s))
+    bound = _U8 * np.einsum("tr,lhtq->lhrq", np.abs(U_s), Z) * (1 + _U8) + _U8 * np.abs(C) * (1 + _U8) ** 2
+    return float(np.max(np.abs(Cs - C) / (bound + 1e-300)))
+
+
+def test_stored_core_within_two_bf16_roundings_of_tucker_core():
+    assert _core_vs_tucker(O.stored_core) <= 1.0
+
+
+def test_recon_operator_worked_example(golden_dir):
+    g = _golden_map(golden_dir, "recon_operator_worked_example.txt")
+    P = O.recon_operator(np.ones((1, 1, 1, 1)), np.ones((2, 1)), np.array(g["sigma"]), 1)
+    assert list(P.ravel()) == g["p_rot"]
+
+
+def _decode_vs_tucker(monkeypatch=None):
+    """At b = 0 the decoder over the stored bytes is the Tucker reconstruction of the stored
+    factors, U_s C_s W_s^T, up to the bf16 rounding of P' (Phi is orthogonal):
+    ||decode - U_s C_s W_s^T||_F <= ||U_s||_2 u ||C_s W_s^T||_F per slice.  Returns the
+    largest ratio of the deviation to that bound over several (r_T, r_D)."""
+    from kv_cache_compression_group_b200 import synth
+    w = synth.WORKLOADS["tiny"]
+    K, V = (synth.to_f64(t) for t in synth.make_cache(w, 3))
+    X = K[:2]
+    opts = O.Options((4, 8, 16, 32), (4, 8, 16), (0, 2), method="exact")
+    f = O.unit_factors(X, 0, 0, opts, 5)
+    worst = 0.0
+    for rT in (4, 16, 32):
+        for rD in (4, 8, 16):
+            c = opts.token_ranks.index(rT) * len(opts.feature_ranks) * len(opts.bits) \
+                + opts.feature_ranks.index(rD) * len(opts.bits)        # b = 0
+            rec = O.encode_unit(X, f, opts, c, 0.0)
+            assert rec.b == 0 and rec.r_T == rT and rec.r_D == rD
+            got = O.decode_unit(rec)
+            want = O.tucker_reconstruct(f.U_s[:, :rT], f.C_s[:, :, :rT, :rD], f.W_s[:, :rD])
+            P = np.einsum("lhrq,dq->lhrd", f.C_s[:, :, :rT, :rD], f.W_s[:, :rD])
+            nU = np.linalg.norm(f.U_s[:, :rT], 2)
+            for l in range(X.shape[0]):
+                for h in range(X.shape[1]):
+                    dev = np.linalg.norm(got[l, h] - want[l, h])
+                    bound = nU * _U8 * np.linalg.norm(P[l, h]) * (1 + 1e-12) + 1e-300
+                    worst = max(worst, dev / bound)
+    return worst
+
+
+def test_decode_b0_is_tucker_reconstruction_of_stored_factors():
+    assert _decode_vs_tucker() <= 1.0
+
+
+def test_full_rank_unrounded_table_entry_is_zero(monkeypatch):
+    """With r_T = T, r_D = D and every storage rounding replaced by the identity, the
+    stored-format pipeline (core, rotated operator, rotated residual) reconstructs X
+    exactly: the b = 0 table entry is ||rho||^2 = 0 (full-rank Tucker is exact)."""
+    monkeypatch.setattr(JR, "bf16_rn", lambda x: np.asarray(x, dtype=np.float64))
+    rng = np.random.default_rng(23)
+    X = _rand_cache(rng, 2, 2, 24, 16)          # T = 24 <= M = 64
+    _, W = O.feature_factor(X)
+    U = O.token_factor_exact(X, 24)
+    C_s = O.stored_core(X, U, W)
+    sigma = O.rotation_signs(1, 0, 0, 16)
+    opts = O.Options((8, 24), (4, 16), (0, 3))
+    tab = O.distortion_table(X, U, W, C_s, sigma, opts)
+    assert tab[1, 1, 0] <= 1e-12 * np.sum(X * X)
+    assert tab[0, 0, 0] > 1e-3 * np.sum(X * X)          # a truncated choice is not exact
+
+
+# --- planted mistakes: each must be caught by one of the pins above --------------------
+def _core_transposed(X, U_s, W_s):
+    Z = O.bf16_rn(np.einsum("lhtd,dq->lhtq", X, W_s))
+    return O.bf16_rn(np.einsum("tr,lhtq->lhqr", U_s, Z))
+
+
+def _core_unrounded_z(X, U_s, W_s):
+    Z = np.einsum("lhtd,dq->lhtq", X, W_s)
+    return O.bf16_rn(np.einsum("tr,lhtq->lhrq", U_s, Z))
+
+
+def _core_token_side_first(X, U_s, W_s):
+    Y = O.bf16_rn(np.einsum("tr,lhtd->lhrd", U_s, X))
+    return O.bf16_rn(np.einsum("lhrd,dq->lhrq", Y, W_s))
+
+
+def _recon_phi_transposed(C_s, W_s, sigma, r_D):
+    P = np.einsum("lhrq,dq->lhrd", C_s[..., :r_D], W_s[:, :r_D])
+    return O.bf16_rn(O.fwht(P) / math.sqrt(P.shape[-1]) * sigma)
+
+
+def _recon_unrotated(C_s, W_s, sigma, r_D):
+    return O.bf16_rn(np.einsum("lhrq,dq->lhrd", C_s[..., :r_D], W_s[:, :r_D]))
+
+
+def test_planted_core_mistakes_are_caught(golden_dir):
+    assert _core_by_selection(_core_transposed) > 0          # transposed core einsum
+    got, g = _core_worked_example(_core_unrounded_z, golden_dir)
+    assert got == g["core_without_z_rounding"][0] != g["core"][0]   # Z left unrounded
+    got, _ = _core_worked_example(_core_token_side_first, golden_dir)
+    assert got != g["core"][0]                                      # rounded on the token side first
+
+
+def test_planted_operator_mistakes_are_caught(golden_dir, monkeypatch):
+    g = _golden_map(golden_dir, "recon_operator_worked_example.txt")
+    P = _recon_phi_transposed(np.ones((1, 1, 1, 1)), np.ones((2, 1)), np.array(g["sigma"]), 1)
+    assert list(P.ravel()) == g["p_rot_transposed"] != g["p_rot"]
+    for mutant in (_recon_phi_transposed, _recon_unrotated):
+        with monkeypatch.context() as m:
+            m.setattr(JR, "recon_operator", mutant)
+            assert _decode_vs_tucker() > 100.0
