@@ -26,9 +26,14 @@
  *
  * Conventions for every call:
  *   - every pointer named *_dev is device memory the caller owns; the library keeps no
- *     pointer after the call returns and allocates no device memory of its own (the one
- *     exception: eigen-solver and Cholesky calls go through a cuSOLVER handle that the
- *     library creates once per thread and device, which holds cuSOLVER's own state);
+ *     pointer after the call returns and takes no workspace from cudaMalloc.  It does own
+ *     these per-thread resources, created on first use and kept until jolt_release() or
+ *     thread exit: a cuSOLVER handle and parameter object for each of two streams (eigen
+ *     solves that are not the library's own kernels), one auxiliary non-blocking stream with
+ *     two events (the feature factor runs on it beside the token factor), one capture stream
+ *     and up to 8 instantiated CUDA graphs of compress calls (see jolt_set_graphs), and the
+ *     CUDA events of stage timing (jolt_profile_begin/end).  The compiled-in 64 KiB array of
+ *     jolt_frobenius_noalloc is held by every device that loads the library;
  *   - calls are stream-ordered on `stream` (a cudaStream_t, NULL = legacy default stream)
  *     and return before the GPU work finishes, except where a call says it synchronises;
  *   - argument errors are detected on the host and returned before anything is launched;
@@ -224,7 +229,10 @@ jolt_status jolt_frobenius(const jolt_shape* shape, const void* k_dev, const voi
  *   - at most 64 units (2 * n_layers / layers_per_group <= 64); more returns
  *     JOLT_ERR_WORKSPACE_TOO_SMALL with a message naming the limit;
  *   - the first call on each device looks up the array's device address with that device
- *     current (a one-time set-up); make that first call before any stream capture;
+ *     current (a one-time set-up); make that first call before any stream capture.  The
+ *     looked-up address is kept for the process: after cudaDeviceReset the device's module
+ *     is loaded again and the array may move, so do not call this entry point on a device
+ *     that has been reset since its first call;
  *   - all calls share the one array: two calls whose GPU work overlaps (different streams or
  *     threads without ordering between them) race on it and may return wrong sums;
  *   - allocates nothing.  Asynchronous. */
@@ -253,6 +261,31 @@ jolt_status jolt_profile_begin(void);
  * launched inside cuSOLVER is not counted). */
 uint64_t jolt_launch_count(void);
 jolt_status jolt_profile_end(char* buf, size_t cap);
+
+/* Release this thread's library-owned resources (no counterpart on the pages): the cached
+ * CUDA graphs and their capture stream, the auxiliary stream and its events, the cuSOLVER
+ * handles and the stage-timing events.  Call it after this thread's library work has
+ * finished (for example after synchronising its streams); later calls recreate what they
+ * need.  Returns JOLT_ERR_CUDA if a stream could not be destroyed. */
+jolt_status jolt_release(void);
+
+/* FP32-pipe rate probe for the roofline of the ALU-bound kernels (no counterpart on the
+ * pages; measurement only).  Launches 8 CTAs of 256 threads per SM; every thread runs
+ * `iters` rounds of 8 independent fused multiply-add chains, scalar (packed = 0) or on
+ * packed pairs (packed != 0, two FMAs per instruction).  *fma_ops receives the number of
+ * FMAs the launch performs (each counted as one operation); time the launch with events on
+ * `stream`.  sink_dev: 8 * 256 * SMs floats the kernel may write (it never does in
+ * practice).  Asynchronous. */
+jolt_status jolt_fp32_rate_probe(int32_t packed, int32_t iters, float* sink_dev, uint64_t* fma_ops, void* stream);
+
+/* Self-test of the bounded device wait the tensor-core pipeline uses (no counterpart on the
+ * pages; failure-detection check).  One thread initialises an mbarrier for one arrival,
+ * arrives on it only if `arrive` != 0, and waits for it with a limit of limit_us
+ * microseconds (1 .. 5e6).  With no arrival the wait gives up, the kernel sets the timeout
+ * bit in *status_dev and returns normally, and this call returns JOLT_ERR_TIMEOUT; with the
+ * arrival it returns JOLT_OK.  status_dev: one uint32 of device memory.  SYNCHRONISES the
+ * stream. */
+jolt_status jolt_wait_selftest(int32_t arrive, uint32_t limit_us, uint32_t* status_dev, void* stream);
 
 #ifdef __cplusplus
 }

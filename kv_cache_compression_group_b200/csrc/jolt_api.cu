@@ -1437,6 +1437,35 @@ jolt_status jolt_profile_end(char* buf, size_t cap) {
   return JOLT_OK;
 }
 
+jolt_status jolt_fp32_rate_probe(int32_t packed, int32_t iters, float* sink_dev, uint64_t* fma_ops, void* stream) {
+  if (!sink_dev || !fma_ops || iters < 1) return fail(JOLT_ERR_INVALID_ARG, "null sink / ops or iters < 1");
+  int dev = 0, sms = 0;
+  CUDA_TRY(cudaGetDevice(&dev));
+  CUDA_TRY(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
+  const unsigned blocks = (unsigned)sms * 8u;
+  count_launch(), fma_probe_kernel<<<blocks, 256, 0, (cudaStream_t)stream>>>(sink_dev, iters, packed ? 1 : 0,
+                                                                              0.99993896484375f, 6.103515625e-05f);
+  CUDA_TRY(cudaGetLastError());
+  *fma_ops = (uint64_t)blocks * 256ull * (uint64_t)iters * (uint64_t)FP32_CHAINS * (packed ? 2ull : 1ull);
+  return JOLT_OK;
+}
+
+jolt_status jolt_wait_selftest(int32_t arrive, uint32_t limit_us, uint32_t* status_dev, void* stream) {
+  if (!status_dev) return fail(JOLT_ERR_INVALID_ARG, "null status word");
+  if (limit_us < 1 || limit_us > 5000000u) return fail(JOLT_ERR_INVALID_ARG, "limit_us %u not in [1, 5e6]", limit_us);
+  cudaStream_t st = (cudaStream_t)stream;
+  CUDA_TRY(cudaMemsetAsync(status_dev, 0, 4, st));
+  count_launch(), umma::wait_selftest_kernel<<<1, 32, 0, st>>>(arrive ? 1 : 0, (uint64_t)limit_us * 1000ull,
+                                                                 status_dev);
+  CUDA_TRY(cudaGetLastError());
+  uint32_t h = 0;
+  CUDA_TRY(cudaMemcpyAsync(&h, status_dev, 4, cudaMemcpyDeviceToHost, st));
+  CUDA_TRY(cudaStreamSynchronize(st));
+  if (h & DEV_ERR_TIMEOUT) return fail(JOLT_ERR_TIMEOUT, "bounded device wait gave up after %u us", limit_us);
+  if (h) return fail(JOLT_ERR_CUDA, "unexpected device status %u", h);
+  return JOLT_OK;
+}
+
 jolt_status jolt_workspace_size(const jolt_shape* shape, const jolt_options* opts, size_t* ws_bytes,
                                 size_t* blob_bytes, size_t* dws_bytes) {
   Plan p;
@@ -1743,6 +1772,40 @@ void jolt_set_graphs(int32_t enable) {
       if (g.exec) cudaGraphExecDestroy(g.exec);
     g_graphs.e.clear();
   }
+}
+
+jolt_status jolt_release(void) {
+  jolt_status ret = JOLT_OK;
+  for (auto& g : g_graphs.e)
+    if (g.exec) cudaGraphExecDestroy(g.exec);
+  g_graphs.e.clear();
+  if (g_graphs.cap_stream && cudaStreamDestroy(g_graphs.cap_stream) != cudaSuccess) ret = JOLT_ERR_CUDA;
+  g_graphs.cap_stream = nullptr;
+  g_graphs.cap_device = -1;
+  if (g_aux.st) {
+    if (cudaStreamDestroy(g_aux.st) != cudaSuccess) ret = JOLT_ERR_CUDA;
+    cudaEventDestroy(g_aux.fork);
+    cudaEventDestroy(g_aux.join);
+  }
+  g_aux = Aux();
+  for (auto& sv : g_solver) {
+    if (sv.h) {
+      cusolverDnDestroyParams(sv.params);
+      cusolverDnDestroy(sv.h);
+    }
+    sv = Solver();
+  }
+  for (auto& r : g_prof.recs) {
+    cudaEventDestroy(r.a);
+    cudaEventDestroy(r.b);
+  }
+  for (auto e : g_prof.pool) cudaEventDestroy(e);
+  g_prof.recs.clear();
+  g_prof.pool.clear();
+  g_prof.on = false;
+  cudaGetLastError();
+  if (ret != JOLT_OK) return fail(ret, "a stream of this thread could not be destroyed");
+  return JOLT_OK;
 }
 
 jolt_status jolt_read_header(const void* blob_dev, jolt_shape* shape_out, uint64_t* total_bytes,

@@ -762,4 +762,39 @@ __global__ void frob_final_kernel(const double* part, int nunits, int nblk, doub
   sq[i] = acc;
 }
 
+// ---------------------------------------------------------------------------------------
+// FP32-pipe rate probe (measurement only): every thread runs `iters` rounds of FP32_CHAINS
+// independent fused multiply-add chains, scalar (FFMA) or on packed pairs (FFMA2, two lanes'
+// worth of FMAs per instruction).  The chains start at 1 and contract towards 1, so no value
+// overflows or goes subnormal; one value per thread is stored only when it is impossible, so
+// the work is kept without memory traffic.
+// ---------------------------------------------------------------------------------------
+constexpr int FP32_CHAINS = 8;
+__global__ void __launch_bounds__(256) fma_probe_kernel(float* sink, int iters, int packed, float a, float b) {
+  if (packed) {
+    float2 x[FP32_CHAINS];
+#pragma unroll
+    for (int i = 0; i < FP32_CHAINS; ++i) x[i] = make_float2(1.f + i * 1e-3f, 1.f - i * 1e-3f);
+    const float2 a2 = make_float2(a, a), b2 = make_float2(b, b);
+    for (int it = 0; it < iters; ++it)
+#pragma unroll
+      for (int i = 0; i < FP32_CHAINS; ++i) x[i] = __ffma2_rn(x[i], a2, b2);
+    float s = 0.f;
+#pragma unroll
+    for (int i = 0; i < FP32_CHAINS; ++i) s += x[i].x + x[i].y;
+    if (s == -1.f) sink[blockIdx.x * blockDim.x + threadIdx.x] = s;
+  } else {
+    float x[FP32_CHAINS];
+#pragma unroll
+    for (int i = 0; i < FP32_CHAINS; ++i) x[i] = 1.f + i * 1e-3f;
+    for (int it = 0; it < iters; ++it)
+#pragma unroll
+      for (int i = 0; i < FP32_CHAINS; ++i) x[i] = fmaf(x[i], a, b);
+    float s = 0.f;
+#pragma unroll
+    for (int i = 0; i < FP32_CHAINS; ++i) s += x[i];
+    if (s == -1.f) sink[blockIdx.x * blockDim.x + threadIdx.x] = s;
+  }
+}
+
 }  // namespace jolt

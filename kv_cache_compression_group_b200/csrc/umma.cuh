@@ -96,14 +96,30 @@ __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
-// bounded wait for the phase with the given parity to complete
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+// bounded wait for the phase with the given parity to complete: false once `limit_ns` of
+// global time has passed without it
+__device__ __forceinline__ bool mbar_wait_for(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
   if (mbar_try(bar, parity)) return true;
   const uint64_t t0 = global_ns();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try(bar, parity)) return true;
-    if ((i & 255u) == 0 && global_ns() - t0 > kWaitNs) return false;
+    if ((i & 255u) == 0 && global_ns() - t0 > limit_ns) return false;
   }
+}
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) { return mbar_wait_for(bar, parity, kWaitNs); }
+
+// Self-test of the bounded wait: thread 0 initialises an mbarrier for one arrival, arrives
+// on it only if `arrive` is set, and waits for phase 0 with the given limit.  Without the
+// arrival the phase never completes, the wait gives up and DEV_ERR_TIMEOUT is raised; the
+// kernel then returns normally.
+__global__ void wait_selftest_kernel(int arrive, uint64_t limit_ns, uint32_t* status) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x != 0) return;
+  const uint32_t b = smem_u32(&bar);
+  mbar_init(b, 1);
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  if (arrive) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(b) : "memory");
+  if (!mbar_wait_for(b, 0, limit_ns)) atomicOr(status, DEV_ERR_TIMEOUT);
 }
 
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, int c0, int c1, int c2,

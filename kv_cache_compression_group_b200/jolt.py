@@ -28,7 +28,8 @@ EXPORTED = [
     "jolt_version", "jolt_last_error", "jolt_workspace_size", "jolt_counts", "jolt_choice_bytes",
     "jolt_compress", "jolt_factor", "jolt_table", "jolt_allocate", "jolt_encode", "jolt_read_header",
     "jolt_decompress", "jolt_frobenius", "jolt_profile_begin", "jolt_profile_end", "jolt_recon_operator",
-    "jolt_launch_count", "jolt_frobenius_noalloc", "jolt_set_graphs",
+    "jolt_launch_count", "jolt_frobenius_noalloc", "jolt_set_graphs", "jolt_release", "jolt_fp32_rate_probe",
+    "jolt_wait_selftest",
 ]
 
 
@@ -89,6 +90,9 @@ def lib():
             "jolt_recon_operator": [pS, pO, u64, vp, vp, ctypes.c_int64, vp, vp, sz, vp],
             "jolt_profile_begin": [],
             "jolt_profile_end": [ctypes.c_char_p, sz],
+            "jolt_release": [],
+            "jolt_fp32_rate_probe": [i32, i32, vp, ctypes.POINTER(u64), vp],
+            "jolt_wait_selftest": [i32, ctypes.c_uint32, vp, vp],
         }
         L.jolt_launch_count.argtypes = []
         L.jolt_launch_count.restype = ctypes.c_uint64
@@ -369,6 +373,24 @@ def profile_end():
         name, ms, n, u = line.split()
         out[name] = (float(ms), int(n), int(u))
     return out
+
+
+def release():
+    """Release this thread's library-owned streams, events, cached graphs and solver handles."""
+    _check(lib().jolt_release())
+
+
+def fp32_rate_probe(packed: bool, iters: int, sink: torch.Tensor, stream=None) -> int:
+    """Launch the FP32-pipe rate probe on the stream; returns the FMAs the launch performs."""
+    ops = ctypes.c_uint64()
+    _check(lib().jolt_fp32_rate_probe(1 if packed else 0, int(iters), _ptr(sink), ctypes.byref(ops),
+                                      _stream(stream)))
+    return int(ops.value)
+
+
+def wait_selftest(arrive: bool, limit_us: int, status: torch.Tensor, stream=None):
+    """Bounded device wait self-test (synchronises); raises JoltError TIMEOUT when it gives up."""
+    _check(lib().jolt_wait_selftest(1 if arrive else 0, int(limit_us), _ptr(status), _stream(stream)))
 
 
 def frobenius_noalloc(K, V, K_hat=None, V_hat=None, layers_per_group=1, stream=None):

@@ -53,16 +53,20 @@ def as_record(g, w, rec, group, kv, seed, block=16):
                         codes, lo, step, rec["distortion"])
 
 
-def check_codes(g, rho, xr, b):
+def check_codes(g, rho, xr, b, rho_oracle=None):
     """Scales and codes of the library against the oracle's quantiser on the same rho.
 
     The library forms rho in fp32 from x' and the reconstruction: its error is absolute,
     bounded per block by w = 2^-17 (max |x'| + max |x_hat|).  A differing scale must be the
     rounding of a block minimum / maximum inside that window; codes are compared under the
     library's own scales and may differ only where the oracle's scaled value lies within
-    w / step of a rounding tie.  Returns (n_scales, n_scale_bad, n_codes, n_code_bad); a
+    w / step of a rounding tie.  A
     differing scale is only possible in a block whose window straddles an fp16 rounding
-    boundary, and their number is asserted not to exceed the number of such blocks."""
+    boundary, and their number is asserted not to exceed the number of such blocks.
+
+    ``rho_oracle`` (the residual on the oracle's own reconstruction operator) adds the strict
+    count: codes that differ from the oracle's own codes (its scales, its operator), which is
+    the quantity the 1e-4 target bounds.  Returns a dict of counts."""
     codes, lo, step, _, _ = O.quantize(rho, b)
     codes, lo, step = codes.reshape(-1, 16), lo.reshape(-1), step.reshape(-1)
     rb = rho.reshape(-1, 16)
@@ -93,4 +97,29 @@ def check_codes(g, rho, xr, b):
         tie = np.abs(q - np.floor(q) - 0.5)
         tw = (win[:, None] / np.where(gs > 0, gs, 1.0)) + 1e-6
         assert np.all(tie[diff] <= np.broadcast_to(tw, tie.shape)[diff]), tie[diff].max()
-    return lo.size, int(bad.size), want.size, int(diff.sum())
+    out = dict(scales=lo.size, scale_bad=int(bad.size), codes=want.size, code_bad=int(diff.sum()),
+               code_vs_oracle=int(np.count_nonzero(g["codes"] != codes)))
+    if rho_oracle is not None:
+        oc = O.quantize(rho_oracle, b)[0].reshape(-1, 16)
+        out["code_vs_oracle"] = int(np.count_nonzero(g["codes"] != oc))
+    return out
+
+
+def add_counts(acc, c):
+    for k, v in c.items():
+        acc[k] = acc.get(k, 0) + v
+    return acc
+
+
+def assert_code_counts(acc, label=""):
+    """Report both code-mismatch fractions and bound them by the 1e-4 target: the codes the
+    library stored against the oracle's own codes (strict), and against the oracle's quantiser
+    evaluated under the library's scales."""
+    n = acc.get("codes", 0)
+    if not n:
+        return
+    print(f"\n[codes {label}] {n} codes: {acc['code_vs_oracle']} differ from the oracle's own codes "
+          f"({acc['code_vs_oracle'] / n:.2e}), {acc['code_bad']} under the library's scales "
+          f"({acc['code_bad'] / n:.2e}); {acc['scale_bad']} of {acc['scales']} block scales differ")
+    assert acc["code_bad"] <= max(1, 1e-4 * n), acc
+    assert acc["code_vs_oracle"] <= max(1, 1e-4 * n), acc

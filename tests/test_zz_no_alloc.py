@@ -34,3 +34,21 @@ def test_noalloc_rejects_too_many_units():
     with pytest.raises(J.JoltError) as e:
         J.frobenius_noalloc(K, V, None, None, 1)
     assert e.value.name == "WORKSPACE_TOO_SMALL" and "64" in str(e.value)
+
+
+def test_noalloc_largest_accepted_unit_count_and_fp32_cache():
+    """64 units (the limit: the highest slots of the compiled-in array) and an fp32 cache
+    with an fp32 second operand, each against the workspace entry point, twice in a row."""
+    w = synth.small_workload("mistral7b", n_layers=32, n_heads=1, T=32)
+    K, V = (t.cuda() for t in synth.make_cache(w, 5))
+    Kh, Vh = (K.float() * 0.99).contiguous(), (V.float() + 0.01).contiguous()
+    want = J.frobenius(K, V, Kh, Vh, 1)
+    assert want.shape[0] == 64
+    for _ in range(2):
+        got = J.frobenius_noalloc(K, V, Kh, Vh, 1)
+        assert torch.allclose(got, want, rtol=1e-12, atol=0.0)
+    Kf, Vf = K.float().contiguous(), V.float().contiguous()
+    want = J.frobenius(Kf, Vf, Kh, Vh, 2)
+    for _ in range(2):
+        got = J.frobenius_noalloc(Kf, Vf, Kh, Vh, 2)
+        assert torch.allclose(got, want, rtol=1e-12, atol=0.0)
