@@ -1,11 +1,13 @@
-"""KV compress throughput of the JoLT / FlashJoLT library on a Mistral-7B-shaped cache.
+"""KV compress throughput of the JoLT / FlashJoLT library on a LLaMA-3.1-8B-shaped 64K cache.
 
-One step = jolt_compress of the whole cache (K and V, 32 layers x 8 KV heads x 1024 tokens
-x 128 features, bf16) at the 2x budget, then again at the 3x budget.  `value` is input
-GB/s over the timed steps (inputs resident in HBM, L2 flushed between steps), `e2e` is
-the same metric through the public API with the caches copied in from pinned host memory
-and the blobs read back every step.  For N > 1 every rank compresses its own cache (weak
-scaling; the units of different caches are independent, so no collective is involved).
+One step = jolt_compress (FlashJoLT) of the whole cache (K and V, 32 layers x 8 KV heads x
+65536 tokens x 128 features, bf16, 8 GiB) at the 2x budget, then again at the 3x budget.
+`value` is input GB/s over the timed steps (inputs resident in HBM and larger than L2; the
+L2 is also flushed between steps), `e2e` is the same metric through the public API with
+the caches copied in from pinned host memory and the blobs read back every step.  The
+Mistral-7B-shaped cache (1024 tokens) is timed beside it as an extra key, with the JoLT
+(exact) arm.  For N > 1 every rank compresses its own cache (weak scaling; the units of
+different caches are independent, so no collective is involved).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--method randomized|exact]
   python bench.py --impl reference ...   # the float64 CPU oracle on a bounded sample
@@ -27,12 +29,9 @@ sys.path.insert(0, ROOT)
 METRIC = "KV compress throughput (input GB/s) at 2x/3x budget"
 RATIOS = (2.0, 3.0)
 L2_BYTES = 126 * 1024 * 1024
-# FP32 pipe: 148 SMs x 128 lanes, one FMA-class instruction per lane per clock
-SMS, FP32_LANES = 148, 128
-# DRAM bytes (read + write) of one table_kernel launch over the 16 units of the bench workload
-# from an ncu capture of that launch (profiles/table_kernel_mistral7b.md: 268.1 MB read +
-# 8.9 MB written); None whenever the kernel has changed since.
-TABLE_KERNEL_TRAFFIC_BYTES = 277.0e6
+# DRAM bytes (read + write) per launch of the dominant kernel from an ncu capture of the
+# current kernel, keyed by workload; a workload without an entry reports null
+KERNEL_TRAFFIC_BYTES = {}
 
 
 def parse():
@@ -42,7 +41,7 @@ def parse():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="jolt", choices=["jolt", "reference"])
     ap.add_argument("--method", default="randomized", choices=["randomized", "exact"])
-    ap.add_argument("--workload", default="mistral7b")
+    ap.add_argument("--workload", default="llama31_8b_64k")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extras", action="store_true", help="skip the exact-arm and decompress side figures")
     ap.add_argument("--profile-case", default=None, choices=["mistral7b_4layers", "mistral7b", "llama31_8b_64k"],
@@ -220,28 +219,43 @@ def load_peaks():
 
 
 # ------------------------------------------------------------------------------------------
-def oracle_sample(w, opts_j, seed, ratio, K=None, V=None):
-    """The float64 oracle as it stands on one unit (the keys of layer group 0) of the workload:
-    factors, distortion table, allocation at the unit's share of the budget, encoding."""
-    import numpy as np
+SAMPLE_TOKENS = 1024
+
+
+def oracle_sample_input(w, seed):
+    """The bounded sample the float64 oracle is timed on: the keys of layer group 0 of the
+    workload, restricted to its first SAMPLE_TOKENS tokens ([L_g, H, 1024, D]; for the
+    1024-token Mistral shape that is the whole unit)."""
+    from kv_cache_compression_group_b200 import synth
+    K = synth.make_cache(w, seed, kv=0, layers=range(0, w.layers_per_group))
+    return K[:, :, :min(w.T, SAMPLE_TOKENS)].contiguous()
+
+
+def oracle_sample(w, opts_j, seed, ratio, K):
+    """The float64 oracle as it stands on the sample unit K: factors, distortion table with
+    the workload's candidate sets, allocation at the unit's share of the budget, encoding."""
     import oracle as O
     from kv_cache_compression_group_b200 import synth
-    if K is None:
-        K = synth.make_cache(w, seed, kv=0, layers=range(0, w.layers_per_group))
     X = synth.to_f64(K)
+    Lg, H, T, D = X.shape
     oo = O.Options(opts_j.token_ranks, opts_j.feature_ranks, opts_j.bits, opts_j.method,
                    opts_j.oversample, opts_j.power_iters)
     t0 = time.perf_counter()
     f = O.unit_factors(X, 0, 0, oo, seed)
     tab = O.distortion_table(X, f.U_s, f.W_s, f.C_s, f.sigma, oo).reshape(1, -1)
-    S = w.layers_per_group * w.n_heads
-    B = O.bytes_table(w.T, w.D, S, oo).reshape(1, -1)
+    B = O.bytes_table(T, D, Lg * H, oo).reshape(1, -1)
     budget = int(X.size * 2 / ratio) - O.header_bytes(1)
     al = O.allocate(tab, B, budget)
     if al.status == "ok":
         O.encode_unit(X, f, oo, int(al.choice[0]), float(tab[0, al.choice[0]]))
     dt = time.perf_counter() - t0
     return dt, X.size * 2
+
+
+def sample_text(w, K, extra=""):
+    Lg, H, T, D = K.shape
+    return (f"one unit: keys of layer group 0 of {w.name}, first {T} of {w.T} tokens ([{Lg}, {H}, {T}, {D}] bf16, "
+            f"{K.numel() * 2 / 2**20:.0f} MiB), the workload's candidate sets{extra}")
 
 
 def cpu_threads():
@@ -256,34 +270,149 @@ def cpu_threads():
 
 # ------------------------------------------------------------------------------------------
 def run_reference(args, rank, world):
-    """The oracle on the host cores: each step is one unit of the workload at 2x or 3x."""
+    """The oracle on the host cores: each step is the sample unit at 2x or 3x (alternating)."""
     from kv_cache_compression_group_b200 import synth, jolt as J
     if rank != 0:
         return
     w = synth.WORKLOADS[args.workload]
     opts = J.default_options(w.T, w.D, args.method)
-    K = synth.make_cache(w, 0, kv=0, layers=range(0, w.layers_per_group))
+    K = oracle_sample_input(w, 0)
     times, nbytes = [], 0
     for i in range(args.warmup + args.steps):
-        dt, nb = oracle_sample(w, opts, 0, RATIOS[i % 2], K=K)
+        dt, nb = oracle_sample(w, opts, 0, RATIOS[i % 2], K)
         if i >= args.warmup:
             times.append(dt)
             nbytes += nb
     tot = sum(times)
     value = nbytes / tot / 1e9
     threads, cores = cpu_threads()
-    sample = (f"one unit per step (keys of layer group 0: [{w.layers_per_group}, {w.n_heads}, {w.T}, {w.D}] bf16, "
-              f"{w.layers_per_group * w.n_heads * w.T * w.D * 2 / 2**20:.0f} MiB), budgets alternating 2x / 3x")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": tot / len(times) * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": workload_config(w, args.method, opts),
         "cpu_baseline": {"value": value, "unit": "GB/s", "cores": threads, "host_cores": cores, "kind": "oracle",
-                         "sample": sample},
+                         "sample": sample_text(w, K, ", budgets alternating 2x / 3x, one unit per step")},
         "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------------------------------
+def fp32_peak(J, dev, stream):
+    """FP32-pipe rate measured in this process: FMAs per second of the library's probe kernel,
+    scalar (FFMA) and packed (FFMA2), best of three launches each after a warm-up.  Each FMA
+    counts as one operation, as in the algorithmic operation counts."""
+    import torch
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    sink = torch.empty(sms * 8 * 256, dtype=torch.float32, device=dev)
+    out = {}
+    for packed in (False, True):
+        J.fp32_rate_probe(packed, 2000, sink)
+        best = 0.0
+        for _ in range(3):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            ops = J.fp32_rate_probe(packed, 20000, sink)
+            b.record(stream)
+            torch.cuda.synchronize()
+            best = max(best, ops / (a.elapsed_time(b) / 1e3) / 1e12)
+        out["ffma2_tops" if packed else "ffma_tops"] = best
+    out["peak_tops"] = max(out["ffma_tops"], out["ffma2_tops"])
+    out["note"] = "measured in this run: FMAs per second of a probe kernel, 8 CTAs of 256 threads per SM"
+    return out
+
+
+def stage_rooflines(w, opts, n_units, prof, n_calls, per_call_ms, peaks, peak_src, alu):
+    """Algorithmic work of each library stage (per compress call) against its own bound, for
+    the stages that take more than 5 % of a compress.  Work counts what the method computes,
+    not what the implementation adds (the bf16 hi + lo halves of fp32 operands, recomputed
+    operators): achieved = algorithmic work / measured stage time."""
+    S = w.layers_per_group * w.n_heads
+    N = S * w.T * w.D                       # elements per unit
+    M = S * w.D
+    T = w.T
+    k = max(opts.token_ranks) + opts.oversample
+    q = opts.power_iters
+    rT, nD = max(opts.token_ranks), len(opts.feature_ranks)
+    hbm = float(peaks["hbm_gbs"])
+    tens = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
+    work = {
+        # products with the cache: Y = X Omega, then (Z = X^T Q, Y = X Q_z) per power iteration,
+        # then Z = X^T Q for the Rayleigh-Ritz Gram: 2 T M k each
+        "sketch_product": ("tensor", (2 + 2 * q) * 2.0 * T * M * k * n_units, "FLOP"),
+        # Cholesky-QR Grams: (q + 2) passes on T x k, q on M x k; m k^2 each (symmetric)
+        "qr_gram": ("tensor", ((q + 2) * T + q * M) * float(k) * k * n_units, "FLOP"),
+        # Q = Y L^{-T}: m k^2 per pass (triangular)
+        "qr_trsm": ("tensor", ((q + 2) * T + q * M) * float(k) * k * n_units, "FLOP"),
+        "ritz_vectors": ("tensor", 2.0 * T * k * rT * n_units, "FLOP"),
+        "table_kernel": ("alu", table_alu_ops(w, opts, n_units)[0], "op"),
+        "encode": ("hbm", (2.0 * N) * n_units, "B"),
+        "feature_factor": ("hbm", 2.0 * N * n_units, "B"),
+        "core": ("hbm", (2.0 * N + 2.0 * N * max(opts.feature_ranks) / w.D) * n_units, "B"),
+    }
+    lines = []
+    for name, (ms, launches, _) in sorted(prof.items(), key=lambda kv: -kv[1][0]):
+        ms_call = ms / n_calls
+        if ms_call < 0.05 * per_call_ms:
+            continue
+        line = {"kernel": name, "ms_per_launch": ms_call, "share_of_compress": ms_call / per_call_ms}
+        if name in work:
+            bound, amount, unit = work[name]
+            t = ms_call / 1e3
+            if bound == "tensor":
+                ach, peak, u = amount / t / 1e12, tens, "TFLOP/s"
+                src = f"{peak_src} bf16 dense, sustained"
+            elif bound == "hbm":
+                ach, peak, u = amount / t / 1e9, hbm, "GB/s"
+                src = f"{peak_src} HBM copy"
+            else:
+                ach, peak, u = amount / t / 1e12, alu["peak_tops"], "Top/s"
+                src = "measured FP32-pipe probe (best of scalar FFMA and packed FFMA2)"
+            line.update({"bound": bound, "achieved": ach, "peak": peak, "unit": u, "frac": ach / peak,
+                         "work_per_launch": amount, "work_unit": unit, "peak_source": src})
+        else:
+            line["bound"] = "latency"
+        lines.append(line)
+    return lines
+
+
+def mistral_extras(J, synth, dev, stream, flush):
+    """The Mistral-7B-shaped cache (1024 tokens): FlashJoLT compress at 2x and 3x (graph
+    replays, events around each call, L2 flushed before), and JoLT (exact) at 2x."""
+    import torch
+    w = synth.WORKLOADS["mistral7b"]
+    K, V = synth.make_cache(w, 0)
+    Kd, Vd = K.to(dev), V.to(dev)
+    out = {"workload": f"mistral7b: K and V [{w.n_layers}, {w.n_heads}, {w.T}, {w.D}] bf16, layer groups of 4"}
+    for meth in ("randomized", "exact"):
+        o2 = J.default_options(w.T, w.D, meth)
+        c2 = J.Compressor(w.n_layers, w.n_heads, w.T, w.D, w.layers_per_group, K.dtype, o2, dev)
+        res = {}
+        for ratio in ((2.0, 3.0) if meth == "randomized" else (2.0,)):
+            budget = int(w.bf16_bytes() / ratio)
+            blob = torch.empty(min(budget, c2.blob_max), dtype=torch.uint8, device=dev)
+            for _ in range(3):   # direct run, graph capture, one replay
+                c2.compress(Kd, Vd, budget, 0, blob=blob)
+            ts = []
+            for _ in range(5):
+                flush.zero_()
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                c2.compress(Kd, Vd, budget, 0, blob=blob)
+                b.record(stream)
+                torch.cuda.synchronize()
+                ts.append(a.elapsed_time(b))
+            ms = sorted(ts)[len(ts) // 2]
+            Ko, Vo = c2.decompress(blob)
+            ek, ev = J.relative_errors(Kd, Vd, Ko, Vo, w.layers_per_group)
+            res[f"{ratio:g}x"] = {"compress_ms": ms, "gbs": w.input_bytes() / ms / 1e6, "rel_err_K": ek, "rel_err_V": ev}
+        out["FlashJoLT" if meth == "randomized" else "JoLT"] = res
+        del c2
+    out["flashjolt_speedup_over_jolt_2x"] = out["JoLT"]["2x"]["compress_ms"] / out["FlashJoLT"]["2x"]["compress_ms"]
+    del Kd, Vd
+    torch.cuda.empty_cache()
+    return out
 
 
 # ------------------------------------------------------------------------------------------
@@ -435,22 +564,23 @@ def main():
     torch.cuda.synchronize()
     prof = J.profile_end()
 
-    # ---- roofline of the dominant stage ----------------------------------------------------
+    # ---- measured FP32-pipe peak (scalar FFMA and packed FFMA2 probes) -------------------
+    alu = fp32_peak(J, dev, stream)
+
+    # ---- roofline of every stage above 5 % of a compress ---------------------------------
     peaks, peak_src = load_peaks()
     stages = {k: {"ms_total": v[0], "launches": v[1], "ms_per_launch": v[0] / max(1, v[1])} for k, v in prof.items()}
-    dom = max(prof.items(), key=lambda kv: kv[1][0])[0] if prof else None
+    n_calls = 2 * len(RATIOS)
+    per_call_ms = t_ms / args.steps / len(RATIOS)
+    lines = stage_rooflines(w, opts, comp.n_units, prof, n_calls, per_call_ms, peaks, peak_src, alu)
+    leaf = [l for l in lines if l.get("bound") in ("alu", "tensor", "hbm")]
+    dom = max(leaf, key=lambda l: l["ms_per_launch"]) if leaf else None
     roofline = None
-    if "table_kernel" in prof:
-        ms, n, _ = prof["table_kernel"]
-        ops, per = table_alu_ops(w, opts, comp.n_units)
-        mhz = float(peaks.get("sm_max_mhz", 1965.0))
-        peak = SMS * FP32_LANES * mhz * 1e6 / 1e12
-        achieved = ops / (ms / n / 1e3) / 1e12
-        roofline = {"kernel": "table_kernel", "bound": "alu", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                    "frac": achieved / peak, "traffic": TABLE_KERNEL_TRAFFIC_BYTES,
-                    "note": f"peak = {SMS} SMs x {FP32_LANES} FP32 lanes x {mhz:.0f} MHz ({peak_src} max clock); "
-                            f"algorithmic work = {per} FP32-pipe ops per element per (r_T, r_D) candidate",
-                    "dominant_stage": dom}
+    if dom is not None:
+        roofline = dict(dom)
+        roofline["traffic"] = KERNEL_TRAFFIC_BYTES.get((w.name, dom["kernel"]))
+        roofline["timing"] = ("per-launch time from a separate pass with CUDA events around the stage on its "
+                              "launch stream (the timed steps replay CUDA graphs, which hold no events)")
 
     out = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
@@ -458,45 +588,30 @@ def main():
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": workload_config(w, args.method, opts),
         "e2e": e2e, "gpu_launches": int(launches), "clocks": clk, "roofline": roofline,
-        "stages": stages,
+        "stage_rooflines": lines, "alu_peak": alu, "stages": stages,
     }
 
     if rank == 0 and not args.no_extras:
-        # side figures: the exact (JoLT) arm and decompress, on the same cache
-        ex = {}
-        for meth in ("exact", "randomized"):
-            o2 = J.default_options(w.T, w.D, meth)
-            c2 = J.Compressor(w.n_layers, w.n_heads, w.T, w.D, w.layers_per_group, K.dtype, o2, dev)
-            for _ in range(3):   # direct run, graph capture, one replay
-                c2.compress(Kd, Vd, budgets[0], seed, blob=blobs[0])
-            torch.cuda.synchronize()
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            c2.compress(Kd, Vd, budgets[0], seed, blob=blobs[0])
-            b.record(stream)
-            torch.cuda.synchronize()
-            ms = a.elapsed_time(b)
-            Ko, Vo = c2.decompress(blobs[0])
-            torch.cuda.synchronize()
-            a.record(stream)
-            Ko, Vo = c2.decompress(blobs[0], K_out=Ko, V_out=Vo)
-            b.record(stream)
-            torch.cuda.synchronize()
-            dms = a.elapsed_time(b)
-            ek, evv = J.relative_errors(Kd, Vd, Ko.float(), Vo.float(), w.layers_per_group)
-            ex[meth] = {"compress_2x_ms": ms, "compress_2x_gbs": in_bytes / ms / 1e6,
-                        "latency_per_layer_group_ms": ms / w.n_groups, "decompress_ms": dms,
-                        "decompress_out_gbs": in_bytes / dms / 1e6, "rel_err_K": ek, "rel_err_V": evv}
-        ex["flashjolt_speedup_over_jolt"] = ex["exact"]["compress_2x_ms"] / ex["randomized"]["compress_2x_ms"]
-        out["arms_2x"] = ex
+        out["mistral7b"] = mistral_extras(J, synth, dev, stream, flush)
+        # decompress of the headline cache (output GB/s) and its relative errors
+        Ko, Vo = comp.decompress(blobs[0])
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        Ko, Vo = comp.decompress(blobs[0], K_out=Ko, V_out=Vo)
+        b.record(stream)
+        torch.cuda.synchronize()
+        dms = a.elapsed_time(b)
+        ek, evv = J.relative_errors(Kd, Vd, Ko, Vo, w.layers_per_group)
+        out["decompress_2x"] = {"ms": dms, "out_gbs": in_bytes / dms / 1e6, "rel_err_K": ek, "rel_err_V": evv}
+        del Ko, Vo
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        dt, nb = oracle_sample(w, opts, 0, RATIOS[0])
+        Ks = oracle_sample_input(w, 0)
+        dt, nb = oracle_sample(w, opts, 0, RATIOS[0], Ks)
         threads, cores = cpu_threads()
         out["cpu_baseline"] = {"value": nb / dt / 1e9, "unit": "GB/s", "cores": threads, "host_cores": cores,
-                               "kind": "oracle",
-                               "sample": f"one unit (keys of layer group 0, [{w.layers_per_group}, {w.n_heads}, "
-                                         f"{w.T}, {w.D}] bf16) at the 2x budget, {dt:.1f} s"}
+                               "kind": "oracle", "sample": sample_text(w, Ks, f", 2x budget, {dt:.1f} s")}
     ranks.barrier(world)
     ranks.shutdown(world)
     if rank == 0:

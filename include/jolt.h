@@ -146,7 +146,7 @@ jolt_status jolt_compress(const jolt_shape* shape, const void* k_dev, const void
  * modes; FlashJoLT swaps the exact token-mode SVD for a randomized one, abstract).
  *   u_dev : [n_units][n_tokens][ld_u] fp32, unrounded token factor (leading max r_T columns)
  *   w_dev : [n_units][head_dim][ld_w] fp32, unrounded feature factor (leading max r_D columns)
- *   ld_u >= max r_T, ld_w >= max r_D.  Columns ordered by descending singular value, the
+ *   ld_u >= max r_T and a multiple of 8, ld_w >= max r_D.  Columns ordered by descending singular value, the
  *   entry of largest magnitude of every column positive.  Asynchronous. */
 jolt_status jolt_factor(const jolt_shape* shape, const void* k_dev, const void* v_dev, const jolt_options* opts,
                         uint64_t seed, float* u_dev, int64_t ld_u, float* w_dev, int64_t ld_w, void* ws_dev,

@@ -10,7 +10,8 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libjolt.so")
 SOURCES = ["jolt_api.cu"]
-DEPS = ["jolt_api.cu", "common.cuh", "gemm.cuh", "kernels.cuh", "misc.cuh", "umma.cuh", "eig_cluster.cuh", "chol.cuh", "fp16_exact.cuh"]
+DEPS = ["jolt_api.cu", "common.cuh", "gemm.cuh", "kernels.cuh", "misc.cuh", "umma.cuh", "eig_cluster.cuh", "chol.cuh",
+        "fp16_exact.cuh", "table_tc.cuh"]
 
 
 def nvcc_cmd(out: str = LIB, extra=()) -> list:

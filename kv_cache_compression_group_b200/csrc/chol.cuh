@@ -417,3 +417,112 @@ __global__ void __launch_bounds__(CF_THREADS, 2)
 }
 
 }  // namespace jolt
+
+namespace jolt {
+
+// ------------------------------------------------------------------------------------------
+// Inverses of the 32 x 32 diagonal blocks of a Cholesky factor L held in the lower triangle
+// of G (column-major, ld gld; the layout a batched LAPACK-style Cholesky leaves), written in
+// fp64 to the upper part of the same diagonal block, W_II[r][s] at G[(I0 + r) * gld + I0 + s]
+// (s <= r): the convention of chol_factor_kernel, so tri_inv_large_kernel reads either.
+// One warp per (block, unit); lane c solves L_II x = e_c by forward substitution.  The warp
+// reads the whole block before any lane writes (the diagonal is overwritten).
+// ------------------------------------------------------------------------------------------
+__global__ void __launch_bounds__(32) diag_inv64_kernel(double* G, int k, long long gld, long long sG) {
+  const int I = blockIdx.x, u = blockIdx.y, lane = threadIdx.x;
+  const int I0 = I * CF_NB, nb = min(CF_NB, k - I0);
+  double* Gu = G + (long long)u * sG;
+  double x[CF_NB];
+#pragma unroll
+  for (int r = 0; r < CF_NB; ++r) {
+    double v = (r == lane) ? 1.0 : 0.0;
+    if (r < nb) {
+#pragma unroll
+      for (int q = 0; q < r; ++q) v = fma(-Gu[(long long)(I0 + q) * gld + I0 + r], x[q], v);
+      v = v / Gu[(long long)(I0 + r) * gld + I0 + r];
+    }
+    x[r] = v;
+  }
+  __syncwarp();
+  if (lane < nb) {
+#pragma unroll
+    for (int r = 0; r < CF_NB; ++r)
+      if (r >= lane && r < nb) Gu[(long long)(I0 + r) * gld + I0 + lane] = x[r];
+  }
+}
+
+// ------------------------------------------------------------------------------------------
+// W = L^{-1} for any k (the block-column recursion of tri_inv_kernel with the block column
+// kept in global fp64 scratch instead of shared memory):
+//   W_JJ = inv(L_JJ),   W_IJ = -inv(L_II) sum_{J <= K < I} L_IK W_KJ   (I > J).
+// G: L's blocks below the diagonal in the lower triangle, inv(L_II) in the upper part of
+// the diagonal blocks.  One CTA per (block column J, unit), 256 threads, thread (r, cg)
+// computes entries (r, cg + 8 j) of each 32 x 32 block.  scr: per unit and block column a
+// kq32 x 32 fp64 slab (row i of the slab = row i of W).  Output as tri_inv_kernel: WT[q][i] =
+// W[i][q] in fp32 at pitch ldw, zeros for i < J0 and for k <= i < ldw.
+// ------------------------------------------------------------------------------------------
+__global__ void __launch_bounds__(CF_THREADS) tri_inv_large_kernel(const double* G, int k, long long gld, long long sG,
+                                                                  double* scr, int kq32, float* WT, long long ldw,
+                                                                  long long sW) {
+  __shared__ double Ls[CF_NB][CF_P];    // L_IK, [r][q]
+  __shared__ double Xs[CF_NB][CF_P];    // W_KJ, [q][c]
+  __shared__ double Ts[CF_NB][CF_P];    // sum_K L_IK W_KJ
+  __shared__ double Ds[CF_NB][CF_P];    // inv(L_II)
+  const int J = blockIdx.x, u = blockIdx.y, tid = threadIdx.x;
+  const int nbk = (k + CF_NB - 1) / CF_NB;
+  const int J0 = J * CF_NB, nbJ = min(CF_NB, k - J0);
+  const double* Gu = G + (long long)u * sG;
+  double* X = scr + ((long long)u * nbk + J) * (long long)kq32 * CF_NB;   // X[i * 32 + c]
+  const int r = tid >> 3, cg = tid & 7;
+  // W_JJ
+  for (int idx = tid; idx < CF_NB * CF_NB; idx += CF_THREADS) {
+    const int rr = idx / CF_NB, c = idx % CF_NB;
+    X[(long long)(J0 + rr) * CF_NB + c] =
+        (rr < nbJ && c < nbJ && c <= rr) ? Gu[(long long)(J0 + rr) * gld + J0 + c] : 0.0;
+  }
+  __syncthreads();
+  for (int I = J + 1; I < nbk; ++I) {
+    const int I0 = I * CF_NB, nbI = min(CF_NB, k - I0);
+    double acc[4] = {0.0, 0.0, 0.0, 0.0};
+    for (int K = J; K < I; ++K) {
+      const int K0 = K * CF_NB, nbK = min(CF_NB, k - K0);
+      for (int idx = tid; idx < CF_NB * CF_NB; idx += CF_THREADS) {
+        const int a = idx / CF_NB, b = idx % CF_NB;
+        // L_IK[b][a] = L[I0 + b][K0 + a], column-major at G[(K0 + a) * gld + I0 + b]: consecutive
+        // threads read consecutive rows of one column
+        Ls[b][a] = (b < nbI && a < nbK) ? Gu[(long long)(K0 + a) * gld + I0 + b] : 0.0;
+        Xs[a][b] = a < nbK ? X[(long long)(K0 + a) * CF_NB + b] : 0.0;
+      }
+      __syncthreads();
+#pragma unroll 8
+      for (int q = 0; q < CF_NB; ++q) {
+        const double l = Ls[r][q];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[j] = fma(l, Xs[q][cg + 8 * j], acc[j]);
+      }
+      __syncthreads();
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) Ts[r][cg + 8 * j] = acc[j];
+    for (int idx = tid; idx < CF_NB * CF_NB; idx += CF_THREADS) {
+      const int rr = idx / CF_NB, s = idx % CF_NB;
+      Ds[rr][s] = (rr < nbI && s <= rr) ? Gu[(long long)(I0 + rr) * gld + I0 + s] : 0.0;
+    }
+    __syncthreads();
+    double out[4] = {0.0, 0.0, 0.0, 0.0};
+    for (int s = 0; s <= r; ++s) {
+      const double d = Ds[r][s];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) out[j] = fma(d, Ts[s][cg + 8 * j], out[j]);
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) X[(long long)(I0 + r) * CF_NB + cg + 8 * j] = r < nbI ? -out[j] : 0.0;
+    __syncthreads();
+  }
+  float* Wu = WT + (long long)u * sW;
+  for (int c = tid >> 5; c < nbJ; c += CF_THREADS / 32)
+    for (int i = tid & 31; i < ldw; i += 32)
+      Wu[(long long)(J0 + c) * ldw + i] = (i >= J0 && i < k) ? (float)X[(long long)i * CF_NB + c] : 0.f;
+}
+
+}  // namespace jolt

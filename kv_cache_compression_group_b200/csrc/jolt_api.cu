@@ -16,6 +16,7 @@
 #include "umma.cuh"
 #include "eig_cluster.cuh"
 #include "chol.cuh"
+#include "table_tc.cuh"
 
 using namespace jolt;
 
@@ -157,6 +158,11 @@ struct Bump {
   }
 };
 
+// Cholesky QR runs its Gram and its triangular product on the tensor cores for block widths
+// of at least QR_TC_MINK columns; a Gram partial sums QR_TC_CHUNK rows in fp32
+constexpr int QR_TC_MINK = 64;
+constexpr int QR_TC_CHUNK = 4096;
+
 struct Plan {
   int nL, H, T, D, Lg, S, G, NU, M, dtype;
   Cands cd;
@@ -169,9 +175,12 @@ struct Plan {
   size_t solver_host;
   // workspace offsets (bytes)
   size_t o_status, o_gd_part, o_gd, o_evals, o_Wf, o_Ws, o_Uf, o_Us, o_core, o_zc, o_ptmp, o_P, o_partial,
-      o_table, o_bytes, o_choice, o_lambda, o_hdr, o_umap, o_info, o_solver, o_fsolver, o_finfo, o_fevals, o_eigvec, o_eigscr;
+      o_table, o_bytes, o_choice, o_lambda, o_hdr, o_umap, o_info, o_solver, o_fsolver, o_finfo, o_fevals, o_eigvec, o_eigscr,
+      o_feigvec, o_feigscr;
+  int eig_n;              // order of the token-side eigen problems solved by the own solver (0: none)
   // token factor scratch (all units)
   size_t o_gt32, o_gt, o_vsel, o_lam, o_omega, o_Y, o_Zm, o_h, o_l, o_gpart, o_G, o_ptrs, o_Lr, o_Linv;
+  size_t o_wth, o_wtl, o_winv, o_vh, o_vl;   // tensor-core Cholesky QR: W^T = L^-T split, fp64 scratch; V split
   int qr_split_max;       // split-K of the Cholesky-QR Grams
   size_t ws_total;
   int tiles;
@@ -264,7 +273,16 @@ jolt_status make_plan(const jolt_shape* sh, const jolt_options* op, Plan* p) {
   // Cholesky-QR Grams: split-K so every fp32 partial sums at most 256 terms
   {
     long long mrows = op->method == JOLT_RANDOMIZED ? (M > T ? M : T) : (p->m_side ? T : 0);
-    p->qr_split_max = mrows > 0 ? (int)ceil_div(mrows, 256) : 1;
+    const int kq = op->method == JOLT_RANDOMIZED ? (int)round_up(p->rTmax + op->oversample, 8) : p->rTmax;
+    if (kq >= QR_TC_MINK) {
+      // tensor-core Grams: two products x split-K chunks of QR_TC_CHUNK rows; the
+      // Rayleigh-Ritz Gram (M rows, chunks of 256) shares the buffer
+      long long need = 2 * ceil_div(mrows, QR_TC_CHUNK);
+      if (op->method == JOLT_RANDOMIZED && ceil_div(M, 256) > need) need = ceil_div(M, 256);
+      p->qr_split_max = mrows > 0 ? (int)need : 1;
+    } else {
+      p->qr_split_max = mrows > 0 ? (int)ceil_div(mrows, 256) : 1;
+    }
   }
   // cuSOLVER device workspace: with a device present the batched eigen solver is asked for
   // its exact need; without one (size queries on a host) a bound is used.
@@ -339,9 +357,10 @@ jolt_status make_plan(const jolt_shape* sh, const jolt_options* op, Plan* p) {
     p->o_gt = b.take((size_t)NU * n * n * 8);
     p->o_lam = b.take((size_t)NU * p->rTmax * 8 + 256);
     if (p->m_side) {
+      // split copies of V (M rows) for the back-projection and of U (T rows) for its QR
       p->o_vsel = b.take((size_t)NU * M * p->ldU * 4);
-      p->o_h = b.take((size_t)NU * M * p->ldU * 2);
-      p->o_l = b.take((size_t)NU * M * p->ldU * 2);
+      p->o_h = b.take((size_t)NU * (M > T ? M : T) * p->ldU * 2);
+      p->o_l = b.take((size_t)NU * (M > T ? M : T) * p->ldU * 2);
     }
   } else {
     const int kp = p->kp;
@@ -352,12 +371,20 @@ jolt_status make_plan(const jolt_shape* sh, const jolt_options* op, Plan* p) {
     p->o_h = b.take((size_t)NU * big * kp * 2);
     p->o_l = b.take((size_t)NU * big * kp * 2);
     p->o_vsel = b.take((size_t)NU * kp * p->ldU * 4);
-    if (p->k >= 2 && p->k <= eigc::MAXN) {
-      p->o_eigvec = b.take((size_t)NU * p->k * p->k * 8);
-      p->o_eigscr = b.take((size_t)NU * eigc::scratch_doubles(p->k) * 8);
+  }
+  // the own eigen solver (order <= 256): the feature factor (n = D, auxiliary stream) and the
+  // token-side problem (Rayleigh-Ritz, n = k; exact route, n = T or M) have separate buffers
+  p->o_feigvec = b.take((size_t)NU * D * D * 8);
+  p->o_feigscr = b.take((size_t)NU * eigc::scratch_doubles(D) * 8);
+  {
+    const long long ntok = op->method == JOLT_EXACT ? (p->m_side ? M : T) : p->k;
+    p->eig_n = (ntok >= 2 && ntok <= eigc::MAXN) ? (int)ntok : 0;
+    if (p->eig_n) {
+      p->o_eigvec = b.take((size_t)NU * ntok * ntok * 8);
+      p->o_eigscr = b.take((size_t)NU * eigc::scratch_doubles((int)ntok) * 8);
     }
   }
-  p->o_Lr = p->o_Linv = 0;
+  p->o_Lr = p->o_Linv = p->o_wth = p->o_wtl = p->o_winv = p->o_vh = p->o_vl = 0;
   if (op->method == JOLT_RANDOMIZED || p->m_side) {
     p->o_gpart = b.take((size_t)NU * p->qr_split_max * kq * kq * 4);
     p->o_G = b.take((size_t)NU * kq * kq * 8);
@@ -365,6 +392,16 @@ jolt_status make_plan(const jolt_shape* sh, const jolt_options* op, Plan* p) {
     p->o_Lr = b.take((size_t)NU * round_up(kq, 32) * round_up(kq, 32) * 4);
     p->o_ptrs = b.take((size_t)NU * 8 + 64);
     p->o_Linv = b.take((size_t)NU * round_up(kq, 32) * 32 * 4);   // inverses of the 32 x 32 diagonal blocks
+    if (kq >= QR_TC_MINK) {
+      const size_t kq32 = round_up(kq, 32);
+      p->o_wth = b.take((size_t)NU * kq32 * kq32 * 2);
+      p->o_wtl = b.take((size_t)NU * kq32 * kq32 * 2);
+      p->o_winv = b.take((size_t)NU * kq32 * kq32 * 8);
+      if (op->method == JOLT_RANDOMIZED) {
+        p->o_vh = b.take((size_t)NU * kq * p->ldU * 2);
+        p->o_vl = b.take((size_t)NU * kq * p->ldU * 2);
+      }
+    }
   }
   p->ws_total = b.off;
 
@@ -504,11 +541,16 @@ jolt_status sym_eig_batched(const Ctx& c, double* A, int64_t n, double* w, int64
 jolt_status sym_eig_top(const Ctx& c, double* S, int n, int nbatch, int r, float* out_f32, bf16* out_bf16,
                         long long ldo, long long sout, double* out_vals) {
   double* w = c.at<double>(c.side ? c.p.o_fevals : c.p.o_evals);
-  if (c.p.o_eigscr && n == c.p.k && n >= 2 && n <= eigc::MAXN) {
-    // the Rayleigh-Ritz problem: one 8-CTA cluster per matrix
-    ProfScope ps("sym_eig", c.st, nbatch);
-    double* V = c.at<double>(c.p.o_eigvec);
-    double* scr = c.at<double>(c.p.o_eigscr);
+  const bool own = c.side ? (n == c.p.D && n >= 2 && n <= eigc::MAXN) : (c.p.eig_n != 0 && n == c.p.eig_n);
+  if (own) {
+    // one 8-CTA cluster per matrix (csrc/eig_cluster.cuh)
+    ProfScope ps(c.side ? "feature_eig" : "sym_eig", c.st, nbatch);
+    double* V = c.at<double>(c.side ? c.p.o_feigvec : c.p.o_eigvec);
+    double* scr = c.at<double>(c.side ? c.p.o_feigscr : c.p.o_eigscr);
+    // a non-finite matrix becomes the identity (and raises the status), as before cuSOLVER
+    count_launch(), sanitize_sym_batched_kernel<<<(unsigned)nbatch, 1024, 0, c.st>>>(S, n, n, (long long)n * n,
+                                                                                      c.status());
+    CUDA_TRY(cudaGetLastError());
     const size_t sm = eigc::smem_bytes();
     CUDA_TRY(cudaFuncSetAttribute(sym_eig_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm));
     count_launch(), sym_eig_cluster_kernel<<<(unsigned)(nbatch * eigc::CL), eigc::THREADS, sm, c.st>>>(
@@ -541,8 +583,14 @@ jolt_status launch_trsm_panel(const Ctx& c, float* Y, long long m, int k, int ld
   return JOLT_OK;
 }
 
+jolt_status cholqr_tc(const Ctx& c, float* Y, long long m, int k, int ld, int passes);
+
 jolt_status cholqr_batched(const Ctx& c, float* Y, long long m, int k, int ld, int passes) {
   const Plan& p = c.p;
+  if (p.o_wth) {
+    if (ld % 8) return fail(JOLT_ERR_INVALID_ARG, "token factor pitch %d not a multiple of 8", ld);
+    return cholqr_tc(c, Y, m, k, ld, passes);
+  }
   ProfScope ps("cholesky_qr", c.st, p.NU);
   Solver* s = nullptr;
   JTRY(solver_get(c.st, &s));
@@ -684,6 +732,135 @@ jolt_status cache_maps(const Ctx& c, bool rows, CUtensorMap* mk, CUtensorMap* mv
 jolt_status umma_run(const UmmaMaps& m, const UmmaArgs& a, int nb, cudaStream_t st) {
   cudaError_t e = launch_umma(m, a, nb, st);
   if (e != cudaSuccess) return fail(JOLT_ERR_CUDA, "tensor-core GEMM: %s", cudaGetErrorString(e));
+  return JOLT_OK;
+}
+
+// Cholesky QR on the tensor cores (block widths >= QR_TC_MINK), in place on every unit's
+// m x k block Y (fp32, pitch ld, unit stride m * ld; columns k..ld zero):
+//   Y = Yh + Yl (bf16 hi + lo, Y - Yh - Yl = O(2^-17 |Y|));
+//   G = Yh^T Yh + Yh^T Yl + Yl^T Yh on tcgen05 (upper tiles only, split-K partials of
+//       QR_TC_CHUNK rows in fp32, summed in fp64) -- the dropped Yl^T Yl is O(2^-18 |Y|^2);
+//   G = L L^T in fp64 (own kernel for k <= 256, else the batched LAPACK-style Cholesky) and
+//   W = L^{-1} block column by block column in fp64 (tri_inv_kernel / tri_inv_large_kernel);
+//   Q = Y W^T = Yh (Wh + Wl)^T + Yl Wh^T on tcgen05, the K range of each output tile cut at
+//       the diagonal (W^T is upper triangular).
+// `passes` = 2 gives CholeskyQR2.
+jolt_status cholqr_tc(const Ctx& c, float* Y, long long m, int k, int ld, int passes) {
+  const Plan& p = c.p;
+  ProfScope ps("cholesky_qr", c.st, p.NU);
+  if (k > 1024) return fail(JOLT_ERR_UNSUPPORTED_SHAPE, "Cholesky QR of more than 1024 columns");
+  if (ld % 8) return fail(JOLT_ERR_UNSUPPORTED_SHAPE, "Cholesky QR pitch %d not a multiple of 8", ld);
+  bf16* yh = c.at<bf16>(p.o_h);
+  bf16* yl = c.at<bf16>(p.o_l);
+  float* gpart = c.at<float>(p.o_gpart);
+  double* G = c.at<double>(p.o_G);
+  float* WT = c.at<float>(p.o_Lr);
+  bf16* wth = c.at<bf16>(p.o_wth);
+  bf16* wtl = c.at<bf16>(p.o_wtl);
+  double** ptrs = c.at<double*>(p.o_ptrs);
+  int* info = c.at<int>(p.o_info);
+  const int gld = ld, kq32 = (int)round_up(k, 32), nbk = (int)ceil_div(k, 32);
+  const long long sG = (long long)k * gld, sW = (long long)kq32 * kq32;
+  const int ns = (int)ceil_div(m, QR_TC_CHUNK);
+  if (2 * ns > p.qr_split_max) return fail(JOLT_ERR_WORKSPACE_TOO_SMALL, "Gram partial slots");
+  const long long nY = (long long)p.NU * m * ld;
+  UmmaMaps my, mw;
+  if (!map_dense(&my.a0, yh, ld, m, p.NU) || !map_dense(&my.a1, yl, ld, m, p.NU) ||
+      !map_dense(&mw.b0, wth, kq32, kq32, p.NU) || !map_dense(&mw.b1, wtl, kq32, kq32, p.NU))
+    return fail(JOLT_ERR_CUDA, "tensor map of the Cholesky QR operands refused");
+  // rows k..kq32 of W^T are never written: zero them once (they meet zero columns of Y)
+  CUDA_TRY(cudaMemsetAsync(WT, 0, (size_t)p.NU * sW * 4, c.st));
+  for (int pass = 0; pass < passes; ++pass) {
+    count_launch(), split_bf16_cols_kernel<<<grid1d(nY), 256, 0, c.st>>>(Y, yh, yl, nY, ld, k);
+    CUDA_TRY(cudaGetLastError());
+    {
+      ProfScope ps1("qr_gram", c.st, p.NU);
+      UmmaArgs g;
+      g.M = g.N = k;
+      g.K = (int)m;
+      g.batch = p.NU;
+      g.splits = ns;
+      g.kchunk = QR_TC_CHUNK;
+      g.A.mode = UM_DENSE_MN;
+      g.B.mode = UM_DENSE_MN;
+      g.tri = 1;
+      g.bn = 128;
+      g.C = gpart;
+      g.ldc = gld;
+      g.sC = (long long)2 * ns * k * gld;
+      g.ssplit = (long long)k * gld;
+      g.status = c.status();
+      UmmaMaps m1;   // Yh^T (Yh + Yl)
+      m1.a0 = m1.a1 = my.a0;
+      m1.b0 = my.a0;
+      m1.b1 = my.a1;
+      JTRY(umma_run(m1, g, 2, c.st));
+      UmmaMaps m2;   // Yl^T Yh
+      m2.a0 = m2.a1 = my.a1;
+      m2.b0 = m2.b1 = my.a0;
+      g.C = gpart + (long long)ns * k * gld;
+      JTRY(umma_run(m2, g, 1, c.st));
+      count_launch(), reduce_upper_sym_kernel<<<grid1d((long long)p.NU * k * k), 256, 0, c.st>>>(gpart, G, p.NU,
+                                                                                                  2 * ns, k, gld);
+      CUDA_TRY(cudaGetLastError());
+    }
+    {
+      ProfScope ps2("qr_factor", c.st, p.NU);
+      if (k <= CF_MAXK && gld % 4 == 0) {
+        CUDA_TRY(cudaFuncSetAttribute(chol_factor_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)chol_factor_smem()));
+        count_launch(), chol_factor_kernel<<<p.NU, CF_FT, chol_factor_smem(), c.st>>>(G, k, gld, sG, c.status());
+        CUDA_TRY(cudaGetLastError());
+        CUDA_TRY(cudaFuncSetAttribute(tri_inv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)tri_inv_smem()));
+        count_launch(), tri_inv_kernel<<<dim3(nbk, p.NU), CF_THREADS, tri_inv_smem(), c.st>>>(G, k, gld, sG, WT, kq32,
+                                                                                               sW);
+        CUDA_TRY(cudaGetLastError());
+      } else {
+        Solver* s = nullptr;
+        JTRY(solver_get(c.st, &s));
+        count_launch(), sanitize_sym_batched_kernel<<<p.NU, 1024, 0, c.st>>>(G, k, gld, sG, c.status());
+        count_launch(), ptr_array_kernel<<<1, 64, 0, c.st>>>(ptrs, G, sG, p.NU);
+        CUDA_TRY(cudaGetLastError());
+        SOLVER_TRY(cusolverDnDpotrfBatched(s->h, CUBLAS_FILL_MODE_LOWER, k, ptrs, gld, info, p.NU));
+        count_launch(), info_check_kernel<<<(unsigned)ceil_div(p.NU, 32), 32, 0, c.st>>>(info, p.NU, c.status(),
+                                                                                          DEV_ERR_FACTOR);
+        count_launch(), diag_inv64_kernel<<<dim3(nbk, p.NU), 32, 0, c.st>>>(G, k, gld, sG);
+        count_launch(), tri_inv_large_kernel<<<dim3(nbk, p.NU), CF_THREADS, 0, c.st>>>(
+            G, k, gld, sG, c.at<double>(p.o_winv), kq32, WT, kq32, sW);
+        CUDA_TRY(cudaGetLastError());
+      }
+    }
+    {
+      ProfScope ps3("qr_trsm", c.st, p.NU);
+      const long long nW = (long long)p.NU * sW;
+      count_launch(), split_bf16_kernel<<<grid1d(nW), 256, 0, c.st>>>(WT, wth, wtl, nW);
+      CUDA_TRY(cudaGetLastError());
+      UmmaArgs q;
+      q.M = (int)m;
+      q.N = k;
+      q.K = k;
+      q.batch = p.NU;
+      q.A.mode = UM_DENSE_K;
+      q.B.mode = UM_DENSE_MN;
+      q.tri = 2;
+      q.bn = 128;
+      q.C = Y;
+      q.ldc = ld;
+      q.sC = m * ld;
+      q.status = c.status();
+      UmmaMaps m1;   // Yh (Wh + Wl)^T
+      m1.a0 = m1.a1 = my.a0;
+      m1.b0 = mw.b0;
+      m1.b1 = mw.b1;
+      JTRY(umma_run(m1, q, 2, c.st));
+      UmmaMaps m2;   // + Yl Wh^T
+      m2.a0 = m2.a1 = my.a1;
+      m2.b0 = m2.b1 = mw.b0;
+      q.c_accum = 1;
+      JTRY(umma_run(m2, q, 1, c.st));
+    }
+  }
   return JOLT_OK;
 }
 
@@ -970,9 +1147,47 @@ jolt_status run_token_randomized(const Ctx& c, float* Uf, long long ldUf) {
     CUDA_TRY(cudaGetLastError());
   }
   float* V = c.at<float>(p.o_vsel);
+  CUDA_TRY(cudaMemsetAsync(V, 0, (size_t)NU * kp * p.ldU * 4, c.st));   // rows k..kp stay zero
   JTRY(sym_eig_top(c, S, k, NU, p.rTmax, V, nullptr, p.ldU, (long long)kp * p.ldU, nullptr));
   // U = Q V
   ProfScope ps2("ritz_vectors", c.st, NU);
+  if (p.o_vh) {
+    // on the tensor cores: Q = Qh + Ql, V = Vh + Vl (bf16 hi + lo); U = Qh (Vh + Vl) + Ql Vh
+    bf16* qh = c.at<bf16>(p.o_h);
+    bf16* ql = c.at<bf16>(p.o_l);
+    bf16* vh = c.at<bf16>(p.o_vh);
+    bf16* vl = c.at<bf16>(p.o_vl);
+    const long long nQ = (long long)NU * T * kp, nV = (long long)NU * kp * p.ldU;
+    count_launch(), split_bf16_cols_kernel<<<grid1d(nQ), 256, 0, c.st>>>(Y, qh, ql, nQ, kp, k);
+    count_launch(), split_bf16_kernel<<<grid1d(nV), 256, 0, c.st>>>(V, vh, vl, nV);
+    CUDA_TRY(cudaGetLastError());
+    UmmaMaps mq, mv;
+    if (!map_dense(&mq.a0, qh, kp, T, NU) || !map_dense(&mq.a1, ql, kp, T, NU) ||
+        !map_dense(&mv.b0, vh, p.ldU, kp, NU) || !map_dense(&mv.b1, vl, p.ldU, kp, NU))
+      return fail(JOLT_ERR_CUDA, "tensor map of the Ritz vectors refused");
+    UmmaArgs a;
+    a.M = T;
+    a.N = p.rTmax;
+    a.K = kp;
+    a.batch = NU;
+    a.A.mode = UM_DENSE_K;
+    a.B.mode = UM_DENSE_MN;
+    a.C = Uf;
+    a.ldc = ldUf;
+    a.sC = (long long)T * ldUf;
+    a.status = c.status();
+    UmmaMaps m1;
+    m1.a0 = m1.a1 = mq.a0;
+    m1.b0 = mv.b0;
+    m1.b1 = mv.b1;
+    JTRY(umma_run(m1, a, 2, c.st));
+    UmmaMaps m2;
+    m2.a0 = m2.a1 = mq.a1;
+    m2.b0 = m2.b1 = mv.b0;
+    a.c_accum = 1;
+    JTRY(umma_run(m2, a, 1, c.st));
+    return JOLT_OK;
+  }
   GemmParams uq;
   uq.M = T;
   uq.N = p.rTmax;
@@ -1138,56 +1353,41 @@ jolt_status rotate_rows(const Ctx& c, const float* in, bf16* out, long long nrow
 
 // P'(r_D) for one unit: bf16(rotate(C_s[:, :rT, :r_D] W_s[:, :r_D]^T)), rows rT of every slice
 // out layout [S][rTslice][D] (rows >= rT of a slice are not written meaningfully)
-jolt_status pmat_unit(const Ctx& c, int u, const bf16* core_u, long long ldC, int rT, int rTslice, const bf16* Ws_u,
-                      long long ldW, int rD, float* ptmp, bf16* out, const int* umap) {
-  const Plan& p = c.p;
-  GemmParams g;
-  g.M = rT;
-  g.N = p.D;
-  g.K = rD;
-  g.batch = p.S;
-  g.A.ptr = core_u;
-  g.A.kmajor = true;
-  g.A.ld = ldC;
-  g.A.sbatch = (long long)rT * ldC;
-  g.B.ptr = Ws_u;
-  g.B.kmajor = true;  // B(j, d) = W_s[d][j]
-  g.B.ld = ldW;
-  g.C = ptmp;
-  g.ldc = p.D;
-  g.sbatchC = (long long)rTslice * p.D;
-  g.c_type = 0;
-  JTRY(gemm(g, 0, 0, c.st));
-  JTRY(rotate_rows(c, ptmp, out, (long long)p.S * rTslice, (long long)p.S * rTslice, umap + u));
+template <int D>
+jolt_status launch_pmat(const Ctx& c, const bf16* core, long long ldC, long long sC, int rT, int rD, const bf16* Ws,
+                        long long ldW, long long sW, int nb, const int* umap, bf16* out, long long sOut) {
+  count_launch(), pmat_exact_kernel<D><<<dim3((unsigned)ceil_div(rT, PX_ROWS), (unsigned)nb), 256, 0, c.st>>>(
+      core, ldC, sC, rT, rD, Ws, ldW, sW, c.p.S, umap, c.seed, out, sOut);
+  CUDA_TRY(cudaGetLastError());
   return JOLT_OK;
 }
 
-// P'(r_D) of every unit: bf16(rotate(C_s[:, :rT, :r_D] W_s[:, :r_D]^T)); out layout
-// [unit][S][rTslice][D] (unit stride S*rTslice*D)
-jolt_status pmat_all(const Ctx& c, const bf16* core, long long ldC, int rT, int rTslice, const bf16* Ws, long long ldW,
-                     int rD, float* ptmp, bf16* out, const int* umap) {
+// P'(r_D) of the rT leading token ranks of nb batch entries (slices; entry b of unit umap[b / S]):
+// bf16(rotate(C_b[:rT, :r_D] W[:, :r_D]^T)) in fp64 (pmat_exact_kernel); out entry stride sOut
+jolt_status pmat_run(const Ctx& c, const bf16* core, long long ldC, long long sC, int rT, const bf16* Ws, long long ldW,
+                     long long sW, int rD, int nb, const int* umap, bf16* out, long long sOut) {
+  switch (c.p.D) {
+    case 16: return launch_pmat<16>(c, core, ldC, sC, rT, rD, Ws, ldW, sW, nb, umap, out, sOut);
+    case 32: return launch_pmat<32>(c, core, ldC, sC, rT, rD, Ws, ldW, sW, nb, umap, out, sOut);
+    case 64: return launch_pmat<64>(c, core, ldC, sC, rT, rD, Ws, ldW, sW, nb, umap, out, sOut);
+    default: return launch_pmat<128>(c, core, ldC, sC, rT, rD, Ws, ldW, sW, nb, umap, out, sOut);
+  }
+}
+
+// one unit's operator (the decoder): S slices of core_u (slice stride rT * ldC), W of unit u
+jolt_status pmat_unit(const Ctx& c, int u, const bf16* core_u, long long ldC, int rT, int rTslice, const bf16* Ws_u,
+                      long long ldW, int rD, float* /*ptmp*/, bf16* out, const int* umap) {
   const Plan& p = c.p;
-  GemmParams g;
-  g.M = rT;
-  g.N = p.D;
-  g.K = rD;
-  g.batch = p.NU * p.S;
-  g.A.ptr = core;
-  g.A.kmajor = true;
-  g.A.ld = ldC;
-  g.A.sbatch = (long long)rT * ldC;
-  g.B.ptr = Ws;
-  g.B.kmajor = true;  // B(j, d) = W_s[d][j]
-  g.B.ld = ldW;
-  g.B.sbatch = (long long)p.D * ldW;
-  g.B.bdiv = p.S;
-  g.C = ptmp;
-  g.ldc = p.D;
-  g.sbatchC = (long long)rTslice * p.D;
-  g.c_type = 0;
-  JTRY(gemm(g, 0, 0, c.st));
-  JTRY(rotate_rows(c, ptmp, out, (long long)p.NU * p.S * rTslice, (long long)p.S * rTslice, umap));
-  return JOLT_OK;
+  return pmat_run(c, core_u, ldC, (long long)rT * ldC, rT, Ws_u, ldW, 0, rD, p.S, umap + u, out,
+                  (long long)rTslice * p.D);
+}
+
+// P'(r_D) of every unit; out layout [unit][S][rTslice][D] (unit stride S*rTslice*D)
+jolt_status pmat_all(const Ctx& c, const bf16* core, long long ldC, int rT, int rTslice, const bf16* Ws, long long ldW,
+                     int rD, float* /*ptmp*/, bf16* out, const int* umap) {
+  const Plan& p = c.p;
+  return pmat_run(c, core, ldC, (long long)rT * ldC, rT, Ws, ldW, (long long)p.D * ldW, rD, p.NU * p.S, umap, out,
+                  (long long)rTslice * p.D);
 }
 
 jolt_status fill_umap(const Ctx& c, int* umap, int n) {
@@ -1219,6 +1419,36 @@ jolt_status launch_table_D(const Ctx& c, const TableArgs& a) {
   return c.p.dtype == JOLT_BF16 ? launch_table_T<D, bf16>(c, a) : launch_table_T<D, float>(c, a);
 }
 
+// the tensor-core table kernel takes D = 128 with at most 4 token-rank cuts, each a multiple
+// of 16 (one K step of the MMA never straddles two cuts), and a U pitch of 16-byte rows
+bool table_tc_ok(const Plan& p, long long ldU) {
+  if (p.D != ttc::DIM || p.cd.nT > ttc::MAXT || ldU % 8) return false;
+  for (int i = 0; i < p.cd.nT; ++i)
+    if (p.cd.rT[i] % 16) return false;
+  return true;
+}
+
+template <typename TX, typename BITS>
+jolt_status launch_table_tc_B(const Ctx& c, const CUtensorMap& mu, const CUtensorMap& mp, const TableTcArgs& a) {
+  CUDA_TRY(cudaFuncSetAttribute(table_tc_kernel<TX, BITS>, cudaFuncAttributeMaxDynamicSharedMemorySize, ttc::SMEM));
+  count_launch(), table_tc_kernel<TX, BITS><<<dim3(a.tiles, c.p.S, c.p.NU), ttc::THREADS, ttc::SMEM, c.st>>>(mu, mp, a);
+  CUDA_TRY(cudaGetLastError());
+  return JOLT_OK;
+}
+
+jolt_status launch_table_tc(const Ctx& c, const bf16* Us, long long ldU, const bf16* P, const TableTcArgs& a) {
+  const Plan& p = c.p;
+  CUtensorMap mu, mp;
+  if (!map_dense(&mu, Us, ldU, p.T, p.NU) || !map_dense(&mp, P, p.D, p.rTmax, (long long)p.cd.nD * p.NU * p.S))
+    return fail(JOLT_ERR_CUDA, "tensor map of the table operands refused");
+  const Cands& cd = p.cd;
+  const bool dflt = cd.nB == 6 && cd.bits[0] == 0 && cd.bits[1] == 1 && cd.bits[2] == 2 && cd.bits[3] == 3 &&
+                    cd.bits[4] == 4 && cd.bits[5] == 8;
+  if (p.dtype == JOLT_BF16)
+    return dflt ? launch_table_tc_B<bf16, DefaultBits>(c, mu, mp, a) : launch_table_tc_B<bf16, void>(c, mu, mp, a);
+  return dflt ? launch_table_tc_B<float, DefaultBits>(c, mu, mp, a) : launch_table_tc_B<float, void>(c, mu, mp, a);
+}
+
 jolt_status run_table(const Ctx& c, const bf16* Us, long long ldU, const bf16* Ws, long long ldW, bf16* core,
                       double* table) {
   const Plan& p = c.p;
@@ -1247,7 +1477,19 @@ jolt_status run_table(const Ctx& c, const bf16* Us, long long ldU, const bf16* W
   a.seed = c.seed;
   a.partial = c.at<double>(p.o_partial);
   a.tiles = p.tiles;
-  {
+  int tiles = p.tiles;
+  if (table_tc_ok(p, ldU)) {
+    ProfScope ps("table_kernel", c.st, p.NU);
+    TableTcArgs t;
+    t.cv = a.cv;
+    t.rTmax = p.rTmax;
+    t.cand = p.cd;
+    t.seed = c.seed;
+    t.partial = a.partial;
+    t.tiles = tiles = (int)ceil_div(p.T, ttc::ROWS);
+    t.status = c.status();
+    JTRY(launch_table_tc(c, Us, ldU, P, t));
+  } else {
     ProfScope ps("table_kernel", c.st, p.NU);
     switch (p.D) {
       case 16: JTRY(launch_table_D<16>(c, a)); break;
@@ -1257,7 +1499,7 @@ jolt_status run_table(const Ctx& c, const bf16* Us, long long ldU, const bf16* W
     }
   }
   count_launch(), table_reduce_kernel<<<(unsigned)ceil_div((long long)p.NU * p.nC, 128), 128, 0, c.st>>>(
-      a.partial, table, p.NU, p.S, p.tiles, p.cd.nT, p.cd.nD, p.cd.nB);
+      a.partial, table, p.NU, p.S, tiles, p.cd.nT, p.cd.nD, p.cd.nB);
   CUDA_TRY(cudaGetLastError());
   return JOLT_OK;
 }
@@ -1503,6 +1745,7 @@ jolt_status jolt_factor(const jolt_shape* shape, const void* k_dev, const void* 
   JTRY(check_ws(p, ws_dev, ws_bytes));
   JTRY(check_inputs(p, k_dev, v_dev));
   if (!u_dev || !w_dev || ld_u < p.rTmax || ld_w < p.rDmax) return fail(JOLT_ERR_INVALID_ARG, "factor outputs");
+  if (ld_u % 8) return fail(JOLT_ERR_INVALID_ARG, "ld_u %lld not a multiple of 8", (long long)ld_u);
   Ctx c{p, (unsigned char*)ws_dev, (cudaStream_t)stream, k_dev, v_dev, seed};
   return run_factor(c, u_dev, ld_u, w_dev, ld_w, nullptr, nullptr);
 }

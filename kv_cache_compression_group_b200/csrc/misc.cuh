@@ -99,7 +99,9 @@ __global__ void eig_select_kernel(const double* vals, const double* vecs, int n,
     }
     __syncthreads();
   }
-  const double sgn = col[besti[0] * inc] < 0 ? -1.0 : 1.0;
+  // no finite entry (a non-finite input, already reported in the status word): sign +1
+  const int piv = besti[0] < n ? besti[0] : 0;
+  const double sgn = col[(long long)piv * inc] < 0 ? -1.0 : 1.0;
   for (int i = threadIdx.x; i < n; i += blockDim.x) {
     double v = sgn * col[i * inc];
     long long o = (long long)u * sout + (long long)i * ldo + j;
@@ -135,7 +137,8 @@ __global__ void col_sign_fix_kernel(float* A, long long lda, long long sA, int n
     }
     __syncthreads();
   }
-  const float sgn = a[(long long)besti[0] * lda + j] < 0 ? -1.f : 1.f;
+  const int piv = besti[0] < n ? besti[0] : 0;   // no finite entry: sign +1
+  const float sgn = a[(long long)piv * lda + j] < 0 ? -1.f : 1.f;
   __syncthreads();
   for (int i = threadIdx.x; i < n; i += blockDim.x) {
     float v = sgn * a[(long long)i * lda + j];
@@ -165,6 +168,17 @@ __global__ void omega_kernel(bf16* om, int M, int k, long long ld, long long sun
 __global__ void split_bf16_kernel(const float* x, bf16* hi, bf16* lo, long long n) {
   for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
     float v = x[i];
+    bf16 h = __float2bfloat16_rn(v);
+    hi[i] = h;
+    lo[i] = __float2bfloat16_rn(v - __bfloat162float(h));
+  }
+}
+
+// the same split of a row-major block of pitch ld, columns k..ld written as zeros (they enter
+// tensor-core K blocks that must contribute nothing)
+__global__ void split_bf16_cols_kernel(const float* x, bf16* hi, bf16* lo, long long n, int ld, int k) {
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
+    const float v = (int)(i % ld) < k ? x[i] : 0.f;
     bf16 h = __float2bfloat16_rn(v);
     hi[i] = h;
     lo[i] = __float2bfloat16_rn(v - __bfloat162float(h));
@@ -797,4 +811,133 @@ __global__ void __launch_bounds__(256) fma_probe_kernel(float* sink, int iters, 
   }
 }
 
+}  // namespace jolt
+
+namespace jolt {
+// Symmetric Gram from the tensor-core partial products: G[u][i * gld + j] (fp64, i, j < k) =
+// sum over the nsplit partial slots s of part[u][s] at the upper entry (min(i,j), max(i,j)),
+// added in fp64 (only the tiles on and above the diagonal were computed).
+__global__ void reduce_upper_sym_kernel(const float* part, double* G, int nbatch, int nsplit, int k, long long gld) {
+  const long long per = (long long)k * k, n = (long long)nbatch * per;
+  for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < n;
+       idx += (long long)gridDim.x * blockDim.x) {
+    const int u = (int)(idx / per);
+    const long long r = idx - u * per;
+    const int i = (int)(r / k), j = (int)(r - (long long)i * k);
+    const int a = i < j ? i : j, b = i < j ? j : i;
+    const float* p = part + (long long)u * nsplit * k * gld + (long long)a * gld + b;
+    double s = 0.0;
+    for (int q = 0; q < nsplit; ++q) s += (double)p[(long long)q * k * gld];
+    G[(long long)u * k * gld + (long long)i * gld + j] = s;
+  }
+}
+}  // namespace jolt
+
+namespace jolt {
+// ---------------------------------------------------------------------------------------
+// Rotated reconstruction operator in fp64:  P'[b][i][:] = bf16_rn( (C_b[i][:rD] W_u[:, :rD]^T)
+// diag(sigma_u) H_D / sqrt(D) ), every step in fp64 (products of bf16 operands, fp64 sums,
+// the Walsh-Hadamard butterflies in the order of strides 1, 2, ..., D/2, the division by
+// sqrt(D)) and one round-to-nearest-even to 8 significant bits at the end.  Only the sums'
+// order differs from a plain fp64 evaluation, so the bf16 result equals the exactly rounded
+// operator except at ties closer than about 1e-16 relative.
+// grid (ceil(rT / 32), batch entries); 256 threads; entry b uses W of unit u = umap[b / S].
+// ---------------------------------------------------------------------------------------
+__device__ __forceinline__ bf16 bf16_rn_from_f64(double x) {
+  // round to 8 significant bits (quantum at least 2^-133, the bf16 subnormal step) with ties
+  // to even, then the now exact conversion
+  if (x == 0.0 || !isfinite(x)) return __float2bfloat16_rn((float)x);
+  int e;
+  (void)frexp(x, &e);                 // x = m 2^e, 0.5 <= |m| < 1
+  const int qe = e - 8 > -133 ? e - 8 : -133;
+  const double y = rint(ldexp(x, -qe));
+  return __float2bfloat16_rn((float)ldexp(y, qe));
+}
+
+constexpr int PX_ROWS = 32;
+template <int D>
+__global__ void __launch_bounds__(256) pmat_exact_kernel(const bf16* C, long long ldC, long long sC, int rT, int rD,
+                                                         const bf16* W, long long ldW, long long sW, int S,
+                                                         const int* umap, uint64_t seed, bf16* out, long long sOut) {
+  constexpr int CPT = D >= 32 ? D / 32 : 1;   // columns per thread (and per lane in the rotation)
+  constexpr int LANES = D / CPT;              // lanes that hold columns (32, or D when D < 32)
+  constexpr int CS_BYTES = PX_ROWS * (128 + 8) * 2, WT_BYTES = 128 * (D + 8) * 2, PS_BYTES = PX_ROWS * (D + 1) * 8;
+  constexpr int BYTES = CS_BYTES + WT_BYTES > PS_BYTES ? CS_BYTES + WT_BYTES : PS_BYTES;
+  __shared__ __align__(16) unsigned char px_sm[BYTES];
+  auto cs = reinterpret_cast<bf16(*)[128 + 8]>(px_sm);                 // C rows of the tile
+  auto wt = reinterpret_cast<bf16(*)[D + 8]>(px_sm + CS_BYTES);        // W^T: wt[q][d]
+  auto ps = reinterpret_cast<double(*)[D + 1]>(px_sm);                 // the products (after the GEMM)
+  const int b = blockIdx.y, i0 = blockIdx.x * PX_ROWS, tid = threadIdx.x;
+  const int u = umap[b / S];
+  const bf16* Cb = C + (long long)b * sC;
+  const bf16* Wu = W + (long long)(b / S) * sW;
+  for (int idx = tid; idx < PX_ROWS * rD; idx += 256) {
+    const int r = idx / rD, q = idx - r * rD;
+    cs[r][q] = (i0 + r < rT) ? Cb[(long long)(i0 + r) * ldC + q] : __float2bfloat16_rn(0.f);
+  }
+  for (int idx = tid; idx < D * rD; idx += 256) {
+    const int d = idx / rD, q = idx - d * rD;
+    wt[q][d] = Wu[(long long)d * ldW + q];
+  }
+  __syncthreads();
+  const int rg = tid >> 5, cg = tid & 31;   // rows 4 rg .. 4 rg + 3, columns CPT cg .. + CPT - 1
+  double acc[4][CPT];
+#pragma unroll
+  for (int r = 0; r < 4; ++r)
+#pragma unroll
+    for (int e = 0; e < CPT; ++e) acc[r][e] = 0.0;
+  for (int q = 0; q < rD && cg < LANES; ++q) {
+    double cv[4], wv[CPT];
+#pragma unroll
+    for (int r = 0; r < 4; ++r) cv[r] = (double)__bfloat162float(cs[4 * rg + r][q]);
+#pragma unroll
+    for (int e = 0; e < CPT; ++e) wv[e] = (double)__bfloat162float(wt[q][CPT * cg + e]);
+#pragma unroll
+    for (int r = 0; r < 4; ++r)
+#pragma unroll
+      for (int e = 0; e < CPT; ++e) acc[r][e] = fma(cv[r], wv[e], acc[r][e]);
+  }
+  __syncthreads();   // ps overlays cs and wt
+  if (cg < LANES)
+#pragma unroll
+    for (int r = 0; r < 4; ++r)
+#pragma unroll
+      for (int e = 0; e < CPT; ++e) ps[4 * rg + r][CPT * cg + e] = acc[r][e];
+  __syncthreads();
+  // rotation: warp w takes rows 4w .. 4w + 3, lane l holds columns CPT l .. CPT l + CPT - 1
+  const int lane = tid & 31, warp = tid >> 5;
+  double sg[CPT];
+#pragma unroll
+  for (int e = 0; e < CPT; ++e) sg[e] = lane < LANES ? (double)rotation_sign(seed, u, CPT * lane + e) : 0.0;
+  const double rs = sqrt((double)D);
+  for (int rr = 0; rr < 4; ++rr) {
+    const int r = 4 * warp + rr;
+    double v[CPT];
+#pragma unroll
+    for (int e = 0; e < CPT; ++e) v[e] = lane < LANES ? ps[r][CPT * lane + e] * sg[e] : 0.0;
+#pragma unroll
+    for (int h = 1; h < CPT; h <<= 1)
+#pragma unroll
+      for (int e = 0; e < CPT; ++e)
+        if (!(e & h)) {
+          const double a = v[e], c = v[e + h];
+          v[e] = a + c;
+          v[e + h] = a - c;
+        }
+#pragma unroll
+    for (int hl = 1; hl < LANES; hl <<= 1) {
+      const bool upper = (lane & hl) != 0;
+#pragma unroll
+      for (int e = 0; e < CPT; ++e) {
+        const double mine = v[e], other = __shfl_xor_sync(0xffffffffu, mine, hl);
+        v[e] = upper ? other - mine : mine + other;
+      }
+    }
+    if (i0 + r < rT && lane < LANES) {
+      bf16* o = out + (long long)b * sOut + (long long)(i0 + r) * D + CPT * lane;
+#pragma unroll
+      for (int e = 0; e < CPT; ++e) o[e] = bf16_rn_from_f64(v[e] / rs);
+    }
+  }
+}
 }  // namespace jolt

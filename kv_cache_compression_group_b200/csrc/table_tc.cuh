@@ -1,0 +1,305 @@
+// Distortion table on the 5th-generation tensor cores (D = 128, up to 4 token-rank cuts).
+//
+// One CTA owns 128 consecutive tokens of one slice s of unit u (TMEM lane = token row) and
+// walks every feature-rank candidate r_D.  For a candidate, the reconstruction of the tile in
+// the rotated basis, U_s[:, :r_T] P'(r_D)[:r_T, :], is needed at every token-rank cut r_T.
+// The token-rank axis is cut into segments [c_{i-1}, c_i) and the tensor cores accumulate
+// each segment in its own TMEM accumulator (4 x 128 fp32 columns, all of tensor memory):
+//   * one thread issues the TMA copies of the U tile (128 x 64 bf16, K-major) and of P'
+//     (64 x 128 bf16, rows of the operator) for every 64-wide K block;
+//   * one thread issues tcgen05.mma (M = 128, N = 128, K = 16) into the accumulator of the
+//     segment the K step belongs to and commits an mbarrier when a segment is complete;
+//   * eight epilogue warps (two per TMEM lane quarter, each half of the 128 columns) read a
+//     finished segment with tcgen05.ld, release it at once (the next candidate's MMAs into
+//     that segment may start), add it to a running sum kept in registers, and evaluate the
+//     quantiser of every bit-width on rho = x' - running sum, block by block -- the
+//     arithmetic of table_kernel (kernels.cuh), which is why the two give the same entries.
+// x' (the tile rotated along the features) is formed once per CTA in shared memory.
+//
+// Every mbarrier wait is bounded (umma::mbar_wait); a wait that gives up raises
+// DEV_ERR_TIMEOUT and the CTA stops issuing work, keeps its named-barrier schedule, and waits
+// (bounded) for its issued MMAs before it frees tensor memory.
+#pragma once
+
+#include "kernels.cuh"
+#include "umma.cuh"
+
+namespace jolt {
+namespace ttc {
+constexpr int ROWS = 128;                                  // tokens per CTA
+constexpr int DIM = 128;                                   // features = MMA N
+constexpr int BK = 64;
+constexpr int STAGES = 4;
+constexpr int U_BYTES = ROWS * BK * 2;                     // 16 KB
+constexpr int P_BYTES = BK * DIM * 2;                      // 16 KB
+constexpr int STAGE_BYTES = U_BYTES + P_BYTES;
+constexpr int XS_LD = DIM + 4;                             // fp32 pitch of the rotated tile
+constexpr int XS_BYTES = ROWS * XS_LD * 4;
+constexpr int EPI_WARPS = 8;
+constexpr int THREADS = (EPI_WARPS + 2) * 32;              // + TMA warp + MMA warp
+constexpr int MAXT = 4;                                    // token-rank cuts
+constexpr int BAR_OFF = STAGES * STAGE_BYTES + XS_BYTES;
+constexpr int SMEM = 1024 + BAR_OFF + 512;                 // alignment slack + barriers
+constexpr int TMEM_COLS = 512;
+}  // namespace ttc
+
+struct TableTcArgs {
+  CacheView cv;
+  int rTmax;
+  Cands cand;
+  uint64_t seed;
+  double* partial;      // [unit][S][tiles][nD][nT][nB]
+  int tiles;            // ceil(T / 128)
+  uint32_t* status;
+};
+
+// the tile's rows rotated along the features into xs (fp32, pitch XS_LD): sign flip, the
+// Walsh-Hadamard butterflies in the order of fwht_regs (strides 1, 2, ..., 64), 1 / sqrt(D)
+template <typename TX>
+__device__ __forceinline__ void ttc_rotate_tile(const TX* X, int T, int t0, const float* sig, float* xs) {
+  using namespace ttc;
+  for (int idx = threadIdx.x; idx < ROWS * DIM; idx += THREADS) {
+    const int r = idx / DIM, d = idx - r * DIM, t = t0 + r;
+    xs[r * XS_LD + d] = t < T ? ld_as_float(X + (long long)t * DIM + d) * sig[d] : 0.f;
+  }
+  __syncthreads();
+  if (threadIdx.x < ROWS) {
+    float* row = xs + threadIdx.x * XS_LD;
+#pragma unroll 1
+    for (int half = 0; half < 2; ++half) {
+      float v[64];
+#pragma unroll
+      for (int q = 0; q < 16; ++q) {
+        const float4 f = *reinterpret_cast<const float4*>(row + half * 64 + 4 * q);
+        v[4 * q] = f.x;
+        v[4 * q + 1] = f.y;
+        v[4 * q + 2] = f.z;
+        v[4 * q + 3] = f.w;
+      }
+      fwht_regs<64>(v);
+#pragma unroll
+      for (int q = 0; q < 16; ++q)
+        *reinterpret_cast<float4*>(row + half * 64 + 4 * q) = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+    }
+    const float sc = (float)(1.0 / sqrt((double)DIM));
+#pragma unroll 4
+    for (int j = 0; j < 64; ++j) {
+      const float a = row[j], b = row[j + 64];
+      row[j] = (a + b) * sc;
+      row[j + 64] = (a - b) * sc;
+    }
+  }
+  __syncthreads();
+}
+
+__device__ __forceinline__ void ttc_tmem_ld16(uint32_t taddr, float* v) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ void ttc_epi_sync() { asm volatile("bar.sync 1, %0;" ::"n"(ttc::EPI_WARPS * 32) : "memory"); }
+
+// grid (tiles, S, units); ttc::THREADS threads; ttc::SMEM bytes of dynamic shared memory
+template <typename TX, typename BITS>
+__global__ void __launch_bounds__(ttc::THREADS, 1)
+    table_tc_kernel(const __grid_constant__ CUtensorMap map_u, const __grid_constant__ CUtensorMap map_p,
+                    TableTcArgs a) {
+  using namespace ttc;
+  extern __shared__ uint8_t ttc_raw[];
+  uint8_t* smem = (uint8_t*)(((uintptr_t)ttc_raw + 1023) & ~(uintptr_t)1023);
+  float* xs = reinterpret_cast<float*>(smem + STAGES * STAGE_BYTES);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + BAR_OFF);
+  // full[STAGES] empty[STAGES] accfull[MAXT] accfree[MAXT] done
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 2 * MAXT + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  __shared__ float sig[DIM];
+  __shared__ float red[EPI_WARPS][MAXT * MAXC];
+
+  const int tile = blockIdx.x, s = blockIdx.y, u = blockIdx.z;
+  const int T = a.cv.T, S = a.cv.S, NU = 2 * (a.cv.n_layers / a.cv.Lg);
+  const int t0 = tile * ROWS;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const Cands& cd = a.cand;
+  const int nT = cd.nT, nD = cd.nD, nB = cd.nB;
+  const int klast = cd.rT[nT - 1];
+  const int nkb = (klast + BK - 1) / BK;
+  const uint32_t full0 = umma::smem_u32(bars), empty0 = full0 + 8 * STAGES, accfull0 = empty0 + 8 * STAGES;
+  const uint32_t accfree0 = accfull0 + 8 * MAXT, done_bar = accfree0 + 8 * MAXT;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < STAGES; ++i) {
+      umma::mbar_init(full0 + 8 * i, 1);
+      umma::mbar_init(empty0 + 8 * i, 1);
+    }
+    for (int i = 0; i < MAXT; ++i) {
+      umma::mbar_init(accfull0 + 8 * i, 1);
+      umma::mbar_init(accfree0 + 8 * i, EPI_WARPS);
+    }
+    umma::mbar_init(done_bar, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (warp == EPI_WARPS) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(umma::smem_u32(tmem_slot)),
+                 "n"(TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  for (int d = threadIdx.x; d < DIM; d += THREADS) sig[d] = rotation_sign(a.seed, u, d);
+  __syncthreads();
+  const TX* X = reinterpret_cast<const TX*>(a.cv.unit_ptr(u)) + (long long)s * T * DIM;
+  ttc_rotate_tile<TX>(X, T, t0, sig, xs);
+  umma::fence_before_sync();
+  __syncthreads();
+  umma::fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == EPI_WARPS) {
+    if (lane == 0) {
+      // ---- TMA producer: for every candidate r_D, the K blocks of U and P' ----
+      int it = 0;
+      for (int iD = 0; iD < nD && !*abort_flag; ++iD) {
+        const int ep = (iD * NU + u) * S + s;
+        for (int j = 0; j < nkb; ++j, ++it) {
+          const int st = it % STAGES;
+          if (it >= STAGES && !umma::mbar_wait(empty0 + 8 * st, ((it / STAGES) & 1) ^ 1)) {
+            *abort_flag = 1;
+            break;
+          }
+          const uint32_t fb = full0 + 8 * st;
+          const uint32_t sa = umma::smem_u32(smem + st * STAGE_BYTES);
+          umma::mbar_expect_tx(fb, STAGE_BYTES);
+          umma::tma_load_3d(sa, &map_u, j * BK, t0, u, fb);
+          umma::tma_load_3d(sa + umma::BOX_BYTES, &map_u, j * BK, t0 + 64, u, fb);
+          umma::tma_load_3d(sa + U_BYTES, &map_p, 0, j * BK, ep, fb);
+          umma::tma_load_3d(sa + U_BYTES + umma::BOX_BYTES, &map_p, 64, j * BK, ep, fb);
+        }
+      }
+    }
+  } else if (warp == EPI_WARPS + 1) {
+    if (lane == 0) {
+      // ---- MMA issuer: K step k16 goes to the accumulator of the segment holding it ----
+      constexpr uint32_t idesc = umma::instr_desc(DIM, false, true);
+      int it = 0;
+      for (int iD = 0; iD < nD && !*abort_flag; ++iD) {
+        int seg = 0;
+        for (int j = 0; j < nkb && !*abort_flag; ++j, ++it) {
+          const int st = it % STAGES;
+          if (!umma::mbar_wait(full0 + 8 * st, (it / STAGES) & 1)) {
+            *abort_flag = 1;
+            break;
+          }
+          umma::fence_after_sync();
+          const uint32_t sa = umma::smem_u32(smem + st * STAGE_BYTES);
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            const int k0 = j * BK + kk * 16;
+            if (k0 >= klast) break;
+            while (k0 >= cd.rT[seg]) ++seg;
+            const int lo = seg ? cd.rT[seg - 1] : 0;
+            if (k0 == lo && iD > 0) {
+              // the previous candidate's epilogue must have read this segment
+              if (!umma::mbar_wait(accfree0 + 8 * seg, (iD - 1) & 1)) {
+                *abort_flag = 1;
+                break;
+              }
+              umma::fence_after_sync();
+            }
+            const uint64_t ad = umma::smem_desc(sa + kk * 32, 16, 1024);
+            const uint64_t bd = umma::smem_desc(sa + U_BYTES + kk * 2048, umma::BOX_BYTES, 1024);
+            umma::mma_bf16(tmem + (uint32_t)(seg * DIM), ad, bd, idesc, k0 != lo ? 1u : 0u);
+            if (k0 + 16 == cd.rT[seg]) umma::mma_commit(accfull0 + 8 * seg);
+          }
+          umma::mma_commit(empty0 + 8 * st);
+        }
+      }
+      umma::mma_commit(done_bar);   // fires when every MMA issued above has completed
+    }
+  } else {
+    // ---- epilogue: warp w owns TMEM lanes 32 (w % 4) .. +31 and columns 64 (w / 4) .. +63 ----
+    const int row = 32 * (warp & 3) + lane;
+    const int cbase = 64 * (warp >> 2);
+    const uint32_t lane_addr = (uint32_t)(32 * (warp & 3)) << 16;
+    const BitConsts kb = bit_consts(cd);
+    double* out = a.partial + (((long long)u * S + s) * a.tiles + tile) * (long long)(nD * nT * nB);
+    const float* xrow = xs + row * XS_LD + cbase;
+    for (int iD = 0; iD < nD; ++iD) {
+      float run[64];
+#pragma unroll
+      for (int j = 0; j < 64; ++j) run[j] = 0.f;
+#pragma unroll 1
+      for (int i = 0; i < nT; ++i) {
+        bool ok = !*abort_flag && umma::mbar_wait(accfull0 + 8 * i, iD & 1);
+        ok = __all_sync(0xffffffffu, ok);   // the TMEM loads below are warp-collective
+        if (!ok) *abort_flag = 1;
+        float err[MAXC];
+#pragma unroll
+        for (int b = 0; b < MAXC; ++b) err[b] = 0.f;
+        if (ok) {
+          umma::fence_after_sync();
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            float seg[32];
+            ttc_tmem_ld16(tmem + lane_addr + (uint32_t)(i * DIM + cbase + 32 * hh), seg);
+            ttc_tmem_ld16(tmem + lane_addr + (uint32_t)(i * DIM + cbase + 32 * hh + 16), seg + 16);
+            asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+            for (int j = 0; j < 32; ++j) run[32 * hh + j] += seg[j];
+          }
+          // the segment is in registers: release it to the next candidate's MMAs
+          umma::fence_before_sync();
+          __syncwarp();
+          if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(accfree0 + 8 * i) : "memory");
+          if (t0 + row < T) {
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+              float v[16];
+              load16(xrow + 16 * m, v);
+#pragma unroll
+              for (int j = 0; j < 16; ++j) v[j] -= run[16 * m + j];
+              if constexpr (std::is_same<BITS, void>::value) block_errors(v, kb, err);
+              else block_errors_fixed(v, err, BITS{});
+            }
+          }
+        }
+        // this cut's sums over the warp (every lane takes part, also after an abort)
+#pragma unroll
+        for (int b = 0; b < MAXC; ++b) {
+          if (b >= nB) break;
+          float v = err[b];
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+          if (lane == 0) red[warp][i * MAXC + b] = v;
+        }
+      }
+      // over the eight epilogue warps in fixed order (fp64)
+      ttc_epi_sync();
+      if (threadIdx.x < nT * nB) {
+        const int i = threadIdx.x / nB, b = threadIdx.x - i * nB;
+        double v = 0.0;
+        for (int w = 0; w < EPI_WARPS; ++w) v += (double)red[w][i * MAXC + b];
+        out[(iD * nT + i) * nB + b] = v;
+      }
+      ttc_epi_sync();
+    }
+  }
+  // every issued MMA has completed before tensor memory is freed
+  __syncwarp();
+  const bool drained = umma::mbar_wait(done_bar, 0);
+  if ((*abort_flag || !drained) && threadIdx.x == 0 && a.status) atomicOr(a.status, DEV_ERR_TIMEOUT);
+  umma::fence_before_sync();
+  __syncthreads();
+  if (warp == EPI_WARPS) {
+    umma::fence_after_sync();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "n"(TMEM_COLS) : "memory");
+  }
+}
+
+}  // namespace jolt

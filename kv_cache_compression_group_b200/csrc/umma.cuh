@@ -55,6 +55,12 @@ struct UmmaArgs {
   bool b_is_a = false;        // Gram of one operand: B's tile is A's tile (M = N = 128, one tile)
   void* C = nullptr;
   int c_bf16 = 0;             // 0: fp32 output, 1: bf16 (round to nearest)
+  int c_accum = 0;            // fp32 output only: add the product to what C holds
+  int tri = 0;                // 1: only output tiles that reach the diagonal or above it
+                              //    (n0 + BN > m0; the upper triangle of a symmetric product);
+                              // 2: B upper triangular (row k of B is zero for k > every column
+                              //    of the tile): the K range ends at n0 + BN
+  int bn = 0;                 // N tile: 0 chooses (256 when N > 128), else 128 or 256
   long long ldc = 0, sC = 0, ssplit = 0;   // row pitch, batch stride, split stride (elements)
   uint32_t* status = nullptr;
 };
@@ -257,9 +263,10 @@ __global__ void __launch_bounds__(128, 1)
   uint32_t* tmem_slot = (uint32_t*)(bars + 2 * C::STAGES + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n0 = blockIdx.x * BN, m0 = blockIdx.y * umma::BM;
+  if (a.tri == 1 && n0 + BN <= m0) return;   // wholly below the diagonal: not needed
   const int bz = blockIdx.z / a.splits, sp = blockIdx.z - bz * a.splits;
   const int kb0 = sp * (a.kchunk / umma::BK);
-  const int kend = min(a.K, (sp + 1) * a.kchunk);
+  const int kend = min(a.tri == 2 ? min(a.K, n0 + BN) : a.K, (sp + 1) * a.kchunk);
   const int nk = kend > kb0 * umma::BK ? (kend - kb0 * umma::BK + umma::BK - 1) / umma::BK : 0;
   const uint32_t full0 = umma::smem_u32(bars), empty0 = full0 + 8 * C::STAGES, accb = full0 + 16 * C::STAGES;
   const bool b_is_a = a.b_is_a;
@@ -392,11 +399,21 @@ __global__ void __launch_bounds__(128, 1)
       float* crow = (float*)a.C + off;
       if (vec && n + 32 <= a.N) {
 #pragma unroll
-        for (int j = 0; j < 32; j += 4) *(float4*)(crow + n + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+        for (int j = 0; j < 32; j += 4) {
+          float4 o = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+          if (a.c_accum) {
+            const float4 c = *(const float4*)(crow + n + j);
+            o.x += c.x;
+            o.y += c.y;
+            o.z += c.z;
+            o.w += c.w;
+          }
+          *(float4*)(crow + n + j) = o;
+        }
       } else {
 #pragma unroll
         for (int j = 0; j < 32; ++j)
-          if (n + j < a.N) crow[n + j] = v[j];
+          if (n + j < a.N) crow[n + j] = a.c_accum ? crow[n + j] + v[j] : v[j];
       }
     }
   }
@@ -487,7 +504,9 @@ inline cudaError_t launch_umma(const UmmaMaps& m, UmmaArgs a, int nb, cudaStream
       (nb == 2 && umma::cache_mode(a.B.mode)) || (a.b_is_a && (a.M > 128 || a.N > 128 || nb != 1)))
     return cudaErrorInvalidValue;
   if (a.splits == 1) a.kchunk = (int)round_up(a.K, umma::BK);
-  if (a.N > 128) return nb == 2 ? launch_umma_bn<256, 2>(m, a, st) : launch_umma_bn<256, 1>(m, a, st);
+  if (a.c_accum && a.c_bf16) return cudaErrorInvalidValue;
+  if (a.bn == 256 || (a.bn == 0 && a.N > 128))
+    return nb == 2 ? launch_umma_bn<256, 2>(m, a, st) : launch_umma_bn<256, 1>(m, a, st);
   return nb == 2 ? launch_umma_bn<128, 2>(m, a, st) : launch_umma_bn<128, 1>(m, a, st);
 }
 

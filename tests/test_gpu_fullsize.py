@@ -78,7 +78,7 @@ def _sampled_rows_check(blob_np, rec, w, u, K, V, comp, opts):
     Pl = _library_operator(comp, opts, w, u, gb)
     Po = O.recon_operator(r.C_s, r.W_s, r.sigma, r.r_D).reshape(Pl.shape)
     diff = Pl != Po
-    assert diff.mean() <= 1e-3, diff.mean()
+    assert diff.mean() <= 1e-6, diff.mean()   # fp64 operator, one rounding: equal but for fp64 ties
     step = np.abs(Po) * 2.0 ** -7 * 1.0001 + 2.0 ** -16 * np.abs(Po).max(-1, keepdims=True)
     assert np.all(np.abs(Pl - Po)[diff] <= step[diff])
     Xrows = _unit_x(K, V, w, u, (t0, t0 + ROWS))

@@ -157,12 +157,16 @@ def test_core_table_and_operator(name):
         Z = O.bf16_rn(np.einsum("lhtd,dq->lhtq", X, f.W_s)).reshape(-1, X.shape[2], f.W_s.shape[1])
         slack = 4 * 2.0 ** -8 * np.abs(f.U_s).max(0)[None, :, None] * np.abs(Z).max(1)[:, None, :]
         frac, ok = _ulp_close(core[u], want, slack)
-        assert frac <= 1e-2 and ok, (u, frac)
+        # every difference is a rounding flip within the bound; how many entries flip depends
+        # on how many sit near cancellation (about 2 % with 4 slices per unit)
+        assert frac <= 5e-2 and ok, (u, frac)
         Cg = core[u].reshape(Lg, H, *core[u].shape[1:])
         for iD, rD in enumerate(d["oo"].feature_ranks):
+            # the library forms P' in fp64 and rounds once: equal to the oracle's operator
+            # except at a tie closer than fp64 resolution
             Pw = O.recon_operator(Cg, f.W_s, f.sigma, rD).reshape(P[iD, u].shape)
-            frac, ok = _ulp_close(P[iD, u], Pw, 2.0 ** -16 * np.abs(Pw).max(-1, keepdims=True))
-            assert frac <= 1e-3 and ok, (u, rD, frac)
+            frac, ok = _ulp_close(P[iD, u], Pw, 0.0)
+            assert frac <= 1e-6 and ok, (u, rD, frac)
         # the table kernel against the oracle's table built from the same stored core.
         # The library forms rho in fp32: |d rho| <= c u_32 |x| per element, so an entry
         # sum_i e_i^2 moves by at most 2 sqrt(entry) ||d rho|| (+ ties, which move e^2 by
