@@ -93,6 +93,11 @@ typedef struct {
   int32_t method;                             /* jolt_method */
   int32_t oversample;                         /* FlashJoLT sketch width = max r_T + oversample */
   int32_t power_iters;                        /* FlashJoLT power iterations */
+  int32_t unit_offset;                        /* global index of this cache's first unit, 0 for a whole
+                                                 cache; a shard holding layer groups g0.. of a larger
+                                                 cache passes 2 * g0, so the rotation signs and the
+                                                 sketch of its units are those of the whole cache
+                                                 (recorded in the blob header for the decoder) */
 } jolt_options;
 
 /* Per-unit record of a compressed blob, as returned by jolt_read_header. */

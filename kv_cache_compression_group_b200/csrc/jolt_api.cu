@@ -167,6 +167,7 @@ struct Plan {
   int nL, H, T, D, Lg, S, G, NU, M, dtype;
   Cands cd;
   int nC, rTmax, rDmax, ldU, ldW, ldC, method, q, k, kp;
+  int u0;                 // global index of this cache's first unit (RNG streams)
   bool m_side;            // exact token factor through the M x M Gram (T > M)
   int gd_split;           // split-K of the feature Gram
   int gt_split;           // split-K of the token Gram
@@ -249,6 +250,8 @@ jolt_status make_plan(const jolt_shape* sh, const jolt_options* op, Plan* p) {
   p->ldW = p->rDmax;
   p->ldC = p->rDmax;
   p->method = op->method;
+  if (op->unit_offset < 0 || op->unit_offset > (1 << 24)) return fail(JOLT_ERR_INVALID_ARG, "unit_offset %d", op->unit_offset);
+  p->u0 = op->unit_offset;
   p->q = op->power_iters;
   p->k = 0;
   p->kp = 0;
@@ -486,6 +489,7 @@ struct Ctx {
     c.D = p.D;
     c.Lg = p.Lg;
     c.S = p.S;
+    c.u0 = p.u0;
     c.unit_elems = (long long)p.S * p.T * p.D;
     return c;
   }
@@ -1070,7 +1074,7 @@ jolt_status run_token_randomized(const Ctx& c, float* Uf, long long ldUf) {
   CUDA_TRY(cudaMemsetAsync(Y, 0, (size_t)NU * T * kp * 4, c.st));
   CUDA_TRY(cudaMemsetAsync(Z, 0, (size_t)NU * M * kp * 4, c.st));
   count_launch(), omega_kernel<<<grid1d((long long)NU * M * kp), 256, 0, c.st>>>(Om, M, k, kp, (long long)M * kp,
-                                                                                  c.seed, 0, NU);
+                                                                                  c.seed, p.u0, NU);
   CUDA_TRY(cudaGetLastError());
   // products with X_(T) (Y side, T x k) and X_(T)^T (Z side, M x k)
   GemmParams gy;
@@ -1391,7 +1395,7 @@ jolt_status pmat_all(const Ctx& c, const bf16* core, long long ldC, int rT, int 
 }
 
 jolt_status fill_umap(const Ctx& c, int* umap, int n) {
-  count_launch(), iota_kernel<<<(unsigned)ceil_div(n, 128), 128, 0, c.st>>>(umap, n);
+  count_launch(), iota_kernel<<<(unsigned)ceil_div(n, 128), 128, 0, c.st>>>(umap, n, c.p.u0);
   CUDA_TRY(cudaGetLastError());
   return JOLT_OK;
 }
@@ -1534,6 +1538,7 @@ BlobHeader header_proto(const Plan& p, uint64_t seed) {
   h.layers_per_group = p.Lg;
   h.dtype = p.dtype;
   h.block = 16;
+  h.unit_offset = p.u0;
   h.seed = seed;
   return h;
 }
@@ -2115,6 +2120,7 @@ jolt_status jolt_decompress(const void* blob_dev, int32_t out_dtype, void* k_out
   op.feature_ranks[0] = (int)round_up(rDm, 8) > sh.head_dim ? rDm : (int)round_up(rDm, 8);
   op.n_bits = 1;
   op.method = JOLT_EXACT;
+  op.unit_offset = h.unit_offset;
   Plan p;
   JTRY(make_plan(&sh, &op, &p));
   if (ws_bytes < p.dws_total)
@@ -2153,6 +2159,7 @@ jolt_status jolt_decompress(const void* blob_dev, int32_t out_dtype, void* k_out
   a.T = p.T;
   a.S = p.S;
   a.Lg = p.Lg;
+  a.u0 = p.u0;
   a.seed = h.seed;
   a.k_out = k_out_dev;
   a.v_out = v_out_dev;

@@ -22,6 +22,7 @@ struct CacheView {
   const void* v;
   int dtype;              // 0 bf16, 1 fp32
   int n_layers, H, T, D, Lg, S;
+  int u0;                 // global index of unit 0 (a shard of a larger cache): RNG streams use u + u0
   long long unit_elems;   // S * T * D
   __host__ __device__ const void* unit_ptr(int u) const {
     const char* base = (const char*)((u & 1) ? v : k);
@@ -472,7 +473,7 @@ __global__ void __launch_bounds__(table_threads<D>(), D >= 64 ? 2 : 1) table_ker
   const int T = a.cv.T;
   const int t0 = tile * TROWS;
   const TX* X = reinterpret_cast<const TX*>(a.cv.unit_ptr(u)) + (long long)s * T * D;
-  for (int d = threadIdx.x; d < D; d += blockDim.x) sig[d] = rotation_sign(a.seed, u, d);
+  for (int d = threadIdx.x; d < D; d += blockDim.x) sig[d] = rotation_sign(a.seed, u + a.cv.u0, d);
   __syncthreads();
   rotate_tile_smem<D, TX>(X, T, t0, sig, rho);   // x' staged through the rho buffer
   __syncthreads();
@@ -538,7 +539,7 @@ __global__ void __launch_bounds__(table_threads<D>(), D >= 64 ? 2 : 1) table_ker
 // ---------------------------------------------------------------------------------------
 struct BlobHeader {      // 64 bytes at offset 0
   uint32_t magic, version, n_units, status;
-  int32_t n_layers, n_heads, n_tokens, head_dim, layers_per_group, dtype, block, reserved;
+  int32_t n_layers, n_heads, n_tokens, head_dim, layers_per_group, dtype, block, unit_offset;
   uint64_t seed, total_bytes;
 };
 struct UnitHeader {      // 64 bytes per unit after the global header
@@ -586,7 +587,7 @@ __global__ void __launch_bounds__(TTHREADS) encode_kernel(EncodeArgs a) {
   while (iD < a.cand.nD && a.cand.rD[iD] != uh.r_D) ++iD;
 
   const TX* X = reinterpret_cast<const TX*>(a.cv.unit_ptr(u)) + (long long)s * T * D;
-  for (int d = threadIdx.x; d < D; d += blockDim.x) sig[d] = rotation_sign(a.seed, u, d);
+  for (int d = threadIdx.x; d < D; d += blockDim.x) sig[d] = rotation_sign(a.seed, u + a.cv.u0, d);
   __syncthreads();
   rotate_tile_to_smem<D, TX>(X, T, t0, sig, rho);
   __syncthreads();
@@ -659,6 +660,7 @@ struct DecodeArgs {
   long long sP_unit;
   int rTmax;
   int T, S, Lg;
+  int u0;                // global index of unit 0 (from the blob header)
   uint64_t seed;
   void* k_out;
   void* v_out;
@@ -713,7 +715,7 @@ __global__ void __launch_bounds__(TTHREADS) decode_kernel(DecodeArgs a) {
   const int T = a.T;
   const int t0 = tile * TROWS;
   const UnitHeader uh = reinterpret_cast<const UnitHeader*>(a.blob + sizeof(BlobHeader))[u];
-  for (int d = threadIdx.x; d < D; d += blockDim.x) sig[d] = rotation_sign(a.seed, u, d);
+  for (int d = threadIdx.x; d < D; d += blockDim.x) sig[d] = rotation_sign(a.seed, u + a.u0, d);
   __syncthreads();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   constexpr int NT = D / 8;

@@ -701,9 +701,9 @@ __global__ void copy_factors_kernel(unsigned char* blob, const bf16* U, long lon
   }
 }
 
-__global__ void iota_kernel(int* out, int n) {
+__global__ void iota_kernel(int* out, int n, int first) {
   int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i < n) out[i] = i;
+  if (i < n) out[i] = first + i;
 }
 
 // device-side errors of the factor stage go into the blob header status word

@@ -153,7 +153,7 @@ __global__ void __launch_bounds__(ttc::THREADS, 1)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
-  for (int d = threadIdx.x; d < DIM; d += THREADS) sig[d] = rotation_sign(a.seed, u, d);
+  for (int d = threadIdx.x; d < DIM; d += THREADS) sig[d] = rotation_sign(a.seed, u + a.cv.u0, d);
   __syncthreads();
   const TX* X = reinterpret_cast<const TX*>(a.cv.unit_ptr(u)) + (long long)s * T * DIM;
   ttc_rotate_tile<TX>(X, T, t0, sig, xs);

@@ -49,7 +49,8 @@ class COptions(ctypes.Structure):
     _fields_ = [("n_token_ranks", ctypes.c_int32), ("token_ranks", ctypes.c_int32 * MAXC),
                 ("n_feature_ranks", ctypes.c_int32), ("feature_ranks", ctypes.c_int32 * MAXC),
                 ("n_bits", ctypes.c_int32), ("bits", ctypes.c_int32 * MAXC),
-                ("method", ctypes.c_int32), ("oversample", ctypes.c_int32), ("power_iters", ctypes.c_int32)]
+                ("method", ctypes.c_int32), ("oversample", ctypes.c_int32), ("power_iters", ctypes.c_int32),
+                ("unit_offset", ctypes.c_int32)]
 
 
 class CUnitRecord(ctypes.Structure):
@@ -132,6 +133,7 @@ class Options:
     method: str = "exact"
     oversample: int = 10
     power_iters: int = 2
+    unit_offset: int = 0    # global index of the first unit (a shard of a larger cache)
 
     def c(self) -> COptions:
         o = COptions()
@@ -146,6 +148,7 @@ class Options:
         o.method = {"exact": JOLT_EXACT, "randomized": JOLT_RANDOMIZED}[self.method]
         o.oversample = self.oversample
         o.power_iters = self.power_iters
+        o.unit_offset = self.unit_offset
         return o
 
     @property

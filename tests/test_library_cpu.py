@@ -112,7 +112,7 @@ def test_null_pointer_calls_fail_before_any_launch():
 
 def test_struct_layouts():
     assert ctypes.sizeof(J.CShape) == 24
-    assert ctypes.sizeof(J.COptions) == 4 * (3 + 3 * J.MAXC + 3)
+    assert ctypes.sizeof(J.COptions) == 4 * (3 + 3 * J.MAXC + 4)   # + method, oversample, power_iters, unit_offset
     assert ctypes.sizeof(J.CUnitRecord) == 64
 
 
