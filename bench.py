@@ -44,7 +44,7 @@ def parse():
     ap.add_argument("--workload", default="llama31_8b_64k")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extras", action="store_true", help="skip the exact-arm and decompress side figures")
-    ap.add_argument("--profile-case", default=None, choices=["mistral7b_4layers", "mistral7b", "llama31_8b_64k"],
+    ap.add_argument("--profile-case", default=None, choices=["mistral7b_4layers", "mistral7b", "llama31_8b_64k", "llama31_8b_4layers_T8192"],
                     help="run two compress + decompress calls of one case (for ncu captures) and exit")
     ap.add_argument("--sweep", action="store_true",
                     help="one JSON line per workload of the other shapes (LLaMA-2-13B, LLaMA-3.1-8B/64K) and "
@@ -54,12 +54,17 @@ def parse():
 
 def profile_case(args):
     """Two FlashJoLT (or JoLT) compress + decompress calls of one case, for ncu captures:
-    mistral7b_4layers (16 MiB of K and V) or the full Mistral-shaped cache (128 MiB, about
-    1 GiB of workspace with FlashJoLT), with the same kernels as the timed run."""
+    mistral7b_4layers (16 MiB of K and V), the full Mistral-shaped cache (128 MiB, about 1 GiB
+    of workspace with FlashJoLT), the LLaMA-3.1-8B/64K cache (8 GiB; for launch lists only) or
+    one layer group of it at 8192 tokens (128 MiB), with the same kernels as the timed run."""
     import torch
     from kv_cache_compression_group_b200 import synth, jolt as J
     if args.profile_case in ("mistral7b", "llama31_8b_64k"):
         w = synth.WORKLOADS[args.profile_case]
+    elif args.profile_case == "llama31_8b_4layers_T8192":
+        # the LLaMA-3.1-8B generator and candidate sets (token ranks up to 960) on one layer
+        # group of 8192 tokens: the long-context kernels at a size a full ncu capture can take
+        w = synth.small_workload("llama31_8b_64k", n_layers=4, T=8192)
     else:
         w = synth.small_workload("mistral7b", n_layers=4)
     K, V = synth.make_cache(w, 0)

@@ -218,6 +218,32 @@ jolt_status jolt_read_header(const void* blob_dev, jolt_shape* shape_out, uint64
 jolt_status jolt_decompress(const void* blob_dev, int32_t out_dtype, void* k_out_dev, void* v_out_dev, void* ws_dev,
                             size_t ws_bytes, void* stream);
 
+/* Decode-side attention over the stored factors (abstract of "A JoLT for the KV cache ...
+ * Joint Rank-bit Allocation": the decode path evaluates attention directly over the stored
+ * factors, without forming dense K and V).  One decode step of n_q_heads query heads against
+ * every token of one layer: query head j reads KV head j / (n_q_heads / n_heads), scores
+ * s_t = k_hat_t . q / sqrt(head_dim) with k_hat the decoder's reconstruction of the stored K,
+ * weights p = softmax(s), output p^T v_hat.  Computed as U_K (P'_K q') + rho_hat_K . q' and
+ * ((p^T U_V) P'_V + p^T rho_hat_V) Phi_V^T with q' = Phi_K^T q: the stored token factors,
+ * codes and scales are read, no dense K or V row is formed.  fp32 arithmetic.
+ *
+ * jolt_attend_prepare: the aligned token factors and the rotated operators P' of every unit
+ *   into ws_dev (the workspace of jolt_decompress, dws_bytes of jolt_workspace_size for the
+ *   blob's shape and candidate sets); reads the blob's headers (SYNCHRONISES once).  Call it
+ *   once per blob; any number of jolt_attend calls then read the prepared workspace.
+ * jolt_attend_scratch_size: bytes of the per-call scratch for n_q_heads query heads when the
+ *   stored token ranks are at most max_token_rank.
+ * jolt_attend: q_dev [n_q_heads][head_dim] fp32 (read only), out_dev [n_q_heads][head_dim]
+ *   fp32; layer in [0, n_layers); n_q_heads a multiple of n_heads with at most 8 query heads
+ *   per KV head; stored token ranks at most 1024.  Reads the blob's header (SYNCHRONISES once),
+ *   then runs asynchronously.  Errors: INVALID_ARG (layer, heads, null pointers),
+ *   WORKSPACE_TOO_SMALL (ws or scratch), BAD_BLOB. */
+jolt_status jolt_attend_prepare(const void* blob_dev, void* ws_dev, size_t ws_bytes, void* stream);
+jolt_status jolt_attend_scratch_size(const jolt_shape* shape, int32_t max_token_rank, int32_t n_q_heads,
+                                     size_t* bytes);
+jolt_status jolt_attend(const void* blob_dev, const void* ws_dev, size_t ws_bytes, int32_t layer, const float* q_dev,
+                        int32_t n_q_heads, float* out_dev, void* scratch_dev, size_t scratch_bytes, void* stream);
+
 /* Per-unit sums of squares (the introduction reports the relative Frobenius error of K and
  * of V separately): sq_dev[2*u] = ||X_u||^2, sq_dev[2*u+1] = ||X_u - Y_u||^2
  * (fp64), X and Y of the same shape; y may be NULL (then only ||X_u||^2).  ydtype is Y's

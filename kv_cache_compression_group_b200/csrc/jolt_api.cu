@@ -17,6 +17,7 @@
 #include "eig_cluster.cuh"
 #include "chol.cuh"
 #include "table_tc.cuh"
+#include "attend.cuh"
 
 using namespace jolt;
 
@@ -2089,65 +2090,97 @@ jolt_status jolt_read_header(const void* blob_dev, jolt_shape* shape_out, uint64
   return JOLT_OK;
 }
 
+}  // extern "C"
+
+namespace {
+// The decoder's preparation of a blob (shared by jolt_decompress and the decode-side
+// attention): read and validate the headers (synchronises once), plan a workspace for the
+// stored ranks, copy every unit's U, W and core to aligned buffers, and form its rotated
+// operator P' from the stored core and feature factor.
+struct Prepared {
+  BlobHeader h;
+  jolt_shape sh;
+  std::vector<jolt_unit_record> rec;
+  Plan p;
+};
+
+jolt_status decode_prepare(const void* blob_dev, void* ws_dev, size_t ws_bytes, cudaStream_t st, Prepared* out,
+                           bool compute) {
+  Prepared& pr = *out;
+  uint64_t total = 0;
+  CUDA_TRY(cudaMemcpyAsync(&pr.h, blob_dev, sizeof pr.h, cudaMemcpyDeviceToHost, st));
+  CUDA_TRY(cudaStreamSynchronize(st));
+  const BlobHeader& h = pr.h;
+  if (h.magic != kMagic || h.version != kVersion || h.n_units == 0 || h.n_units > 4096)
+    return fail(JOLT_ERR_BAD_BLOB, "bad blob header");
+  pr.rec.resize(h.n_units);
+  JTRY(jolt_read_header(blob_dev, &pr.sh, &total, pr.rec.data(), (int32_t)h.n_units, st));
+  // a plan for this shape with candidate sets made of the ranks actually stored
+  jolt_options op;
+  memset(&op, 0, sizeof op);
+  int rTm = 8, rDm = 8;
+  for (auto& r : pr.rec) {
+    if (r.r_T < 1 || r.r_T > pr.sh.n_tokens || r.r_D < 1 || r.r_D > pr.sh.head_dim || r.bits < 0 || r.bits > 8)
+      return fail(JOLT_ERR_BAD_BLOB, "unit record out of range");
+    if (r.off_U + 2ull * pr.sh.n_tokens * r.r_T > total) return fail(JOLT_ERR_BAD_BLOB, "unit record offsets");
+    rTm = r.r_T > rTm ? r.r_T : rTm;
+    rDm = r.r_D > rDm ? r.r_D : rDm;
+  }
+  op.n_token_ranks = 1;
+  op.token_ranks[0] = (int)round_up(rTm, 8) > pr.sh.n_tokens ? rTm : (int)round_up(rTm, 8);
+  op.n_feature_ranks = 1;
+  op.feature_ranks[0] = (int)round_up(rDm, 8) > pr.sh.head_dim ? rDm : (int)round_up(rDm, 8);
+  op.n_bits = 1;
+  op.method = JOLT_EXACT;
+  op.unit_offset = h.unit_offset;
+  JTRY(make_plan(&pr.sh, &op, &pr.p));
+  const Plan& p = pr.p;
+  if (ws_bytes < p.dws_total)
+    return fail(JOLT_ERR_WORKSPACE_TOO_SMALL, "decompress workspace %zu bytes, need %zu", ws_bytes, p.dws_total);
+  if (!compute) return JOLT_OK;
+  Ctx c{p, (unsigned char*)ws_dev, st, nullptr, nullptr, h.seed};
+  bf16* Ucp = c.at<bf16>(p.d_U);
+  bf16* Wcp = c.at<bf16>(p.d_W);
+  bf16* Ccp = c.at<bf16>(p.d_C);
+  bf16* P = c.at<bf16>(p.d_P);
+  int* umap = c.at<int>(p.d_umap);
+  JTRY(fill_umap(c, umap, p.NU));
+  const unsigned char* blob = (const unsigned char*)blob_dev;
+  const long long sP_unit = (long long)p.S * p.rTmax * p.D;
+  for (int u = 0; u < p.NU; ++u) {
+    const jolt_unit_record& r = pr.rec[u];
+    bf16* Uu = Ucp + (size_t)u * p.T * p.ldU;
+    bf16* Wu = Wcp + (size_t)u * p.D * p.ldW;
+    bf16* Cu = Ccp + (size_t)u * p.S * p.rTmax * p.ldC;
+    count_launch(), copy2d_kernel<<<grid1d((long long)p.T * p.ldU), 256, 0, st>>>((const bf16*)(blob + r.off_U), p.T,
+                                                                                r.r_T, Uu, p.ldU);
+    count_launch(), copy2d_kernel<<<grid1d((long long)p.D * p.ldW), 256, 0, st>>>((const bf16*)(blob + r.off_W), p.D,
+                                                                                r.r_D, Wu, p.ldW);
+    count_launch(), copy2d_kernel<<<grid1d((long long)p.S * r.r_T * p.ldC), 256, 0, st>>>(
+        (const bf16*)(blob + r.off_C), (long long)p.S * r.r_T, r.r_D, Cu, p.ldC);
+    CUDA_TRY(cudaGetLastError());
+    JTRY(pmat_unit(c, u, Cu, p.ldC, r.r_T, p.rTmax, Wu, p.ldW, r.r_D, nullptr, P + u * sP_unit, umap));
+  }
+  return JOLT_OK;
+}
+}  // namespace
+
+extern "C" {
+
 jolt_status jolt_decompress(const void* blob_dev, int32_t out_dtype, void* k_out_dev, void* v_out_dev, void* ws_dev,
                             size_t ws_bytes, void* stream) {
   if (out_dtype != JOLT_BF16 && out_dtype != JOLT_F32) return fail(JOLT_ERR_INVALID_ARG, "out_dtype %d", out_dtype);
   if (!k_out_dev || !v_out_dev || !ws_dev) return fail(JOLT_ERR_INVALID_ARG, "null pointer");
   cudaStream_t st = (cudaStream_t)stream;
-  jolt_shape sh;
-  uint64_t total = 0;
-  BlobHeader h;
-  CUDA_TRY(cudaMemcpyAsync(&h, blob_dev, sizeof h, cudaMemcpyDeviceToHost, st));
-  CUDA_TRY(cudaStreamSynchronize(st));
-  if (h.magic != kMagic || h.version != kVersion || h.n_units == 0 || h.n_units > 4096)
-    return fail(JOLT_ERR_BAD_BLOB, "bad blob header");
-  std::vector<jolt_unit_record> rec(h.n_units);
-  JTRY(jolt_read_header(blob_dev, &sh, &total, rec.data(), (int32_t)h.n_units, stream));
-  // a plan for this shape with candidate sets made of the ranks actually stored
-  jolt_options op;
-  memset(&op, 0, sizeof op);
-  int rTm = 8, rDm = 8;
-  for (auto& r : rec) {
-    if (r.r_T < 1 || r.r_T > sh.n_tokens || r.r_D < 1 || r.r_D > sh.head_dim || r.bits < 0 || r.bits > 8)
-      return fail(JOLT_ERR_BAD_BLOB, "unit record out of range");
-    if (r.off_U + 2ull * sh.n_tokens * r.r_T > total) return fail(JOLT_ERR_BAD_BLOB, "unit record offsets");
-    rTm = r.r_T > rTm ? r.r_T : rTm;
-    rDm = r.r_D > rDm ? r.r_D : rDm;
-  }
-  op.n_token_ranks = 1;
-  op.token_ranks[0] = (int)round_up(rTm, 8) > sh.n_tokens ? rTm : (int)round_up(rTm, 8);
-  op.n_feature_ranks = 1;
-  op.feature_ranks[0] = (int)round_up(rDm, 8) > sh.head_dim ? rDm : (int)round_up(rDm, 8);
-  op.n_bits = 1;
-  op.method = JOLT_EXACT;
-  op.unit_offset = h.unit_offset;
-  Plan p;
-  JTRY(make_plan(&sh, &op, &p));
-  if (ws_bytes < p.dws_total)
-    return fail(JOLT_ERR_WORKSPACE_TOO_SMALL, "decompress workspace %zu bytes, need %zu", ws_bytes, p.dws_total);
+  Prepared pr;
+  JTRY(decode_prepare(blob_dev, ws_dev, ws_bytes, st, &pr, true));
+  const Plan& p = pr.p;
+  const BlobHeader& h = pr.h;
   Ctx c{p, (unsigned char*)ws_dev, st, nullptr, nullptr, h.seed};
   bf16* Ucp = c.at<bf16>(p.d_U);
-  bf16* Wcp = c.at<bf16>(p.d_W);
-  bf16* Ccp = c.at<bf16>(p.d_C);
-  float* ptmp = c.at<float>(p.d_ptmp);
   bf16* P = c.at<bf16>(p.d_P);
-  int* umap = c.at<int>(p.d_umap);
-  JTRY(fill_umap(c, umap, p.NU));
-  CUDA_TRY(cudaMemsetAsync(ptmp, 0, (size_t)p.S * p.rTmax * p.D * 4, st));
   const unsigned char* blob = (const unsigned char*)blob_dev;
   const long long sP_unit = (long long)p.S * p.rTmax * p.D;
-  for (int u = 0; u < p.NU; ++u) {
-    const jolt_unit_record& r = rec[u];
-    bf16* Uu = Ucp + (size_t)u * p.T * p.ldU;
-    bf16* Wu = Wcp + (size_t)u * p.D * p.ldW;
-    bf16* Cu = Ccp + (size_t)u * p.S * p.rTmax * p.ldC;
-    count_launch(), copy2d_kernel<<<grid1d((long long)p.T * p.ldU), 256, 0, st>>>((const bf16*)(blob + r.off_U), p.T, r.r_T, Uu, p.ldU);
-    count_launch(), copy2d_kernel<<<grid1d((long long)p.D * p.ldW), 256, 0, st>>>((const bf16*)(blob + r.off_W), p.D, r.r_D, Wu, p.ldW);
-    count_launch(), copy2d_kernel<<<grid1d((long long)p.S * r.r_T * p.ldC), 256, 0, st>>>((const bf16*)(blob + r.off_C),
-                                                                          (long long)p.S * r.r_T, r.r_D, Cu, p.ldC);
-    CUDA_TRY(cudaGetLastError());
-    JTRY(pmat_unit(c, u, Cu, p.ldC, r.r_T, p.rTmax, Wu, p.ldW, r.r_D, ptmp, P + u * sP_unit, umap));
-  }
   DecodeArgs a;
   a.blob = blob;
   a.U = Ucp;
@@ -2183,6 +2216,105 @@ jolt_status jolt_decompress(const void* blob_dev, int32_t out_dtype, void* k_out
   }
   CUDA_TRY(cudaGetLastError());
   return JOLT_OK;
+}
+
+}  // extern "C"
+
+namespace {
+// token chunks per KV head for the decode-side attention: about two CTAs per SM in all,
+// at least 64 tokens per chunk, at most 64 chunks
+int attend_chunks(int T, int H) {
+  long long n = ceil_div(2 * 148, H);
+  n = n < 1 ? 1 : (n > 64 ? 64 : n);
+  const long long byT = ceil_div(T, att::TT);
+  return (int)(n < byT ? n : byT);
+}
+size_t attend_scratch(int T, int H, int D, int rTmax, int nq) {
+  const int G = nq / H;
+  return sizeof(float) * ((size_t)nq * D + (size_t)nq * rTmax +
+                          (size_t)H * attend_chunks(T, H) * G * (2 + (size_t)rTmax + D)) + 256;
+}
+
+template <int D>
+jolt_status launch_attend(const AttendArgs& a, cudaStream_t st) {
+  count_launch(), attend_query_kernel<D><<<a.nq, att::THREADS, 0, st>>>(a);
+  CUDA_TRY(cudaGetLastError());
+  const size_t sm = attend_chunk_smem(D, a.rTmax, a.G);
+  CUDA_TRY(cudaFuncSetAttribute(attend_chunk_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm));
+  count_launch(), attend_chunk_kernel<D><<<dim3(a.nch, a.H), att::THREADS, sm, st>>>(a);
+  CUDA_TRY(cudaGetLastError());
+  count_launch(), attend_combine_kernel<D><<<a.nq, att::THREADS, 0, st>>>(a);
+  CUDA_TRY(cudaGetLastError());
+  return JOLT_OK;
+}
+}  // namespace
+
+extern "C" {
+
+jolt_status jolt_attend_prepare(const void* blob_dev, void* ws_dev, size_t ws_bytes, void* stream) {
+  if (!blob_dev || !ws_dev) return fail(JOLT_ERR_INVALID_ARG, "null pointer");
+  Prepared pr;
+  return decode_prepare(blob_dev, ws_dev, ws_bytes, (cudaStream_t)stream, &pr, true);
+}
+
+jolt_status jolt_attend_scratch_size(const jolt_shape* shape, int32_t max_token_rank, int32_t n_q_heads,
+                                     size_t* bytes) {
+  if (!shape || !bytes || n_q_heads < 1 || max_token_rank < 1) return fail(JOLT_ERR_INVALID_ARG, "attend sizes");
+  if (shape->n_heads < 1 || n_q_heads % shape->n_heads) return fail(JOLT_ERR_INVALID_ARG, "n_q_heads % n_heads");
+  const int rT = (int)round_up(max_token_rank, 8);
+  *bytes = attend_scratch(shape->n_tokens, shape->n_heads, shape->head_dim, rT, n_q_heads);
+  return JOLT_OK;
+}
+
+jolt_status jolt_attend(const void* blob_dev, const void* ws_dev, size_t ws_bytes, int32_t layer, const float* q_dev,
+                        int32_t n_q_heads, float* out_dev, void* scratch_dev, size_t scratch_bytes, void* stream) {
+  if (!blob_dev || !ws_dev || !q_dev || !out_dev || !scratch_dev) return fail(JOLT_ERR_INVALID_ARG, "null pointer");
+  cudaStream_t st = (cudaStream_t)stream;
+  Prepared pr;
+  JTRY(decode_prepare(blob_dev, const_cast<void*>(ws_dev), ws_bytes, st, &pr, false));
+  const Plan& p = pr.p;
+  if (layer < 0 || layer >= p.nL) return fail(JOLT_ERR_INVALID_ARG, "layer %d not in [0, %d)", layer, p.nL);
+  if (n_q_heads < p.H || n_q_heads % p.H || n_q_heads / p.H > att::MAXG)
+    return fail(JOLT_ERR_INVALID_ARG, "n_q_heads %d: a multiple of the %d KV heads, at most %d per KV head",
+                n_q_heads, p.H, att::MAXG);
+  if (p.rTmax > att::MAXR) return fail(JOLT_ERR_UNSUPPORTED_SHAPE, "stored token rank above %d", att::MAXR);
+  if (p.D < 16) return fail(JOLT_ERR_UNSUPPORTED_SHAPE, "head_dim");
+  const size_t need = attend_scratch(p.T, p.H, p.D, p.rTmax, n_q_heads);
+  if (scratch_bytes < need) return fail(JOLT_ERR_WORKSPACE_TOO_SMALL, "attend scratch %zu bytes, need %zu",
+                                        scratch_bytes, need);
+  Ctx c{p, (unsigned char*)const_cast<void*>(ws_dev), st, nullptr, nullptr, pr.h.seed};
+  AttendArgs a;
+  a.blob = (const unsigned char*)blob_dev;
+  a.U = c.at<bf16>(p.d_U);
+  a.ldU = p.ldU;
+  a.sU = (long long)p.T * p.ldU;
+  a.P = c.at<bf16>(p.d_P);
+  a.sP_unit = (long long)p.S * p.rTmax * p.D;
+  a.rTmax = p.rTmax;
+  a.T = p.T;
+  a.S = p.S;
+  a.H = p.H;
+  a.D = p.D;
+  a.Lg = p.Lg;
+  a.u0 = p.u0;
+  a.seed = pr.h.seed;
+  a.layer = layer;
+  a.nq = n_q_heads;
+  a.G = n_q_heads / p.H;
+  a.q = q_dev;
+  float* sc = (float*)(((uintptr_t)scratch_dev + 255) & ~(uintptr_t)255);
+  a.qrot = sc;
+  a.a = a.qrot + (size_t)n_q_heads * p.D;
+  a.part = a.a + (size_t)n_q_heads * p.rTmax;
+  a.nch = attend_chunks(p.T, p.H);
+  a.out = out_dev;
+  ProfScope ps("attend", st, 1);
+  switch (p.D) {
+    case 16: return launch_attend<16>(a, st);
+    case 32: return launch_attend<32>(a, st);
+    case 64: return launch_attend<64>(a, st);
+    default: return launch_attend<128>(a, st);
+  }
 }
 
 jolt_status jolt_frobenius(const jolt_shape* shape, const void* k_dev, const void* v_dev, const void* ky_dev,

@@ -205,11 +205,12 @@ __device__ __forceinline__ void recon_mma_k16(const bf16* st, int kk, int kabs, 
 }
 
 // Walk the token-rank axis [0, kmax) in KC chunks; call epi(i) whenever the
-// accumulated prefix reaches cut[i] (cuts ascending, all <= kmax).
-template <int D, int SPLIT = 1, typename Epi>
-__device__ __forceinline__ void recon_walk(bf16* smem_stages, const bf16* U, long long ldU, int T, int t0,
-                                           const bf16* P, int kmax, const int* cuts, int ncuts,
-                                           float (*acc)[4], Epi&& epi) {
+// accumulated prefix reaches cut[i] (cuts ascending, all <= kmax), and fold() after every
+// whole chunk (the encoder moves the chunk's sums out of the accumulator there).
+template <int D, int SPLIT = 1, typename Epi, typename Fold>
+__device__ __forceinline__ void recon_walk_fold(bf16* smem_stages, const bf16* U, long long ldU, int T, int t0,
+                                                const bf16* P, int kmax, const int* cuts, int ncuts,
+                                                float (*acc)[4], Epi&& epi, Fold&& fold) {
   using namespace gemm_detail;
   const int nchunks = (kmax + KC - 1) / KC;
   int ci = 0;
@@ -235,9 +236,24 @@ __device__ __forceinline__ void recon_walk(bf16* smem_stages, const bf16* U, lon
         while (ci < ncuts && cuts[ci] == lo) { epi(ci); ++ci; }
       }
     }
+    if (ci < ncuts) fold();
     __syncthreads();
   }
   cp_async_wait<0>();
+}
+
+template <int D, int SPLIT = 1, typename Epi>
+__device__ __forceinline__ void recon_walk(bf16* smem_stages, const bf16* U, long long ldU, int T, int t0,
+                                           const bf16* P, int kmax, const int* cuts, int ncuts,
+                                           float (*acc)[4], Epi&& epi) {
+  recon_walk_fold<D, SPLIT>(smem_stages, U, ldU, T, t0, P, kmax, cuts, ncuts, acc, epi, [] {});
+}
+
+// error-free sum of two floats (Knuth's TwoSum): s + e == a + b exactly
+__device__ __forceinline__ void two_sum(float a, float b, float& s, float& e) {
+  s = __fadd_rn(a, b);
+  const float bb = __fsub_rn(s, a);
+  e = __fadd_rn(__fsub_rn(a, __fsub_rn(s, bb)), __fsub_rn(b, bb));
 }
 
 // ---------------------------------------------------------------------------------------
@@ -611,7 +627,37 @@ __global__ void __launch_bounds__(TTHREADS) encode_kernel(EncodeArgs a) {
   const int brow = block_row<D>();
   const bool has_blocks = (RhoTile<D>::BLK_PER_THREAD > 0) || threadIdx.x < TROWS;
 
+  // the residual x' - U P' is kept as an unevaluated sum hi + lo: every whole chunk of token
+  // ranks is subtracted from it without rounding error (TwoSum), so only the fp32 sums inside
+  // one chunk round -- the reconstruction is subtracted from x' with a chunk's error, not the
+  // error of the whole sum
+  TileFrag<D> xl;
+#pragma unroll
+  for (int h = 0; h < 2; ++h)
+#pragma unroll
+    for (int j = 0; j < NT; ++j) xl.v[h][j][0] = xl.v[h][j][1] = 0.f;
+  auto fold = [&]() {
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+      for (int j = 0; j < NT; ++j)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          float sum, err;
+          two_sum(xf.v[h][j][e], -acc[j][h * 2 + e], sum, err);
+          xf.v[h][j][e] = sum;
+          xl.v[h][j][e] = __fadd_rn(xl.v[h][j][e], err);
+          acc[j][h * 2 + e] = 0.f;
+        }
+  };
   auto epi = [&](int) {
+    fold();
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+      for (int j = 0; j < NT; ++j)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) xf.v[h][j][e] = __fadd_rn(xf.v[h][j][e], xl.v[h][j][e]);
     write_rho<D>(rho, xf, acc);
     __syncthreads();
     const int t = t0 + brow;
@@ -645,7 +691,7 @@ __global__ void __launch_bounds__(TTHREADS) encode_kernel(EncodeArgs a) {
     }
   };
   int cut = uh.r_T;
-  recon_walk<D>(stages, U, a.ldU, T, t0, P, cut, &cut, 1, acc, epi);
+  recon_walk_fold<D>(stages, U, a.ldU, T, t0, P, cut, &cut, 1, acc, epi, fold);
 }
 
 // ---------------------------------------------------------------------------------------

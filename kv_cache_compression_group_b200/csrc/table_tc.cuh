@@ -9,7 +9,7 @@
 //     (64 x 128 bf16, rows of the operator) for every 64-wide K block;
 //   * one thread issues tcgen05.mma (M = 128, N = 128, K = 16) into the accumulator of the
 //     segment the K step belongs to and commits an mbarrier when a segment is complete;
-//   * eight epilogue warps (two per TMEM lane quarter, each half of the 128 columns) read a
+//   * sixteen epilogue warps (four per TMEM lane quarter, 32 columns each) read a
 //     finished segment with tcgen05.ld, release it at once (the next candidate's MMAs into
 //     that segment may start), add it to a running sum kept in registers, and evaluate the
 //     quantiser of every bit-width on rho = x' - running sum, block by block -- the
@@ -35,7 +35,8 @@ constexpr int P_BYTES = BK * DIM * 2;                      // 16 KB
 constexpr int STAGE_BYTES = U_BYTES + P_BYTES;
 constexpr int XS_LD = DIM + 4;                             // fp32 pitch of the rotated tile
 constexpr int XS_BYTES = ROWS * XS_LD * 4;
-constexpr int EPI_WARPS = 8;
+constexpr int EPI_WARPS = 16;                             // four per TMEM lane quarter
+constexpr int EPI_COLS = DIM / (EPI_WARPS / 4);            // columns per epilogue warp
 constexpr int THREADS = (EPI_WARPS + 2) * 32;              // + TMA warp + MMA warp
 constexpr int MAXT = 4;                                    // token-rank cuts
 constexpr int BAR_OFF = STAGES * STAGE_BYTES + XS_BYTES;
@@ -223,17 +224,17 @@ __global__ void __launch_bounds__(ttc::THREADS, 1)
       umma::mma_commit(done_bar);   // fires when every MMA issued above has completed
     }
   } else {
-    // ---- epilogue: warp w owns TMEM lanes 32 (w % 4) .. +31 and columns 64 (w / 4) .. +63 ----
+    // ---- epilogue: warp w owns TMEM lanes 32 (w % 4) .. +31 and columns EPI_COLS (w / 4) .. ----
     const int row = 32 * (warp & 3) + lane;
-    const int cbase = 64 * (warp >> 2);
+    const int cbase = EPI_COLS * (warp >> 2);
     const uint32_t lane_addr = (uint32_t)(32 * (warp & 3)) << 16;
     const BitConsts kb = bit_consts(cd);
     double* out = a.partial + (((long long)u * S + s) * a.tiles + tile) * (long long)(nD * nT * nB);
     const float* xrow = xs + row * XS_LD + cbase;
     for (int iD = 0; iD < nD; ++iD) {
-      float run[64];
+      float run[EPI_COLS];
 #pragma unroll
-      for (int j = 0; j < 64; ++j) run[j] = 0.f;
+      for (int j = 0; j < EPI_COLS; ++j) run[j] = 0.f;
 #pragma unroll 1
       for (int i = 0; i < nT; ++i) {
         bool ok = !*abort_flag && umma::mbar_wait(accfull0 + 8 * i, iD & 1);
@@ -245,13 +246,12 @@ __global__ void __launch_bounds__(ttc::THREADS, 1)
         if (ok) {
           umma::fence_after_sync();
 #pragma unroll
-          for (int hh = 0; hh < 2; ++hh) {
-            float seg[32];
-            ttc_tmem_ld16(tmem + lane_addr + (uint32_t)(i * DIM + cbase + 32 * hh), seg);
-            ttc_tmem_ld16(tmem + lane_addr + (uint32_t)(i * DIM + cbase + 32 * hh + 16), seg + 16);
+          for (int hh = 0; hh < EPI_COLS / 16; ++hh) {
+            float seg[16];
+            ttc_tmem_ld16(tmem + lane_addr + (uint32_t)(i * DIM + cbase + 16 * hh), seg);
             asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
-            for (int j = 0; j < 32; ++j) run[32 * hh + j] += seg[j];
+            for (int j = 0; j < 16; ++j) run[16 * hh + j] += seg[j];
           }
           // the segment is in registers: release it to the next candidate's MMAs
           umma::fence_before_sync();
@@ -259,7 +259,7 @@ __global__ void __launch_bounds__(ttc::THREADS, 1)
           if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(accfree0 + 8 * i) : "memory");
           if (t0 + row < T) {
 #pragma unroll
-            for (int m = 0; m < 4; ++m) {
+            for (int m = 0; m < EPI_COLS / 16; ++m) {
               float v[16];
               load16(xrow + 16 * m, v);
 #pragma unroll
@@ -279,7 +279,7 @@ __global__ void __launch_bounds__(ttc::THREADS, 1)
           if (lane == 0) red[warp][i * MAXC + b] = v;
         }
       }
-      // over the eight epilogue warps in fixed order (fp64)
+      // over the epilogue warps in fixed order (fp64)
       ttc_epi_sync();
       if (threadIdx.x < nT * nB) {
         const int i = threadIdx.x / nB, b = threadIdx.x - i * nB;

@@ -29,7 +29,7 @@ EXPORTED = [
     "jolt_compress", "jolt_factor", "jolt_table", "jolt_allocate", "jolt_encode", "jolt_read_header",
     "jolt_decompress", "jolt_frobenius", "jolt_profile_begin", "jolt_profile_end", "jolt_recon_operator",
     "jolt_launch_count", "jolt_frobenius_noalloc", "jolt_set_graphs", "jolt_release", "jolt_fp32_rate_probe",
-    "jolt_wait_selftest",
+    "jolt_wait_selftest", "jolt_attend_prepare", "jolt_attend_scratch_size", "jolt_attend",
 ]
 
 
@@ -94,6 +94,9 @@ def lib():
             "jolt_release": [],
             "jolt_fp32_rate_probe": [i32, i32, vp, ctypes.POINTER(u64), vp],
             "jolt_wait_selftest": [i32, ctypes.c_uint32, vp, vp],
+            "jolt_attend_prepare": [vp, vp, sz, vp],
+            "jolt_attend_scratch_size": [pS, i32, i32, ctypes.POINTER(sz)],
+            "jolt_attend": [vp, vp, sz, i32, vp, i32, vp, vp, sz, vp],
         }
         L.jolt_launch_count.argtypes = []
         L.jolt_launch_count.restype = ctypes.c_uint64
@@ -308,6 +311,35 @@ class Compressor:
                                      _ptr(K_out), _ptr(V_out), self._ws_ptr(self.dws), self.dws_bytes,
                                      _stream(stream)))
         return K_out, V_out
+
+
+class Attention:
+    """Decode-side attention over one compressed blob: prepare once (the aligned factors and
+    rotated operators in a workspace it owns), then attend(layer, q) for any layer."""
+
+    def __init__(self, comp: "Compressor", blob: torch.Tensor, n_q_heads: int, stream=None):
+        self.blob = blob
+        self.nq = int(n_q_heads)
+        self.D = comp.shape.head_dim
+        self.ws = torch.empty(comp.dws_bytes + 256, dtype=torch.uint8, device=blob.device)
+        self.ws_ptr = comp._ws_ptr(self.ws)
+        self.ws_bytes = comp.dws_bytes
+        nbytes = ctypes.c_size_t()
+        _check(lib().jolt_attend_scratch_size(ctypes.byref(comp.shape), max(comp.opts.token_ranks), self.nq,
+                                              ctypes.byref(nbytes)))
+        self.scratch = torch.empty(nbytes.value, dtype=torch.uint8, device=blob.device)
+        _check(lib().jolt_attend_prepare(_ptr(blob), self.ws_ptr, self.ws_bytes, _stream(stream)))
+
+    def attend(self, layer: int, q: torch.Tensor, out: torch.Tensor | None = None, stream=None):
+        """q [n_q_heads, head_dim] fp32 on the device; returns the attention output (same shape)."""
+        q = q.to(torch.float32).contiguous()
+        if q.shape != (self.nq, self.D):
+            raise ValueError(f"q must be [{self.nq}, {self.D}]")
+        if out is None:
+            out = torch.empty_like(q)
+        _check(lib().jolt_attend(_ptr(self.blob), self.ws_ptr, self.ws_bytes, int(layer), _ptr(q), self.nq, _ptr(out),
+                                 _ptr(self.scratch), self.scratch.numel(), _stream(stream)))
+        return out
 
 
 def read_header(blob: torch.Tensor, stream=None):
