@@ -382,6 +382,38 @@ def stage_rooflines(w, opts, n_units, prof, n_calls, per_call_ms, peaks, peak_sr
     return lines
 
 
+def attend_extras(J, comp, blob, w, dev, stream):
+    """Decode-side attention over the stored factors of the 2x blob: one decode step of 4
+    query heads per KV head against every cached token, layer by layer (all layers timed
+    together with CUDA events after a warm-up pass).  Bytes are those the kernels must read
+    for a layer: both token factors, the codes and the scales of the layer's slices."""
+    import torch
+    nq = 4 * w.n_heads
+    att = J.Attention(comp, blob, nq)
+    q = torch.randn((nq, w.D), dtype=torch.float32, device=dev, generator=torch.Generator(dev).manual_seed(1))
+    outs = torch.empty_like(q)
+    for layer in range(w.n_layers):
+        att.attend(layer, q, out=outs)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for layer in range(w.n_layers):
+        att.attend(layer, q, out=outs)
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / w.n_layers
+    _, _, recs = J.read_header(blob)
+    nbytes = 0.0
+    for g in range(w.n_groups):
+        rk, rv = recs[2 * g], recs[2 * g + 1]
+        for r in (rk, rv):
+            nbytes += 2.0 * w.T * r["r_T"]                                   # token factor
+            nbytes += w.n_heads * w.T * (w.D // 16) * (2 * r["bits"] + 4) if r["bits"] else 0.0
+    nbytes /= w.n_groups
+    return {"query_heads": nq, "ms_per_layer": ms, "bytes_per_layer": nbytes, "gbs": nbytes / ms / 1e6,
+            "note": "host sync per call to read the blob header is inside the timed region"}
+
+
 def mistral_extras(J, synth, dev, stream, flush):
     """The Mistral-7B-shaped cache (1024 tokens): FlashJoLT compress at 2x and 3x (graph
     replays, events around each call, L2 flushed before), and JoLT (exact) at 2x."""
@@ -610,6 +642,7 @@ def main():
         ek, evv = J.relative_errors(Kd, Vd, Ko, Vo, w.layers_per_group)
         out["decompress_2x"] = {"ms": dms, "out_gbs": in_bytes / dms / 1e6, "rel_err_K": ek, "rel_err_V": evv}
         del Ko, Vo
+        out["attend_2x"] = attend_extras(J, comp, blobs[0], w, dev, stream)
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         Ks = oracle_sample_input(w, 0)

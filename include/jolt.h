@@ -244,6 +244,21 @@ jolt_status jolt_attend_scratch_size(const jolt_shape* shape, int32_t max_token_
 jolt_status jolt_attend(const void* blob_dev, const void* ws_dev, size_t ws_bytes, int32_t layer, const float* q_dev,
                         int32_t n_q_heads, float* out_dev, void* scratch_dev, size_t scratch_bytes, void* stream);
 
+/* Per-block b-bit quantisation of the caches themselves, without factors or rotation: the
+ * plain quantisation baseline of the introduction of "A JoLT for the KV Cache ... Joint Tucker
+ * and JL-Residual Allocation for LLMs" (JoLT's error is roughly an order of magnitude below it
+ * and below cross-layer SVD; the cross-layer SVD baseline is jolt_compress with the feature
+ * ranks {head_dim} and the bit-widths {0}).  The quantiser of the residual: 16 consecutive
+ * features per block, fp16 lo = round-down(min), step = round-up((max - lo)/(2^b - 1)).
+ *   bits: 1..8; sq_dev [n_units][2] fp64 out: ||X_u||^2 and ||X_u - Q(X_u)||^2 (+inf if a
+ *   block's scale overflows fp16); codes_dev (2b bytes per block) and scales_dev (fp16 pairs)
+ *   optional (both or neither), blocks of unit u after those of units < u, 16-byte aligned;
+ *   ws_dev: 148 * 16 bytes per unit.  The stored form takes 2b + 4 bytes per 16 values.
+ *   Asynchronous. */
+jolt_status jolt_quant_baseline(const jolt_shape* shape, const void* k_dev, const void* v_dev, int32_t bits,
+                                void* codes_dev, void* scales_dev, double* sq_dev, void* ws_dev, size_t ws_bytes,
+                                void* stream);
+
 /* Per-unit sums of squares (the introduction reports the relative Frobenius error of K and
  * of V separately): sq_dev[2*u] = ||X_u||^2, sq_dev[2*u+1] = ||X_u - Y_u||^2
  * (fp64), X and Y of the same shape; y may be NULL (then only ||X_u||^2).  ydtype is Y's

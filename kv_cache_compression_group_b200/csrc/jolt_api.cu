@@ -2317,6 +2317,46 @@ jolt_status jolt_attend(const void* blob_dev, const void* ws_dev, size_t ws_byte
   }
 }
 
+jolt_status jolt_quant_baseline(const jolt_shape* shape, const void* k_dev, const void* v_dev, int32_t bits,
+                                void* codes_dev, void* scales_dev, double* sq_dev, void* ws_dev, size_t ws_bytes,
+                                void* stream) {
+  if (!shape || !k_dev || !v_dev || !sq_dev || !ws_dev) return fail(JOLT_ERR_INVALID_ARG, "null pointer");
+  if (bits < 1 || bits > 8) return fail(JOLT_ERR_INVALID_ARG, "bits %d not in [1, 8]", bits);
+  if ((codes_dev == nullptr) != (scales_dev == nullptr)) return fail(JOLT_ERR_INVALID_ARG, "give both or neither output");
+  if (shape->dtype != JOLT_BF16 && shape->dtype != JOLT_F32) return fail(JOLT_ERR_INVALID_ARG, "dtype");
+  if (shape->n_layers < 1 || shape->layers_per_group < 1 || shape->n_layers % shape->layers_per_group ||
+      shape->head_dim % 16 || shape->n_heads < 1 || shape->n_tokens < 1)
+    return fail(JOLT_ERR_UNSUPPORTED_SHAPE, "shape");
+  const int G = shape->n_layers / shape->layers_per_group, NU = 2 * G, nblk = 148;
+  if (ws_bytes < (size_t)NU * nblk * 16) return fail(JOLT_ERR_WORKSPACE_TOO_SMALL, "baseline workspace");
+  if (((uintptr_t)codes_dev % 16) || ((uintptr_t)scales_dev % 4)) return fail(JOLT_ERR_INVALID_ARG, "alignment");
+  CacheView cv;
+  cv.k = k_dev;
+  cv.v = v_dev;
+  cv.dtype = shape->dtype;
+  cv.n_layers = shape->n_layers;
+  cv.H = shape->n_heads;
+  cv.T = shape->n_tokens;
+  cv.D = shape->head_dim;
+  cv.Lg = shape->layers_per_group;
+  cv.S = cv.Lg * cv.H;
+  cv.u0 = 0;
+  cv.unit_elems = (long long)cv.S * cv.T * cv.D;
+  cudaStream_t st = (cudaStream_t)stream;
+  double* part = (double*)ws_dev;
+  ProfScope ps("quant_baseline", st, NU);
+  if (shape->dtype == JOLT_BF16)
+    count_launch(), quant_baseline_kernel<bf16><<<dim3(nblk, NU), 256, 0, st>>>(
+        cv, bits, (unsigned char*)codes_dev, (__half2*)scales_dev, part, nblk);
+  else
+    count_launch(), quant_baseline_kernel<float><<<dim3(nblk, NU), 256, 0, st>>>(
+        cv, bits, (unsigned char*)codes_dev, (__half2*)scales_dev, part, nblk);
+  CUDA_TRY(cudaGetLastError());
+  count_launch(), frob_final_kernel<<<(unsigned)ceil_div(2 * NU, 128), 128, 0, st>>>(part, NU, nblk, sq_dev);
+  CUDA_TRY(cudaGetLastError());
+  return JOLT_OK;
+}
+
 jolt_status jolt_frobenius(const jolt_shape* shape, const void* k_dev, const void* v_dev, const void* ky_dev,
                            const void* vy_dev, int32_t ydtype, double* sq_dev, void* ws_dev, size_t ws_bytes,
                            void* stream) {

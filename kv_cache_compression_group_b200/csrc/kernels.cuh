@@ -830,3 +830,69 @@ inline size_t decode_smem() {
 }
 
 }  // namespace jolt
+
+namespace jolt {
+// ---------------------------------------------------------------------------------------
+// Per-block b-bit quantisation of the cache itself (no factors, no rotation): the plain
+// quantisation baseline the pages set JoLT against ("A JoLT for the KV Cache ... Joint Tucker
+// and JL-Residual Allocation for LLMs", introduction: the error is roughly an order of
+// magnitude below cross-layer SVD and 4-bit quantisation).  Same quantiser as the residual:
+// asymmetric min-max over 16 consecutive features with fp16 (lo, step).  Every thread takes
+// whole blocks (consecutive threads consecutive blocks: coalesced 32- or 64-byte reads);
+// per CTA and unit the fp64 sums of x^2 and of the squared error; codes and scales written
+// when the output pointers are given (layout of the blob's residual arrays).
+// grid (nblk, units); 256 threads.
+// ---------------------------------------------------------------------------------------
+template <typename TX>
+__global__ void __launch_bounds__(256) quant_baseline_kernel(CacheView cv, int b, unsigned char* codes,
+                                                             __half2* scales, double* part, int nblk) {
+  const int u = blockIdx.y;
+  const TX* X = reinterpret_cast<const TX*>(cv.unit_ptr(u));
+  const long long nb = cv.unit_elems / 16;
+  const float flev = (float)((1 << b) - 1), inv_lev = 1.0f / flev;
+  double sx = 0.0, se = 0.0;
+  for (long long q = blockIdx.x * (long long)blockDim.x + threadIdx.x; q < nb; q += (long long)nblk * blockDim.x) {
+    float v[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = ld_as_float(X + q * 16 + i);
+    float mn, mx;
+    minmax16(v, mn, mx);
+    const float lo = rd16(mn);
+    const float step = quant_step(mx, lo, flev, inv_lev);
+    const bool ok = isfinite(lo) && step <= kFp16Max;
+    const float inv = (ok && step > 0.f) ? __frcp_rn(step) : 0.f;
+    uint32_t w[4] = {0u, 0u, 0u, 0u};
+    float ex = 0.f, ee = 0.f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const uint32_t c = ok ? block_code(v[i], lo, inv, flev) : 0u;
+      pack_code(w, i, b, c);
+      const float e = v[i] - fmaf((float)c, step, lo);
+      ex = fmaf(v[i], v[i], ex);
+      ee = fmaf(e, e, ee);
+    }
+    sx += (double)ex;
+    se += ok ? (double)ee : (double)INFINITY;
+    if (codes) {
+      unsigned char* dst = codes + ((long long)u * nb + q) * (2 * b);
+      for (int byte = 0; byte < 2 * b; ++byte) dst[byte] = (unsigned char)(w[byte >> 2] >> ((byte & 3) * 8));
+    }
+    if (scales) scales[(long long)u * nb + q] = __halves2half2(__float2half_rn(lo), __float2half_rn(step));
+  }
+  __shared__ double s1[256], s2[256];
+  s1[threadIdx.x] = sx;
+  s2[threadIdx.x] = se;
+  __syncthreads();
+  for (int st = blockDim.x / 2; st > 0; st >>= 1) {
+    if ((int)threadIdx.x < st) {
+      s1[threadIdx.x] += s1[threadIdx.x + st];
+      s2[threadIdx.x] += s2[threadIdx.x + st];
+    }
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    part[((long long)u * nblk + blockIdx.x) * 2 + 0] = s1[0];
+    part[((long long)u * nblk + blockIdx.x) * 2 + 1] = s2[0];
+  }
+}
+}  // namespace jolt

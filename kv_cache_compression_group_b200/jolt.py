@@ -29,7 +29,7 @@ EXPORTED = [
     "jolt_compress", "jolt_factor", "jolt_table", "jolt_allocate", "jolt_encode", "jolt_read_header",
     "jolt_decompress", "jolt_frobenius", "jolt_profile_begin", "jolt_profile_end", "jolt_recon_operator",
     "jolt_launch_count", "jolt_frobenius_noalloc", "jolt_set_graphs", "jolt_release", "jolt_fp32_rate_probe",
-    "jolt_wait_selftest", "jolt_attend_prepare", "jolt_attend_scratch_size", "jolt_attend",
+    "jolt_wait_selftest", "jolt_attend_prepare", "jolt_attend_scratch_size", "jolt_attend", "jolt_quant_baseline",
 ]
 
 
@@ -97,6 +97,7 @@ def lib():
             "jolt_attend_prepare": [vp, vp, sz, vp],
             "jolt_attend_scratch_size": [pS, i32, i32, ctypes.POINTER(sz)],
             "jolt_attend": [vp, vp, sz, i32, vp, i32, vp, vp, sz, vp],
+            "jolt_quant_baseline": [pS, vp, vp, i32, vp, vp, vp, vp, sz, vp],
         }
         L.jolt_launch_count.argtypes = []
         L.jolt_launch_count.restype = ctypes.c_uint64
@@ -438,6 +439,21 @@ def frobenius_noalloc(K, V, K_hat=None, V_hat=None, layers_per_group=1, stream=N
     _check(lib().jolt_frobenius_noalloc(ctypes.byref(shape), _ptr(K), _ptr(V), _ptr(K_hat), _ptr(V_hat), yd,
                                         _ptr(sq), _stream(stream)))
     return sq.view(2 * G, 2)
+
+
+def quant_baseline(K, V, bits: int, layers_per_group: int, keep_codes: bool = False, stream=None):
+    """Per-block b-bit quantisation of K and V themselves: per-unit [||X_u||^2, ||X_u - Q(X_u)||^2]
+    (fp64, device), and (keep_codes) the codes and fp16 scales."""
+    shape = make_shape(K, layers_per_group)
+    G = K.shape[0] // layers_per_group
+    nblk_all = 2 * K.numel() // 16
+    sq = torch.zeros(2 * 2 * G, dtype=torch.float64, device=K.device)
+    ws = torch.empty(2 * G * 148 * 16, dtype=torch.uint8, device=K.device)
+    codes = torch.empty(nblk_all * 2 * bits, dtype=torch.uint8, device=K.device) if keep_codes else None
+    scales = torch.empty(nblk_all * 2, dtype=torch.float16, device=K.device) if keep_codes else None
+    _check(lib().jolt_quant_baseline(ctypes.byref(shape), _ptr(K), _ptr(V), int(bits), _ptr(codes), _ptr(scales),
+                                     _ptr(sq), _ptr(ws), ws.numel(), _stream(stream)))
+    return sq.view(2 * G, 2), codes, scales
 
 
 def relative_errors(K, V, K_hat, V_hat, layers_per_group):
