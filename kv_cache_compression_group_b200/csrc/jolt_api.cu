@@ -1592,11 +1592,34 @@ jolt_status run_encode(const Ctx& c, const bf16* Us, long long ldU, const bf16* 
   a.seed = c.seed;
   a.blob = blob;
   ProfScope ps("encode", c.st, p.NU);
-  switch (p.D) {
-    case 16: JTRY(launch_encode_D<16>(c, a)); break;
-    case 32: JTRY(launch_encode_D<32>(c, a)); break;
-    case 64: JTRY(launch_encode_D<64>(c, a)); break;
-    default: JTRY(launch_encode_D<128>(c, a)); break;
+  if (table_tc_ok(p, ldU)) {
+    // the tensor-core encoder (every candidate token rank a multiple of 16, D = 128)
+    CUtensorMap mu, mp;
+    if (!map_dense(&mu, Us, ldU, p.T, p.NU) || !map_dense(&mp, a.P, p.D, p.rTmax, (long long)p.cd.nD * p.NU * p.S))
+      return fail(JOLT_ERR_CUDA, "tensor map of the encoder operands refused");
+    EncodeTcArgs e;
+    e.cv = a.cv;
+    e.rTmax = p.rTmax;
+    e.cand = p.cd;
+    e.seed = c.seed;
+    e.blob = blob;
+    e.status = c.status();
+    const dim3 grid((unsigned)ceil_div(p.T, ttc::ROWS), p.S, p.NU);
+    if (p.dtype == JOLT_BF16) {
+      CUDA_TRY(cudaFuncSetAttribute(encode_tc_kernel<bf16>, cudaFuncAttributeMaxDynamicSharedMemorySize, ttc::SMEM));
+      count_launch(), encode_tc_kernel<bf16><<<grid, etc::THREADS, ttc::SMEM, c.st>>>(mu, mp, e);
+    } else {
+      CUDA_TRY(cudaFuncSetAttribute(encode_tc_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, ttc::SMEM));
+      count_launch(), encode_tc_kernel<float><<<grid, etc::THREADS, ttc::SMEM, c.st>>>(mu, mp, e);
+    }
+    CUDA_TRY(cudaGetLastError());
+  } else {
+    switch (p.D) {
+      case 16: JTRY(launch_encode_D<16>(c, a)); break;
+      case 32: JTRY(launch_encode_D<32>(c, a)); break;
+      case 64: JTRY(launch_encode_D<64>(c, a)); break;
+      default: JTRY(launch_encode_D<128>(c, a)); break;
+    }
   }
   count_launch(), copy_factors_kernel<<<dim3(64, p.NU), 256, 0, c.st>>>(blob, Us, ldU, (long long)p.T * ldU, Ws, ldW,
                                                          (long long)p.D * ldW, core, p.ldC, (long long)p.rTmax * p.ldC,

@@ -56,10 +56,10 @@ struct TableTcArgs {
 
 // the tile's rows rotated along the features into xs (fp32, pitch XS_LD): sign flip, the
 // Walsh-Hadamard butterflies in the order of fwht_regs (strides 1, 2, ..., 64), 1 / sqrt(D)
-template <typename TX>
+template <typename TX, int NTHREADS>
 __device__ __forceinline__ void ttc_rotate_tile(const TX* X, int T, int t0, const float* sig, float* xs) {
   using namespace ttc;
-  for (int idx = threadIdx.x; idx < ROWS * DIM; idx += THREADS) {
+  for (int idx = threadIdx.x; idx < ROWS * DIM; idx += NTHREADS) {
     const int r = idx / DIM, d = idx - r * DIM, t = t0 + r;
     xs[r * XS_LD + d] = t < T ? ld_as_float(X + (long long)t * DIM + d) * sig[d] : 0.f;
   }
@@ -103,6 +103,96 @@ __device__ __forceinline__ void ttc_tmem_ld16(uint32_t taddr, float* v) {
       : "r"(taddr));
 #pragma unroll
   for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// ---------------------------------------------------------------------------------------
+// Quantiser error sums of one 16-wide block for the table (packed pairs throughout):
+//   * block min / max by three-input min / max (exact, the same values as a two-input tree);
+//   * lo and the fp16 step exactly as the encoder forms them (rd16, quant_step);
+//   * code = round-half-even(d / step) through the approximate reciprocal of step, the error
+//     (d - code * step)^2 summed in four packed partial sums.
+// The approximate reciprocal can move a code only where d / step lies within a few ulp of a
+// half-integer, where both neighbouring codes give the same squared error to that precision,
+// so the table entry (a sum of squared errors) is unchanged to fp32 resolution; the stored
+// codes come from the encoder, which uses the correctly rounded reciprocal.
+// ---------------------------------------------------------------------------------------
+__device__ __forceinline__ float ttc_min3(float a, float b, float c) {
+  float r;
+  asm("min.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+__device__ __forceinline__ float ttc_max3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+__device__ __forceinline__ float ttc_rcp_approx(float x) {
+  float r;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
+}
+
+template <int B>
+__device__ __forceinline__ void ttc_bit_error(const float2* v, const float2* d, float mx, float lo, float& err) {
+  if constexpr (B == 0) {
+    float2 a0 = make_float2(0.f, 0.f), a1 = a0, a2 = a0, a3 = a0;
+#pragma unroll
+    for (int j = 0; j < 8; j += 4) {
+      a0 = __ffma2_rn(v[j], v[j], a0);
+      a1 = __ffma2_rn(v[j + 1], v[j + 1], a1);
+      a2 = __ffma2_rn(v[j + 2], v[j + 2], a2);
+      a3 = __ffma2_rn(v[j + 3], v[j + 3], a3);
+    }
+    err += ((a0.x + a0.y) + (a1.x + a1.y)) + ((a2.x + a2.y) + (a3.x + a3.y));
+  } else {
+    constexpr float flev = (float)((1 << B) - 1);
+    const float inv_lev = 1.0f / flev;
+    const float step = quant_step(mx, lo, flev, inv_lev);
+    if (!(isfinite(lo) && step <= kFp16Max)) {
+      err = INFINITY;
+      return;
+    }
+    const float inv = step > 0.f ? ttc_rcp_approx(step) : 0.f;
+    const float2 inv2 = make_float2(inv, inv), nstep2 = make_float2(-step, -step);
+    const float2 sh = make_float2(kRoundShift, kRoundShift), nsh = make_float2(-kRoundShift, -kRoundShift);
+    float2 a0 = make_float2(0.f, 0.f), a1 = a0, a2 = a0, a3 = a0;
+#pragma unroll
+    for (int j = 0; j < 8; j += 4) {
+      const float2 c0 = __fadd2_rn(__ffma2_rn(d[j], inv2, sh), nsh);
+      const float2 c1 = __fadd2_rn(__ffma2_rn(d[j + 1], inv2, sh), nsh);
+      const float2 c2 = __fadd2_rn(__ffma2_rn(d[j + 2], inv2, sh), nsh);
+      const float2 c3 = __fadd2_rn(__ffma2_rn(d[j + 3], inv2, sh), nsh);
+      const float2 e0 = __ffma2_rn(c0, nstep2, d[j]);
+      const float2 e1 = __ffma2_rn(c1, nstep2, d[j + 1]);
+      const float2 e2 = __ffma2_rn(c2, nstep2, d[j + 2]);
+      const float2 e3 = __ffma2_rn(c3, nstep2, d[j + 3]);
+      a0 = __ffma2_rn(e0, e0, a0);
+      a1 = __ffma2_rn(e1, e1, a1);
+      a2 = __ffma2_rn(e2, e2, a2);
+      a3 = __ffma2_rn(e3, e3, a3);
+    }
+    err += ((a0.x + a0.y) + (a1.x + a1.y)) + ((a2.x + a2.y) + (a3.x + a3.y));
+  }
+}
+
+// every bit-width of the set for one block of rho given as 8 packed pairs
+template <int... Bs>
+__device__ __forceinline__ void ttc_block_errors(const float2* v, float* err, BitSet<Bs...>) {
+  const float m0 = ttc_min3(v[0].x, v[0].y, v[1].x), m1 = ttc_min3(v[1].y, v[2].x, v[2].y);
+  const float m2 = ttc_min3(v[3].x, v[3].y, v[4].x), m3 = ttc_min3(v[4].y, v[5].x, v[5].y);
+  const float m4 = ttc_min3(v[6].x, v[6].y, v[7].x);
+  const float mn = fminf(ttc_min3(m0, m1, m2), ttc_min3(m3, m4, v[7].y));
+  const float x0 = ttc_max3(v[0].x, v[0].y, v[1].x), x1 = ttc_max3(v[1].y, v[2].x, v[2].y);
+  const float x2 = ttc_max3(v[3].x, v[3].y, v[4].x), x3 = ttc_max3(v[4].y, v[5].x, v[5].y);
+  const float x4 = ttc_max3(v[6].x, v[6].y, v[7].x);
+  const float mx = fmaxf(ttc_max3(x0, x1, x2), ttc_max3(x3, x4, v[7].y));
+  const float lo = rd16(mn);
+  const float2 nlo = make_float2(-lo, -lo);
+  float2 d[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) d[j] = __fadd2_rn(v[j], nlo);
+  int i = 0;
+  (ttc_bit_error<Bs>(v, d, mx, lo, err[i++]), ...);
 }
 
 __device__ __forceinline__ void ttc_epi_sync() { asm volatile("bar.sync 1, %0;" ::"n"(ttc::EPI_WARPS * 32) : "memory"); }
@@ -157,7 +247,7 @@ __global__ void __launch_bounds__(ttc::THREADS, 1)
   for (int d = threadIdx.x; d < DIM; d += THREADS) sig[d] = rotation_sign(a.seed, u + a.cv.u0, d);
   __syncthreads();
   const TX* X = reinterpret_cast<const TX*>(a.cv.unit_ptr(u)) + (long long)s * T * DIM;
-  ttc_rotate_tile<TX>(X, T, t0, sig, xs);
+  ttc_rotate_tile<TX, THREADS>(X, T, t0, sig, xs);
   umma::fence_before_sync();
   __syncthreads();
   umma::fence_after_sync();
@@ -231,10 +321,11 @@ __global__ void __launch_bounds__(ttc::THREADS, 1)
     const BitConsts kb = bit_consts(cd);
     double* out = a.partial + (((long long)u * S + s) * a.tiles + tile) * (long long)(nD * nT * nB);
     const float* xrow = xs + row * XS_LD + cbase;
+    const float2 neg1 = make_float2(-1.f, -1.f);
     for (int iD = 0; iD < nD; ++iD) {
-      float run[EPI_COLS];
+      float2 nrun[EPI_COLS / 2];   // minus the running sum of the finished segments
 #pragma unroll
-      for (int j = 0; j < EPI_COLS; ++j) run[j] = 0.f;
+      for (int j = 0; j < EPI_COLS / 2; ++j) nrun[j] = make_float2(0.f, 0.f);
 #pragma unroll 1
       for (int i = 0; i < nT; ++i) {
         bool ok = !*abort_flag && umma::mbar_wait(accfull0 + 8 * i, iD & 1);
@@ -251,7 +342,8 @@ __global__ void __launch_bounds__(ttc::THREADS, 1)
             ttc_tmem_ld16(tmem + lane_addr + (uint32_t)(i * DIM + cbase + 16 * hh), seg);
             asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
-            for (int j = 0; j < 16; ++j) run[16 * hh + j] += seg[j];
+            for (int j = 0; j < 8; ++j)
+              nrun[8 * hh + j] = __ffma2_rn(make_float2(seg[2 * j], seg[2 * j + 1]), neg1, nrun[8 * hh + j]);
           }
           // the segment is in registers: release it to the next candidate's MMAs
           umma::fence_before_sync();
@@ -260,12 +352,18 @@ __global__ void __launch_bounds__(ttc::THREADS, 1)
           if (t0 + row < T) {
 #pragma unroll
             for (int m = 0; m < EPI_COLS / 16; ++m) {
-              float v[16];
-              load16(xrow + 16 * m, v);
+              float2 v2[8];
 #pragma unroll
-              for (int j = 0; j < 16; ++j) v[j] -= run[16 * m + j];
-              if constexpr (std::is_same<BITS, void>::value) block_errors(v, kb, err);
-              else block_errors_fixed(v, err, BITS{});
+              for (int q = 0; q < 4; ++q) {
+                const float4 xv = reinterpret_cast<const float4*>(xrow + 16 * m)[q];
+                v2[2 * q] = __fadd2_rn(make_float2(xv.x, xv.y), nrun[8 * m + 2 * q]);
+                v2[2 * q + 1] = __fadd2_rn(make_float2(xv.z, xv.w), nrun[8 * m + 2 * q + 1]);
+              }
+              if constexpr (std::is_same<BITS, void>::value) {
+                block_errors(reinterpret_cast<const float*>(v2), kb, err);
+              } else {
+                ttc_block_errors(v2, err, BITS{});
+              }
             }
           }
         }
@@ -302,4 +400,205 @@ __global__ void __launch_bounds__(ttc::THREADS, 1)
   }
 }
 
+}  // namespace jolt
+
+namespace jolt {
+// ---------------------------------------------------------------------------------------
+// Encoder on the tensor cores (D = 128): the chosen (r_T, r_D, b) of the unit from the blob's
+// unit table; one CTA per 128 tokens of one slice.  The token-rank axis [0, r_T) is cut into
+// 64-rank segments that rotate through the four TMEM accumulators.  The epilogue subtracts
+// every finished segment from the rotated tile without rounding error (TwoSum into hi + lo),
+// so the residual carries the fp32 error of one 64-rank segment, not of the whole sum; then
+// it quantises rho = hi + lo block by block, packs the codes and writes codes and scales.
+// Sixteen epilogue warps (four per TMEM lane quarter, 32 columns each).
+// ---------------------------------------------------------------------------------------
+namespace etc {
+constexpr int EPI_WARPS = 16;
+constexpr int THREADS = (EPI_WARPS + 2) * 32;
+constexpr int COLS = ttc::DIM / (EPI_WARPS / 4);   // 32
+}  // namespace etc
+
+struct EncodeTcArgs {
+  CacheView cv;
+  int rTmax;
+  Cands cand;
+  uint64_t seed;
+  unsigned char* blob;
+  uint32_t* status;
+};
+
+template <typename TX>
+__global__ void __launch_bounds__(etc::THREADS, 1)
+    encode_tc_kernel(const __grid_constant__ CUtensorMap map_u, const __grid_constant__ CUtensorMap map_p,
+                     EncodeTcArgs a) {
+  using namespace ttc;
+  extern __shared__ uint8_t etc_raw[];
+  uint8_t* smem = (uint8_t*)(((uintptr_t)etc_raw + 1023) & ~(uintptr_t)1023);
+  float* xs = reinterpret_cast<float*>(smem + STAGES * STAGE_BYTES);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + BAR_OFF);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 2 * MAXT + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  __shared__ float sig[DIM];
+
+  const int tile = blockIdx.x, s = blockIdx.y, u = blockIdx.z;
+  const BlobHeader* gh = reinterpret_cast<const BlobHeader*>(a.blob);
+  const UnitHeader uh = reinterpret_cast<const UnitHeader*>(a.blob + sizeof(BlobHeader))[u];
+  if (gh->status != 0 || uh.bits == 0) return;   // uniform over the CTA: nothing to write
+  const int T = a.cv.T, S = a.cv.S, NU = 2 * (a.cv.n_layers / a.cv.Lg);
+  const int t0 = tile * ROWS;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int rT = uh.r_T, b = uh.bits;
+  int iD = 0;
+  while (iD < a.cand.nD && a.cand.rD[iD] != uh.r_D) ++iD;
+  const int nkb = (rT + BK - 1) / BK;     // K blocks = segments (64 ranks each)
+  const uint32_t full0 = umma::smem_u32(bars), empty0 = full0 + 8 * STAGES, accfull0 = empty0 + 8 * STAGES;
+  const uint32_t accfree0 = accfull0 + 8 * MAXT, done_bar = accfree0 + 8 * MAXT;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < STAGES; ++i) {
+      umma::mbar_init(full0 + 8 * i, 1);
+      umma::mbar_init(empty0 + 8 * i, 1);
+    }
+    for (int i = 0; i < MAXT; ++i) {
+      umma::mbar_init(accfull0 + 8 * i, 1);
+      umma::mbar_init(accfree0 + 8 * i, etc::EPI_WARPS);
+    }
+    umma::mbar_init(done_bar, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (warp == etc::EPI_WARPS) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(umma::smem_u32(tmem_slot)),
+                 "n"(TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  for (int d = threadIdx.x; d < DIM; d += etc::THREADS) sig[d] = rotation_sign(a.seed, u + a.cv.u0, d);
+  __syncthreads();
+  ttc_rotate_tile<TX, etc::THREADS>(reinterpret_cast<const TX*>(a.cv.unit_ptr(u)) + (long long)s * T * DIM, T, t0,
+                                   sig, xs);
+  umma::fence_before_sync();
+  __syncthreads();
+  umma::fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+  const int ep = (iD * NU + u) * S + s;
+
+  if (warp == etc::EPI_WARPS) {
+    if (lane == 0) {
+      for (int j = 0; j < nkb; ++j) {
+        const int st = j % STAGES;
+        if (j >= STAGES && !umma::mbar_wait(empty0 + 8 * st, ((j / STAGES) & 1) ^ 1)) {
+          *abort_flag = 1;
+          break;
+        }
+        const uint32_t fb = full0 + 8 * st;
+        const uint32_t sa = umma::smem_u32(smem + st * STAGE_BYTES);
+        umma::mbar_expect_tx(fb, STAGE_BYTES);
+        umma::tma_load_3d(sa, &map_u, j * BK, t0, u, fb);
+        umma::tma_load_3d(sa + umma::BOX_BYTES, &map_u, j * BK, t0 + 64, u, fb);
+        umma::tma_load_3d(sa + U_BYTES, &map_p, 0, j * BK, ep, fb);
+        umma::tma_load_3d(sa + U_BYTES + umma::BOX_BYTES, &map_p, 64, j * BK, ep, fb);
+      }
+    }
+  } else if (warp == etc::EPI_WARPS + 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = umma::instr_desc(DIM, false, true);
+      for (int j = 0; j < nkb && !*abort_flag; ++j) {
+        const int st = j % STAGES, acc = j % MAXT, use = j / MAXT;
+        if (!umma::mbar_wait(full0 + 8 * st, (j / STAGES) & 1)) {
+          *abort_flag = 1;
+          break;
+        }
+        if (use > 0 && !umma::mbar_wait(accfree0 + 8 * acc, (use - 1) & 1)) {
+          *abort_flag = 1;
+          break;
+        }
+        umma::fence_after_sync();
+        const uint32_t sa = umma::smem_u32(smem + st * STAGE_BYTES);
+        for (int kk = 0; kk < BK / 16 && j * BK + kk * 16 < rT; ++kk) {
+          const uint64_t ad = umma::smem_desc(sa + kk * 32, 16, 1024);
+          const uint64_t bd = umma::smem_desc(sa + U_BYTES + kk * 2048, umma::BOX_BYTES, 1024);
+          umma::mma_bf16(tmem + (uint32_t)(acc * DIM), ad, bd, idesc, kk ? 1u : 0u);
+        }
+        umma::mma_commit(accfull0 + 8 * acc);
+        umma::mma_commit(empty0 + 8 * st);
+      }
+      umma::mma_commit(done_bar);
+    }
+  } else {
+    const int row = 32 * (warp & 3) + lane;
+    const int cbase = etc::COLS * (warp >> 2);
+    const uint32_t lane_addr = (uint32_t)(32 * (warp & 3)) << 16;
+    float hi[etc::COLS], lo[etc::COLS];
+#pragma unroll
+    for (int j = 0; j < etc::COLS; ++j) {
+      hi[j] = xs[row * XS_LD + cbase + j];
+      lo[j] = 0.f;
+    }
+    for (int j = 0; j < nkb; ++j) {
+      const int acc = j % MAXT, use = j / MAXT;
+      bool ok = !*abort_flag && umma::mbar_wait(accfull0 + 8 * acc, use & 1);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) {
+        *abort_flag = 1;
+        break;
+      }
+      umma::fence_after_sync();
+#pragma unroll
+      for (int hh = 0; hh < etc::COLS / 16; ++hh) {
+        float seg[16];
+        ttc_tmem_ld16(tmem + lane_addr + (uint32_t)(acc * DIM + cbase + 16 * hh), seg);
+        asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          float sum, err;
+          two_sum(hi[16 * hh + i], -seg[i], sum, err);
+          hi[16 * hh + i] = sum;
+          lo[16 * hh + i] = __fadd_rn(lo[16 * hh + i], err);
+        }
+      }
+      umma::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(accfree0 + 8 * acc) : "memory");
+    }
+    const int t = t0 + row;
+    if (!*abort_flag && t < T) {
+      const float flev = (float)((1 << b) - 1), inv_lev = 1.0f / flev;
+      unsigned char* codes = a.blob + uh.off_codes;
+      __half2* scales = reinterpret_cast<__half2*>(a.blob + uh.off_scales);
+#pragma unroll
+      for (int m = 0; m < etc::COLS / 16; ++m) {
+        float v[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) v[i] = __fadd_rn(hi[16 * m + i], lo[16 * m + i]);
+        float mn, mx;
+        minmax16(v, mn, mx);
+        const float l16 = rd16(mn);
+        const float step = quant_step(mx, l16, flev, inv_lev);
+        const float inv = (step > 0.f && step <= kFp16Max) ? __frcp_rn(step) : 0.f;
+        uint32_t w[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+        for (int i = 0; i < 16; ++i) pack_code(w, i, b, block_code(v[i], l16, inv, flev));
+        const long long blk = ((long long)s * T + t) * (DIM / 16) + cbase / 16 + m;
+        unsigned char* dst = codes + blk * (2 * b);
+        if (b == 8) *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+        else if (b == 4) *reinterpret_cast<uint2*>(dst) = make_uint2(w[0], w[1]);
+        else if (b == 2) *reinterpret_cast<uint32_t*>(dst) = w[0];
+        else
+          for (int byte = 0; byte < 2 * b; ++byte) dst[byte] = (unsigned char)(w[byte >> 2] >> ((byte & 3) * 8));
+        scales[blk] = __halves2half2(__float2half_rn(l16), __float2half_rn(step));
+      }
+    }
+  }
+  __syncwarp();
+  const bool drained = umma::mbar_wait(done_bar, 0);
+  if ((*abort_flag || !drained) && threadIdx.x == 0 && a.status) atomicOr(a.status, DEV_ERR_TIMEOUT);
+  umma::fence_before_sync();
+  __syncthreads();
+  if (warp == etc::EPI_WARPS) {
+    umma::fence_after_sync();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "n"(TMEM_COLS) : "memory");
+  }
+}
 }  // namespace jolt

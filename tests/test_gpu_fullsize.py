@@ -162,3 +162,28 @@ def test_full_size_factors_mistral():
                     checked += 1
         print(f"\n[mistral7b {method}] {checked} subspace cuts checked")
         assert checked >= 4, (method, checked)
+
+
+def test_free_zone_flashjolt_matches_jolt():
+    """Budget sweep 2x..5x on the Mistral-shaped cache, JoLT (exact token SVD) against FlashJoLT
+    (randomized): the randomized sketch must lose nothing measurable in the free zone ("A JoLT
+    for the KV cache ... Joint Rank-bit Allocation", abstract: FlashJoLT matches JoLT at a
+    fraction of the compression cost).  Criterion: FlashJoLT's relative Frobenius error of K and
+    of V at most 1.05 x JoLT's + 1e-4 at every budget."""
+    w = synth.WORKLOADS["mistral7b"]
+    K, V = synth.make_cache(w, SEED)
+    Kd, Vd = K.cuda(), V.cuda()
+    comps = {m: J.Compressor(w.n_layers, w.n_heads, w.T, w.D, w.layers_per_group, K.dtype,
+                             J.default_options(w.T, w.D, m)) for m in ("exact", "randomized")}
+    for ratio in (2.0, 3.0, 4.0, 5.0):
+        budget = int(w.bf16_bytes() / ratio)
+        err = {}
+        for m, comp in comps.items():
+            blob = comp.compress(Kd, Vd, budget, SEED)
+            _, total, _ = J.read_header(blob)
+            assert total <= budget
+            Kh, Vh = comp.decompress(blob, torch.float32)
+            err[m] = J.relative_errors(Kd, Vd, Kh, Vh, w.layers_per_group)
+        print(f"\n[free zone {ratio:g}x] JoLT K/V {err['exact']}, FlashJoLT K/V {err['randomized']}")
+        for kv in (0, 1):
+            assert err["randomized"][kv] <= 1.05 * err["exact"][kv] + 1e-4, (ratio, kv, err)
