@@ -11,7 +11,7 @@ CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libjolt.so")
 SOURCES = ["jolt_api.cu"]
 DEPS = ["jolt_api.cu", "common.cuh", "gemm.cuh", "kernels.cuh", "misc.cuh", "umma.cuh", "eig_cluster.cuh", "chol.cuh",
-        "fp16_exact.cuh", "table_tc.cuh", "attend.cuh"]
+        "fp16_exact.cuh", "table_tc.cuh", "attend.cuh", "eig_large.cuh"]
 
 
 def nvcc_cmd(out: str = LIB, extra=()) -> list:

@@ -1,4 +1,5 @@
-// Cholesky QR of the sketch blocks for widths k <= 256: Q = Y L^{-T} with G = Y^T Y = L L^T.
+// Cholesky QR of the sketch blocks: Q = Y L^{-T} with G = Y^T Y = L L^T (the factor kernels;
+// the products run on the tensor cores).
 //
 // Three kernels, all in fp64 up to the last product:
 //   chol_factor_kernel   one CTA per unit: the Cholesky factor L of the Gram, left-looking,
@@ -12,6 +13,8 @@
 // diagonal blocks to the upper triangle of their own diagonal block (W[i][c] at G[i*gld+c],
 // c <= i), both places the factorisation no longer reads.
 #pragma once
+
+#include <cooperative_groups.h>
 
 #include "common.cuh"
 
@@ -525,4 +528,141 @@ __global__ void __launch_bounds__(CF_THREADS) tri_inv_large_kernel(const double*
       Wu[(long long)(J0 + c) * ldw + i] = (i >= J0 && i < k) ? (float)X[(long long)i * CF_NB + c] : 0.f;
 }
 
+}  // namespace jolt
+
+namespace jolt {
+// ------------------------------------------------------------------------------------------
+// Cholesky factor for 256 < k <= 1024: one cluster of 8 CTAs per matrix, right-looking by
+// 32-column block columns, block column K owned by CTA K % 8.  Per block column J:
+//   1. its owner factors the diagonal block (one warp, column by column) and inverts it
+//      (forward substitution, one lane per column), then forms the panel
+//      L_IJ = A_IJ inv(L_JJ)^T for every block row I > J;
+//   2. cluster barrier;
+//   3. every CTA updates its block columns K > J: A_IK -= L_IJ L_KJ^T for I >= K.
+// The owner of block column J + 1 updated it in step 3 itself, so one barrier per block
+// column suffices.  Output in the layout of chol_factor_kernel: L below the diagonal blocks
+// in the lower triangle, inv(L_JJ) in the upper part of its diagonal block (W[i][c] at
+// G[i * gld + c], c <= i).  A pivot that is not positive: DEV_ERR_FACTOR, pivot taken as 1.
+// grid (8 * matrices), clusters of 8, 256 threads.
+// ------------------------------------------------------------------------------------------
+constexpr int CC_CL = 8;
+__global__ void __cluster_dims__(CC_CL, 1, 1) __launch_bounds__(256)
+    chol_cluster_kernel(double* G, int k, long long gld, long long sG, uint32_t* status) {
+  namespace cg = cooperative_groups;
+  cg::cluster_group cluster = cg::this_cluster();
+  const int q = (int)cluster.block_rank(), u = blockIdx.x / CC_CL, tid = threadIdx.x;
+  const int lane = tid & 31, warp = tid >> 5;
+  __shared__ double Ls[CF_NB][CF_P];    // L_JJ, then (rows) a panel block / L_IJ
+  __shared__ double Wi[CF_NB][CF_P];    // inv(L_JJ)
+  __shared__ double Bs[CF_NB][CF_P];    // L_KJ
+  __shared__ int bad;
+  double* Gu = G + (long long)u * sG;
+  const int nbk = (k + CF_NB - 1) / CF_NB;
+  auto at = [&](int r, int c) -> double& { return Gu[(long long)c * gld + r]; };   // column-major
+  if (tid == 0) bad = 0;
+  __syncthreads();
+  for (int J = 0; J < nbk; ++J) {
+    const int J0 = J * CF_NB, nbJ = min(CF_NB, k - J0);
+    __syncthreads();   // this CTA's updates of block column J are done
+    if (J % CC_CL == q) {
+      for (int idx = tid; idx < CF_NB * CF_NB; idx += blockDim.x) {
+        const int r = idx % CF_NB, c = idx / CF_NB;
+        Ls[r][c] = (r < nbJ && c < nbJ) ? at(J0 + r, J0 + c) : (r == c ? 1.0 : 0.0);
+      }
+      __syncthreads();
+      if (warp == 0) {
+        // factor: lane r holds row r
+        for (int c = 0; c < CF_NB; ++c) {
+          double d = Ls[c][c];
+          if (!(d > 0.0) || !isfinite(d)) {
+            if (lane == 0 && c < nbJ) bad = 1;
+            d = 1.0;
+          }
+          d = sqrt(d);
+          __syncwarp();
+          if (lane == c) Ls[c][c] = d;
+          if (lane > c) Ls[lane][c] /= d;
+          __syncwarp();
+          if (lane > c)
+            for (int s = c + 1; s <= lane; ++s) Ls[lane][s] -= Ls[lane][c] * Ls[s][c];
+          __syncwarp();
+        }
+        // inverse: lane c solves L x = e_c
+        double x[CF_NB];
+#pragma unroll
+        for (int r = 0; r < CF_NB; ++r) {
+          double v = (r == lane) ? 1.0 : 0.0;
+#pragma unroll
+          for (int p = 0; p < r; ++p) v = fma(-Ls[r][p], x[p], v);
+          x[r] = v / Ls[r][r];
+        }
+#pragma unroll
+        for (int r = 0; r < CF_NB; ++r) Wi[r][lane] = r >= lane ? x[r] : 0.0;
+      }
+      __syncthreads();
+      // the diagonal block's inverse into the upper part (W[r][c] at (row c, column r)); rows
+      // of L below it follow as the panel
+      for (int idx = tid; idx < CF_NB * CF_NB; idx += blockDim.x) {
+        const int r = idx / CF_NB, c = idx % CF_NB;
+        if (r < nbJ && c <= r) at(J0 + c, J0 + r) = Wi[r][c];
+      }
+      for (int I = J + 1; I < nbk; ++I) {
+        const int I0 = I * CF_NB, nbI = min(CF_NB, k - I0);
+        __syncthreads();
+        for (int idx = tid; idx < CF_NB * CF_NB; idx += blockDim.x) {
+          const int r = idx % CF_NB, c = idx / CF_NB;
+          Ls[r][c] = (r < nbI && c < nbJ) ? at(I0 + r, J0 + c) : 0.0;
+        }
+        __syncthreads();
+        // L_IJ[r][c] = sum_s A_IJ[r][s] inv(L_JJ)[c][s]
+        const int r = tid >> 3, cg0 = tid & 7;
+        double o[4];
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+          const int c = cg0 + 8 * jj;
+          double acc = 0.0;
+          for (int s2 = 0; s2 <= c; ++s2) acc = fma(Ls[r][s2], Wi[c][s2], acc);
+          o[jj] = acc;
+        }
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+          const int c = cg0 + 8 * jj;
+          if (r < nbI && c < nbJ) at(I0 + r, J0 + c) = o[jj];
+        }
+      }
+    }
+    __threadfence();
+    cluster.sync();   // the panel of block column J is in global memory
+    // trailing update of my block columns K > J
+    for (int K = J + 1; K < nbk; ++K) {
+      if (K % CC_CL != q) continue;
+      const int K0 = K * CF_NB, nbK = min(CF_NB, k - K0);
+      __syncthreads();
+      for (int idx = tid; idx < CF_NB * CF_NB; idx += blockDim.x) {
+        const int r = idx % CF_NB, c = idx / CF_NB;
+        Bs[r][c] = (r < nbK && c < nbJ) ? at(K0 + r, J0 + c) : 0.0;
+      }
+      for (int I = K; I < nbk; ++I) {
+        const int I0 = I * CF_NB, nbI = min(CF_NB, k - I0);
+        __syncthreads();
+        for (int idx = tid; idx < CF_NB * CF_NB; idx += blockDim.x) {
+          const int r = idx % CF_NB, c = idx / CF_NB;
+          Ls[r][c] = (r < nbI && c < nbJ) ? at(I0 + r, J0 + c) : 0.0;
+        }
+        __syncthreads();
+        const int r = tid & 31, cg0 = tid >> 5;   // row r, columns cg0 + 8 jj (coalesced writes)
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+          const int c = cg0 + 8 * jj;
+          double acc = 0.0;
+#pragma unroll 8
+          for (int s2 = 0; s2 < CF_NB; ++s2) acc = fma(Ls[r][s2], Bs[c][s2], acc);
+          if (r < nbI && c < nbK) at(I0 + r, K0 + c) -= acc;
+        }
+      }
+    }
+  }
+  __syncthreads();
+  if (tid == 0 && bad) raise_status(status, DEV_ERR_FACTOR);
+}
 }  // namespace jolt

@@ -15,6 +15,7 @@
 #include "misc.cuh"
 #include "umma.cuh"
 #include "eig_cluster.cuh"
+#include "eig_large.cuh"
 #include "chol.cuh"
 #include "table_tc.cuh"
 #include "attend.cuh"
@@ -181,7 +182,7 @@ struct Plan {
       o_feigvec, o_feigscr;
   int eig_n;              // order of the token-side eigen problems solved by the own solver (0: none)
   // token factor scratch (all units)
-  size_t o_gt32, o_gt, o_vsel, o_lam, o_omega, o_Y, o_Zm, o_h, o_l, o_gpart, o_G, o_ptrs, o_Lr, o_Linv;
+  size_t o_gt32, o_gt, o_vsel, o_lam, o_omega, o_Y, o_Zm, o_h, o_l, o_gpart, o_G, o_Lr;
   size_t o_wth, o_wtl, o_winv, o_vh, o_vl;   // tensor-core Cholesky QR: W^T = L^-T split, fp64 scratch; V split
   int qr_split_max;       // split-K of the Cholesky-QR Grams
   size_t ws_total;
@@ -353,7 +354,7 @@ jolt_status make_plan(const jolt_shape* sh, const jolt_options* op, Plan* p) {
   p->o_fevals = b.take((size_t)NU * D * 8 + 256);
   // token factor scratch
   p->o_gt32 = p->o_gt = p->o_vsel = p->o_lam = p->o_omega = 0;
-  p->o_Y = p->o_Zm = p->o_h = p->o_l = p->o_gpart = p->o_G = p->o_ptrs = p->o_eigvec = p->o_eigscr = 0;
+  p->o_Y = p->o_Zm = p->o_h = p->o_l = p->o_gpart = p->o_G = p->o_eigvec = p->o_eigscr = 0;
   const int kq = op->method == JOLT_RANDOMIZED ? p->kp : p->ldU;   // width of the QR'ed blocks
   if (op->method == JOLT_EXACT) {
     long long n = p->m_side ? M : T;
@@ -381,21 +382,21 @@ jolt_status make_plan(const jolt_shape* sh, const jolt_options* op, Plan* p) {
   p->o_feigvec = b.take((size_t)NU * D * D * 8);
   p->o_feigscr = b.take((size_t)NU * eigc::scratch_doubles(D) * 8);
   {
+    // order <= 256: the cluster solver in shared memory; <= 1024: the global-memory solver
     const long long ntok = op->method == JOLT_EXACT ? (p->m_side ? M : T) : p->k;
-    p->eig_n = (ntok >= 2 && ntok <= eigc::MAXN) ? (int)ntok : 0;
+    p->eig_n = (ntok >= 2 && ntok <= eigl::MAXN) ? (int)ntok : 0;
     if (p->eig_n) {
+      const size_t scr = ntok <= eigc::MAXN ? eigc::scratch_doubles((int)ntok) : eigl::scratch_doubles((int)ntok);
       p->o_eigvec = b.take((size_t)NU * ntok * ntok * 8);
-      p->o_eigscr = b.take((size_t)NU * eigc::scratch_doubles((int)ntok) * 8);
+      p->o_eigscr = b.take((size_t)NU * scr * 8);
     }
   }
-  p->o_Lr = p->o_Linv = p->o_wth = p->o_wtl = p->o_winv = p->o_vh = p->o_vl = 0;
+  p->o_Lr = p->o_wth = p->o_wtl = p->o_winv = p->o_vh = p->o_vl = 0;
   if (op->method == JOLT_RANDOMIZED || p->m_side) {
     p->o_gpart = b.take((size_t)NU * p->qr_split_max * kq * kq * 4);
     p->o_G = b.take((size_t)NU * kq * kq * 8);
     // L as fp32 row-major, or (k <= 256) the transposed inverse of L at the padded width
     p->o_Lr = b.take((size_t)NU * round_up(kq, 32) * round_up(kq, 32) * 4);
-    p->o_ptrs = b.take((size_t)NU * 8 + 64);
-    p->o_Linv = b.take((size_t)NU * round_up(kq, 32) * 32 * 4);   // inverses of the 32 x 32 diagonal blocks
     if (kq >= QR_TC_MINK) {
       const size_t kq32 = round_up(kq, 32);
       p->o_wth = b.take((size_t)NU * kq32 * kq32 * 2);
@@ -547,6 +548,34 @@ jolt_status sym_eig_top(const Ctx& c, double* S, int n, int nbatch, int r, float
                         long long ldo, long long sout, double* out_vals) {
   double* w = c.at<double>(c.side ? c.p.o_fevals : c.p.o_evals);
   const bool own = c.side ? (n == c.p.D && n >= 2 && n <= eigc::MAXN) : (c.p.eig_n != 0 && n == c.p.eig_n);
+  if (own && n > eigc::MAXN) {
+    // the global-memory solver (csrc/eig_large.cuh)
+    ProfScope ps("sym_eig", c.st, nbatch);
+    double* V = c.at<double>(c.p.o_eigvec);
+    double* scr = c.at<double>(c.p.o_eigscr);
+    count_launch(), sanitize_sym_batched_kernel<<<(unsigned)nbatch, 1024, 0, c.st>>>(S, n, n, (long long)n * n,
+                                                                                      c.status());
+    count_launch(), symmetrize_lower_kernel<<<dim3(64, (unsigned)nbatch), 256, 0, c.st>>>(S, n, (long long)n * n);
+    CUDA_TRY(cudaGetLastError());
+    CUDA_TRY(cudaFuncSetAttribute(tridiag_gm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)eigl::TRI_SMEM));
+    count_launch(), tridiag_gm_kernel<<<(unsigned)(nbatch * eigl::CL), eigl::THREADS, eigl::TRI_SMEM, c.st>>>(
+        S, n, (long long)n * n, scr);
+    CUDA_TRY(cudaGetLastError());
+    count_launch(), tri_eig_kernel<<<dim3((unsigned)ceil_div(n, eigl::EV_PER_CTA), (unsigned)nbatch), eigl::THREADS, 0,
+                                     c.st>>>(n, w, n, V, scr);
+    CUDA_TRY(cudaGetLastError());
+    count_launch(), tight_mgs_kernel<<<(unsigned)nbatch, 32, 0, c.st>>>(n, w, n, V);
+    CUDA_TRY(cudaGetLastError());
+    const size_t bsm = backtransform_smem(n);
+    CUDA_TRY(cudaFuncSetAttribute(backtransform_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bsm));
+    count_launch(), backtransform_kernel<<<dim3((unsigned)ceil_div(n, eigl::BT_COLS), (unsigned)nbatch), eigl::THREADS,
+                                           bsm, c.st>>>(n, V, scr);
+    CUDA_TRY(cudaGetLastError());
+    count_launch(), eig_select_kernel<<<dim3(r, nbatch), 256, 0, c.st>>>(w, V, n, 1, n, n, (long long)n * n, r,
+                                                                         out_f32, out_bf16, ldo, sout, out_vals);
+    CUDA_TRY(cudaGetLastError());
+    return JOLT_OK;
+  }
   if (own) {
     // one 8-CTA cluster per matrix (csrc/eig_cluster.cuh)
     ProfScope ps(c.side ? "feature_eig" : "sym_eig", c.st, nbatch);
@@ -577,16 +606,6 @@ jolt_status sym_eig_top(const Ctx& c, double* S, int n, int nbatch, int r, float
 // place: G = Y^T Y (fp32 partial sums of <= 256 terms, added in fp64), G = L L^T (cuSOLVER's
 // batched Cholesky, fp64), Q = Y L^{-T} (blocked row-panel solve).  `passes` = 2 gives
 // CholeskyQR2.
-template <int RB>
-jolt_status launch_trsm_panel(const Ctx& c, float* Y, long long m, int k, int ld, const float* Lr, long long ldl,
-                              long long sL, const float* Dinv, long long sD) {
-  const size_t sm = trsm_smem(RB, k);
-  CUDA_TRY(cudaFuncSetAttribute(trsm_panel_kernel<RB>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm));
-  count_launch(), trsm_panel_kernel<RB><<<dim3((unsigned)ceil_div(m, RB), c.p.NU), 256, sm, c.st>>>(
-      Y, m, k, ld, m * ld, Lr, ldl, sL, Dinv, sD);
-  CUDA_TRY(cudaGetLastError());
-  return JOLT_OK;
-}
 
 jolt_status cholqr_tc(const Ctx& c, float* Y, long long m, int k, int ld, int passes);
 
@@ -596,13 +615,10 @@ jolt_status cholqr_batched(const Ctx& c, float* Y, long long m, int k, int ld, i
     if (ld % 8) return fail(JOLT_ERR_INVALID_ARG, "token factor pitch %d not a multiple of 8", ld);
     return cholqr_tc(c, Y, m, k, ld, passes);
   }
+  // block widths below the tensor-core width (k < 64): fp32 Gram, own factor and inverse product
   ProfScope ps("cholesky_qr", c.st, p.NU);
-  Solver* s = nullptr;
-  JTRY(solver_get(c.st, &s));
   float* gpart = c.at<float>(p.o_gpart);
   double* G = c.at<double>(p.o_G);
-  double** ptrs = c.at<double*>(p.o_ptrs);
-  int* info = c.at<int>(p.o_info);
   // split-K chunk: 256 rows, halved (down to 64) while fewer than two CTAs per SM would run
   // and the partial buffer (qr_split_max splits) still holds the splits
   int kchunk = 256;
@@ -642,9 +658,7 @@ jolt_status cholqr_batched(const Ctx& c, float* Y, long long m, int k, int ld, i
         gpart, G, p.NU, ns, k, gld, sgemm_detail::BM);
     }
     float* Lr = c.at<float>(p.o_Lr);
-    float* Dinv = c.at<float>(p.o_Linv);
-    const int nbk = (int)ceil_div(k, TS_NB);
-    const long long sL = (long long)k * gld, sD = (long long)nbk * TS_NB * TS_NB;
+    const int nbk = (int)ceil_div(k, CF_NB);
     if (k <= CF_MAXK && ld % 4 == 0) {
       // own factor, block-column inverse and inverse product (chol.cuh; 16-byte row loads)
       const int kq32 = (int)round_up(k, 32);
@@ -670,21 +684,7 @@ jolt_status cholqr_batched(const Ctx& c, float* Y, long long m, int k, int ld, i
       CUDA_TRY(cudaGetLastError());
       continue;
     }
-    {
-      count_launch(), sanitize_sym_batched_kernel<<<p.NU, 1024, 0, c.st>>>(G, k, gld, n, c.status());
-      count_launch(), ptr_array_kernel<<<1, 64, 0, c.st>>>(ptrs, G, n, p.NU);
-      CUDA_TRY(cudaGetLastError());
-      ProfScope ps2("qr_potrf", c.st, p.NU);
-      SOLVER_TRY(cusolverDnDpotrfBatched(s->h, CUBLAS_FILL_MODE_LOWER, k, ptrs, gld, info, p.NU));
-      count_launch(), info_check_kernel<<<(unsigned)ceil_div(p.NU, 32), 32, 0, c.st>>>(info, p.NU, c.status(),
-                                                                                        DEV_ERR_FACTOR);
-      count_launch(), trsm_prep_kernel<<<dim3(nbk, p.NU), 32, 0, c.st>>>(G, k, gld, n, Lr, gld, sL, Dinv, sD);
-      CUDA_TRY(cudaGetLastError());
-    }
-    ProfScope ps3("qr_trsm", c.st, p.NU);
-    // rows per CTA: 64 (two CTAs per SM), 32 for wide blocks
-    if (k <= 512) JTRY(launch_trsm_panel<64>(c, Y, m, k, ld, Lr, gld, sL, Dinv, sD));
-    else JTRY(launch_trsm_panel<32>(c, Y, m, k, ld, Lr, gld, sL, Dinv, sD));
+    return fail(JOLT_ERR_UNSUPPORTED_SHAPE, "Cholesky QR of %d columns below the tensor-core width", k);
   }
   return JOLT_OK;
 }
@@ -762,8 +762,6 @@ jolt_status cholqr_tc(const Ctx& c, float* Y, long long m, int k, int ld, int pa
   float* WT = c.at<float>(p.o_Lr);
   bf16* wth = c.at<bf16>(p.o_wth);
   bf16* wtl = c.at<bf16>(p.o_wtl);
-  double** ptrs = c.at<double*>(p.o_ptrs);
-  int* info = c.at<int>(p.o_info);
   const int gld = ld, kq32 = (int)round_up(k, 32), nbk = (int)ceil_div(k, 32);
   const long long sG = (long long)k * gld, sW = (long long)kq32 * kq32;
   const int ns = (int)ceil_div(m, QR_TC_CHUNK);
@@ -822,15 +820,10 @@ jolt_status cholqr_tc(const Ctx& c, float* Y, long long m, int k, int ld, int pa
                                                                                                sW);
         CUDA_TRY(cudaGetLastError());
       } else {
-        Solver* s = nullptr;
-        JTRY(solver_get(c.st, &s));
+        // 256 < k <= 1024: the cluster Cholesky (chol.cuh), then the block-column inverse
         count_launch(), sanitize_sym_batched_kernel<<<p.NU, 1024, 0, c.st>>>(G, k, gld, sG, c.status());
-        count_launch(), ptr_array_kernel<<<1, 64, 0, c.st>>>(ptrs, G, sG, p.NU);
+        count_launch(), chol_cluster_kernel<<<(unsigned)(p.NU * CC_CL), 256, 0, c.st>>>(G, k, gld, sG, c.status());
         CUDA_TRY(cudaGetLastError());
-        SOLVER_TRY(cusolverDnDpotrfBatched(s->h, CUBLAS_FILL_MODE_LOWER, k, ptrs, gld, info, p.NU));
-        count_launch(), info_check_kernel<<<(unsigned)ceil_div(p.NU, 32), 32, 0, c.st>>>(info, p.NU, c.status(),
-                                                                                          DEV_ERR_FACTOR);
-        count_launch(), diag_inv64_kernel<<<dim3(nbk, p.NU), 32, 0, c.st>>>(G, k, gld, sG);
         count_launch(), tri_inv_large_kernel<<<dim3(nbk, p.NU), CF_THREADS, 0, c.st>>>(
             G, k, gld, sG, c.at<double>(p.o_winv), kq32, WT, kq32, sW);
         CUDA_TRY(cudaGetLastError());
@@ -1331,30 +1324,6 @@ jolt_status run_core(const Ctx& c, const bf16* Us, long long ldU, const bf16* Ws
   return JOLT_OK;
 }
 
-template <int D>
-void launch_rotate_rows(const float* in, bf16* out, long long nrows, long long rows_per_unit, const int* umap,
-                        uint64_t seed, cudaStream_t st) {
-  if constexpr (D >= 32) {
-    const long long blocks = ceil_div(nrows, 8) < 148 * 16 ? ceil_div(nrows, 8) : 148 * 16;   // 8 warps per block
-    count_launch(), rotate_rows_warp_kernel<D><<<(unsigned)blocks, 256, 0, st>>>(in, out, nrows, rows_per_unit, umap,
-                                                                               seed);
-  } else {
-    count_launch(), rotate_rows_kernel<D><<<(unsigned)ceil_div(nrows, 64), 64, 0, st>>>(in, out, nrows, rows_per_unit,
-                                                                                      umap, seed);
-  }
-}
-
-jolt_status rotate_rows(const Ctx& c, const float* in, bf16* out, long long nrows, long long rows_per_unit,
-                        const int* umap) {
-  switch (c.p.D) {
-    case 16: launch_rotate_rows<16>(in, out, nrows, rows_per_unit, umap, c.seed, c.st); break;
-    case 32: launch_rotate_rows<32>(in, out, nrows, rows_per_unit, umap, c.seed, c.st); break;
-    case 64: launch_rotate_rows<64>(in, out, nrows, rows_per_unit, umap, c.seed, c.st); break;
-    default: launch_rotate_rows<128>(in, out, nrows, rows_per_unit, umap, c.seed, c.st); break;
-  }
-  CUDA_TRY(cudaGetLastError());
-  return JOLT_OK;
-}
 
 // P'(r_D) for one unit: bf16(rotate(C_s[:, :rT, :r_D] W_s[:, :r_D]^T)), rows rT of every slice
 // out layout [S][rTslice][D] (rows >= rT of a slice are not written meaningfully)

@@ -860,19 +860,24 @@ __global__ void __launch_bounds__(256) quant_baseline_kernel(CacheView cv, int b
     const float lo = rd16(mn);
     const float step = quant_step(mx, lo, flev, inv_lev);
     const bool ok = isfinite(lo) && step <= kFp16Max;
-    const float inv = (ok && step > 0.f) ? __frcp_rn(step) : 0.f;
+    // codes and errors in fp64: v - lo, its quotient by the step and the rounding to the
+    // nearest level (ties to even) are then those of the definition; the inputs of this
+    // baseline are coarse (bf16 values, fp16 scales), so exact ties are common and a product
+    // with a rounded reciprocal would settle them differently.  The kernel stays HBM-bound.
     uint32_t w[4] = {0u, 0u, 0u, 0u};
-    float ex = 0.f, ee = 0.f;
+    double ex = 0.0, ee = 0.0;
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
-      const uint32_t c = ok ? block_code(v[i], lo, inv, flev) : 0u;
-      pack_code(w, i, b, c);
-      const float e = v[i] - fmaf((float)c, step, lo);
-      ex = fmaf(v[i], v[i], ex);
-      ee = fmaf(e, e, ee);
+      const double d = (double)v[i] - (double)lo;
+      double c = (ok && step > 0.f) ? rint(d / (double)step) : 0.0;
+      c = fmin(fmax(c, 0.0), (double)flev);
+      pack_code(w, i, b, (uint32_t)c);
+      const double e = (double)v[i] - fma(c, (double)step, (double)lo);
+      ex = fma((double)v[i], (double)v[i], ex);
+      ee = fma(e, e, ee);
     }
-    sx += (double)ex;
-    se += ok ? (double)ee : (double)INFINITY;
+    sx += ex;
+    se += ok ? ee : (double)INFINITY;
     if (codes) {
       unsigned char* dst = codes + ((long long)u * nb + q) * (2 * b);
       for (int byte = 0; byte < 2 * b; ++byte) dst[byte] = (unsigned char)(w[byte >> 2] >> ((byte & 3) * 8));

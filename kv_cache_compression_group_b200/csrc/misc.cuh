@@ -185,83 +185,6 @@ __global__ void split_bf16_cols_kernel(const float* x, bf16* hi, bf16* lo, long 
   }
 }
 
-// rows of fp32 [nrows][D] -> bf16(FWHT(sigma * row) / sqrt(D)) ; sigma of unit (row / rows_per_unit)
-template <int D>
-__global__ void rotate_rows_kernel(const float* in, bf16* out, long long nrows, long long rows_per_unit,
-                                   const int* unit_of_batch, uint64_t seed) {
-  long long r = blockIdx.x * (long long)blockDim.x + threadIdx.x;
-  if (r >= nrows) return;
-  int u = unit_of_batch[r / rows_per_unit];
-  float v[D];
-  const float* row = in + r * D;
-#pragma unroll
-  for (int d = 0; d < D; ++d) v[d] = row[d] * rotation_sign(seed, u, d);
-  fwht_regs<D>(v);
-  const float sc = (float)(1.0 / sqrt((double)D));
-  bf16* o = out + r * D;
-#pragma unroll
-  for (int d = 0; d < D; ++d) o[d] = __float2bfloat16_rn(v[d] * sc);
-}
-
-// The same rotation with one warp per row (D >= 32): lane l holds the E = D/32 consecutive
-// elements [l E, l E + E), so loads and stores are coalesced; the Walsh-Hadamard stages of
-// stride < E run inside the thread, the others across lanes (shfl_xor); each output is the
-// same sum or difference of the same two values as in fwht_regs, so the result is bitwise
-// the same.  The signs of a unit are recomputed only when a warp's row changes unit.
-template <int D>
-__global__ void rotate_rows_warp_kernel(const float* in, bf16* out, long long nrows, long long rows_per_unit,
-                                        const int* unit_of_batch, uint64_t seed) {
-  constexpr int E = D / 32;
-  const int lane = threadIdx.x & 31;
-  const long long warp0 = (blockIdx.x * (long long)blockDim.x + threadIdx.x) >> 5;
-  const long long nwarps = ((long long)gridDim.x * blockDim.x) >> 5;
-  const float sc = (float)(1.0 / sqrt((double)D));
-  int ucur = -1;
-  float sg[E];
-  for (long long r = warp0; r < nrows; r += nwarps) {
-    const int u = unit_of_batch[r / rows_per_unit];
-    if (u != ucur) {
-#pragma unroll
-      for (int e = 0; e < E; ++e) sg[e] = rotation_sign(seed, u, lane * E + e);
-      ucur = u;
-    }
-    float v[E];
-    const float* row = in + r * D + lane * E;
-    if (E == 4) {
-      const float4 t = *reinterpret_cast<const float4*>(row);
-      v[0] = t.x;
-      v[E > 1 ? 1 : 0] = t.y;
-      v[E > 2 ? 2 : 0] = t.z;
-      v[E > 3 ? 3 : 0] = t.w;
-    } else {
-#pragma unroll
-      for (int e = 0; e < E; ++e) v[e] = row[e];
-    }
-#pragma unroll
-    for (int e = 0; e < E; ++e) v[e] *= sg[e];
-#pragma unroll
-    for (int h = 1; h < E; h <<= 1)
-#pragma unroll
-      for (int e = 0; e < E; ++e)
-        if (!(e & h)) {
-          const float a = v[e], b = v[e + h];
-          v[e] = a + b;
-          v[e + h] = a - b;
-        }
-#pragma unroll
-    for (int hl = 1; hl < 32; hl <<= 1) {
-      const bool upper = (lane & hl) != 0;
-#pragma unroll
-      for (int e = 0; e < E; ++e) {
-        const float mine = v[e], other = __shfl_xor_sync(0xffffffffu, mine, hl);
-        v[e] = upper ? other - mine : mine + other;
-      }
-    }
-    bf16* o = out + r * D + lane * E;
-#pragma unroll
-    for (int e = 0; e < E; ++e) o[e] = __float2bfloat16_rn(v[e] * sc);
-  }
-}
 
 // zero the strict upper triangle of column-major n x n matrices (lda)
 __global__ void tril_zero_kernel(double* A, int n, long long lda, long long sA, int nbatch) {
@@ -311,147 +234,6 @@ __global__ void sanitize_sym_batched_kernel(double* A, int n, long long lda, lon
   for (long long i = threadIdx.x; i < (long long)n * n; i += blockDim.x) {
     long long r = i / n, c = i - r * n;
     M[c * lda + r] = (r == c) ? 1.0 : 0.0;
-  }
-}
-
-// device pointer array for the batched Cholesky: P[u] = A + u * sA
-__global__ void ptr_array_kernel(double** P, double* A, long long sA, int n) {
-  int u = blockIdx.x * blockDim.x + threadIdx.x;
-  if (u < n) P[u] = A + (long long)u * sA;
-}
-
-// ------------------------------------------------------------------------------------------
-// Q = Y L^{-T} in place (the triangular solve of Cholesky QR), blocked by 32 columns:
-//   Q[:, J] = (Y[:, J] - Q[:, :J] L[J, :J]^T) inv(L[J, J])^T
-// trsm_prep_kernel: per (block J, unit) one warp writes rows J of L as fp32 row-major (zeros
-//   above the diagonal) and inv(L_JJ) (fp64 forward substitution, rounded to fp32);
-// trsm_panel_kernel<RB>: one CTA per RB rows of one unit keeps its rows of Y in shared memory
-//   and solves them block column by block column (GEMM update from staged chunks of L, then
-//   the product with inv(L_JJ)^T), then writes the k solved columns back.
-// ------------------------------------------------------------------------------------------
-constexpr int TS_NB = 32;
-constexpr int TS_PC = 128;
-
-__global__ void trsm_prep_kernel(const double* L, int k, long long gld, long long sG, float* Lr, long long ldl,
-                                 long long sL, float* Dinv, long long sD) {
-  const int J = blockIdx.x, u = blockIdx.y, lane = threadIdx.x;
-  const int J0 = J * TS_NB, nb = min(TS_NB, k - J0);
-  const double* Lu = L + (long long)u * sG;   // column-major: (i, j) at Lu[j * gld + i]
-  float* Lru = Lr + (long long)u * sL;
-  for (int r = 0; r < nb; ++r) {
-    const int i = J0 + r;
-    for (int c = lane; c < k; c += 32) Lru[(long long)i * ldl + c] = c <= i ? (float)Lu[(long long)c * gld + i] : 0.f;
-  }
-  double x[TS_NB];
-#pragma unroll
-  for (int r = 0; r < TS_NB; ++r) {
-    double v = (r == lane) ? 1.0 : 0.0;
-    if (r < nb && lane < nb) {
-#pragma unroll
-      for (int q = 0; q < r; ++q) v = fma(-Lu[(long long)(J0 + q) * gld + J0 + r], x[q], v);
-      x[r] = lane <= r ? v / Lu[(long long)(J0 + r) * gld + J0 + r] : 0.0;
-    } else {
-      x[r] = 0.0;
-    }
-  }
-  float* D = Dinv + (long long)u * sD + (long long)J * TS_NB * TS_NB;
-#pragma unroll
-  for (int r = 0; r < TS_NB; ++r) D[r * TS_NB + lane] = (float)x[r];
-}
-
-// row pitches: multiples of 4 floats (16-byte vector loads) that are 4 mod 32, so the rows a
-// warp reads together fall on distinct banks
-__host__ __device__ inline int trsm_pitch(int k) { return (int)round_up(k, TS_NB) + 4; }
-constexpr int TS_LP = TS_PC + 4;
-inline size_t trsm_smem(int rb, int k) {
-  return ((size_t)rb * trsm_pitch(k) + (size_t)TS_NB * TS_LP + (size_t)TS_NB * (TS_NB + 1)) * sizeof(float);
-}
-
-template <int RB>
-__global__ void __launch_bounds__(256) trsm_panel_kernel(float* Y, long long m, int k, long long ld, long long sY,
-                                                         const float* Lr, long long ldl, long long sL,
-                                                         const float* Dinv, long long sD) {
-  extern __shared__ __align__(16) float ts_sm[];
-  const int P = trsm_pitch(k), kq = P - 4;
-  float* panel = ts_sm;                        // RB x P
-  float* lch = panel + RB * P;                 // 32 x TS_LP
-  float* dv = lch + TS_NB * TS_LP;             // 32 x 33
-  const int u = blockIdx.y, tid = threadIdx.x;
-  const long long r0 = (long long)blockIdx.x * RB;
-  float* Yu = Y + (long long)u * sY;
-  const float* Lu = Lr + (long long)u * sL;
-  const float* Du = Dinv + (long long)u * sD;
-  for (int idx = tid; idx < RB * kq; idx += blockDim.x) {
-    const int r = idx / kq, c = idx - r * kq;
-    panel[r * P + c] = (r0 + r < m && c < k) ? Yu[(r0 + r) * ld + c] : 0.f;
-  }
-  __syncthreads();
-  constexpr int RI = RB / 32;
-  const int ty = tid >> 3, tx = tid & 7;
-  for (int J0 = 0; J0 < k; J0 += TS_NB) {
-    float acc[RI][4];
-#pragma unroll
-    for (int i = 0; i < RI; ++i)
-#pragma unroll
-      for (int j = 0; j < 4; ++j) acc[i][j] = panel[(ty + 32 * i) * P + J0 + tx + 8 * j];
-    for (int p0 = 0; p0 < J0; p0 += TS_PC) {
-      const int pc = min(TS_PC, J0 - p0);
-      __syncthreads();
-      for (int idx = tid; idx < TS_NB * TS_PC; idx += blockDim.x) {
-        const int rr = idx / TS_PC, cc = idx - rr * TS_PC;
-        lch[rr * TS_LP + cc] = (cc < pc && J0 + rr < k) ? Lu[(long long)(J0 + rr) * ldl + p0 + cc] : 0.f;
-      }
-      __syncthreads();
-      // pc is a multiple of 4 (block columns of 32, chunks of 128): four p per vector load
-      for (int p = 0; p < pc; p += 4) {
-        float4 q[RI], l[4];
-#pragma unroll
-        for (int i = 0; i < RI; ++i) q[i] = *reinterpret_cast<const float4*>(panel + (ty + 32 * i) * P + p0 + p);
-#pragma unroll
-        for (int j = 0; j < 4; ++j) l[j] = *reinterpret_cast<const float4*>(lch + (tx + 8 * j) * TS_LP + p);
-#pragma unroll
-        for (int i = 0; i < RI; ++i)
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            float a = acc[i][j];
-            a = fmaf(-q[i].x, l[j].x, a);
-            a = fmaf(-q[i].y, l[j].y, a);
-            a = fmaf(-q[i].z, l[j].z, a);
-            a = fmaf(-q[i].w, l[j].w, a);
-            acc[i][j] = a;
-          }
-      }
-    }
-    __syncthreads();
-#pragma unroll
-    for (int i = 0; i < RI; ++i)
-#pragma unroll
-      for (int j = 0; j < 4; ++j) panel[(ty + 32 * i) * P + J0 + tx + 8 * j] = acc[i][j];
-    for (int idx = tid; idx < TS_NB * TS_NB; idx += blockDim.x)
-      dv[(idx / TS_NB) * (TS_NB + 1) + (idx % TS_NB)] = Du[(long long)(J0 / TS_NB) * TS_NB * TS_NB + idx];
-    __syncthreads();
-    float out[RI][4];
-#pragma unroll
-    for (int i = 0; i < RI; ++i)
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const float* row = panel + (ty + 32 * i) * P + J0;
-        const float* dr = dv + (tx + 8 * j) * (TS_NB + 1);
-        float s = 0.f;
-#pragma unroll
-        for (int q = 0; q < TS_NB; ++q) s = fmaf(row[q], dr[q], s);
-        out[i][j] = s;
-      }
-    __syncthreads();
-#pragma unroll
-    for (int i = 0; i < RI; ++i)
-#pragma unroll
-      for (int j = 0; j < 4; ++j) panel[(ty + 32 * i) * P + J0 + tx + 8 * j] = out[i][j];
-    __syncthreads();
-  }
-  for (int idx = tid; idx < RB * kq; idx += blockDim.x) {
-    const int r = idx / kq, c = idx - r * kq;
-    if (r0 + r < m && c < k) Yu[(r0 + r) * ld + c] = panel[r * P + c];
   }
 }
 
