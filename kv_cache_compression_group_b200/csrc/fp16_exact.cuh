@@ -95,6 +95,28 @@ __host__ __device__ __forceinline__ float quant_step(float mx, float lo, float f
   return s;
 }
 
+// The same step as quant_step, decided without data-dependent branches where the float
+// comparisons are conclusive (the common case): the fp16 round-up of (max - lo) / levels in
+// the normal fp16 range by bit operations, then the one-step corrections of quant_step chosen
+// by selects.  Where a comparison is inconclusive, or the value leaves the range where the
+// neighbouring fp16 numbers are one bit step away, it calls quant_step itself; so the result
+// is quant_step's in every case.
+__host__ __device__ __forceinline__ float quant_step_sel(float mx, float lo, float flev, float inv_lev) {
+  const float R = mx - lo;
+  const float q = R * inv_lev;
+  const bool inside = (mx > lo) && q >= 2.0f * kFp16MinNormal && q <= 16384.f;
+  uint32_t u = f32_bits(q);
+  u = (u & 0x1FFFu) ? ((u | 0x1FFFu) + 1u) : u;
+  const float s = bits_f32(u), sp = bits_f32(u - 0x2000u), su = bits_f32(u + 0x2000u);
+  const float a = s * flev, ap = sp * flev;
+  const float Rhi = R * 1.0000002384185791f, Rlo = R * 0.9999997615814209f;
+  const bool a_ge = a > Rhi, a_lt = a < Rlo;
+  const bool ap_ge = ap > Rhi, ap_lt = ap < Rlo;
+  const bool sure = inside && (a_lt || (a_ge && (ap_ge || ap_lt)));
+  if (!sure) return quant_step(mx, lo, flev, inv_lev);
+  return a_lt ? su : (ap_ge ? sp : s);
+}
+
 // ---------------------------------------------------------------------------------------
 // codes of the b-bit block quantiser and their packing
 // ---------------------------------------------------------------------------------------

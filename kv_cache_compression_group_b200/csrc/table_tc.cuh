@@ -132,52 +132,43 @@ __device__ __forceinline__ float ttc_rcp_approx(float x) {
   return r;
 }
 
+// squared-error sums of one bit-width over one block, added into two packed partial sums
+// (a[0], a[1]) that run over all blocks of the thread for the current cut; a block whose
+// scale overflows fp16 makes the sums +inf
 template <int B>
-__device__ __forceinline__ void ttc_bit_error(const float2* v, const float2* d, float mx, float lo, float& err) {
+__device__ __forceinline__ void ttc_bit_error(const float2* v, const float2* d, float mx, float lo, float2* a) {
   if constexpr (B == 0) {
-    float2 a0 = make_float2(0.f, 0.f), a1 = a0, a2 = a0, a3 = a0;
 #pragma unroll
-    for (int j = 0; j < 8; j += 4) {
-      a0 = __ffma2_rn(v[j], v[j], a0);
-      a1 = __ffma2_rn(v[j + 1], v[j + 1], a1);
-      a2 = __ffma2_rn(v[j + 2], v[j + 2], a2);
-      a3 = __ffma2_rn(v[j + 3], v[j + 3], a3);
+    for (int j = 0; j < 8; j += 2) {
+      a[0] = __ffma2_rn(v[j], v[j], a[0]);
+      a[1] = __ffma2_rn(v[j + 1], v[j + 1], a[1]);
     }
-    err += ((a0.x + a0.y) + (a1.x + a1.y)) + ((a2.x + a2.y) + (a3.x + a3.y));
   } else {
     constexpr float flev = (float)((1 << B) - 1);
     const float inv_lev = 1.0f / flev;
-    const float step = quant_step(mx, lo, flev, inv_lev);
-    if (!(isfinite(lo) && step <= kFp16Max)) {
-      err = INFINITY;
-      return;
-    }
+    const float step = quant_step_sel(mx, lo, flev, inv_lev);
+    const bool ok = isfinite(lo) && step <= kFp16Max;
     const float inv = step > 0.f ? ttc_rcp_approx(step) : 0.f;
     const float2 inv2 = make_float2(inv, inv), nstep2 = make_float2(-step, -step);
     const float2 sh = make_float2(kRoundShift, kRoundShift), nsh = make_float2(-kRoundShift, -kRoundShift);
-    float2 a0 = make_float2(0.f, 0.f), a1 = a0, a2 = a0, a3 = a0;
+    float2 b0 = a[0], b1 = a[1];
 #pragma unroll
-    for (int j = 0; j < 8; j += 4) {
+    for (int j = 0; j < 8; j += 2) {
       const float2 c0 = __fadd2_rn(__ffma2_rn(d[j], inv2, sh), nsh);
       const float2 c1 = __fadd2_rn(__ffma2_rn(d[j + 1], inv2, sh), nsh);
-      const float2 c2 = __fadd2_rn(__ffma2_rn(d[j + 2], inv2, sh), nsh);
-      const float2 c3 = __fadd2_rn(__ffma2_rn(d[j + 3], inv2, sh), nsh);
       const float2 e0 = __ffma2_rn(c0, nstep2, d[j]);
       const float2 e1 = __ffma2_rn(c1, nstep2, d[j + 1]);
-      const float2 e2 = __ffma2_rn(c2, nstep2, d[j + 2]);
-      const float2 e3 = __ffma2_rn(c3, nstep2, d[j + 3]);
-      a0 = __ffma2_rn(e0, e0, a0);
-      a1 = __ffma2_rn(e1, e1, a1);
-      a2 = __ffma2_rn(e2, e2, a2);
-      a3 = __ffma2_rn(e3, e3, a3);
+      b0 = __ffma2_rn(e0, e0, b0);
+      b1 = __ffma2_rn(e1, e1, b1);
     }
-    err += ((a0.x + a0.y) + (a1.x + a1.y)) + ((a2.x + a2.y) + (a3.x + a3.y));
+    a[0] = ok ? b0 : make_float2(INFINITY, INFINITY);
+    a[1] = ok ? b1 : make_float2(INFINITY, INFINITY);
   }
 }
 
 // every bit-width of the set for one block of rho given as 8 packed pairs
 template <int... Bs>
-__device__ __forceinline__ void ttc_block_errors(const float2* v, float* err, BitSet<Bs...>) {
+__device__ __forceinline__ void ttc_block_errors(const float2* v, float2 (*acc)[2], BitSet<Bs...>) {
   const float m0 = ttc_min3(v[0].x, v[0].y, v[1].x), m1 = ttc_min3(v[1].y, v[2].x, v[2].y);
   const float m2 = ttc_min3(v[3].x, v[3].y, v[4].x), m3 = ttc_min3(v[4].y, v[5].x, v[5].y);
   const float m4 = ttc_min3(v[6].x, v[6].y, v[7].x);
@@ -192,14 +183,14 @@ __device__ __forceinline__ void ttc_block_errors(const float2* v, float* err, Bi
 #pragma unroll
   for (int j = 0; j < 8; ++j) d[j] = __fadd2_rn(v[j], nlo);
   int i = 0;
-  (ttc_bit_error<Bs>(v, d, mx, lo, err[i++]), ...);
+  (ttc_bit_error<Bs>(v, d, mx, lo, acc[i++]), ...);
 }
 
 __device__ __forceinline__ void ttc_epi_sync() { asm volatile("bar.sync 1, %0;" ::"n"(ttc::EPI_WARPS * 32) : "memory"); }
 
 // grid (tiles, S, units); ttc::THREADS threads; ttc::SMEM bytes of dynamic shared memory
 template <typename TX, typename BITS>
-__global__ void __launch_bounds__(ttc::THREADS, 1)
+__global__ void __maxnreg__(112)
     table_tc_kernel(const __grid_constant__ CUtensorMap map_u, const __grid_constant__ CUtensorMap map_p,
                     TableTcArgs a) {
   using namespace ttc;
@@ -334,6 +325,9 @@ __global__ void __launch_bounds__(ttc::THREADS, 1)
         float err[MAXC];
 #pragma unroll
         for (int b = 0; b < MAXC; ++b) err[b] = 0.f;
+        float2 acc2[MAXC][2];   // packed partial sums of the fixed bit set (horizontal sum per cut)
+#pragma unroll
+        for (int b = 0; b < MAXC; ++b) acc2[b][0] = acc2[b][1] = make_float2(0.f, 0.f);
         if (ok) {
           umma::fence_after_sync();
 #pragma unroll
@@ -362,9 +356,13 @@ __global__ void __launch_bounds__(ttc::THREADS, 1)
               if constexpr (std::is_same<BITS, void>::value) {
                 block_errors(reinterpret_cast<const float*>(v2), kb, err);
               } else {
-                ttc_block_errors(v2, err, BITS{});
+                ttc_block_errors(v2, acc2, BITS{});
               }
             }
+          }
+          if constexpr (!std::is_same<BITS, void>::value) {
+#pragma unroll
+            for (int b = 0; b < BITS::N; ++b) err[b] = (acc2[b][0].x + acc2[b][0].y) + (acc2[b][1].x + acc2[b][1].y);
           }
         }
         // this cut's sums over the warp (every lane takes part, also after an abort)
@@ -428,7 +426,7 @@ struct EncodeTcArgs {
 };
 
 template <typename TX>
-__global__ void __launch_bounds__(etc::THREADS, 1)
+__global__ void __maxnreg__(112)
     encode_tc_kernel(const __grid_constant__ CUtensorMap map_u, const __grid_constant__ CUtensorMap map_p,
                      EncodeTcArgs a) {
   using namespace ttc;

@@ -505,7 +505,9 @@ inline cudaError_t launch_umma(const UmmaMaps& m, UmmaArgs a, int nb, cudaStream
     return cudaErrorInvalidValue;
   if (a.splits == 1) a.kchunk = (int)round_up(a.K, umma::BK);
   if (a.c_accum && a.c_bf16) return cudaErrorInvalidValue;
-  if (a.bn == 256 || (a.bn == 0 && a.N > 128))
+  // N tiles of 256 only with one B operand: with two (hi + lo) a 256-wide stage takes 80 KB and
+  // leaves room for two pipeline stages, a 128-wide one 48 KB and four
+  if (a.bn == 256 || (a.bn == 0 && a.N > 128 && nb == 1))
     return nb == 2 ? launch_umma_bn<256, 2>(m, a, st) : launch_umma_bn<256, 1>(m, a, st);
   return nb == 2 ? launch_umma_bn<128, 2>(m, a, st) : launch_umma_bn<128, 1>(m, a, st);
 }

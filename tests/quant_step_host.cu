@@ -1,6 +1,7 @@
 // Host driver for the library's exact fp16 helpers (the same source the table and encode
 // kernels compile for the device): reads (block minimum, block maximum) pairs as fp32 from
-// stdin, writes lo = rd16(min) and quant_step(max, lo) for b = 1, 2, 3, 4, 8 as fp32.
+// stdin, writes lo = rd16(min), quant_step(max, lo) for b = 1, 2, 3, 4, 8 and the branch-free
+// quant_step_sel for the same b, as fp32.
 #include <cstdio>
 #include <vector>
 
@@ -15,13 +16,14 @@ int main() {
     in.push_back(v[1]);
   }
   for (size_t i = 0; i < in.size(); i += 2) {
-    float out[6];
+    float out[11];
     out[0] = jolt::rd16(in[i]);
     for (int j = 0; j < 5; ++j) {
       const float flev = (float)((1 << bits[j]) - 1);
       out[1 + j] = jolt::quant_step(in[i + 1], out[0], flev, 1.0f / flev);
+      out[6 + j] = jolt::quant_step_sel(in[i + 1], out[0], flev, 1.0f / flev);
     }
-    fwrite(out, sizeof(float), 6, stdout);
+    fwrite(out, sizeof(float), 11, stdout);
   }
   return 0;
 }
