@@ -534,13 +534,15 @@ namespace jolt {
 // ------------------------------------------------------------------------------------------
 // Cholesky factor for 256 < k <= 1024: one cluster of 8 CTAs per matrix, right-looking by
 // 32-column block columns, block column K owned by CTA K % 8.  Per block column J:
-//   1. its owner factors the diagonal block (one warp, column by column) and inverts it
-//      (forward substitution, one lane per column), then forms the panel
-//      L_IJ = A_IJ inv(L_JJ)^T for every block row I > J;
+//   1. its owner factors the diagonal block (one warp, column by column), inverts it (forward
+//      substitution, one lane per column) and writes the inverse into every CTA's shared
+//      memory (distributed shared memory);
 //   2. cluster barrier;
-//   3. every CTA updates its block columns K > J: A_IK -= L_IJ L_KJ^T for I >= K.
-// The owner of block column J + 1 updated it in step 3 itself, so one barrier per block
-// column suffices.  Output in the layout of chol_factor_kernel: L below the diagonal blocks
+//   3. every CTA forms the panel rows it owns, L_IJ = A_IJ inv(L_JJ)^T for I > J, I % 8 == q;
+//   4. cluster barrier;
+//   5. every CTA updates its block columns K > J: A_IK -= L_IJ L_KJ^T for I >= K.
+// The owner of block column J + 1 updated it in step 5 itself, so its factorisation needs no
+// further barrier.  Output in the layout of chol_factor_kernel: L below the diagonal blocks
 // in the lower triangle, inv(L_JJ) in the upper part of its diagonal block (W[i][c] at
 // G[i * gld + c], c <= i).  A pivot that is not positive: DEV_ERR_FACTOR, pivot taken as 1.
 // grid (8 * matrices), clusters of 8, 256 threads.
@@ -587,7 +589,7 @@ __global__ void __cluster_dims__(CC_CL, 1, 1) __launch_bounds__(256)
             for (int s = c + 1; s <= lane; ++s) Ls[lane][s] -= Ls[lane][c] * Ls[s][c];
           __syncwarp();
         }
-        // inverse: lane c solves L x = e_c
+        // inverse: lane c solves L x = e_c; the result goes to every CTA of the cluster
         double x[CF_NB];
 #pragma unroll
         for (int r = 0; r < CF_NB; ++r) {
@@ -596,39 +598,43 @@ __global__ void __cluster_dims__(CC_CL, 1, 1) __launch_bounds__(256)
           for (int p = 0; p < r; ++p) v = fma(-Ls[r][p], x[p], v);
           x[r] = v / Ls[r][r];
         }
+        for (int t = 0; t < CC_CL; ++t) {
+          double* wt = cluster.map_shared_rank(&Wi[0][0], t);
 #pragma unroll
-        for (int r = 0; r < CF_NB; ++r) Wi[r][lane] = r >= lane ? x[r] : 0.0;
+          for (int r = 0; r < CF_NB; ++r) wt[r * CF_P + lane] = r >= lane ? x[r] : 0.0;
+        }
       }
       __syncthreads();
-      // the diagonal block's inverse into the upper part (W[r][c] at (row c, column r)); rows
-      // of L below it follow as the panel
+      // the diagonal block's inverse into the upper part (W[r][c] at (row c, column r))
       for (int idx = tid; idx < CF_NB * CF_NB; idx += blockDim.x) {
         const int r = idx / CF_NB, c = idx % CF_NB;
         if (r < nbJ && c <= r) at(J0 + c, J0 + r) = Wi[r][c];
       }
-      for (int I = J + 1; I < nbk; ++I) {
-        const int I0 = I * CF_NB, nbI = min(CF_NB, k - I0);
-        __syncthreads();
-        for (int idx = tid; idx < CF_NB * CF_NB; idx += blockDim.x) {
-          const int r = idx % CF_NB, c = idx / CF_NB;
-          Ls[r][c] = (r < nbI && c < nbJ) ? at(I0 + r, J0 + c) : 0.0;
-        }
-        __syncthreads();
-        // L_IJ[r][c] = sum_s A_IJ[r][s] inv(L_JJ)[c][s]
-        const int r = tid >> 3, cg0 = tid & 7;
-        double o[4];
+    }
+    __threadfence();
+    cluster.sync();   // inv(L_JJ) in every CTA
+    // my rows of the panel: L_IJ[r][c] = sum_s A_IJ[r][s] inv(L_JJ)[c][s]
+    for (int I = J + 1 + ((q - (J + 1)) % CC_CL + CC_CL) % CC_CL; I < nbk; I += CC_CL) {
+      const int I0 = I * CF_NB, nbI = min(CF_NB, k - I0);
+      __syncthreads();
+      for (int idx = tid; idx < CF_NB * CF_NB; idx += blockDim.x) {
+        const int r = idx % CF_NB, c = idx / CF_NB;
+        Ls[r][c] = (r < nbI && c < nbJ) ? at(I0 + r, J0 + c) : 0.0;
+      }
+      __syncthreads();
+      const int r = tid >> 3, cg0 = tid & 7;
+      double o[4];
 #pragma unroll
-        for (int jj = 0; jj < 4; ++jj) {
-          const int c = cg0 + 8 * jj;
-          double acc = 0.0;
-          for (int s2 = 0; s2 <= c; ++s2) acc = fma(Ls[r][s2], Wi[c][s2], acc);
-          o[jj] = acc;
-        }
+      for (int jj = 0; jj < 4; ++jj) {
+        const int c = cg0 + 8 * jj;
+        double acc = 0.0;
+        for (int s2 = 0; s2 <= c; ++s2) acc = fma(Ls[r][s2], Wi[c][s2], acc);
+        o[jj] = acc;
+      }
 #pragma unroll
-        for (int jj = 0; jj < 4; ++jj) {
-          const int c = cg0 + 8 * jj;
-          if (r < nbI && c < nbJ) at(I0 + r, J0 + c) = o[jj];
-        }
+      for (int jj = 0; jj < 4; ++jj) {
+        const int c = cg0 + 8 * jj;
+        if (r < nbI && c < nbJ) at(I0 + r, J0 + c) = o[jj];
       }
     }
     __threadfence();

@@ -3,18 +3,19 @@
 // tokens).  The same algorithm as the cluster solver of eig_cluster.cuh -- Householder
 // tridiagonalisation, multisection on Sturm counts, inverse iteration, the back-transformation
 // -- with the matrix in global memory (it does not fit the shared memory of a cluster):
-//   1. tridiag_gm_kernel: one cluster of 8 CTAs per matrix; CTA q owns the columns c with
-//      c % 8 == q (contiguous in the column-major matrix).  Per column j: the owner forms the
-//      reflector and writes it into every CTA's shared memory (distributed shared memory) and
-//      to global memory; every CTA computes p = beta A v on its columns and sends p and its
-//      partial p.v to all; every CTA applies the rank-2 update to its columns.  Two cluster
-//      barriers per column; vectors alternate between two buffers (as in eig_cluster.cuh).
+//   1. tridiag_gm_kernel: one cluster of 8 CTAs of 1024 threads per matrix; CTA q owns the
+//      columns c with c % 8 == q (contiguous in the column-major matrix).  Per column j: the
+//      owner forms the reflector and writes it into every CTA's shared memory (distributed
+//      shared memory) and to global memory; every CTA computes p = beta A v on its columns
+//      (one warp per column) and sends p and its warps' partial p.v to all; every CTA applies
+//      the rank-2 update to its columns.  Two cluster barriers per column; vectors alternate
+//      between two buffers (as in eig_cluster.cuh).
 //   2. tri_eig_kernel: 128 eigenvalues per CTA by multisection (8 threads each), then their
 //      eigenvectors of T by inverse iteration (one thread each, the factors in global memory).
 //   3. tight_mgs_kernel: vectors of eigenvalues closer than 1e-10 ||T|| orthonormalised in
 //      order by one warp (they span their cluster's invariant subspace).
-//   4. backtransform_kernel: V = H_0 ... H_{n-3} Z on 16 eigenvectors per CTA, the vectors in
-//      shared memory, the reflectors staged 8 at a time, one warp per two vectors.
+//   4. wy_tfactor_kernel, wy_apply_kernel: V = H_0 ... H_{n-3} Z with the reflectors taken 32 at
+//      a time in compact WY form (I - Y T Y^T), 16 eigenvectors per CTA in shared memory.
 // Output as the cluster solver: w ascending; V[r * n + i] = component r of eigenvector i.
 // Non-finite input raises DEV_ERR_NONFINITE (the matrices are sanitised before, so the
 // arithmetic stays finite).  Every thread of every CTA of a cluster passes the same cluster
@@ -33,14 +34,21 @@ constexpr int CL = 8;             // CTAs per matrix in the tridiagonalisation
 constexpr int MAXN = 1024;
 constexpr int THREADS = 256;
 constexpr int WARPS = THREADS / 32;
-constexpr int RED = CL * WARPS;
-// tridiagonalisation shared memory (doubles): v[2][MAXN] | p[2][MAXN] | red[2][RED] | beta[2] | tmp[THREADS]
-constexpr size_t TRI_SMEM = sizeof(double) * (4 * (size_t)MAXN + 2 * RED + 2 + THREADS);
+// the tridiagonalisation runs 1024 threads per CTA: one warp per column in the matrix-vector
+// product and the update, so that many loads of the (L2-resident) matrix are in flight
+constexpr int TRI_THREADS = 1024;
+constexpr int TRI_WARPS = TRI_THREADS / 32;
+constexpr int TRED = CL * TRI_WARPS;   // partial sums of p.v: one per warp of the cluster
+// tridiagonalisation shared memory (doubles): v[2][MAXN] | p[2][MAXN] | red[2][TRED] | beta[2] | tmp[TRI_WARPS]
+constexpr size_t TRI_SMEM = sizeof(double) * (4 * (size_t)MAXN + 2 * TRED + 2 + TRI_WARPS);
 // per matrix global scratch (doubles): reflectors n*n | LU factors 5*n*n | d, e, beta 3*n
 __host__ __device__ inline size_t scratch_doubles(int n) { return (size_t)6 * n * n + 3 * (size_t)n; }
 constexpr int EV_PER_CTA = 128;   // eigenvalues / eigenvectors per CTA of tri_eig_kernel
-constexpr int BT_COLS = 16;       // eigenvectors per CTA of the back-transformation
-constexpr int BT_REFL = 8;        // reflectors staged together
+// back-transformation in blocks of WY_NB reflectors (compact WY form I - Y T Y^T)
+constexpr int WY_NB = 32;
+constexpr int WY_COLS = 16;       // eigenvectors per CTA
+constexpr int WY_ROWS = 128;      // rows of Y staged together
+constexpr int WY_THREADS = 256;
 }  // namespace eigl
 
 __device__ __forceinline__ double eigl_block_sum(double v, double* tmp) {
@@ -65,9 +73,9 @@ __global__ void symmetrize_lower_kernel(double* A, int n, long long sA) {
   }
 }
 
-// grid (8 * matrices), clusters of 8, eigl::THREADS threads, eigl::TRI_SMEM dynamic shared
+// grid (8 * matrices), clusters of 8, eigl::TRI_THREADS threads, eigl::TRI_SMEM dynamic shared
 // memory.  A: n x n symmetric, column-major (both triangles), stride sA, overwritten.
-__global__ void __cluster_dims__(eigl::CL, 1, 1) __launch_bounds__(eigl::THREADS)
+__global__ void __cluster_dims__(eigl::CL, 1, 1) __launch_bounds__(eigl::TRI_THREADS)
     tridiag_gm_kernel(double* A, int n, long long sA, double* scr) {
   using namespace eigl;
   cg::cluster_group cluster = cg::this_cluster();
@@ -77,9 +85,9 @@ __global__ void __cluster_dims__(eigl::CL, 1, 1) __launch_bounds__(eigl::THREADS
   extern __shared__ double tg_sm[];
   double* vb = tg_sm;                     // [2][MAXN]
   double* pb = vb + 2 * MAXN;             // [2][MAXN]
-  double* red = pb + 2 * MAXN;            // [2][RED]
-  double* sbeta = red + 2 * RED;          // [2]
-  double* tmp = sbeta + 2;                // [THREADS]
+  double* red = pb + 2 * MAXN;            // [2][TRED]
+  double* sbeta = red + 2 * TRED;         // [2]
+  double* tmp = sbeta + 2;                // [TRI_WARPS]
   double* Au = A + (long long)u * sA;
   double* base = scr + (long long)u * scratch_doubles(n);
   double* refl = base;                    // [n][n]
@@ -119,42 +127,43 @@ __global__ void __cluster_dims__(eigl::CL, 1, 1) __launch_bounds__(eigl::THREADS
     cluster.sync();   // (A) v and beta everywhere
     const double beta = sbeta[buf];
     const double* v = vb + buf * MAXN;
+    // my first column after j (the columns c with c % CL == q), then every CL-th; warp w takes
+    // the columns cf + CL (w + TRI_WARPS i)
+    const int cf = j + 1 + ((q - (j + 1)) % CL + CL) % CL;
     if (beta != 0.0) {
-      // p_c = beta * (column c) . v on my columns c > j: 8 threads per column
+      // p_c = beta * (column c) . v: one warp per column, lanes over rows, four partial sums
       double pv = 0.0;
-      const int part = tid & 7;
-      // the same trip count on every lane (the shuffles below take the whole warp)
-      const int iters = (n + CL * (THREADS / 8) - 1) / (CL * (THREADS / 8));
-      for (int it = 0; it < iters; ++it) {
-        const int c = q + CL * (tid >> 3) + CL * (THREADS / 8) * it;
-        double s = 0.0;
-        if (c > j && c < n) {
-          const double* col = Au + (long long)c * n;
-          for (int r = j + 1 + part; r < n; r += 8) s = fma(col[r], v[r], s);
+      for (int c = cf + CL * warp; c < n; c += CL * TRI_WARPS) {
+        const double* col = Au + (long long)c * n;
+        double s0 = 0.0, s1 = 0.0, s2 = 0.0, s3 = 0.0;
+        int r = j + 1 + lane;
+        for (; r + 96 < n; r += 128) {
+          s0 = fma(col[r], v[r], s0);
+          s1 = fma(col[r + 32], v[r + 32], s1);
+          s2 = fma(col[r + 64], v[r + 64], s2);
+          s3 = fma(col[r + 96], v[r + 96], s3);
         }
-#pragma unroll
-        for (int o = 4; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-        if (part == 0 && c > j && c < n) {
-          const double pc = beta * s;
-          for (int t = 0; t < CL; ++t) cluster.map_shared_rank(pb, t)[buf * MAXN + c] = pc;
-          pv = fma(pc, v[c], pv);
-        }
+        for (; r < n; r += 32) s0 = fma(col[r], v[r], s0);
+        const double pc = beta * eigc::warp_sum((s0 + s1) + (s2 + s3));
+        if (lane < CL) cluster.map_shared_rank(pb, lane)[buf * MAXN + c] = pc;
+        pv = fma(pc, v[c], pv);   // the same on every lane
       }
-      pv = eigc::warp_sum(pv);
-      if (lane == 0)
-        for (int t = 0; t < CL; ++t) cluster.map_shared_rank(red, t)[buf * RED + q * WARPS + warp] = pv;
+      if (lane < CL) cluster.map_shared_rank(red, lane)[buf * TRED + q * TRI_WARPS + warp] = pv;
     }
     cluster.sync();   // (B) p and the partial sums of p.v everywhere
     if (beta != 0.0) {
+      // p.v over the cluster's warps, in the same order in every warp of every CTA
       double ptv = 0.0;
-      for (int t = 0; t < RED; ++t) ptv += red[buf * RED + t];
+#pragma unroll
+      for (int t = 0; t < TRED / 32; ++t) ptv += red[buf * TRED + lane * (TRED / 32) + t];
+      ptv = eigc::warp_sum(ptv);
       const double K = 0.5 * beta * ptv;
       const double* pf = pb + buf * MAXN;
       // A -= v w^T + w v^T on my columns, w = p - K v; one warp per column, lanes over rows
-      for (int c = q + CL * warp; c < n; c += CL * WARPS) {
-        if (c <= j) continue;
+      for (int c = cf + CL * warp; c < n; c += CL * TRI_WARPS) {
         double* col = Au + (long long)c * n;
         const double vc = v[c], wc = fma(-K, vc, pf[c]);
+#pragma unroll 4
         for (int r = j + 1 + lane; r < n; r += 32) col[r] = col[r] - (v[r] * wc + fma(-K, v[r], pf[r]) * vc);
       }
     }
@@ -283,52 +292,155 @@ __global__ void tight_mgs_kernel(int n, const double* w, long long sw, double* V
   }
 }
 
-// grid (ceil(n / 16), matrices), eigl::THREADS threads, dynamic shared memory backtransform_smem(n).
-// Z (16 eigenvectors of T) staged in shared memory; H_{n-3} .. H_0 applied in turn, 8
-// reflectors staged together; warp w updates vectors 2w and 2w + 1, lanes over rows.
-inline size_t backtransform_smem(int n) {
-  return sizeof(double) * ((size_t)n * eigl::BT_COLS + (size_t)eigl::BT_REFL * n);
-}
-__global__ void __launch_bounds__(eigl::THREADS) backtransform_kernel(int n, double* V, const double* scr) {
+// ---- back-transformation V = H_0 H_1 ... H_{n-3} Z in blocks of 32 reflectors ----
+// The product of the reflectors j0 .. j0 + jn - 1 of a block is I - Y T Y^T (Y = [v_j0 ..], T
+// upper triangular: T_ii = beta_i, T[0:i, i] = -beta_i T[0:i, 0:i] Y[:, 0:i]^T v_i, the forward
+// accumulation of Schreiber and Van Loan's compact WY form).  V = P_0 (P_1 (... (P_last Z))).
+// T of block b goes to the scratch area of the inverse-iteration factors (free by then).
+inline __host__ __device__ int wy_blocks(int n) { return (n - 2 + eigl::WY_NB - 1) / eigl::WY_NB; }
+
+// grid (wy_blocks(n), matrices), eigl::WY_THREADS threads
+__global__ void __launch_bounds__(eigl::WY_THREADS) wy_tfactor_kernel(int n, double* scr) {
   using namespace eigl;
-  extern __shared__ double bt_sm[];
-  double* Z = bt_sm;                      // [n][BT_COLS]
-  double* R = Z + (size_t)n * BT_COLS;    // [BT_REFL][n]
-  const int u = blockIdx.y, c0 = blockIdx.x * BT_COLS, tid = threadIdx.x;
-  const int lane = tid & 31, warp = tid >> 5;
-  const double* base = scr + (long long)u * scratch_doubles(n);
+  constexpr int TF_ROWS = 64;   // rows of Y staged together (static shared memory stays under 48 KB)
+  __shared__ double Yc[TF_ROWS][WY_NB + 1];
+  __shared__ double Ss[WY_NB][WY_NB + 1];
+  __shared__ double Ts[WY_NB][WY_NB + 1];
+  const int u = blockIdx.y, b = blockIdx.x, tid = threadIdx.x;
+  double* base = scr + (long long)u * scratch_doubles(n);
   const double* refl = base;
   const double* bg = base + 6 * (long long)n * n + 2 * (long long)n;
-  double* Vu = V + (long long)u * n * n;
-  for (int idx = tid; idx < n * BT_COLS; idx += blockDim.x) {
-    const int r = idx / BT_COLS, c = idx - r * BT_COLS;
-    Z[idx] = c0 + c < n ? Vu[(long long)r * n + c0 + c] : 0.0;
-  }
-  for (int jh = n - 3; jh >= 0; jh -= BT_REFL) {
-    const int jl = jh - BT_REFL + 1 > 0 ? jh - BT_REFL + 1 : 0;   // reflectors jh, jh-1, .., jl
+  double* Tg = base + (long long)n * n + (long long)b * WY_NB * WY_NB;
+  const int j0 = b * WY_NB, jn = min(WY_NB, n - 2 - j0), r0 = j0 + 1;
+  // S = Y^T Y: thread (i, mg) accumulates S[i][mg + 8 k]
+  const int i = tid >> 3, mg = tid & 7;
+  double sacc[4] = {0.0, 0.0, 0.0, 0.0};
+  for (int rc = r0; rc < n; rc += TF_ROWS) {
+    const int nr = min(TF_ROWS, n - rc);
     __syncthreads();
-    for (int idx = tid; idx < (jh - jl + 1) * n; idx += blockDim.x) {
-      const int k = idx / n, r = idx - k * n;
-      R[k * n + r] = refl[(long long)(jh - k) * n + r];
+    for (int idx = tid; idx < WY_NB * TF_ROWS; idx += blockDim.x) {
+      const int ii = idx / TF_ROWS, rr = idx - ii * TF_ROWS;
+      Yc[rr][ii] = (ii < jn && rr < nr) ? refl[(long long)(j0 + ii) * n + rc + rr] : 0.0;
     }
     __syncthreads();
-    for (int k = 0; k <= jh - jl; ++k) {
-      const int j = jh - k;
-      const double bj = bg[j];
-      const double* v = R + k * n;
+    for (int rr = 0; rr < nr; ++rr) {
+      const double y = Yc[rr][i];
 #pragma unroll
-      for (int cc = 0; cc < 2; ++cc) {
-        const int c = 2 * warp + cc;
-        double s = 0.0;
-        for (int r = j + 1 + lane; r < n; r += 32) s = fma(v[r], Z[r * BT_COLS + c], s);
-        s = eigc::warp_sum(s) * bj;
-        for (int r = j + 1 + lane; r < n; r += 32) Z[r * BT_COLS + c] = fma(-s, v[r], Z[r * BT_COLS + c]);
+      for (int k = 0; k < 4; ++k) sacc[k] = fma(y, Yc[rr][mg + 8 * k], sacc[k]);
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < 4; ++k) Ss[i][mg + 8 * k] = sacc[k];
+  __syncthreads();
+  if (tid < 32) {
+    // T column by column; lane l owns row l (and reads only its own row of T)
+    const int l = tid;
+    for (int c = 0; c < WY_NB; ++c) {
+      double t = 0.0;
+      if (c < jn) {
+        const double tau = bg[j0 + c];
+        if (l < c) {
+          double acc = 0.0;
+          for (int m = l; m < c; ++m) acc = fma(Ts[l][m], Ss[m][c], acc);
+          t = -tau * acc;
+        } else if (l == c) {
+          t = tau;
+        }
       }
+      Ts[l][c] = t;
     }
   }
   __syncthreads();
-  for (int idx = tid; idx < n * BT_COLS; idx += blockDim.x) {
-    const int r = idx / BT_COLS, c = idx - r * BT_COLS;
+  for (int idx = tid; idx < WY_NB * WY_NB; idx += blockDim.x) Tg[idx] = Ts[idx / WY_NB][idx % WY_NB];
+}
+
+inline size_t wy_apply_smem(int n) {
+  using namespace eigl;
+  return sizeof(double) * ((size_t)n * WY_COLS + (size_t)WY_ROWS * (WY_NB + 1) + WY_NB * WY_COLS +
+                           WY_NB * (WY_NB + 1));
+}
+
+// grid (ceil(n / 16), matrices), eigl::WY_THREADS threads, wy_apply_smem(n) bytes of dynamic
+// shared memory.  Z (16 eigenvectors of T) in shared memory; for every block from the last:
+// W = Y^T Z, W = T W, Z -= Y W, with Y staged 128 rows at a time.
+__global__ void __launch_bounds__(eigl::WY_THREADS) wy_apply_kernel(int n, double* V, const double* scr) {
+  using namespace eigl;
+  extern __shared__ double wy_sm[];
+  double* Z = wy_sm;                                                  // [n][WY_COLS]
+  double(*Yc)[WY_NB + 1] = reinterpret_cast<double(*)[WY_NB + 1]>(Z + (size_t)n * WY_COLS);   // [WY_ROWS]
+  double* Wb = reinterpret_cast<double*>(Yc + WY_ROWS);               // [WY_NB][WY_COLS]
+  double* Tb = Wb + WY_NB * WY_COLS;                                  // [WY_NB][WY_NB + 1]
+  const int u = blockIdx.y, c0 = blockIdx.x * WY_COLS, tid = threadIdx.x;
+  const double* base = scr + (long long)u * scratch_doubles(n);
+  const double* refl = base;
+  double* Vu = V + (long long)u * n * n;
+  for (int idx = tid; idx < n * WY_COLS; idx += blockDim.x) {
+    const int r = idx / WY_COLS, c = idx - r * WY_COLS;
+    Z[idx] = c0 + c < n ? Vu[(long long)r * n + c0 + c] : 0.0;
+  }
+  const int iw = tid >> 3, cp = (tid & 7) * 2;     // W phase: row iw of W, columns cp, cp + 1
+  const int cu = tid & 15, rg = tid >> 4;          // update phase: column cu, rows rg + 16 k
+  auto load_y = [&](int j0, int jn, int rc, int nr) {
+    __syncthreads();
+    for (int idx = tid; idx < WY_NB * WY_ROWS; idx += blockDim.x) {
+      const int ii = idx / WY_ROWS, rr = idx - ii * WY_ROWS;
+      Yc[rr][ii] = (ii < jn && rr < nr) ? refl[(long long)(j0 + ii) * n + rc + rr] : 0.0;
+    }
+    __syncthreads();
+  };
+  for (int b = wy_blocks(n) - 1; b >= 0; --b) {
+    const int j0 = b * WY_NB, jn = min(WY_NB, n - 2 - j0), r0 = j0 + 1;
+    const double* Tg = base + (long long)n * n + (long long)b * WY_NB * WY_NB;
+    for (int idx = tid; idx < WY_NB * WY_NB; idx += blockDim.x) Tb[(idx / WY_NB) * (WY_NB + 1) + idx % WY_NB] = Tg[idx];
+    // W = Y^T Z
+    double w0 = 0.0, w1 = 0.0;
+    for (int rc = r0; rc < n; rc += WY_ROWS) {
+      const int nr = min(WY_ROWS, n - rc);
+      load_y(j0, jn, rc, nr);
+      for (int rr = 0; rr < nr; ++rr) {
+        const double y = Yc[rr][iw];
+        const double2 z = *reinterpret_cast<const double2*>(Z + (size_t)(rc + rr) * WY_COLS + cp);
+        w0 = fma(y, z.x, w0);
+        w1 = fma(y, z.y, w1);
+      }
+    }
+    Wb[iw * WY_COLS + cp] = w0;
+    Wb[iw * WY_COLS + cp + 1] = w1;
+    __syncthreads();
+    // W = T W (T upper triangular)
+    double a0 = 0.0, a1 = 0.0;
+    for (int m = iw; m < WY_NB; ++m) {
+      const double t = Tb[iw * (WY_NB + 1) + m];
+      a0 = fma(t, Wb[m * WY_COLS + cp], a0);
+      a1 = fma(t, Wb[m * WY_COLS + cp + 1], a1);
+    }
+    __syncthreads();
+    Wb[iw * WY_COLS + cp] = a0;
+    Wb[iw * WY_COLS + cp + 1] = a1;
+    __syncthreads();
+    double wc[WY_NB];
+#pragma unroll
+    for (int m = 0; m < WY_NB; ++m) wc[m] = Wb[m * WY_COLS + cu];
+    // Z -= Y W
+    for (int rc = r0; rc < n; rc += WY_ROWS) {
+      const int nr = min(WY_ROWS, n - rc);
+      load_y(j0, jn, rc, nr);
+#pragma unroll 2
+      for (int k = 0; k < WY_ROWS / 16; ++k) {
+        const int rr = rg + 16 * k;
+        if (rr < nr) {
+          double acc = 0.0;
+#pragma unroll
+          for (int m = 0; m < WY_NB; ++m) acc = fma(Yc[rr][m], wc[m], acc);
+          Z[(size_t)(rc + rr) * WY_COLS + cu] -= acc;
+        }
+      }
+    }
+    __syncthreads();
+  }
+  __syncthreads();
+  for (int idx = tid; idx < n * WY_COLS; idx += blockDim.x) {
+    const int r = idx / WY_COLS, c = idx - r * WY_COLS;
     if (c0 + c < n) Vu[(long long)r * n + c0 + c] = Z[idx];
   }
 }

@@ -480,6 +480,9 @@ struct Ctx {
   template <typename T>
   T* at(size_t off) const { return reinterpret_cast<T*>(ws + off); }
   uint32_t* status() const { return at<uint32_t>(p.o_status); }
+  // the tile counter of the tensor-core GEMMs launched on this context's stream (bytes 64.. of
+  // the 256-byte status block; one per stream, since the two streams' GEMMs may overlap)
+  int* sched() const { return at<int>(p.o_status) + 16 + 8 * side; }
   CacheView view() const {
     CacheView c;
     c.k = k;
@@ -558,19 +561,31 @@ jolt_status sym_eig_top(const Ctx& c, double* S, int n, int nbatch, int r, float
     count_launch(), symmetrize_lower_kernel<<<dim3(64, (unsigned)nbatch), 256, 0, c.st>>>(S, n, (long long)n * n);
     CUDA_TRY(cudaGetLastError());
     CUDA_TRY(cudaFuncSetAttribute(tridiag_gm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)eigl::TRI_SMEM));
-    count_launch(), tridiag_gm_kernel<<<(unsigned)(nbatch * eigl::CL), eigl::THREADS, eigl::TRI_SMEM, c.st>>>(
-        S, n, (long long)n * n, scr);
-    CUDA_TRY(cudaGetLastError());
-    count_launch(), tri_eig_kernel<<<dim3((unsigned)ceil_div(n, eigl::EV_PER_CTA), (unsigned)nbatch), eigl::THREADS, 0,
-                                     c.st>>>(n, w, n, V, scr);
-    CUDA_TRY(cudaGetLastError());
-    count_launch(), tight_mgs_kernel<<<(unsigned)nbatch, 32, 0, c.st>>>(n, w, n, V);
-    CUDA_TRY(cudaGetLastError());
-    const size_t bsm = backtransform_smem(n);
-    CUDA_TRY(cudaFuncSetAttribute(backtransform_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bsm));
-    count_launch(), backtransform_kernel<<<dim3((unsigned)ceil_div(n, eigl::BT_COLS), (unsigned)nbatch), eigl::THREADS,
-                                           bsm, c.st>>>(n, V, scr);
-    CUDA_TRY(cudaGetLastError());
+    {
+      ProfScope ps1("eig_tridiag", c.st, nbatch);
+      count_launch(), tridiag_gm_kernel<<<(unsigned)(nbatch * eigl::CL), eigl::TRI_THREADS, eigl::TRI_SMEM, c.st>>>(
+          S, n, (long long)n * n, scr);
+      CUDA_TRY(cudaGetLastError());
+    }
+    {
+      ProfScope ps2("eig_tridiag_solve", c.st, nbatch);
+      count_launch(), tri_eig_kernel<<<dim3((unsigned)ceil_div(n, eigl::EV_PER_CTA), (unsigned)nbatch),
+                                       eigl::THREADS, 0, c.st>>>(n, w, n, V, scr);
+      CUDA_TRY(cudaGetLastError());
+      count_launch(), tight_mgs_kernel<<<(unsigned)nbatch, 32, 0, c.st>>>(n, w, n, V);
+      CUDA_TRY(cudaGetLastError());
+    }
+    const size_t wsm = wy_apply_smem(n);
+    CUDA_TRY(cudaFuncSetAttribute(wy_apply_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)wsm));
+    {
+      ProfScope ps3("eig_backtransform", c.st, nbatch);
+      count_launch(), wy_tfactor_kernel<<<dim3((unsigned)wy_blocks(n), (unsigned)nbatch), eigl::WY_THREADS, 0,
+                                          c.st>>>(n, scr);
+      CUDA_TRY(cudaGetLastError());
+      count_launch(), wy_apply_kernel<<<dim3((unsigned)ceil_div(n, eigl::WY_COLS), (unsigned)nbatch),
+                                        eigl::WY_THREADS, wsm, c.st>>>(n, V, scr);
+      CUDA_TRY(cudaGetLastError());
+    }
     count_launch(), eig_select_kernel<<<dim3(r, nbatch), 256, 0, c.st>>>(w, V, n, 1, n, n, (long long)n * n, r,
                                                                          out_f32, out_bf16, ldo, sout, out_vals);
     CUDA_TRY(cudaGetLastError());
@@ -734,8 +749,9 @@ jolt_status cache_maps(const Ctx& c, bool rows, CUtensorMap* mk, CUtensorMap* mv
   return JOLT_OK;
 }
 
-jolt_status umma_run(const UmmaMaps& m, const UmmaArgs& a, int nb, cudaStream_t st) {
-  cudaError_t e = launch_umma(m, a, nb, st);
+jolt_status umma_run(const Ctx& c, const UmmaMaps& m, UmmaArgs a, int nb) {
+  a.sched = c.sched();
+  cudaError_t e = launch_umma(m, a, nb, c.st);
   if (e != cudaSuccess) return fail(JOLT_ERR_CUDA, "tensor-core GEMM: %s", cudaGetErrorString(e));
   return JOLT_OK;
 }
@@ -797,12 +813,12 @@ jolt_status cholqr_tc(const Ctx& c, float* Y, long long m, int k, int ld, int pa
       m1.a0 = m1.a1 = my.a0;
       m1.b0 = my.a0;
       m1.b1 = my.a1;
-      JTRY(umma_run(m1, g, 2, c.st));
+      JTRY(umma_run(c, m1, g, 2));
       UmmaMaps m2;   // Yl^T Yh
       m2.a0 = m2.a1 = my.a1;
       m2.b0 = m2.b1 = my.a0;
       g.C = gpart + (long long)ns * k * gld;
-      JTRY(umma_run(m2, g, 1, c.st));
+      JTRY(umma_run(c, m2, g, 1));
       count_launch(), reduce_upper_sym_kernel<<<grid1d((long long)p.NU * k * k), 256, 0, c.st>>>(gpart, G, p.NU,
                                                                                                   2 * ns, k, gld);
       CUDA_TRY(cudaGetLastError());
@@ -822,8 +838,12 @@ jolt_status cholqr_tc(const Ctx& c, float* Y, long long m, int k, int ld, int pa
       } else {
         // 256 < k <= 1024: the cluster Cholesky (chol.cuh), then the block-column inverse
         count_launch(), sanitize_sym_batched_kernel<<<p.NU, 1024, 0, c.st>>>(G, k, gld, sG, c.status());
-        count_launch(), chol_cluster_kernel<<<(unsigned)(p.NU * CC_CL), 256, 0, c.st>>>(G, k, gld, sG, c.status());
-        CUDA_TRY(cudaGetLastError());
+        {
+          ProfScope ps4("chol_cluster", c.st, p.NU);
+          count_launch(), chol_cluster_kernel<<<(unsigned)(p.NU * CC_CL), 256, 0, c.st>>>(G, k, gld, sG, c.status());
+          CUDA_TRY(cudaGetLastError());
+        }
+        ProfScope ps5("tri_inv_large", c.st, p.NU);
         count_launch(), tri_inv_large_kernel<<<dim3(nbk, p.NU), CF_THREADS, 0, c.st>>>(
             G, k, gld, sG, c.at<double>(p.o_winv), kq32, WT, kq32, sW);
         CUDA_TRY(cudaGetLastError());
@@ -851,12 +871,12 @@ jolt_status cholqr_tc(const Ctx& c, float* Y, long long m, int k, int ld, int pa
       m1.a0 = m1.a1 = my.a0;
       m1.b0 = mw.b0;
       m1.b1 = mw.b1;
-      JTRY(umma_run(m1, q, 2, c.st));
+      JTRY(umma_run(c, m1, q, 2));
       UmmaMaps m2;   // + Yl Wh^T
       m2.a0 = m2.a1 = my.a1;
       m2.b0 = m2.b1 = mw.b0;
       q.c_accum = 1;
-      JTRY(umma_run(m2, q, 1, c.st));
+      JTRY(umma_run(c, m2, q, 1));
     }
   }
   return JOLT_OK;
@@ -879,7 +899,7 @@ jolt_status umma_product(const Ctx& c, bool z_side, const bf16* F16, const float
     f1 = lo;
   }
   cudaError_t e = umma_x_product(c.k, c.v, p.nL, p.H, p.T, p.D, p.S, p.NU, z_side, f0, f1, p.kp, p.k, out, p.kp,
-                                 c.status(), c.st);
+                                 c.status(), c.sched(), c.st);
   if (e != cudaSuccess) return fail(JOLT_ERR_CUDA, "tensor-core X-product: %s", cudaGetErrorString(e));
   return JOLT_OK;
 }
@@ -934,7 +954,7 @@ jolt_status run_feature_factor(const Ctx& c, float* Wf, long long ldWf, bf16* Ws
     a.sC = (long long)p.gd_split * D * D;
     a.ssplit = (long long)D * D;
     a.status = c.status();
-    JTRY(umma_run(m, a, 1, c.st));
+    JTRY(umma_run(c, m, a, 1));
   } else {
     const int kchunk = (int)round_up(ceil_div(rows, p.gd_split), 32);
     GemmParams g;
@@ -1012,7 +1032,7 @@ jolt_status run_token_exact(const Ctx& c, float* Uf, long long ldUf) {
       a.ldc = n;
       a.sC = n * n;
       a.status = c.status();
-      JTRY(umma_run(m, a, 1, c.st));
+      JTRY(umma_run(c, m, a, 1));
     } else {
       JTRY(gemm(g, xtype(c), xtype(c), c.st));
     }
@@ -1047,7 +1067,7 @@ jolt_status run_token_exact(const Ctx& c, float* Uf, long long ldUf) {
     count_launch(), split_bf16_kernel<<<grid1d(nF), 256, 0, c.st>>>(V, hi, lo, nF);
     CUDA_TRY(cudaGetLastError());
     cudaError_t e = umma_x_product(c.k, c.v, p.nL, p.H, T, p.D, p.S, p.NU, false, hi, lo, p.ldU, p.rTmax, Uf, ldUf,
-                                   c.status(), c.st);
+                                   c.status(), c.sched(), c.st);
     if (e != cudaSuccess) return fail(JOLT_ERR_CUDA, "tensor-core X-product: %s", cudaGetErrorString(e));
   } else {
     JTRY(gemm_xf(c, y, false, V, (long long)p.NU * M * p.ldU));
@@ -1178,12 +1198,12 @@ jolt_status run_token_randomized(const Ctx& c, float* Uf, long long ldUf) {
     m1.a0 = m1.a1 = mq.a0;
     m1.b0 = mv.b0;
     m1.b1 = mv.b1;
-    JTRY(umma_run(m1, a, 2, c.st));
+    JTRY(umma_run(c, m1, a, 2));
     UmmaMaps m2;
     m2.a0 = m2.a1 = mq.a1;
     m2.b0 = m2.b1 = mv.b0;
     a.c_accum = 1;
-    JTRY(umma_run(m2, a, 1, c.st));
+    JTRY(umma_run(c, m2, a, 1));
     return JOLT_OK;
   }
   GemmParams uq;
@@ -1259,7 +1279,7 @@ jolt_status run_core(const Ctx& c, const bf16* Us, long long ldU, const bf16* Ws
     a.ldc = p.ldW;
     a.sC = (long long)S * T * p.ldW;
     a.status = c.status();
-    JTRY(umma_run(m, a, 1, c.st));
+    JTRY(umma_run(c, m, a, 1));
     // C_s = bf16(U_s^T Z_s) per (unit, slice): A = U_s^T (MN-major, shared by the S slices)
     UmmaMaps m2;
     if (!map_dense(&m2.a0, Us, ldU, T, p.NU) || !map_dense(&m2.b0, Zc, p.ldW, T, (long long)p.NU * S))
@@ -1279,7 +1299,7 @@ jolt_status run_core(const Ctx& c, const bf16* Us, long long ldU, const bf16* Ws
     a2.ldc = p.ldC;
     a2.sC = (long long)p.rTmax * p.ldC;
     a2.status = c.status();
-    return umma_run(m2, a2, 1, c.st);
+    return umma_run(c, m2, a2, 1);
   }
   // Z = bf16(X_(D) W_s)   ((S T) x rDmax per unit)
   GemmParams z;

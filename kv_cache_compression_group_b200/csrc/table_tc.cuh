@@ -14,7 +14,8 @@
 //     that segment may start), add it to a running sum kept in registers, and evaluate the
 //     quantiser of every bit-width on rho = x' - running sum, block by block -- the
 //     arithmetic of table_kernel (kernels.cuh), which is why the two give the same entries.
-// x' (the tile rotated along the features) is formed once per CTA in shared memory.
+// x' (the tile rotated along the features) is formed once per CTA in shared memory by the
+// epilogue warps while the copy and MMA warps start on the first operands.
 //
 // Every mbarrier wait is bounded (umma::mbar_wait); a wait that gives up raises
 // DEV_ERR_TIMEOUT and the CTA stops issuing work, keeps its named-barrier schedule, and waits
@@ -55,15 +56,30 @@ struct TableTcArgs {
 };
 
 // the tile's rows rotated along the features into xs (fp32, pitch XS_LD): sign flip, the
-// Walsh-Hadamard butterflies in the order of fwht_regs (strides 1, 2, ..., 64), 1 / sqrt(D)
+// Walsh-Hadamard butterflies in the order of fwht_regs (strides 1, 2, ..., 64), 1 / sqrt(D).
+// Run by the NTHREADS epilogue threads (threads 0 .. NTHREADS-1) alone, synchronised by
+// named barrier 1, while the copy and MMA warps start on the operands.
 template <typename TX, int NTHREADS>
 __device__ __forceinline__ void ttc_rotate_tile(const TX* X, int T, int t0, const float* sig, float* xs) {
   using namespace ttc;
-  for (int idx = threadIdx.x; idx < ROWS * DIM; idx += NTHREADS) {
-    const int r = idx / DIM, d = idx - r * DIM, t = t0 + r;
-    xs[r * XS_LD + d] = t < T ? ld_as_float(X + (long long)t * DIM + d) * sig[d] : 0.f;
+  constexpr int V = 16 / sizeof(TX);   // elements per 16-byte load
+  for (int idx = threadIdx.x; idx < ROWS * DIM / V; idx += NTHREADS) {
+    const int r = idx / (DIM / V), d0 = (idx - r * (DIM / V)) * V, t = t0 + r;
+    float f[V];
+    if (t < T) {
+      const uint4 w = *reinterpret_cast<const uint4*>(X + (long long)t * DIM + d0);
+      const TX* e = reinterpret_cast<const TX*>(&w);
+#pragma unroll
+      for (int i = 0; i < V; ++i) f[i] = ld_as_float(e + i) * sig[d0 + i];
+    } else {
+#pragma unroll
+      for (int i = 0; i < V; ++i) f[i] = 0.f;
+    }
+#pragma unroll
+    for (int i = 0; i < V; i += 4)
+      *reinterpret_cast<float4*>(xs + r * XS_LD + d0 + i) = make_float4(f[i], f[i + 1], f[i + 2], f[i + 3]);
   }
-  __syncthreads();
+  asm volatile("bar.sync 1, %0;" ::"n"(NTHREADS) : "memory");
   if (threadIdx.x < ROWS) {
     float* row = xs + threadIdx.x * XS_LD;
 #pragma unroll 1
@@ -90,7 +106,7 @@ __device__ __forceinline__ void ttc_rotate_tile(const TX* X, int T, int t0, cons
       row[j + 64] = (a - b) * sc;
     }
   }
-  __syncthreads();
+  asm volatile("bar.sync 1, %0;" ::"n"(NTHREADS) : "memory");
 }
 
 __device__ __forceinline__ void ttc_tmem_ld16(uint32_t taddr, float* v) {
@@ -132,17 +148,14 @@ __device__ __forceinline__ float ttc_rcp_approx(float x) {
   return r;
 }
 
-// squared-error sums of one bit-width over one block, added into two packed partial sums
-// (a[0], a[1]) that run over all blocks of the thread for the current cut; a block whose
-// scale overflows fp16 makes the sums +inf
+// squared-error sums of one bit-width over one block, added into one packed partial sum `a`
+// that runs over all blocks of the thread for the current cut (the five bit-widths give the
+// scheduler independent chains); a block whose scale overflows fp16 makes the sums +inf
 template <int B>
-__device__ __forceinline__ void ttc_bit_error(const float2* v, const float2* d, float mx, float lo, float2* a) {
+__device__ __forceinline__ void ttc_bit_error(const float2* v, const float2* d, float mx, float lo, float2& a) {
   if constexpr (B == 0) {
 #pragma unroll
-    for (int j = 0; j < 8; j += 2) {
-      a[0] = __ffma2_rn(v[j], v[j], a[0]);
-      a[1] = __ffma2_rn(v[j + 1], v[j + 1], a[1]);
-    }
+    for (int j = 0; j < 8; ++j) a = __ffma2_rn(v[j], v[j], a);
   } else {
     constexpr float flev = (float)((1 << B) - 1);
     const float inv_lev = 1.0f / flev;
@@ -151,24 +164,20 @@ __device__ __forceinline__ void ttc_bit_error(const float2* v, const float2* d, 
     const float inv = step > 0.f ? ttc_rcp_approx(step) : 0.f;
     const float2 inv2 = make_float2(inv, inv), nstep2 = make_float2(-step, -step);
     const float2 sh = make_float2(kRoundShift, kRoundShift), nsh = make_float2(-kRoundShift, -kRoundShift);
-    float2 b0 = a[0], b1 = a[1];
+    float2 b0 = a;
 #pragma unroll
-    for (int j = 0; j < 8; j += 2) {
-      const float2 c0 = __fadd2_rn(__ffma2_rn(d[j], inv2, sh), nsh);
-      const float2 c1 = __fadd2_rn(__ffma2_rn(d[j + 1], inv2, sh), nsh);
-      const float2 e0 = __ffma2_rn(c0, nstep2, d[j]);
-      const float2 e1 = __ffma2_rn(c1, nstep2, d[j + 1]);
-      b0 = __ffma2_rn(e0, e0, b0);
-      b1 = __ffma2_rn(e1, e1, b1);
+    for (int j = 0; j < 8; ++j) {
+      const float2 c = __fadd2_rn(__ffma2_rn(d[j], inv2, sh), nsh);
+      const float2 e = __ffma2_rn(c, nstep2, d[j]);
+      b0 = __ffma2_rn(e, e, b0);
     }
-    a[0] = ok ? b0 : make_float2(INFINITY, INFINITY);
-    a[1] = ok ? b1 : make_float2(INFINITY, INFINITY);
+    a = ok ? b0 : make_float2(INFINITY, INFINITY);
   }
 }
 
 // every bit-width of the set for one block of rho given as 8 packed pairs
 template <int... Bs>
-__device__ __forceinline__ void ttc_block_errors(const float2* v, float2 (*acc)[2], BitSet<Bs...>) {
+__device__ __forceinline__ void ttc_block_errors(const float2* v, float2* acc, BitSet<Bs...>) {
   const float m0 = ttc_min3(v[0].x, v[0].y, v[1].x), m1 = ttc_min3(v[1].y, v[2].x, v[2].y);
   const float m2 = ttc_min3(v[3].x, v[3].y, v[4].x), m3 = ttc_min3(v[4].y, v[5].x, v[5].y);
   const float m4 = ttc_min3(v[6].x, v[6].y, v[7].x);
@@ -188,9 +197,11 @@ __device__ __forceinline__ void ttc_block_errors(const float2* v, float2 (*acc)[
 
 __device__ __forceinline__ void ttc_epi_sync() { asm volatile("bar.sync 1, %0;" ::"n"(ttc::EPI_WARPS * 32) : "memory"); }
 
-// grid (tiles, S, units); ttc::THREADS threads; ttc::SMEM bytes of dynamic shared memory
+// grid (tiles, S, units); ttc::THREADS threads; ttc::SMEM bytes of dynamic shared memory.
+// Registers: the SM's file is four partitions of 16K, one per scheduler, and the 18 warps put
+// five on one partition, so a thread gets at most 96 (the launch bound makes ptxas keep to it).
 template <typename TX, typename BITS>
-__global__ void __maxnreg__(112)
+__global__ void __launch_bounds__(ttc::THREADS, 1)
     table_tc_kernel(const __grid_constant__ CUtensorMap map_u, const __grid_constant__ CUtensorMap map_p,
                     TableTcArgs a) {
   using namespace ttc;
@@ -236,9 +247,6 @@ __global__ void __maxnreg__(112)
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
   for (int d = threadIdx.x; d < DIM; d += THREADS) sig[d] = rotation_sign(a.seed, u + a.cv.u0, d);
-  __syncthreads();
-  const TX* X = reinterpret_cast<const TX*>(a.cv.unit_ptr(u)) + (long long)s * T * DIM;
-  ttc_rotate_tile<TX, THREADS>(X, T, t0, sig, xs);
   umma::fence_before_sync();
   __syncthreads();
   umma::fence_after_sync();
@@ -312,6 +320,8 @@ __global__ void __maxnreg__(112)
     const BitConsts kb = bit_consts(cd);
     double* out = a.partial + (((long long)u * S + s) * a.tiles + tile) * (long long)(nD * nT * nB);
     const float* xrow = xs + row * XS_LD + cbase;
+    ttc_rotate_tile<TX, EPI_WARPS * 32>(reinterpret_cast<const TX*>(a.cv.unit_ptr(u)) + (long long)s * T * DIM, T,
+                                         t0, sig, xs);
     const float2 neg1 = make_float2(-1.f, -1.f);
     for (int iD = 0; iD < nD; ++iD) {
       float2 nrun[EPI_COLS / 2];   // minus the running sum of the finished segments
@@ -325,9 +335,9 @@ __global__ void __maxnreg__(112)
         float err[MAXC];
 #pragma unroll
         for (int b = 0; b < MAXC; ++b) err[b] = 0.f;
-        float2 acc2[MAXC][2];   // packed partial sums of the fixed bit set (horizontal sum per cut)
+        float2 acc2[MAXC];   // packed partial sums of the fixed bit set (horizontal sum per cut)
 #pragma unroll
-        for (int b = 0; b < MAXC; ++b) acc2[b][0] = acc2[b][1] = make_float2(0.f, 0.f);
+        for (int b = 0; b < MAXC; ++b) acc2[b] = make_float2(0.f, 0.f);
         if (ok) {
           umma::fence_after_sync();
 #pragma unroll
@@ -362,7 +372,7 @@ __global__ void __maxnreg__(112)
           }
           if constexpr (!std::is_same<BITS, void>::value) {
 #pragma unroll
-            for (int b = 0; b < BITS::N; ++b) err[b] = (acc2[b][0].x + acc2[b][0].y) + (acc2[b][1].x + acc2[b][1].y);
+            for (int b = 0; b < BITS::N; ++b) err[b] = acc2[b].x + acc2[b].y;
           }
         }
         // this cut's sums over the warp (every lane takes part, also after an abort)
@@ -426,7 +436,7 @@ struct EncodeTcArgs {
 };
 
 template <typename TX>
-__global__ void __maxnreg__(112)
+__global__ void __launch_bounds__(etc::THREADS, 1)
     encode_tc_kernel(const __grid_constant__ CUtensorMap map_u, const __grid_constant__ CUtensorMap map_p,
                      EncodeTcArgs a) {
   using namespace ttc;
@@ -473,9 +483,6 @@ __global__ void __maxnreg__(112)
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
   for (int d = threadIdx.x; d < DIM; d += etc::THREADS) sig[d] = rotation_sign(a.seed, u + a.cv.u0, d);
-  __syncthreads();
-  ttc_rotate_tile<TX, etc::THREADS>(reinterpret_cast<const TX*>(a.cv.unit_ptr(u)) + (long long)s * T * DIM, T, t0,
-                                   sig, xs);
   umma::fence_before_sync();
   __syncthreads();
   umma::fence_after_sync();
@@ -528,6 +535,8 @@ __global__ void __maxnreg__(112)
     const int row = 32 * (warp & 3) + lane;
     const int cbase = etc::COLS * (warp >> 2);
     const uint32_t lane_addr = (uint32_t)(32 * (warp & 3)) << 16;
+    ttc_rotate_tile<TX, etc::EPI_WARPS * 32>(reinterpret_cast<const TX*>(a.cv.unit_ptr(u)) + (long long)s * T * DIM,
+                                             T, t0, sig, xs);
     float hi[etc::COLS], lo[etc::COLS];
 #pragma unroll
     for (int j = 0; j < etc::COLS; ++j) {

@@ -8,8 +8,9 @@
 //   * one thread issues tcgen05.mma (M = 128, N = BN, K = 16, bf16 x bf16 -> fp32) with the
 //     accumulator in tensor memory; tcgen05.commit releases a shared-memory stage back to the
 //     copy thread through an mbarrier, so copies of later K blocks overlap the MMAs;
-//   * the epilogue reads the accumulator with tcgen05.ld (warp w owns TMEM lanes 32w..32w+31,
-//     i.e. output rows m0 + 32w + lane) and stores fp32 or bf16 rows.
+//   * persistent CTAs (one per SM) walk the output tiles; two TMEM accumulators alternate
+//     between tiles, so four epilogue warps read one (tcgen05.ld; warp w owns TMEM lanes
+//     32 (w % 4) .. +31) and store fp32 or bf16 rows while the MMAs of the next tile run.
 //
 // Each operand is a 128 (A) or BN (B) x 64 tile assembled from 64 x 64 boxes; the box
 // coordinates come from the operand's addressing mode, so the cache is read in place:
@@ -26,8 +27,8 @@
 // multiple of 64 (a 64-row box never straddles two units).
 //
 // Every mbarrier wait is bounded (about two seconds of global time); a wait that gives up
-// sets DEV_ERR_TIMEOUT in the status word, stops issuing work, and the CTA still waits for
-// its issued MMAs (through the final commit) before it frees its tensor memory.
+// sets DEV_ERR_TIMEOUT in the status word, every role stops, and the CTA still waits for
+// its issued MMAs (through a final commit) before it frees its tensor memory.
 #pragma once
 
 #include <cuda.h>
@@ -63,6 +64,7 @@ struct UmmaArgs {
   int bn = 0;                 // N tile: 0 chooses (256 when N > 128), else 128 or 256
   long long ldc = 0, sC = 0, ssplit = 0;   // row pitch, batch stride, split stride (elements)
   uint32_t* status = nullptr;
+  int* sched = nullptr;       // device int: the next output tile to hand out (zeroed before the launch)
 };
 
 namespace umma {
@@ -204,7 +206,7 @@ struct Cfg {
   static constexpr int STAGE_BYTES = A_BYTES + NB * B_BYTES;
   static constexpr int STAGES = (200 * 1024) / STAGE_BYTES > 6 ? 6 : (200 * 1024) / STAGE_BYTES;
   static constexpr int BAR_OFF = STAGES * STAGE_BYTES;
-  static constexpr int SMEM = BAR_OFF + 256 + 1024;    // barriers + TMEM address + alignment slack
+  static constexpr int SMEM = BAR_OFF + 512 + 1024;    // barriers, TMEM address, flag, tile ring + slack
   static_assert(STAGES >= 2, "pipeline needs two stages");
 };
 
@@ -249,41 +251,97 @@ __host__ __device__ __forceinline__ bool cache_mode(int mode) { return mode <= U
 
 }  // namespace umma
 
-// One CTA computes the 128 x BN output tile (m0, n0) of batch entry b (split sp of its K
-// range): C = A * sum_b B_b.  Grid: (N tiles, M tiles, batch * splits); 128 threads.
+// Persistent: grid = min(tiles, SMs).  The output tiles, in the order (batch entry and split,
+// M tile, N tile), N fastest, are handed out by an atomic counter, so CTAs that start late
+// (their SM busy with other work) take fewer tiles.  Tile (m0, n0) of batch entry b (split sp
+// of its K range) is C = A * sum_b B_b.  Six warps: warp 0 takes tiles from the counter,
+// passes their indices to the other roles through a ring in shared memory and issues the TMA
+// copies of every tile's K blocks through one ring of shared-memory stages (it runs ahead
+// across tile boundaries); warp 1 issues the MMAs into one of two TMEM accumulators
+// (alternating by tile); warps 2-5 (one per TMEM lane quarter) drain the other accumulator:
+// the epilogue of one tile overlaps the MMAs of the next.
+namespace umma {
+constexpr int RING = 4;   // tile indices in flight between the roles
+}
 template <int BN, int NB, bool A_MN, bool B_MN>
-__global__ void __launch_bounds__(128, 1)
+__global__ void __launch_bounds__(192, 1)
     umma_gemm_kernel(const __grid_constant__ CUtensorMap map_a0, const __grid_constant__ CUtensorMap map_a1,
                      const __grid_constant__ CUtensorMap map_b0, const __grid_constant__ CUtensorMap map_b1,
                      UmmaArgs a) {
   using C = umma::Cfg<BN, NB>;
+  using umma::RING;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  uint64_t* bars = (uint64_t*)(smem + C::BAR_OFF);  // full[STAGES], empty[STAGES], acc
-  uint32_t* tmem_slot = (uint32_t*)(bars + 2 * C::STAGES + 1);
+  // full[S] empty[S] accfull[2] accempty[2] done ringfull[RING] ringempty[RING]
+  uint64_t* bars = (uint64_t*)(smem + C::BAR_OFF);
+  uint32_t* tmem_slot = (uint32_t*)(bars + 2 * C::STAGES + 5 + 2 * RING);
+  volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
+  volatile int* ring = (volatile int*)(tmem_slot + 2);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n0 = blockIdx.x * BN, m0 = blockIdx.y * umma::BM;
-  if (a.tri == 1 && n0 + BN <= m0) return;   // wholly below the diagonal: not needed
-  const int bz = blockIdx.z / a.splits, sp = blockIdx.z - bz * a.splits;
-  const int kb0 = sp * (a.kchunk / umma::BK);
-  const int kend = min(a.tri == 2 ? min(a.K, n0 + BN) : a.K, (sp + 1) * a.kchunk);
-  const int nk = kend > kb0 * umma::BK ? (kend - kb0 * umma::BK + umma::BK - 1) / umma::BK : 0;
-  const uint32_t full0 = umma::smem_u32(bars), empty0 = full0 + 8 * C::STAGES, accb = full0 + 16 * C::STAGES;
+  const int tN = (a.N + BN - 1) / BN, tM = (a.M + umma::BM - 1) / umma::BM;
+  const int per = tN * tM, total = a.batch * a.splits * per;
+  const uint32_t full0 = umma::smem_u32(bars), empty0 = full0 + 8 * C::STAGES;
+  const uint32_t accfull0 = empty0 + 8 * C::STAGES, accempty0 = accfull0 + 16, done_bar = accempty0 + 16;
+  const uint32_t ringfull0 = done_bar + 8, ringempty0 = ringfull0 + 8 * RING;
   const bool b_is_a = a.b_is_a;
+  // tile t: batch entry bz, split sp, origin (m0, n0), K blocks [kb0, kb0 + nk)
+  auto tile = [&](int t, int& bz, int& sp, int& m0, int& n0, int& kb0, int& nk) -> bool {
+    const int zz = t / per, rem = t - zz * per;
+    bz = zz / a.splits;
+    sp = zz - bz * a.splits;
+    m0 = (rem / tN) * umma::BM;
+    n0 = (rem - (rem / tN) * tN) * BN;
+    if (a.tri == 1 && n0 + BN <= m0) return false;   // wholly below the diagonal: not needed
+    kb0 = sp * (a.kchunk / umma::BK);
+    const int kend = min(a.tri == 2 ? min(a.K, n0 + BN) : a.K, (sp + 1) * a.kchunk);
+    nk = kend > kb0 * umma::BK ? (kend - kb0 * umma::BK + umma::BK - 1) / umma::BK : 0;
+    return true;
+  };
+  // the next tile that is needed, or -1 when none is left
+  auto fetch = [&]() -> int {
+    int bz, sp, m0, n0, kb0, nk;
+    for (;;) {
+      const int t = atomicAdd(a.sched, 1);
+      if (t >= total) return -1;
+      if (tile(t, bz, sp, m0, n0, kb0, nk)) return t;
+    }
+  };
+  // the j-th tile index of the ring (all roles read the same sequence); -1: stop, -2: the wait
+  // gave up.  warp_wide: every lane of the warp calls it and gets the same answer.
+  auto ring_take = [&](int j, bool warp_wide) -> int {
+    const int slot = j % RING;
+    const bool ok = umma::mbar_wait(ringfull0 + 8 * slot, (j / RING) & 1);
+    int t = ok ? ring[slot] : -2;
+    if (warp_wide) {
+      if (!__all_sync(0xffffffffu, ok)) t = -2;
+      __syncwarp();   // every lane has read the slot before it is handed back
+    }
+    if (lane == 0 && ok) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(ringempty0 + 8 * slot) : "memory");
+    return t;
+  };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
       umma::mbar_init(full0 + 8 * s, 1);
       umma::mbar_init(empty0 + 8 * s, 1);
     }
-    umma::mbar_init(accb, 1);
+    for (int b = 0; b < 2; ++b) {
+      umma::mbar_init(accfull0 + 8 * b, 1);
+      umma::mbar_init(accempty0 + 8 * b, 4);
+    }
+    umma::mbar_init(done_bar, 1);
+    for (int r = 0; r < RING; ++r) {
+      umma::mbar_init(ringfull0 + 8 * r, 1);
+      umma::mbar_init(ringempty0 + 8 * r, 5);   // the MMA thread + the four epilogue warps
+    }
+    *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
   if (warp == 0) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                      umma::smem_u32(tmem_slot)),
-                 "r"(BN)
+                 "r"(2 * BN)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
@@ -291,138 +349,204 @@ __global__ void __launch_bounds__(128, 1)
   __syncthreads();
   umma::fence_after_sync();
   const uint32_t tmem = *tmem_slot;
-  bool ok = true;
 
-  if (warp == 0 && lane == 0) {
-    // ---- TMA producer ----
-    const int ea = bz / a.A.ediv, eb = bz / a.B.ediv;
-    const CUtensorMap* ma = (umma::cache_mode(a.A.mode) && (ea & 1)) ? &map_a1 : &map_a0;
-    const uint32_t bytes = b_is_a ? (uint32_t)C::A_BYTES : (uint32_t)C::STAGE_BYTES;
-    for (int i = 0; i < nk && ok; ++i) {
-      const int s = i % C::STAGES;
-      if (i >= C::STAGES && !umma::mbar_wait(empty0 + 8 * s, ((i / C::STAGES) & 1) ^ 1)) {
-        ok = false;
-        break;
-      }
-      const uint32_t fb = full0 + 8 * s;
-      const uint32_t sa = umma::smem_u32(smem + s * C::STAGE_BYTES);
-      const int k = (kb0 + i) * umma::BK;
-      umma::mbar_expect_tx(fb, bytes);
-      int c0, c1, c2;
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---- tile fetcher and TMA producer ----
+      int it = 0;
+      int next = fetch();
+      for (int j = 0;; ++j) {
+        const int t = *abort_flag ? -1 : next;
+        const int slot = j % RING;
+        if (j >= RING && !umma::mbar_wait(ringempty0 + 8 * slot, ((j / RING) & 1) ^ 1)) {
+          *abort_flag = 1;
+          break;
+        }
+        ring[slot] = t;
+        asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(ringfull0 + 8 * slot) : "memory");
+        if (t < 0) break;
+        next = fetch();   // its latency overlaps the copies below
+        int bz, sp, m0, n0, kb0, nk;
+        tile(t, bz, sp, m0, n0, kb0, nk);
+        const int ea = bz / a.A.ediv, eb = bz / a.B.ediv;
+        const CUtensorMap* ma = (umma::cache_mode(a.A.mode) && (ea & 1)) ? &map_a1 : &map_a0;
+        const uint32_t bytes = b_is_a ? (uint32_t)C::A_BYTES : (uint32_t)C::STAGE_BYTES;
+        for (int i = 0; i < nk; ++i, ++it) {
+          const int s = it % C::STAGES;
+          if (it >= C::STAGES && !umma::mbar_wait(empty0 + 8 * s, ((it / C::STAGES) & 1) ^ 1)) {
+            *abort_flag = 1;
+            break;
+          }
+          const uint32_t fb = full0 + 8 * s;
+          const uint32_t sa = umma::smem_u32(smem + s * C::STAGE_BYTES);
+          const int k = (kb0 + i) * umma::BK;
+          umma::mbar_expect_tx(fb, bytes);
+          int c0, c1, c2;
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        umma::box_coords(a.A, ea, m0 + 64 * h, k, c0, c1, c2);
-        umma::tma_load_3d(sa + h * umma::BOX_BYTES, ma, c0, c1, c2, fb);
-      }
-      if (!b_is_a) {
+          for (int h = 0; h < 2; ++h) {
+            umma::box_coords(a.A, ea, m0 + 64 * h, k, c0, c1, c2);
+            umma::tma_load_3d(sa + h * umma::BOX_BYTES, ma, c0, c1, c2, fb);
+          }
+          if (!b_is_a) {
 #pragma unroll
-        for (int b = 0; b < NB; ++b) {
-          const CUtensorMap* mb = umma::cache_mode(a.B.mode) ? ((eb & 1) ? &map_b1 : &map_b0) : (b ? &map_b1 : &map_b0);
-          const uint32_t sb = sa + C::A_BYTES + b * C::B_BYTES;
+            for (int b = 0; b < NB; ++b) {
+              const CUtensorMap* mb =
+                  umma::cache_mode(a.B.mode) ? ((eb & 1) ? &map_b1 : &map_b0) : (b ? &map_b1 : &map_b0);
+              const uint32_t sb = sa + C::A_BYTES + b * C::B_BYTES;
 #pragma unroll
-          for (int j = 0; j < BN / 64; ++j) {
-            umma::box_coords(a.B, eb, n0 + 64 * j, k, c0, c1, c2);
-            umma::tma_load_3d(sb + j * umma::BOX_BYTES, mb, c0, c1, c2, fb);
+              for (int jj = 0; jj < BN / 64; ++jj) {
+                umma::box_coords(a.B, eb, n0 + 64 * jj, k, c0, c1, c2);
+                umma::tma_load_3d(sb + jj * umma::BOX_BYTES, mb, c0, c1, c2, fb);
+              }
+            }
           }
         }
       }
     }
-  } else if (warp == 1 && lane == 0) {
-    // ---- MMA issuer ----
-    constexpr uint32_t idesc = umma::instr_desc(BN, A_MN, B_MN);
-    for (int i = 0; i < nk; ++i) {
-      const int s = i % C::STAGES;
-      if (!umma::mbar_wait(full0 + 8 * s, (i / C::STAGES) & 1)) {
-        ok = false;
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---- MMA issuer ----
+      constexpr uint32_t idesc = umma::instr_desc(BN, A_MN, B_MN);
+      int it = 0, tc = 0;
+      for (int j = 0;; ++j) {
+        const int t = ring_take(j, false);
+        if (t == -2) *abort_flag = 1;
+        if (t < 0) break;
+        int bz, sp, m0, n0, kb0, nk;
+        tile(t, bz, sp, m0, n0, kb0, nk);
+        const int buf = tc & 1, use = tc >> 1;
+        if (use > 0 && !umma::mbar_wait(accempty0 + 8 * buf, (use - 1) & 1)) {
+          *abort_flag = 1;
+          break;
+        }
+        umma::fence_after_sync();
+        const uint32_t acc = tmem + (uint32_t)(buf * BN);
+        bool ok = true;
+        for (int i = 0; i < nk; ++i, ++it) {
+          const int s = it % C::STAGES;
+          if (!umma::mbar_wait(full0 + 8 * s, (it / C::STAGES) & 1)) {
+            ok = false;
+            break;
+          }
+          umma::fence_after_sync();
+          const uint32_t sa = umma::smem_u32(smem + s * C::STAGE_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < umma::BK / 16; ++kk) {
+            // K step of 16: K-major advances 32 bytes inside the swizzle row, MN-major two
+            // 8-row groups (2 x 1024 bytes)
+            const uint64_t ad = A_MN ? umma::smem_desc(sa + kk * 2048, umma::BOX_BYTES, 1024)
+                                     : umma::smem_desc(sa + kk * 32, 16, 1024);
+#pragma unroll
+            for (int b = 0; b < NB; ++b) {
+              const uint32_t sb = b_is_a ? sa : sa + C::A_BYTES + b * C::B_BYTES;
+              const uint64_t bd = B_MN ? umma::smem_desc(sb + kk * 2048, umma::BOX_BYTES, 1024)
+                                       : umma::smem_desc(sb + kk * 32, 16, 1024);
+              umma::mma_bf16(acc, ad, bd, idesc, (i | kk | b) != 0);
+            }
+          }
+          umma::mma_commit(empty0 + 8 * s);
+        }
+        if (!ok) {
+          *abort_flag = 1;
+          break;
+        }
+        umma::mma_commit(accfull0 + 8 * buf);   // fires once this tile's MMAs have completed
+        ++tc;
+      }
+      umma::mma_commit(done_bar);
+    }
+  } else {
+    // ---- epilogue: warp w owns TMEM lanes 32 (w % 4) .. +31, i.e. output rows m0 + 32 (w % 4) + lane ----
+    const int q4 = warp & 3;
+    const int esz = a.c_bf16 ? 2 : 4;
+    const bool vec = ((a.ldc * esz) % 16 == 0) && ((((uintptr_t)a.C) & 15) == 0) && ((a.sC * esz) % 16 == 0) &&
+                     ((a.ssplit * esz) % 16 == 0);
+    int tc = 0;
+    for (int j = 0;; ++j) {
+      const int t = ring_take(j, true);
+      if (t == -2) *abort_flag = 1;
+      if (t < 0) break;
+      int bz, sp, m0, n0, kb0, nk;
+      tile(t, bz, sp, m0, n0, kb0, nk);
+      const int buf = tc & 1, use = tc >> 1;
+      bool ok = !*abort_flag && umma::mbar_wait(accfull0 + 8 * buf, use & 1);
+      ok = __all_sync(0xffffffffu, ok);   // the TMEM loads are warp-collective
+      if (!ok) {
+        *abort_flag = 1;
         break;
       }
       umma::fence_after_sync();
-      const uint32_t sa = umma::smem_u32(smem + s * C::STAGE_BYTES);
+      const int row = m0 + q4 * 32 + lane;
+      const long long off = (long long)bz * a.sC + (long long)sp * a.ssplit + (long long)row * a.ldc;
+#pragma unroll 1
+      for (int c0 = 0; c0 < BN; c0 += 32) {
+        float v[32];
+        umma::tmem_ld32(tmem + (uint32_t)(buf * BN) + ((uint32_t)(q4 * 32) << 16) + (uint32_t)c0, v);
+        if (c0 + 32 >= BN) {
+          // the accumulator is in registers: hand it back to the MMA warp
+          umma::fence_before_sync();
+          __syncwarp();
+          if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(accempty0 + 8 * buf) : "memory");
+        }
+        if (nk == 0) {  // an empty K range (a trailing split): its partial sum is zero
 #pragma unroll
-      for (int kk = 0; kk < umma::BK / 16; ++kk) {
-        // K step of 16: K-major advances 32 bytes inside the swizzle row, MN-major two
-        // 8-row groups (2 x 1024 bytes)
-        const uint64_t ad = A_MN ? umma::smem_desc(sa + kk * 2048, umma::BOX_BYTES, 1024)
-                                 : umma::smem_desc(sa + kk * 32, 16, 1024);
+          for (int j = 0; j < 32; ++j) v[j] = 0.f;
+        }
+        if (row >= a.M) continue;
+        const int n = n0 + c0;
+        if (a.c_bf16) {
+          bf16* crow = (bf16*)a.C + off;
+          if (vec && n + 32 <= a.N) {
 #pragma unroll
-        for (int b = 0; b < NB; ++b) {
-          const uint32_t sb = b_is_a ? sa : sa + C::A_BYTES + b * C::B_BYTES;
-          const uint64_t bd = B_MN ? umma::smem_desc(sb + kk * 2048, umma::BOX_BYTES, 1024)
-                                   : umma::smem_desc(sb + kk * 32, 16, 1024);
-          umma::mma_bf16(tmem, ad, bd, idesc, (i | kk | b) != 0);
+            for (int j = 0; j < 32; j += 8) {
+              uint4 w;
+              __nv_bfloat162 h0 = __floats2bfloat162_rn(v[j], v[j + 1]), h1 = __floats2bfloat162_rn(v[j + 2], v[j + 3]);
+              __nv_bfloat162 h2 = __floats2bfloat162_rn(v[j + 4], v[j + 5]), h3 = __floats2bfloat162_rn(v[j + 6], v[j + 7]);
+              w.x = *(uint32_t*)&h0;
+              w.y = *(uint32_t*)&h1;
+              w.z = *(uint32_t*)&h2;
+              w.w = *(uint32_t*)&h3;
+              *(uint4*)(crow + n + j) = w;
+            }
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (n + j < a.N) crow[n + j] = __float2bfloat16_rn(v[j]);
+          }
+        } else {
+          float* crow = (float*)a.C + off;
+          if (vec && n + 32 <= a.N) {
+#pragma unroll
+            for (int j = 0; j < 32; j += 4) {
+              float4 o = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+              if (a.c_accum) {
+                const float4 cc = *(const float4*)(crow + n + j);
+                o.x += cc.x;
+                o.y += cc.y;
+                o.z += cc.z;
+                o.w += cc.w;
+              }
+              *(float4*)(crow + n + j) = o;
+            }
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (n + j < a.N) crow[n + j] = a.c_accum ? crow[n + j] + v[j] : v[j];
+          }
         }
       }
-      umma::mma_commit(empty0 + 8 * s);
+      ++tc;
     }
-    umma::mma_commit(accb);  // fires once every MMA issued above has completed
   }
   __syncwarp();
-
-  // ---- epilogue: all four warps ----
-  const bool acc_ok = umma::mbar_wait(accb, 0);
-  umma::fence_after_sync();
-  const int row = m0 + warp * 32 + lane;
-  const long long off = (long long)bz * a.sC + (long long)sp * a.ssplit + (long long)row * a.ldc;
-  const int esz = a.c_bf16 ? 2 : 4;
-  const bool vec = ((a.ldc * esz) % 16 == 0) && ((((uintptr_t)a.C) & 15) == 0) && ((a.sC * esz) % 16 == 0) &&
-                   ((a.ssplit * esz) % 16 == 0);
-#pragma unroll 1
-  for (int c0 = 0; c0 < BN; c0 += 32) {
-    float v[32];
-    umma::tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)c0, v);
-    if (nk == 0) {  // an empty K range (a trailing split): its partial sum is zero
-#pragma unroll
-      for (int j = 0; j < 32; ++j) v[j] = 0.f;
-    }
-    if (!acc_ok || row >= a.M) continue;
-    const int n = n0 + c0;
-    if (a.c_bf16) {
-      bf16* crow = (bf16*)a.C + off;
-      if (vec && n + 32 <= a.N) {
-#pragma unroll
-        for (int j = 0; j < 32; j += 8) {
-          uint4 w;
-          __nv_bfloat162 h0 = __floats2bfloat162_rn(v[j], v[j + 1]), h1 = __floats2bfloat162_rn(v[j + 2], v[j + 3]);
-          __nv_bfloat162 h2 = __floats2bfloat162_rn(v[j + 4], v[j + 5]), h3 = __floats2bfloat162_rn(v[j + 6], v[j + 7]);
-          w.x = *(uint32_t*)&h0;
-          w.y = *(uint32_t*)&h1;
-          w.z = *(uint32_t*)&h2;
-          w.w = *(uint32_t*)&h3;
-          *(uint4*)(crow + n + j) = w;
-        }
-      } else {
-#pragma unroll
-        for (int j = 0; j < 32; ++j)
-          if (n + j < a.N) crow[n + j] = __float2bfloat16_rn(v[j]);
-      }
-    } else {
-      float* crow = (float*)a.C + off;
-      if (vec && n + 32 <= a.N) {
-#pragma unroll
-        for (int j = 0; j < 32; j += 4) {
-          float4 o = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
-          if (a.c_accum) {
-            const float4 c = *(const float4*)(crow + n + j);
-            o.x += c.x;
-            o.y += c.y;
-            o.z += c.z;
-            o.w += c.w;
-          }
-          *(float4*)(crow + n + j) = o;
-        }
-      } else {
-#pragma unroll
-        for (int j = 0; j < 32; ++j)
-          if (n + j < a.N) crow[n + j] = a.c_accum ? crow[n + j] + v[j] : v[j];
-      }
-    }
-  }
-  if ((!ok || !acc_ok) && a.status) atomicOr(a.status, DEV_ERR_TIMEOUT);
+  // every issued MMA has completed before tensor memory is freed
+  const bool drained = umma::mbar_wait(done_bar, 0);
+  if ((*abort_flag || !drained) && threadIdx.x == 0 && a.status) atomicOr(a.status, DEV_ERR_TIMEOUT);
   umma::fence_before_sync();
   __syncthreads();
   if (warp == 0) {
     umma::fence_after_sync();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(BN) : "memory");
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(2 * BN) : "memory");
   }
 }
 
@@ -483,9 +607,15 @@ cudaError_t launch_umma_t(const UmmaMaps& m, const UmmaArgs& a, cudaStream_t st)
   cudaError_t e = cudaFuncSetAttribute(umma_gemm_kernel<BN, NB, A_MN, B_MN>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  dim3 grid((unsigned)ceil_div(a.N, BN), (unsigned)ceil_div(a.M, umma::BM), (unsigned)(a.batch * a.splits));
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const long long tiles = ceil_div(a.N, BN) * ceil_div(a.M, umma::BM) * (long long)a.batch * a.splits;
+  if (tiles <= 0 || !a.sched) return cudaErrorInvalidValue;
+  const unsigned grid = (unsigned)(tiles < sms ? tiles : sms);
+  e = cudaMemsetAsync(a.sched, 0, sizeof(int), st);
+  if (e != cudaSuccess) return e;
   count_launch();
-  umma_gemm_kernel<BN, NB, A_MN, B_MN><<<grid, 128, smem, st>>>(m.a0, m.a1, m.b0, m.b1, a);
+  umma_gemm_kernel<BN, NB, A_MN, B_MN><<<grid, 192, smem, st>>>(m.a0, m.a1, m.b0, m.b1, a);
   return cudaGetLastError();
 }
 
@@ -518,7 +648,7 @@ inline cudaError_t launch_umma(const UmmaMaps& m, UmmaArgs a, int nb, cudaStream
 // xk / xv: the K and V caches [n_layers][H][T][D] bf16; F1 may be null (one B operand).
 inline cudaError_t umma_x_product(const void* xk, const void* xv, int n_layers, int H, int T, int D, int S,
                                   int nunits, bool z_side, const bf16* F0, const bf16* F1, int ldf, int N, float* C,
-                                  long long ldc, uint32_t* status, cudaStream_t st) {
+                                  long long ldc, uint32_t* status, int* sched, cudaStream_t st) {
   if (D % 64 || ldf % 8 || N > ldf) return cudaErrorInvalidValue;
   int dshift = 0;
   while ((1 << dshift) < D) ++dshift;
@@ -541,6 +671,7 @@ inline cudaError_t umma_x_product(const void* xk, const void* xv, int n_layers, 
   a.ldc = ldc;
   a.sC = (long long)a.M * ldc;
   a.status = status;
+  a.sched = sched;
   return launch_umma(m, a, F1 ? 2 : 1, st);
 }
 

@@ -2,15 +2,19 @@
 seeded inputs.  Tolerances:
   factor subspaces        : largest principal-angle sine <= 1e-3 where the relative eigengap
                             at the cut is >= 1e-4 (elsewhere the subspace is not determined)
-  stored core             : <= 1e-2 of entries differ, each by at most one bf16 step
-  reconstruction operator : same bound as the core (bf16 rounding of fp32 vs fp64 sums)
+  stored core             : <= 5e-2 of entries differ, each by at most one bf16 step plus four
+                            flips of a bf16 rounding of Z = bf16(X W) (two rounding points of
+                            fp32 vs fp64 sums; entries near cancellation flip)
+  reconstruction operator : formed in fp64 and rounded once: equal to the oracle's except at a
+                            tie closer than fp64 resolution (<= 1e-6 of entries, one bf16 step)
   distortion table        : 1e-6 relative + 2 sqrt(entry) * 64 u_32 ||X|| (fp32 residual vs fp64)
   block scales            : equal, except where the oracle's block minimum / maximum lies within
                             w = 2^-17 (max|x'| + max|x_hat|) of an fp16 rounding boundary (the
                             fp32 residual's absolute error); then the library's scale must be
                             the rounding of a value inside that window
-  codes                   : <= 1e-4 of codes differ (under the library's scales), and only where
-                            the oracle's scaled value lies within w / step of a rounding tie
+  codes                   : <= 1e-4 of codes differ from the oracle's own codes (its scales,
+                            its operator); under the library's scales every differing code lies
+                            within w / step of a rounding tie
   allocation              : bit-exact choices and lambda given identical tables
   end to end              : relative Frobenius error within 1e-4 absolute of the oracle's
 """
