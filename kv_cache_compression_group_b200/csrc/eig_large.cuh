@@ -7,9 +7,9 @@
 //      columns c with c % 8 == q (contiguous in the column-major matrix).  Per column j: the
 //      owner forms the reflector and writes it into every CTA's shared memory (distributed
 //      shared memory) and to global memory; every CTA computes p = beta A v on its columns
-//      (one warp per column) and sends p and its warps' partial p.v to all; every CTA applies
-//      the rank-2 update to its columns.  Two cluster barriers per column; vectors alternate
-//      between two buffers (as in eig_cluster.cuh).
+//      (one warp per column), applying the previous step's rank-2 update to the column in the
+//      same pass, and sends p and its warps' partial p.v to all.  Two cluster barriers per
+//      column; vectors alternate between two buffers (as in eig_cluster.cuh).
 //   2. tri_eig_kernel: 128 eigenvalues per CTA by multisection (8 threads each), then their
 //      eigenvectors of T by inverse iteration (one thread each, the factors in global memory).
 //   3. tight_mgs_kernel: vectors of eigenvalues closer than 1e-10 ||T|| orthonormalised in
@@ -75,6 +75,12 @@ __global__ void symmetrize_lower_kernel(double* A, int n, long long sA) {
 
 // grid (8 * matrices), clusters of 8, eigl::TRI_THREADS threads, eigl::TRI_SMEM dynamic shared
 // memory.  A: n x n symmetric, column-major (both triangles), stride sA, overwritten.
+//
+// Look-ahead order: the rank-2 update of step j - 1, A -= v w^T + w v^T, is not applied in a
+// pass of its own; at step j the owner of column j first applies it to that column and forms
+// the reflector v_j from it, and then every CTA applies it to each of its columns c > j in the
+// same pass over the column that forms p_c = beta_j (column c) . v_j.  One read and one write
+// of the trailing matrix per step, two cluster barriers.
 __global__ void __cluster_dims__(eigl::CL, 1, 1) __launch_bounds__(eigl::TRI_THREADS)
     tridiag_gm_kernel(double* A, int n, long long sA, double* scr) {
   using namespace eigl;
@@ -83,8 +89,8 @@ __global__ void __cluster_dims__(eigl::CL, 1, 1) __launch_bounds__(eigl::TRI_THR
   const int u = blockIdx.x / CL;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   extern __shared__ double tg_sm[];
-  double* vb = tg_sm;                     // [2][MAXN]
-  double* pb = vb + 2 * MAXN;             // [2][MAXN]
+  double* vb = tg_sm;                     // [2][MAXN] reflectors v_j (by the parity of j)
+  double* pb = vb + 2 * MAXN;             // [2][MAXN] p_j
   double* red = pb + 2 * MAXN;            // [2][TRED]
   double* sbeta = red + 2 * TRED;         // [2]
   double* tmp = sbeta + 2;                // [TRI_WARPS]
@@ -96,11 +102,19 @@ __global__ void __cluster_dims__(eigl::CL, 1, 1) __launch_bounds__(eigl::TRI_THR
   double* bg = eg + n;
   for (int i = tid; i < 4 * MAXN; i += blockDim.x) tg_sm[i] = 0.0;
   cluster.sync();
+  double Kp = 0.0;   // K of the previous step (the same in every thread)
   for (int j = 0; j + 2 < n; ++j) {
-    const int buf = j & 1;
+    const int cur = j & 1, prv = cur ^ 1;
+    const double* vp = vb + prv * MAXN;   // v_{j-1} (zero at j = 0)
+    const double* pp = pb + prv * MAXN;   // p_{j-1} (zero at j = 0)
     if (j % CL == q) {
-      // the reflector of column j (rows j+1 .. n-1); every thread takes part in the sums
-      const double* col = Au + (long long)j * n;
+      // column j brought up to date (update j - 1 on rows >= j), then its reflector
+      double* col = Au + (long long)j * n;
+      if (j > 0) {
+        const double vj = vp[j], wj = fma(-Kp, vj, pp[j]);
+        for (int r = j + tid; r < n; r += blockDim.x) col[r] = col[r] - (vp[r] * wj + fma(-Kp, vp[r], pp[r]) * vj);
+        __syncthreads();
+      }
       double part = 0.0;
       for (int r = j + 2 + tid; r < n; r += blockDim.x) part = fma(col[r], col[r], part);
       const double tail2 = eigl_block_sum(part, tmp);
@@ -114,29 +128,50 @@ __global__ void __cluster_dims__(eigl::CL, 1, 1) __launch_bounds__(eigl::TRI_THR
       }
       for (int r = tid; r < MAXN; r += blockDim.x) {
         const double v = (r <= j || r >= n) ? 0.0 : (r == j + 1 ? x0 - alpha : col[r]);
-        for (int t = 0; t < CL; ++t) cluster.map_shared_rank(vb, t)[buf * MAXN + r] = v;
+        for (int t = 0; t < CL; ++t) cluster.map_shared_rank(vb, t)[cur * MAXN + r] = v;
         if (r < n) refl[(long long)j * n + r] = v;
       }
       if (tid == 0) {
-        for (int t = 0; t < CL; ++t) cluster.map_shared_rank(sbeta, t)[buf] = beta;
+        for (int t = 0; t < CL; ++t) cluster.map_shared_rank(sbeta, t)[cur] = beta;
         dg[j] = col[j];
         eg[j] = alpha;
         bg[j] = beta;
       }
     }
-    cluster.sync();   // (A) v and beta everywhere
-    const double beta = sbeta[buf];
-    const double* v = vb + buf * MAXN;
+    cluster.sync();   // (A) v_j and beta_j everywhere
+    const double beta = sbeta[cur];
+    const double* v = vb + cur * MAXN;
     // my first column after j (the columns c with c % CL == q), then every CL-th; warp w takes
-    // the columns cf + CL (w + TRI_WARPS i)
+    // the columns cf + CL (w + TRI_WARPS i); one warp per column, lanes over rows
     const int cf = j + 1 + ((q - (j + 1)) % CL + CL) % CL;
-    if (beta != 0.0) {
-      // p_c = beta * (column c) . v: one warp per column, lanes over rows, four partial sums
-      double pv = 0.0;
-      for (int c = cf + CL * warp; c < n; c += CL * TRI_WARPS) {
-        const double* col = Au + (long long)c * n;
-        double s0 = 0.0, s1 = 0.0, s2 = 0.0, s3 = 0.0;
-        int r = j + 1 + lane;
+    double pv = 0.0;
+    for (int c = cf + CL * warp; c < n; c += CL * TRI_WARPS) {
+      double* col = Au + (long long)c * n;
+      const double vc = vp[c], wc = fma(-Kp, vc, pp[c]);
+      double s0 = 0.0, s1 = 0.0, s2 = 0.0, s3 = 0.0;
+      int r = j + 1 + lane;
+      if (j > 0) {
+        for (; r + 96 < n; r += 128) {
+          const double a0 = col[r], a1 = col[r + 32], a2 = col[r + 64], a3 = col[r + 96];
+          const double b0 = a0 - (vp[r] * wc + fma(-Kp, vp[r], pp[r]) * vc);
+          const double b1 = a1 - (vp[r + 32] * wc + fma(-Kp, vp[r + 32], pp[r + 32]) * vc);
+          const double b2 = a2 - (vp[r + 64] * wc + fma(-Kp, vp[r + 64], pp[r + 64]) * vc);
+          const double b3 = a3 - (vp[r + 96] * wc + fma(-Kp, vp[r + 96], pp[r + 96]) * vc);
+          col[r] = b0;
+          col[r + 32] = b1;
+          col[r + 64] = b2;
+          col[r + 96] = b3;
+          s0 = fma(b0, v[r], s0);
+          s1 = fma(b1, v[r + 32], s1);
+          s2 = fma(b2, v[r + 64], s2);
+          s3 = fma(b3, v[r + 96], s3);
+        }
+        for (; r < n; r += 32) {
+          const double b0 = col[r] - (vp[r] * wc + fma(-Kp, vp[r], pp[r]) * vc);
+          col[r] = b0;
+          s0 = fma(b0, v[r], s0);
+        }
+      } else {
         for (; r + 96 < n; r += 128) {
           s0 = fma(col[r], v[r], s0);
           s1 = fma(col[r + 32], v[r + 32], s1);
@@ -144,32 +179,32 @@ __global__ void __cluster_dims__(eigl::CL, 1, 1) __launch_bounds__(eigl::TRI_THR
           s3 = fma(col[r + 96], v[r + 96], s3);
         }
         for (; r < n; r += 32) s0 = fma(col[r], v[r], s0);
-        const double pc = beta * eigc::warp_sum((s0 + s1) + (s2 + s3));
-        if (lane < CL) cluster.map_shared_rank(pb, lane)[buf * MAXN + c] = pc;
-        pv = fma(pc, v[c], pv);   // the same on every lane
       }
-      if (lane < CL) cluster.map_shared_rank(red, lane)[buf * TRED + q * TRI_WARPS + warp] = pv;
+      const double pc = beta * eigc::warp_sum((s0 + s1) + (s2 + s3));
+      if (lane < CL) cluster.map_shared_rank(pb, lane)[cur * MAXN + c] = pc;
+      pv = fma(pc, v[c], pv);   // the same on every lane
     }
-    cluster.sync();   // (B) p and the partial sums of p.v everywhere
-    if (beta != 0.0) {
-      // p.v over the cluster's warps, in the same order in every warp of every CTA
-      double ptv = 0.0;
+    if (lane < CL) cluster.map_shared_rank(red, lane)[cur * TRED + q * TRI_WARPS + warp] = pv;
+    cluster.sync();   // (B) p_j and the partial sums of p_j . v_j everywhere
+    // K_j = beta_j p_j . v_j / 2, summed in the same order in every warp of every CTA
+    double ptv = 0.0;
 #pragma unroll
-      for (int t = 0; t < TRED / 32; ++t) ptv += red[buf * TRED + lane * (TRED / 32) + t];
-      ptv = eigc::warp_sum(ptv);
-      const double K = 0.5 * beta * ptv;
-      const double* pf = pb + buf * MAXN;
-      // A -= v w^T + w v^T on my columns, w = p - K v; one warp per column, lanes over rows
-      for (int c = cf + CL * warp; c < n; c += CL * TRI_WARPS) {
-        double* col = Au + (long long)c * n;
-        const double vc = v[c], wc = fma(-K, vc, pf[c]);
-#pragma unroll 4
-        for (int r = j + 1 + lane; r < n; r += 32) col[r] = col[r] - (v[r] * wc + fma(-K, v[r], pf[r]) * vc);
-      }
+    for (int t = 0; t < TRED / 32; ++t) ptv += red[cur * TRED + lane * (TRED / 32) + t];
+    Kp = 0.5 * beta * eigc::warp_sum(ptv);
+  }
+  // the last update on the last two columns, then the last 2 x 2 block of T
+  {
+    const int jl = n - 3, cur = jl & 1;
+    const double* vp = vb + cur * MAXN;
+    const double* pp = pb + cur * MAXN;
+    for (int c = n - 2; c < n; ++c) {
+      if (c % CL != q) continue;
+      double* col = Au + (long long)c * n;
+      const double vc = vp[c], wc = fma(-Kp, vc, pp[c]);
+      for (int r = n - 2 + tid; r < n; r += blockDim.x) col[r] = col[r] - (vp[r] * wc + fma(-Kp, vp[r], pp[r]) * vc);
     }
     __syncthreads();
   }
-  // the last 2 x 2 block of T
   if (tid == 0) {
     const int c2 = n - 2, c1 = n - 1;
     if (c2 % CL == q) {

@@ -275,14 +275,14 @@ jolt_status make_plan(const jolt_shape* sh, const jolt_options* op, Plan* p) {
   if (p->gt_split > 64) p->gt_split = 64;
 
   const int NU = p->NU, T = p->T, S = p->S, M = p->M;
-  // Cholesky-QR Grams: split-K so every fp32 partial sums at most 256 terms
+  // Cholesky-QR Grams: split-K partials in fp32, summed in fp64
   {
     long long mrows = op->method == JOLT_RANDOMIZED ? (M > T ? M : T) : (p->m_side ? T : 0);
     const int kq = op->method == JOLT_RANDOMIZED ? (int)round_up(p->rTmax + op->oversample, 8) : p->rTmax;
     if (kq >= QR_TC_MINK) {
-      // tensor-core Grams: two products x split-K chunks of QR_TC_CHUNK rows; the
-      // Rayleigh-Ritz Gram (M rows, chunks of 256) shares the buffer
-      long long need = 2 * ceil_div(mrows, QR_TC_CHUNK);
+      // tensor-core Grams: split-K chunks of QR_TC_CHUNK rows; the Rayleigh-Ritz Gram (M rows,
+      // chunks of 256) shares the buffer
+      long long need = ceil_div(mrows, QR_TC_CHUNK);
       if (op->method == JOLT_RANDOMIZED && ceil_div(M, 256) > need) need = ceil_div(M, 256);
       p->qr_split_max = mrows > 0 ? (int)need : 1;
     } else {
@@ -781,7 +781,7 @@ jolt_status cholqr_tc(const Ctx& c, float* Y, long long m, int k, int ld, int pa
   const int gld = ld, kq32 = (int)round_up(k, 32), nbk = (int)ceil_div(k, 32);
   const long long sG = (long long)k * gld, sW = (long long)kq32 * kq32;
   const int ns = (int)ceil_div(m, QR_TC_CHUNK);
-  if (2 * ns > p.qr_split_max) return fail(JOLT_ERR_WORKSPACE_TOO_SMALL, "Gram partial slots");
+  if (ns > p.qr_split_max) return fail(JOLT_ERR_WORKSPACE_TOO_SMALL, "Gram partial slots");
   const long long nY = (long long)p.NU * m * ld;
   UmmaMaps my, mw;
   if (!map_dense(&my.a0, yh, ld, m, p.NU) || !map_dense(&my.a1, yl, ld, m, p.NU) ||
@@ -806,21 +806,17 @@ jolt_status cholqr_tc(const Ctx& c, float* Y, long long m, int k, int ld, int pa
       g.bn = 128;
       g.C = gpart;
       g.ldc = gld;
-      g.sC = (long long)2 * ns * k * gld;
+      g.sC = (long long)ns * k * gld;
       g.ssplit = (long long)k * gld;
       g.status = c.status();
-      UmmaMaps m1;   // Yh^T (Yh + Yl)
-      m1.a0 = m1.a1 = my.a0;
-      m1.b0 = my.a0;
-      m1.b1 = my.a1;
-      JTRY(umma_run(c, m1, g, 2));
-      UmmaMaps m2;   // Yl^T Yh
-      m2.a0 = m2.a1 = my.a1;
-      m2.b0 = m2.b1 = my.a0;
-      g.C = gpart + (long long)ns * k * gld;
-      JTRY(umma_run(c, m2, g, 1));
+      UmmaMaps m3;   // Yh^T Yh + Yh^T Yl + Yl^T Yh in one pass
+      m3.a0 = my.a0;
+      m3.a1 = my.a1;
+      m3.b0 = my.a0;
+      m3.b1 = my.a1;
+      JTRY(umma_run(c, m3, g, 3));
       count_launch(), reduce_upper_sym_kernel<<<grid1d((long long)p.NU * k * k), 256, 0, c.st>>>(gpart, G, p.NU,
-                                                                                                  2 * ns, k, gld);
+                                                                                                  ns, k, gld);
       CUDA_TRY(cudaGetLastError());
     }
     {
@@ -867,16 +863,12 @@ jolt_status cholqr_tc(const Ctx& c, float* Y, long long m, int k, int ld, int pa
       q.ldc = ld;
       q.sC = m * ld;
       q.status = c.status();
-      UmmaMaps m1;   // Yh (Wh + Wl)^T
-      m1.a0 = m1.a1 = my.a0;
-      m1.b0 = mw.b0;
-      m1.b1 = mw.b1;
-      JTRY(umma_run(c, m1, q, 2));
-      UmmaMaps m2;   // + Yl Wh^T
-      m2.a0 = m2.a1 = my.a1;
-      m2.b0 = m2.b1 = mw.b0;
-      q.c_accum = 1;
-      JTRY(umma_run(c, m2, q, 1));
+      UmmaMaps m3;   // Yh Wh^T + Yh Wl^T + Yl Wh^T in one pass
+      m3.a0 = my.a0;
+      m3.a1 = my.a1;
+      m3.b0 = mw.b0;
+      m3.b1 = mw.b1;
+      JTRY(umma_run(c, m3, q, 3));
     }
   }
   return JOLT_OK;
@@ -1194,16 +1186,12 @@ jolt_status run_token_randomized(const Ctx& c, float* Uf, long long ldUf) {
     a.ldc = ldUf;
     a.sC = (long long)T * ldUf;
     a.status = c.status();
-    UmmaMaps m1;
-    m1.a0 = m1.a1 = mq.a0;
-    m1.b0 = mv.b0;
-    m1.b1 = mv.b1;
-    JTRY(umma_run(c, m1, a, 2));
-    UmmaMaps m2;
-    m2.a0 = m2.a1 = mq.a1;
-    m2.b0 = m2.b1 = mv.b0;
-    a.c_accum = 1;
-    JTRY(umma_run(c, m2, a, 1));
+    UmmaMaps m3;   // Qh Vh + Qh Vl + Ql Vh in one pass
+    m3.a0 = mq.a0;
+    m3.a1 = mq.a1;
+    m3.b0 = mv.b0;
+    m3.b1 = mv.b1;
+    JTRY(umma_run(c, m3, a, 3));
     return JOLT_OK;
   }
   GemmParams uq;

@@ -199,11 +199,15 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// NB = 1: C = A B; NB = 2: C = A (B0 + B1); NB = 3: C = A0 B0 + A0 B1 + A1 B0 (the products of
+// fp32 operands split as bf16 hi + lo, without the lo * lo term)
 template <int BN, int NB>
 struct Cfg {
+  static constexpr int NA_OP = NB == 3 ? 2 : 1;        // A operands in a stage
+  static constexpr int NB_OP = NB == 3 ? 2 : NB;       // B operands in a stage
   static constexpr int A_BYTES = BM * BK * 2;          // 16 KB
   static constexpr int B_BYTES = BN * BK * 2;          // BN/64 boxes
-  static constexpr int STAGE_BYTES = A_BYTES + NB * B_BYTES;
+  static constexpr int STAGE_BYTES = NA_OP * A_BYTES + NB_OP * B_BYTES;
   static constexpr int STAGES = (200 * 1024) / STAGE_BYTES > 6 ? 6 : (200 * 1024) / STAGE_BYTES;
   static constexpr int BAR_OFF = STAGES * STAGE_BYTES;
   static constexpr int SMEM = BAR_OFF + 512 + 1024;    // barriers, TMEM address, flag, tile ring + slack
@@ -386,13 +390,14 @@ __global__ void __launch_bounds__(192, 1)
           for (int h = 0; h < 2; ++h) {
             umma::box_coords(a.A, ea, m0 + 64 * h, k, c0, c1, c2);
             umma::tma_load_3d(sa + h * umma::BOX_BYTES, ma, c0, c1, c2, fb);
+            if constexpr (C::NA_OP == 2) umma::tma_load_3d(sa + C::A_BYTES + h * umma::BOX_BYTES, &map_a1, c0, c1, c2, fb);
           }
           if (!b_is_a) {
 #pragma unroll
-            for (int b = 0; b < NB; ++b) {
+            for (int b = 0; b < C::NB_OP; ++b) {
               const CUtensorMap* mb =
                   umma::cache_mode(a.B.mode) ? ((eb & 1) ? &map_b1 : &map_b0) : (b ? &map_b1 : &map_b0);
-              const uint32_t sb = sa + C::A_BYTES + b * C::B_BYTES;
+              const uint32_t sb = sa + C::NA_OP * C::A_BYTES + b * C::B_BYTES;
 #pragma unroll
               for (int jj = 0; jj < BN / 64; ++jj) {
                 umma::box_coords(a.B, eb, n0 + 64 * jj, k, c0, c1, c2);
@@ -437,11 +442,20 @@ __global__ void __launch_bounds__(192, 1)
             const uint64_t ad = A_MN ? umma::smem_desc(sa + kk * 2048, umma::BOX_BYTES, 1024)
                                      : umma::smem_desc(sa + kk * 32, 16, 1024);
 #pragma unroll
-            for (int b = 0; b < NB; ++b) {
-              const uint32_t sb = b_is_a ? sa : sa + C::A_BYTES + b * C::B_BYTES;
+            for (int b = 0; b < C::NB_OP; ++b) {
+              const uint32_t sb = b_is_a ? sa : sa + C::NA_OP * C::A_BYTES + b * C::B_BYTES;
               const uint64_t bd = B_MN ? umma::smem_desc(sb + kk * 2048, umma::BOX_BYTES, 1024)
                                        : umma::smem_desc(sb + kk * 32, 16, 1024);
               umma::mma_bf16(acc, ad, bd, idesc, (i | kk | b) != 0);
+            }
+            if constexpr (C::NA_OP == 2) {
+              // A1 B0
+              const uint32_t sa1 = sa + C::A_BYTES, sb0 = sa + 2 * C::A_BYTES;
+              const uint64_t ad1 = A_MN ? umma::smem_desc(sa1 + kk * 2048, umma::BOX_BYTES, 1024)
+                                        : umma::smem_desc(sa1 + kk * 32, 16, 1024);
+              const uint64_t bd0 = B_MN ? umma::smem_desc(sb0 + kk * 2048, umma::BOX_BYTES, 1024)
+                                        : umma::smem_desc(sb0 + kk * 32, 16, 1024);
+              umma::mma_bf16(acc, ad1, bd0, idesc, 1u);
             }
           }
           umma::mma_commit(empty0 + 8 * s);
@@ -627,16 +641,19 @@ cudaError_t launch_umma_bn(const UmmaMaps& m, const UmmaArgs& a, cudaStream_t st
   return bmn ? launch_umma_t<BN, NB, false, true>(m, a, st) : launch_umma_t<BN, NB, false, false>(m, a, st);
 }
 
-// C = A * sum_{b < nb} B_b on the tensor cores.  nb = 2 requires dense B operands (maps b0,
-// b1); b_is_a requires M = N <= 128 and identical A and B operands.
+// C = A * sum_{b < nb} B_b on the tensor cores (nb = 1, 2), or C = A0 B0 + A0 B1 + A1 B0
+// (nb = 3; maps a0, a1, b0, b1; N tiles of 128).  nb >= 2 requires dense B operands, nb = 3
+// dense A operands too; b_is_a requires M = N <= 128 and identical A and B operands.
 inline cudaError_t launch_umma(const UmmaMaps& m, UmmaArgs a, int nb, cudaStream_t st) {
-  if (a.splits < 1 || (a.splits > 1 && (a.kchunk <= 0 || a.kchunk % umma::BK)) || a.batch < 1 || nb < 1 || nb > 2 ||
-      (nb == 2 && umma::cache_mode(a.B.mode)) || (a.b_is_a && (a.M > 128 || a.N > 128 || nb != 1)))
+  if (a.splits < 1 || (a.splits > 1 && (a.kchunk <= 0 || a.kchunk % umma::BK)) || a.batch < 1 || nb < 1 || nb > 3 ||
+      (nb >= 2 && umma::cache_mode(a.B.mode)) || (nb == 3 && (umma::cache_mode(a.A.mode) || a.b_is_a)) ||
+      (a.b_is_a && (a.M > 128 || a.N > 128 || nb != 1)))
     return cudaErrorInvalidValue;
   if (a.splits == 1) a.kchunk = (int)round_up(a.K, umma::BK);
   if (a.c_accum && a.c_bf16) return cudaErrorInvalidValue;
   // N tiles of 256 only with one B operand: with two (hi + lo) a 256-wide stage takes 80 KB and
   // leaves room for two pipeline stages, a 128-wide one 48 KB and four
+  if (nb == 3) return launch_umma_bn<128, 3>(m, a, st);   // a 64 KB stage: three stages
   if (a.bn == 256 || (a.bn == 0 && a.N > 128 && nb == 1))
     return nb == 2 ? launch_umma_bn<256, 2>(m, a, st) : launch_umma_bn<256, 1>(m, a, st);
   return nb == 2 ? launch_umma_bn<128, 2>(m, a, st) : launch_umma_bn<128, 1>(m, a, st);
