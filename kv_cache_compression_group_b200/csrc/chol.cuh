@@ -14,7 +14,6 @@
 // c <= i), both places the factorisation no longer reads.
 #pragma once
 
-#include <cooperative_groups.h>
 
 #include "common.cuh"
 
@@ -424,37 +423,6 @@ __global__ void __launch_bounds__(CF_THREADS, 2)
 namespace jolt {
 
 // ------------------------------------------------------------------------------------------
-// Inverses of the 32 x 32 diagonal blocks of a Cholesky factor L held in the lower triangle
-// of G (column-major, ld gld; the layout a batched LAPACK-style Cholesky leaves), written in
-// fp64 to the upper part of the same diagonal block, W_II[r][s] at G[(I0 + r) * gld + I0 + s]
-// (s <= r): the convention of chol_factor_kernel, so tri_inv_large_kernel reads either.
-// One warp per (block, unit); lane c solves L_II x = e_c by forward substitution.  The warp
-// reads the whole block before any lane writes (the diagonal is overwritten).
-// ------------------------------------------------------------------------------------------
-__global__ void __launch_bounds__(32) diag_inv64_kernel(double* G, int k, long long gld, long long sG) {
-  const int I = blockIdx.x, u = blockIdx.y, lane = threadIdx.x;
-  const int I0 = I * CF_NB, nb = min(CF_NB, k - I0);
-  double* Gu = G + (long long)u * sG;
-  double x[CF_NB];
-#pragma unroll
-  for (int r = 0; r < CF_NB; ++r) {
-    double v = (r == lane) ? 1.0 : 0.0;
-    if (r < nb) {
-#pragma unroll
-      for (int q = 0; q < r; ++q) v = fma(-Gu[(long long)(I0 + q) * gld + I0 + r], x[q], v);
-      v = v / Gu[(long long)(I0 + r) * gld + I0 + r];
-    }
-    x[r] = v;
-  }
-  __syncwarp();
-  if (lane < nb) {
-#pragma unroll
-    for (int r = 0; r < CF_NB; ++r)
-      if (r >= lane && r < nb) Gu[(long long)(I0 + r) * gld + I0 + lane] = x[r];
-  }
-}
-
-// ------------------------------------------------------------------------------------------
 // W = L^{-1} for any k (the block-column recursion of tri_inv_kernel with the block column
 // kept in global fp64 scratch instead of shared memory):
 //   W_JJ = inv(L_JJ),   W_IJ = -inv(L_II) sum_{J <= K < I} L_IK W_KJ   (I > J).
@@ -532,143 +500,125 @@ __global__ void __launch_bounds__(CF_THREADS) tri_inv_large_kernel(const double*
 
 namespace jolt {
 // ------------------------------------------------------------------------------------------
-// Cholesky factor for 256 < k <= 1024: one cluster of 8 CTAs per matrix, right-looking by
-// 32-column block columns, block column K owned by CTA K % 8.  Per block column J:
-//   1. its owner factors the diagonal block (one warp, column by column), inverts it (forward
-//      substitution, one lane per column) and writes the inverse into every CTA's shared
-//      memory (distributed shared memory);
-//   2. cluster barrier;
-//   3. every CTA forms the panel rows it owns, L_IJ = A_IJ inv(L_JJ)^T for I > J, I % 8 == q;
-//   4. cluster barrier;
-//   5. every CTA updates its block columns K > J: A_IK -= L_IJ L_KJ^T for I >= K.
-// The owner of block column J + 1 updated it in step 5 itself, so its factorisation needs no
-// further barrier.  Output in the layout of chol_factor_kernel: L below the diagonal blocks
-// in the lower triangle, inv(L_JJ) in the upper part of its diagonal block (W[i][c] at
-// G[i * gld + c], c <= i).  A pivot that is not positive: DEV_ERR_FACTOR, pivot taken as 1.
-// grid (8 * matrices), clusters of 8, 256 threads.
+// Cholesky factor for 256 < k <= 1024 as a sequence of small steps over all matrices at once,
+// right-looking by 32-column block columns J (the blocked arithmetic of chol_factor_kernel,
+// with every block of a step handled by its own CTA, so the whole GPU works on each step):
+//   chol_step_diag_kernel   L_JJ = chol(A_JJ) and inv(L_JJ) (one warp per matrix);
+//   chol_step_panel_kernel  L_IJ = A_IJ inv(L_JJ)^T for I > J (one CTA per block);
+//   chol_step_update_kernel A_IK -= L_IJ L_KJ^T for J < K <= I (one CTA per block pair).
+// Output as chol_factor_kernel: L below the diagonal blocks in the lower triangle, inv(L_JJ)
+// in the upper part of its diagonal block (W[r][c] at row J0 + c, column J0 + r).  A pivot
+// that is not positive raises DEV_ERR_FACTOR and is taken as 1.  G column-major, pitch gld,
+// matrix stride sG.
 // ------------------------------------------------------------------------------------------
-constexpr int CC_CL = 8;
-__global__ void __cluster_dims__(CC_CL, 1, 1) __launch_bounds__(256)
-    chol_cluster_kernel(double* G, int k, long long gld, long long sG, uint32_t* status) {
-  namespace cg = cooperative_groups;
-  cg::cluster_group cluster = cg::this_cluster();
-  const int q = (int)cluster.block_rank(), u = blockIdx.x / CC_CL, tid = threadIdx.x;
-  const int lane = tid & 31, warp = tid >> 5;
-  __shared__ double Ls[CF_NB][CF_P];    // L_JJ, then (rows) a panel block / L_IJ
-  __shared__ double Wi[CF_NB][CF_P];    // inv(L_JJ)
-  __shared__ double Bs[CF_NB][CF_P];    // L_KJ
-  __shared__ int bad;
-  double* Gu = G + (long long)u * sG;
-  const int nbk = (k + CF_NB - 1) / CF_NB;
-  auto at = [&](int r, int c) -> double& { return Gu[(long long)c * gld + r]; };   // column-major
-  if (tid == 0) bad = 0;
-  __syncthreads();
-  for (int J = 0; J < nbk; ++J) {
-    const int J0 = J * CF_NB, nbJ = min(CF_NB, k - J0);
-    __syncthreads();   // this CTA's updates of block column J are done
-    if (J % CC_CL == q) {
-      for (int idx = tid; idx < CF_NB * CF_NB; idx += blockDim.x) {
-        const int r = idx % CF_NB, c = idx / CF_NB;
-        Ls[r][c] = (r < nbJ && c < nbJ) ? at(J0 + r, J0 + c) : (r == c ? 1.0 : 0.0);
-      }
-      __syncthreads();
-      if (warp == 0) {
-        // factor: lane r holds row r
-        for (int c = 0; c < CF_NB; ++c) {
-          double d = Ls[c][c];
-          if (!(d > 0.0) || !isfinite(d)) {
-            if (lane == 0 && c < nbJ) bad = 1;
-            d = 1.0;
-          }
-          d = sqrt(d);
-          __syncwarp();
-          if (lane == c) Ls[c][c] = d;
-          if (lane > c) Ls[lane][c] /= d;
-          __syncwarp();
-          if (lane > c)
-            for (int s = c + 1; s <= lane; ++s) Ls[lane][s] -= Ls[lane][c] * Ls[s][c];
-          __syncwarp();
-        }
-        // inverse: lane c solves L x = e_c; the result goes to every CTA of the cluster
-        double x[CF_NB];
-#pragma unroll
-        for (int r = 0; r < CF_NB; ++r) {
-          double v = (r == lane) ? 1.0 : 0.0;
-#pragma unroll
-          for (int p = 0; p < r; ++p) v = fma(-Ls[r][p], x[p], v);
-          x[r] = v / Ls[r][r];
-        }
-        for (int t = 0; t < CC_CL; ++t) {
-          double* wt = cluster.map_shared_rank(&Wi[0][0], t);
-#pragma unroll
-          for (int r = 0; r < CF_NB; ++r) wt[r * CF_P + lane] = r >= lane ? x[r] : 0.0;
-        }
-      }
-      __syncthreads();
-      // the diagonal block's inverse into the upper part (W[r][c] at (row c, column r))
-      for (int idx = tid; idx < CF_NB * CF_NB; idx += blockDim.x) {
-        const int r = idx / CF_NB, c = idx % CF_NB;
-        if (r < nbJ && c <= r) at(J0 + c, J0 + r) = Wi[r][c];
-      }
+// grid (matrices), 32 threads
+__global__ void __launch_bounds__(32) chol_step_diag_kernel(double* G, int k, long long gld, long long sG, int J,
+                                                            uint32_t* status) {
+  __shared__ double Ls[CF_NB][CF_P];
+  const int lane = threadIdx.x;
+  double* Gu = G + (long long)blockIdx.x * sG;
+  const int J0 = J * CF_NB, nbJ = min(CF_NB, k - J0);
+  auto at = [&](int r, int c) -> double& { return Gu[(long long)c * gld + r]; };
+  for (int c = 0; c < CF_NB; ++c) Ls[lane][c] = (lane < nbJ && c < nbJ) ? at(J0 + lane, J0 + c) : (lane == c ? 1.0 : 0.0);
+  __syncwarp();
+  bool bad = false;
+  // lane r holds row r
+  for (int c = 0; c < CF_NB; ++c) {
+    double d = Ls[c][c];
+    if (!(d > 0.0) || !isfinite(d)) {
+      if (c < nbJ) bad = true;
+      d = 1.0;
     }
-    __threadfence();
-    cluster.sync();   // inv(L_JJ) in every CTA
-    // my rows of the panel: L_IJ[r][c] = sum_s A_IJ[r][s] inv(L_JJ)[c][s]
-    for (int I = J + 1 + ((q - (J + 1)) % CC_CL + CC_CL) % CC_CL; I < nbk; I += CC_CL) {
-      const int I0 = I * CF_NB, nbI = min(CF_NB, k - I0);
-      __syncthreads();
-      for (int idx = tid; idx < CF_NB * CF_NB; idx += blockDim.x) {
-        const int r = idx % CF_NB, c = idx / CF_NB;
-        Ls[r][c] = (r < nbI && c < nbJ) ? at(I0 + r, J0 + c) : 0.0;
-      }
-      __syncthreads();
-      const int r = tid >> 3, cg0 = tid & 7;
-      double o[4];
+    d = sqrt(d);
+    __syncwarp();
+    if (lane == c) Ls[c][c] = d;
+    if (lane > c) Ls[lane][c] /= d;
+    __syncwarp();
+    if (lane > c)
+      for (int s = c + 1; s <= lane; ++s) Ls[lane][s] -= Ls[lane][c] * Ls[s][c];
+    __syncwarp();
+  }
+  // inverse: lane c solves L x = e_c
+  double x[CF_NB];
 #pragma unroll
-      for (int jj = 0; jj < 4; ++jj) {
-        const int c = cg0 + 8 * jj;
-        double acc = 0.0;
-        for (int s2 = 0; s2 <= c; ++s2) acc = fma(Ls[r][s2], Wi[c][s2], acc);
-        o[jj] = acc;
-      }
+  for (int r = 0; r < CF_NB; ++r) {
+    double v = (r == lane) ? 1.0 : 0.0;
 #pragma unroll
-      for (int jj = 0; jj < 4; ++jj) {
-        const int c = cg0 + 8 * jj;
-        if (r < nbI && c < nbJ) at(I0 + r, J0 + c) = o[jj];
-      }
-    }
-    __threadfence();
-    cluster.sync();   // the panel of block column J is in global memory
-    // trailing update of my block columns K > J
-    for (int K = J + 1; K < nbk; ++K) {
-      if (K % CC_CL != q) continue;
-      const int K0 = K * CF_NB, nbK = min(CF_NB, k - K0);
-      __syncthreads();
-      for (int idx = tid; idx < CF_NB * CF_NB; idx += blockDim.x) {
-        const int r = idx % CF_NB, c = idx / CF_NB;
-        Bs[r][c] = (r < nbK && c < nbJ) ? at(K0 + r, J0 + c) : 0.0;
-      }
-      for (int I = K; I < nbk; ++I) {
-        const int I0 = I * CF_NB, nbI = min(CF_NB, k - I0);
-        __syncthreads();
-        for (int idx = tid; idx < CF_NB * CF_NB; idx += blockDim.x) {
-          const int r = idx % CF_NB, c = idx / CF_NB;
-          Ls[r][c] = (r < nbI && c < nbJ) ? at(I0 + r, J0 + c) : 0.0;
-        }
-        __syncthreads();
-        const int r = tid & 31, cg0 = tid >> 5;   // row r, columns cg0 + 8 jj (coalesced writes)
+    for (int p = 0; p < r; ++p) v = fma(-Ls[r][p], x[p], v);
+    x[r] = v / Ls[r][r];
+  }
+  // W[r][lane] = x[r] (r >= lane) at row J0 + lane, column J0 + r
 #pragma unroll
-        for (int jj = 0; jj < 4; ++jj) {
-          const int c = cg0 + 8 * jj;
-          double acc = 0.0;
-#pragma unroll 8
-          for (int s2 = 0; s2 < CF_NB; ++s2) acc = fma(Ls[r][s2], Bs[c][s2], acc);
-          if (r < nbI && c < nbK) at(I0 + r, K0 + c) -= acc;
-        }
-      }
-    }
+  for (int r = 0; r < CF_NB; ++r)
+    if (r >= lane && r < nbJ && lane < nbJ) at(J0 + lane, J0 + r) = x[r];
+  if (bad && status) raise_status(status, DEV_ERR_FACTOR);
+}
+
+// grid (blocks below J, matrices), CF_THREADS threads
+__global__ void __launch_bounds__(CF_THREADS) chol_step_panel_kernel(double* G, int k, long long gld, long long sG,
+                                                                     int J) {
+  __shared__ double As[CF_NB][CF_P];
+  __shared__ double Wi[CF_NB][CF_P];
+  const int tid = threadIdx.x;
+  double* Gu = G + (long long)blockIdx.y * sG;
+  const int J0 = J * CF_NB, nbJ = min(CF_NB, k - J0);
+  const int I = J + 1 + blockIdx.x, I0 = I * CF_NB, nbI = min(CF_NB, k - I0);
+  auto at = [&](int r, int c) -> double& { return Gu[(long long)c * gld + r]; };
+  for (int idx = tid; idx < CF_NB * CF_NB; idx += blockDim.x) {
+    const int r = idx % CF_NB, c = idx / CF_NB;
+    As[r][c] = (r < nbI && c < nbJ) ? at(I0 + r, J0 + c) : 0.0;
+    // inv(L_JJ)[c][r] sits at row J0 + r, column J0 + c (r <= c)
+    Wi[c][r] = (r <= c && c < nbJ) ? at(J0 + r, J0 + c) : 0.0;
   }
   __syncthreads();
-  if (tid == 0 && bad) raise_status(status, DEV_ERR_FACTOR);
+  // L_IJ[r][c] = sum_s A_IJ[r][s] inv(L_JJ)[c][s]  (s <= c)
+  const int r = tid & 31, cg0 = tid >> 5;   // row r, columns cg0 + 8 jj (coalesced writes)
+#pragma unroll
+  for (int jj = 0; jj < 4; ++jj) {
+    const int c = cg0 + 8 * jj;
+    double acc = 0.0;
+    for (int s2 = 0; s2 <= c; ++s2) acc = fma(As[r][s2], Wi[c][s2], acc);
+    if (r < nbI && c < nbJ) at(I0 + r, J0 + c) = acc;
+  }
+}
+
+// grid (block pairs (I, K) with J < K <= I < nbk, matrices), CF_THREADS threads
+__global__ void __launch_bounds__(CF_THREADS) chol_step_update_kernel(double* G, int k, long long gld, long long sG,
+                                                                      int J) {
+  __shared__ double Li[CF_NB][CF_P];
+  __shared__ double Lk[CF_NB][CF_P];
+  const int tid = threadIdx.x;
+  double* Gu = G + (long long)blockIdx.y * sG;
+  const int J0 = J * CF_NB, nbJ = min(CF_NB, k - J0);
+  // pair index -> (i, kk) with 0 <= kk <= i: row-major lower triangle
+  const int idx = blockIdx.x;
+  int i = (int)((sqrt(8.0 * idx + 1.0) - 1.0) * 0.5);
+  while ((i + 1) * (i + 2) / 2 <= idx) ++i;
+  while (i * (i + 1) / 2 > idx) --i;
+  const int kk = idx - i * (i + 1) / 2;
+  const int I = J + 1 + i, K = J + 1 + kk;
+  const int I0 = I * CF_NB, K0 = K * CF_NB, nbI = min(CF_NB, k - I0), nbK = min(CF_NB, k - K0);
+  auto at = [&](int r, int c) -> double& { return Gu[(long long)c * gld + r]; };
+  for (int e = tid; e < CF_NB * CF_NB; e += blockDim.x) {
+    const int r = e % CF_NB, c = e / CF_NB;
+    Li[r][c] = (r < nbI && c < nbJ) ? at(I0 + r, J0 + c) : 0.0;
+    Lk[r][c] = (r < nbK && c < nbJ) ? at(K0 + r, J0 + c) : 0.0;
+  }
+  const int r = tid & 31, cg0 = tid >> 5;
+  double aold[4];
+#pragma unroll
+  for (int jj = 0; jj < 4; ++jj) {
+    const int c = cg0 + 8 * jj;
+    aold[jj] = (r < nbI && c < nbK) ? at(I0 + r, K0 + c) : 0.0;
+  }
+  __syncthreads();
+#pragma unroll
+  for (int jj = 0; jj < 4; ++jj) {
+    const int c = cg0 + 8 * jj;
+    double acc = 0.0;
+#pragma unroll 8
+    for (int s2 = 0; s2 < CF_NB; ++s2) acc = fma(Li[r][s2], Lk[c][s2], acc);
+    if (r < nbI && c < nbK) at(I0 + r, K0 + c) = aold[jj] - acc;
+  }
 }
 }  // namespace jolt

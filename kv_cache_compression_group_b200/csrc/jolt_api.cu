@@ -835,8 +835,16 @@ jolt_status cholqr_tc(const Ctx& c, float* Y, long long m, int k, int ld, int pa
         // 256 < k <= 1024: the cluster Cholesky (chol.cuh), then the block-column inverse
         count_launch(), sanitize_sym_batched_kernel<<<p.NU, 1024, 0, c.st>>>(G, k, gld, sG, c.status());
         {
-          ProfScope ps4("chol_cluster", c.st, p.NU);
-          count_launch(), chol_cluster_kernel<<<(unsigned)(p.NU * CC_CL), 256, 0, c.st>>>(G, k, gld, sG, c.status());
+          ProfScope ps4("chol_steps", c.st, p.NU);
+          for (int J = 0; J < nbk; ++J) {
+            count_launch(), chol_step_diag_kernel<<<p.NU, 32, 0, c.st>>>(G, k, gld, sG, J, c.status());
+            const int below = nbk - J - 1;
+            if (below > 0) {
+              count_launch(), chol_step_panel_kernel<<<dim3(below, p.NU), CF_THREADS, 0, c.st>>>(G, k, gld, sG, J);
+              count_launch(), chol_step_update_kernel<<<dim3(below * (below + 1) / 2, p.NU), CF_THREADS, 0, c.st>>>(
+                  G, k, gld, sG, J);
+            }
+          }
           CUDA_TRY(cudaGetLastError());
         }
         ProfScope ps5("tri_inv_large", c.st, p.NU);
