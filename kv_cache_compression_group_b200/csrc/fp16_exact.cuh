@@ -117,6 +117,58 @@ __host__ __device__ __forceinline__ float quant_step_sel(float mx, float lo, flo
   return a_lt ? su : (ap_ge ? sp : s);
 }
 
+// 1 / (2^b - 1) rounded down and up to fp32, b = 1 .. 8 (hexadecimal float literals)
+__host__ __device__ __forceinline__ float inv_levels_rd(int b) {
+  switch (b) {
+    case 1: return 0x1.000000p+0f;
+    case 2: return 0x1.555554p-2f;
+    case 3: return 0x1.249248p-3f;
+    case 4: return 0x1.111110p-4f;
+    case 5: return 0x1.084210p-5f;
+    case 6: return 0x1.041040p-6f;
+    case 7: return 0x1.020408p-7f;
+    default: return 0x1.010100p-8f;
+  }
+}
+__host__ __device__ __forceinline__ float inv_levels_ru(int b) {
+  switch (b) {
+    case 1: return 0x1.000000p+0f;
+    case 2: return 0x1.555556p-2f;
+    case 3: return 0x1.24924ap-3f;
+    case 4: return 0x1.111112p-4f;
+    case 5: return 0x1.084212p-5f;
+    case 6: return 0x1.041042p-6f;
+    case 7: return 0x1.02040ap-7f;
+    default: return 0x1.010102p-8f;
+  }
+}
+
+// The same step as quant_step, from a bracket of the quotient: lower and upper fp32 bounds of
+// (mx - lo) / levels (directed roundings of the difference and of the product with the
+// directed reciprocal), each rounded up to fp16 by the conversion instruction.  When the two
+// agree, the fp16 round-up of the exact quotient is that value (the round-up is monotone);
+// otherwise (the quotient lies within a few fp32 ulps of an fp16 number) quant_step decides.
+// The conversion also covers the fp16 subnormal range and the overflow to +inf.  On the host
+// the bracket is widened by one ulp on each side in place of the directed roundings.
+__host__ __device__ __forceinline__ float quant_step_cvt(float mx, float lo, int b) {
+  if (!(mx > lo)) return 0.f;
+#ifdef __CUDA_ARCH__
+  const float rlo = __fsub_rd(mx, lo), rhi = __fsub_ru(mx, lo);
+  const float qlo = __fmul_rd(rlo, inv_levels_rd(b)), qhi = __fmul_ru(rhi, inv_levels_ru(b));
+#else
+  const float r = mx - lo;
+  const float rlo = nextafterf(r, -INFINITY), rhi = nextafterf(r, INFINITY);
+  const float qlo = nextafterf(fmaxf(rlo, 0.f) * inv_levels_rd(b), -INFINITY);
+  const float qhi = nextafterf(rhi * inv_levels_ru(b), INFINITY);
+#endif
+  const __half hlo = __float2half_ru(qlo), hhi = __float2half_ru(qhi);
+  if (__half_as_ushort(hlo) != __half_as_ushort(hhi)) {
+    const float flev = (float)((1 << b) - 1);
+    return quant_step(mx, lo, flev, 1.0f / flev);
+  }
+  return __half2float(hlo);
+}
+
 // ---------------------------------------------------------------------------------------
 // codes of the b-bit block quantiser and their packing
 // ---------------------------------------------------------------------------------------

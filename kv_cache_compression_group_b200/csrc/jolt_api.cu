@@ -177,6 +177,7 @@ struct Plan {
   size_t fsolver_dev;     // cuSOLVER device workspace (feature factor, on the auxiliary stream)
   size_t solver_host;
   // workspace offsets (bytes)
+  size_t o_signkey, o_sign;
   size_t o_status, o_gd_part, o_gd, o_evals, o_Wf, o_Ws, o_Uf, o_Us, o_core, o_zc, o_ptmp, o_P, o_partial,
       o_table, o_bytes, o_choice, o_lambda, o_hdr, o_umap, o_info, o_solver, o_fsolver, o_finfo, o_fevals, o_eigvec, o_eigscr,
       o_feigvec, o_feigscr;
@@ -325,6 +326,8 @@ jolt_status make_plan(const jolt_shape* sh, const jolt_options* op, Plan* p) {
 
   Bump b;
   p->o_status = b.take(256);
+  p->o_signkey = b.take((size_t)NU * p->rTmax * 8);   // token-factor column signs: keys, signs
+  p->o_sign = b.take((size_t)NU * p->rTmax * 4);
   p->o_gd_part = b.take((size_t)NU * p->gd_split * D * D * 4);
   p->o_gd = b.take((size_t)NU * D * D * 8);
   {
@@ -1242,9 +1245,19 @@ jolt_status run_factor(const Ctx& c, float* Uf, long long ldUf, float* Wf, long 
   CUDA_TRY(cudaStreamWaitEvent(c.st, ax->join, 0));
   // sign convention of the token factor columns (the randomized and back-projected routes
   // need it; for the eigenvector route it is already in place) and the bf16 copy
-  count_launch(), col_sign_fix_kernel<<<dim3(p.rTmax, p.NU), 256, 0, c.st>>>(
-      Uf, ldUf, (long long)p.T * ldUf, p.T, p.rTmax, Us, ldUf, (long long)p.T * ldUf);
-  CUDA_TRY(cudaGetLastError());
+  {
+    ProfScope ps("sign_fix", c.st, p.NU);
+    unsigned long long* keys = c.at<unsigned long long>(p.o_signkey);
+    float* signs = c.at<float>(p.o_sign);
+    const long long sU = (long long)p.T * ldUf;
+    CUDA_TRY(cudaMemsetAsync(keys, 0, (size_t)p.NU * p.rTmax * 8, c.st));
+    count_launch(), sign_key_kernel<<<dim3((unsigned)ceil_div(p.T, SK_ROWS), p.NU), 256, 0, c.st>>>(
+        Uf, ldUf, sU, p.T, p.rTmax, keys);
+    count_launch(), sign_of_kernel<<<p.NU, 1024, 0, c.st>>>(Uf, ldUf, sU, p.rTmax, keys, signs);
+    count_launch(), sign_apply_kernel<<<grid1d((long long)p.NU * p.T * (p.rTmax / 4)), 256, 0, c.st>>>(
+        Uf, ldUf, sU, p.T, p.rTmax, signs, Us, ldUf, sU, p.NU);
+    CUDA_TRY(cudaGetLastError());
+  }
   return JOLT_OK;
 }
 
@@ -1488,7 +1501,7 @@ jolt_status run_table(const Ctx& c, const bf16* Us, long long ldU, const bf16* W
       default: JTRY(launch_table_D<128>(c, a)); break;
     }
   }
-  count_launch(), table_reduce_kernel<<<(unsigned)ceil_div((long long)p.NU * p.nC, 128), 128, 0, c.st>>>(
+  count_launch(), table_reduce_kernel<<<(unsigned)((long long)p.NU * p.nC), 256, 0, c.st>>>(
       a.partial, table, p.NU, p.S, tiles, p.cd.nT, p.cd.nD, p.cd.nB);
   CUDA_TRY(cudaGetLastError());
   return JOLT_OK;

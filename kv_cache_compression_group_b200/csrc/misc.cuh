@@ -110,40 +110,74 @@ __global__ void eig_select_kernel(const double* vals, const double* vecs, int n,
   }
 }
 
-// Same sign convention on the columns of a row-major fp32 matrix (in place), plus bf16 copy
-__global__ void col_sign_fix_kernel(float* A, long long lda, long long sA, int n, int r, bf16* out_bf16,
-                                    long long ldo, long long so) {
-  const int j = blockIdx.x, u = blockIdx.y;
-  float* a = A + (long long)u * sA;
-  __shared__ float bestv[256];
-  __shared__ int besti[256];
-  float bv = -1.f;
-  int bi = 0x7fffffff;
-  for (int i = threadIdx.x; i < n; i += blockDim.x) {
-    float x = fabsf(a[(long long)i * lda + j]);
-    if (x > bv || (x == bv && i < bi)) { bv = x; bi = i; }
-  }
-  bestv[threadIdx.x] = bv;
-  besti[threadIdx.x] = bi;
-  __syncthreads();
-  for (int st = blockDim.x / 2; st > 0; st >>= 1) {
-    if ((int)threadIdx.x < st) {
-      float ov = bestv[threadIdx.x + st];
-      int oi = besti[threadIdx.x + st];
-      if (ov > bestv[threadIdx.x] || (ov == bestv[threadIdx.x] && oi < besti[threadIdx.x])) {
-        bestv[threadIdx.x] = ov;
-        besti[threadIdx.x] = oi;
-      }
+// Same sign convention on the columns j < r of every unit's row-major fp32 matrix (n rows,
+// pitch lda, unit stride sA), in place, plus a bf16 copy; three coalesced passes:
+//   sign_key_kernel   per column the largest |a| with its first row, as one 64-bit key
+//                     (|a|'s bits above the complement of the row: the atomic maximum of the
+//                     keys is the largest magnitude, ties to the lowest row; non-finite
+//                     magnitudes never win, a column without any keeps the key 0);
+//   sign_of_kernel    the sign of the entry the key names (+1 for key 0);
+//   sign_apply_kernel a *= sign, bf16 copy.
+// keys: [units][r] uint64, zeroed before sign_key_kernel; signs: [units][r] fp32.
+constexpr int SK_ROWS = 512;   // rows per CTA of sign_key_kernel
+// grid (ceil(n / SK_ROWS), units), 256 threads
+__global__ void __launch_bounds__(256) sign_key_kernel(const float* A, long long lda, long long sA, int n, int r,
+                                                       unsigned long long* keys) {
+  const int u = blockIdx.y, i0 = blockIdx.x * SK_ROWS, i1 = min(n, i0 + SK_ROWS);
+  const float* a = A + (long long)u * sA;
+  for (int c = threadIdx.x; c < r; c += blockDim.x) {
+    unsigned long long best = 0ull;
+    for (int i = i0; i < i1; ++i) {
+      const float x = fabsf(a[(long long)i * lda + c]);
+      if (!(x <= 3.402823466e38f)) continue;   // NaN or infinite: never the pivot
+      const unsigned long long key =
+          ((unsigned long long)__float_as_uint(x) << 32) | (unsigned long long)(0xFFFFFFFFu - (unsigned)i);
+      best = key > best ? key : best;
     }
-    __syncthreads();
+    if (best) atomicMax(keys + (long long)u * r + c, best);
   }
-  const int piv = besti[0] < n ? besti[0] : 0;   // no finite entry: sign +1
-  const float sgn = a[(long long)piv * lda + j] < 0 ? -1.f : 1.f;
-  __syncthreads();
-  for (int i = threadIdx.x; i < n; i += blockDim.x) {
-    float v = sgn * a[(long long)i * lda + j];
-    a[(long long)i * lda + j] = v;
-    if (out_bf16) out_bf16[(long long)u * so + (long long)i * ldo + j] = __float2bfloat16_rn(v);
+}
+// grid (units), 1024 threads
+__global__ void sign_of_kernel(const float* A, long long lda, long long sA, int r, const unsigned long long* keys,
+                               float* signs) {
+  const int u = blockIdx.x;
+  const float* a = A + (long long)u * sA;
+  for (int c = threadIdx.x; c < r; c += blockDim.x) {
+    const unsigned long long key = keys[(long long)u * r + c];
+    float sg = 1.f;
+    if (key) {
+      const long long piv = (long long)(0xFFFFFFFFu - (unsigned)(key & 0xFFFFFFFFull));
+      sg = a[piv * lda + c] < 0.f ? -1.f : 1.f;
+    }
+    signs[(long long)u * r + c] = sg;
+  }
+}
+// grid-stride over units x n x r (4 columns per thread; lda, ldo, r multiples of 4)
+__global__ void sign_apply_kernel(float* A, long long lda, long long sA, int n, int r, const float* signs,
+                                  bf16* out_bf16, long long ldo, long long so, int nunits) {
+  const int r4 = r / 4;
+  const long long per = (long long)n * r4, total = per * nunits;
+  for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < total;
+       e += (long long)gridDim.x * blockDim.x) {
+    const int u = (int)(e / per);
+    const long long rem = e - (long long)u * per;
+    const long long i = rem / r4;
+    const int c = (int)(rem - i * r4) * 4;
+    float4* pa = reinterpret_cast<float4*>(A + (long long)u * sA + i * lda + c);
+    const float4 sg = *reinterpret_cast<const float4*>(signs + (long long)u * r + c);
+    float4 v = *pa;
+    v.x *= sg.x;
+    v.y *= sg.y;
+    v.z *= sg.z;
+    v.w *= sg.w;
+    *pa = v;
+    if (out_bf16) {
+      __nv_bfloat162 h0 = __floats2bfloat162_rn(v.x, v.y), h1 = __floats2bfloat162_rn(v.z, v.w);
+      uint2 w;
+      w.x = *reinterpret_cast<uint32_t*>(&h0);
+      w.y = *reinterpret_cast<uint32_t*>(&h1);
+      *reinterpret_cast<uint2*>(out_bf16 + (long long)u * so + i * ldo + c) = w;
+    }
   }
 }
 
@@ -224,15 +258,16 @@ __global__ void sanitize_sym_batched_kernel(double* A, int n, long long lda, lon
   __shared__ int bad;
   if (threadIdx.x == 0) bad = (*status & DEV_ERR_NONFINITE) ? 1 : 0;
   __syncthreads();
+  // column by column (consecutive threads read consecutive rows)
   for (long long i = threadIdx.x; i < (long long)n * n && !bad; i += blockDim.x) {
-    long long r = i / n, c = i - r * n;
+    long long c = i / n, r = i - c * n;
     if (!isfinite(M[c * lda + r])) bad = 1;
   }
   __syncthreads();
   if (!bad) return;
   if (threadIdx.x == 0) raise_status(status, DEV_ERR_NONFINITE);
   for (long long i = threadIdx.x; i < (long long)n * n; i += blockDim.x) {
-    long long r = i / n, c = i - r * n;
+    long long c = i / n, r = i - c * n;
     M[c * lda + r] = (r == c) ? 1.0 : 0.0;
   }
 }
@@ -270,18 +305,26 @@ __global__ void scale_cols_kernel(float* V, const double* lam, int n, int r, lon
 // distortion table finalisation, byte table and the Lagrangian dual
 // ------------------------------------------------------------------------------------------
 // table[u][(iT*nD + iD)*nB + ib] = sum over (slice, tile) of partial[u][s][tile][(iD*nT+iT)*nB+ib]
-__global__ void table_reduce_kernel(const double* partial, double* table, int nunits, int S, int tiles, int nT,
-                                    int nD, int nB) {
+// grid (units x choices), 256 threads: the partial sums of every (slice, tile) of one table
+// entry, strided over the threads, then a fixed-order tree (the same order on every call)
+__global__ void __launch_bounds__(256) table_reduce_kernel(const double* partial, double* table, int nunits, int S,
+                                                           int tiles, int nT, int nD, int nB) {
+  __shared__ double red[256];
   const int nc = nT * nD * nB;
-  int idx = blockIdx.x * blockDim.x + threadIdx.x;
-  if (idx >= nunits * nc) return;
-  int u = idx / nc, c = idx - u * nc;
-  int ib = c % nB, iD = (c / nB) % nD, iT = c / (nB * nD);
-  int pc = (iD * nT + iT) * nB + ib;
+  const int idx = blockIdx.x;
+  const int u = idx / nc, c = idx - u * nc;
+  const int ib = c % nB, iD = (c / nB) % nD, iT = c / (nB * nD);
+  const int pc = (iD * nT + iT) * nB + ib;
   const double* p = partial + (long long)u * S * tiles * nc + pc;
   double acc = 0.0;
-  for (long long st = 0; st < (long long)S * tiles; ++st) acc += p[st * nc];
-  table[idx] = acc;
+  for (long long st = threadIdx.x; st < (long long)S * tiles; st += blockDim.x) acc += p[st * nc];
+  red[threadIdx.x] = acc;
+  __syncthreads();
+  for (int w = blockDim.x / 2; w > 0; w >>= 1) {
+    if ((int)threadIdx.x < w) red[threadIdx.x] += red[threadIdx.x + w];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) table[idx] = red[0];
 }
 
 __host__ __device__ inline unsigned long long pad16u(unsigned long long n) { return (n + 15ull) / 16ull * 16ull; }

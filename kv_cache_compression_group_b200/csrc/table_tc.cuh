@@ -124,7 +124,7 @@ __device__ __forceinline__ void ttc_tmem_ld16(uint32_t taddr, float* v) {
 // ---------------------------------------------------------------------------------------
 // Quantiser error sums of one 16-wide block for the table (packed pairs throughout):
 //   * block min / max by three-input min / max (exact, the same values as a two-input tree);
-//   * lo and the fp16 step exactly as the encoder forms them (rd16, quant_step);
+//   * lo and the fp16 step exactly as the encoder forms them (rd16, quant_step_cvt);
 //   * code = round-half-even(d / step) through the approximate reciprocal of step, the error
 //     (d - code * step)^2 summed in four packed partial sums.
 // The approximate reciprocal can move a code only where d / step lies within a few ulp of a
@@ -157,9 +157,7 @@ __device__ __forceinline__ void ttc_bit_error(const float2* v, const float2* d, 
 #pragma unroll
     for (int j = 0; j < 8; ++j) a = __ffma2_rn(v[j], v[j], a);
   } else {
-    constexpr float flev = (float)((1 << B) - 1);
-    const float inv_lev = 1.0f / flev;
-    const float step = quant_step_sel(mx, lo, flev, inv_lev);
+    const float step = quant_step_cvt(mx, lo, B);
     const bool ok = isfinite(lo) && step <= kFp16Max;
     const float inv = step > 0.f ? ttc_rcp_approx(step) : 0.f;
     const float2 inv2 = make_float2(inv, inv), nstep2 = make_float2(-step, -step);
@@ -571,7 +569,7 @@ __global__ void __launch_bounds__(etc::THREADS, 1)
     }
     const int t = t0 + row;
     if (!*abort_flag && t < T) {
-      const float flev = (float)((1 << b) - 1), inv_lev = 1.0f / flev;
+      const float flev = (float)((1 << b) - 1);
       unsigned char* codes = a.blob + uh.off_codes;
       __half2* scales = reinterpret_cast<__half2*>(a.blob + uh.off_scales);
 #pragma unroll
@@ -582,7 +580,7 @@ __global__ void __launch_bounds__(etc::THREADS, 1)
         float mn, mx;
         minmax16(v, mn, mx);
         const float l16 = rd16(mn);
-        const float step = quant_step(mx, l16, flev, inv_lev);
+        const float step = quant_step_cvt(mx, l16, b);
         const float inv = (step > 0.f && step <= kFp16Max) ? __frcp_rn(step) : 0.f;
         uint32_t w[4] = {0u, 0u, 0u, 0u};
 #pragma unroll

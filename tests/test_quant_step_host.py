@@ -2,8 +2,8 @@
 against the oracle:
 
 * the exact fp16 block scales (lo = fp16 round-down of the block minimum, step = smallest
-  fp16 s with s * (2^b - 1) >= max - lo), bit for bit, on random and adversarial blocks, both
-  the branching form and the select form the table kernel uses
+  fp16 s with s * (2^b - 1) >= max - lo), bit for bit, on random and adversarial blocks, in
+  the branching form, the select form and the bracketed conversion form
   (values at and next to fp16 numbers, steps landing exactly on fp16 numbers, the fp16
   subnormal range, overflow, equal minimum and maximum);
 * the packed code bytes, bit for bit with the oracle's packing of the same codes, and their
@@ -131,7 +131,7 @@ def test_block_scales_match_the_oracle_bit_for_bit(host_prog):
     mn, mx = _cases(rng)
     pairs = np.stack([mn, mx], 1).astype(np.float32)
     out = subprocess.run([host_prog], input=pairs.tobytes(), capture_output=True, check=True).stdout
-    got = np.frombuffer(out, dtype=np.float32).reshape(-1, 11).astype(np.float64)
+    got = np.frombuffer(out, dtype=np.float32).reshape(-1, 16).astype(np.float64)
     assert got.shape[0] == pairs.shape[0]
     lo = O.fp16_rd(mn.astype(np.float64))
     np.testing.assert_array_equal(got[:, 0], lo)
@@ -140,8 +140,9 @@ def test_block_scales_match_the_oracle_bit_for_bit(host_prog):
         with np.errstate(invalid="ignore", over="ignore"):
             ref = np.where(mx.astype(np.float64) > lo, O.fp16_ru((mx.astype(np.float64) - lo) / levels), 0.0)
         np.testing.assert_array_equal(got[:, 1 + j], ref, err_msg=f"b = {b}")
-        # the branch-free form the table kernel uses: the same value in every case
+        # the branch-free form and the bracketed conversion form: the same value in every case
         np.testing.assert_array_equal(got[:, 6 + j], ref, err_msg=f"b = {b} (select form)")
+        np.testing.assert_array_equal(got[:, 11 + j], ref, err_msg=f"b = {b} (conversion form)")
     # the cases reach every branch: ties on fp16 numbers, subnormal steps, overflow, zero step
     steps = got[:, 1:]
     assert np.any(steps == 0.0) and np.any(np.isinf(steps)) and np.any((steps > 0) & (steps < 6.103515625e-05))
