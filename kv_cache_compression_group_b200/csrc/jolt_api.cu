@@ -184,6 +184,9 @@ struct Plan {
   int eig_n;              // order of the token-side eigen problems solved by the own solver (0: none)
   // token factor scratch (all units)
   size_t o_gt32, o_gt, o_vsel, o_lam, o_omega, o_Y, o_Zm, o_h, o_l, o_gpart, o_G, o_Lr;
+  // FlashJoLT on the tensor cores: the T x k bases only as bf16 hi + lo pairs (two pairs,
+  // alternating) and the split of the M-side basis
+  size_t o_h2, o_l2, o_mh, o_ml;
   size_t o_wth, o_wtl, o_winv, o_vh, o_vl;   // tensor-core Cholesky QR: W^T = L^-T split, fp64 scratch; V split
   int qr_split_max;       // split-K of the Cholesky-QR Grams
   size_t ws_total;
@@ -358,6 +361,7 @@ jolt_status make_plan(const jolt_shape* sh, const jolt_options* op, Plan* p) {
   // token factor scratch
   p->o_gt32 = p->o_gt = p->o_vsel = p->o_lam = p->o_omega = 0;
   p->o_Y = p->o_Zm = p->o_h = p->o_l = p->o_gpart = p->o_G = p->o_eigvec = p->o_eigscr = 0;
+  p->o_h2 = p->o_l2 = p->o_mh = p->o_ml = 0;
   const int kq = op->method == JOLT_RANDOMIZED ? p->kp : p->ldU;   // width of the QR'ed blocks
   if (op->method == JOLT_EXACT) {
     long long n = p->m_side ? M : T;
@@ -373,11 +377,18 @@ jolt_status make_plan(const jolt_shape* sh, const jolt_options* op, Plan* p) {
   } else {
     const int kp = p->kp;
     long long big = M > T ? M : T;
+    const bool pairs = sh->dtype == JOLT_BF16 && D % 64 == 0 && T % 64 == 0 && kp >= QR_TC_MINK;
     p->o_omega = b.take((size_t)NU * M * kp * 2);
-    p->o_Y = b.take((size_t)NU * T * kp * 4);
+    if (!pairs) p->o_Y = b.take((size_t)NU * T * kp * 4);
     p->o_Zm = b.take((size_t)NU * M * kp * 4);
     p->o_h = b.take((size_t)NU * big * kp * 2);
     p->o_l = b.take((size_t)NU * big * kp * 2);
+    if (pairs) {
+      p->o_h2 = b.take((size_t)NU * T * kp * 2);
+      p->o_l2 = b.take((size_t)NU * T * kp * 2);
+      p->o_mh = b.take((size_t)NU * M * kp * 2);
+      p->o_ml = b.take((size_t)NU * M * kp * 2);
+    }
     p->o_vsel = b.take((size_t)NU * kp * p->ldU * 4);
   }
   // the own eigen solver (order <= 256): the feature factor (n = D, auxiliary stream) and the
@@ -769,13 +780,12 @@ jolt_status umma_run(const Ctx& c, const UmmaMaps& m, UmmaArgs a, int nb) {
 //   Q = Y W^T = Yh (Wh + Wl)^T + Yl Wh^T on tcgen05, the K range of each output tile cut at
 //       the diagonal (W^T is upper triangular).
 // `passes` = 2 gives CholeskyQR2.
-jolt_status cholqr_tc(const Ctx& c, float* Y, long long m, int k, int ld, int passes) {
+// One pass on a block given as its bf16 hi + lo split (yh, yl; columns k..ld zero): the Gram,
+// the factor and its inverse, and Q, written either as fp32 (outY) or as a bf16 pair (oh, ol,
+// all ld columns; the columns k..ld come out zero).
+jolt_status qr_pass_tc(const Ctx& c, const bf16* yh, const bf16* yl, long long m, int k, int ld, float* outY,
+                       bf16* oh, bf16* ol) {
   const Plan& p = c.p;
-  ProfScope ps("cholesky_qr", c.st, p.NU);
-  if (k > 1024) return fail(JOLT_ERR_UNSUPPORTED_SHAPE, "Cholesky QR of more than 1024 columns");
-  if (ld % 8) return fail(JOLT_ERR_UNSUPPORTED_SHAPE, "Cholesky QR pitch %d not a multiple of 8", ld);
-  bf16* yh = c.at<bf16>(p.o_h);
-  bf16* yl = c.at<bf16>(p.o_l);
   float* gpart = c.at<float>(p.o_gpart);
   double* G = c.at<double>(p.o_G);
   float* WT = c.at<float>(p.o_Lr);
@@ -785,126 +795,171 @@ jolt_status cholqr_tc(const Ctx& c, float* Y, long long m, int k, int ld, int pa
   const long long sG = (long long)k * gld, sW = (long long)kq32 * kq32;
   const int ns = (int)ceil_div(m, QR_TC_CHUNK);
   if (ns > p.qr_split_max) return fail(JOLT_ERR_WORKSPACE_TOO_SMALL, "Gram partial slots");
-  const long long nY = (long long)p.NU * m * ld;
   UmmaMaps my, mw;
   if (!map_dense(&my.a0, yh, ld, m, p.NU) || !map_dense(&my.a1, yl, ld, m, p.NU) ||
       !map_dense(&mw.b0, wth, kq32, kq32, p.NU) || !map_dense(&mw.b1, wtl, kq32, kq32, p.NU))
     return fail(JOLT_ERR_CUDA, "tensor map of the Cholesky QR operands refused");
-  // rows k..kq32 of W^T are never written: zero them once (they meet zero columns of Y)
+  // rows k..kq32 of W^T are never written: zeroed (they meet zero columns of Y)
   CUDA_TRY(cudaMemsetAsync(WT, 0, (size_t)p.NU * sW * 4, c.st));
-  for (int pass = 0; pass < passes; ++pass) {
-    count_launch(), split_bf16_cols_kernel<<<grid1d(nY), 256, 0, c.st>>>(Y, yh, yl, nY, ld, k);
+  {
+    ProfScope ps1("qr_gram", c.st, p.NU);
+    UmmaArgs g;
+    g.M = g.N = k;
+    g.K = (int)m;
+    g.batch = p.NU;
+    g.splits = ns;
+    g.kchunk = QR_TC_CHUNK;
+    g.A.mode = UM_DENSE_MN;
+    g.B.mode = UM_DENSE_MN;
+    g.tri = 1;
+    g.bn = 128;
+    g.C = gpart;
+    g.ldc = gld;
+    g.sC = (long long)ns * k * gld;
+    g.ssplit = (long long)k * gld;
+    g.status = c.status();
+    UmmaMaps m3;   // Yh^T Yh + Yh^T Yl + Yl^T Yh in one pass
+    m3.a0 = my.a0;
+    m3.a1 = my.a1;
+    m3.b0 = my.a0;
+    m3.b1 = my.a1;
+    JTRY(umma_run(c, m3, g, 3));
+    count_launch(), reduce_upper_sym_kernel<<<grid1d((long long)p.NU * k * k), 256, 0, c.st>>>(gpart, G, p.NU,
+                                                                                                ns, k, gld);
     CUDA_TRY(cudaGetLastError());
-    {
-      ProfScope ps1("qr_gram", c.st, p.NU);
-      UmmaArgs g;
-      g.M = g.N = k;
-      g.K = (int)m;
-      g.batch = p.NU;
-      g.splits = ns;
-      g.kchunk = QR_TC_CHUNK;
-      g.A.mode = UM_DENSE_MN;
-      g.B.mode = UM_DENSE_MN;
-      g.tri = 1;
-      g.bn = 128;
-      g.C = gpart;
-      g.ldc = gld;
-      g.sC = (long long)ns * k * gld;
-      g.ssplit = (long long)k * gld;
-      g.status = c.status();
-      UmmaMaps m3;   // Yh^T Yh + Yh^T Yl + Yl^T Yh in one pass
-      m3.a0 = my.a0;
-      m3.a1 = my.a1;
-      m3.b0 = my.a0;
-      m3.b1 = my.a1;
-      JTRY(umma_run(c, m3, g, 3));
-      count_launch(), reduce_upper_sym_kernel<<<grid1d((long long)p.NU * k * k), 256, 0, c.st>>>(gpart, G, p.NU,
-                                                                                                  ns, k, gld);
+  }
+  {
+    ProfScope ps2("qr_factor", c.st, p.NU);
+    if (k <= CF_MAXK && gld % 4 == 0) {
+      CUDA_TRY(cudaFuncSetAttribute(chol_factor_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)chol_factor_smem()));
+      count_launch(), chol_factor_kernel<<<p.NU, CF_FT, chol_factor_smem(), c.st>>>(G, k, gld, sG, c.status());
       CUDA_TRY(cudaGetLastError());
-    }
-    {
-      ProfScope ps2("qr_factor", c.st, p.NU);
-      if (k <= CF_MAXK && gld % 4 == 0) {
-        CUDA_TRY(cudaFuncSetAttribute(chol_factor_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      (int)chol_factor_smem()));
-        count_launch(), chol_factor_kernel<<<p.NU, CF_FT, chol_factor_smem(), c.st>>>(G, k, gld, sG, c.status());
-        CUDA_TRY(cudaGetLastError());
-        CUDA_TRY(cudaFuncSetAttribute(tri_inv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      (int)tri_inv_smem()));
-        count_launch(), tri_inv_kernel<<<dim3(nbk, p.NU), CF_THREADS, tri_inv_smem(), c.st>>>(G, k, gld, sG, WT, kq32,
-                                                                                               sW);
-        CUDA_TRY(cudaGetLastError());
-      } else {
-        // 256 < k <= 1024: the cluster Cholesky (chol.cuh), then the block-column inverse
-        count_launch(), sanitize_sym_batched_kernel<<<p.NU, 1024, 0, c.st>>>(G, k, gld, sG, c.status());
-        {
-          ProfScope ps4("chol_steps", c.st, p.NU);
-          for (int J = 0; J < nbk; ++J) {
-            count_launch(), chol_step_diag_kernel<<<p.NU, 32, 0, c.st>>>(G, k, gld, sG, J, c.status());
-            const int below = nbk - J - 1;
-            if (below > 0) {
-              count_launch(), chol_step_panel_kernel<<<dim3(below, p.NU), CF_THREADS, 0, c.st>>>(G, k, gld, sG, J);
-              count_launch(), chol_step_update_kernel<<<dim3(below * (below + 1) / 2, p.NU), CF_THREADS, 0, c.st>>>(
-                  G, k, gld, sG, J);
-            }
+      CUDA_TRY(cudaFuncSetAttribute(tri_inv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)tri_inv_smem()));
+      count_launch(), tri_inv_kernel<<<dim3(nbk, p.NU), CF_THREADS, tri_inv_smem(), c.st>>>(G, k, gld, sG, WT, kq32,
+                                                                                             sW);
+      CUDA_TRY(cudaGetLastError());
+    } else {
+      // 256 < k <= 1024: the cluster Cholesky (chol.cuh), then the block-column inverse
+      count_launch(), sanitize_sym_batched_kernel<<<p.NU, 1024, 0, c.st>>>(G, k, gld, sG, c.status());
+      {
+        ProfScope ps4("chol_steps", c.st, p.NU);
+        for (int J = 0; J < nbk; ++J) {
+          count_launch(), chol_step_diag_kernel<<<p.NU, 32, 0, c.st>>>(G, k, gld, sG, J, c.status());
+          const int below = nbk - J - 1;
+          if (below > 0) {
+            count_launch(), chol_step_panel_kernel<<<dim3(below, p.NU), CF_THREADS, 0, c.st>>>(G, k, gld, sG, J);
+            count_launch(), chol_step_update_kernel<<<dim3(below * (below + 1) / 2, p.NU), CF_THREADS, 0, c.st>>>(
+                G, k, gld, sG, J);
           }
-          CUDA_TRY(cudaGetLastError());
         }
-        ProfScope ps5("tri_inv_large", c.st, p.NU);
-        count_launch(), tri_inv_large_kernel<<<dim3(nbk, p.NU), CF_THREADS, 0, c.st>>>(
-            G, k, gld, sG, c.at<double>(p.o_winv), kq32, WT, kq32, sW);
         CUDA_TRY(cudaGetLastError());
       }
-    }
-    {
-      ProfScope ps3("qr_trsm", c.st, p.NU);
-      const long long nW = (long long)p.NU * sW;
-      count_launch(), split_bf16_kernel<<<grid1d(nW), 256, 0, c.st>>>(WT, wth, wtl, nW);
+      ProfScope ps5("tri_inv_large", c.st, p.NU);
+      count_launch(), tri_inv_large_kernel<<<dim3(nbk, p.NU), CF_THREADS, 0, c.st>>>(
+          G, k, gld, sG, c.at<double>(p.o_winv), kq32, WT, kq32, sW);
       CUDA_TRY(cudaGetLastError());
-      UmmaArgs q;
-      q.M = (int)m;
-      q.N = k;
-      q.K = k;
-      q.batch = p.NU;
-      q.A.mode = UM_DENSE_K;
-      q.B.mode = UM_DENSE_MN;
-      q.tri = 2;
-      q.bn = 128;
-      q.C = Y;
-      q.ldc = ld;
-      q.sC = m * ld;
-      q.status = c.status();
-      UmmaMaps m3;   // Yh Wh^T + Yh Wl^T + Yl Wh^T in one pass
-      m3.a0 = my.a0;
-      m3.a1 = my.a1;
-      m3.b0 = mw.b0;
-      m3.b1 = mw.b1;
-      JTRY(umma_run(c, m3, q, 3));
     }
+  }
+  {
+    ProfScope ps3("qr_trsm", c.st, p.NU);
+    const long long nW = (long long)p.NU * sW;
+    count_launch(), split_bf16_kernel<<<grid1d(nW), 256, 0, c.st>>>(WT, wth, wtl, nW);
+    CUDA_TRY(cudaGetLastError());
+    UmmaArgs q;
+    q.M = (int)m;
+    q.N = k;
+    q.K = k;
+    q.batch = p.NU;
+    q.A.mode = UM_DENSE_K;
+    q.B.mode = UM_DENSE_MN;
+    q.tri = 2;
+    q.bn = 128;
+    if (outY) {
+      q.C = outY;
+    } else {
+      q.N = ld;   // the pair gets every column (k..ld from zero rows of W^T)
+      q.C = oh;
+      q.C2 = ol;
+      q.c_split = 1;
+    }
+    q.ldc = ld;
+    q.sC = m * ld;
+    q.status = c.status();
+    UmmaMaps m3;   // Yh Wh^T + Yh Wl^T + Yl Wh^T in one pass
+    m3.a0 = my.a0;
+    m3.a1 = my.a1;
+    m3.b0 = mw.b0;
+    m3.b1 = mw.b1;
+    JTRY(umma_run(c, m3, q, 3));
   }
   return JOLT_OK;
 }
 
-// z_side = false: out (T x k per unit) = X_(T) F, F = M x kp ; z_side = true: out (M x k) =
-// X_(T)^T F, F = T x kp.  F is bf16 (F16, one operand) or fp32 (F32, split into hi + lo).
-jolt_status umma_product(const Ctx& c, bool z_side, const bf16* F16, const float* F32, float* out) {
+jolt_status cholqr_tc(const Ctx& c, float* Y, long long m, int k, int ld, int passes) {
+  const Plan& p = c.p;
+  ProfScope ps("cholesky_qr", c.st, p.NU);
+  if (k > 1024) return fail(JOLT_ERR_UNSUPPORTED_SHAPE, "Cholesky QR of more than 1024 columns");
+  if (ld % 8) return fail(JOLT_ERR_UNSUPPORTED_SHAPE, "Cholesky QR pitch %d not a multiple of 8", ld);
+  bf16* yh = c.at<bf16>(p.o_h);
+  bf16* yl = c.at<bf16>(p.o_l);
+  const long long nY = (long long)p.NU * m * ld;
+  for (int pass = 0; pass < passes; ++pass) {
+    count_launch(), split_bf16_cols_kernel<<<grid1d(nY), 256, 0, c.st>>>(Y, yh, yl, nY, ld, k);
+    CUDA_TRY(cudaGetLastError());
+    JTRY(qr_pass_tc(c, yh, yl, m, k, ld, Y, nullptr, nullptr));
+  }
+  return JOLT_OK;
+}
+
+// Cholesky QR of a block held as bf16 pairs: pass i reads pair *cur and writes the other pair,
+// so *cur names the pair holding Q afterwards.
+jolt_status cholqr_tc_pairs(const Ctx& c, bf16* const* ph, bf16* const* pl, int* cur, long long m, int k, int ld,
+                            int passes) {
+  const Plan& p = c.p;
+  ProfScope ps("cholesky_qr", c.st, p.NU);
+  if (k > 1024) return fail(JOLT_ERR_UNSUPPORTED_SHAPE, "Cholesky QR of more than 1024 columns");
+  if (ld % 8) return fail(JOLT_ERR_UNSUPPORTED_SHAPE, "Cholesky QR pitch %d not a multiple of 8", ld);
+  for (int pass = 0; pass < passes; ++pass) {
+    const int i = *cur, o = i ^ 1;
+    JTRY(qr_pass_tc(c, ph[i], pl[i], m, k, ld, nullptr, ph[o], pl[o]));
+    *cur = o;
+  }
+  return JOLT_OK;
+}
+
+// z_side = false: out (T x N per unit) = X_(T) F, F = M x kp ; z_side = true: out (M x N) =
+// X_(T)^T F, F = T x kp, with F = f0 (+ f1, bf16 operands).  out is fp32, or with out2 the
+// result as a bf16 hi (out) + lo (out2) pair; pitch kp.
+jolt_status umma_x(const Ctx& c, bool z_side, const bf16* f0, const bf16* f1, int N, void* out, void* out2) {
   const Plan& p = c.p;
   ProfScope ps("sketch_product", c.st, p.NU);
+  cudaError_t e = umma_x_product(c.k, c.v, p.nL, p.H, p.T, p.D, p.S, p.NU, z_side, f0, f1, p.kp, N, out, p.kp,
+                                 c.status(), c.sched(), c.st, out2);
+  if (e != cudaSuccess) return fail(JOLT_ERR_CUDA, "tensor-core X-product: %s", cudaGetErrorString(e));
+  return JOLT_OK;
+}
+
+// the same with F given as bf16 (F16, one operand) or fp32 (F32, split into hi + lo into
+// (hi, lo), which must hold NU x rows(F) x kp); fp32 output with N = k
+jolt_status umma_product(const Ctx& c, bool z_side, const bf16* F16, const float* F32, float* out, bf16* hi = nullptr,
+                         bf16* lo = nullptr) {
+  const Plan& p = c.p;
   const bf16* f0 = F16;
   const bf16* f1 = nullptr;
   if (F32) {
-    bf16* hi = c.at<bf16>(p.o_h);
-    bf16* lo = c.at<bf16>(p.o_l);
+    if (!hi) {
+      hi = c.at<bf16>(p.o_h);
+      lo = c.at<bf16>(p.o_l);
+    }
     const long long nF = (long long)p.NU * (z_side ? p.T : p.M) * p.kp;
     count_launch(), split_bf16_kernel<<<grid1d(nF), 256, 0, c.st>>>(F32, hi, lo, nF);
     CUDA_TRY(cudaGetLastError());
     f0 = hi;
     f1 = lo;
   }
-  cudaError_t e = umma_x_product(c.k, c.v, p.nL, p.H, p.T, p.D, p.S, p.NU, z_side, f0, f1, p.kp, p.k, out, p.kp,
-                                 c.status(), c.sched(), c.st);
-  if (e != cudaSuccess) return fail(JOLT_ERR_CUDA, "tensor-core X-product: %s", cudaGetErrorString(e));
-  return JOLT_OK;
+  return umma_x(c, z_side, f0, f1, p.k, out, nullptr);
 }
 
 // the cache of every unit as a batched operand: X_(T) (T x M, rows t, columns (l,h,d))
@@ -1088,7 +1143,7 @@ jolt_status run_token_randomized(const Ctx& c, float* Uf, long long ldUf) {
   bf16* Om = c.at<bf16>(p.o_omega);
   float* Y = c.at<float>(p.o_Y);
   float* Z = c.at<float>(p.o_Zm);
-  CUDA_TRY(cudaMemsetAsync(Y, 0, (size_t)NU * T * kp * 4, c.st));
+  if (p.o_Y) CUDA_TRY(cudaMemsetAsync(Y, 0, (size_t)NU * T * kp * 4, c.st));   // no fp32 Y with the pairs
   CUDA_TRY(cudaMemsetAsync(Z, 0, (size_t)NU * M * kp * 4, c.st));
   count_launch(), omega_kernel<<<grid1d((long long)NU * M * kp), 256, 0, c.st>>>(Om, M, k, kp, (long long)M * kp,
                                                                                   c.seed, p.u0, NU);
@@ -1113,7 +1168,14 @@ jolt_status run_token_randomized(const Ctx& c, float* Uf, long long ldUf) {
   gz.C = Z;
   gz.sbatchC = (long long)M * kp;
   const bool tc = umma_ok(p);
-  if (tc) {
+  // the pairs path: every T x k basis as bf16 hi + lo, in pair 0 or 1 (cur names Q's)
+  const bool pairs = tc && p.o_h2;
+  bf16* ph[2] = {c.at<bf16>(p.o_h), pairs ? c.at<bf16>(p.o_h2) : nullptr};
+  bf16* pl[2] = {c.at<bf16>(p.o_l), pairs ? c.at<bf16>(p.o_l2) : nullptr};
+  int cur = 0;
+  if (pairs) {
+    JTRY(umma_x(c, false, Om, nullptr, kp, ph[0], pl[0]));   // Y = X_(T) Omega, all kp columns
+  } else if (tc) {
     JTRY(umma_product(c, false, Om, nullptr, Y));   // Y = X_(T) Omega
   } else {
     ProfScope ps0("sketch_product", c.st, NU);
@@ -1130,15 +1192,32 @@ jolt_status run_token_randomized(const Ctx& c, float* Uf, long long ldUf) {
   auto y_of = [&](const float* Qz) -> jolt_status {  // Y = X_(T) Qz
     return tc ? umma_product(c, false, nullptr, Qz, Y) : gemm_xf(c, gy, false, Qz, (long long)NU * M * kp);
   };
-  JTRY(cholqr_batched(c, Y, T, k, kp, p.q == 0 ? 2 : 1));
-  for (int it = 0; it < p.q; ++it) {
+  if (pairs) {
+    bf16* mh = c.at<bf16>(p.o_mh);
+    bf16* ml = c.at<bf16>(p.o_ml);
+    JTRY(cholqr_tc_pairs(c, ph, pl, &cur, T, k, kp, p.q == 0 ? 2 : 1));
+    for (int it = 0; it < p.q; ++it) {
+      JTRY(umma_x(c, true, ph[cur], pl[cur], k, Z, nullptr));    // Z = X_(T)^T Q
+      JTRY(cholqr_batched(c, Z, M, k, kp, 1));   // its scratch pair may overwrite Q: used above
+      const long long nZ = (long long)NU * M * kp;
+      count_launch(), split_bf16_kernel<<<grid1d(nZ), 256, 0, c.st>>>(Z, mh, ml, nZ);
+      CUDA_TRY(cudaGetLastError());
+      cur = 0;
+      JTRY(umma_x(c, false, mh, ml, kp, ph[0], pl[0]));   // Y = X_(T) Qz
+      JTRY(cholqr_tc_pairs(c, ph, pl, &cur, T, k, kp, it + 1 == p.q ? 2 : 1));
+    }
+    JTRY(umma_x(c, true, ph[cur], pl[cur], k, Z, nullptr));   // Rayleigh-Ritz: Z = X_(T)^T Q
+  } else {
+    JTRY(cholqr_batched(c, Y, T, k, kp, p.q == 0 ? 2 : 1));
+    for (int it = 0; it < p.q; ++it) {
+      JTRY(z_of(Y));
+      JTRY(cholqr_batched(c, Z, M, k, kp, 1));
+      JTRY(y_of(Z));
+      JTRY(cholqr_batched(c, Y, T, k, kp, it + 1 == p.q ? 2 : 1));
+    }
+    // Rayleigh-Ritz: S = Z^T Z with Z = X_(T)^T Q  (k x k per unit)
     JTRY(z_of(Y));
-    JTRY(cholqr_batched(c, Z, M, k, kp, 1));
-    JTRY(y_of(Z));
-    JTRY(cholqr_batched(c, Y, T, k, kp, it + 1 == p.q ? 2 : 1));
   }
-  // Rayleigh-Ritz: S = Z^T Z with Z = X_(T)^T Q  (k x k per unit)
-  JTRY(z_of(Y));
   float* gpart = c.at<float>(p.o_gpart);
   double* S = c.at<double>(p.o_G);
   const int ns = (int)ceil_div(M, 256);
@@ -1174,12 +1253,12 @@ jolt_status run_token_randomized(const Ctx& c, float* Uf, long long ldUf) {
   ProfScope ps2("ritz_vectors", c.st, NU);
   if (p.o_vh) {
     // on the tensor cores: Q = Qh + Ql, V = Vh + Vl (bf16 hi + lo); U = Qh (Vh + Vl) + Ql Vh
-    bf16* qh = c.at<bf16>(p.o_h);
-    bf16* ql = c.at<bf16>(p.o_l);
+    bf16* qh = ph[cur];
+    bf16* ql = pl[cur];
     bf16* vh = c.at<bf16>(p.o_vh);
     bf16* vl = c.at<bf16>(p.o_vl);
     const long long nQ = (long long)NU * T * kp, nV = (long long)NU * kp * p.ldU;
-    count_launch(), split_bf16_cols_kernel<<<grid1d(nQ), 256, 0, c.st>>>(Y, qh, ql, nQ, kp, k);
+    if (!pairs) count_launch(), split_bf16_cols_kernel<<<grid1d(nQ), 256, 0, c.st>>>(Y, qh, ql, nQ, kp, k);
     count_launch(), split_bf16_kernel<<<grid1d(nV), 256, 0, c.st>>>(V, vh, vl, nV);
     CUDA_TRY(cudaGetLastError());
     UmmaMaps mq, mv;

@@ -56,6 +56,8 @@ struct UmmaArgs {
   bool b_is_a = false;        // Gram of one operand: B's tile is A's tile (M = N = 128, one tile)
   void* C = nullptr;
   int c_bf16 = 0;             // 0: fp32 output, 1: bf16 (round to nearest)
+  int c_split = 0;            // 1: the fp32 result as a bf16 pair: C = bf16(v), C2 = bf16(v - C)
+  void* C2 = nullptr;
   int c_accum = 0;            // fp32 output only: add the product to what C holds
   int tri = 0;                // 1: only output tiles that reach the diagonal or above it
                               //    (n0 + BN > m0; the upper triangle of a symmetric product);
@@ -472,9 +474,9 @@ __global__ void __launch_bounds__(192, 1)
   } else {
     // ---- epilogue: warp w owns TMEM lanes 32 (w % 4) .. +31, i.e. output rows m0 + 32 (w % 4) + lane ----
     const int q4 = warp & 3;
-    const int esz = a.c_bf16 ? 2 : 4;
+    const int esz = (a.c_bf16 || a.c_split) ? 2 : 4;
     const bool vec = ((a.ldc * esz) % 16 == 0) && ((((uintptr_t)a.C) & 15) == 0) && ((a.sC * esz) % 16 == 0) &&
-                     ((a.ssplit * esz) % 16 == 0);
+                     ((a.ssplit * esz) % 16 == 0) && (!a.c_split || (((uintptr_t)a.C2) & 15) == 0);
     int tc = 0;
     for (int j = 0;; ++j) {
       const int t = ring_take(j, true);
@@ -508,7 +510,34 @@ __global__ void __launch_bounds__(192, 1)
         }
         if (row >= a.M) continue;
         const int n = n0 + c0;
-        if (a.c_bf16) {
+        if (a.c_split) {
+          bf16* hrow = (bf16*)a.C + off;
+          bf16* lrow = (bf16*)a.C2 + off;
+          if (vec && n + 32 <= a.N) {
+#pragma unroll
+            for (int j = 0; j < 32; j += 8) {
+              uint32_t hw[4], lw[4];
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                const __nv_bfloat162 h = __floats2bfloat162_rn(v[j + 2 * q], v[j + 2 * q + 1]);
+                const __nv_bfloat162 l = __floats2bfloat162_rn(v[j + 2 * q] - __low2float(h),
+                                                               v[j + 2 * q + 1] - __high2float(h));
+                hw[q] = *(const uint32_t*)&h;
+                lw[q] = *(const uint32_t*)&l;
+              }
+              *(uint4*)(hrow + n + j) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+              *(uint4*)(lrow + n + j) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+            }
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (n + j < a.N) {
+                const bf16 h = __float2bfloat16_rn(v[j]);
+                hrow[n + j] = h;
+                lrow[n + j] = __float2bfloat16_rn(v[j] - __bfloat162float(h));
+              }
+          }
+        } else if (a.c_bf16) {
           bf16* crow = (bf16*)a.C + off;
           if (vec && n + 32 <= a.N) {
 #pragma unroll
@@ -651,6 +680,7 @@ inline cudaError_t launch_umma(const UmmaMaps& m, UmmaArgs a, int nb, cudaStream
     return cudaErrorInvalidValue;
   if (a.splits == 1) a.kchunk = (int)round_up(a.K, umma::BK);
   if (a.c_accum && a.c_bf16) return cudaErrorInvalidValue;
+  if (a.c_split && (!a.C2 || a.c_bf16 || a.c_accum)) return cudaErrorInvalidValue;
   // N tiles of 256 only with one B operand: with two (hi + lo) a 256-wide stage takes 80 KB and
   // leaves room for two pipeline stages, a 128-wide one 48 KB and four
   if (nb == 3) return launch_umma_bn<128, 3>(m, a, st);   // a 64 KB stage: three stages
@@ -663,9 +693,10 @@ inline cudaError_t launch_umma(const UmmaMaps& m, UmmaArgs a, int nb, cudaStream
 //   z_side = false : C_u (T x N) = X_(T),u   * sum_b F_b,u   with F_b,u = Fb[u] (M x ldf)
 //   z_side = true  : C_u (M x N) = X_(T),u^T * sum_b F_b,u   with F_b,u = Fb[u] (T x ldf)
 // xk / xv: the K and V caches [n_layers][H][T][D] bf16; F1 may be null (one B operand).
+// C: fp32, or with C2 the result as a bf16 hi (C) + lo (C2) pair, pitch ldc.
 inline cudaError_t umma_x_product(const void* xk, const void* xv, int n_layers, int H, int T, int D, int S,
-                                  int nunits, bool z_side, const bf16* F0, const bf16* F1, int ldf, int N, float* C,
-                                  long long ldc, uint32_t* status, int* sched, cudaStream_t st) {
+                                  int nunits, bool z_side, const bf16* F0, const bf16* F1, int ldf, int N, void* C,
+                                  long long ldc, uint32_t* status, int* sched, cudaStream_t st, void* C2 = nullptr) {
   if (D % 64 || ldf % 8 || N > ldf) return cudaErrorInvalidValue;
   int dshift = 0;
   while ((1 << dshift) < D) ++dshift;
@@ -689,6 +720,10 @@ inline cudaError_t umma_x_product(const void* xk, const void* xv, int n_layers, 
   a.sC = (long long)a.M * ldc;
   a.status = status;
   a.sched = sched;
+  if (C2) {
+    a.c_split = 1;
+    a.C2 = C2;
+  }
   return launch_umma(m, a, F1 ? 2 : 1, st);
 }
 
