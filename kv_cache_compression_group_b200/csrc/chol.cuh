@@ -424,29 +424,35 @@ namespace jolt {
 
 // ------------------------------------------------------------------------------------------
 // W = L^{-1} for any k (the block-column recursion of tri_inv_kernel with the block column
-// kept in global fp64 scratch instead of shared memory):
+// kept in global fp64 scratch instead of shared memory; each sum over K split over TI_G thread
+// groups and added in group order):
 //   W_JJ = inv(L_JJ),   W_IJ = -inv(L_II) sum_{J <= K < I} L_IK W_KJ   (I > J).
 // G: L's blocks below the diagonal in the lower triangle, inv(L_II) in the upper part of
-// the diagonal blocks.  One CTA per (block column J, unit), 256 threads, thread (r, cg)
-// computes entries (r, cg + 8 j) of each 32 x 32 block.  scr: per unit and block column a
-// kq32 x 32 fp64 slab (row i of the slab = row i of W).  Output as tri_inv_kernel: WT[q][i] =
-// W[i][q] in fp32 at pitch ldw, zeros for i < J0 and for k <= i < ldw.
+// the diagonal blocks.  One CTA per (block column J, unit), TI_G x 256 threads (dynamic
+// shared memory tri_inv_large_smem()); thread (r, cg) of a group computes entries (r, cg + 8 j)
+// of each 32 x 32 block.  scr: per unit and block column a kq32 x 32 fp64 slab (row i of the
+// slab = row i of W).  Output as tri_inv_kernel: WT[q][i] = W[i][q] in fp32 at pitch ldw, zeros
+// for i < J0 and for k <= i < ldw.
 // ------------------------------------------------------------------------------------------
-__global__ void __launch_bounds__(CF_THREADS) tri_inv_large_kernel(const double* G, int k, long long gld, long long sG,
-                                                                  double* scr, int kq32, float* WT, long long ldw,
-                                                                  long long sW) {
-  __shared__ double Ls[CF_NB][CF_P];    // L_IK, [r][q]
-  __shared__ double Xs[CF_NB][CF_P];    // W_KJ, [q][c]
-  __shared__ double Ts[CF_NB][CF_P];    // sum_K L_IK W_KJ
-  __shared__ double Ds[CF_NB][CF_P];    // inv(L_II)
+constexpr int TI_G = 4;   // K blocks of one sum formed at once, one thread group of CF_THREADS each
+inline size_t tri_inv_large_smem() { return sizeof(double) * (3 * TI_G + 1) * CF_NB * CF_P; }
+__global__ void __launch_bounds__(CF_THREADS * TI_G) tri_inv_large_kernel(const double* G, int k, long long gld,
+                                                                         long long sG, double* scr, int kq32, float* WT,
+                                                                         long long ldw, long long sW) {
+  extern __shared__ double ti_sm[];
+  double(*Ls)[CF_NB][CF_P] = reinterpret_cast<double(*)[CF_NB][CF_P]>(ti_sm);   // [TI_G] L_IK, [r][q]
+  double(*Xs)[CF_NB][CF_P] = Ls + TI_G;                                          // [TI_G] W_KJ, [q][c]
+  double(*Tg)[CF_NB][CF_P] = Xs + TI_G;                                          // [TI_G] partial sums
+  double(*Ds)[CF_P] = reinterpret_cast<double(*)[CF_P]>(Tg + TI_G);            // inv(L_II)
   const int J = blockIdx.x, u = blockIdx.y, tid = threadIdx.x;
+  const int g = tid / CF_THREADS, lt = tid - g * CF_THREADS;
   const int nbk = (k + CF_NB - 1) / CF_NB;
   const int J0 = J * CF_NB, nbJ = min(CF_NB, k - J0);
   const double* Gu = G + (long long)u * sG;
   double* X = scr + ((long long)u * nbk + J) * (long long)kq32 * CF_NB;   // X[i * 32 + c]
-  const int r = tid >> 3, cg = tid & 7;
+  const int r = lt >> 3, cg = lt & 7;
   // W_JJ
-  for (int idx = tid; idx < CF_NB * CF_NB; idx += CF_THREADS) {
+  for (int idx = tid; idx < CF_NB * CF_NB; idx += blockDim.x) {
     const int rr = idx / CF_NB, c = idx % CF_NB;
     X[(long long)(J0 + rr) * CF_NB + c] =
         (rr < nbJ && c < nbJ && c <= rr) ? Gu[(long long)(J0 + rr) * gld + J0 + c] : 0.0;
@@ -454,44 +460,53 @@ __global__ void __launch_bounds__(CF_THREADS) tri_inv_large_kernel(const double*
   __syncthreads();
   for (int I = J + 1; I < nbk; ++I) {
     const int I0 = I * CF_NB, nbI = min(CF_NB, k - I0);
+    // group g sums the K blocks J + g, J + g + TI_G, ... (its own barrier: the trip counts differ)
     double acc[4] = {0.0, 0.0, 0.0, 0.0};
-    for (int K = J; K < I; ++K) {
+    for (int K = J + g; K < I; K += TI_G) {
       const int K0 = K * CF_NB, nbK = min(CF_NB, k - K0);
-      for (int idx = tid; idx < CF_NB * CF_NB; idx += CF_THREADS) {
+      for (int idx = lt; idx < CF_NB * CF_NB; idx += CF_THREADS) {
         const int a = idx / CF_NB, b = idx % CF_NB;
         // L_IK[b][a] = L[I0 + b][K0 + a], column-major at G[(K0 + a) * gld + I0 + b]: consecutive
         // threads read consecutive rows of one column
-        Ls[b][a] = (b < nbI && a < nbK) ? Gu[(long long)(K0 + a) * gld + I0 + b] : 0.0;
-        Xs[a][b] = a < nbK ? X[(long long)(K0 + a) * CF_NB + b] : 0.0;
+        Ls[g][b][a] = (b < nbI && a < nbK) ? Gu[(long long)(K0 + a) * gld + I0 + b] : 0.0;
+        Xs[g][a][b] = a < nbK ? X[(long long)(K0 + a) * CF_NB + b] : 0.0;
       }
-      __syncthreads();
+      asm volatile("bar.sync %0, %1;" ::"r"(1 + g), "n"(CF_THREADS) : "memory");
 #pragma unroll 8
       for (int q = 0; q < CF_NB; ++q) {
-        const double l = Ls[r][q];
+        const double l = Ls[g][r][q];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) acc[j] = fma(l, Xs[q][cg + 8 * j], acc[j]);
+        for (int j = 0; j < 4; ++j) acc[j] = fma(l, Xs[g][q][cg + 8 * j], acc[j]);
       }
-      __syncthreads();
+      asm volatile("bar.sync %0, %1;" ::"r"(1 + g), "n"(CF_THREADS) : "memory");
     }
 #pragma unroll
-    for (int j = 0; j < 4; ++j) Ts[r][cg + 8 * j] = acc[j];
-    for (int idx = tid; idx < CF_NB * CF_NB; idx += CF_THREADS) {
-      const int rr = idx / CF_NB, s = idx % CF_NB;
-      Ds[rr][s] = (rr < nbI && s <= rr) ? Gu[(long long)(I0 + rr) * gld + I0 + s] : 0.0;
+    for (int j = 0; j < 4; ++j) Tg[g][r][cg + 8 * j] = acc[j];
+    for (int idx = tid; idx < CF_NB * CF_NB; idx += blockDim.x) {
+      const int rr = idx / CF_NB, s2 = idx % CF_NB;
+      Ds[rr][s2] = (rr < nbI && s2 <= rr) ? Gu[(long long)(I0 + rr) * gld + I0 + s2] : 0.0;
     }
     __syncthreads();
-    double out[4] = {0.0, 0.0, 0.0, 0.0};
-    for (int s = 0; s <= r; ++s) {
-      const double d = Ds[r][s];
+    if (g == 0) {
+      // W_IJ = -inv(L_II) (sum over the groups, in group order)
+      double out[4] = {0.0, 0.0, 0.0, 0.0};
+      for (int s2 = 0; s2 <= r; ++s2) {
+        const double d = Ds[r][s2];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) out[j] = fma(d, Ts[s][cg + 8 * j], out[j]);
+        for (int j = 0; j < 4; ++j) {
+          double t = Tg[0][s2][cg + 8 * j];
+#pragma unroll
+          for (int gg = 1; gg < TI_G; ++gg) t += Tg[gg][s2][cg + 8 * j];
+          out[j] = fma(d, t, out[j]);
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < 4; ++j) X[(long long)(I0 + r) * CF_NB + cg + 8 * j] = r < nbI ? -out[j] : 0.0;
     }
-#pragma unroll
-    for (int j = 0; j < 4; ++j) X[(long long)(I0 + r) * CF_NB + cg + 8 * j] = r < nbI ? -out[j] : 0.0;
     __syncthreads();
   }
   float* Wu = WT + (long long)u * sW;
-  for (int c = tid >> 5; c < nbJ; c += CF_THREADS / 32)
+  for (int c = tid >> 5; c < nbJ; c += blockDim.x / 32)
     for (int i = tid & 31; i < ldw; i += 32)
       Wu[(long long)(J0 + c) * ldw + i] = (i >= J0 && i < k) ? (float)X[(long long)i * CF_NB + c] : 0.f;
 }

@@ -177,7 +177,7 @@ struct Plan {
   size_t fsolver_dev;     // cuSOLVER device workspace (feature factor, on the auxiliary stream)
   size_t solver_host;
   // workspace offsets (bytes)
-  size_t o_signkey, o_sign;
+  size_t o_signkey, o_sign, o_ctmp;
   size_t o_status, o_gd_part, o_gd, o_evals, o_Wf, o_Ws, o_Uf, o_Us, o_core, o_zc, o_ptmp, o_P, o_partial,
       o_table, o_bytes, o_choice, o_lambda, o_hdr, o_umap, o_info, o_solver, o_fsolver, o_finfo, o_fevals, o_eigvec, o_eigscr,
       o_feigvec, o_feigscr;
@@ -344,6 +344,7 @@ jolt_status make_plan(const jolt_shape* sh, const jolt_options* op, Plan* p) {
   p->o_Us = b.take((size_t)NU * T * p->ldU * 2);
   p->o_core = b.take((size_t)NU * S * p->rTmax * p->ldC * 2);
   p->o_zc = b.take((size_t)NU * S * T * p->ldW * 2);
+  p->o_ctmp = b.take((size_t)NU * S * p->rTmax * p->ldW * 2);   // the core before its permutation
   p->o_ptmp = b.take((size_t)NU * S * p->rTmax * D * 4);
   p->o_P = b.take((size_t)NU * p->cd.nD * S * p->rTmax * D * 2);
   p->o_partial = b.take((size_t)NU * S * p->tiles * p->nC * 8);
@@ -857,7 +858,9 @@ jolt_status qr_pass_tc(const Ctx& c, const bf16* yh, const bf16* yl, long long m
         CUDA_TRY(cudaGetLastError());
       }
       ProfScope ps5("tri_inv_large", c.st, p.NU);
-      count_launch(), tri_inv_large_kernel<<<dim3(nbk, p.NU), CF_THREADS, 0, c.st>>>(
+      CUDA_TRY(cudaFuncSetAttribute(tri_inv_large_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)tri_inv_large_smem()));
+      count_launch(), tri_inv_large_kernel<<<dim3(nbk, p.NU), CF_THREADS * TI_G, tri_inv_large_smem(), c.st>>>(
           G, k, gld, sG, c.at<double>(p.o_winv), kq32, WT, kq32, sW);
       CUDA_TRY(cudaGetLastError());
     }
@@ -1349,45 +1352,56 @@ jolt_status run_core(const Ctx& c, const bf16* Us, long long ldU, const bf16* Ws
   const int T = p.T, D = p.D, S = p.S;
   bf16* Zc = c.at<bf16>(p.o_zc);
   if (umma_ok(p)) {
-    // Z = bf16(X_(D) W_s) : A = X_(D) rows (K-major), B = W_s (D x rDmax, MN-major)
-    UmmaMaps m;
-    JTRY(cache_maps(c, true, &m.a0, &m.a1));
-    if (!map_dense(&m.b0, Ws, ldW, D, p.NU)) return fail(JOLT_ERR_CUDA, "tensor map of W refused");
-    m.b1 = m.b0;
-    UmmaArgs a;
-    a.M = S * T;
-    a.N = p.rDmax;
-    a.K = D;
-    a.batch = p.NU;
-    a.A.mode = UM_ROW_K;
-    a.A.rows = (long long)S * T;
-    a.B.mode = UM_DENSE_MN;
-    a.C = Zc;
-    a.c_bf16 = 1;
-    a.ldc = p.ldW;
-    a.sC = (long long)S * T * p.ldW;
-    a.status = c.status();
-    JTRY(umma_run(c, m, a, 1));
-    // C_s = bf16(U_s^T Z_s) per (unit, slice): A = U_s^T (MN-major, shared by the S slices)
+    // Z_u = bf16(X_u W_u) token-major, Z[u][t][s * ldW + c]: one launch per unit, its slices as
+    // the batch (A = the unit's cache slices [S][T][D], K-major; B = W_u, MN-major)
+    const long long zld = (long long)S * p.ldW;
+    for (int u = 0; u < p.NU; ++u) {
+      const bf16* base = reinterpret_cast<const bf16*>((u & 1) ? c.v : c.k) + (long long)(u >> 1) * S * T * D;
+      UmmaMaps m;
+      if (!map_dense(&m.a0, base, D, T, S) || !map_dense(&m.b0, Ws + (long long)u * D * ldW, ldW, D, 1))
+        return fail(JOLT_ERR_CUDA, "tensor map of X / W refused");
+      m.a1 = m.a0;
+      m.b1 = m.b0;
+      UmmaArgs a;
+      a.M = T;
+      a.N = p.rDmax;
+      a.K = D;
+      a.batch = S;
+      a.A.mode = UM_DENSE_K;
+      a.B.mode = UM_DENSE_MN;
+      a.B.ediv = S;   // every slice uses the unit's W
+      a.C = Zc + (long long)u * T * zld;
+      a.c_bf16 = 1;
+      a.ldc = zld;
+      a.sC = p.ldW;
+      a.status = c.status();
+      JTRY(umma_run(c, m, a, 1));
+    }
+    // C_u = bf16(U_u^T Z_u) (rTmax x S ldW per unit; N tiles of 256), then into the stored
+    // layout [u][s][rTmax][ldC]
+    bf16* Ct = c.at<bf16>(p.o_ctmp);
     UmmaMaps m2;
-    if (!map_dense(&m2.a0, Us, ldU, T, p.NU) || !map_dense(&m2.b0, Zc, p.ldW, T, (long long)p.NU * S))
+    if (!map_dense(&m2.a0, Us, ldU, T, p.NU) || !map_dense(&m2.b0, Zc, zld, T, p.NU))
       return fail(JOLT_ERR_CUDA, "tensor map of U / Z refused");
     m2.a1 = m2.a0;
     m2.b1 = m2.b0;
     UmmaArgs a2;
     a2.M = p.rTmax;
-    a2.N = p.rDmax;
+    a2.N = (int)zld;
     a2.K = T;
-    a2.batch = p.NU * S;
+    a2.batch = p.NU;
     a2.A.mode = UM_DENSE_MN;
-    a2.A.ediv = S;
     a2.B.mode = UM_DENSE_MN;
-    a2.C = core;
+    a2.C = Ct;
     a2.c_bf16 = 1;
-    a2.ldc = p.ldC;
-    a2.sC = (long long)p.rTmax * p.ldC;
+    a2.ldc = zld;
+    a2.sC = (long long)p.rTmax * zld;
     a2.status = c.status();
-    return umma_run(c, m2, a2, 1);
+    JTRY(umma_run(c, m2, a2, 1));
+    const long long n = (long long)p.NU * S * p.rTmax * p.ldC;
+    count_launch(), core_permute_kernel<<<grid1d(n), 256, 0, c.st>>>(Ct, core, p.NU, S, p.rTmax, p.ldW, p.ldC);
+    CUDA_TRY(cudaGetLastError());
+    return JOLT_OK;
   }
   // Z = bf16(X_(D) W_s)   ((S T) x rDmax per unit)
   GemmParams z;

@@ -301,6 +301,22 @@ __global__ void scale_cols_kernel(float* V, const double* lam, int n, int r, lon
   }
 }
 
+// the core from the token-major product, Ct[u][i][s * ldw + c], into its stored layout
+// core[u][s][i][c] (c < ldc <= ldw)
+__global__ void core_permute_kernel(const bf16* Ct, bf16* core, int nunits, int S, int rT, int ldw, int ldc) {
+  const long long total = (long long)nunits * S * rT * ldc;
+  for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < total;
+       e += (long long)gridDim.x * blockDim.x) {
+    const int c = (int)(e % ldc);
+    long long r = e / ldc;
+    const int i = (int)(r % rT);
+    r /= rT;
+    const int s = (int)(r % S);
+    const long long u = r / S;
+    core[e] = Ct[(u * rT + i) * ((long long)S * ldw) + (long long)s * ldw + c];
+  }
+}
+
 // ------------------------------------------------------------------------------------------
 // distortion table finalisation, byte table and the Lagrangian dual
 // ------------------------------------------------------------------------------------------
