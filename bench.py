@@ -328,11 +328,13 @@ def fp32_peak(J, dev, stream):
     return out
 
 
-def stage_rooflines(w, opts, n_units, prof, n_calls, per_call_ms, peaks, peak_src, alu):
+def stage_rooflines(w, opts, n_units, prof, n_calls, per_call_ms, peaks, peak_src, alu, chosen):
     """Algorithmic work of each library stage (per compress call) against its own bound, for
     the stages that take more than 5 % of a compress.  Work counts what the method computes,
     not what the implementation adds (the bf16 hi + lo halves of fp32 operands, recomputed
-    operators): achieved = algorithmic work / measured stage time."""
+    operators, the compensated residual sums of the encoder): achieved = algorithmic work /
+    measured stage time.  `chosen`: the unit records of the blobs of one step (one list per
+    budget), for the stages whose work depends on the allocation."""
     S = w.layers_per_group * w.n_heads
     N = S * w.T * w.D                       # elements per unit
     M = S * w.D
@@ -352,9 +354,14 @@ def stage_rooflines(w, opts, n_units, prof, n_calls, per_call_ms, peaks, peak_sr
         "qr_trsm": ("tensor", ((q + 2) * T + q * M) * float(k) * k * n_units, "FLOP"),
         "ritz_vectors": ("tensor", 2.0 * T * k * rT * n_units, "FLOP"),
         "table_kernel": ("alu", table_alu_ops(w, opts, n_units)[0], "op"),
-        "encode": ("hbm", (2.0 * N) * n_units, "B"),
+        # the reconstruction U_s[:, :r_T] P' of every slice whose unit stores a residual (b > 0),
+        # at the ranks the allocation chose, averaged over the step's budgets
+        "encode": ("tensor", sum(2.0 * w.T * S * w.D * r["r_T"] for recs in chosen for r in recs if r["bits"] > 0)
+                   / max(1, len(chosen)), "FLOP"),
         "feature_factor": ("hbm", 2.0 * N * n_units, "B"),
-        "core": ("hbm", (2.0 * N + 2.0 * N * max(opts.feature_ranks) / w.D) * n_units, "B"),
+        # Z = X W (2 N r_D) and U^T Z (2 r_T T S r_D) at the largest ranks
+        "core": ("tensor", (2.0 * N * max(opts.feature_ranks) + 2.0 * rT * T * S * max(opts.feature_ranks)) * n_units,
+                 "FLOP"),
     }
     lines = []
     for name, (ms, launches, _) in sorted(prof.items(), key=lambda kv: -kv[1][0]):
@@ -494,9 +501,11 @@ def main():
         step(Kd, Vd)
     torch.cuda.synchronize()
     # validity of what is timed: the blobs decode and respect their budgets
+    chosen = []
     for b, blob in zip(budgets, blobs):
-        _, total, _ = J.read_header(blob)
+        _, total, recs = J.read_header(blob)
         assert total <= b
+        chosen.append(recs)
 
     # ---- timed region: device-resident inputs ------------------------------------------
     clocks = ClockSampler(local)
@@ -609,7 +618,7 @@ def main():
     stages = {k: {"ms_total": v[0], "launches": v[1], "ms_per_launch": v[0] / max(1, v[1])} for k, v in prof.items()}
     n_calls = 2 * len(RATIOS)
     per_call_ms = t_ms / args.steps / len(RATIOS)
-    lines = stage_rooflines(w, opts, comp.n_units, prof, n_calls, per_call_ms, peaks, peak_src, alu)
+    lines = stage_rooflines(w, opts, comp.n_units, prof, n_calls, per_call_ms, peaks, peak_src, alu, chosen)
     leaf = [l for l in lines if l.get("bound") in ("alu", "tensor", "hbm")]
     dom = max(leaf, key=lambda l: l["ms_per_launch"]) if leaf else None
     roofline = None

@@ -22,7 +22,7 @@
 //   UM_DENSE_MN dense [entry][K][MN]                                     map {ld, K, entries}
 // Cache modes take map 0 / map 1 for the K / V cache of unit u = 2 g + kv (batch entry u);
 // dense modes take map b for B operand b (NB = 2 sums two B operands, F = hi + lo, into one
-// accumulator).  The K modes are K-major in shared memory, the MN modes MN-major.  D must be
+// accumulator; NB = 4 sums two A operands against one B, which may then be a cache operand).  The K modes are K-major in shared memory, the MN modes MN-major.  D must be
 // a multiple of 64 (a 64-wide box never straddles two slices) and, for the row modes, T a
 // multiple of 64 (a 64-row box never straddles two units).
 //
@@ -59,6 +59,8 @@ struct UmmaArgs {
   int c_split = 0;            // 1: the fp32 result as a bf16 pair: C = bf16(v), C2 = bf16(v - C)
   void* C2 = nullptr;
   int c_accum = 0;            // fp32 output only: add the product to what C holds
+  int c_trans = 0;            // 1: the tile is stored transposed, C[n * ldc + m] (batch stride sC)
+  int m_fast = 0;             // 1: tiles handed out M tile fastest (consecutive tiles share B's tile)
   int tri = 0;                // 1: only output tiles that reach the diagonal or above it
                               //    (n0 + BN > m0; the upper triangle of a symmetric product);
                               // 2: B upper triangular (row k of B is zero for k > every column
@@ -202,11 +204,11 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
 }
 
 // NB = 1: C = A B; NB = 2: C = A (B0 + B1); NB = 3: C = A0 B0 + A0 B1 + A1 B0 (the products of
-// fp32 operands split as bf16 hi + lo, without the lo * lo term)
+// fp32 operands split as bf16 hi + lo, without the lo * lo term); NB = 4: C = (A0 + A1) B
 template <int BN, int NB>
 struct Cfg {
-  static constexpr int NA_OP = NB == 3 ? 2 : 1;        // A operands in a stage
-  static constexpr int NB_OP = NB == 3 ? 2 : NB;       // B operands in a stage
+  static constexpr int NA_OP = NB >= 3 ? 2 : 1;                  // A operands in a stage
+  static constexpr int NB_OP = NB == 3 ? 2 : (NB == 4 ? 1 : NB);  // B operands in a stage
   static constexpr int A_BYTES = BM * BK * 2;          // 16 KB
   static constexpr int B_BYTES = BN * BK * 2;          // BN/64 boxes
   static constexpr int STAGE_BYTES = NA_OP * A_BYTES + NB_OP * B_BYTES;
@@ -295,8 +297,9 @@ __global__ void __launch_bounds__(192, 1)
     const int zz = t / per, rem = t - zz * per;
     bz = zz / a.splits;
     sp = zz - bz * a.splits;
-    m0 = (rem / tN) * umma::BM;
-    n0 = (rem - (rem / tN) * tN) * BN;
+    const int mi = a.m_fast ? rem % tM : rem / tN, ni = a.m_fast ? rem / tM : rem % tN;
+    m0 = mi * umma::BM;
+    n0 = ni * BN;
     if (a.tri == 1 && n0 + BN <= m0) return false;   // wholly below the diagonal: not needed
     kb0 = sp * (a.kchunk / umma::BK);
     const int kend = min(a.tri == 2 ? min(a.K, n0 + BN) : a.K, (sp + 1) * a.kchunk);
@@ -510,6 +513,36 @@ __global__ void __launch_bounds__(192, 1)
         }
         if (row >= a.M) continue;
         const int n = n0 + c0;
+        if (a.c_trans) {
+          // C[n][row]: the warp's lanes hold 32 consecutive rows, so every store of the warp
+          // covers 32 consecutive elements of one output row
+          const long long toff = (long long)bz * a.sC + (long long)sp * a.ssplit + row;
+          if (a.c_split) {
+            bf16* hc = (bf16*)a.C + toff;
+            bf16* lc = (bf16*)a.C2 + toff;
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (n + j < a.N) {
+                const bf16 h = __float2bfloat16_rn(v[j]);
+                hc[(long long)(n + j) * a.ldc] = h;
+                lc[(long long)(n + j) * a.ldc] = __float2bfloat16_rn(v[j] - __bfloat162float(h));
+              }
+          } else if (a.c_bf16) {
+            bf16* cc = (bf16*)a.C + toff;
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (n + j < a.N) cc[(long long)(n + j) * a.ldc] = __float2bfloat16_rn(v[j]);
+          } else {
+            float* cc = (float*)a.C + toff;
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (n + j < a.N) {
+                float* o = cc + (long long)(n + j) * a.ldc;
+                *o = a.c_accum ? *o + v[j] : v[j];
+              }
+          }
+          continue;
+        }
         if (a.c_split) {
           bf16* hrow = (bf16*)a.C + off;
           bf16* lrow = (bf16*)a.C2 + off;
@@ -670,13 +703,14 @@ cudaError_t launch_umma_bn(const UmmaMaps& m, const UmmaArgs& a, cudaStream_t st
   return bmn ? launch_umma_t<BN, NB, false, true>(m, a, st) : launch_umma_t<BN, NB, false, false>(m, a, st);
 }
 
-// C = A * sum_{b < nb} B_b on the tensor cores (nb = 1, 2), or C = A0 B0 + A0 B1 + A1 B0
-// (nb = 3; maps a0, a1, b0, b1; N tiles of 128).  nb >= 2 requires dense B operands, nb = 3
-// dense A operands too; b_is_a requires M = N <= 128 and identical A and B operands.
+// C = A * sum_{b < nb} B_b on the tensor cores (nb = 1, 2), C = A0 B0 + A0 B1 + A1 B0
+// (nb = 3; maps a0, a1, b0, b1; N tiles of 128), or C = (A0 + A1) B (nb = 4; N tiles of 256).
+// nb = 2, 3 require dense B operands, nb = 3, 4 dense A operands; b_is_a requires M = N <= 128
+// and identical A and B operands.
 inline cudaError_t launch_umma(const UmmaMaps& m, UmmaArgs a, int nb, cudaStream_t st) {
-  if (a.splits < 1 || (a.splits > 1 && (a.kchunk <= 0 || a.kchunk % umma::BK)) || a.batch < 1 || nb < 1 || nb > 3 ||
-      (nb >= 2 && umma::cache_mode(a.B.mode)) || (nb == 3 && (umma::cache_mode(a.A.mode) || a.b_is_a)) ||
-      (a.b_is_a && (a.M > 128 || a.N > 128 || nb != 1)))
+  if (a.splits < 1 || (a.splits > 1 && (a.kchunk <= 0 || a.kchunk % umma::BK)) || a.batch < 1 || nb < 1 || nb > 4 ||
+      ((nb == 2 || nb == 3) && umma::cache_mode(a.B.mode)) ||
+      (nb >= 3 && (umma::cache_mode(a.A.mode) || a.b_is_a)) || (a.b_is_a && (a.M > 128 || a.N > 128 || nb != 1)))
     return cudaErrorInvalidValue;
   if (a.splits == 1) a.kchunk = (int)round_up(a.K, umma::BK);
   if (a.c_accum && a.c_bf16) return cudaErrorInvalidValue;
@@ -684,6 +718,7 @@ inline cudaError_t launch_umma(const UmmaMaps& m, UmmaArgs a, int nb, cudaStream
   // N tiles of 256 only with one B operand: with two (hi + lo) a 256-wide stage takes 80 KB and
   // leaves room for two pipeline stages, a 128-wide one 48 KB and four
   if (nb == 3) return launch_umma_bn<128, 3>(m, a, st);   // a 64 KB stage: three stages
+  if (nb == 4) return launch_umma_bn<256, 4>(m, a, st);   // 2 x 16 KB + 32 KB: three stages
   if (a.bn == 256 || (a.bn == 0 && a.N > 128 && nb == 1))
     return nb == 2 ? launch_umma_bn<256, 2>(m, a, st) : launch_umma_bn<256, 1>(m, a, st);
   return nb == 2 ? launch_umma_bn<128, 2>(m, a, st) : launch_umma_bn<128, 1>(m, a, st);
@@ -694,6 +729,12 @@ inline cudaError_t launch_umma(const UmmaMaps& m, UmmaArgs a, int nb, cudaStream
 //   z_side = true  : C_u (M x N) = X_(T),u^T * sum_b F_b,u   with F_b,u = Fb[u] (T x ldf)
 // xk / xv: the K and V caches [n_layers][H][T][D] bf16; F1 may be null (one B operand).
 // C: fp32, or with C2 the result as a bf16 hi (C) + lo (C2) pair, pitch ldc.
+// With F = F0 + F1 (an fp32 operand as bf16 hi + lo) the product runs transposed, C^T =
+// (F0 + F1)^T X^T: the pair is the A operand and the cache a 256-wide B tile, so a stage holds
+// one cache tile for two MMAs (a 128-wide B tile with the pair on the B side needs a third more
+// shared-memory traffic per MMA, which the MMAs then wait on).  The tiles are stored
+// transposed and handed out M tile fastest, so the CTAs working at one time share the cache
+// tile in L2.
 inline cudaError_t umma_x_product(const void* xk, const void* xv, int n_layers, int H, int T, int D, int S,
                                   int nunits, bool z_side, const bf16* F0, const bf16* F1, int ldf, int N, void* C,
                                   long long ldc, uint32_t* status, int* sched, cudaStream_t st, void* C2 = nullptr) {
@@ -703,28 +744,44 @@ inline cudaError_t umma_x_product(const void* xk, const void* xv, int n_layers, 
   const int M = S * D;
   const long long krows = z_side ? T : M;
   UmmaMaps m;
-  if (!map_cache_xt(&m.a0, xk, n_layers, H, T, D) || !map_cache_xt(&m.a1, xv, n_layers, H, T, D) ||
-      !map_dense(&m.b0, F0, ldf, krows, nunits) || !map_dense(&m.b1, F1 ? F1 : F0, ldf, krows, nunits))
-    return cudaErrorInvalidValue;
   UmmaArgs a;
-  a.M = z_side ? M : T;
-  a.N = N;
-  a.K = z_side ? T : M;
+  if (F1) {
+    if (!map_dense(&m.a0, F0, ldf, krows, nunits) || !map_dense(&m.a1, F1, ldf, krows, nunits) ||
+        !map_cache_xt(&m.b0, xk, n_layers, H, T, D) || !map_cache_xt(&m.b1, xv, n_layers, H, T, D))
+      return cudaErrorInvalidValue;
+    a.M = N;
+    a.N = z_side ? M : T;
+    a.K = z_side ? T : M;
+    a.A.mode = UM_DENSE_MN;
+    a.B.mode = z_side ? UM_XT_MN : UM_XT_K;
+    a.B.S = S;
+    a.B.d_shift = dshift;
+    a.c_trans = 1;
+    a.m_fast = 1;
+  } else {
+    if (!map_cache_xt(&m.a0, xk, n_layers, H, T, D) || !map_cache_xt(&m.a1, xv, n_layers, H, T, D) ||
+        !map_dense(&m.b0, F0, ldf, krows, nunits))
+      return cudaErrorInvalidValue;
+    m.b1 = m.b0;
+    a.M = z_side ? M : T;
+    a.N = N;
+    a.K = z_side ? T : M;
+    a.A.mode = z_side ? UM_XT_MN : UM_XT_K;
+    a.A.S = S;
+    a.A.d_shift = dshift;
+    a.B.mode = UM_DENSE_MN;
+  }
   a.batch = nunits;
-  a.A.mode = z_side ? UM_XT_MN : UM_XT_K;
-  a.A.S = S;
-  a.A.d_shift = dshift;
-  a.B.mode = UM_DENSE_MN;
   a.C = C;
   a.ldc = ldc;
-  a.sC = (long long)a.M * ldc;
+  a.sC = (long long)(z_side ? M : T) * ldc;
   a.status = status;
   a.sched = sched;
   if (C2) {
     a.c_split = 1;
     a.C2 = C2;
   }
-  return launch_umma(m, a, F1 ? 2 : 1, st);
+  return launch_umma(m, a, F1 ? 4 : 1, st);
 }
 
 }  // namespace jolt
