@@ -30,8 +30,10 @@ METRIC = "KV compress throughput (input GB/s) at 2x/3x budget"
 RATIOS = (2.0, 3.0)
 L2_BYTES = 126 * 1024 * 1024
 # DRAM bytes (read + write) per launch of the dominant kernel from an ncu capture of the
-# current kernel, keyed by workload; a workload without an entry reports null
-KERNEL_TRAFFIC_BYTES = {}
+# current kernel, keyed by workload; a workload without an entry reports null.  The table
+# kernel on the LLaMA-3.1-8B/64K cache: 11,376,815,104 read + 210,655,744 written (one-pass
+# metrics, full size; the one-pass input is the 8.6 GB cache, U and P', about 11.6 GB)
+KERNEL_TRAFFIC_BYTES = {("llama31_8b_64k", "table_kernel"): 11376815104 + 210655744}
 
 
 def parse():

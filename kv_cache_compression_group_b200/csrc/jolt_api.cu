@@ -1527,7 +1527,7 @@ bool table_tc_ok(const Plan& p, long long ldU) {
 template <typename TX, typename BITS>
 jolt_status launch_table_tc_B(const Ctx& c, const CUtensorMap& mu, const CUtensorMap& mp, const TableTcArgs& a) {
   CUDA_TRY(cudaFuncSetAttribute(table_tc_kernel<TX, BITS>, cudaFuncAttributeMaxDynamicSharedMemorySize, ttc::SMEM));
-  count_launch(), table_tc_kernel<TX, BITS><<<dim3(a.tiles, c.p.S, c.p.NU), ttc::THREADS, ttc::SMEM, c.st>>>(mu, mp, a);
+  count_launch(), table_tc_kernel<TX, BITS><<<dim3((unsigned)(a.tiles * c.p.S), c.p.NU), ttc::THREADS, ttc::SMEM, c.st>>>(mu, mp, a);
   CUDA_TRY(cudaGetLastError());
   return JOLT_OK;
 }
@@ -1695,7 +1695,7 @@ jolt_status run_encode(const Ctx& c, const bf16* Us, long long ldU, const bf16* 
     e.seed = c.seed;
     e.blob = blob;
     e.status = c.status();
-    const dim3 grid((unsigned)ceil_div(p.T, ttc::ROWS), p.S, p.NU);
+    const dim3 grid((unsigned)(ceil_div(p.T, ttc::ROWS) * p.S), p.NU);   // slices fastest
     if (p.dtype == JOLT_BF16) {
       CUDA_TRY(cudaFuncSetAttribute(encode_tc_kernel<bf16>, cudaFuncAttributeMaxDynamicSharedMemorySize, ttc::SMEM));
       count_launch(), encode_tc_kernel<bf16><<<grid, etc::THREADS, ttc::SMEM, c.st>>>(mu, mp, e);

@@ -57,55 +57,49 @@ struct TableTcArgs {
 
 // the tile's rows rotated along the features into xs (fp32, pitch XS_LD): sign flip, the
 // Walsh-Hadamard butterflies in the order of fwht_regs (strides 1, 2, ..., 64), 1 / sqrt(D).
-// Run by the NTHREADS epilogue threads (threads 0 .. NTHREADS-1) alone, synchronised by
-// named barrier 1, while the copy and MMA warps start on the operands.
+// Run by the NTHREADS = 4 x ROWS epilogue threads (threads 0 .. NTHREADS-1) alone, four per
+// row, 32 features each: strides 1 .. 16 in registers, strides 32 and 64 with the partner
+// threads p ^ 1 and p ^ 2 (lanes of the same warp).  The operations are those of one thread
+// per row, so the result is the same bit for bit.  Ends with named barrier 1 over the
+// NTHREADS threads, while the copy and MMA warps start on the operands.
 template <typename TX, int NTHREADS>
 __device__ __forceinline__ void ttc_rotate_tile(const TX* X, int T, int t0, const float* sig, float* xs) {
   using namespace ttc;
+  static_assert(NTHREADS == 4 * ROWS && DIM == 128, "four threads per row, 32 features each");
   constexpr int V = 16 / sizeof(TX);   // elements per 16-byte load
-  for (int idx = threadIdx.x; idx < ROWS * DIM / V; idx += NTHREADS) {
-    const int r = idx / (DIM / V), d0 = (idx - r * (DIM / V)) * V, t = t0 + r;
-    float f[V];
-    if (t < T) {
-      const uint4 w = *reinterpret_cast<const uint4*>(X + (long long)t * DIM + d0);
+  const int r = threadIdx.x >> 2, p = threadIdx.x & 3, t = t0 + r;
+  float v[32];
+  if (t < T) {
+    const TX* src = X + (long long)t * DIM + 32 * p;
+#pragma unroll
+    for (int q = 0; q < 32 / V; ++q) {
+      const uint4 w = *reinterpret_cast<const uint4*>(src + q * V);
       const TX* e = reinterpret_cast<const TX*>(&w);
 #pragma unroll
-      for (int i = 0; i < V; ++i) f[i] = ld_as_float(e + i) * sig[d0 + i];
-    } else {
-#pragma unroll
-      for (int i = 0; i < V; ++i) f[i] = 0.f;
+      for (int i = 0; i < V; ++i) v[q * V + i] = ld_as_float(e + i) * sig[32 * p + q * V + i];
     }
+  } else {
 #pragma unroll
-    for (int i = 0; i < V; i += 4)
-      *reinterpret_cast<float4*>(xs + r * XS_LD + d0 + i) = make_float4(f[i], f[i + 1], f[i + 2], f[i + 3]);
+    for (int i = 0; i < 32; ++i) v[i] = 0.f;
   }
-  asm volatile("bar.sync 1, %0;" ::"n"(NTHREADS) : "memory");
-  if (threadIdx.x < ROWS) {
-    float* row = xs + threadIdx.x * XS_LD;
-#pragma unroll 1
-    for (int half = 0; half < 2; ++half) {
-      float v[64];
+  fwht_regs<32>(v);
+  // a pair (lower a, upper b) becomes (a + b, a - b): the upper thread of the pair forms
+  // partner - own, the lower own + partner
+  const bool up32 = (p & 1) != 0, up64 = (p & 2) != 0;
 #pragma unroll
-      for (int q = 0; q < 16; ++q) {
-        const float4 f = *reinterpret_cast<const float4*>(row + half * 64 + 4 * q);
-        v[4 * q] = f.x;
-        v[4 * q + 1] = f.y;
-        v[4 * q + 2] = f.z;
-        v[4 * q + 3] = f.w;
-      }
-      fwht_regs<64>(v);
-#pragma unroll
-      for (int q = 0; q < 16; ++q)
-        *reinterpret_cast<float4*>(row + half * 64 + 4 * q) = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
-    }
-    const float sc = (float)(1.0 / sqrt((double)DIM));
-#pragma unroll 4
-    for (int j = 0; j < 64; ++j) {
-      const float a = row[j], b = row[j + 64];
-      row[j] = (a + b) * sc;
-      row[j + 64] = (a - b) * sc;
-    }
+  for (int i = 0; i < 32; ++i) {
+    const float o = __shfl_xor_sync(0xffffffffu, v[i], 1);
+    v[i] = up32 ? o - v[i] : v[i] + o;
   }
+  const float sc = (float)(1.0 / sqrt((double)DIM));
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    const float o = __shfl_xor_sync(0xffffffffu, v[i], 2);
+    v[i] = (up64 ? o - v[i] : v[i] + o) * sc;
+  }
+  float* dst = xs + r * XS_LD + 32 * p;
+#pragma unroll
+  for (int i = 0; i < 32; i += 4) *reinterpret_cast<float4*>(dst + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
   asm volatile("bar.sync 1, %0;" ::"n"(NTHREADS) : "memory");
 }
 
@@ -195,7 +189,8 @@ __device__ __forceinline__ void ttc_block_errors(const float2* v, float2* acc, B
 
 __device__ __forceinline__ void ttc_epi_sync() { asm volatile("bar.sync 1, %0;" ::"n"(ttc::EPI_WARPS * 32) : "memory"); }
 
-// grid (tiles, S, units); ttc::THREADS threads; ttc::SMEM bytes of dynamic shared memory.
+// grid (S x tiles, units), slices fastest; ttc::THREADS threads; ttc::SMEM bytes of dynamic
+// shared memory.
 // Registers: the SM's file is four partitions of 16K, one per scheduler, and the 18 warps put
 // five on one partition, so a thread gets at most 96 (the launch bound makes ptxas keep to it).
 template <typename TX, typename BITS>
@@ -213,8 +208,9 @@ __global__ void __launch_bounds__(ttc::THREADS, 1)
   __shared__ float sig[DIM];
   __shared__ float red[EPI_WARPS][MAXT * MAXC];
 
-  const int tile = blockIdx.x, s = blockIdx.y, u = blockIdx.z;
   const int T = a.cv.T, S = a.cv.S, NU = 2 * (a.cv.n_layers / a.cv.Lg);
+  // slices fastest: the CTAs that run together share the token tile of U (one read from memory)
+  const int s = blockIdx.x % S, tile = blockIdx.x / S, u = blockIdx.y;
   const int t0 = tile * ROWS;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const Cands& cd = a.cand;
@@ -446,11 +442,12 @@ __global__ void __launch_bounds__(etc::THREADS, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   __shared__ float sig[DIM];
 
-  const int tile = blockIdx.x, s = blockIdx.y, u = blockIdx.z;
+  const int T = a.cv.T, S = a.cv.S, NU = 2 * (a.cv.n_layers / a.cv.Lg);
+  // slices fastest: the CTAs that run together share the token tile of U (one read from memory)
+  const int s = blockIdx.x % S, tile = blockIdx.x / S, u = blockIdx.y;
   const BlobHeader* gh = reinterpret_cast<const BlobHeader*>(a.blob);
   const UnitHeader uh = reinterpret_cast<const UnitHeader*>(a.blob + sizeof(BlobHeader))[u];
   if (gh->status != 0 || uh.bits == 0) return;   // uniform over the CTA: nothing to write
-  const int T = a.cv.T, S = a.cv.S, NU = 2 * (a.cv.n_layers / a.cv.Lg);
   const int t0 = tile * ROWS;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int rT = uh.r_T, b = uh.bits;
