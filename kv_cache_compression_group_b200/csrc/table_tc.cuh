@@ -408,16 +408,20 @@ namespace jolt {
 // ---------------------------------------------------------------------------------------
 // Encoder on the tensor cores (D = 128): the chosen (r_T, r_D, b) of the unit from the blob's
 // unit table; one CTA per 128 tokens of one slice.  The token-rank axis [0, r_T) is cut into
-// 64-rank segments that rotate through the four TMEM accumulators.  The epilogue subtracts
-// every finished segment from the rotated tile without rounding error (TwoSum into hi + lo),
-// so the residual carries the fp32 error of one 64-rank segment, not of the whole sum; then
-// it quantises rho = hi + lo block by block, packs the codes and writes codes and scales.
+// 128-rank segments (two 64-rank K blocks accumulated in one accumulator) that rotate through
+// the four TMEM accumulators.  The epilogue subtracts every finished segment from the rotated
+// tile without rounding error (TwoSum into hi + lo), so the residual carries the fp32 error of
+// one 128-rank segment, not of the whole sum; then it quantises rho = hi + lo block by block,
+// packs the codes and writes codes and scales.
 // Sixteen epilogue warps (four per TMEM lane quarter, 32 columns each).
 // ---------------------------------------------------------------------------------------
 namespace etc {
 constexpr int EPI_WARPS = 16;
 constexpr int THREADS = (EPI_WARPS + 2) * 32;
 constexpr int COLS = ttc::DIM / (EPI_WARPS / 4);   // 32
+// K blocks (64 ranks each) accumulated in one TMEM accumulator before the epilogue folds it
+// into the residual: the residual carries the fp32 rounding of one 128-rank partial sum
+constexpr int SEG_KB = 2;
 }  // namespace etc
 
 struct EncodeTcArgs {
@@ -453,7 +457,8 @@ __global__ void __launch_bounds__(etc::THREADS, 1)
   const int rT = uh.r_T, b = uh.bits;
   int iD = 0;
   while (iD < a.cand.nD && a.cand.rD[iD] != uh.r_D) ++iD;
-  const int nkb = (rT + BK - 1) / BK;     // K blocks = segments (64 ranks each)
+  const int nkb = (rT + BK - 1) / BK;     // K blocks of 64 ranks
+  const int nseg = (nkb + etc::SEG_KB - 1) / etc::SEG_KB;   // segments of SEG_KB K blocks
   const uint32_t full0 = umma::smem_u32(bars), empty0 = full0 + 8 * STAGES, accfull0 = empty0 + 8 * STAGES;
   const uint32_t accfree0 = accfull0 + 8 * MAXT, done_bar = accfree0 + 8 * MAXT;
 
@@ -505,12 +510,14 @@ __global__ void __launch_bounds__(etc::THREADS, 1)
     if (lane == 0) {
       constexpr uint32_t idesc = umma::instr_desc(DIM, false, true);
       for (int j = 0; j < nkb && !*abort_flag; ++j) {
-        const int st = j % STAGES, acc = j % MAXT, use = j / MAXT;
+        const int seg = j / etc::SEG_KB, jin = j - seg * etc::SEG_KB;
+        const int st = j % STAGES, acc = seg % MAXT, use = seg / MAXT;
         if (!umma::mbar_wait(full0 + 8 * st, (j / STAGES) & 1)) {
           *abort_flag = 1;
           break;
         }
-        if (use > 0 && !umma::mbar_wait(accfree0 + 8 * acc, (use - 1) & 1)) {
+        // a segment's first K block waits until the epilogue has read the accumulator's last use
+        if (jin == 0 && use > 0 && !umma::mbar_wait(accfree0 + 8 * acc, (use - 1) & 1)) {
           *abort_flag = 1;
           break;
         }
@@ -519,9 +526,9 @@ __global__ void __launch_bounds__(etc::THREADS, 1)
         for (int kk = 0; kk < BK / 16 && j * BK + kk * 16 < rT; ++kk) {
           const uint64_t ad = umma::smem_desc(sa + kk * 32, 16, 1024);
           const uint64_t bd = umma::smem_desc(sa + U_BYTES + kk * 2048, umma::BOX_BYTES, 1024);
-          umma::mma_bf16(tmem + (uint32_t)(acc * DIM), ad, bd, idesc, kk ? 1u : 0u);
+          umma::mma_bf16(tmem + (uint32_t)(acc * DIM), ad, bd, idesc, (jin | kk) ? 1u : 0u);
         }
-        umma::mma_commit(accfull0 + 8 * acc);
+        if (jin == etc::SEG_KB - 1 || j == nkb - 1) umma::mma_commit(accfull0 + 8 * acc);
         umma::mma_commit(empty0 + 8 * st);
       }
       umma::mma_commit(done_bar);
@@ -538,7 +545,7 @@ __global__ void __launch_bounds__(etc::THREADS, 1)
       hi[j] = xs[row * XS_LD + cbase + j];
       lo[j] = 0.f;
     }
-    for (int j = 0; j < nkb; ++j) {
+    for (int j = 0; j < nseg; ++j) {
       const int acc = j % MAXT, use = j / MAXT;
       bool ok = !*abort_flag && umma::mbar_wait(accfull0 + 8 * acc, use & 1);
       ok = __all_sync(0xffffffffu, ok);
