@@ -627,6 +627,9 @@ def main():
     if dom is not None:
         roofline = dict(dom)
         roofline["traffic"] = KERNEL_TRAFFIC_BYTES.get((w.name, dom["kernel"]))
+        if roofline["traffic"] is not None:
+            roofline["traffic_source"] = ("ncu dram__bytes_read.sum + dram__bytes_write.sum of one launch of the "
+                                          "current kernel on this workload (one-pass metrics, full size)")
         roofline["timing"] = ("per-launch time from a separate pass with CUDA events around the stage on its "
                               "launch stream (the timed steps replay CUDA graphs, which hold no events)")
 
